@@ -1,0 +1,299 @@
+/*
+ * Dust estimator oracle: plain, slow, fp64 CPU reference of the token-level
+ * node-perturbation gradient estimator for one linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or call
+ * this file: only the tests, the smoke check and the CPU-baseline leg of the
+ * benchmark use it.  It shares no code with the CUDA kernels.
+ *
+ * Source of every formula: the Dust review page (koala.ai.kr, "Dust: 역전파 없이
+ * 트랜스포머를 사전학습하다"), section "신용 할당(credit assignment): 보상에서
+ * 기울기까지":
+ *   noise equation          y_t -> y_t + sigma a_t,  a_t ~ N(0, I), independent per token
+ *   centred loss            c_s = mean-over-draws(l_s) - l_s
+ *   credit equation         r_t = sum_{s >= t} gamma^(s-t) c_s  (later tokens of the sequence)
+ *   output-error equation   g_t = -(1/(K sigma)) sum_i r_t^(i) a_t^(i)
+ *   weight-estimate eq.     G_W = sum_t g_t x_t^T
+ * The page fixes no random generator.  The one used here is Philox4x32-10
+ * (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as 1, 2, 3",
+ * SC'11), written from that paper's description, with the Box-Muller transform
+ * (Box & Muller 1958) on uniforms u(w) = (2*(w >> 9) + 1) * 2^-24.
+ * Counter of the quad that holds channel o of token t in draw i of layer L:
+ *   (o >> 2, token_offset + t, draw_offset + i, L), key = (seed lo32, seed hi32);
+ * channel o takes normal z[o & 3] of that quad.
+ *
+ * Every loop below is the plain definition; OpenMP only splits independent
+ * outer loops (tokens or output rows) across threads and never changes the
+ * order in which one output element is summed.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define PHILOX_M0 0xD2511F53u
+#define PHILOX_M1 0xCD9E8D57u
+#define PHILOX_W0 0x9E3779B9u
+#define PHILOX_W1 0xBB67AE85u
+
+void oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+int oracle_get_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Philox4x32 with 10 rounds (Salmon et al. 2011, section 3 "Philox"): each round
+ * multiplies words 0 and 2 by the two round multipliers into 64-bit products,
+ * and the new block is (hi(M1*c2) ^ c1 ^ k0, lo(M1*c2), hi(M0*c0) ^ c3 ^ k1,
+ * lo(M0*c0)); the key is bumped by the two Weyl constants between rounds. */
+void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) {
+            k0 += PHILOX_W0;
+            k1 += PHILOX_W1;
+        }
+        uint64_t p0 = (uint64_t)PHILOX_M0 * (uint64_t)c0;
+        uint64_t p1 = (uint64_t)PHILOX_M1 * (uint64_t)c2;
+        uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        uint32_t n0 = hi1 ^ c1 ^ k0;
+        uint32_t n1 = lo1;
+        uint32_t n2 = hi0 ^ c3 ^ k1;
+        uint32_t n3 = lo0;
+        c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/* u(w) = (2 * (w >> 9) + 1) * 2^-24: the top 23 bits, centred in their cell; never 0 or 1. */
+double oracle_uniform(uint32_t w)
+{
+    return ldexp(2.0 * (double)(w >> 9) + 1.0, -24);
+}
+
+/* Box-Muller on the four words of one Philox block: (w0, w1) -> (z0, z1), (w2, w3) -> (z2, z3). */
+void oracle_box_muller4(const uint32_t w[4], double z[4])
+{
+    const double two_pi = 6.283185307179586476925286766559;
+    for (int p = 0; p < 2; ++p) {
+        double rho = sqrt(-2.0 * log(oracle_uniform(w[2 * p])));
+        double theta = two_pi * oracle_uniform(w[2 * p + 1]);
+        z[2 * p] = rho * cos(theta);
+        z[2 * p + 1] = rho * sin(theta);
+    }
+}
+
+/* The four normals a[4q .. 4q+3] of token t (global), draw i (global), layer L. */
+void oracle_normal_quad(uint64_t seed, uint32_t q, uint32_t t, uint32_t i, uint32_t layer,
+                        double z[4])
+{
+    uint32_t ctr[4] = {q, t, i, layer};
+    uint32_t key[2] = {(uint32_t)(seed & 0xffffffffu), (uint32_t)(seed >> 32)};
+    uint32_t w[4];
+    oracle_philox4x32_10(ctr, key, w);
+    oracle_box_muller4(w, z);
+}
+
+/* Batch of Philox blocks for arbitrary counters (n x 4 words in, n x 4 words and normals out). */
+void oracle_philox_batch(const uint32_t* ctr, int64_t n, uint64_t seed, uint32_t* words,
+                         double* normals)
+{
+    uint32_t key[2] = {(uint32_t)(seed & 0xffffffffu), (uint32_t)(seed >> 32)};
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < n; ++j) {
+        uint32_t w[4];
+        oracle_philox4x32_10(ctr + 4 * j, key, w);
+        if (words) memcpy(words + 4 * j, w, sizeof w);
+        if (normals) oracle_box_muller4(w, normals + 4 * j);
+    }
+}
+
+/* Noise a_t^(i)[o] for a list of (t, i, o) triples (local indices; offsets added here). */
+static double noise_at(uint64_t seed, uint32_t layer, uint32_t tg, uint32_t ig, int32_t o)
+{
+    double z[4];
+    oracle_normal_quad(seed, (uint32_t)o >> 2, tg, ig, layer, z);
+    return z[o & 3];
+}
+
+/*
+ * Per-token quadratic readout loss of the noisy layer, absolute, for every draw:
+ *   y_t = W x_t;  l_t^(i) = 1/2 || y_t + sigma a_t^(i) - u_t ||^2;  clean_t = 1/2 || y_t - u_t ||^2.
+ * (noise equation of the page; the quadratic readout is the synthetic per-token loss.)
+ * tokens: n_tok local token indices to evaluate (NULL: all N, n_tok = N).
+ * loss: [K][n_tok], clean: [n_tok] (may be NULL).
+ */
+void oracle_noisy_linear_loss(const double* x, const double* W, const double* u, int64_t N,
+                              int32_t d_in, int32_t d_out, int32_t K, double sigma,
+                              uint64_t seed, uint32_t layer_id, uint32_t draw_offset,
+                              uint32_t token_offset, const int64_t* tokens, int64_t n_tok,
+                              double* loss, double* clean)
+{
+    if (!tokens) n_tok = N;
+#pragma omp parallel
+    {
+        double* y = (double*)malloc(sizeof(double) * (size_t)d_out);
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t j = 0; j < n_tok; ++j) {
+            int64_t t = tokens ? tokens[j] : j;
+            const double* xt = x + t * (int64_t)d_in;
+            const double* ut = u + t * (int64_t)d_out;
+            for (int32_t o = 0; o < d_out; ++o) {
+                double acc = 0.0;
+                const double* Wo = W + (int64_t)o * d_in;
+                for (int32_t k = 0; k < d_in; ++k) acc += Wo[k] * xt[k];
+                y[o] = acc;
+            }
+            if (clean) {
+                double l = 0.0;
+                for (int32_t o = 0; o < d_out; ++o) {
+                    double e = y[o] - ut[o];
+                    l += e * e;
+                }
+                clean[j] = 0.5 * l;
+            }
+            for (int32_t i = 0; i < K; ++i) {
+                double l = 0.0;
+                for (int32_t q = 0; 4 * q < d_out; ++q) {
+                    double z[4];
+                    oracle_normal_quad(seed, (uint32_t)q, token_offset + (uint32_t)t,
+                                       draw_offset + (uint32_t)i, layer_id, z);
+                    for (int32_t jj = 0; jj < 4 && 4 * q + jj < d_out; ++jj) {
+                        int32_t o = 4 * q + jj;
+                        double v = y[o] + sigma * z[jj] - ut[o];
+                        l += v * v;
+                    }
+                }
+                loss[(int64_t)i * n_tok + j] = 0.5 * l;
+            }
+        }
+        free(y);
+    }
+}
+
+/* Segment index of every token from cu_seqlens (cu[0] = 0, cu[n_seq] = N). */
+static int32_t* segment_end_of(const int32_t* cu, int32_t n_seq, int64_t N)
+{
+    int32_t* end = (int32_t*)malloc(sizeof(int32_t) * (size_t)(N > 0 ? N : 1));
+    for (int32_t s = 0; s < n_seq; ++s)
+        for (int64_t t = cu[s]; t < cu[s + 1]; ++t) end[t] = cu[s + 1];
+    return end;
+}
+
+/*
+ * Centred loss and discounted credit, as written on the page:
+ *   mean_t = (1/K) sum_i l_t^(i)     (the draw mean includes draw i itself)
+ *   c_t^(i) = mean_t - l_t^(i)
+ *   r_t^(i) = sum_{s = t}^{end(seg(t)) - 1} gamma^(s - t) c_s^(i)
+ * computed as the explicit double sum (O(T^2) per segment).
+ * loss, r: [K][N] row-major with leading dimension N.
+ */
+void oracle_credit(const double* loss, int32_t K, int64_t N, const int32_t* cu, int32_t n_seq,
+                   double gamma, double* r)
+{
+    double* c = (double*)malloc(sizeof(double) * (size_t)(K * N > 0 ? K * N : 1));
+    for (int64_t t = 0; t < N; ++t) {
+        double m = 0.0;
+        for (int32_t i = 0; i < K; ++i) m += loss[(int64_t)i * N + t];
+        m /= (double)K;
+        for (int32_t i = 0; i < K; ++i) c[(int64_t)i * N + t] = m - loss[(int64_t)i * N + t];
+    }
+    int32_t* end = segment_end_of(cu, n_seq, N);
+#pragma omp parallel for schedule(dynamic, 16) collapse(2)
+    for (int32_t i = 0; i < K; ++i) {
+        for (int64_t t = 0; t < N; ++t) {
+            double acc = 0.0, g = 1.0;
+            for (int64_t s = t; s < end[t]; ++s) {
+                acc += g * c[(int64_t)i * N + s];
+                g *= gamma;
+            }
+            r[(int64_t)i * N + t] = acc;
+        }
+    }
+    free(end);
+    free(c);
+}
+
+/* Second route to the same credit: the backward recurrence r_t = c_t + gamma r_{t+1},
+ * restarted at each segment end (used only to check the double sum). */
+void oracle_credit_recurrence(const double* loss, int32_t K, int64_t N, const int32_t* cu,
+                              int32_t n_seq, double gamma, double* r)
+{
+    for (int64_t t = 0; t < N; ++t) {
+        double m = 0.0;
+        for (int32_t i = 0; i < K; ++i) m += loss[(int64_t)i * N + t];
+        m /= (double)K;
+        for (int32_t i = 0; i < K; ++i) r[(int64_t)i * N + t] = m - loss[(int64_t)i * N + t];
+    }
+    for (int32_t i = 0; i < K; ++i)
+        for (int32_t s = 0; s < n_seq; ++s)
+            for (int64_t t = (int64_t)cu[s + 1] - 2; t >= cu[s]; --t)
+                r[(int64_t)i * N + t] += gamma * r[(int64_t)i * N + t + 1];
+}
+
+/*
+ * Output-error estimate (output-error equation of the page):
+ *   g_t[o] = -(1 / (K_total sigma)) sum_{i < K_chunk} r_t^(i) a_t^(draw_offset + i)[o]
+ * r: [K_chunk][N] (leading dimension N).  tokens / chans select the outputs (NULL: all).
+ * g: [n_tok][n_ch].
+ */
+void oracle_output_error(const double* r, int32_t K_chunk, int32_t K_total, int64_t N,
+                         int32_t d_out, double sigma, uint64_t seed, uint32_t layer_id,
+                         uint32_t draw_offset, uint32_t token_offset, const int64_t* tokens,
+                         int64_t n_tok, const int32_t* chans, int32_t n_ch, double* g)
+{
+    if (!tokens) n_tok = N;
+    if (!chans) n_ch = d_out;
+    const double scale = -1.0 / ((double)K_total * sigma);
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t j = 0; j < n_tok; ++j) {
+        int64_t t = tokens ? tokens[j] : j;
+        for (int32_t cc = 0; cc < n_ch; ++cc) {
+            int32_t o = chans ? chans[cc] : cc;
+            double acc = 0.0;
+            for (int32_t i = 0; i < K_chunk; ++i)
+                acc += r[(int64_t)i * N + t] *
+                       noise_at(seed, layer_id, token_offset + (uint32_t)t,
+                                draw_offset + (uint32_t)i, o);
+            g[j * n_ch + cc] = scale * acc;
+        }
+    }
+}
+
+/*
+ * Weight estimate (weight-estimate equation of the page), the explicit sum of outer
+ * products over tokens:  G_W[o][k] = sum_t g_t[o] x_t[k].
+ * g: [N][d_out], x: [N][d_in], GW: [d_out][d_in].
+ */
+void oracle_weight_grad(const double* g, const double* x, int64_t N, int32_t d_in,
+                        int32_t d_out, double* GW)
+{
+#pragma omp parallel for schedule(static)
+    for (int32_t o = 0; o < d_out; ++o) {
+        double* row = GW + (int64_t)o * d_in;
+        for (int32_t k = 0; k < d_in; ++k) row[k] = 0.0;
+        for (int64_t t = 0; t < N; ++t) {
+            double gt = g[t * d_out + o];
+            const double* xt = x + t * (int64_t)d_in;
+            for (int32_t k = 0; k < d_in; ++k) row[k] += gt * xt[k];
+        }
+    }
+}
