@@ -1,0 +1,420 @@
+#!/usr/bin/env python
+"""Benchmark of the Dust estimator hot path for one transformer linear layer on B200.
+
+One step = the whole path over one batch of seeded synthetic input resident in HBM:
+  dust_noisy_linear_fwd (noise + per-draw loss change) -> dust_credit (centring + discounted
+  credit scan) -> dust_weight_grad (output-error estimate g + weight estimate G_W),
+and, on N > 1 GPUs, one NCCL all-reduce of G_W (each rank holds its own batch; weak scaling).
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload C] [--impl ours|reference]
+Multi-GPU: launched by torchrun, one rank per GPU (RANK / LOCAL_RANK / WORLD_SIZE from the env).
+Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle instead (rank 0
+only), on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "Dust estimator tokens*draws/s per layer"
+UNIT = "tokens*draws/s"
+L2_FLUSH_BYTES = 256 << 20
+
+# ALU roofline of the noise kernels: issue slots of all SMs at the maximum SM clock divided by
+# the algorithm's minimal per-normal operation count (one Philox4x32-10 block = 10 rounds x
+# (2 wide multiplies + 2 three-input XORs) per 4 normals; 3 ops per uniform; Box-Muller 10 ops
+# per pair: log, scale, rsqrt, multiply, angle FMA, range scale, sin, cos, 2 products; plus the
+# consumer FMAs: 2 per normal in the forward, 1 in the draw reduction).
+LANES_PER_SM = 128
+OPS_PER_NORMAL = {"fwd_bf16_noise_loss": 20.0, "ghat_reduce_draws": 19.0}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d["bf16_tflops_sustained"],
+                    sm_max_mhz=d.get("sm_max_mhz", 1965.0), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                sm_max_mhz=1965.0, source="fallback")
+
+
+def describe(wl) -> str:
+    shapes = sorted({(l.d_in, l.d_out) for l in wl.layers})
+    s = ", ".join(f"{a}->{b}" for a, b in shapes)
+    return (f"{wl.name} (cfg {wl.cfg_id}): {wl.n_seq}x{wl.seq_len} tokens"
+            f"{' packed' if wl.packed else ''}, {len(wl.layers)} layer(s) {s}, K={wl.K}, "
+            f"sigma={wl.sigma}, gamma={wl.gamma}, {wl.dtype}")
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+def oracle_sample(data, n_tokens: int, max_seconds: float):
+    """Run the oracle's whole estimator on the first n_tokens of each layer until max_seconds
+    of work; returns (token*draws processed per layer, seconds, threads, description)."""
+    import oracle
+    wl = data.wl
+    done = 0
+    t0 = time.perf_counter()
+    layers_run = 0
+    while True:
+        L = data.layers[layers_run % len(data.layers)]
+        n = min(n_tokens, wl.N)
+        cu = np.asarray(data.cu_seqlens, dtype=np.int64)
+        cu = np.unique(np.clip(cu, 0, n)).astype(np.int32)
+        oracle.dust_layer(L.x_f64[:n], L.W_f64, L.u_f64[:n], wl.K, wl.sigma, wl.gamma, cu,
+                          wl.seed, L.shape.layer_id)
+        done += n * wl.K
+        layers_run += 1
+        el = time.perf_counter() - t0
+        if el >= max_seconds or layers_run >= 64:
+            break
+    desc = (f"oracle (fp64 C, OpenMP) whole estimator on the first {min(n_tokens, wl.N)} tokens "
+            f"of {layers_run} layer pass(es) of the workload (credit segments truncated to the "
+            f"sample)")
+    return done, el, oracle.get_threads(), desc
+
+
+def run_reference(args, rank: int, world: int) -> None:
+    if rank != 0:
+        return
+    data = workloads.generate(args.workload, n_layers=1)
+    wl = data.wl
+    n_tok = args.ref_tokens
+    times = []
+    for k in range(args.warmup + args.steps):
+        done, el, cores, desc = oracle_sample(data, n_tok, 0.0)
+        if k >= args.warmup:
+            times.append(el)
+    tot = sum(times)
+    value = done * len(times) / tot
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": describe(wl), "sample_tokens": min(n_tok, wl.N)},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------ GPU arm
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
+        self.proc = None
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(gpu_index), "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for ln in f:
+                p = [x.strip() for x in ln.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    sm.append(float(p[1]))
+                    smax.append(float(p[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, p[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def kernel_work(name, wl, layer):
+    """Algorithmic work of one launch: (bound, amount, unit-scale) for the roofline."""
+    N, K = wl.N, wl.K
+    if name in OPS_PER_NORMAL:
+        return "alu", N * layer.d_out * K, "normals"
+    if name == "gw_bf16_tcgen05":
+        return "tensor", 2.0 * N * layer.d_in * layer.d_out, "flops"
+    if name == "credit_scan":
+        return "hbm", 8.0 * K * N, "bytes"
+    if name == "gw_splitk_reduce":
+        return "hbm", None, "bytes"
+    return None, None, None
+
+
+def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
+    import torch
+    import torch.distributed as dist
+
+    import zeroth_order_transformer_b200 as dust
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=dev)
+    data = workloads.generate(args.workload)
+    wl = data.wl
+    peaks = measured_peaks()
+
+    def dev_t(store, dtype):
+        if dtype == "f32":
+            return torch.from_numpy(np.ascontiguousarray(store)).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(store).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    layers = []
+    for L in data.layers:
+        x, W, u = (dev_t(a, wl.dtype) for a in (L.x_store, L.W_store, L.u_store))
+        layers.append((L.shape, x, W, u))
+    cu = torch.from_numpy(data.cu_seqlens).to(dev)
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    max_in = max(s.d_in for s, *_ in layers)
+    max_out = max(s.d_out for s, *_ in layers)
+    ws_bytes = max(dust.dust_workspace_size(op, 1 if wl.dtype == "bf16" else 0, wl.N, s.d_in,
+                                            s.d_out, wl.K)
+                   for op in range(3) for s, *_ in layers)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    dloss = torch.empty((wl.K, wl.N), dtype=torch.float32, device=dev)
+    r = torch.empty((wl.K, wl.N), dtype=torch.float32, device=dev)
+    GWs = [torch.empty((s.d_out, s.d_in), dtype=torch.float32, device=dev) for s, *_ in layers]
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    gamma = wl.gamma
+
+    def step(inputs=None):
+        for li, (s, x, W, u) in enumerate(inputs or layers):
+            key = dust.NoiseKey(wl.seed, s.layer_id, 0, rank * wl.N)
+            dust.dust_noisy_linear_fwd(x, W, u, wl.K, wl.sigma, key, dloss, ws)
+            dust.dust_credit(dloss, cu, gamma, r, ws)
+            dust.dust_weight_grad(r, x, s.d_out, wl.K, wl.sigma, key, GWs[li], False, None, ws)
+        if world > 1:
+            for G in GWs:
+                dist.all_reduce(G)
+
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+
+    # ---- timed region
+    dust.dust_profile_enable(1 << 16)
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    for k in range(args.steps):
+        flush.zero_()
+        starts[k].record(stream)
+        step()
+        stops[k].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    prof = dust.dust_profile_read()
+    dust.dust_profile_disable()
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    units = wl.N * wl.K * len(layers) * world
+    value = units / (ms_per_step / 1e3) / len(layers)  # per layer
+
+    # ---- per-kernel statistics (rank 0's launches)
+    per = {}
+    for name, ms in prof:
+        d = per.setdefault(name, [0, 0.0])
+        d[0] += 1
+        d[1] += ms
+    kern_total = sum(v[1] for v in per.values())
+    kernels = {n: {"launches": c, "ms_total": round(t, 4), "ms_avg": round(t / c, 5),
+                   "share": round(t / kern_total, 4) if kern_total else None}
+               for n, (c, t) in sorted(per.items(), key=lambda kv: -kv[1][1])}
+    s0 = layers[0][0]
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    for n, info in kernels.items():
+        bound, amount, what = kernel_work(n, wl, s0)
+        if amount is None or len(layers) > 1:
+            continue
+        per_s = amount / (info["ms_avg"] / 1e3)
+        if what == "normals":
+            info["gnormals_per_s"] = round(per_s / 1e9, 2)
+        elif what == "flops":
+            info["tflops"] = round(per_s / 1e12, 2)
+        else:
+            info["gbs"] = round(per_s / 1e9, 2)
+    dominant = next(iter(kernels)) if kernels else None
+    roofline = None
+    if dominant and len(layers) == 1:
+        bound, amount, what = kernel_work(dominant, wl, s0)
+        avg_s = kernels[dominant]["ms_avg"] / 1e3
+        if bound == "alu":
+            peak = sms * LANES_PER_SM * peaks["sm_max_mhz"] * 1e6 / OPS_PER_NORMAL[dominant] / 1e9
+            ach = amount / avg_s / 1e9
+            roofline = {"kernel": dominant, "bound": "alu", "achieved": round(ach, 2),
+                        "peak": round(peak, 2), "unit": "Gnormal/s", "frac": round(ach / peak, 4),
+                        "traffic": None,
+                        "peak_basis": f"{sms} SMs x {LANES_PER_SM} lanes x "
+                                      f"{peaks['sm_max_mhz']:.0f} MHz / "
+                                      f"{OPS_PER_NORMAL[dominant]:.0f} ops per normal"}
+        elif bound == "tensor":
+            ach = amount / avg_s / 1e12
+            roofline = {"kernel": dominant, "bound": "tensor", "achieved": round(ach, 2),
+                        "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                        "frac": round(ach / peaks["bf16_tflops"], 4), "traffic": None}
+        elif bound == "hbm":
+            ach = amount / avg_s / 1e9
+            roofline = {"kernel": dominant, "bound": "hbm", "achieved": round(ach, 2),
+                        "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None}
+        if roofline is not None:
+            roofline["peak_source"] = peaks["source"]
+
+    # ---- end to end through the public API, host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        host_in = []
+        h2d = 0
+        for s, x, W, u in layers:
+            hx, hW, hu = (t.cpu().pin_memory() for t in (x, W, u))
+            host_in.append((s, hx, hW, hu))
+            h2d += sum(t.numel() * t.element_size() for t in (hx, hW, hu))
+        dev_in = [(s, torch.empty_like(x), torch.empty_like(W), torch.empty_like(u))
+                  for s, x, W, u in layers]
+        host_out = [torch.empty(G.shape, dtype=G.dtype, pin_memory=True) for G in GWs]
+        d2h = sum(G.numel() * G.element_size() for G in GWs)
+
+        def e2e_step():
+            for (s, hx, hW, hu), (_, dx, dW, du) in zip(host_in, dev_in):
+                dx.copy_(hx, non_blocking=True)
+                dW.copy_(hW, non_blocking=True)
+                du.copy_(hu, non_blocking=True)
+            step(dev_in)
+            for G, hG in zip(GWs, host_out):
+                hG.copy_(G, non_blocking=True)
+
+        for _ in range(max(1, args.warmup // 2)):
+            flush.zero_()
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        es = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ee = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for k in range(args.steps):
+            flush.zero_()
+            es[k].record(stream)
+            e2e_step()
+            ee[k].record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = sum(a.elapsed_time(b) for a, b in zip(es, ee))
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": units / (e_ms / args.steps / 1e3) / len(layers), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e_ms / args.steps}
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        done, el, cores, desc = oracle_sample(data, args.cpu_tokens, args.cpu_seconds)
+        cpu = {"value": done / el, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": desc, "seconds": round(el, 2)}
+
+    n_launch_per_step = sum(c for c in (v["launches"] for v in kernels.values())) / args.steps
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, f32/u32 noise",
+        "data": "synthetic (seeded; shapes of the Dust page's transformer layers)",
+        "config": {"workload": describe(wl), "tokens_per_gpu": wl.N, "d_in": s0.d_in,
+                   "d_out": s0.d_out, "K": wl.K, "layers": len(layers),
+                   "parallelism": f"dp{world}: one batch per GPU, NCCL all-reduce of G_W",
+                   "l2": "flushed (256 MiB write) before every timed step"},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": int(round(n_launch_per_step * args.steps)),
+        "clocks": clocks,
+        "kernels": kernels,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=2, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-tokens", type=int, default=1024)
+    ap.add_argument("--ref-tokens", type=int, default=256)
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_gpu(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,164 @@
+/*
+ * dust.h: C ABI of libdust, a B200 (sm_100a) implementation of the Dust token-level
+ * node-perturbation gradient estimator for one linear layer y_t = W x_t.
+ *
+ * The method (Dust review page, koala.ai.kr, "Dust: 역전파 없이 트랜스포머를 사전학습하다",
+ * section "신용 할당(credit assignment): 보상에서 기울기까지"):
+ *   noise equation          y_t -> y_t + sigma a_t,  a_t ~ N(0, I) independent per token, draw
+ *   centred loss            c_s = mean_i(l_s^(i)) - l_s^(i)   (mean over the draws, self included)
+ *   credit equation         r_t = sum_{s >= t} gamma^(s-t) c_s   (later tokens of the same sequence)
+ *   output-error equation   g_t = -(1/(K sigma)) sum_i r_t^(i) a_t^(i)
+ *   weight-estimate eq.     G_W = sum_t g_t x_t^T
+ * The per-token loss computed by dust_noisy_linear_fwd is the quadratic readout
+ * l_t = 1/2 || W x_t + sigma a_t - u_t ||^2.
+ *
+ * Noise is never stored: every kernel regenerates a_t^(i)[o] from a counter-based generator,
+ * Philox4x32-10 (Salmon et al., SC'11) with Box-Muller.  The block with counter
+ *     (o >> 2, token_offset + t, draw_offset + i, layer_id),  key (seed lo32, seed hi32)
+ * gives four words w0..w3; with u(w) = (2 (w >> 9) + 1) 2^-24,
+ *     z0 = rho cos(2 pi u(w1)), z1 = rho sin(2 pi u(w1)), rho = sqrt(-2 ln u(w0)),
+ *     z2, z3 likewise from (w2, w3);  a_t^(i)[o] = z_{o & 3}.
+ * Normals are fp32, within 1e-5 (absolute) of the exact value of the same formula.
+ *
+ * Conventions for every call:
+ *   - Pointers named in the signature are DEVICE pointers unless said otherwise; arrays are
+ *     row-major with a contiguous last dimension; pointers are 16-byte aligned.
+ *   - The caller owns every buffer.  The library allocates no device memory; scratch space
+ *     comes from the caller's workspace (size from dust_workspace_size).
+ *   - Calls are asynchronous: they enqueue kernels on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream) and return after the launch.
+ *   - Argument errors return synchronously and launch nothing.  Failures inside a kernel
+ *     (a bounded wait that ran out) set a device error word that dust_last_device_error
+ *     reads.  No C++ exception crosses this interface.
+ *   - Sizes: N >= 1 tokens, 1 <= K.  bf16 layers need d_in and d_out multiples of 16;
+ *     fp32 layers need d_out a multiple of 4.
+ */
+#ifndef DUST_H
+#define DUST_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DUST_OK = 0,
+    DUST_ERR_INVALID_ARG = 1,  /* a size, pointer, alignment or value is out of range       */
+    DUST_ERR_UNSUPPORTED = 2,  /* valid, but outside what the kernels implement              */
+    DUST_ERR_CUDA = 3,         /* a CUDA runtime call failed (launch, attribute, driver)     */
+    DUST_ERR_TIMEOUT = 4,      /* a bounded device-side wait ran out (see dust_credit)       */
+    DUST_ERR_WORKSPACE = 5     /* workspace pointer NULL, misaligned or smaller than needed  */
+} dust_status;
+
+typedef enum { DUST_F32 = 0, DUST_BF16 = 1 } dust_dtype;
+
+typedef enum {
+    DUST_OP_NOISY_LINEAR_FWD = 0,
+    DUST_OP_CREDIT = 1,
+    DUST_OP_WEIGHT_GRAD = 2
+} dust_op;
+
+/* Identifies the noise of one call.  seed: generator key; layer_id: fourth counter word, so
+ * layers draw independent noise; draw_offset: global index of the call's first draw (a
+ * population larger than one call is processed in chunks); token_offset: global index of the
+ * call's first token (a batch sharded over several GPUs keeps the same noise per token). */
+typedef struct {
+    uint64_t seed;
+    uint32_t layer_id;
+    uint32_t draw_offset;
+    uint32_t token_offset;
+    uint32_t reserved; /* must be 0 */
+} dust_noise_key;
+
+/*
+ * Noisy linear forward with the per-draw loss change (noise equation; quadratic readout).
+ *   For each draw i in [0, K) and token t in [0, N):
+ *     dloss[i * ld_dloss + t] = l_t^(i) - l_t^clean
+ *                             = sum_o ( sigma a e_o + sigma^2 a^2 / 2 ),  a = a_t^(i)[o],
+ *   with e = W x_t - u_t the clean residual.  The clean forward y = W x is computed once;
+ *   the noise is added in the epilogue and never stored.
+ * x: [N, d_in], W: [d_out, d_in], u: [N, d_out], all of dtype dt.
+ * dloss: fp32 [K, ld_dloss], ld_dloss >= N.
+ * workspace: dust_workspace_size(DUST_OP_NOISY_LINEAR_FWD, ...) bytes, 256-byte aligned.
+ * Deterministic: the same inputs and key give bit-identical dloss.
+ */
+dust_status dust_noisy_linear_fwd(const void* x, const void* W, const void* u, dust_dtype dt,
+                                  int64_t N, int32_t d_in, int32_t d_out, int32_t K,
+                                  float sigma, dust_noise_key key, float* dloss,
+                                  int64_t ld_dloss, void* workspace, size_t ws_bytes,
+                                  void* stream);
+
+/*
+ * Centred loss and discounted credit (centred-loss and credit equations).
+ *   mean_t = (1/K) sum_i loss[i][t];  c = mean_t - loss[i][t];
+ *   r[i][t] = c_t + gamma * r[i][t+1], restarted (r = c) at the last token of each segment.
+ * loss: fp32 [K, ld_loss] (absolute losses or the dloss of dust_noisy_linear_fwd; the
+ *       centring removes any per-token constant).  r: fp32 [K, ld_r].  ld_* >= N.
+ * cu_seqlens: DEVICE int32 [n_seq + 1], non-decreasing, cu[0] = 0, cu[n_seq] = N; segment s
+ *   is tokens [cu[s], cu[s+1]); credit never crosses a segment end.  Token N-1 always ends a
+ *   segment.  Out-of-order entries give undefined r but no out-of-range access.
+ * 0 <= gamma <= 1.  K >= 2 (with K = 1 the centred loss is identically 0).
+ * The reverse scan chains token blocks by decoupled look-back.  Every wait is bounded (about
+ * one second); a wait that runs out writes NaN to its block and sets DUST_ERR_TIMEOUT in the
+ * device error word.  Deterministic.
+ */
+dust_status dust_credit(const float* loss, int64_t ld_loss, int32_t K, int64_t N,
+                        const int32_t* cu_seqlens, int32_t n_seq, float gamma, float* r,
+                        int64_t ld_r, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Output-error estimate and weight estimate (output-error and weight-estimate equations).
+ *   g_t[o] = -(1/(K_total sigma)) sum_{i < K_chunk} r[i][t] a_t^(draw_offset + i)[o]
+ *   G_W[o][k] (+)= sum_t g_t[o] x_t[k]
+ * r: fp32 [K_chunk, ld_r] holds the credit rows of draws key.draw_offset .. +K_chunk.
+ * x: [N, d_in] of dtype dt.  G_W: fp32 [d_out, d_in]; accumulate != 0 adds to it (chunks of
+ * one population), accumulate == 0 overwrites it.  g_out: optional fp32 [N, d_out] copy of g
+ * (NULL to skip).  For bf16, g enters the tensor-core contraction rounded to bf16 (fp32
+ * accumulation).  Deterministic (split-K partials are reduced in a fixed order).
+ */
+dust_status dust_weight_grad(const float* r, int64_t ld_r, const void* x, dust_dtype dt,
+                             int64_t N, int32_t d_in, int32_t d_out, int32_t K_chunk,
+                             int32_t K_total, float sigma, dust_noise_key key, float* G_W,
+                             int accumulate, float* g_out, void* workspace, size_t ws_bytes,
+                             void* stream);
+
+/* Workspace bytes that `op` needs for these sizes (0 if none).  d_in / d_out are ignored by
+ * DUST_OP_CREDIT, K by DUST_OP_WEIGHT_GRAD. */
+size_t dust_workspace_size(dust_op op, dust_dtype dt, int64_t N, int32_t d_in, int32_t d_out,
+                           int32_t K);
+
+/* Static, NUL-terminated name of a status code. */
+const char* dust_status_string(dust_status s);
+
+/* Synchronizes `stream`, then reads and clears the device error word of the current device:
+ * DUST_OK if no kernel reported a failure since the last read.  *info (if not NULL) receives
+ * the failing block index or wait site recorded with the error. */
+dust_status dust_last_device_error(void* stream, int32_t* info);
+
+/* Profiling.  While enabled, every kernel that libdust launches is bracketed by two CUDA
+ * events on its stream (cheap; no synchronization).  dust_profile_read synchronizes the
+ * device, then returns up to `max` records (static kernel name, duration in ms) in launch
+ * order and clears them.  At most `capacity` launches are kept; later ones are dropped.
+ * Host-side state is one global list (not thread-safe). */
+dust_status dust_profile_enable(int32_t capacity);
+void dust_profile_disable(void);
+int32_t dust_profile_read(const char** names, float* ms, int32_t max);
+
+/* Test support: the generator on its own.  ctr: DEVICE uint32 [n, 4] counters; the key is
+ * (seed lo32, seed hi32).  Writes DEVICE words [n, 4] and fp32 normals [n, 4] (either may be
+ * NULL).  Uses the same device functions as the estimator kernels. */
+dust_status dust_debug_philox(const uint32_t* ctr, int64_t n, uint64_t seed, uint32_t* words,
+                              float* normals, void* stream);
+
+/* Test support: the next dust_credit launch on any stream skips publishing the look-back
+ * status of token block `block` (-1: none), so that the block before it waits until its
+ * bounded wait runs out.  Used to test the timeout path; never set in normal use. */
+void dust_debug_credit_skip_publish(int32_t block);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DUST_H */

@@ -1,0 +1,305 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, on seeded inputs.
+
+Tolerances, from the arithmetic:
+  * Philox words and all integer/segment logic: bit-exact.
+  * Normals: the kernels evaluate Box-Muller in fp32 with logf (about 1 ulp), x * rsqrtf(x)
+    (2 ulp) and the fast sine/cosine on (-pi, pi) (absolute error 2^-21.41); with |z| <= 5.77
+    the bound is a few 1e-6, tested at 1e-5 absolute.
+  * Loss change and fp32 g: sums of d_out (or K) terms in fp32 whose inputs carry the normal
+    error above: element error <= 1e-3 x RMS, relative Frobenius error <= 1e-4.
+  * G_W (bf16): g enters the tensor cores rounded to bf16 (relative rounding error up to 2^-9,
+    RMS about 1.7e-3 for a noise-dominated g); the required bar is 2e-3 relative Frobenius,
+    against the oracle's G_W built from the oracle's own fp64 g.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from tests import _dev
+
+pytestmark = pytest.mark.gpu
+
+z = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    global z
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import zeroth_order_transformer_b200 as zz
+    zz.lib()
+    z = zz
+    yield
+    st, info = z.dust_last_device_error()
+    assert st == 0, (st, info)
+
+
+# ------------------------------------------------------------------------- generator
+def test_philox_words_bit_exact_and_normals_close():
+    import torch
+    rng = np.random.default_rng(100)
+    n = 1 << 18
+    ctr = rng.integers(0, 2**32, size=(n, 4), dtype=np.uint64).astype(np.uint32)
+    ctr[: n // 4, 1:] &= np.uint32(0xFFFF)
+    ctr[n // 4: n // 2] |= np.uint32(0x80000000)
+    seed = 0x5EED0002
+    words_ref, z_ref = oracle.philox_batch(ctr, seed)
+    w, zn = z.dust_debug_philox(torch.from_numpy(ctr.view(np.int32)).cuda(), seed)
+    assert np.array_equal(_dev.host(w).view(np.uint32), words_ref)
+    err = np.abs(_dev.host(zn).astype(np.float64) - z_ref)
+    assert err.max() <= _dev.NORMAL_ATOL, err.max()
+
+
+def test_normals_near_u_one_and_u_zero():
+    """Words whose uniforms sit at the ends of (0, 1): rho -> 0 and rho -> 5.77."""
+    import torch
+    seed = 0x77
+    rng = np.random.default_rng(101)
+    ctr = rng.integers(0, 2**32, size=(1 << 16, 4), dtype=np.uint64).astype(np.uint32)
+    words_ref, z_ref = oracle.philox_batch(ctr, seed)
+    _, zn = z.dust_debug_philox(torch.from_numpy(ctr.view(np.int32)).cuda(), seed)
+    zn = _dev.host(zn).astype(np.float64)
+    u0 = ((words_ref[:, 0] >> 9).astype(np.float64) * 2 + 1) * 2.0**-24
+    extreme = (u0 > 0.999) | (u0 < 0.001)
+    assert extreme.sum() > 50
+    assert np.abs(zn[extreme] - z_ref[extreme]).max() <= _dev.NORMAL_ATOL
+
+
+# ------------------------------------------------------------------------- forward
+def _fwd_case(L, K, sigma, key):
+    import torch
+    x, W, u = _dev.layer_to_device(L)
+    dl = z.dust_noisy_linear_fwd(x, W, u, K, sigma, key)
+    torch.cuda.synchronize()
+    loss, clean = oracle.noisy_linear_loss(L.x_f64, L.W_f64, L.u_f64, K, sigma, key.seed,
+                                           key.layer_id, key.draw_offset, key.token_offset)
+    return _dev.host(dl), loss - clean
+
+
+@pytest.mark.parametrize("N,d_in,d_out,K", [
+    (128, 64, 256, 4),      # one tile
+    (200, 64, 320, 5),      # ragged tokens and channels
+    (385, 144, 528, 3),     # ragged everything, d_in not a multiple of 64
+    (1, 16, 16, 2),         # smallest
+    (700, 768, 512, 8),
+])
+def test_fwd_bf16_matches_oracle(N, d_in, d_out, K):
+    L = workloads.custom_layer(1000 + N, N, d_in, d_out, "bf16", 0.02)
+    key = z.NoiseKey(0x5EED0002, layer_id=3, draw_offset=7, token_offset=11)
+    got, ref = _fwd_case(L, K, 1e-3, key)
+    _dev.assert_fp32_close(got, ref, "dloss")
+
+
+def test_fwd_f32_tiny_workload_matches_oracle():
+    data = workloads.generate(1)
+    L = data.layers[0]
+    wl = data.wl
+    got, ref = _fwd_case(L, wl.K, wl.sigma, z.NoiseKey(wl.seed))
+    _dev.assert_fp32_close(got, ref, "dloss f32")
+
+
+def test_fwd_offsets_above_2_31():
+    L = workloads.custom_layer(5, 130, 32, 48, "bf16", 0.02)
+    key = z.NoiseKey(2**63 + 12345, layer_id=2**31 + 5, draw_offset=2**31 + 3,
+                     token_offset=2**32 - 200)
+    got, ref = _fwd_case(L, 3, 5e-3, key)
+    _dev.assert_fp32_close(got, ref, "dloss offsets")
+
+
+def test_fwd_deterministic():
+    import torch
+    L = workloads.custom_layer(6, 600, 256, 768, "bf16", 0.02)
+    x, W, u = _dev.layer_to_device(L)
+    key = z.NoiseKey(9)
+    a = z.dust_noisy_linear_fwd(x, W, u, 6, 1e-3, key).clone()
+    b = z.dust_noisy_linear_fwd(x, W, u, 6, 1e-3, key)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+# ------------------------------------------------------------------------- credit
+def _credit_gpu(loss_np, cu, gamma):
+    import torch
+    loss = torch.from_numpy(np.ascontiguousarray(loss_np, dtype=np.float32)).cuda()
+    r = z.dust_credit(loss, _dev.cu_to_device(cu), gamma)
+    torch.cuda.synchronize()
+    return _dev.host(r)
+
+
+CREDIT_SEGMENTS = {
+    "single-tokens": lambda N: np.arange(N + 1, dtype=np.int32),
+    "whole-stream": lambda N: np.array([0, N], dtype=np.int32),
+    "straddling": lambda N: workloads.random_segments(31, N, 200, 700),
+    "short": lambda N: workloads.random_segments(32, N, 1, 40),
+    "packed-256-2048": lambda N: workloads.random_segments(33, N, 256, 2048),
+}
+
+
+@pytest.mark.parametrize("seg", list(CREDIT_SEGMENTS))
+@pytest.mark.parametrize("gamma", [0.0, 1.0])
+@pytest.mark.parametrize("K", [2, 8, 32, 128])
+def test_credit_bit_exact_on_integer_losses(seg, gamma, K):
+    """Integer losses in [-8, 8], K a power of two, segments <= 2048 tokens: every mean,
+    centred loss and (for gamma in {0, 1}) every partial sum is a multiple of 1/K below 2^15,
+    exact in fp32 in any order, so the GPU must equal the oracle bit for bit.  This pins the
+    segment resets, the look-back chaining and all indexing."""
+    N = 3000 if K <= 32 else 1500
+    cu = CREDIT_SEGMENTS[seg](N)
+    if seg == "whole-stream" and gamma == 1.0:
+        cu = np.array([0, 1000, N], dtype=np.int32)  # keep every segment <= 2048
+    loss = workloads.dyadic_losses(40 + K, K, N, scale_bits=0, max_abs=8)
+    got = _credit_gpu(loss, cu, gamma)
+    ref = oracle.credit(loss, cu, gamma)
+    assert np.array_equal(got.astype(np.float64), ref), np.abs(got - ref).max()
+
+
+def _credit_tol(ref_c, cu, gamma):
+    """fp32 rounding bound of the reverse scan: each step rounds by 2^-24 relative and the
+    rounding errors decay by gamma, so the error is below a few 2^-24 times the discounted sum
+    of |r| (taken here as 1e-6 x (min(L, 1/(1-gamma)) + 1) x max|r| of the row) plus the
+    centring's rounding."""
+    K, N = ref_c.shape
+    L = np.max(np.diff(cu))
+    eff = min(L, 1.0 / (1.0 - gamma) if gamma < 1 else L) + 1
+    return 2e-6 * eff * np.max(np.abs(ref_c), axis=1, keepdims=True) + 1e-6
+
+
+@pytest.mark.parametrize("gamma", [0.5, 0.9, 0.95, 0.99])
+def test_credit_general_gamma(gamma):
+    K, N = 16, 5000
+    cu = workloads.random_segments(50, N, 1, 1200)
+    loss = workloads.gaussian_losses(51, K, N)
+    got = _credit_gpu(loss, cu, gamma)
+    ref = oracle.credit(loss, cu, gamma)
+    assert np.all(np.abs(got - ref) <= _credit_tol(ref, cu, gamma))
+
+
+def test_credit_ragged_and_minimal_sizes():
+    for N, K in [(1, 2), (255, 3), (257, 5), (513, 64)]:
+        cu = np.array([0, N], dtype=np.int32)
+        loss = workloads.gaussian_losses(60 + N, K, N)
+        got = _credit_gpu(loss, cu, 0.9)
+        ref = oracle.credit(loss, cu, 0.9)
+        assert np.all(np.abs(got - ref) <= _credit_tol(ref, cu, 0.9)), (N, K)
+
+
+def test_credit_timeout_is_reported_and_context_survives():
+    """A block that never publishes makes its predecessor's bounded wait run out: the call
+    reports DUST_ERR_TIMEOUT, writes NaN there, and the next call is correct."""
+    import torch
+    K, N = 4, 256 * 6
+    cu = np.array([0, N], dtype=np.int32)
+    loss = workloads.gaussian_losses(70, K, N)
+    z.dust_debug_credit_skip_publish(3)
+    r = z.dust_credit(torch.from_numpy(loss).cuda(), _dev.cu_to_device(cu), 0.9)
+    st, info = z.dust_last_device_error()
+    # block 2 waits for block 3; blocks 1 and 0 may look past block 2's aggregate and time
+    # out on block 3 themselves, or receive block 2's NaN: either way they are NaN.
+    assert st == z.DUST_ERR_TIMEOUT and 0 <= info <= 2, (st, info)
+    rh = _dev.host(r)
+    assert np.isnan(rh[:, :3 * 256]).all()
+    ref = oracle.credit(loss, cu, 0.9)
+    tail = slice(3 * 256, N)
+    assert np.all(np.abs(rh[:, tail] - ref[:, tail]) <= _credit_tol(ref, cu, 0.9)[:, :1])
+    got = _credit_gpu(loss, cu, 0.9)
+    ref = oracle.credit(loss, cu, 0.9)
+    assert np.all(np.abs(got - ref) <= _credit_tol(ref, cu, 0.9))
+    assert z.dust_last_device_error()[0] == 0
+
+
+# ------------------------------------------------------------------------- weight estimate
+def _wgrad_case(L, K_chunk, K_total, sigma, key, r_seed, dtype):
+    import torch
+    N = L.x_store.shape[0]
+    d_out = L.W_store.shape[0]
+    r = workloads.gaussian_losses(r_seed, K_chunk, N, scale=0.05)
+    x = _dev.to_device(L.x_store, dtype)
+    GW, g = z.dust_weight_grad(torch.from_numpy(r).cuda(), x, d_out, K_total, sigma, key,
+                               g_out=True)
+    torch.cuda.synchronize()
+    g_ref = oracle.output_error(r, K_total, sigma, key.seed, d_out, key.layer_id,
+                                key.draw_offset, key.token_offset)
+    GW_ref = oracle.weight_grad(g_ref, L.x_f64)
+    return _dev.host(GW), _dev.host(g), GW_ref, g_ref
+
+
+@pytest.mark.parametrize("N,d_in,d_out,K", [
+    (256, 256, 128, 4),
+    (300, 272, 144, 6),      # ragged tokens, columns and rows
+    (4100, 768, 512, 8),     # several token tiles: split-K
+    (16, 16, 16, 2),
+])
+def test_weight_grad_bf16_matches_oracle(N, d_in, d_out, K):
+    L = workloads.custom_layer(2000 + N, N, d_in, d_out, "bf16", 0.02)
+    key = z.NoiseKey(0x5EED0003, layer_id=1, draw_offset=40, token_offset=3)
+    GW, g, GW_ref, g_ref = _wgrad_case(L, K, K + 40, 1e-3, key, 80 + N, "bf16")
+    _dev.assert_fp32_close(g, g_ref, "g")
+    assert _dev.rel_fro(GW, GW_ref) <= _dev.GW_FRO, _dev.rel_fro(GW, GW_ref)
+
+
+def test_weight_grad_f32_matches_oracle():
+    L = workloads.custom_layer(3, 128, 64, 64, "f32", None)
+    key = z.NoiseKey(0x5EED0001)
+    GW, g, GW_ref, g_ref = _wgrad_case(L, 8, 8, 1e-2, key, 90, "f32")
+    _dev.assert_fp32_close(g, g_ref, "g f32")
+    _dev.assert_fp32_close(GW, GW_ref, "G_W f32")
+
+
+def test_weight_grad_accumulates_draw_chunks():
+    """Two chunks (draw offsets 0 and K1) with accumulate give the full-population G_W."""
+    import torch
+    N, d_in, d_out, K, K1 = 512, 128, 256, 12, 5
+    L = workloads.custom_layer(7, N, d_in, d_out, "bf16", 0.02)
+    x = _dev.to_device(L.x_store, "bf16")
+    r = workloads.gaussian_losses(91, K, N, scale=0.05)
+    rt = torch.from_numpy(r).cuda()
+    key0 = z.NoiseKey(11, layer_id=4, draw_offset=0)
+    key1 = z.NoiseKey(11, layer_id=4, draw_offset=K1)
+    GW, _ = z.dust_weight_grad(rt[:K1].contiguous(), x, d_out, K, 1e-3, key0)
+    z.dust_weight_grad(rt[K1:].contiguous(), x, d_out, K, 1e-3, key1, G_W=GW, accumulate=True)
+    torch.cuda.synchronize()
+    g_ref = oracle.output_error(r, K, 1e-3, 11, d_out, 4)
+    assert _dev.rel_fro(_dev.host(GW), oracle.weight_grad(g_ref, L.x_f64)) <= _dev.GW_FRO
+
+
+# ------------------------------------------------------------------------- whole chain
+def _chain(L, cu, K, sigma, gamma, key, dtype):
+    import torch
+    x, W, u = (_dev.to_device(a, dtype) for a in (L.x_store, L.W_store, L.u_store))
+    d_out = W.shape[0]
+    dl = z.dust_noisy_linear_fwd(x, W, u, K, sigma, key)
+    r = z.dust_credit(dl, _dev.cu_to_device(cu), gamma)
+    GW, g = z.dust_weight_grad(r, x, d_out, K, sigma, key, g_out=True)
+    torch.cuda.synchronize()
+    return {k: _dev.host(v) for k, v in dict(dloss=dl, r=r, g=g, G_W=GW).items()}
+
+
+@pytest.mark.parametrize("gamma", [0.9, 0.0])
+def test_chain_tiny_f32_workload(gamma):
+    data = workloads.generate(1)
+    L, wl = data.layers[0], data.wl
+    got = _chain(L, data.cu_seqlens, wl.K, wl.sigma, gamma, z.NoiseKey(wl.seed), "f32")
+    ref = oracle.dust_layer(L.x_f64, L.W_f64, L.u_f64, wl.K, wl.sigma, gamma, data.cu_seqlens,
+                            wl.seed)
+    _dev.assert_fp32_close(got["dloss"], ref["loss"] - ref["clean"], "dloss")
+    _dev.assert_fp32_close(got["r"], ref["r"], "r")
+    assert _dev.rel_fro(got["g"], ref["g"]) <= _dev.GW_FRO
+    assert _dev.rel_fro(got["G_W"], ref["G_W"]) <= _dev.GW_FRO
+
+
+def test_chain_bf16_ragged_packed():
+    N, d_in, d_out, K = 1000, 160, 272, 8
+    L = workloads.custom_layer(8, N, d_in, d_out, "bf16", 0.02)
+    cu = workloads.random_segments(9, N, 50, 400)
+    key = z.NoiseKey(0x5EED0003, layer_id=2)
+    got = _chain(L, cu, K, 1e-3, 0.99, key, "bf16")
+    ref = oracle.dust_layer(L.x_f64, L.W_f64, L.u_f64, K, 1e-3, 0.99, cu, key.seed, 2)
+    _dev.assert_fp32_close(got["dloss"], ref["loss"] - ref["clean"], "dloss")
+    assert _dev.rel_fro(got["r"], ref["r"]) <= 1e-4
+    assert _dev.rel_fro(got["g"], ref["g"]) <= _dev.GW_FRO
+    assert _dev.rel_fro(got["G_W"], ref["G_W"]) <= _dev.GW_FRO
+    # the credit sums to zero over draws at every token (centring), to fp32 rounding
+    assert np.abs(got["r"].sum(axis=0)).max() <= 1e-4 * np.abs(got["r"]).max()

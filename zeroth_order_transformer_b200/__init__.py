@@ -1,0 +1,294 @@
+"""Python binding of libdust, the B200 implementation of the Dust token-level
+node-perturbation gradient estimator for one linear layer.
+
+The binding only marshals arguments: it checks tensors, takes their device pointers and the
+current CUDA stream, allocates outputs and workspaces with PyTorch, and calls the C ABI
+declared in ``include/dust.h``.  Every step of the estimator runs in the CUDA kernels of
+``libdust.so``; there is no other code path.  If the library is missing, every call raises.
+
+Function names follow the C ABI:
+  dust_noisy_linear_fwd  per-draw loss change of the noisy layer (noise equation)
+  dust_credit            centred loss and discounted credit (centred-loss, credit equations)
+  dust_weight_grad       output-error estimate g and weight estimate G_W
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import NamedTuple, Optional, Tuple
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdust.so")
+
+DUST_OK = 0
+DUST_ERR_INVALID_ARG = 1
+DUST_ERR_UNSUPPORTED = 2
+DUST_ERR_CUDA = 3
+DUST_ERR_TIMEOUT = 4
+DUST_ERR_WORKSPACE = 5
+
+DUST_F32 = 0
+DUST_BF16 = 1
+
+DUST_OP_NOISY_LINEAR_FWD = 0
+DUST_OP_CREDIT = 1
+DUST_OP_WEIGHT_GRAD = 2
+
+EXPORTED_SYMBOLS = (
+    "dust_noisy_linear_fwd", "dust_credit", "dust_weight_grad", "dust_workspace_size",
+    "dust_status_string", "dust_last_device_error", "dust_debug_philox",
+    "dust_debug_credit_skip_publish", "dust_profile_enable", "dust_profile_disable",
+    "dust_profile_read",
+)
+
+
+class DustError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+class dust_noise_key(ctypes.Structure):
+    _fields_ = [("seed", ctypes.c_uint64), ("layer_id", ctypes.c_uint32),
+                ("draw_offset", ctypes.c_uint32), ("token_offset", ctypes.c_uint32),
+                ("reserved", ctypes.c_uint32)]
+
+
+class NoiseKey(NamedTuple):
+    seed: int
+    layer_id: int = 0
+    draw_offset: int = 0
+    token_offset: int = 0
+
+    def c(self) -> dust_noise_key:
+        return dust_noise_key(self.seed & 0xFFFFFFFFFFFFFFFF, self.layer_id, self.draw_offset,
+                              self.token_offset, 0)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libdust.so; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libdust.so is not built ({LIB_PATH}); run "
+                               "`python -m zeroth_order_transformer_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32, f32, sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32,
+                                 ctypes.c_float, ctypes.c_size_t)
+        L.dust_noisy_linear_fwd.argtypes = [vp, vp, vp, ctypes.c_int, i64, i32, i32, i32, f32,
+                                            dust_noise_key, vp, i64, vp, sz, vp]
+        L.dust_credit.argtypes = [vp, i64, i32, i64, vp, i32, f32, vp, i64, vp, sz, vp]
+        L.dust_weight_grad.argtypes = [vp, i64, vp, ctypes.c_int, i64, i32, i32, i32, i32, f32,
+                                       dust_noise_key, vp, ctypes.c_int, vp, vp, sz, vp]
+        L.dust_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, i64, i32, i32, i32]
+        L.dust_workspace_size.restype = sz
+        L.dust_status_string.argtypes = [ctypes.c_int]
+        L.dust_status_string.restype = ctypes.c_char_p
+        L.dust_last_device_error.argtypes = [vp, ctypes.POINTER(i32)]
+        L.dust_debug_philox.argtypes = [vp, i64, ctypes.c_uint64, vp, vp, vp]
+        L.dust_debug_credit_skip_publish.argtypes = [i32]
+        L.dust_debug_credit_skip_publish.restype = None
+        L.dust_profile_enable.argtypes = [i32]
+        L.dust_profile_enable.restype = ctypes.c_int
+        L.dust_profile_disable.argtypes = []
+        L.dust_profile_disable.restype = None
+        L.dust_profile_read.argtypes = [ctypes.POINTER(ctypes.c_char_p),
+                                        ctypes.POINTER(ctypes.c_float), i32]
+        L.dust_profile_read.restype = i32
+        for name in ("dust_noisy_linear_fwd", "dust_credit", "dust_weight_grad",
+                     "dust_last_device_error", "dust_debug_philox"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().dust_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != DUST_OK:
+        raise DustError(status, where)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return DUST_BF16
+    if t.dtype == torch.float32:
+        return DUST_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; layers are bf16 or fp32")
+
+
+def _cuda(t, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _stream(device, stream) -> int:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return int(stream.cuda_stream)
+
+
+def _workspace(ws, nbytes: int, device):
+    torch = _torch()
+    if nbytes == 0:
+        return None, 0
+    if ws is None or ws.numel() * ws.element_size() < nbytes:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return ws, ws.numel() * ws.element_size()
+
+
+def dust_workspace_size(op: int, dtype: int, N: int, d_in: int, d_out: int, K: int) -> int:
+    return int(lib().dust_workspace_size(op, dtype, N, d_in, d_out, K))
+
+
+def dust_noisy_linear_fwd(x, W, u, K: int, sigma: float, key: NoiseKey, dloss=None,
+                          workspace=None, stream=None):
+    """Per-draw loss change dloss[K, N] (fp32) of the layer W x_t + sigma a_t against u_t."""
+    torch = _torch()
+    _cuda(x, "x"), _cuda(W, "W"), _cuda(u, "u")
+    N, d_in = x.shape
+    d_out = W.shape[0]
+    if W.shape != (d_out, d_in) or u.shape != (N, d_out) or not (x.dtype == W.dtype == u.dtype):
+        raise ValueError("shapes/dtypes: x [N, d_in], W [d_out, d_in], u [N, d_out], one dtype")
+    dt = _dtype_code(x)
+    if dloss is None:
+        dloss = torch.empty((K, N), dtype=torch.float32, device=x.device)
+    _cuda(dloss, "dloss")
+    ws, nb = _workspace(workspace, dust_workspace_size(DUST_OP_NOISY_LINEAR_FWD, dt, N, d_in,
+                                                       d_out, K), x.device)
+    st = lib().dust_noisy_linear_fwd(x.data_ptr(), W.data_ptr(), u.data_ptr(), dt, N, d_in,
+                                     d_out, K, float(sigma), key.c(), dloss.data_ptr(),
+                                     dloss.stride(0), ws.data_ptr() if ws is not None else None,
+                                     nb, _stream(x.device, stream))
+    _check(st, "dust_noisy_linear_fwd")
+    return dloss
+
+
+def dust_credit(loss, cu_seqlens, gamma: float, r=None, workspace=None, stream=None):
+    """Credit r[K, N] from losses [K, N] and int32 cu_seqlens [n_seq + 1] (device)."""
+    torch = _torch()
+    _cuda(loss, "loss"), _cuda(cu_seqlens, "cu_seqlens")
+    if loss.dtype != torch.float32 or cu_seqlens.dtype != torch.int32:
+        raise TypeError("loss must be float32 and cu_seqlens int32")
+    K, N = loss.shape
+    if r is None:
+        r = torch.empty((K, N), dtype=torch.float32, device=loss.device)
+    _cuda(r, "r")
+    ws, nb = _workspace(workspace, dust_workspace_size(DUST_OP_CREDIT, DUST_F32, N, 0, 0, K),
+                        loss.device)
+    st = lib().dust_credit(loss.data_ptr(), loss.stride(0), K, N, cu_seqlens.data_ptr(),
+                           cu_seqlens.numel() - 1, float(gamma), r.data_ptr(), r.stride(0),
+                           ws.data_ptr() if ws is not None else None, nb,
+                           _stream(loss.device, stream))
+    _check(st, "dust_credit")
+    return r
+
+
+def dust_weight_grad(r, x, d_out: int, K_total: int, sigma: float, key: NoiseKey, G_W=None,
+                     accumulate: bool = False, g_out=None, workspace=None, stream=None
+                     ) -> Tuple[object, Optional[object]]:
+    """G_W[d_out, d_in] (fp32) and, if g_out is a tensor or True, g[N, d_out] (fp32)."""
+    torch = _torch()
+    _cuda(r, "r"), _cuda(x, "x")
+    K_chunk, N = r.shape
+    d_in = x.shape[1]
+    dt = _dtype_code(x)
+    if G_W is None:
+        G_W = torch.empty((d_out, d_in), dtype=torch.float32, device=x.device)
+        accumulate = False
+    _cuda(G_W, "G_W")
+    if g_out is True:
+        g_out = torch.empty((N, d_out), dtype=torch.float32, device=x.device)
+    if g_out is False:
+        g_out = None
+    need = dust_workspace_size(DUST_OP_WEIGHT_GRAD, dt, N, d_in, d_out, K_chunk)
+    if dt == DUST_F32 and g_out is not None:
+        need = 0
+    ws, nb = _workspace(workspace, need, x.device)
+    st = lib().dust_weight_grad(r.data_ptr(), r.stride(0), x.data_ptr(), dt, N, d_in, d_out,
+                                K_chunk, K_total, float(sigma), key.c(), G_W.data_ptr(),
+                                1 if accumulate else 0,
+                                g_out.data_ptr() if g_out is not None else None,
+                                ws.data_ptr() if ws is not None else None, nb,
+                                _stream(x.device, stream))
+    _check(st, "dust_weight_grad")
+    return G_W, g_out
+
+
+def dust_last_device_error(stream=None, device=None) -> Tuple[int, int]:
+    """(status, info) of the device error word, which is then cleared."""
+    torch = _torch()
+    dev = device if device is not None else torch.cuda.current_device()
+    info = ctypes.c_int32(0)
+    st = lib().dust_last_device_error(_stream(dev, stream), ctypes.byref(info))
+    return int(st), int(info.value)
+
+
+def dust_debug_philox(ctr, seed: int, stream=None):
+    """Words (uint32 as int64) and fp32 normals for counters ctr [n, 4] (uint32 as int32)."""
+    torch = _torch()
+    _cuda(ctr, "ctr")
+    n = ctr.shape[0]
+    words = torch.empty((n, 4), dtype=torch.int32, device=ctr.device)
+    normals = torch.empty((n, 4), dtype=torch.float32, device=ctr.device)
+    st = lib().dust_debug_philox(ctr.data_ptr(), n, seed & 0xFFFFFFFFFFFFFFFF, words.data_ptr(),
+                                 normals.data_ptr(), _stream(ctr.device, stream))
+    _check(st, "dust_debug_philox")
+    return words, normals
+
+
+def dust_debug_credit_skip_publish(block: int) -> None:
+    lib().dust_debug_credit_skip_publish(int(block))
+
+
+def dust_profile_enable(capacity: int) -> None:
+    _check(lib().dust_profile_enable(int(capacity)), "dust_profile_enable")
+
+
+def dust_profile_disable() -> None:
+    lib().dust_profile_disable()
+
+
+def dust_profile_read(max_records: int = 1 << 16):
+    """[(kernel name, milliseconds)] of the launches recorded since enabling (synchronizes)."""
+    names = (ctypes.c_char_p * max_records)()
+    ms = (ctypes.c_float * max_records)()
+    n = lib().dust_profile_read(names, ms, max_records)
+    return [(names[i].decode(), float(ms[i])) for i in range(n)]
+
+
+class DustLayer:
+    """One layer's estimator with workspaces kept between calls (fwd -> credit -> weight grad)."""
+
+    def __init__(self, N: int, d_in: int, d_out: int, K: int, dtype, device):
+        torch = _torch()
+        dt = DUST_BF16 if dtype == torch.bfloat16 else DUST_F32
+        self.N, self.d_in, self.d_out, self.K = N, d_in, d_out, K
+        nbytes = max(dust_workspace_size(op, dt, N, d_in, d_out, K) for op in range(3))
+        self.ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        self.dloss = torch.empty((K, N), dtype=torch.float32, device=device)
+        self.r = torch.empty((K, N), dtype=torch.float32, device=device)
+        self.G_W = torch.empty((d_out, d_in), dtype=torch.float32, device=device)
+
+    def estimate(self, x, W, u, cu_seqlens, sigma: float, gamma: float, key: NoiseKey,
+                 stream=None):
+        dust_noisy_linear_fwd(x, W, u, self.K, sigma, key, self.dloss, self.ws, stream)
+        dust_credit(self.dloss, cu_seqlens, gamma, self.r, self.ws, stream)
+        dust_weight_grad(self.r, x, self.d_out, self.K, sigma, key, self.G_W, False, None,
+                         self.ws, stream)
+        return self.G_W

@@ -1,0 +1,309 @@
+// C-ABI entry points of libdust: argument validation, workspace checks, the per-device error
+// word, TMA descriptor encoding, and the generator test export.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <mutex>
+#include <vector>
+
+#include "dust_device.cuh"
+#include "dust_internal.h"
+
+namespace dust {
+
+__device__ ErrorWord g_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+int current_device() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return dev;
+}
+
+__global__ void philox_debug_kernel(const uint32_t* __restrict__ ctr, int64_t n, NoiseKey key,
+                                    uint32_t* words, float* normals) {
+    for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < n;
+         j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const uint4 c = reinterpret_cast<const uint4*>(ctr)[j];
+        const U4 w = philox4x32_10(c.x, c.y, c.z, c.w, key.k0, key.k1);
+        if (words) reinterpret_cast<uint4*>(words)[j] = make_uint4(w.x, w.y, w.z, w.w);
+        if (normals) {
+            const F4 z = normal_quad(c.x, c.y, c.z, c.w, key.k0, key.k1);
+            reinterpret_cast<float4*>(normals)[j] = make_float4(z.x, z.y, z.z, z.w);
+        }
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+}  // namespace
+
+ErrorWord* device_error_word() {
+    static ErrorWord* addr[kMaxDevices] = {};
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<ErrorWord*>(p);
+    }
+    return addr[dev];
+}
+
+int num_sms() {
+    static int cache[kMaxDevices] = {};
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return 148;
+    if (!cache[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                       uint32_t box_rows, uint32_t box_cols) {
+    auto fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+namespace {
+struct ProfRecord {
+    const char* name;
+    cudaEvent_t start, stop;
+};
+std::vector<ProfRecord> g_prof;       // completed records
+std::vector<cudaEvent_t> g_prof_pool;  // free events
+int g_prof_capacity = 0;
+bool g_prof_on = false;
+cudaEvent_t g_prof_open = nullptr;
+
+cudaEvent_t prof_event() {
+    if (!g_prof_pool.empty()) {
+        cudaEvent_t e = g_prof_pool.back();
+        g_prof_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+}  // namespace
+
+void prof_begin(cudaStream_t s) {
+    if (!g_prof_on || static_cast<int>(g_prof.size()) >= g_prof_capacity) return;
+    g_prof_open = prof_event();
+    if (g_prof_open) cudaEventRecord(g_prof_open, s);
+}
+
+void prof_end(cudaStream_t s, const char* name) {
+    if (!g_prof_on || !g_prof_open) return;
+    cudaEvent_t stop = prof_event();
+    if (stop) {
+        cudaEventRecord(stop, s);
+        g_prof.push_back(ProfRecord{name, g_prof_open, stop});
+    } else {
+        g_prof_pool.push_back(g_prof_open);
+    }
+    g_prof_open = nullptr;
+}
+
+dust_status philox_debug_launch(const uint32_t* ctr, int64_t n, NoiseKey key, uint32_t* words,
+                                float* normals, cudaStream_t s) {
+    if (n == 0) return DUST_OK;
+    const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, static_cast<int64_t>(num_sms()) * 8));
+    prof_begin(s);
+    philox_debug_kernel<<<blocks, 256, 0, s>>>(ctr, n, key, words, normals);
+    prof_end(s, "philox_debug");
+    return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
+}
+
+}  // namespace dust
+
+using namespace dust;
+
+namespace {
+
+bool valid_dtype(dust_dtype dt) { return dt == DUST_F32 || dt == DUST_BF16; }
+
+dust_status check_layer(const void* x, dust_dtype dt, int64_t N, int32_t d_in, int32_t d_out) {
+    if (!valid_dtype(dt) || !x || N < 1 || d_in < 1 || d_out < 1) return DUST_ERR_INVALID_ARG;
+    if (!aligned16(x)) return DUST_ERR_INVALID_ARG;
+    if (N > 0xFFFFFFFFLL) return DUST_ERR_UNSUPPORTED;  // token index is one counter word
+    if (dt == DUST_BF16 && (d_in % 16 != 0 || d_out % 16 != 0)) return DUST_ERR_UNSUPPORTED;
+    if (dt == DUST_F32 && d_out % 4 != 0) return DUST_ERR_UNSUPPORTED;
+    return DUST_OK;
+}
+
+dust_status check_ws(void* ws, size_t have, size_t need) {
+    if (need == 0) return DUST_OK;
+    if (!ws || !aligned256(ws) || have < need) return DUST_ERR_WORKSPACE;
+    return DUST_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dust_status_string(dust_status s) {
+    switch (s) {
+        case DUST_OK: return "DUST_OK";
+        case DUST_ERR_INVALID_ARG: return "DUST_ERR_INVALID_ARG";
+        case DUST_ERR_UNSUPPORTED: return "DUST_ERR_UNSUPPORTED";
+        case DUST_ERR_CUDA: return "DUST_ERR_CUDA";
+        case DUST_ERR_TIMEOUT: return "DUST_ERR_TIMEOUT";
+        case DUST_ERR_WORKSPACE: return "DUST_ERR_WORKSPACE";
+    }
+    return "DUST_ERR_UNKNOWN";
+}
+
+size_t dust_workspace_size(dust_op op, dust_dtype dt, int64_t N, int32_t d_in, int32_t d_out,
+                           int32_t K) {
+    if (N < 1 || K < 0) return 0;
+    switch (op) {
+        case DUST_OP_NOISY_LINEAR_FWD: return fwd_workspace_bytes(dt, N, d_out, K);
+        case DUST_OP_CREDIT: return credit_workspace_bytes(N, K);
+        case DUST_OP_WEIGHT_GRAD: return wgrad_workspace_bytes(dt, N, d_in, d_out);
+    }
+    return 0;
+}
+
+dust_status dust_noisy_linear_fwd(const void* x, const void* W, const void* u, dust_dtype dt,
+                                  int64_t N, int32_t d_in, int32_t d_out, int32_t K,
+                                  float sigma, dust_noise_key key, float* dloss,
+                                  int64_t ld_dloss, void* workspace, size_t ws_bytes,
+                                  void* stream) {
+    dust_status st = check_layer(x, dt, N, d_in, d_out);
+    if (st != DUST_OK) return st;
+    if (!W || !u || !dloss || !aligned16(W) || !aligned16(u) || !aligned16(dloss))
+        return DUST_ERR_INVALID_ARG;
+    if (K < 1 || ld_dloss < N || !std::isfinite(sigma) || key.reserved != 0)
+        return DUST_ERR_INVALID_ARG;
+    if (static_cast<uint64_t>(key.draw_offset) + static_cast<uint64_t>(K) > 0x100000000ull ||
+        static_cast<uint64_t>(key.token_offset) + static_cast<uint64_t>(N) > 0x100000000ull)
+        return DUST_ERR_INVALID_ARG;
+    st = check_ws(workspace, ws_bytes, fwd_workspace_bytes(dt, N, d_out, K));
+    if (st != DUST_OK) return st;
+    return fwd_launch(x, W, u, dt, N, d_in, d_out, K, sigma, make_key(key), dloss, ld_dloss,
+                      workspace, static_cast<cudaStream_t>(stream));
+}
+
+dust_status dust_credit(const float* loss, int64_t ld_loss, int32_t K, int64_t N,
+                        const int32_t* cu_seqlens, int32_t n_seq, float gamma, float* r,
+                        int64_t ld_r, void* workspace, size_t ws_bytes, void* stream) {
+    if (!loss || !r || !cu_seqlens || N < 1 || K < 2 || n_seq < 1 || ld_loss < N || ld_r < N)
+        return DUST_ERR_INVALID_ARG;
+    if (!(gamma >= 0.f && gamma <= 1.f)) return DUST_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0 || !aligned16(loss) || !aligned16(r))
+        return DUST_ERR_INVALID_ARG;
+    dust_status st = check_ws(workspace, ws_bytes, credit_workspace_bytes(N, K));
+    if (st != DUST_OK) return st;
+    return credit_launch(loss, ld_loss, K, N, cu_seqlens, n_seq, gamma, r, ld_r, workspace,
+                         static_cast<cudaStream_t>(stream));
+}
+
+dust_status dust_weight_grad(const float* r, int64_t ld_r, const void* x, dust_dtype dt,
+                             int64_t N, int32_t d_in, int32_t d_out, int32_t K_chunk,
+                             int32_t K_total, float sigma, dust_noise_key key, float* G_W,
+                             int accumulate, float* g_out, void* workspace, size_t ws_bytes,
+                             void* stream) {
+    dust_status st = check_layer(x, dt, N, d_in, d_out);
+    if (st != DUST_OK) return st;
+    if (!r || !G_W || !aligned16(G_W) || (g_out && !aligned16(g_out))) return DUST_ERR_INVALID_ARG;
+    if (K_chunk < 1 || K_total < K_chunk || ld_r < N || key.reserved != 0)
+        return DUST_ERR_INVALID_ARG;
+    if (!(sigma > 0.f) || !std::isfinite(sigma)) return DUST_ERR_INVALID_ARG;
+    if (static_cast<uint64_t>(key.draw_offset) + static_cast<uint64_t>(K_chunk) > 0x100000000ull ||
+        static_cast<uint64_t>(key.token_offset) + static_cast<uint64_t>(N) > 0x100000000ull)
+        return DUST_ERR_INVALID_ARG;
+    size_t need = wgrad_workspace_bytes(dt, N, d_in, d_out);
+    if (dt == DUST_F32 && g_out) need = 0;
+    st = check_ws(workspace, ws_bytes, need);
+    if (st != DUST_OK) return st;
+    return wgrad_launch(r, ld_r, x, dt, N, d_in, d_out, K_chunk, K_total, sigma, make_key(key),
+                        G_W, accumulate, g_out, workspace, static_cast<cudaStream_t>(stream));
+}
+
+dust_status dust_last_device_error(void* stream, int32_t* info) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DUST_ERR_CUDA;
+    ErrorWord* ew = device_error_word();
+    if (!ew) return DUST_ERR_CUDA;
+    ErrorWord h{0, 0};
+    if (cudaMemcpy(&h, ew, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) return DUST_ERR_CUDA;
+    if (h.code != 0) {
+        const ErrorWord zero{0, 0};
+        if (cudaMemcpy(ew, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess)
+            return DUST_ERR_CUDA;
+    }
+    if (info) *info = h.info;
+    return h.code == 0 ? DUST_OK : static_cast<dust_status>(h.code);
+}
+
+dust_status dust_debug_philox(const uint32_t* ctr, int64_t n, uint64_t seed, uint32_t* words,
+                              float* normals, void* stream) {
+    if (n < 0 || (n > 0 && !ctr)) return DUST_ERR_INVALID_ARG;
+    if ((ctr && !aligned16(ctr)) || (words && !aligned16(words)) || (normals && !aligned16(normals)))
+        return DUST_ERR_INVALID_ARG;
+    dust_noise_key k{seed, 0, 0, 0, 0};
+    return philox_debug_launch(ctr, n, make_key(k), words, normals,
+                               static_cast<cudaStream_t>(stream));
+}
+
+void dust_debug_credit_skip_publish(int32_t block) { g_credit_skip_publish = block; }
+
+dust_status dust_profile_enable(int32_t capacity) {
+    if (capacity < 0) return DUST_ERR_INVALID_ARG;
+    g_prof_capacity = capacity;
+    g_prof_on = capacity > 0;
+    return DUST_OK;
+}
+
+void dust_profile_disable(void) { g_prof_on = false; }
+
+int32_t dust_profile_read(const char** names, float* ms, int32_t max) {
+    cudaDeviceSynchronize();
+    int32_t n = 0;
+    for (const ProfRecord& r : g_prof) {
+        if (n < max) {
+            float t = 0.f;
+            cudaEventElapsedTime(&t, r.start, r.stop);
+            if (names) names[n] = r.name;
+            if (ms) ms[n] = t;
+            ++n;
+        }
+        g_prof_pool.push_back(r.start);
+        g_prof_pool.push_back(r.stop);
+    }
+    g_prof.clear();
+    return n;
+}
+
+}  // extern "C"

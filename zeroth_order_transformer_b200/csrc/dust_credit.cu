@@ -1,0 +1,291 @@
+// Centred loss and discounted credit (Dust review page, section "신용 할당": c_s = mean over
+// draws of l_s minus l_s; r_t = sum_{s >= t} gamma^(s-t) c_s over later tokens of the same
+// sequence).
+//
+// One block per 256 tokens and all K draws.  The block stages its [K, 256] slab of losses in
+// shared memory, centres every token over the draws, and runs, per draw row, a reverse scan
+// of the affine maps r_t = c_t + g_t r_{t+1} (g_t = gamma, or 0 at a segment's last token):
+// each lane composes 8 consecutive tokens serially, the warp composes the 32 lane maps with
+// shuffles.  Blocks are chained from the end of the stream to its start by decoupled
+// look-back: a block publishes its aggregate map (A, G) with r_first = A + G * r_next, then
+// its inclusive value once its successor's is known.  Block indices come from an atomic
+// ticket in reverse order, so a block only ever waits for blocks that started before it.
+// Waits are bounded; a wait that runs out records the error, writes NaN and still publishes,
+// so no other block waits forever.
+#include "dust_device.cuh"
+#include "dust_internal.h"
+
+namespace dust {
+
+int g_credit_skip_publish = -1;
+
+namespace {
+
+constexpr int kCB = 256;       // tokens per block
+constexpr int kThreads = 256;  // 8 warps
+constexpr int kKMax = 128;     // draws held in shared memory at once
+constexpr unsigned kAgg = 1u, kInc = 2u;
+
+struct CreditParams {
+    const float* loss;
+    float* r;
+    const int32_t* cu;
+    unsigned* ticket;
+    unsigned* flags;  // [nblk]
+    float2* agg;      // [nblk, K]
+    float* inc;       // [nblk, K]
+    ErrorWord* ew;
+    int64_t ld_loss, ld_r, N;
+    int n_seq, K, nblk, skip_publish;
+    float gamma;
+};
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+size_t smem_bytes(int K) {
+    return static_cast<size_t>(K) * kCB * 4 + kCB * 4 + static_cast<size_t>(K) * 32 * 4 * 2 +
+           static_cast<size_t>(K) * 4 * 3 + kCB;
+}
+
+__global__ void __launch_bounds__(kThreads) credit_kernel(const CreditParams p) {
+    extern __shared__ float sm[];
+    const int K = p.K;
+    float* slab = sm;                 // [K][kCB]: loss, then c, then r
+    float* exA = slab + K * kCB;      // [K][32]: map of the tokens after each lane's range
+    float* exG = exA + K * 32;
+    float* carry = exG + K * 32;      // [K]: r at the first token after the block
+    float* aggA = carry + K;          // [K]
+    float* aggG = aggA + K;           // [K]
+    float* mean = aggG + K;           // [kCB]
+    unsigned char* isend = reinterpret_cast<unsigned char*>(mean + kCB);  // [kCB]
+    __shared__ int s_blk;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) s_blk = p.nblk - 1 - static_cast<int>(atomicAdd(p.ticket, 1u));
+    __syncthreads();
+    const int b = s_blk;
+    const int64_t t0 = static_cast<int64_t>(b) * kCB;
+    const int nb = static_cast<int>(min(static_cast<int64_t>(kCB), p.N - t0));
+
+    for (int idx = tid; idx < K * kCB; idx += kThreads) {
+        const int i = idx / kCB, j = idx % kCB;
+        slab[idx] = (j < nb) ? __ldg(&p.loss[static_cast<int64_t>(i) * p.ld_loss + t0 + j]) : 0.f;
+    }
+    for (int j = tid; j < kCB; j += kThreads) isend[j] = (j >= nb || t0 + j == p.N - 1) ? 1 : 0;
+    __syncthreads();
+    if (warp == 0) {
+        // segment ends e = cu[s] with t0 < e <= t0 + nb end token e - 1 of this block
+        int lo = 0, hi = p.n_seq + 1;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (static_cast<int64_t>(__ldg(&p.cu[mid])) > t0) hi = mid;
+            else lo = mid + 1;
+        }
+        for (int s = lo + lane; s <= p.n_seq; s += 32) {
+            const int64_t e = __ldg(&p.cu[s]);
+            if (e > t0 + nb) break;
+            if (e > t0) isend[e - 1 - t0] = 1;
+        }
+    }
+    // centring over the draws (the mean includes every draw)
+    for (int j = tid; j < kCB; j += kThreads) {
+        float m = 0.f;
+        for (int i = 0; i < K; ++i) m += slab[i * kCB + j];
+        m = m / static_cast<float>(K);
+        for (int i = 0; i < K; ++i) slab[i * kCB + j] = m - slab[i * kCB + j];
+    }
+    __syncthreads();
+
+    const float gam = p.gamma;
+    for (int i = warp; i < K; i += kThreads / 32) {
+        const float* row = slab + i * kCB + lane * 8;
+        float A = 0.f, G = 1.f;
+#pragma unroll
+        for (int k = 7; k >= 0; --k) {
+            const float g = isend[lane * 8 + k] ? 0.f : gam;
+            A = row[k] + g * A;
+            G = g * G;
+        }
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float A2 = __shfl_down_sync(0xffffffffu, A, off);
+            const float G2 = __shfl_down_sync(0xffffffffu, G, off);
+            if (lane + off < 32) {
+                A = A + G * A2;
+                G = G * G2;
+            }
+        }
+        float eA = __shfl_down_sync(0xffffffffu, A, 1);
+        float eG = __shfl_down_sync(0xffffffffu, G, 1);
+        if (lane == 31) {
+            eA = 0.f;
+            eG = 1.f;
+        }
+        exA[i * 32 + lane] = eA;
+        exG[i * 32 + lane] = eG;
+        if (lane == 0) {
+            aggA[i] = A;
+            aggG[i] = G;
+            p.agg[static_cast<int64_t>(b) * K + i] = make_float2(A, G);
+        }
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        const bool publish = (b != p.skip_publish);
+        if (b == p.nblk - 1) {
+            for (int i = lane; i < K; i += 32) carry[i] = 0.f;
+        } else {
+            if (lane == 0) {
+                __threadfence();
+                if (publish) st_release(&p.flags[b], kAgg);
+            }
+            __syncwarp();
+            constexpr int kRows = kKMax / 32;
+            float accA[kRows], accG[kRows];
+#pragma unroll
+            for (int k = 0; k < kRows; ++k) {
+                accA[k] = 0.f;
+                accG[k] = 1.f;
+            }
+            int j = b + 1;
+            const uint64_t start = global_timer_ns();
+            while (true) {
+                if (j >= p.nblk) {
+#pragma unroll
+                    for (int k = 0; k < kRows; ++k)
+                        if (lane + 32 * k < K) carry[lane + 32 * k] = accA[k];
+                    break;
+                }
+                unsigned st = 0;
+                int timed_out = 0;
+                if (lane == 0) {
+                    st = ld_acquire(&p.flags[j]);
+                    while (st == 0) {
+                        if (global_timer_ns() - start > kWaitLimitNs) {
+                            timed_out = 1;
+                            break;
+                        }
+                        __nanosleep(64);
+                        st = ld_acquire(&p.flags[j]);
+                    }
+                }
+                st = __shfl_sync(0xffffffffu, st, 0);
+                timed_out = __shfl_sync(0xffffffffu, timed_out, 0);
+                __threadfence();
+                if (timed_out) {
+                    if (lane == 0) report_error(p.ew, kDevTimeout, b);
+                    for (int i = lane; i < K; i += 32) carry[i] = __int_as_float(0x7fc00000);
+                    break;
+                }
+                if (st == kInc) {
+#pragma unroll
+                    for (int k = 0; k < kRows; ++k) {
+                        const int i = lane + 32 * k;
+                        if (i < K)
+                            carry[i] = accA[k] + accG[k] * __ldcg(&p.inc[static_cast<int64_t>(j) * K + i]);
+                    }
+                    break;
+                }
+                bool all_zero = true;
+#pragma unroll
+                for (int k = 0; k < kRows; ++k) {
+                    const int i = lane + 32 * k;
+                    if (i < K) {
+                        const float2 a = __ldcg(&p.agg[static_cast<int64_t>(j) * K + i]);
+                        accA[k] = accA[k] + accG[k] * a.x;
+                        accG[k] = accG[k] * a.y;
+                        all_zero = all_zero && (accG[k] == 0.f);
+                    }
+                }
+                if (__all_sync(0xffffffffu, all_zero)) {
+#pragma unroll
+                    for (int k = 0; k < kRows; ++k)
+                        if (lane + 32 * k < K) carry[lane + 32 * k] = accA[k];
+                    break;
+                }
+                ++j;
+            }
+        }
+        for (int i = lane; i < K; i += 32)
+            p.inc[static_cast<int64_t>(b) * K + i] = aggA[i] + aggG[i] * carry[i];
+        __syncwarp();
+        if (lane == 0) {
+            __threadfence();
+            if (publish) st_release(&p.flags[b], kInc);
+        }
+    }
+    __syncthreads();
+
+    for (int i = warp; i < K; i += kThreads / 32) {
+        float* row = slab + i * kCB + lane * 8;
+        float rn = exA[i * 32 + lane] + exG[i * 32 + lane] * carry[i];
+#pragma unroll
+        for (int k = 7; k >= 0; --k) {
+            const float g = isend[lane * 8 + k] ? 0.f : gam;
+            rn = row[k] + g * rn;
+            row[k] = rn;
+        }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < K * kCB; idx += kThreads) {
+        const int i = idx / kCB, j = idx % kCB;
+        if (j < nb) p.r[static_cast<int64_t>(i) * p.ld_r + t0 + j] = slab[idx];
+    }
+}
+
+}  // namespace
+
+size_t credit_workspace_bytes(int64_t N, int32_t K) {
+    const int64_t nblk = (N + kCB - 1) / kCB;
+    return 256 + align_up(static_cast<size_t>(nblk) * 4, 256) +
+           align_up(static_cast<size_t>(nblk) * K * 8, 256) +
+           align_up(static_cast<size_t>(nblk) * K * 4, 256);
+}
+
+dust_status credit_launch(const float* loss, int64_t ld_loss, int32_t K, int64_t N,
+                          const int32_t* cu, int32_t n_seq, float gamma, float* r, int64_t ld_r,
+                          void* ws, cudaStream_t s) {
+    if (K > kKMax) return DUST_ERR_UNSUPPORTED;
+    const int64_t nblk = (N + kCB - 1) / kCB;
+    if (nblk > 2147483647LL) return DUST_ERR_UNSUPPORTED;
+    char* base = static_cast<char*>(ws);
+    CreditParams p;
+    p.loss = loss;
+    p.r = r;
+    p.cu = cu;
+    p.ticket = reinterpret_cast<unsigned*>(base);
+    p.flags = reinterpret_cast<unsigned*>(base + 256);
+    const size_t off_agg = 256 + align_up(static_cast<size_t>(nblk) * 4, 256);
+    p.agg = reinterpret_cast<float2*>(base + off_agg);
+    p.inc = reinterpret_cast<float*>(base + off_agg + align_up(static_cast<size_t>(nblk) * K * 8, 256));
+    p.ew = device_error_word();
+    p.ld_loss = ld_loss;
+    p.ld_r = ld_r;
+    p.N = N;
+    p.n_seq = n_seq;
+    p.K = K;
+    p.nblk = static_cast<int>(nblk);
+    p.skip_publish = g_credit_skip_publish;
+    g_credit_skip_publish = -1;
+    p.gamma = gamma;
+    const size_t smem = smem_bytes(K);
+    if (cudaFuncSetAttribute(credit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return DUST_ERR_CUDA;
+    if (cudaMemsetAsync(base, 0, 256 + static_cast<size_t>(nblk) * 4, s) != cudaSuccess)
+        return DUST_ERR_CUDA;
+    prof_begin(s);
+    credit_kernel<<<static_cast<unsigned>(nblk), kThreads, smem, s>>>(p);
+    prof_end(s, "credit_scan");
+    return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
+}
+
+}  // namespace dust

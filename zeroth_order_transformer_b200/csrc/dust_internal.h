@@ -1,0 +1,66 @@
+// Host-side interface between the C-ABI entry points (dust_api.cu) and the kernel launchers
+// of each stage.  Arguments arrive already validated.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/dust.h"
+
+namespace dust {
+
+struct ErrorWord;
+
+struct NoiseKey {
+    uint32_t k0, k1;        // Philox key words (seed lo32, seed hi32)
+    uint32_t layer;         // fourth counter word
+    uint32_t draw_offset;   // added to the draw index (third counter word)
+    uint32_t token_offset;  // added to the token index (second counter word)
+};
+
+inline NoiseKey make_key(const dust_noise_key& k) {
+    return NoiseKey{static_cast<uint32_t>(k.seed & 0xffffffffu), static_cast<uint32_t>(k.seed >> 32),
+                    k.layer_id, k.draw_offset, k.token_offset};
+}
+
+ErrorWord* device_error_word();  // of the current device
+int num_sms();                   // of the current device
+
+// Encodes a 2-D row-major bf16 tensor [rows, cols] for TMA with a (box_cols x box_rows) box
+// and 128-byte swizzle.  Returns false if the driver rejects it.
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                       uint32_t box_rows, uint32_t box_cols);
+
+// ---- noisy linear forward (dust_fwd.cu)
+size_t fwd_workspace_bytes(dust_dtype dt, int64_t N, int32_t d_out, int32_t K);
+dust_status fwd_launch(const void* x, const void* W, const void* u, dust_dtype dt, int64_t N,
+                       int32_t d_in, int32_t d_out, int32_t K, float sigma, NoiseKey key,
+                       float* dloss, int64_t ld, void* ws, cudaStream_t s);
+
+// ---- credit (dust_credit.cu)
+size_t credit_workspace_bytes(int64_t N, int32_t K);
+dust_status credit_launch(const float* loss, int64_t ld_loss, int32_t K, int64_t N,
+                          const int32_t* cu, int32_t n_seq, float gamma, float* r, int64_t ld_r,
+                          void* ws, cudaStream_t s);
+extern int g_credit_skip_publish;
+
+// ---- weight estimate (dust_wgrad.cu)
+size_t wgrad_workspace_bytes(dust_dtype dt, int64_t N, int32_t d_in, int32_t d_out);
+dust_status wgrad_launch(const float* r, int64_t ld_r, const void* x, dust_dtype dt, int64_t N,
+                         int32_t d_in, int32_t d_out, int32_t K_chunk, int32_t K_total,
+                         float sigma, NoiseKey key, float* G_W, int accumulate, float* g_out,
+                         void* ws, cudaStream_t s);
+
+// ---- generator test export (dust_api.cu)
+dust_status philox_debug_launch(const uint32_t* ctr, int64_t n, NoiseKey key, uint32_t* words,
+                                float* normals, cudaStream_t s);
+
+// Profiling hooks around each kernel launch (no-ops unless dust_profile_enable was called).
+void prof_begin(cudaStream_t s);
+void prof_end(cudaStream_t s, const char* name);
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace dust
