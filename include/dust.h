@@ -124,6 +124,27 @@ dust_status dust_weight_grad(const float* r, int64_t ld_r, const void* x, dust_d
                              int accumulate, float* g_out, void* workspace, size_t ws_bytes,
                              void* stream);
 
+/*
+ * dust_credit without a caller workspace (the paper has no counterpart: this is a packaging
+ * variant for callers that cannot allocate device memory, for example a plugin run by a host
+ * engine that owns every buffer and forbids allocation while it executes, or a process under a
+ * fixed memory budget).  Same arguments, result and errors as dust_credit, minus the
+ * workspace: the look-back scratch lives in a 4 MiB static device array of the library, which
+ * every device that loads the library holds until the process exits.  The call allocates
+ * nothing (no cudaMalloc, no allocating library routine).
+ *   - Sizes whose scratch (dust_workspace_size(DUST_OP_CREDIT, ...)) exceeds 4 MiB are
+ *     rejected with DUST_ERR_WORKSPACE; the scratch is about 12 K + 4 bytes per 256 tokens,
+ *     so K = 32 allows N up to about 2.7 million tokens and K = 64 about 1.4 million.
+ *   - The first call on a device looks up the array's device address (once per device, with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call shares the one array, and the ticket and flags are cleared on `stream` before
+ *     each launch.  Calls whose kernels overlap on the GPU (other streams, other threads)
+ *     race on the scratch and give wrong results: serialize them.
+ */
+dust_status dust_credit_no_alloc(const float* loss, int64_t ld_loss, int32_t K, int64_t N,
+                                 const int32_t* cu_seqlens, int32_t n_seq, float gamma,
+                                 float* r, int64_t ld_r, void* stream);
+
 /* Workspace bytes that `op` needs for these sizes (0 if none).  d_in / d_out are ignored by
  * DUST_OP_CREDIT, K by DUST_OP_WEIGHT_GRAD. */
 size_t dust_workspace_size(dust_op op, dust_dtype dt, int64_t N, int32_t d_in, int32_t d_out,

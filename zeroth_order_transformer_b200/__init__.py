@@ -38,7 +38,7 @@ EXPORTED_SYMBOLS = (
     "dust_noisy_linear_fwd", "dust_credit", "dust_weight_grad", "dust_workspace_size",
     "dust_status_string", "dust_last_device_error", "dust_debug_philox",
     "dust_debug_credit_skip_publish", "dust_profile_enable", "dust_profile_disable",
-    "dust_profile_read",
+    "dust_profile_read", "dust_credit_no_alloc",
 )
 
 
@@ -83,6 +83,8 @@ def lib() -> ctypes.CDLL:
         L.dust_credit.argtypes = [vp, i64, i32, i64, vp, i32, f32, vp, i64, vp, sz, vp]
         L.dust_weight_grad.argtypes = [vp, i64, vp, ctypes.c_int, i64, i32, i32, i32, i32, f32,
                                        dust_noise_key, vp, ctypes.c_int, vp, vp, sz, vp]
+        L.dust_credit_no_alloc.argtypes = [vp, i64, i32, i64, vp, i32, f32, vp, i64, vp]
+        L.dust_credit_no_alloc.restype = ctypes.c_int
         L.dust_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, i64, i32, i32, i32]
         L.dust_workspace_size.restype = sz
         L.dust_status_string.argtypes = [ctypes.c_int]
@@ -196,6 +198,22 @@ def dust_credit(loss, cu_seqlens, gamma: float, r=None, workspace=None, stream=N
                            ws.data_ptr() if ws is not None else None, nb,
                            _stream(loss.device, stream))
     _check(st, "dust_credit")
+    return r
+
+
+def dust_credit_no_alloc(loss, cu_seqlens, gamma: float, r, stream=None):
+    """dust_credit with the library's static 4 MiB scratch instead of a workspace, for callers
+    that cannot allocate device memory; ``r`` must be given (float32 [K, N]).  Calls that
+    overlap on the GPU share the scratch and race: serialize them."""
+    torch = _torch()
+    _cuda(loss, "loss"), _cuda(cu_seqlens, "cu_seqlens"), _cuda(r, "r")
+    if loss.dtype != torch.float32 or r.dtype != torch.float32 or cu_seqlens.dtype != torch.int32:
+        raise TypeError("loss and r must be float32 and cu_seqlens int32")
+    K, N = loss.shape
+    st = lib().dust_credit_no_alloc(loss.data_ptr(), loss.stride(0), K, N, cu_seqlens.data_ptr(),
+                                    cu_seqlens.numel() - 1, float(gamma), r.data_ptr(),
+                                    r.stride(0), _stream(loss.device, stream))
+    _check(st, "dust_credit_no_alloc")
     return r
 
 

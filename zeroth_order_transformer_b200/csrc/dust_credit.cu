@@ -288,4 +288,85 @@ dust_status credit_launch(const float* loss, int64_t ld_loss, int32_t K, int64_t
     return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------------------------------
+// Credit without a caller workspace.  Some callers cannot allocate device memory at all: a
+// plugin run by a host engine that owns every buffer and forbids allocation while it executes,
+// or a process working under a fixed memory budget where a cudaMalloc could fail or stall the
+// device.  For them the look-back scratch (ticket, status flags, per-block aggregates) lives
+// in this fixed device array instead.  Each device that loads the library keeps it until the
+// process exits.
+// ------------------------------------------------------------------------------------------
+constexpr size_t kStaticCreditScratchBytes = 4u << 20;  // 4 MiB per device
+
+static __device__ __align__(256) unsigned char g_credit_scratch[kStaticCreditScratchBytes];
+
+namespace {
+
+// Device address of g_credit_scratch on the current device.  Host code cannot pass the
+// array's name to a kernel (on the host it is only a stand-in symbol), so the address is
+// looked up once per device, with that device current, and cached.
+void* static_credit_scratch() {
+    constexpr int kMaxDev = 64;
+    static void* addr[kMaxDev] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_credit_scratch) != cudaSuccess) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+}  // namespace
+
 }  // namespace dust
+
+extern "C" dust_status dust_credit_no_alloc(const float* loss, int64_t ld_loss, int32_t K,
+                                            int64_t N, const int32_t* cu_seqlens, int32_t n_seq,
+                                            float gamma, float* r, int64_t ld_r, void* stream) {
+    using namespace dust;
+    if (!loss || !r || !cu_seqlens || N < 1 || K < 2 || n_seq < 1 || ld_loss < N || ld_r < N)
+        return DUST_ERR_INVALID_ARG;
+    if (!(gamma >= 0.f && gamma <= 1.f)) return DUST_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0 ||
+        (reinterpret_cast<uintptr_t>(loss) & 15u) != 0 || (reinterpret_cast<uintptr_t>(r) & 15u) != 0)
+        return DUST_ERR_INVALID_ARG;
+    if (K > kKMax) return DUST_ERR_UNSUPPORTED;
+    if (credit_workspace_bytes(N, K) > kStaticCreditScratchBytes) return DUST_ERR_WORKSPACE;
+    void* scratch = static_credit_scratch();
+    if (!scratch) return DUST_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t nblk = (N + kCB - 1) / kCB;
+    char* base = static_cast<char*>(scratch);
+    CreditParams p;
+    p.loss = loss;
+    p.r = r;
+    p.cu = cu_seqlens;
+    p.ticket = reinterpret_cast<unsigned*>(base);
+    p.flags = reinterpret_cast<unsigned*>(base + 256);
+    const size_t off_agg = 256 + align_up(static_cast<size_t>(nblk) * 4, 256);
+    p.agg = reinterpret_cast<float2*>(base + off_agg);
+    p.inc = reinterpret_cast<float*>(base + off_agg + align_up(static_cast<size_t>(nblk) * K * 8, 256));
+    p.ew = device_error_word();
+    p.ld_loss = ld_loss;
+    p.ld_r = ld_r;
+    p.N = N;
+    p.n_seq = n_seq;
+    p.K = K;
+    p.nblk = static_cast<int>(nblk);
+    p.skip_publish = -1;
+    p.gamma = gamma;
+    const size_t smem = smem_bytes(K);
+    if (cudaFuncSetAttribute(credit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return DUST_ERR_CUDA;
+    // The ticket and the status flags must start at zero; the array keeps the previous
+    // call's contents, so they are cleared on the stream before every launch.
+    if (cudaMemsetAsync(base, 0, 256 + static_cast<size_t>(nblk) * 4, s) != cudaSuccess)
+        return DUST_ERR_CUDA;
+    prof_begin(s);
+    credit_kernel<<<static_cast<unsigned>(nblk), kThreads, smem, s>>>(p);
+    prof_end(s, "credit_scan_no_alloc");
+    return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
+}
