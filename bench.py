@@ -289,7 +289,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
             info["tflops"] = round(per_s / 1e12, 2)
         else:
             info["gbs"] = round(per_s / 1e9, 2)
-    dominant = next(iter(kernels)) if kernels else None
+    # dominant kernel: the largest total time among kernels with a defined algorithmic work
+    dominant = next((n for n in kernels if kernel_work(n, wl, s0)[1] is not None), None)
     roofline = None
     if dominant and len(layers) == 1:
         bound, amount, what = kernel_work(dominant, wl, s0)

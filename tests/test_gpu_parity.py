@@ -50,6 +50,7 @@ def test_philox_words_bit_exact_and_normals_close():
     w, zn = z.dust_debug_philox(torch.from_numpy(ctr.view(np.int32)).cuda(), seed)
     assert np.array_equal(_dev.host(w).view(np.uint32), words_ref)
     err = np.abs(_dev.host(zn).astype(np.float64) - z_ref)
+    print(f"max |z_gpu - z_exact| over {4 * n} normals: {err.max():.3e}")
     assert err.max() <= _dev.NORMAL_ATOL, err.max()
 
 
@@ -65,7 +66,9 @@ def test_normals_near_u_one_and_u_zero():
     u0 = ((words_ref[:, 0] >> 9).astype(np.float64) * 2 + 1) * 2.0**-24
     extreme = (u0 > 0.999) | (u0 < 0.001)
     assert extreme.sum() > 50
-    assert np.abs(zn[extreme] - z_ref[extreme]).max() <= _dev.NORMAL_ATOL
+    err = np.abs(zn[extreme] - z_ref[extreme]).max()
+    print(f"max error at u0 < 0.001 or u0 > 0.999: {err:.3e}")
+    assert err <= _dev.NORMAL_ATOL
 
 
 # ------------------------------------------------------------------------- forward

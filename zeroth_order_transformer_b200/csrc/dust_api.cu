@@ -29,10 +29,10 @@ __global__ void philox_debug_kernel(const uint32_t* __restrict__ ctr, int64_t n,
     for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < n;
          j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const uint4 c = reinterpret_cast<const uint4*>(ctr)[j];
-        const U4 w = philox4x32_10(c.x, c.y, c.z, c.w, key.k0, key.k1);
+        const U4 w = philox4x32_10(c.x, c.y, c.z, c.w, key);
         if (words) reinterpret_cast<uint4*>(words)[j] = make_uint4(w.x, w.y, w.z, w.w);
         if (normals) {
-            const F4 z = normal_quad(c.x, c.y, c.z, c.w, key.k0, key.k1);
+            const F4 z = normal_quad(c.x, c.y, c.z, c.w, key);
             reinterpret_cast<float4*>(normals)[j] = make_float4(z.x, z.y, z.z, z.w);
         }
     }

@@ -8,6 +8,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "dust_internal.h"
+
 namespace dust {
 
 // ----------------------------------------------------------------------------------------
@@ -34,35 +36,31 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 // ----------------------------------------------------------------------------------------
-// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): 10 rounds of two 32x32->64 products
-// of counter words 0 and 2 with the round multipliers, XORs with the other two words and
-// the key, and a Weyl-sequence key bump between rounds.
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): 10 rounds; each multiplies counter
+// words 0 and 2 by the two round multipliers into 64-bit products and forms
+// (hi1 ^ c1 ^ key0, lo1, hi0 ^ c3 ^ key1, lo0).  The round keys come precomputed in
+// NoiseKey::rk (parameter space), so each round is two widening multiplies and two
+// three-input XORs.
 // ----------------------------------------------------------------------------------------
 constexpr uint32_t kPhiloxM0 = 0xD2511F53u;
 constexpr uint32_t kPhiloxM1 = 0xCD9E8D57u;
-constexpr uint32_t kPhiloxW0 = 0x9E3779B9u;
-constexpr uint32_t kPhiloxW1 = 0xBB67AE85u;
 
 struct U4 {
     uint32_t x, y, z, w;
 };
 
 __device__ __forceinline__ U4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
-                                            uint32_t k0, uint32_t k1) {
+                                            const NoiseKey& key) {
 #pragma unroll
     for (int round = 0; round < 10; ++round) {
-        const uint32_t lo0 = kPhiloxM0 * c0;
-        const uint32_t hi0 = __umulhi(kPhiloxM0, c0);
-        const uint32_t lo1 = kPhiloxM1 * c2;
-        const uint32_t hi1 = __umulhi(kPhiloxM1, c2);
-        const uint32_t n0 = hi1 ^ c1 ^ k0;
-        const uint32_t n2 = hi0 ^ c3 ^ k1;
+        const uint64_t p0 = static_cast<uint64_t>(kPhiloxM0) * c0;
+        const uint64_t p1 = static_cast<uint64_t>(kPhiloxM1) * c2;
+        const uint32_t n0 = static_cast<uint32_t>(p1 >> 32) ^ c1 ^ key.rk[2 * round];
+        const uint32_t n2 = static_cast<uint32_t>(p0 >> 32) ^ c3 ^ key.rk[2 * round + 1];
+        c1 = static_cast<uint32_t>(p1);
+        c3 = static_cast<uint32_t>(p0);
         c0 = n0;
-        c1 = lo1;
         c2 = n2;
-        c3 = lo0;
-        k0 += kPhiloxW0;
-        k1 += kPhiloxW1;
     }
     return U4{c0, c1, c2, c3};
 }
@@ -73,32 +71,80 @@ __device__ __forceinline__ float uniform_from_word(uint32_t w) {
     return __uint_as_float(0x3f800000u | (w >> 9)) - 0.99999994f;
 }
 
-// Box-Muller: rho = sqrt(-2 ln u0), angle 2 pi u1.  The angle is shifted by -pi into
-// (-pi, pi), where the fast sine/cosine have their documented absolute error bound, and the
-// shift is undone by the sign: cos(x - pi) = -cos x, sin(x - pi) = -sin x.
-__device__ __forceinline__ void box_muller(uint32_t w0, uint32_t w1, float& z0, float& z1) {
-    const float u0 = uniform_from_word(w0);
-    const float u1 = uniform_from_word(w1);
-    const float m2lnu = -2.0f * logf(u0);
-    const float rho = m2lnu * rsqrtf(m2lnu);
-    float s, c;
-    __sincosf(fmaf(u1, 6.28318530717958647692f, -3.14159265358979323846f), &s, &c);
-    z0 = -rho * c;
-    z1 = -rho * s;
+// Hardware approximations (PTX .approx with flush-to-zero; every input here is a normal
+// float): base-2 logarithm, reciprocal square root, sine and cosine in radians.
+__device__ __forceinline__ float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
+__device__ __forceinline__ float rsqrt_approx(float x) {
+    float y;
+    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float sin_approx(float x) {
+    float y;
+    asm("sin.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float cos_approx(float x) {
+    float y;
+    asm("cos.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// X = -2 ln u for u in [2^-24, 1 - 2^-24], from the hardware base-2 logarithm.  Its small
+// absolute error is amplified in rho = sqrt(X) by 1 / (2 rho), which matters only for u close
+// to 1; there (u > 1 - 2^-10) the Taylor series of
+// -2 ln(1 - v) = 2v + v^2 + (2/3) v^3 + (1/2) v^4 + ... in the exact v = 1 - u replaces it (the
+// omitted terms are below v^3 / 4 relative, i.e. under 2^-32).
+__device__ __forceinline__ float neg2_ln_fast(float u) {
+    return -1.3862943611198906f * lg2_approx(u);  // -2 ln(2) log2(u)
+}
+__device__ __forceinline__ float neg2_ln_near_one(float u, float x_fast) {
+    if (u > 0.9990234375f) {
+        const float v = 1.0f - u;
+        return v * fmaf(v, fmaf(v, 0.6666666667f, 1.0f), 2.0f);
+    }
+    return x_fast;
+}
+// Words whose uniform exceeds 1 - 2^-10 have their top ten bits set.
+constexpr uint32_t kNearOneWord = 0xFFC00000u;
 
 struct F4 {
     float x, y, z, w;
 };
 
+// Box-Muller on one Philox block: (w0, w1) -> (z0, z1), (w2, w3) -> (z2, z3), with
+// rho = sqrt(-2 ln u(w0)) and angle 2 pi u(w1).  The angle is shifted by -pi into (-pi, pi),
+// where the hardware sine/cosine keep their absolute error bound, and the shift is undone by
+// the sign: cos(x - pi) = -cos x, sin(x - pi) = -sin x.
+__device__ __forceinline__ F4 box_muller4(const U4& w) {
+    const float u0 = uniform_from_word(w.x);
+    const float u2 = uniform_from_word(w.z);
+    float x0 = neg2_ln_fast(u0);
+    float x2 = neg2_ln_fast(u2);
+    if (max(w.x, w.z) >= kNearOneWord) {  // rare: about 1 block in 500
+        x0 = neg2_ln_near_one(u0, x0);
+        x2 = neg2_ln_near_one(u2, x2);
+    }
+    const float r0 = x0 * rsqrt_approx(x0);
+    const float r2 = x2 * rsqrt_approx(x2);
+    const float a1 = fmaf(uniform_from_word(w.y), 6.28318530717958647692f, -3.14159265358979323846f);
+    const float a3 = fmaf(uniform_from_word(w.w), 6.28318530717958647692f, -3.14159265358979323846f);
+    F4 z;
+    z.x = -r0 * cos_approx(a1);
+    z.y = -r0 * sin_approx(a1);
+    z.z = -r2 * cos_approx(a3);
+    z.w = -r2 * sin_approx(a3);
+    return z;
+}
+
 // The four normals of channels 4q .. 4q+3 of (token, draw, layer).
 __device__ __forceinline__ F4 normal_quad(uint32_t q, uint32_t t, uint32_t i, uint32_t layer,
-                                          uint32_t k0, uint32_t k1) {
-    const U4 w = philox4x32_10(q, t, i, layer, k0, k1);
-    F4 z;
-    box_muller(w.x, w.y, z.x, z.y);
-    box_muller(w.z, w.w, z.z, z.w);
-    return z;
+                                          const NoiseKey& key) {
+    return box_muller4(philox4x32_10(q, t, i, layer, key));
 }
 
 // ----------------------------------------------------------------------------------------

@@ -22,7 +22,8 @@ constexpr int kBM = 128;  // tokens per tile
 constexpr int kBN = 256;  // channels per tile
 constexpr int kBK = 64;   // d_in per pipeline stage (128 bytes of bf16: one swizzle row)
 constexpr int kStages = 2;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;  // 3 groups of 4 warps
+constexpr int kGroups = kThreads / 128;
 constexpr uint32_t kABytes = kBM * kBK * 2;
 constexpr uint32_t kBBytes = kBN * kBK * 2;
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
@@ -129,17 +130,18 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncwarp();
     tc_fence_after();
 
-    // ---------------- epilogue: every warp; TMEM lane quarter = warp % 4.
+    // ---------------- epilogue: every warp; TMEM lane quarter = warp % 4, and the kGroups
+    // warps that share a lane quarter split the work (chunks in phase 1, draws in phase 2).
     const int lq = warp & 3;
-    const int half = warp >> 2;
+    const int grp = warp >> 2;
     const int row = lq * 32 + lane;
     const int64_t t = m0 + row;
     const bool valid = t < p.N;
     const uint32_t trow = tmem + (static_cast<uint32_t>(lq * 32) << 16);
     const int nchunks = min(kBN, p.d_out - n0) / 16;
 
-    // Phase 1: s_e = sigma (y - u), written back in place (each half does alternate chunks).
-    for (int c = half; c < nchunks; c += 2) {
+    // Phase 1: s_e = sigma (y - u), written back in place.
+    for (int c = grp; c < nchunks; c += kGroups) {
         float v[16];
         tmem_ld16(trow + c * 16, v);
         tmem_wait_ld();
@@ -163,28 +165,29 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fence_after();
 
     // Phase 2: per draw, regenerate the noise and sum the loss change over this tile's
-    // channels.  The two warp halves take alternate draws.
+    // channels (four independent partial sums, one per quad of a 16-channel chunk).
     const uint32_t tg = p.key.token_offset + static_cast<uint32_t>(t);
     const uint32_t qbase = static_cast<uint32_t>(n0 >> 2);
     const float h = p.half_sigma2;
-    for (int i = half; i < p.K; i += 2) {
+    for (int i = grp; i < p.K; i += kGroups) {
         const uint32_t di = p.key.draw_offset + static_cast<uint32_t>(i);
-        float acc = 0.f;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
         for (int c = 0; c < nchunks; ++c) {
             float se[16];
             tmem_ld16(trow + c * 16, se);
             tmem_wait_ld();
 #pragma unroll
             for (int qq = 0; qq < 4; ++qq) {
-                const F4 z = normal_quad(qbase + c * 4 + qq, tg, di, p.key.layer, p.key.k0,
-                                         p.key.k1);
-                acc = fmaf(z.x, fmaf(h, z.x, se[4 * qq + 0]), acc);
-                acc = fmaf(z.y, fmaf(h, z.y, se[4 * qq + 1]), acc);
-                acc = fmaf(z.z, fmaf(h, z.z, se[4 * qq + 2]), acc);
-                acc = fmaf(z.w, fmaf(h, z.w, se[4 * qq + 3]), acc);
+                const F4 z = normal_quad(qbase + c * 4 + qq, tg, di, p.key.layer, p.key);
+                acc[qq] = fmaf(z.x, fmaf(h, z.x, se[4 * qq + 0]), acc[qq]);
+                acc[qq] = fmaf(z.y, fmaf(h, z.y, se[4 * qq + 1]), acc[qq]);
+                acc[qq] = fmaf(z.z, fmaf(h, z.z, se[4 * qq + 2]), acc[qq]);
+                acc[qq] = fmaf(z.w, fmaf(h, z.w, se[4 * qq + 3]), acc[qq]);
             }
         }
-        if (valid) p.partial[(static_cast<int64_t>(n_tile) * p.K + i) * p.N + t] = acc;
+        if (valid)
+            p.partial[(static_cast<int64_t>(n_tile) * p.K + i) * p.N + t] =
+                (acc[0] + acc[1]) + (acc[2] + acc[3]);
     }
 
     // Release tensor memory early, then the last channel tile of this token block reduces.
@@ -255,8 +258,7 @@ __global__ void __launch_bounds__(256) fwd_f32_kernel(const FwdF32Params p) {
         float acc = 0.f;
         if (ch_ok[0]) {
             const F4 z = normal_quad(static_cast<uint32_t>(q), tg,
-                                     p.key.draw_offset + static_cast<uint32_t>(i), p.key.layer,
-                                     p.key.k0, p.key.k1);
+                                     p.key.draw_offset + static_cast<uint32_t>(i), p.key.layer, p.key);
             const float zz[4] = {z.x, z.y, z.z, z.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j)

@@ -13,16 +13,28 @@ namespace dust {
 
 struct ErrorWord;
 
+// Philox4x32-10 round keys: key word j of round r is key_j + r * W_j (Weyl sequence with the
+// constants of Salmon et al. 2011).  Computed once on the host so that kernels read them from
+// parameter space instead of recomputing them per thread.
+constexpr uint32_t kPhiloxWeyl0 = 0x9E3779B9u;
+constexpr uint32_t kPhiloxWeyl1 = 0xBB67AE85u;
+
 struct NoiseKey {
     uint32_t k0, k1;        // Philox key words (seed lo32, seed hi32)
     uint32_t layer;         // fourth counter word
     uint32_t draw_offset;   // added to the draw index (third counter word)
     uint32_t token_offset;  // added to the token index (second counter word)
+    uint32_t rk[20];        // round keys: rk[2r] = k0 + r W0, rk[2r+1] = k1 + r W1
 };
 
 inline NoiseKey make_key(const dust_noise_key& k) {
-    return NoiseKey{static_cast<uint32_t>(k.seed & 0xffffffffu), static_cast<uint32_t>(k.seed >> 32),
-                    k.layer_id, k.draw_offset, k.token_offset};
+    NoiseKey n{static_cast<uint32_t>(k.seed & 0xffffffffu), static_cast<uint32_t>(k.seed >> 32),
+               k.layer_id, k.draw_offset, k.token_offset, {}};
+    for (uint32_t r = 0; r < 10; ++r) {
+        n.rk[2 * r] = n.k0 + r * kPhiloxWeyl0;
+        n.rk[2 * r + 1] = n.k1 + r * kPhiloxWeyl1;
+    }
+    return n;
 }
 
 ErrorWord* device_error_word();  // of the current device

@@ -45,8 +45,7 @@ __global__ void __launch_bounds__(kGThreads) ghat_kernel(const GhatParams p) {
         for (int i = 0; i < p.K; ++i) {
             const float ri = __ldg(rt + static_cast<int64_t>(i) * p.ld_r);
             const F4 z = normal_quad(static_cast<uint32_t>(q), tg,
-                                     p.key.draw_offset + static_cast<uint32_t>(i), p.key.layer,
-                                     p.key.k0, p.key.k1);
+                                     p.key.draw_offset + static_cast<uint32_t>(i), p.key.layer, p.key);
             a0 = fmaf(ri, z.x, a0);
             a1 = fmaf(ri, z.y, a1);
             a2 = fmaf(ri, z.z, a2);
