@@ -264,7 +264,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         total_ms = float(t.item())
     ms_per_step = total_ms / args.steps
     units = wl.N * wl.K * len(layers) * world
-    value = units / (ms_per_step / 1e3) / len(layers)  # per layer
+    # tokens*draws per layer processed per second: N K n_layers n_gpus / step time
+    value = units / (ms_per_step / 1e3)
 
     # ---- per-kernel statistics (rank 0's launches)
     per = {}
@@ -359,7 +360,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
             t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e_ms = float(t.item())
-        e2e = {"value": units / (e_ms / args.steps / 1e3) / len(layers), "unit": UNIT,
+        e2e = {"value": units / (e_ms / args.steps / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e_ms / args.steps}
 

@@ -116,35 +116,48 @@ struct F4 {
     float x, y, z, w;
 };
 
-// Box-Muller on one Philox block: (w0, w1) -> (z0, z1), (w2, w3) -> (z2, z3), with
-// rho = sqrt(-2 ln u(w0)) and angle 2 pi u(w1).  The angle is shifted by -pi into (-pi, pi),
-// where the hardware sine/cosine keep their absolute error bound, and the shift is undone by
-// the sign: cos(x - pi) = -cos x, sin(x - pi) = -sin x.
-__device__ __forceinline__ F4 box_muller4(const U4& w) {
+// Box-Muller on one Philox block in polar form: pair p (words 2p, 2p+1) has radius
+// rho_p = sqrt(x_p), x_p = -2 ln u(w_2p), and angle 2 pi u(w_2p+1).  The angle is shifted by
+// -pi into (-pi, pi), where the hardware sine/cosine keep their absolute error bound; the
+// shift flips both signs, cos(x - pi) = -cos x and sin(x - pi) = -sin x, so
+//     z_2p = -rho_p cos_p,   z_2p+1 = -rho_p sin_p,   z_2p^2 + z_2p+1^2 = x_p.
+// Consumers that need sums of a and a^2 use this form directly.
+struct Polar4 {
+    float x0, r0, c0, s0;  // pair 0: channels 4q, 4q+1
+    float x1, r1, c1, s1;  // pair 1: channels 4q+2, 4q+3
+};
+
+__device__ __forceinline__ Polar4 box_muller_polar(const U4& w) {
     const float u0 = uniform_from_word(w.x);
     const float u2 = uniform_from_word(w.z);
-    float x0 = neg2_ln_fast(u0);
-    float x2 = neg2_ln_fast(u2);
+    Polar4 p;
+    p.x0 = neg2_ln_fast(u0);
+    p.x1 = neg2_ln_fast(u2);
     if (max(w.x, w.z) >= kNearOneWord) {  // rare: about 1 block in 500
-        x0 = neg2_ln_near_one(u0, x0);
-        x2 = neg2_ln_near_one(u2, x2);
+        p.x0 = neg2_ln_near_one(u0, p.x0);
+        p.x1 = neg2_ln_near_one(u2, p.x1);
     }
-    const float r0 = x0 * rsqrt_approx(x0);
-    const float r2 = x2 * rsqrt_approx(x2);
+    p.r0 = p.x0 * rsqrt_approx(p.x0);
+    p.r1 = p.x1 * rsqrt_approx(p.x1);
     const float a1 = fmaf(uniform_from_word(w.y), 6.28318530717958647692f, -3.14159265358979323846f);
     const float a3 = fmaf(uniform_from_word(w.w), 6.28318530717958647692f, -3.14159265358979323846f);
-    F4 z;
-    z.x = -r0 * cos_approx(a1);
-    z.y = -r0 * sin_approx(a1);
-    z.z = -r2 * cos_approx(a3);
-    z.w = -r2 * sin_approx(a3);
-    return z;
+    p.c0 = cos_approx(a1);
+    p.s0 = sin_approx(a1);
+    p.c1 = cos_approx(a3);
+    p.s1 = sin_approx(a3);
+    return p;
 }
 
-// The four normals of channels 4q .. 4q+3 of (token, draw, layer).
+__device__ __forceinline__ Polar4 normal_quad_polar(uint32_t q, uint32_t t, uint32_t i,
+                                                    uint32_t layer, const NoiseKey& key) {
+    return box_muller_polar(philox4x32_10(q, t, i, layer, key));
+}
+
+// The four normals a[4q .. 4q+3] of (token, draw, layer).
 __device__ __forceinline__ F4 normal_quad(uint32_t q, uint32_t t, uint32_t i, uint32_t layer,
                                           const NoiseKey& key) {
-    return box_muller4(philox4x32_10(q, t, i, layer, key));
+    const Polar4 p = normal_quad_polar(q, t, i, layer, key);
+    return F4{-p.r0 * p.c0, -p.r0 * p.s0, -p.r1 * p.c1, -p.r1 * p.s1};
 }
 
 // ----------------------------------------------------------------------------------------

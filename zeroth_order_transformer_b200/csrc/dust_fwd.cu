@@ -32,7 +32,7 @@ constexpr uint32_t kTmemCols = 256;
 
 struct FwdParams {
     const __nv_bfloat16* u;
-    float* partial;  // [n_tiles, K, N]
+    float* partial;  // [2 n_tiles, K, N]: (channel tile, half) x draw x token
     float* dloss;    // [K, ld]
     int* counters;   // [m_tiles], zero on entry
     ErrorWord* ew;
@@ -164,29 +164,37 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     tc_fence_after();
 
-    // Phase 2: per draw, regenerate the noise and sum the loss change over this tile's
-    // channels (four independent partial sums, one per quad of a 16-channel chunk).
+    // Phase 2: work units are (draw, half of the tile's channels), dealt round-robin to the
+    // warp groups so that they finish together.  Per unit: regenerate the noise and sum the
+    // loss change over the half's channels.  In polar form a pair (z, z') = -rho (cos, sin)
+    // contributes sigma (z e + z' e') + sigma^2 / 2 (z^2 + z'^2)
+    //           = -rho (cos s_e + sin s_e') + h x,   with x = rho^2 = -2 ln u.
     const uint32_t tg = p.key.token_offset + static_cast<uint32_t>(t);
     const uint32_t qbase = static_cast<uint32_t>(n0 >> 2);
     const float h = p.half_sigma2;
-    for (int i = grp; i < p.K; i += kGroups) {
+    const int half_chunks = (nchunks + 1) / 2;
+    for (int unit = grp; unit < 2 * p.K; unit += kGroups) {
+        const int i = unit >> 1;
+        const int hf = unit & 1;
         const uint32_t di = p.key.draw_offset + static_cast<uint32_t>(i);
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int c = 0; c < nchunks; ++c) {
+        const int c_end = hf ? nchunks : half_chunks;
+        for (int c = hf ? half_chunks : 0; c < c_end; ++c) {
             float se[16];
             tmem_ld16(trow + c * 16, se);
             tmem_wait_ld();
 #pragma unroll
             for (int qq = 0; qq < 4; ++qq) {
-                const F4 z = normal_quad(qbase + c * 4 + qq, tg, di, p.key.layer, p.key);
-                acc[qq] = fmaf(z.x, fmaf(h, z.x, se[4 * qq + 0]), acc[qq]);
-                acc[qq] = fmaf(z.y, fmaf(h, z.y, se[4 * qq + 1]), acc[qq]);
-                acc[qq] = fmaf(z.z, fmaf(h, z.z, se[4 * qq + 2]), acc[qq]);
-                acc[qq] = fmaf(z.w, fmaf(h, z.w, se[4 * qq + 3]), acc[qq]);
+                const Polar4 z = normal_quad_polar(qbase + c * 4 + qq, tg, di, p.key.layer, p.key);
+                const float l0 = fmaf(z.s0, se[4 * qq + 1], z.c0 * se[4 * qq + 0]);
+                const float l1 = fmaf(z.s1, se[4 * qq + 3], z.c1 * se[4 * qq + 2]);
+                acc[qq] = fmaf(-z.r0, l0, acc[qq]);
+                acc[qq] = fmaf(-z.r1, l1, acc[qq]);
+                acc[qq] = fmaf(h, z.x0 + z.x1, acc[qq]);
             }
         }
         if (valid)
-            p.partial[(static_cast<int64_t>(n_tile) * p.K + i) * p.N + t] =
+            p.partial[((static_cast<int64_t>(n_tile) * 2 + hf) * p.K + i) * p.N + t] =
                 (acc[0] + acc[1]) + (acc[2] + acc[3]);
     }
 
@@ -207,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int64_t tt = m0 + (idx % kBM);
             if (tt < p.N) {
                 float s = 0.f;
-                for (int pp = 0; pp < p.n_tiles; ++pp)
+                for (int pp = 0; pp < 2 * p.n_tiles; ++pp)
                     s += __ldcg(&p.partial[(static_cast<int64_t>(pp) * p.K + i) * p.N + tt]);
                 p.dloss[static_cast<int64_t>(i) * p.ld + tt] = s;
             }
@@ -287,7 +295,7 @@ size_t fwd_workspace_bytes(dust_dtype dt, int64_t N, int32_t d_out, int32_t K) {
     if (dt == DUST_BF16) {
         const int64_t n_tiles = (d_out + kBN - 1) / kBN;
         const int64_t m_tiles = (N + kBM - 1) / kBM;
-        return align_up(static_cast<size_t>(n_tiles * K * N) * 4, 256) +
+        return align_up(static_cast<size_t>(2 * n_tiles * K * N) * 4, 256) +
                align_up(static_cast<size_t>(m_tiles) * 4, 256);
     }
     const int64_t n_cb = (d_out + 4 * kF32Quads - 1) / (4 * kF32Quads);
@@ -309,7 +317,7 @@ dust_status fwd_launch(const void* x, const void* W, const void* u, dust_dtype d
         p.u = static_cast<const __nv_bfloat16*>(u);
         p.partial = static_cast<float*>(ws);
         p.counters = reinterpret_cast<int*>(static_cast<char*>(ws) +
-                                            align_up(static_cast<size_t>(n_tiles) * K * N * 4, 256));
+                                            align_up(static_cast<size_t>(2 * n_tiles) * K * N * 4, 256));
         p.dloss = dloss;
         p.ew = device_error_word();
         p.N = N;

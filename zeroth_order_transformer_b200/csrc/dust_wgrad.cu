@@ -42,14 +42,20 @@ __global__ void __launch_bounds__(kGThreads) ghat_kernel(const GhatParams p) {
         const uint32_t tg = p.key.token_offset + static_cast<uint32_t>(t);
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
         const float* rt = p.r + t;
+        // unrolled so that independent Philox chains of consecutive draws interleave
+#pragma unroll 2
         for (int i = 0; i < p.K; ++i) {
             const float ri = __ldg(rt + static_cast<int64_t>(i) * p.ld_r);
-            const F4 z = normal_quad(static_cast<uint32_t>(q), tg,
-                                     p.key.draw_offset + static_cast<uint32_t>(i), p.key.layer, p.key);
-            a0 = fmaf(ri, z.x, a0);
-            a1 = fmaf(ri, z.y, a1);
-            a2 = fmaf(ri, z.z, a2);
-            a3 = fmaf(ri, z.w, a3);
+            const Polar4 z = normal_quad_polar(static_cast<uint32_t>(q), tg,
+                                               p.key.draw_offset + static_cast<uint32_t>(i),
+                                               p.key.layer, p.key);
+            // r a = -(r rho) (cos, sin) per pair
+            const float rr0 = ri * z.r0;
+            const float rr1 = ri * z.r1;
+            a0 = fmaf(-rr0, z.c0, a0);
+            a1 = fmaf(-rr0, z.s0, a1);
+            a2 = fmaf(-rr1, z.c1, a2);
+            a3 = fmaf(-rr1, z.s1, a3);
         }
         a0 *= p.scale;
         a1 *= p.scale;
