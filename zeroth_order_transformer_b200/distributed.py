@@ -1,0 +1,82 @@
+"""Data-parallel plumbing for the Dust estimator across GPUs (one process per GPU).
+
+The estimator shards by tokens.  Each rank takes whole sequences (the credit scan never
+crosses a sequence end), generates the noise of its tokens with their GLOBAL index
+(token_offset), so no noise and no loss is ever exchanged.  The only exchange is the sum
+of the partial weight estimates G_W over ranks: one all-reduce per layer.  This follows the
+pages' remark that zeroth-order training needs to share only seeds and scalars
+(gist.science 2605.15622, seed-based communication; gist.science 2502.10239, seed and scalar
+upload), and the weight-estimate equation of the Dust page (G_W = sum over ALL tokens).
+
+Nothing here computes any step of the estimator; `estimate_sharded` calls the CUDA path.
+"""
+from __future__ import annotations
+
+from typing import List, Sequence, Tuple
+
+import numpy as np
+
+
+def shard_by_sequences(cu_seqlens: Sequence[int], world: int) -> List[Tuple[int, int]]:
+    """Contiguous token ranges [t0, t1), one per rank, made of whole sequences, with token
+    counts as even as the sequence boundaries allow (greedy on the ideal cut points).
+    Ranks may receive an empty range when there are fewer sequences than ranks."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    if cu.ndim != 1 or cu.size < 2 or cu[0] != 0 or np.any(np.diff(cu) < 0):
+        raise ValueError("cu_seqlens must be non-decreasing, start at 0, have >= 2 entries")
+    if world < 1:
+        raise ValueError("world must be >= 1")
+    N = int(cu[-1])
+    cuts = [0]
+    for r in range(1, world):
+        ideal = r * N / world
+        j = int(np.argmin(np.abs(cu - ideal)))
+        cuts.append(max(int(cu[j]), cuts[-1]))
+    cuts.append(N)
+    return [(cuts[r], cuts[r + 1]) for r in range(world)]
+
+
+def local_problem(cu_seqlens: Sequence[int], world: int, rank: int):
+    """(t0, t1, local cu_seqlens as int32) of this rank's shard."""
+    t0, t1 = shard_by_sequences(cu_seqlens, world)[rank]
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    inside = cu[(cu > t0) & (cu < t1)]
+    local = np.concatenate([[0], inside - t0, [t1 - t0]]).astype(np.int32)
+    if t1 == t0:
+        local = np.zeros(1, dtype=np.int32)
+    return t0, t1, local
+
+
+def check_same_problem(group=None, **fields) -> None:
+    """Raise on every rank if the ranks disagree on any field (seed, K, sigma, gamma, layer,
+    shapes): a mismatch would silently combine estimates of different problems."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    mine = tuple(sorted(fields.items()))
+    everyone = [None] * world
+    dist.all_gather_object(everyone, mine, group=group)
+    bad = [r for r, v in enumerate(everyone) if v != mine]
+    if bad:
+        raise RuntimeError(f"ranks {bad} disagree on the estimator problem: {everyone}")
+
+
+def allreduce_weight_estimate(G_W, group=None):
+    """Sum of the per-rank partial weight estimates (in place)."""
+    import torch.distributed as dist
+    dist.all_reduce(G_W, op=dist.ReduceOp.SUM, group=group)
+    return G_W
+
+
+def estimate_sharded(x, W, u, cu_local, K: int, sigma: float, gamma: float, seed: int,
+                     token_offset: int, layer_id: int = 0, group=None, layer=None):
+    """One layer's estimate on this rank's shard (CUDA path), summed over ranks."""
+    from . import DustLayer, NoiseKey
+    import torch
+    N, d_in = x.shape
+    d_out = W.shape[0]
+    if layer is None:
+        layer = DustLayer(N, d_in, d_out, K, x.dtype, x.device)
+    cu = torch.as_tensor(cu_local, dtype=torch.int32, device=x.device)
+    key = NoiseKey(seed, layer_id, 0, token_offset)
+    G_W = layer.estimate(x, W, u, cu, sigma, gamma, key)
+    return allreduce_weight_estimate(G_W, group)
