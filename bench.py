@@ -40,7 +40,8 @@ L2_FLUSH_BYTES = 256 << 20
 # per pair: log, scale, rsqrt, multiply, angle FMA, range scale, sin, cos, 2 products; plus the
 # consumer FMAs: 2 per normal in the forward, 1 in the draw reduction).
 LANES_PER_SM = 128
-OPS_PER_NORMAL = {"fwd_bf16_noise_loss": 20.0, "ghat_reduce_draws": 19.0}
+OPS_PER_NORMAL = {"fwd_bf16_noise_loss": 20.0, "ghat_reduce_draws": 19.0,
+                  "fwd_bf16_noise_loss_grouped": 20.0, "ghat_reduce_draws_grouped": 19.0}
 
 
 def measured_peaks():
@@ -167,17 +168,15 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
-def kernel_work(name, wl, layer):
-    """Algorithmic work of one launch: (bound, amount, unit-scale) for the roofline."""
+def kernel_work(name, wl, shapes):
+    """Algorithmic work of one launch over the given layer shapes: (bound, amount, what)."""
     N, K = wl.N, wl.K
     if name in OPS_PER_NORMAL:
-        return "alu", N * layer.d_out * K, "normals"
-    if name == "gw_bf16_tcgen05":
-        return "tensor", 2.0 * N * layer.d_in * layer.d_out, "flops"
-    if name == "credit_scan":
-        return "hbm", 8.0 * K * N, "bytes"
-    if name == "gw_splitk_reduce":
-        return "hbm", None, "bytes"
+        return "alu", sum(N * s.d_out * K for s in shapes), "normals"
+    if name.startswith("gw_bf16_tcgen05"):
+        return "tensor", sum(2.0 * N * s.d_in * s.d_out for s in shapes), "flops"
+    if name.startswith("credit_scan"):
+        return "hbm", 8.0 * K * N * len(shapes), "bytes"
     return None, None, None
 
 
@@ -219,15 +218,29 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     gamma = wl.gamma
 
+    stacks = {}
+
     def step(inputs=None):
-        for li, (s, x, W, u) in enumerate(inputs or layers):
+        inputs = inputs or layers
+        if len(inputs) > 1:
+            # a block stack: the grouped calls, one launch per step for all layers
+            st = stacks.get(id(inputs))
+            if st is None:
+                st = dust.DustStack([(x, W, u, s.layer_id) for s, x, W, u in inputs], wl.K)
+                stacks[id(inputs)] = st
+            st.estimate(cu, wl.sigma, gamma, wl.seed, 0, rank * wl.N)
+            out = st.G_W
+        else:
+            s, x, W, u = inputs[0]
             key = dust.NoiseKey(wl.seed, s.layer_id, 0, rank * wl.N)
             dust.dust_noisy_linear_fwd(x, W, u, wl.K, wl.sigma, key, dloss, ws)
             dust.dust_credit(dloss, cu, gamma, r, ws)
-            dust.dust_weight_grad(r, x, s.d_out, wl.K, wl.sigma, key, GWs[li], False, None, ws)
+            dust.dust_weight_grad(r, x, s.d_out, wl.K, wl.sigma, key, GWs[0], False, None, ws)
+            out = GWs
         if world > 1:
-            for G in GWs:
+            for G in out:
                 dist.all_reduce(G)
+        return out
 
     stream = torch.cuda.current_stream(dev)
     for _ in range(args.warmup):
@@ -278,10 +291,11 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                    "share": round(t / kern_total, 4) if kern_total else None}
                for n, (c, t) in sorted(per.items(), key=lambda kv: -kv[1][1])}
     s0 = layers[0][0]
+    shapes = [s for s, *_ in layers]
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     for n, info in kernels.items():
-        bound, amount, what = kernel_work(n, wl, s0)
-        if amount is None or len(layers) > 1:
+        bound, amount, what = kernel_work(n, wl, shapes if n.endswith("_grouped") else [s0])
+        if amount is None or (len(layers) > 1 and not n.endswith("_grouped")):
             continue
         per_s = amount / (info["ms_avg"] / 1e3)
         if what == "normals":
@@ -291,10 +305,13 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         else:
             info["gbs"] = round(per_s / 1e9, 2)
     # dominant kernel: the largest total time among kernels with a defined algorithmic work
-    dominant = next((n for n in kernels if kernel_work(n, wl, s0)[1] is not None), None)
+    def work_of(n):
+        return kernel_work(n, wl, shapes if n.endswith("_grouped") else [s0])
+
+    dominant = next((n for n in kernels if work_of(n)[1] is not None), None)
     roofline = None
-    if dominant and len(layers) == 1:
-        bound, amount, what = kernel_work(dominant, wl, s0)
+    if dominant:
+        bound, amount, what = work_of(dominant)
         avg_s = kernels[dominant]["ms_avg"] / 1e3
         if bound == "alu":
             peak = sms * LANES_PER_SM * peaks["sm_max_mhz"] * 1e6 / OPS_PER_NORMAL[dominant] / 1e9
@@ -337,8 +354,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                 dx.copy_(hx, non_blocking=True)
                 dW.copy_(hW, non_blocking=True)
                 du.copy_(hu, non_blocking=True)
-            step(dev_in)
-            for G, hG in zip(GWs, host_out):
+            out = step(dev_in)
+            for G, hG in zip(out, host_out):
                 hG.copy_(G, non_blocking=True)
 
         for _ in range(max(1, args.warmup // 2)):

@@ -145,6 +145,54 @@ dust_status dust_credit_no_alloc(const float* loss, int64_t ld_loss, int32_t K, 
                                  const int32_t* cu_seqlens, int32_t n_seq, float gamma,
                                  float* r, int64_t ld_r, void* stream);
 
+/*
+ * Grouped forms: the same three steps for many bf16 layers that share the token batch
+ * (N tokens, the same sequences, K, sigma, seed), one kernel launch per step for up to 64
+ * layers (more layers take more launches).  A transformer block stack perturbs each linear
+ * layer on its own (Dust page, section "간섭 줄이기": each block and layer type is perturbed
+ * separately with its own noise), so each layer has its own noise (its layer_id) and its own
+ * per-token loss.  Grouping fills the GPU when single layers are too small to.
+ * `layers` is a HOST array of n_layers descriptors; the pointers inside are DEVICE pointers.
+ * Per layer: x [N, d_in], W [d_out, d_in], u [N, d_out] (bf16; d_in, d_out multiples of 16);
+ * dloss fp32 [K, ld_dloss]; r fp32 [K, ld_r]; G_W fp32 [d_out, d_in]; g_out optional fp32
+ * [N, d_out].  key.layer_id is ignored (each descriptor's layer_id is used).  The workspace is
+ * dust_workspace_size_grouped bytes; each layer gets its own region.  dloss and r equal the
+ * single-layer calls bit for bit; G_W can differ by rounding, because the split of the token
+ * sum (split-K) is chosen for the whole group.
+ */
+typedef struct {
+    const void* x;
+    const void* W;
+    const void* u;
+    int32_t d_in, d_out;
+    uint32_t layer_id;
+    uint32_t reserved; /* must be 0 */
+    float* dloss;
+    int64_t ld_dloss;
+    float* r;
+    int64_t ld_r;
+    float* G_W;
+    float* g_out;
+} dust_layer_desc;
+
+/* dust_noisy_linear_fwd for every layer: reads x, W, u; writes dloss. */
+dust_status dust_noisy_linear_fwd_grouped(const dust_layer_desc* layers, int32_t n_layers,
+                                          int64_t N, int32_t K, float sigma, dust_noise_key key,
+                                          void* workspace, size_t ws_bytes, void* stream);
+/* dust_credit for every layer: reads dloss, writes r (cu_seqlens shared by all layers). */
+dust_status dust_credit_grouped(const dust_layer_desc* layers, int32_t n_layers, int32_t K,
+                                int64_t N, const int32_t* cu_seqlens, int32_t n_seq, float gamma,
+                                void* workspace, size_t ws_bytes, void* stream);
+/* dust_weight_grad for every layer: reads r (K_chunk rows) and x; writes (or adds to) G_W and,
+ * where not NULL, g_out. */
+dust_status dust_weight_grad_grouped(const dust_layer_desc* layers, int32_t n_layers, int64_t N,
+                                     int32_t K_chunk, int32_t K_total, float sigma,
+                                     dust_noise_key key, int accumulate, void* workspace,
+                                     size_t ws_bytes, void* stream);
+/* Workspace bytes of a grouped call of step `op`. */
+size_t dust_workspace_size_grouped(dust_op op, const dust_layer_desc* layers, int32_t n_layers,
+                                   int64_t N, int32_t K);
+
 /* Workspace bytes that `op` needs for these sizes (0 if none).  d_in / d_out are ignored by
  * DUST_OP_CREDIT, K by DUST_OP_WEIGHT_GRAD. */
 size_t dust_workspace_size(dust_op op, dust_dtype dt, int64_t N, int32_t d_in, int32_t d_out,

@@ -1,0 +1,80 @@
+"""Grouped calls (several layers sharing one token batch, one launch per step) against the
+single-layer calls and against the oracle."""
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from tests import _dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def z():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import zeroth_order_transformer_b200 as zz
+    zz.lib()
+    return zz
+
+
+def _stack(N, d, seed):
+    """Two blocks of {QKV d->3d, O d->d, W_in d->4d, W_out 4d->d} (layer ids 4b + j)."""
+    rng = np.random.default_rng(seed)
+    shapes = []
+    for b in range(2):
+        shapes += [workloads.LayerShape(d, 3 * d, 4 * b), workloads.LayerShape(d, d, 4 * b + 1),
+                   workloads.LayerShape(d, 4 * d, 4 * b + 2), workloads.LayerShape(4 * d, d, 4 * b + 3)]
+    return [workloads.make_layer(rng, s, N, "bf16", 0.02) for s in shapes]
+
+
+def test_grouped_equals_single_layer_calls(z):
+    import torch
+    N, K, sigma, gamma, seed = 700, 6, 1e-3, 0.9, 0x5EED0005
+    layers = _stack(N, 64, 1)
+    cu = workloads.random_segments(2, N, 50, 300)
+    cu_d = _dev.cu_to_device(cu)
+    dev_layers = [(*_dev.layer_to_device(L), L.shape.layer_id) for L in layers]
+    st = z.DustStack(dev_layers, K, want_g=True)
+    st.estimate(cu_d, sigma, gamma, seed)
+    torch.cuda.synchronize()
+    for l, (x, W, u, lid) in enumerate(dev_layers):
+        key = z.NoiseKey(seed, lid)
+        dl = z.dust_noisy_linear_fwd(x, W, u, K, sigma, key)
+        r = z.dust_credit(dl, cu_d, gamma)
+        GW, g = z.dust_weight_grad(r, x, W.shape[0], K, sigma, key, g_out=True)
+        torch.cuda.synchronize()
+        assert torch.equal(st.dloss[l], dl), l
+        assert torch.equal(st.r[l], r), l
+        assert torch.equal(st.g[l], g), l
+        assert _dev.rel_fro(_dev.host(st.G_W[l]), _dev.host(GW)) < 1e-6, l
+
+
+def test_grouped_stack_matches_oracle(z):
+    import torch
+    N, K, sigma, gamma, seed = 520, 8, 1e-3, 0.99, 0x5EED0005
+    layers = _stack(N, 32, 3)
+    cu = workloads.random_segments(4, N, 64, 256)
+    dev_layers = [(*_dev.layer_to_device(L), L.shape.layer_id) for L in layers]
+    st = z.DustStack(dev_layers, K, want_g=True)
+    st.estimate(_dev.cu_to_device(cu), sigma, gamma, seed)
+    torch.cuda.synchronize()
+    for l, L in enumerate(layers):
+        ref = oracle.dust_layer(L.x_f64, L.W_f64, L.u_f64, K, sigma, gamma, cu, seed,
+                                L.shape.layer_id)
+        _dev.assert_fp32_close(_dev.host(st.dloss[l]), ref["loss"] - ref["clean"], f"dloss {l}")
+        assert _dev.rel_fro(_dev.host(st.g[l]), ref["g"]) <= _dev.GW_FRO, l
+        assert _dev.rel_fro(_dev.host(st.G_W[l]), ref["G_W"]) <= _dev.GW_FRO, l
+
+
+def test_grouped_rejects_bad_descriptors(z):
+    import ctypes
+    d = (z.dust_layer_desc * 1)()
+    d[0].d_in, d[0].d_out = 64, 72          # not a multiple of 16
+    key = z.NoiseKey(1).c()
+    assert z.lib().dust_noisy_linear_fwd_grouped(d, 1, 256, 4, 1e-3, key, None, 0, None) == \
+        z.DUST_ERR_UNSUPPORTED
+    assert z.lib().dust_noisy_linear_fwd_grouped(d, 0, 256, 4, 1e-3, key, None, 0, None) == \
+        z.DUST_ERR_INVALID_ARG

@@ -38,7 +38,8 @@ EXPORTED_SYMBOLS = (
     "dust_noisy_linear_fwd", "dust_credit", "dust_weight_grad", "dust_workspace_size",
     "dust_status_string", "dust_last_device_error", "dust_debug_philox",
     "dust_debug_credit_skip_publish", "dust_profile_enable", "dust_profile_disable",
-    "dust_profile_read", "dust_credit_no_alloc",
+    "dust_profile_read", "dust_credit_no_alloc", "dust_noisy_linear_fwd_grouped",
+    "dust_credit_grouped", "dust_weight_grad_grouped", "dust_workspace_size_grouped",
 )
 
 
@@ -52,6 +53,14 @@ class dust_noise_key(ctypes.Structure):
     _fields_ = [("seed", ctypes.c_uint64), ("layer_id", ctypes.c_uint32),
                 ("draw_offset", ctypes.c_uint32), ("token_offset", ctypes.c_uint32),
                 ("reserved", ctypes.c_uint32)]
+
+
+class dust_layer_desc(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("W", ctypes.c_void_p), ("u", ctypes.c_void_p),
+                ("d_in", ctypes.c_int32), ("d_out", ctypes.c_int32), ("layer_id", ctypes.c_uint32),
+                ("reserved", ctypes.c_uint32), ("dloss", ctypes.c_void_p),
+                ("ld_dloss", ctypes.c_int64), ("r", ctypes.c_void_p), ("ld_r", ctypes.c_int64),
+                ("G_W", ctypes.c_void_p), ("g_out", ctypes.c_void_p)]
 
 
 class NoiseKey(NamedTuple):
@@ -85,6 +94,17 @@ def lib() -> ctypes.CDLL:
                                        dust_noise_key, vp, ctypes.c_int, vp, vp, sz, vp]
         L.dust_credit_no_alloc.argtypes = [vp, i64, i32, i64, vp, i32, f32, vp, i64, vp]
         L.dust_credit_no_alloc.restype = ctypes.c_int
+        dp = ctypes.POINTER(dust_layer_desc)
+        L.dust_noisy_linear_fwd_grouped.argtypes = [dp, i32, i64, i32, f32, dust_noise_key, vp,
+                                                    sz, vp]
+        L.dust_credit_grouped.argtypes = [dp, i32, i32, i64, vp, i32, f32, vp, sz, vp]
+        L.dust_weight_grad_grouped.argtypes = [dp, i32, i64, i32, i32, f32, dust_noise_key,
+                                               ctypes.c_int, vp, sz, vp]
+        L.dust_workspace_size_grouped.argtypes = [ctypes.c_int, dp, i32, i64, i32]
+        L.dust_workspace_size_grouped.restype = sz
+        for name in ("dust_noisy_linear_fwd_grouped", "dust_credit_grouped",
+                     "dust_weight_grad_grouped"):
+            getattr(L, name).restype = ctypes.c_int
         L.dust_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, i64, i32, i32, i32]
         L.dust_workspace_size.restype = sz
         L.dust_status_string.argtypes = [ctypes.c_int]
@@ -288,6 +308,61 @@ def dust_profile_read(max_records: int = 1 << 16):
     ms = (ctypes.c_float * max_records)()
     n = lib().dust_profile_read(names, ms, max_records)
     return [(names[i].decode(), float(ms[i])) for i in range(n)]
+
+
+class DustStack:
+    """Many bf16 layers sharing one token batch (a transformer block stack), estimated with the
+    grouped calls: one launch per step for up to 64 layers.  ``layers`` is a list of
+    (x, W, u, layer_id) device tensors; outputs live in ``dloss[l]``, ``r[l]``, ``G_W[l]``."""
+
+    def __init__(self, layers, K: int, want_g: bool = False):
+        torch = _torch()
+        self.K = K
+        self.layers = layers
+        x0 = layers[0][0]
+        self.N = x0.shape[0]
+        dev = x0.device
+        n = len(layers)
+        self.dloss = [torch.empty((K, self.N), dtype=torch.float32, device=dev) for _ in range(n)]
+        self.r = [torch.empty((K, self.N), dtype=torch.float32, device=dev) for _ in range(n)]
+        self.G_W = [torch.empty((W.shape[0], W.shape[1]), dtype=torch.float32, device=dev)
+                    for (_, W, _, _) in layers]
+        self.g = ([torch.empty((self.N, W.shape[0]), dtype=torch.float32, device=dev)
+                   for (_, W, _, _) in layers] if want_g else None)
+        self.desc = (dust_layer_desc * n)()
+        for l, (x, W, u, layer_id) in enumerate(layers):
+            for t, nm in ((x, "x"), (W, "W"), (u, "u")):
+                _cuda(t, nm)
+                if t.dtype != torch.bfloat16:
+                    raise TypeError("grouped calls take bf16 layers")
+            d = self.desc[l]
+            d.x, d.W, d.u = x.data_ptr(), W.data_ptr(), u.data_ptr()
+            d.d_in, d.d_out = x.shape[1], W.shape[0]
+            d.layer_id, d.reserved = layer_id, 0
+            d.dloss, d.ld_dloss = self.dloss[l].data_ptr(), self.N
+            d.r, d.ld_r = self.r[l].data_ptr(), self.N
+            d.G_W = self.G_W[l].data_ptr()
+            d.g_out = self.g[l].data_ptr() if want_g else None
+        nbytes = max(int(lib().dust_workspace_size_grouped(op, self.desc, n, self.N, K))
+                     for op in range(3))
+        self.ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+
+    def estimate(self, cu_seqlens, sigma: float, gamma: float, seed: int, draw_offset: int = 0,
+                 token_offset: int = 0, stream=None):
+        n = len(self.layers)
+        s = _stream(self.ws.device, stream)
+        nb = self.ws.numel()
+        key = NoiseKey(seed, 0, draw_offset, token_offset).c()
+        _check(lib().dust_noisy_linear_fwd_grouped(self.desc, n, self.N, self.K, float(sigma), key,
+                                                   self.ws.data_ptr(), nb, s),
+               "dust_noisy_linear_fwd_grouped")
+        _check(lib().dust_credit_grouped(self.desc, n, self.K, self.N, cu_seqlens.data_ptr(),
+                                         cu_seqlens.numel() - 1, float(gamma), self.ws.data_ptr(),
+                                         nb, s), "dust_credit_grouped")
+        _check(lib().dust_weight_grad_grouped(self.desc, n, self.N, self.K, self.K, float(sigma),
+                                              key, 0, self.ws.data_ptr(), nb, s),
+               "dust_weight_grad_grouped")
+        return self.G_W
 
 
 class DustLayer:

@@ -279,6 +279,116 @@ dust_status dust_debug_philox(const uint32_t* ctr, int64_t n, uint64_t seed, uin
 
 void dust_debug_credit_skip_publish(int32_t block) { g_credit_skip_publish = block; }
 
+}  // extern "C"
+
+namespace {
+
+dust_status check_group(const dust_layer_desc* layers, int32_t n_layers, int64_t N, int32_t K,
+                        dust_noise_key key, int step) {
+    if (!layers || n_layers < 1 || N < 1 || K < 1 || key.reserved != 0) return DUST_ERR_INVALID_ARG;
+    if (N > 0xFFFFFFFFLL) return DUST_ERR_UNSUPPORTED;
+    if (static_cast<uint64_t>(key.draw_offset) + static_cast<uint64_t>(K) > 0x100000000ull ||
+        static_cast<uint64_t>(key.token_offset) + static_cast<uint64_t>(N) > 0x100000000ull)
+        return DUST_ERR_INVALID_ARG;
+    for (int32_t l = 0; l < n_layers; ++l) {
+        const dust_layer_desc& d = layers[l];
+        if (d.reserved != 0 || d.d_in < 1 || d.d_out < 1) return DUST_ERR_INVALID_ARG;
+        if (d.d_in % 16 != 0 || d.d_out % 16 != 0) return DUST_ERR_UNSUPPORTED;
+        if (step == 0 && (!d.x || !d.W || !d.u || !d.dloss || !aligned16(d.x) || !aligned16(d.W) ||
+                          !aligned16(d.u) || !aligned16(d.dloss) || d.ld_dloss < N))
+            return DUST_ERR_INVALID_ARG;
+        if (step == 1 && (!d.dloss || !d.r || !aligned16(d.dloss) || !aligned16(d.r) ||
+                          d.ld_dloss < N || d.ld_r < N))
+            return DUST_ERR_INVALID_ARG;
+        if (step == 2 && (!d.x || !d.r || !d.G_W || !aligned16(d.x) || !aligned16(d.G_W) ||
+                          (d.g_out && !aligned16(d.g_out)) || d.ld_r < N))
+            return DUST_ERR_INVALID_ARG;
+    }
+    return DUST_OK;
+}
+
+std::vector<FwdLayerArgs> fwd_args(const dust_layer_desc* layers, int32_t n) {
+    std::vector<FwdLayerArgs> v(n);
+    for (int32_t l = 0; l < n; ++l)
+        v[l] = FwdLayerArgs{layers[l].x, layers[l].W, layers[l].u, layers[l].d_in, layers[l].d_out,
+                            layers[l].layer_id, layers[l].dloss, layers[l].ld_dloss};
+    return v;
+}
+
+std::vector<WgradLayerArgs> wgrad_args(const dust_layer_desc* layers, int32_t n) {
+    std::vector<WgradLayerArgs> v(n);
+    for (int32_t l = 0; l < n; ++l)
+        v[l] = WgradLayerArgs{layers[l].r, layers[l].ld_r, layers[l].x, layers[l].d_in,
+                              layers[l].d_out, layers[l].layer_id, layers[l].G_W, layers[l].g_out};
+    return v;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dust_workspace_size_grouped(dust_op op, const dust_layer_desc* layers, int32_t n_layers,
+                                   int64_t N, int32_t K) {
+    if (!layers || n_layers < 1 || N < 1 || K < 0) return 0;
+    switch (op) {
+        case DUST_OP_NOISY_LINEAR_FWD: {
+            auto a = fwd_args(layers, n_layers);
+            return fwd_grouped_workspace_bytes(a.data(), n_layers, N, K);
+        }
+        case DUST_OP_CREDIT: return credit_grouped_workspace_bytes(n_layers, N, K);
+        case DUST_OP_WEIGHT_GRAD: {
+            auto a = wgrad_args(layers, n_layers);
+            return wgrad_grouped_workspace_bytes(a.data(), n_layers, N);
+        }
+    }
+    return 0;
+}
+
+dust_status dust_noisy_linear_fwd_grouped(const dust_layer_desc* layers, int32_t n_layers,
+                                          int64_t N, int32_t K, float sigma, dust_noise_key key,
+                                          void* workspace, size_t ws_bytes, void* stream) {
+    dust_status st = check_group(layers, n_layers, N, K, key, 0);
+    if (st != DUST_OK) return st;
+    if (!std::isfinite(sigma)) return DUST_ERR_INVALID_ARG;
+    auto a = fwd_args(layers, n_layers);
+    st = check_ws(workspace, ws_bytes, fwd_grouped_workspace_bytes(a.data(), n_layers, N, K));
+    if (st != DUST_OK) return st;
+    return fwd_grouped_launch(a.data(), n_layers, N, K, sigma, make_key(key), workspace,
+                              static_cast<cudaStream_t>(stream));
+}
+
+dust_status dust_credit_grouped(const dust_layer_desc* layers, int32_t n_layers, int32_t K,
+                                int64_t N, const int32_t* cu_seqlens, int32_t n_seq, float gamma,
+                                void* workspace, size_t ws_bytes, void* stream) {
+    dust_noise_key none{0, 0, 0, 0, 0};
+    dust_status st = check_group(layers, n_layers, N, K, none, 1);
+    if (st != DUST_OK) return st;
+    if (!cu_seqlens || n_seq < 1 || K < 2 || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0)
+        return DUST_ERR_INVALID_ARG;
+    if (!(gamma >= 0.f && gamma <= 1.f)) return DUST_ERR_INVALID_ARG;
+    st = check_ws(workspace, ws_bytes, credit_grouped_workspace_bytes(n_layers, N, K));
+    if (st != DUST_OK) return st;
+    std::vector<CreditLayerArgs> a(n_layers);
+    for (int32_t l = 0; l < n_layers; ++l)
+        a[l] = CreditLayerArgs{layers[l].dloss, layers[l].ld_dloss, layers[l].r, layers[l].ld_r};
+    return credit_grouped_launch(a.data(), n_layers, K, N, cu_seqlens, n_seq, gamma, workspace,
+                                 static_cast<cudaStream_t>(stream));
+}
+
+dust_status dust_weight_grad_grouped(const dust_layer_desc* layers, int32_t n_layers, int64_t N,
+                                     int32_t K_chunk, int32_t K_total, float sigma,
+                                     dust_noise_key key, int accumulate, void* workspace,
+                                     size_t ws_bytes, void* stream) {
+    dust_status st = check_group(layers, n_layers, N, K_chunk, key, 2);
+    if (st != DUST_OK) return st;
+    if (K_total < K_chunk || !(sigma > 0.f) || !std::isfinite(sigma)) return DUST_ERR_INVALID_ARG;
+    auto a = wgrad_args(layers, n_layers);
+    st = check_ws(workspace, ws_bytes, wgrad_grouped_workspace_bytes(a.data(), n_layers, N));
+    if (st != DUST_OK) return st;
+    return wgrad_grouped_launch(a.data(), n_layers, N, K_chunk, K_total, sigma, make_key(key),
+                                accumulate, workspace, static_cast<cudaStream_t>(stream));
+}
+
 dust_status dust_profile_enable(int32_t capacity) {
     if (capacity < 0) return DUST_ERR_INVALID_ARG;
     g_prof_capacity = capacity;

@@ -26,16 +26,24 @@ constexpr int kThreads = 256;  // 8 warps
 constexpr int kKMax = 128;     // draws held in shared memory at once
 constexpr unsigned kAgg = 1u, kInc = 2u;
 
-struct CreditParams {
+struct CreditLayer {
     const float* loss;
     float* r;
-    const int32_t* cu;
     unsigned* ticket;
     unsigned* flags;  // [nblk]
     float2* agg;      // [nblk, K]
     float* inc;       // [nblk, K]
+    int64_t ld_loss, ld_r;
+};
+
+// One launch covers the layers of the table (blockIdx.y = layer); every layer has its own
+// ticket and look-back state, so blocks of different layers never wait for one another.
+template <int kMax>
+struct CreditTable {
+    CreditLayer layer[kMax];
+    const int32_t* cu;
     ErrorWord* ew;
-    int64_t ld_loss, ld_r, N;
+    int64_t N;
     int n_seq, K, nblk, skip_publish;
     float gamma;
 };
@@ -54,9 +62,11 @@ size_t smem_bytes(int K) {
            static_cast<size_t>(K) * 4 * 3 + kCB;
 }
 
-__global__ void __launch_bounds__(kThreads) credit_kernel(const CreditParams p) {
+template <int kMax>
+__global__ void __launch_bounds__(kThreads) credit_kernel(const __grid_constant__ CreditTable<kMax> T) {
+    const CreditLayer& L = T.layer[blockIdx.y];
     extern __shared__ float sm[];
-    const int K = p.K;
+    const int K = T.K;
     float* slab = sm;                 // [K][kCB]: loss, then c, then r
     float* exA = slab + K * kCB;      // [K][32]: map of the tokens after each lane's range
     float* exG = exA + K * 32;
@@ -68,28 +78,28 @@ __global__ void __launch_bounds__(kThreads) credit_kernel(const CreditParams p) 
     __shared__ int s_blk;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (tid == 0) s_blk = p.nblk - 1 - static_cast<int>(atomicAdd(p.ticket, 1u));
+    if (tid == 0) s_blk = T.nblk - 1 - static_cast<int>(atomicAdd(L.ticket, 1u));
     __syncthreads();
     const int b = s_blk;
     const int64_t t0 = static_cast<int64_t>(b) * kCB;
-    const int nb = static_cast<int>(min(static_cast<int64_t>(kCB), p.N - t0));
+    const int nb = static_cast<int>(min(static_cast<int64_t>(kCB), T.N - t0));
 
     for (int idx = tid; idx < K * kCB; idx += kThreads) {
         const int i = idx / kCB, j = idx % kCB;
-        slab[idx] = (j < nb) ? __ldg(&p.loss[static_cast<int64_t>(i) * p.ld_loss + t0 + j]) : 0.f;
+        slab[idx] = (j < nb) ? __ldg(&L.loss[static_cast<int64_t>(i) * L.ld_loss + t0 + j]) : 0.f;
     }
-    for (int j = tid; j < kCB; j += kThreads) isend[j] = (j >= nb || t0 + j == p.N - 1) ? 1 : 0;
+    for (int j = tid; j < kCB; j += kThreads) isend[j] = (j >= nb || t0 + j == T.N - 1) ? 1 : 0;
     __syncthreads();
     if (warp == 0) {
         // segment ends e = cu[s] with t0 < e <= t0 + nb end token e - 1 of this block
-        int lo = 0, hi = p.n_seq + 1;
+        int lo = 0, hi = T.n_seq + 1;
         while (lo < hi) {
             const int mid = (lo + hi) >> 1;
-            if (static_cast<int64_t>(__ldg(&p.cu[mid])) > t0) hi = mid;
+            if (static_cast<int64_t>(__ldg(&T.cu[mid])) > t0) hi = mid;
             else lo = mid + 1;
         }
-        for (int s = lo + lane; s <= p.n_seq; s += 32) {
-            const int64_t e = __ldg(&p.cu[s]);
+        for (int s = lo + lane; s <= T.n_seq; s += 32) {
+            const int64_t e = __ldg(&T.cu[s]);
             if (e > t0 + nb) break;
             if (e > t0) isend[e - 1 - t0] = 1;
         }
@@ -103,7 +113,7 @@ __global__ void __launch_bounds__(kThreads) credit_kernel(const CreditParams p) 
     }
     __syncthreads();
 
-    const float gam = p.gamma;
+    const float gam = T.gamma;
     for (int i = warp; i < K; i += kThreads / 32) {
         const float* row = slab + i * kCB + lane * 8;
         float A = 0.f, G = 1.f;
@@ -133,19 +143,19 @@ __global__ void __launch_bounds__(kThreads) credit_kernel(const CreditParams p) 
         if (lane == 0) {
             aggA[i] = A;
             aggG[i] = G;
-            p.agg[static_cast<int64_t>(b) * K + i] = make_float2(A, G);
+            L.agg[static_cast<int64_t>(b) * K + i] = make_float2(A, G);
         }
     }
     __syncthreads();
 
     if (warp == 0) {
-        const bool publish = (b != p.skip_publish);
-        if (b == p.nblk - 1) {
+        const bool publish = (b != T.skip_publish);
+        if (b == T.nblk - 1) {
             for (int i = lane; i < K; i += 32) carry[i] = 0.f;
         } else {
             if (lane == 0) {
                 __threadfence();
-                if (publish) st_release(&p.flags[b], kAgg);
+                if (publish) st_release(&L.flags[b], kAgg);
             }
             __syncwarp();
             constexpr int kRows = kKMax / 32;
@@ -158,7 +168,7 @@ __global__ void __launch_bounds__(kThreads) credit_kernel(const CreditParams p) 
             int j = b + 1;
             const uint64_t start = global_timer_ns();
             while (true) {
-                if (j >= p.nblk) {
+                if (j >= T.nblk) {
 #pragma unroll
                     for (int k = 0; k < kRows; ++k)
                         if (lane + 32 * k < K) carry[lane + 32 * k] = accA[k];
@@ -167,21 +177,21 @@ __global__ void __launch_bounds__(kThreads) credit_kernel(const CreditParams p) 
                 unsigned st = 0;
                 int timed_out = 0;
                 if (lane == 0) {
-                    st = ld_acquire(&p.flags[j]);
+                    st = ld_acquire(&L.flags[j]);
                     while (st == 0) {
                         if (global_timer_ns() - start > kWaitLimitNs) {
                             timed_out = 1;
                             break;
                         }
                         __nanosleep(64);
-                        st = ld_acquire(&p.flags[j]);
+                        st = ld_acquire(&L.flags[j]);
                     }
                 }
                 st = __shfl_sync(0xffffffffu, st, 0);
                 timed_out = __shfl_sync(0xffffffffu, timed_out, 0);
                 __threadfence();
                 if (timed_out) {
-                    if (lane == 0) report_error(p.ew, kDevTimeout, b);
+                    if (lane == 0) report_error(T.ew, kDevTimeout, b);
                     for (int i = lane; i < K; i += 32) carry[i] = __int_as_float(0x7fc00000);
                     break;
                 }
@@ -190,7 +200,7 @@ __global__ void __launch_bounds__(kThreads) credit_kernel(const CreditParams p) 
                     for (int k = 0; k < kRows; ++k) {
                         const int i = lane + 32 * k;
                         if (i < K)
-                            carry[i] = accA[k] + accG[k] * __ldcg(&p.inc[static_cast<int64_t>(j) * K + i]);
+                            carry[i] = accA[k] + accG[k] * __ldcg(&L.inc[static_cast<int64_t>(j) * K + i]);
                     }
                     break;
                 }
@@ -199,7 +209,7 @@ __global__ void __launch_bounds__(kThreads) credit_kernel(const CreditParams p) 
                 for (int k = 0; k < kRows; ++k) {
                     const int i = lane + 32 * k;
                     if (i < K) {
-                        const float2 a = __ldcg(&p.agg[static_cast<int64_t>(j) * K + i]);
+                        const float2 a = __ldcg(&L.agg[static_cast<int64_t>(j) * K + i]);
                         accA[k] = accA[k] + accG[k] * a.x;
                         accG[k] = accG[k] * a.y;
                         all_zero = all_zero && (accG[k] == 0.f);
@@ -215,11 +225,11 @@ __global__ void __launch_bounds__(kThreads) credit_kernel(const CreditParams p) 
             }
         }
         for (int i = lane; i < K; i += 32)
-            p.inc[static_cast<int64_t>(b) * K + i] = aggA[i] + aggG[i] * carry[i];
+            L.inc[static_cast<int64_t>(b) * K + i] = aggA[i] + aggG[i] * carry[i];
         __syncwarp();
         if (lane == 0) {
             __threadfence();
-            if (publish) st_release(&p.flags[b], kInc);
+            if (publish) st_release(&L.flags[b], kInc);
         }
     }
     __syncthreads();
@@ -237,7 +247,7 @@ __global__ void __launch_bounds__(kThreads) credit_kernel(const CreditParams p) 
     __syncthreads();
     for (int idx = tid; idx < K * kCB; idx += kThreads) {
         const int i = idx / kCB, j = idx % kCB;
-        if (j < nb) p.r[static_cast<int64_t>(i) * p.ld_r + t0 + j] = slab[idx];
+        if (j < nb) L.r[static_cast<int64_t>(i) * L.ld_r + t0 + j] = slab[idx];
     }
 }
 
@@ -250,42 +260,96 @@ size_t credit_workspace_bytes(int64_t N, int32_t K) {
            align_up(static_cast<size_t>(nblk) * K * 4, 256);
 }
 
+namespace {
+
+// Points a layer's look-back state at `base` (credit_workspace_bytes(N, K) bytes) and clears
+// the ticket and flags on the stream.
+bool place_credit_state(CreditLayer& L, char* base, int64_t nblk, int32_t K, cudaStream_t s) {
+    L.ticket = reinterpret_cast<unsigned*>(base);
+    L.flags = reinterpret_cast<unsigned*>(base + 256);
+    const size_t off_agg = 256 + align_up(static_cast<size_t>(nblk) * 4, 256);
+    L.agg = reinterpret_cast<float2*>(base + off_agg);
+    L.inc = reinterpret_cast<float*>(base + off_agg + align_up(static_cast<size_t>(nblk) * K * 8, 256));
+    return cudaMemsetAsync(base, 0, 256 + static_cast<size_t>(nblk) * 4, s) == cudaSuccess;
+}
+
+template <int kMax>
+dust_status launch_credit_table(const CreditTable<kMax>& T, int n_layers, cudaStream_t s,
+                                const char* name) {
+    const size_t smem = smem_bytes(T.K);
+    if (cudaFuncSetAttribute(credit_kernel<kMax>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return DUST_ERR_CUDA;
+    prof_begin(s);
+    credit_kernel<kMax><<<dim3(static_cast<unsigned>(T.nblk), static_cast<unsigned>(n_layers)),
+                          kThreads, smem, s>>>(T);
+    prof_end(s, name);
+    return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
+}
+
+template <int kMax>
+void fill_common(CreditTable<kMax>& T, const int32_t* cu, int32_t n_seq, int32_t K, int64_t N,
+                 float gamma, int skip) {
+    T.cu = cu;
+    T.ew = device_error_word();
+    T.N = N;
+    T.n_seq = n_seq;
+    T.K = K;
+    T.nblk = static_cast<int>((N + kCB - 1) / kCB);
+    T.skip_publish = skip;
+    T.gamma = gamma;
+}
+
+constexpr int kMaxGroup = 64;
+
+}  // namespace
+
 dust_status credit_launch(const float* loss, int64_t ld_loss, int32_t K, int64_t N,
                           const int32_t* cu, int32_t n_seq, float gamma, float* r, int64_t ld_r,
                           void* ws, cudaStream_t s) {
     if (K > kKMax) return DUST_ERR_UNSUPPORTED;
     const int64_t nblk = (N + kCB - 1) / kCB;
     if (nblk > 2147483647LL) return DUST_ERR_UNSUPPORTED;
-    char* base = static_cast<char*>(ws);
-    CreditParams p;
-    p.loss = loss;
-    p.r = r;
-    p.cu = cu;
-    p.ticket = reinterpret_cast<unsigned*>(base);
-    p.flags = reinterpret_cast<unsigned*>(base + 256);
-    const size_t off_agg = 256 + align_up(static_cast<size_t>(nblk) * 4, 256);
-    p.agg = reinterpret_cast<float2*>(base + off_agg);
-    p.inc = reinterpret_cast<float*>(base + off_agg + align_up(static_cast<size_t>(nblk) * K * 8, 256));
-    p.ew = device_error_word();
-    p.ld_loss = ld_loss;
-    p.ld_r = ld_r;
-    p.N = N;
-    p.n_seq = n_seq;
-    p.K = K;
-    p.nblk = static_cast<int>(nblk);
-    p.skip_publish = g_credit_skip_publish;
+    CreditTable<1> T;
+    fill_common(T, cu, n_seq, K, N, gamma, g_credit_skip_publish);
     g_credit_skip_publish = -1;
-    p.gamma = gamma;
-    const size_t smem = smem_bytes(K);
-    if (cudaFuncSetAttribute(credit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-        return DUST_ERR_CUDA;
-    if (cudaMemsetAsync(base, 0, 256 + static_cast<size_t>(nblk) * 4, s) != cudaSuccess)
-        return DUST_ERR_CUDA;
-    prof_begin(s);
-    credit_kernel<<<static_cast<unsigned>(nblk), kThreads, smem, s>>>(p);
-    prof_end(s, "credit_scan");
-    return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
+    T.layer[0].loss = loss;
+    T.layer[0].r = r;
+    T.layer[0].ld_loss = ld_loss;
+    T.layer[0].ld_r = ld_r;
+    if (!place_credit_state(T.layer[0], static_cast<char*>(ws), nblk, K, s)) return DUST_ERR_CUDA;
+    return launch_credit_table(T, 1, s, "credit_scan");
+}
+
+size_t credit_grouped_workspace_bytes(int n_layers, int64_t N, int32_t K) {
+    return static_cast<size_t>(n_layers) * credit_workspace_bytes(N, K);
+}
+
+dust_status credit_grouped_launch(const CreditLayerArgs* layers, int n, int32_t K, int64_t N,
+                                  const int32_t* cu, int32_t n_seq, float gamma, void* ws,
+                                  cudaStream_t s) {
+    if (K > kKMax) return DUST_ERR_UNSUPPORTED;
+    const int64_t nblk = (N + kCB - 1) / kCB;
+    if (nblk > 2147483647LL) return DUST_ERR_UNSUPPORTED;
+    char* base = static_cast<char*>(ws);
+    const size_t per = credit_workspace_bytes(N, K);
+    for (int l0 = 0; l0 < n; l0 += kMaxGroup) {
+        const int cnt = n - l0 < kMaxGroup ? n - l0 : kMaxGroup;
+        CreditTable<kMaxGroup> T;
+        fill_common(T, cu, n_seq, K, N, gamma, -1);
+        for (int l = 0; l < cnt; ++l) {
+            CreditLayer& L = T.layer[l];
+            L.loss = layers[l0 + l].loss;
+            L.r = layers[l0 + l].r;
+            L.ld_loss = layers[l0 + l].ld_loss;
+            L.ld_r = layers[l0 + l].ld_r;
+            if (!place_credit_state(L, base, nblk, K, s)) return DUST_ERR_CUDA;
+            base += per;
+        }
+        const dust_status st = launch_credit_table(T, cnt, s, "credit_scan_grouped");
+        if (st != DUST_OK) return st;
+    }
+    return DUST_OK;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -338,35 +402,15 @@ extern "C" dust_status dust_credit_no_alloc(const float* loss, int64_t ld_loss, 
     if (!scratch) return DUST_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t nblk = (N + kCB - 1) / kCB;
-    char* base = static_cast<char*>(scratch);
-    CreditParams p;
-    p.loss = loss;
-    p.r = r;
-    p.cu = cu_seqlens;
-    p.ticket = reinterpret_cast<unsigned*>(base);
-    p.flags = reinterpret_cast<unsigned*>(base + 256);
-    const size_t off_agg = 256 + align_up(static_cast<size_t>(nblk) * 4, 256);
-    p.agg = reinterpret_cast<float2*>(base + off_agg);
-    p.inc = reinterpret_cast<float*>(base + off_agg + align_up(static_cast<size_t>(nblk) * K * 8, 256));
-    p.ew = device_error_word();
-    p.ld_loss = ld_loss;
-    p.ld_r = ld_r;
-    p.N = N;
-    p.n_seq = n_seq;
-    p.K = K;
-    p.nblk = static_cast<int>(nblk);
-    p.skip_publish = -1;
-    p.gamma = gamma;
-    const size_t smem = smem_bytes(K);
-    if (cudaFuncSetAttribute(credit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-        return DUST_ERR_CUDA;
+    CreditTable<1> T;
+    fill_common(T, cu_seqlens, n_seq, K, N, gamma, -1);
+    T.layer[0].loss = loss;
+    T.layer[0].r = r;
+    T.layer[0].ld_loss = ld_loss;
+    T.layer[0].ld_r = ld_r;
     // The ticket and the status flags must start at zero; the array keeps the previous
     // call's contents, so they are cleared on the stream before every launch.
-    if (cudaMemsetAsync(base, 0, 256 + static_cast<size_t>(nblk) * 4, s) != cudaSuccess)
+    if (!place_credit_state(T.layer[0], static_cast<char*>(scratch), nblk, K, s))
         return DUST_ERR_CUDA;
-    prof_begin(s);
-    credit_kernel<<<static_cast<unsigned>(nblk), kThreads, smem, s>>>(p);
-    prof_end(s, "credit_scan_no_alloc");
-    return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
+    return launch_credit_table(T, 1, s, "credit_scan_no_alloc");
 }

@@ -1,17 +1,21 @@
 // Noisy linear forward with the per-draw loss change (Dust review page, section "신용 할당",
 // noise equation y_t -> y_t + sigma a_t, with the quadratic readout l = 1/2 |y + sigma a - u|^2).
 //
-// bf16 layers: one tcgen05 kernel per 128-token x 256-channel tile.  TMA brings x and W tiles
-// (128-byte swizzle, 2-stage ring) into shared memory, one thread issues tcgen05.mma into a
-// 128 x 256 fp32 accumulator in tensor memory.  The epilogue turns the accumulator into
-// s_e = sigma (y - u) in place, then every thread owns one token and walks every draw:
-// it regenerates the normals of its 256 channels (never stored) and sums
-//   sigma a e + sigma^2 a^2 / 2
-// into a per-tile partial.  The last tile of each token block (an atomic ticket) adds the
-// partials of all channel tiles in a fixed order, so the result is deterministic.
+// bf16 layers: one tcgen05 kernel; each CTA owns a 128-token x 256-channel tile of one layer
+// (a launch may hold the tiles of up to kMaxGroup layers, described by a table in parameter
+// space).  TMA brings x and W tiles (128-byte swizzle, 2-stage ring) into shared memory, one
+// thread issues tcgen05.mma into a 128 x 256 fp32 accumulator in tensor memory.  The epilogue
+// turns the accumulator into s_e = sigma (y - u) in place; then the CTA's twelve warps share
+// (draw, channel-half) work units: each thread owns one token, regenerates the normals of the
+// unit's 128 channels (never stored) and sums sigma a e + sigma^2 a^2 / 2 into a per-unit
+// partial.  The last tile of each token block (an atomic ticket) adds the partials of all
+// units in a fixed order, so the result is deterministic.
 //
 // fp32 layers: a SIMT kernel (one warp per token, one quad of channels per lane) and a
 // partial-sum reduction kernel.
+#include <algorithm>
+#include <vector>
+
 #include "dust_device.cuh"
 #include "dust_internal.h"
 
@@ -29,16 +33,26 @@ constexpr uint32_t kBBytes = kBN * kBK * 2;
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 + 256;
 constexpr uint32_t kTmemCols = 256;
+constexpr int kMaxGroup = 64;  // layers per grouped launch (parameter space holds their table)
 
-struct FwdParams {
+struct FwdLayer {
     const __nv_bfloat16* u;
     float* partial;  // [2 n_tiles, K, N]: (channel tile, half) x draw x token
     float* dloss;    // [K, ld]
     int* counters;   // [m_tiles], zero on entry
+    int64_t ld;
+    int d_in, d_out, n_tiles, tile_begin;
+    uint32_t layer_id;
+};
+
+template <int kMax>
+struct FwdTable {
+    CUtensorMap tmx[kMax];
+    CUtensorMap tmw[kMax];
+    FwdLayer layer[kMax];
     ErrorWord* ew;
     int64_t N;
-    int64_t ld;
-    int d_in, d_out, K, n_tiles;
+    int n_layers, m_tiles, K;
     float sigma, half_sigma2;
     NoiseKey key;
 };
@@ -53,9 +67,8 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& v, float* f) {
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
-    fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
-                    const FwdParams p) {
+template <int kMax>
+__global__ void __launch_bounds__(kThreads, 2) fwd_bf16_kernel(const __grid_constant__ FwdTable<kMax> T) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -65,13 +78,24 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
     int* is_last = reinterpret_cast<int*>(tmem_slot + 1);
 
+    // this CTA's layer and tile (tiles are numbered layer by layer, token tile fastest)
+    int l = 0;
+    const int tile = blockIdx.x;
+    while (l + 1 < T.n_layers && tile >= T.layer[l + 1].tile_begin) ++l;
+    const FwdLayer& L = T.layer[l];
+    const CUtensorMap* tmx = &T.tmx[l];
+    const CUtensorMap* tmw = &T.tmw[l];
+    const int local = tile - L.tile_begin;
+    const int m_tile = local % T.m_tiles;
+    const int n_tile = local / T.m_tiles;
+    const int64_t N = T.N;
+    const int K = T.K;
+
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int m_tile = blockIdx.x;
-    const int n_tile = blockIdx.y;
     const int64_t m0 = static_cast<int64_t>(m_tile) * kBM;
     const int n0 = n_tile * kBN;
-    const int nk = (p.d_in + kBK - 1) / kBK;
+    const int nk = (L.d_in + kBK - 1) / kBK;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -93,17 +117,17 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     if (warp == 0 && lane == 0) {
         // TMA producer
-        prefetch_tensormap(&tmx);
-        prefetch_tensormap(&tmw);
+        prefetch_tensormap(tmx);
+        prefetch_tensormap(tmw);
         for (int kb = 0; kb < nk; ++kb) {
             const int s = kb % kStages;
             if (kb >= kStages &&
-                !mbar_wait_bounded(&empty[s], ((kb / kStages) - 1) & 1, p.ew, 101))
+                !mbar_wait_bounded(&empty[s], ((kb / kStages) - 1) & 1, T.ew, 101))
                 break;
             uint8_t* a = smem + s * kStageBytes;
             mbar_arrive_expect_tx(&full[s], kStageBytes);
-            tma_load_2d(a, &tmx, &full[s], kb * kBK, static_cast<int32_t>(m0));
-            tma_load_2d(a + kABytes, &tmw, &full[s], kb * kBK, n0);
+            tma_load_2d(a, tmx, &full[s], kb * kBK, static_cast<int32_t>(m0));
+            tma_load_2d(a + kABytes, tmw, &full[s], kb * kBK, n0);
         }
     } else if (warp == 1 && lane == 0) {
         // MMA issuer: 4 MMAs of K = 16 per stage; operands K-major, 128-byte swizzle,
@@ -111,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, 0, 0);
         for (int kb = 0; kb < nk; ++kb) {
             const int s = kb % kStages;
-            if (!mbar_wait_bounded(&full[s], (kb / kStages) & 1, p.ew, 102)) break;
+            if (!mbar_wait_bounded(&full[s], (kb / kStages) & 1, T.ew, 102)) break;
             tc_fence_after();
             const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
             const uint32_t b_addr = a_addr + kABytes;
@@ -126,19 +150,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         umma_commit(acc_full);
     }
 
-    mbar_wait_bounded(acc_full, 0, p.ew, 103);
+    mbar_wait_bounded(acc_full, 0, T.ew, 103);
     __syncwarp();
     tc_fence_after();
 
     // ---------------- epilogue: every warp; TMEM lane quarter = warp % 4, and the kGroups
-    // warps that share a lane quarter split the work (chunks in phase 1, draws in phase 2).
+    // warps that share a lane quarter split the work (chunks in phase 1, units in phase 2).
     const int lq = warp & 3;
     const int grp = warp >> 2;
     const int row = lq * 32 + lane;
     const int64_t t = m0 + row;
-    const bool valid = t < p.N;
+    const bool valid = t < N;
     const uint32_t trow = tmem + (static_cast<uint32_t>(lq * 32) << 16);
-    const int nchunks = min(kBN, p.d_out - n0) / 16;
+    const int nchunks = min(kBN, L.d_out - n0) / 16;
 
     // Phase 1: s_e = sigma (y - u), written back in place.
     for (int c = grp; c < nchunks; c += kGroups) {
@@ -147,12 +171,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         tmem_wait_ld();
         if (valid) {
             const uint4* up =
-                reinterpret_cast<const uint4*>(p.u + t * p.d_out + n0 + c * 16);
+                reinterpret_cast<const uint4*>(L.u + t * L.d_out + n0 + c * 16);
             float uf[16];
             unpack_bf16x8(__ldg(up), uf);
             unpack_bf16x8(__ldg(up + 1), uf + 8);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = p.sigma * (v[j] - uf[j]);
+            for (int j = 0; j < 16; ++j) v[j] = T.sigma * (v[j] - uf[j]);
         } else {
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = 0.f;
@@ -169,14 +193,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     // loss change over the half's channels.  In polar form a pair (z, z') = -rho (cos, sin)
     // contributes sigma (z e + z' e') + sigma^2 / 2 (z^2 + z'^2)
     //           = -rho (cos s_e + sin s_e') + h x,   with x = rho^2 = -2 ln u.
-    const uint32_t tg = p.key.token_offset + static_cast<uint32_t>(t);
+    const uint32_t tg = T.key.token_offset + static_cast<uint32_t>(t);
     const uint32_t qbase = static_cast<uint32_t>(n0 >> 2);
-    const float h = p.half_sigma2;
+    const float h = T.half_sigma2;
     const int half_chunks = (nchunks + 1) / 2;
-    for (int unit = grp; unit < 2 * p.K; unit += kGroups) {
+    for (int unit = grp; unit < 2 * K; unit += kGroups) {
         const int i = unit >> 1;
         const int hf = unit & 1;
-        const uint32_t di = p.key.draw_offset + static_cast<uint32_t>(i);
+        const uint32_t di = T.key.draw_offset + static_cast<uint32_t>(i);
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         const int c_end = hf ? nchunks : half_chunks;
         for (int c = hf ? half_chunks : 0; c < c_end; ++c) {
@@ -185,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             tmem_wait_ld();
 #pragma unroll
             for (int qq = 0; qq < 4; ++qq) {
-                const Polar4 z = normal_quad_polar(qbase + c * 4 + qq, tg, di, p.key.layer, p.key);
+                const Polar4 z = normal_quad_polar(qbase + c * 4 + qq, tg, di, L.layer_id, T.key);
                 const float l0 = fmaf(z.s0, se[4 * qq + 1], z.c0 * se[4 * qq + 0]);
                 const float l1 = fmaf(z.s1, se[4 * qq + 3], z.c1 * se[4 * qq + 2]);
                 acc[qq] = fmaf(-z.r0, l0, acc[qq]);
@@ -194,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
         if (valid)
-            p.partial[((static_cast<int64_t>(n_tile) * 2 + hf) * p.K + i) * p.N + t] =
+            L.partial[((static_cast<int64_t>(n_tile) * 2 + hf) * K + i) * N + t] =
                 (acc[0] + acc[1]) + (acc[2] + acc[3]);
     }
 
@@ -204,24 +228,85 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
     if (threadIdx.x == 0) {
-        const int old = atomicAdd(&p.counters[m_tile], 1);
-        *is_last = (old == p.n_tiles - 1);
+        const int old = atomicAdd(&L.counters[m_tile], 1);
+        *is_last = (old == L.n_tiles - 1);
     }
     __syncthreads();
     if (*is_last) {
         __threadfence();
-        for (int idx = threadIdx.x; idx < p.K * kBM; idx += kThreads) {
+        for (int idx = threadIdx.x; idx < K * kBM; idx += kThreads) {
             const int i = idx / kBM;
             const int64_t tt = m0 + (idx % kBM);
-            if (tt < p.N) {
+            if (tt < N) {
                 float s = 0.f;
-                for (int pp = 0; pp < 2 * p.n_tiles; ++pp)
-                    s += __ldcg(&p.partial[(static_cast<int64_t>(pp) * p.K + i) * p.N + tt]);
-                p.dloss[static_cast<int64_t>(i) * p.ld + tt] = s;
+                for (int pp = 0; pp < 2 * L.n_tiles; ++pp)
+                    s += __ldcg(&L.partial[(static_cast<int64_t>(pp) * K + i) * N + tt]);
+                L.dloss[static_cast<int64_t>(i) * L.ld + tt] = s;
             }
         }
-        if (threadIdx.x == 0) p.counters[m_tile] = 0;
+        if (threadIdx.x == 0) L.counters[m_tile] = 0;
     }
+}
+
+size_t bf16_layer_ws(int64_t N, int32_t d_out, int32_t K) {
+    const int64_t n_tiles = (d_out + kBN - 1) / kBN;
+    const int64_t m_tiles = (N + kBM - 1) / kBM;
+    return align_up(static_cast<size_t>(2 * n_tiles * K * N) * 4, 256) +
+           align_up(static_cast<size_t>(m_tiles) * 4, 256);
+}
+
+// Fills and launches one table of up to kMax layers.
+template <int kMax>
+dust_status launch_bf16_table(const FwdLayerArgs* layers, int n, int64_t N, int K, float sigma,
+                              const NoiseKey& key, char* ws, cudaStream_t s) {
+    FwdTable<kMax> T;  // copied into the launch's parameter space
+    T.ew = device_error_word();
+    T.N = N;
+    T.n_layers = n;
+    T.m_tiles = static_cast<int>((N + kBM - 1) / kBM);
+    T.K = K;
+    T.sigma = sigma;
+    T.half_sigma2 = 0.5f * sigma * sigma;
+    T.key = key;
+    int64_t tiles = 0;
+    size_t off = 0;
+    for (int l = 0; l < n; ++l) {
+        const FwdLayerArgs& a = layers[l];
+        if (!make_tmap_bf16_2d(&T.tmx[l], a.x, static_cast<uint64_t>(N), a.d_in, kBM, kBK) ||
+            !make_tmap_bf16_2d(&T.tmw[l], a.W, static_cast<uint64_t>(a.d_out), a.d_in, kBN, kBK))
+            return DUST_ERR_CUDA;
+        FwdLayer& L = T.layer[l];
+        const int n_tiles = (a.d_out + kBN - 1) / kBN;
+        L.u = static_cast<const __nv_bfloat16*>(a.u);
+        L.partial = reinterpret_cast<float*>(ws + off);
+        L.counters = reinterpret_cast<int*>(
+            ws + off + align_up(static_cast<size_t>(2 * n_tiles) * K * N * 4, 256));
+        L.dloss = a.dloss;
+        L.ld = a.ld;
+        L.d_in = a.d_in;
+        L.d_out = a.d_out;
+        L.n_tiles = n_tiles;
+        L.tile_begin = static_cast<int>(tiles);
+        L.layer_id = a.layer_id;
+        if (cudaMemsetAsync(L.counters, 0, static_cast<size_t>(T.m_tiles) * 4, s) != cudaSuccess)
+            return DUST_ERR_CUDA;
+        tiles += static_cast<int64_t>(n_tiles) * T.m_tiles;
+        if (tiles > 2147483647LL) return DUST_ERR_UNSUPPORTED;
+        off += bf16_layer_ws(N, a.d_out, K);
+    }
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !attr_done[dev]) {
+        if (cudaFuncSetAttribute(fwd_bf16_kernel<kMax>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSmemBytes) != cudaSuccess)
+            return DUST_ERR_CUDA;
+        if (dev < 64) attr_done[dev] = true;
+    }
+    prof_begin(s);
+    fwd_bf16_kernel<kMax><<<static_cast<unsigned>(tiles), kThreads, kSmemBytes, s>>>(T);
+    prof_end(s, kMax == 1 ? "fwd_bf16_noise_loss" : "fwd_bf16_noise_loss_grouped");
+    return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------------------ fp32 path
@@ -292,59 +377,37 @@ __global__ void reduce_partials_kernel(const float* __restrict__ partial, int n_
 }  // namespace
 
 size_t fwd_workspace_bytes(dust_dtype dt, int64_t N, int32_t d_out, int32_t K) {
-    if (dt == DUST_BF16) {
-        const int64_t n_tiles = (d_out + kBN - 1) / kBN;
-        const int64_t m_tiles = (N + kBM - 1) / kBM;
-        return align_up(static_cast<size_t>(2 * n_tiles * K * N) * 4, 256) +
-               align_up(static_cast<size_t>(m_tiles) * 4, 256);
-    }
+    if (dt == DUST_BF16) return bf16_layer_ws(N, d_out, K);
     const int64_t n_cb = (d_out + 4 * kF32Quads - 1) / (4 * kF32Quads);
     return align_up(static_cast<size_t>(n_cb * K * N) * 4, 256);
+}
+
+size_t fwd_grouped_workspace_bytes(const FwdLayerArgs* layers, int n, int64_t N, int32_t K) {
+    size_t total = 0;
+    for (int l = 0; l < n; ++l) total += bf16_layer_ws(N, layers[l].d_out, K);
+    return total;
+}
+
+dust_status fwd_grouped_launch(const FwdLayerArgs* layers, int n, int64_t N, int32_t K,
+                               float sigma, NoiseKey key, void* ws, cudaStream_t s) {
+    char* base = static_cast<char*>(ws);
+    for (int l0 = 0; l0 < n; l0 += kMaxGroup) {
+        const int cnt = std::min(kMaxGroup, n - l0);
+        const dust_status st = launch_bf16_table<kMaxGroup>(layers + l0, cnt, N, K, sigma, key, base, s);
+        if (st != DUST_OK) return st;
+        base += fwd_grouped_workspace_bytes(layers + l0, cnt, N, K);
+    }
+    return DUST_OK;
 }
 
 dust_status fwd_launch(const void* x, const void* W, const void* u, dust_dtype dt, int64_t N,
                        int32_t d_in, int32_t d_out, int32_t K, float sigma, NoiseKey key,
                        float* dloss, int64_t ld, void* ws, cudaStream_t s) {
     if (dt == DUST_BF16) {
-        const int n_tiles = (d_out + kBN - 1) / kBN;
-        const int64_t m_tiles = (N + kBM - 1) / kBM;
-        if (m_tiles > 2147483647LL) return DUST_ERR_UNSUPPORTED;
-        CUtensorMap tmx, tmw;
-        if (!make_tmap_bf16_2d(&tmx, x, static_cast<uint64_t>(N), d_in, kBM, kBK) ||
-            !make_tmap_bf16_2d(&tmw, W, static_cast<uint64_t>(d_out), d_in, kBN, kBK))
-            return DUST_ERR_CUDA;
-        FwdParams p;
-        p.u = static_cast<const __nv_bfloat16*>(u);
-        p.partial = static_cast<float*>(ws);
-        p.counters = reinterpret_cast<int*>(static_cast<char*>(ws) +
-                                            align_up(static_cast<size_t>(2 * n_tiles) * K * N * 4, 256));
-        p.dloss = dloss;
-        p.ew = device_error_word();
-        p.N = N;
-        p.ld = ld;
-        p.d_in = d_in;
-        p.d_out = d_out;
-        p.K = K;
-        p.n_tiles = n_tiles;
-        p.sigma = sigma;
-        p.half_sigma2 = 0.5f * sigma * sigma;
-        p.key = key;
-        static bool attr_done[64] = {};
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (dev >= 64 || !attr_done[dev]) {
-            if (cudaFuncSetAttribute(fwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     kSmemBytes) != cudaSuccess)
-                return DUST_ERR_CUDA;
-            if (dev < 64) attr_done[dev] = true;
-        }
-        if (cudaMemsetAsync(p.counters, 0, static_cast<size_t>(m_tiles) * 4, s) != cudaSuccess)
-            return DUST_ERR_CUDA;
-        dim3 grid(static_cast<unsigned>(m_tiles), static_cast<unsigned>(n_tiles));
-        prof_begin(s);
-        fwd_bf16_kernel<<<grid, kThreads, kSmemBytes, s>>>(tmx, tmw, p);
-        prof_end(s, "fwd_bf16_noise_loss");
-        return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
+        const int64_t tiles = (N + kBM - 1) / kBM * ((d_out + kBN - 1) / kBN);
+        if (tiles > 2147483647LL) return DUST_ERR_UNSUPPORTED;
+        FwdLayerArgs a{x, W, u, d_in, d_out, key.layer, dloss, ld};
+        return launch_bf16_table<1>(&a, 1, N, K, sigma, key, static_cast<char*>(ws), s);
     }
     const int n_cb = (d_out + 4 * kF32Quads - 1) / (4 * kF32Quads);
     FwdF32Params p;

@@ -46,6 +46,18 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64
                        uint32_t box_rows, uint32_t box_cols);
 
 // ---- noisy linear forward (dust_fwd.cu)
+struct FwdLayerArgs {
+    const void* x;
+    const void* W;
+    const void* u;
+    int32_t d_in, d_out;
+    uint32_t layer_id;
+    float* dloss;
+    int64_t ld;
+};
+size_t fwd_grouped_workspace_bytes(const FwdLayerArgs* layers, int n, int64_t N, int32_t K);
+dust_status fwd_grouped_launch(const FwdLayerArgs* layers, int n, int64_t N, int32_t K,
+                               float sigma, NoiseKey key, void* ws, cudaStream_t s);
 size_t fwd_workspace_bytes(dust_dtype dt, int64_t N, int32_t d_out, int32_t K);
 dust_status fwd_launch(const void* x, const void* W, const void* u, dust_dtype dt, int64_t N,
                        int32_t d_in, int32_t d_out, int32_t K, float sigma, NoiseKey key,
@@ -57,8 +69,31 @@ dust_status credit_launch(const float* loss, int64_t ld_loss, int32_t K, int64_t
                           const int32_t* cu, int32_t n_seq, float gamma, float* r, int64_t ld_r,
                           void* ws, cudaStream_t s);
 extern int g_credit_skip_publish;
+struct CreditLayerArgs {
+    const float* loss;
+    int64_t ld_loss;
+    float* r;
+    int64_t ld_r;
+};
+size_t credit_grouped_workspace_bytes(int n_layers, int64_t N, int32_t K);
+dust_status credit_grouped_launch(const CreditLayerArgs* layers, int n, int32_t K, int64_t N,
+                                  const int32_t* cu, int32_t n_seq, float gamma, void* ws,
+                                  cudaStream_t s);
 
 // ---- weight estimate (dust_wgrad.cu)
+struct WgradLayerArgs {
+    const float* r;
+    int64_t ld_r;
+    const void* x;
+    int32_t d_in, d_out;
+    uint32_t layer_id;
+    float* G_W;
+    float* g_out;
+};
+size_t wgrad_grouped_workspace_bytes(const WgradLayerArgs* layers, int n, int64_t N);
+dust_status wgrad_grouped_launch(const WgradLayerArgs* layers, int n, int64_t N, int32_t K_chunk,
+                                 int32_t K_total, float sigma, NoiseKey key, int accumulate,
+                                 void* ws, cudaStream_t s);
 size_t wgrad_workspace_bytes(dust_dtype dt, int64_t N, int32_t d_in, int32_t d_out);
 dust_status wgrad_launch(const float* r, int64_t ld_r, const void* x, dust_dtype dt, int64_t N,
                          int32_t d_in, int32_t d_out, int32_t K_chunk, int32_t K_total,

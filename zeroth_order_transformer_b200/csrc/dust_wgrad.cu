@@ -3,14 +3,15 @@
 //
 // Stage 1 (ghat_kernel): one thread per (token, channel quad) regenerates the quad's normals
 // for every draw and accumulates the reward-weighted sum; g is written as bf16 (the tensor
-// core operand) and optionally as fp32.  A grid-stride loop over (token, 128-quad block)
-// units keeps every SM busy to the end.
+// core operand) and optionally as fp32.  A grid-stride loop over (layer, token, 128-quad
+// block) units keeps every SM busy to the end.
 // Stage 2 (gw_bf16_kernel): G_W = g^T x on the tensor cores.  Both operands are MN-major
 // (tokens are the contraction index and the slow index of g [N, d_out] and x [N, d_in]):
 // TMA loads 64-token x 64-element boxes with 128-byte swizzle, one thread issues
 // tcgen05.mma (M = 128 output rows, N = 256 output columns, K = 16 tokens per instruction)
-// into a TMEM accumulator.  Small outputs split the token range (split-K) and a fixed-order
-// reduction adds the partials, so the result is deterministic.
+// into a TMEM accumulator.  When the outputs have fewer tiles than SMs the token range is
+// split (split-K) and a fixed-order reduction adds the partials, so the result is
+// deterministic.  One launch covers up to kMaxGroup layers (tables in parameter space).
 // fp32 layers use a SIMT tiled contraction on the fp32 g.
 #include <algorithm>
 
@@ -20,35 +21,49 @@
 namespace dust {
 namespace {
 
+constexpr int kMaxGroup = 64;
+
 // ------------------------------------------------------------------ stage 1: g
 constexpr int kGThreads = 128;
 
-struct GhatParams {
+struct GhatLayer {
     const float* r;
     __nv_bfloat16* gb;  // [N, d_out] or null
     float* gf;          // [N, d_out] or null
-    int64_t ld_r, N, units;
-    int d_out, K, nqb;
+    int64_t ld_r, unit_begin;
+    int d_out, nqb;
+    uint32_t layer_id;
+};
+
+template <int kMax>
+struct GhatTable {
+    GhatLayer layer[kMax];
+    int64_t total_units;
+    int n_layers, K;
     float scale;  // -1 / (K_total sigma)
     NoiseKey key;
 };
 
-__global__ void __launch_bounds__(kGThreads) ghat_kernel(const GhatParams p) {
-    const int nq = p.d_out >> 2;
-    for (int64_t u = blockIdx.x; u < p.units; u += gridDim.x) {
-        const int64_t t = u / p.nqb;
-        const int q = static_cast<int>(u % p.nqb) * kGThreads + threadIdx.x;
-        if (q >= nq) continue;
-        const uint32_t tg = p.key.token_offset + static_cast<uint32_t>(t);
+template <int kMax>
+__global__ void __launch_bounds__(kGThreads) ghat_kernel(const __grid_constant__ GhatTable<kMax> T) {
+    int l = 0;
+    for (int64_t u = blockIdx.x; u < T.total_units; u += gridDim.x) {
+        while (l + 1 < T.n_layers && u >= T.layer[l + 1].unit_begin) ++l;
+        const GhatLayer& L = T.layer[l];
+        const int64_t local = u - L.unit_begin;
+        const int64_t t = local / L.nqb;
+        const int q = static_cast<int>(local % L.nqb) * kGThreads + threadIdx.x;
+        if (q >= (L.d_out >> 2)) continue;
+        const uint32_t tg = T.key.token_offset + static_cast<uint32_t>(t);
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-        const float* rt = p.r + t;
+        const float* rt = L.r + t;
         // unrolled so that independent Philox chains of consecutive draws interleave
 #pragma unroll 2
-        for (int i = 0; i < p.K; ++i) {
-            const float ri = __ldg(rt + static_cast<int64_t>(i) * p.ld_r);
+        for (int i = 0; i < T.K; ++i) {
+            const float ri = __ldg(rt + static_cast<int64_t>(i) * L.ld_r);
             const Polar4 z = normal_quad_polar(static_cast<uint32_t>(q), tg,
-                                               p.key.draw_offset + static_cast<uint32_t>(i),
-                                               p.key.layer, p.key);
+                                               T.key.draw_offset + static_cast<uint32_t>(i),
+                                               L.layer_id, T.key);
             // r a = -(r rho) (cos, sin) per pair
             const float rr0 = ri * z.r0;
             const float rr1 = ri * z.r1;
@@ -57,20 +72,20 @@ __global__ void __launch_bounds__(kGThreads) ghat_kernel(const GhatParams p) {
             a2 = fmaf(-rr1, z.c1, a2);
             a3 = fmaf(-rr1, z.s1, a3);
         }
-        a0 *= p.scale;
-        a1 *= p.scale;
-        a2 *= p.scale;
-        a3 *= p.scale;
-        const int64_t off = t * p.d_out + 4 * q;
-        if (p.gb) {
+        a0 *= T.scale;
+        a1 *= T.scale;
+        a2 *= T.scale;
+        a3 *= T.scale;
+        const int64_t off = t * L.d_out + 4 * q;
+        if (L.gb) {
             __nv_bfloat162 lo = __floats2bfloat162_rn(a0, a1);
             __nv_bfloat162 hi = __floats2bfloat162_rn(a2, a3);
             uint2 v;
             v.x = *reinterpret_cast<uint32_t*>(&lo);
             v.y = *reinterpret_cast<uint32_t*>(&hi);
-            *reinterpret_cast<uint2*>(p.gb + off) = v;
+            *reinterpret_cast<uint2*>(L.gb + off) = v;
         }
-        if (p.gf) *reinterpret_cast<float4*>(p.gf + off) = make_float4(a0, a1, a2, a3);
+        if (L.gf) *reinterpret_cast<float4*>(L.gf + off) = make_float4(a0, a1, a2, a3);
     }
 }
 
@@ -87,16 +102,24 @@ constexpr uint32_t kGStageBytes = kGABytes + kGBBytes;
 constexpr uint32_t kGSmem = kGStages * kGStageBytes + 1024 + 256;
 constexpr uint32_t kGTmemCols = 256;
 
-struct GwParams {
-    float* out;  // G_W (split == 1) or partial [S, d_out, d_in]
-    ErrorWord* ew;
-    int64_t N, tokens_per_split;
-    int d_in, d_out, accumulate;
+struct GwLayer {
+    float* out;  // G_W (splits == 1) or partial [S, d_out, d_in]
+    int64_t tokens_per_split;
+    int d_in, d_out, o_tiles, k_tiles, splits, tile_begin, accumulate;
 };
 
-__global__ void __launch_bounds__(kGWThreads, 1)
-    gw_bf16_kernel(const __grid_constant__ CUtensorMap tmg, const __grid_constant__ CUtensorMap tmx,
-                   const GwParams p) {
+template <int kMax>
+struct GwTable {
+    CUtensorMap tmg[kMax];
+    CUtensorMap tmx[kMax];
+    GwLayer layer[kMax];
+    ErrorWord* ew;
+    int64_t N;
+    int n_layers;
+};
+
+template <int kMax>
+__global__ void __launch_bounds__(kGWThreads, 1) gw_bf16_kernel(const __grid_constant__ GwTable<kMax> T) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -105,12 +128,21 @@ __global__ void __launch_bounds__(kGWThreads, 1)
     uint64_t* acc_full = empty + kGStages;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
 
+    int l = 0;
+    const int tile = blockIdx.x;
+    while (l + 1 < T.n_layers && tile >= T.layer[l + 1].tile_begin) ++l;
+    const GwLayer& L = T.layer[l];
+    const CUtensorMap* tmg = &T.tmg[l];
+    const CUtensorMap* tmx = &T.tmx[l];
+    const int local = tile - L.tile_begin;
+    const int per_split = L.o_tiles * L.k_tiles;
+    const int split = local / per_split;
+    const int o0 = (local % per_split % L.o_tiles) * kGM;
+    const int k0 = (local % per_split / L.o_tiles) * kGN;
+
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int o0 = blockIdx.x * kGM;
-    const int k0 = blockIdx.y * kGN;
-    const int split = blockIdx.z;
-    const int64_t t_begin = static_cast<int64_t>(split) * p.tokens_per_split;
-    const int64_t t_end = min(p.N, t_begin + p.tokens_per_split);
+    const int64_t t_begin = static_cast<int64_t>(split) * L.tokens_per_split;
+    const int64_t t_end = min(T.N, t_begin + L.tokens_per_split);
     const int nk = t_end > t_begin ? static_cast<int>((t_end - t_begin + kGK - 1) / kGK) : 0;
 
     if (threadIdx.x == 0) {
@@ -131,22 +163,22 @@ __global__ void __launch_bounds__(kGWThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0 && lane == 0) {
-        prefetch_tensormap(&tmg);
-        prefetch_tensormap(&tmx);
+        prefetch_tensormap(tmg);
+        prefetch_tensormap(tmx);
         for (int kb = 0; kb < nk; ++kb) {
             const int s = kb % kGStages;
             if (kb >= kGStages &&
-                !mbar_wait_bounded(&empty[s], ((kb / kGStages) - 1) & 1, p.ew, 201))
+                !mbar_wait_bounded(&empty[s], ((kb / kGStages) - 1) & 1, T.ew, 201))
                 break;
             uint8_t* a = smem + s * kGStageBytes;
             uint8_t* bsm = a + kGABytes;
             const int32_t tok = static_cast<int32_t>(t_begin + static_cast<int64_t>(kb) * kGK);
             mbar_arrive_expect_tx(&full[s], kGStageBytes);
 #pragma unroll
-            for (int j = 0; j < kGM / 64; ++j) tma_load_2d(a + j * kBox, &tmg, &full[s], o0 + 64 * j, tok);
+            for (int j = 0; j < kGM / 64; ++j) tma_load_2d(a + j * kBox, tmg, &full[s], o0 + 64 * j, tok);
 #pragma unroll
             for (int j = 0; j < kGN / 64; ++j)
-                tma_load_2d(bsm + j * kBox, &tmx, &full[s], k0 + 64 * j, tok);
+                tma_load_2d(bsm + j * kBox, tmx, &full[s], k0 + 64 * j, tok);
         }
     } else if (warp == 1 && lane == 0) {
         // MN-major operands: 64-element (128-byte) rows, one row per token; 8-token core
@@ -155,7 +187,7 @@ __global__ void __launch_bounds__(kGWThreads, 1)
         constexpr uint32_t idesc = idesc_bf16_f32(kGM, kGN, 1, 1);
         for (int kb = 0; kb < nk; ++kb) {
             const int s = kb % kGStages;
-            if (!mbar_wait_bounded(&full[s], (kb / kGStages) & 1, p.ew, 202)) break;
+            if (!mbar_wait_bounded(&full[s], (kb / kGStages) & 1, T.ew, 202)) break;
             tc_fence_after();
             const uint32_t a_addr = smem_u32(smem + s * kGStageBytes);
             const uint32_t b_addr = a_addr + kGABytes;
@@ -170,14 +202,14 @@ __global__ void __launch_bounds__(kGWThreads, 1)
         umma_commit(acc_full);
     }
 
-    mbar_wait_bounded(acc_full, 0, p.ew, 203);
+    mbar_wait_bounded(acc_full, 0, T.ew, 203);
     __syncwarp();
     tc_fence_after();
 
     const int o = o0 + warp * 32 + lane;
     const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const int ncols = min(kGN, p.d_in - k0);
-    float* dst = p.out + static_cast<int64_t>(split) * p.d_out * p.d_in;
+    const int ncols = min(kGN, L.d_in - k0);
+    float* dst = L.out + static_cast<int64_t>(split) * L.d_out * L.d_in;
     for (int c = 0; c < ncols / 16; ++c) {
         float v[16];
         tmem_ld16(trow + c * 16, v);
@@ -186,12 +218,12 @@ __global__ void __launch_bounds__(kGWThreads, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = 0.f;
         }
-        if (o < p.d_out) {
-            float4* d4 = reinterpret_cast<float4*>(dst + static_cast<int64_t>(o) * p.d_in + k0 + c * 16);
+        if (o < L.d_out) {
+            float4* d4 = reinterpret_cast<float4*>(dst + static_cast<int64_t>(o) * L.d_in + k0 + c * 16);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 float4 w = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-                if (p.accumulate) {
+                if (L.accumulate) {
                     const float4 old = d4[j];
                     w.x += old.x;
                     w.y += old.y;
@@ -207,19 +239,33 @@ __global__ void __launch_bounds__(kGWThreads, 1)
     if (warp == 1) tmem_dealloc(tmem, kGTmemCols);
 }
 
-__global__ void splitk_reduce_kernel(const float4* __restrict__ part, int S, int64_t n4,
-                                     float4* __restrict__ out, int accumulate) {
-    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < n4;
+struct SplitLayer {
+    const float4* part;  // [S, n4]
+    float4* out;         // [n4]
+    int64_t n4;
+    int S, accumulate;
+};
+
+template <int kMax>
+struct SplitTable {
+    SplitLayer layer[kMax];
+};
+
+// out = (accumulate ? out : 0) + sum_s part[s] in order s = 0 .. S-1; blockIdx.y = layer.
+template <int kMax>
+__global__ void splitk_reduce_kernel(const __grid_constant__ SplitTable<kMax> T) {
+    const SplitLayer& L = T.layer[blockIdx.y];
+    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < L.n4;
          idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        float4 s = accumulate ? out[idx] : make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int k = 0; k < S; ++k) {
-            const float4 v = __ldg(&part[static_cast<int64_t>(k) * n4 + idx]);
+        float4 s = L.accumulate ? L.out[idx] : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k = 0; k < L.S; ++k) {
+            const float4 v = __ldg(&L.part[static_cast<int64_t>(k) * L.n4 + idx]);
             s.x += v.x;
             s.y += v.y;
             s.z += v.z;
             s.w += v.w;
         }
-        out[idx] = s;
+        L.out[idx] = s;
     }
 }
 
@@ -273,98 +319,181 @@ __global__ void __launch_bounds__(256) gw_f32_kernel(const float* __restrict__ g
     }
 }
 
-int choose_splits(int64_t N, int32_t d_in, int32_t d_out) {
-    const int64_t tiles = static_cast<int64_t>((d_out + kGM - 1) / kGM) * ((d_in + kGN - 1) / kGN);
+int64_t gw_tiles(int32_t d_in, int32_t d_out) {
+    return static_cast<int64_t>((d_out + kGM - 1) / kGM) * ((d_in + kGN - 1) / kGN);
+}
+
+// Split factor for a launch whose layers have `tiles` output tiles in total: fill the SMs once,
+// keeping at least 8 token blocks of 64 per split.
+int choose_splits(int64_t tiles, int64_t N) {
     const int64_t nkb = (N + kGK - 1) / kGK;
-    int64_t S = num_sms() / tiles;
+    int64_t S = num_sms() / std::max<int64_t>(tiles, 1);
     S = std::min<int64_t>(S, nkb / 8);
     return static_cast<int>(std::max<int64_t>(S, 1));
+}
+
+size_t bf16_layer_ws(int64_t N, int32_t d_in, int32_t d_out, int S) {
+    return align_up(static_cast<size_t>(N) * d_out * 2, 256) +
+           (S > 1 ? align_up(static_cast<size_t>(S) * d_out * d_in * 4, 256) : 0);
+}
+
+template <int kMax>
+dust_status launch_bf16_tables(const WgradLayerArgs* layers, int n, int64_t N, int32_t K_chunk,
+                               int32_t K_total, float sigma, const NoiseKey& key, int accumulate,
+                               char* ws, cudaStream_t s) {
+    int64_t tiles0 = 0;
+    for (int l = 0; l < n; ++l) tiles0 += gw_tiles(layers[l].d_in, layers[l].d_out);
+    const int S = choose_splits(tiles0, N);
+    const int64_t nkb = (N + kGK - 1) / kGK;
+    const int64_t tps = ((nkb + S - 1) / S) * kGK;
+
+    // stage 1: g for every layer
+    GhatTable<kMax> G;
+    G.n_layers = n;
+    G.K = K_chunk;
+    G.scale = -1.0f / (static_cast<float>(K_total) * sigma);
+    G.key = key;
+    int64_t units = 0;
+    size_t off = 0;
+    for (int l = 0; l < n; ++l) {
+        const WgradLayerArgs& a = layers[l];
+        GhatLayer& L = G.layer[l];
+        L.r = a.r;
+        L.ld_r = a.ld_r;
+        L.gb = reinterpret_cast<__nv_bfloat16*>(ws + off);
+        L.gf = a.g_out;
+        L.d_out = a.d_out;
+        L.nqb = (a.d_out / 4 + kGThreads - 1) / kGThreads;
+        L.unit_begin = units;
+        L.layer_id = a.layer_id;
+        units += N * L.nqb;
+        off += bf16_layer_ws(N, a.d_in, a.d_out, S);
+    }
+    G.total_units = units;
+    const int64_t max_blocks = static_cast<int64_t>(num_sms()) * 16;
+    prof_begin(s);
+    ghat_kernel<kMax><<<static_cast<unsigned>(std::min(units, max_blocks)), kGThreads, 0, s>>>(G);
+    prof_end(s, kMax == 1 ? "ghat_reduce_draws" : "ghat_reduce_draws_grouped");
+
+    // stage 2: G_W for every layer
+    GwTable<kMax> W;
+    W.ew = device_error_word();
+    W.N = N;
+    W.n_layers = n;
+    SplitTable<kMax> R;
+    int n_split_layers = 0;
+    int64_t max_n4 = 0;
+    int64_t tiles = 0;
+    off = 0;
+    for (int l = 0; l < n; ++l) {
+        const WgradLayerArgs& a = layers[l];
+        if (!make_tmap_bf16_2d(&W.tmg[l], ws + off, static_cast<uint64_t>(N), a.d_out, kGK, 64) ||
+            !make_tmap_bf16_2d(&W.tmx[l], a.x, static_cast<uint64_t>(N), a.d_in, kGK, 64))
+            return DUST_ERR_CUDA;
+        GwLayer& L = W.layer[l];
+        L.o_tiles = (a.d_out + kGM - 1) / kGM;
+        L.k_tiles = (a.d_in + kGN - 1) / kGN;
+        L.splits = S;
+        L.tokens_per_split = tps;
+        L.d_in = a.d_in;
+        L.d_out = a.d_out;
+        L.tile_begin = static_cast<int>(tiles);
+        tiles += static_cast<int64_t>(L.o_tiles) * L.k_tiles * S;
+        if (tiles > 2147483647LL) return DUST_ERR_UNSUPPORTED;
+        if (S == 1) {
+            L.out = a.G_W;
+            L.accumulate = accumulate;
+        } else {
+            L.out = reinterpret_cast<float*>(ws + off + align_up(static_cast<size_t>(N) * a.d_out * 2, 256));
+            L.accumulate = 0;
+            SplitLayer& Rl = R.layer[n_split_layers++];
+            Rl.part = reinterpret_cast<const float4*>(L.out);
+            Rl.out = reinterpret_cast<float4*>(a.G_W);
+            Rl.n4 = static_cast<int64_t>(a.d_out) * a.d_in / 4;
+            Rl.S = S;
+            Rl.accumulate = accumulate;
+            max_n4 = std::max(max_n4, Rl.n4);
+        }
+        off += bf16_layer_ws(N, a.d_in, a.d_out, S);
+    }
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !attr_done[dev]) {
+        if (cudaFuncSetAttribute(gw_bf16_kernel<kMax>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGSmem) != cudaSuccess)
+            return DUST_ERR_CUDA;
+        if (dev < 64) attr_done[dev] = true;
+    }
+    prof_begin(s);
+    gw_bf16_kernel<kMax><<<static_cast<unsigned>(tiles), kGWThreads, kGSmem, s>>>(W);
+    prof_end(s, kMax == 1 ? "gw_bf16_tcgen05" : "gw_bf16_tcgen05_grouped");
+    if (n_split_layers > 0) {
+        const unsigned bx = static_cast<unsigned>(
+            std::min<int64_t>((max_n4 + 255) / 256, std::max<int64_t>(1, max_blocks / n_split_layers)));
+        prof_begin(s);
+        splitk_reduce_kernel<kMax><<<dim3(bx, n_split_layers), 256, 0, s>>>(R);
+        prof_end(s, kMax == 1 ? "gw_splitk_reduce" : "gw_splitk_reduce_grouped");
+    }
+    return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
 }
 
 }  // namespace
 
 size_t wgrad_workspace_bytes(dust_dtype dt, int64_t N, int32_t d_in, int32_t d_out) {
-    if (dt == DUST_BF16) {
-        const int S = choose_splits(N, d_in, d_out);
-        return align_up(static_cast<size_t>(N) * d_out * 2, 256) +
-               (S > 1 ? align_up(static_cast<size_t>(S) * d_out * d_in * 4, 256) : 0);
-    }
+    if (dt == DUST_BF16) return bf16_layer_ws(N, d_in, d_out, choose_splits(gw_tiles(d_in, d_out), N));
     return align_up(static_cast<size_t>(N) * d_out * 4, 256);
+}
+
+size_t wgrad_grouped_workspace_bytes(const WgradLayerArgs* layers, int n, int64_t N) {
+    size_t total = 0;
+    for (int l0 = 0; l0 < n; l0 += kMaxGroup) {
+        const int cnt = std::min(kMaxGroup, n - l0);
+        int64_t tiles = 0;
+        for (int l = l0; l < l0 + cnt; ++l) tiles += gw_tiles(layers[l].d_in, layers[l].d_out);
+        const int S = choose_splits(tiles, N);
+        for (int l = l0; l < l0 + cnt; ++l)
+            total += bf16_layer_ws(N, layers[l].d_in, layers[l].d_out, S);
+    }
+    return total;
+}
+
+dust_status wgrad_grouped_launch(const WgradLayerArgs* layers, int n, int64_t N, int32_t K_chunk,
+                                 int32_t K_total, float sigma, NoiseKey key, int accumulate,
+                                 void* ws, cudaStream_t s) {
+    char* base = static_cast<char*>(ws);
+    for (int l0 = 0; l0 < n; l0 += kMaxGroup) {
+        const int cnt = std::min(kMaxGroup, n - l0);
+        const dust_status st = launch_bf16_tables<kMaxGroup>(layers + l0, cnt, N, K_chunk, K_total,
+                                                             sigma, key, accumulate, base, s);
+        if (st != DUST_OK) return st;
+        base += wgrad_grouped_workspace_bytes(layers + l0, cnt, N);
+    }
+    return DUST_OK;
 }
 
 dust_status wgrad_launch(const float* r, int64_t ld_r, const void* x, dust_dtype dt, int64_t N,
                          int32_t d_in, int32_t d_out, int32_t K_chunk, int32_t K_total,
                          float sigma, NoiseKey key, float* G_W, int accumulate, float* g_out,
                          void* ws, cudaStream_t s) {
-    const int nq = d_out / 4;
-    GhatParams gp;
-    gp.r = r;
-    gp.ld_r = ld_r;
-    gp.N = N;
-    gp.d_out = d_out;
-    gp.K = K_chunk;
-    gp.nqb = (nq + kGThreads - 1) / kGThreads;
-    gp.units = N * gp.nqb;
-    gp.scale = -1.0f / (static_cast<float>(K_total) * sigma);
-    gp.key = key;
-    const int64_t max_blocks = static_cast<int64_t>(num_sms()) * 16;
-    const unsigned gblocks = static_cast<unsigned>(std::min<int64_t>(gp.units, max_blocks));
-
     if (dt == DUST_BF16) {
-        gp.gb = static_cast<__nv_bfloat16*>(ws);
-        gp.gf = g_out;
-        prof_begin(s);
-        ghat_kernel<<<gblocks, kGThreads, 0, s>>>(gp);
-        prof_end(s, "ghat_reduce_draws");
-        const int S = choose_splits(N, d_in, d_out);
-        CUtensorMap tmg, tmx;
-        if (!make_tmap_bf16_2d(&tmg, gp.gb, static_cast<uint64_t>(N), d_out, kGK, 64) ||
-            !make_tmap_bf16_2d(&tmx, x, static_cast<uint64_t>(N), d_in, kGK, 64))
-            return DUST_ERR_CUDA;
-        GwParams p;
-        p.ew = device_error_word();
-        p.N = N;
-        p.d_in = d_in;
-        p.d_out = d_out;
-        const int64_t nkb = (N + kGK - 1) / kGK;
-        p.tokens_per_split = ((nkb + S - 1) / S) * kGK;
-        if (S == 1) {
-            p.out = G_W;
-            p.accumulate = accumulate;
-        } else {
-            p.out = reinterpret_cast<float*>(static_cast<char*>(ws) +
-                                             align_up(static_cast<size_t>(N) * d_out * 2, 256));
-            p.accumulate = 0;
-        }
-        static bool attr_done[64] = {};
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (dev < 64 && !attr_done[dev]) {
-            if (cudaFuncSetAttribute(gw_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     kGSmem) != cudaSuccess)
-                return DUST_ERR_CUDA;
-            attr_done[dev] = true;
-        }
-        dim3 grid((d_out + kGM - 1) / kGM, (d_in + kGN - 1) / kGN, S);
-        prof_begin(s);
-        gw_bf16_kernel<<<grid, kGWThreads, kGSmem, s>>>(tmg, tmx, p);
-        prof_end(s, "gw_bf16_tcgen05");
-        if (S > 1) {
-            const int64_t n4 = static_cast<int64_t>(d_out) * d_in / 4;
-            const unsigned rb = static_cast<unsigned>(std::min<int64_t>((n4 + 255) / 256, max_blocks));
-            prof_begin(s);
-            splitk_reduce_kernel<<<rb, 256, 0, s>>>(reinterpret_cast<const float4*>(p.out), S, n4,
-                                                    reinterpret_cast<float4*>(G_W), accumulate);
-            prof_end(s, "gw_splitk_reduce");
-        }
-        return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
+        WgradLayerArgs a{r, ld_r, x, d_in, d_out, key.layer, G_W, g_out};
+        return launch_bf16_tables<1>(&a, 1, N, K_chunk, K_total, sigma, key, accumulate,
+                                     static_cast<char*>(ws), s);
     }
     // fp32: g in fp32 (into g_out when given, else the workspace), SIMT contraction.
     float* gf = g_out ? g_out : static_cast<float*>(ws);
-    gp.gb = nullptr;
-    gp.gf = gf;
+    GhatTable<1> G;
+    G.n_layers = 1;
+    G.K = K_chunk;
+    G.scale = -1.0f / (static_cast<float>(K_total) * sigma);
+    G.key = key;
+    G.layer[0] = GhatLayer{r, nullptr, gf, ld_r, 0, d_out, (d_out / 4 + kGThreads - 1) / kGThreads,
+                           key.layer};
+    G.total_units = N * G.layer[0].nqb;
+    const int64_t max_blocks = static_cast<int64_t>(num_sms()) * 16;
     prof_begin(s);
-    ghat_kernel<<<gblocks, kGThreads, 0, s>>>(gp);
+    ghat_kernel<1><<<static_cast<unsigned>(std::min(G.total_units, max_blocks)), kGThreads, 0, s>>>(G);
     prof_end(s, "ghat_reduce_draws");
     dim3 grid((d_in + kFT - 1) / kFT, (d_out + kFT - 1) / kFT);
     prof_begin(s);
