@@ -413,6 +413,44 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     print(json.dumps(line), flush=True)
 
 
+def run_credit_stress(args) -> None:
+    """The credit step alone on a stress shape larger than L2 (default K = 64 draws x 4 Mi
+    tokens: 1 GiB of losses in, 1 GiB of credit out), packed sequences U[256, 2048]; prints
+    the achieved HBM bandwidth of the algorithmic bytes (8 K N per launch)."""
+    import torch
+
+    import zeroth_order_transformer_b200 as dust
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    K, N = args.stress_K, args.stress_N
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234)
+    loss = torch.randn((K, N), generator=g, device=dev, dtype=torch.float32)
+    r = torch.empty_like(loss)
+    cu = torch.from_numpy(workloads.random_segments(77, N, 256, 2048)).to(dev)
+    ws = torch.empty(dust.dust_workspace_size(dust.DUST_OP_CREDIT, dust.DUST_F32, N, 0, 0, K),
+                     dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        dust.dust_credit(loss, cu, 0.99, r, ws)
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for a, b in evs:
+        a.record()
+        dust.dust_credit(loss, cu, 0.99, r, ws)
+        b.record()
+    torch.cuda.synchronize(dev)
+    ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    st = dust.dust_last_device_error()[0]
+    peaks = measured_peaks()
+    gbs = 8.0 * K * N / (ms / 1e3) / 1e9
+    print(json.dumps({"stage": "credit_scan", "K": K, "N": N, "ms": ms, "GB/s": gbs,
+                      "frac_hbm": gbs / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"],
+                      "peak_source": peaks["source"], "status": st,
+                      "note": "inputs exceed L2 (2 GiB moved per launch); no flush needed"}),
+          flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -425,7 +463,14 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--cpu-tokens", type=int, default=1024)
     ap.add_argument("--ref-tokens", type=int, default=256)
+    ap.add_argument("--credit-stress", action="store_true",
+                    help="time dust_credit alone on a shape larger than L2 and exit")
+    ap.add_argument("--stress-K", type=int, default=64)
+    ap.add_argument("--stress-N", type=int, default=1 << 22)
     args = ap.parse_args()
+    if args.credit_stress:
+        run_credit_stress(args)
+        return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -189,11 +189,15 @@ def test_credit_ragged_and_minimal_sizes():
         assert np.all(np.abs(got - ref) <= _credit_tol(ref, cu, 0.9)), (N, K)
 
 
+CREDIT_BLOCK = 128  # tokens per look-back block of the credit kernel
+
+
 def test_credit_timeout_is_reported_and_context_survives():
     """A block that never publishes makes its predecessor's bounded wait run out: the call
     reports DUST_ERR_TIMEOUT, writes NaN there, and the next call is correct."""
     import torch
-    K, N = 4, 256 * 6
+    B = CREDIT_BLOCK
+    K, N = 4, B * 6
     cu = np.array([0, N], dtype=np.int32)
     loss = workloads.gaussian_losses(70, K, N)
     z.dust_debug_credit_skip_publish(3)
@@ -203,14 +207,54 @@ def test_credit_timeout_is_reported_and_context_survives():
     # out on block 3 themselves, or receive block 2's NaN: either way they are NaN.
     assert st == z.DUST_ERR_TIMEOUT and 0 <= info <= 2, (st, info)
     rh = _dev.host(r)
-    assert np.isnan(rh[:, :3 * 256]).all()
+    assert np.isnan(rh[:, :3 * B]).all()
     ref = oracle.credit(loss, cu, 0.9)
-    tail = slice(3 * 256, N)
+    tail = slice(3 * B, N)
     assert np.all(np.abs(rh[:, tail] - ref[:, tail]) <= _credit_tol(ref, cu, 0.9)[:, :1])
     got = _credit_gpu(loss, cu, 0.9)
     ref = oracle.credit(loss, cu, 0.9)
     assert np.all(np.abs(got - ref) <= _credit_tol(ref, cu, 0.9))
     assert z.dust_last_device_error()[0] == 0
+
+
+@pytest.mark.parametrize("K", [129, 300])
+def test_credit_many_draws_row_groups(K):
+    """More than 128 draws: the per-token mean comes from a separate pass and the rows are
+    scanned in groups with their own look-back chains."""
+    N = 2000
+    cu = workloads.random_segments(80, N, 100, 900)
+    loss = workloads.dyadic_losses(81, K, N, scale_bits=0, max_abs=8)
+    got = _credit_gpu(loss, cu, 1.0)
+    ref = oracle.credit(loss, cu, 1.0)
+    tol = 1e-6 * np.max(np.abs(ref)) + 1e-6   # mean over K not a power of two rounds
+    assert np.abs(got - ref).max() <= tol
+    g = workloads.gaussian_losses(82, K, N)
+    got = _credit_gpu(g, cu, 0.95)
+    ref = oracle.credit(g, cu, 0.95)
+    assert np.all(np.abs(got - ref) <= _credit_tol(ref, cu, 0.95))
+
+
+def test_credit_unaligned_leading_dimension():
+    """Rows that do not start on 16 bytes (ld not a multiple of 4) take the plain-load path."""
+    import torch
+    K, N, ld = 8, 1001, 1003
+    cu = workloads.random_segments(83, N, 50, 400)
+    loss = workloads.gaussian_losses(84, K, N)
+    buf = torch.zeros((K, ld), dtype=torch.float32, device="cuda")
+    buf[:, :N] = torch.from_numpy(loss).cuda()
+    out = torch.full((K, ld), float("nan"), dtype=torch.float32, device="cuda")
+    ws = torch.empty(z.dust_workspace_size(z.DUST_OP_CREDIT, z.DUST_F32, N, 0, 0, K),
+                     dtype=torch.uint8, device="cuda")
+    cu_d = _dev.cu_to_device(cu)
+    st = z.lib().dust_credit(buf.data_ptr(), ld, K, N, cu_d.data_ptr(), len(cu) - 1,
+                             0.9, out.data_ptr(), ld, ws.data_ptr(), ws.numel(),
+                             torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    torch.cuda.synchronize()
+    got = _dev.host(out)[:, :N]
+    ref = oracle.credit(loss, cu, 0.9)
+    assert np.all(np.abs(got - ref) <= _credit_tol(ref, cu, 0.9))
+    assert np.isnan(_dev.host(out)[:, N:]).all()     # nothing written past N
 
 
 # ------------------------------------------------------------------------- weight estimate

@@ -108,6 +108,6 @@ dust_status philox_debug_launch(const uint32_t* ctr, int64_t n, NoiseKey key, ui
 void prof_begin(cudaStream_t s);
 void prof_end(cudaStream_t s, const char* name);
 
-inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+__host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 }  // namespace dust
