@@ -66,6 +66,11 @@ def lib():
             _c_i64p, ctypes.c_int64, _c_i32p, ctypes.c_int32, _c_f64p]
         L.oracle_weight_grad.argtypes = [_c_f64p, _c_f64p, ctypes.c_int64, ctypes.c_int32,
                                          ctypes.c_int32, _c_f64p]
+        L.oracle_sgd_momentum.argtypes = [_c_f64p, _c_f64p, _c_f64p, ctypes.c_int64,
+                                          ctypes.c_double, ctypes.c_double, ctypes.c_double]
+        L.oracle_adam.argtypes = [_c_f64p, _c_f64p, _c_f64p, _c_f64p, ctypes.c_int64,
+                                  ctypes.c_double, ctypes.c_double, ctypes.c_double,
+                                  ctypes.c_double, ctypes.c_double, ctypes.c_int32]
         L.oracle_set_threads.argtypes = [ctypes.c_int]
         L.oracle_get_threads.restype = ctypes.c_int
         _lib = L
@@ -192,3 +197,19 @@ def dust_layer(x, W, u, K: int, sigma: float, gamma: float, cu_seqlens, seed: in
     g = output_error(r, K, sigma, seed, W.shape[0], layer_id, 0, token_offset)
     GW = weight_grad(g, x)
     return dict(loss=loss, clean=clean, r=r, g=g, G_W=GW)
+
+
+# --------------------------------------------------------------------------- optimizers
+def sgd_momentum(W, m, G, lr: float, mu: float, wd: float = 0.0):
+    """One SGD-with-momentum step (heavy ball): returns new (W, m).  Dust page, "설정"."""
+    W, m, G = _f64(W).copy(), _f64(m).copy(), _f64(G)
+    lib().oracle_sgd_momentum(_p(W, _c_f64p), _p(m, _c_f64p), _p(G, _c_f64p), W.size, lr, mu, wd)
+    return W, m
+
+
+def adam(W, m, v, G, lr: float, b1: float, b2: float, eps: float, t: int, wd: float = 0.0):
+    """One bias-corrected Adam step t >= 1 (Kingma & Ba): returns new (W, m, v)."""
+    W, m, v, G = _f64(W).copy(), _f64(m).copy(), _f64(v).copy(), _f64(G)
+    lib().oracle_adam(_p(W, _c_f64p), _p(m, _c_f64p), _p(v, _c_f64p), _p(G, _c_f64p), W.size,
+                      lr, b1, b2, eps, wd, int(t))
+    return W, m, v

@@ -297,3 +297,36 @@ void oracle_weight_grad(const double* g, const double* x, int64_t N, int32_t d_i
         }
     }
 }
+
+/*
+ * Optimizer steps on the weight estimate (Dust page, section "설정": training with SGD and
+ * momentum; section "Adam에서도 통할까?": the same estimate fed to Adam).  The page names the
+ * optimizers only; these are their standard published forms:
+ *   SGD with momentum (heavy ball, no dampening):  m <- mu m + G;  W <- W - lr m
+ *   Adam (Kingma & Ba 2015, bias-corrected), step t >= 1:
+ *     m <- b1 m + (1 - b1) G;  v <- b2 v + (1 - b2) G^2;
+ *     W <- W - lr (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps)
+ * Decoupled weight decay, when wd != 0, is applied first: W <- W - lr wd W.
+ */
+void oracle_sgd_momentum(double* W, double* m, const double* G, int64_t n, double lr, double mu,
+                         double wd)
+{
+    for (int64_t j = 0; j < n; ++j) {
+        W[j] -= lr * wd * W[j];
+        m[j] = mu * m[j] + G[j];
+        W[j] -= lr * m[j];
+    }
+}
+
+void oracle_adam(double* W, double* m, double* v, const double* G, int64_t n, double lr,
+                 double b1, double b2, double eps, double wd, int32_t t)
+{
+    const double c1 = 1.0 - pow(b1, (double)t);
+    const double c2 = 1.0 - pow(b2, (double)t);
+    for (int64_t j = 0; j < n; ++j) {
+        W[j] -= lr * wd * W[j];
+        m[j] = b1 * m[j] + (1.0 - b1) * G[j];
+        v[j] = b2 * v[j] + (1.0 - b2) * G[j] * G[j];
+        W[j] -= lr * (m[j] / c1) / (sqrt(v[j] / c2) + eps);
+    }
+}
