@@ -71,6 +71,10 @@ def lib():
         L.oracle_adam.argtypes = [_c_f64p, _c_f64p, _c_f64p, _c_f64p, ctypes.c_int64,
                                   ctypes.c_double, ctypes.c_double, ctypes.c_double,
                                   ctypes.c_double, ctypes.c_double, ctypes.c_int32]
+        L.oracle_noisy_logits_ce.argtypes = [
+            _c_f64p, _c_i32p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+            ctypes.c_int32, ctypes.c_double, ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32,
+            ctypes.c_uint32, _c_i64p, ctypes.c_int64, _c_f64p, _c_f64p]
         L.oracle_set_threads.argtypes = [ctypes.c_int]
         L.oracle_get_threads.restype = ctypes.c_int
         _lib = L
@@ -213,3 +217,21 @@ def adam(W, m, v, G, lr: float, b1: float, b2: float, eps: float, t: int, wd: fl
     lib().oracle_adam(_p(W, _c_f64p), _p(m, _c_f64p), _p(v, _c_f64p), _p(G, _c_f64p), W.size,
                       lr, b1, b2, eps, wd, int(t))
     return W, m, v
+
+
+# --------------------------------------------------------------------------- LM head
+def noisy_logits_ce(z, y, v0: int, S: int, K: int, sigma: float, seed: int, layer_id: int = 0,
+                    draw_offset: int = 0, token_offset: int = 0, tokens=None):
+    """Absolute cross-entropy losses [K, n_tok] with noise on the logit slab [v0, v0 + S), and the
+    clean losses [n_tok] (Dust page, "간섭 줄이기": the LM head perturbed on cached logits)."""
+    z = _f64(z)
+    N, V = z.shape
+    yy = np.ascontiguousarray(y, dtype=np.int32)
+    tk = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int64)
+    n_tok = N if tk is None else tk.shape[0]
+    loss = np.zeros((K, n_tok), dtype=np.float64)
+    clean = np.zeros(n_tok, dtype=np.float64)
+    lib().oracle_noisy_logits_ce(_p(z, _c_f64p), _p(yy, _c_i32p), N, V, v0, S, K, float(sigma),
+                                 int(seed), layer_id, draw_offset, token_offset, _p(tk, _c_i64p),
+                                 n_tok, _p(loss, _c_f64p), _p(clean, _c_f64p))
+    return loss, clean

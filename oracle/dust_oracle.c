@@ -330,3 +330,48 @@ void oracle_adam(double* W, double* m, double* v, const double* G, int64_t n, do
         W[j] -= lr * (m[j] / c1) / (sqrt(v[j] / c2) + eps);
     }
 }
+
+/*
+ * LM-head perturbation on cached logits (Dust page, section "간섭(interference) 줄이기",
+ * third point: the LM head is perturbed directly on the cached logits; only the cross-entropy
+ * is recomputed, on a slab of the vocabulary).  Reading: noise sigma a_t^(i)[v] is added to
+ * the logits of the slab v in [v0, v0 + S) (channel index v, so the noise of a logit does not
+ * depend on the slab); the per-token loss is the full-vocabulary cross-entropy
+ *   l_t^(i) = log sum_v exp(z_t[v] + sigma a_t^(i)[v] [v in slab]) - (z_t[y_t] + sigma a_t^(i)[y_t] [y_t in slab]).
+ * Computed as the plain definition in fp64 (max-shifted log-sum-exp).
+ * z: [N][V], y: [N]; loss: [K][n_tok] absolute, clean: [n_tok] (unperturbed), tokens as above.
+ */
+void oracle_noisy_logits_ce(const double* z, const int32_t* y, int64_t N, int32_t V, int32_t v0,
+                            int32_t S, int32_t K, double sigma, uint64_t seed, uint32_t layer_id,
+                            uint32_t draw_offset, uint32_t token_offset, const int64_t* tokens,
+                            int64_t n_tok, double* loss, double* clean)
+{
+    if (!tokens) n_tok = N;
+#pragma omp parallel
+    {
+        double* zp = (double*)malloc(sizeof(double) * (size_t)V);
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t j = 0; j < n_tok; ++j) {
+            int64_t t = tokens ? tokens[j] : j;
+            const double* zt = z + t * (int64_t)V;
+            int32_t yt = y[t];
+            double mx = zt[0];
+            for (int32_t v = 1; v < V; ++v) mx = zt[v] > mx ? zt[v] : mx;
+            double s = 0.0;
+            for (int32_t v = 0; v < V; ++v) s += exp(zt[v] - mx);
+            if (clean) clean[j] = mx + log(s) - zt[yt];
+            for (int32_t i = 0; i < K; ++i) {
+                for (int32_t v = 0; v < V; ++v) zp[v] = zt[v];
+                for (int32_t v = v0; v < v0 + S; ++v)
+                    zp[v] += sigma * noise_at(seed, layer_id, token_offset + (uint32_t)t,
+                                              draw_offset + (uint32_t)i, v);
+                double m2 = zp[0];
+                for (int32_t v = 1; v < V; ++v) m2 = zp[v] > m2 ? zp[v] : m2;
+                double s2 = 0.0;
+                for (int32_t v = 0; v < V; ++v) s2 += exp(zp[v] - m2);
+                loss[(int64_t)i * n_tok + j] = m2 + log(s2) - zp[yt];
+            }
+        }
+        free(zp);
+    }
+}
