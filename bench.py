@@ -381,6 +381,42 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e_ms / args.steps}
 
+    # ---- optional: the optimizer step fused into the weight estimate (single-layer workloads)
+    opt_line = None
+    if args.optimizer != "none" and len(layers) == 1:
+        s1, x1, W1, u1 = layers[0]
+        Wm = torch.zeros((s1.d_out, s1.d_in), dtype=torch.float32, device=dev)
+        mm = torch.zeros_like(Wm)
+        vv = torch.zeros_like(Wm) if args.optimizer == "adam" else None
+        Wb = torch.empty((s1.d_out, s1.d_in), dtype=torch.bfloat16, device=dev)
+        key = dust.NoiseKey(wl.seed, s1.layer_id, 0, rank * wl.N)
+
+        def opt_params(t):
+            return dust.sgd_momentum(1e-2, 0.9) if args.optimizer == "sgd" else dust.adam(1e-3, t)
+
+        for t in range(1, 3):
+            dust.dust_weight_grad_step(r, x1, s1.d_out, wl.K, wl.sigma, key, opt_params(t), Wm,
+                                       mm, vv, W_bf16=Wb, workspace=ws)
+        torch.cuda.synchronize(dev)
+        ea = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        eb = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        reps = max(5, args.steps)
+        ea[0].record(stream)
+        for t in range(reps):
+            dust.dust_weight_grad(r, x1, s1.d_out, wl.K, wl.sigma, key, GWs[0], False, None, ws)
+        eb[0].record(stream)
+        ea[1].record(stream)
+        for t in range(reps):
+            dust.dust_weight_grad_step(r, x1, s1.d_out, wl.K, wl.sigma, key, opt_params(t + 3),
+                                       Wm, mm, vv, W_bf16=Wb, workspace=ws)
+        eb[1].record(stream)
+        torch.cuda.synchronize(dev)
+        t_plain = ea[0].elapsed_time(eb[0]) / reps
+        t_step = ea[1].elapsed_time(eb[1]) / reps
+        opt_line = {"kind": args.optimizer, "weight_grad_ms": round(t_plain, 5),
+                    "weight_grad_with_step_ms": round(t_step, 5),
+                    "step_overhead_ms": round(t_step - t_plain, 5)}
+
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -410,6 +446,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         "clocks": clocks,
         "kernels": kernels,
     }
+    if opt_line is not None:
+        line["optimizer"] = opt_line
     print(json.dumps(line), flush=True)
 
 
@@ -463,6 +501,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--cpu-tokens", type=int, default=1024)
     ap.add_argument("--ref-tokens", type=int, default=256)
+    ap.add_argument("--optimizer", choices=["none", "sgd", "adam"], default="none",
+                    help="also time the optimizer step fused into the weight estimate (reported "
+                         "under 'optimizer'; the headline value stays the estimator alone)")
     ap.add_argument("--credit-stress", action="store_true",
                     help="time dust_credit alone on a shape larger than L2 and exit")
     ap.add_argument("--stress-K", type=int, default=64)

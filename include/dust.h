@@ -57,19 +57,23 @@ typedef enum { DUST_F32 = 0, DUST_BF16 = 1 } dust_dtype;
 typedef enum {
     DUST_OP_NOISY_LINEAR_FWD = 0,
     DUST_OP_CREDIT = 1,
-    DUST_OP_WEIGHT_GRAD = 2
+    DUST_OP_WEIGHT_GRAD = 2,
+    DUST_OP_LOGITS_CE = 3 /* d_in = vocabulary size V, d_out = slab size S */
 } dust_op;
 
 /* Identifies the noise of one call.  seed: generator key; layer_id: fourth counter word, so
  * layers draw independent noise; draw_offset: global index of the call's first draw (a
  * population larger than one call is processed in chunks); token_offset: global index of the
- * call's first token (a batch sharded over several GPUs keeps the same noise per token). */
+ * call's first token (a batch sharded over several GPUs keeps the same noise per token);
+ * channel_offset: global index of the call's first output channel, a multiple of 4 (0 for a
+ * whole layer; the slab start when only a slab of a layer's outputs is perturbed, as for the
+ * LM head, so that a channel's noise does not depend on the slab). */
 typedef struct {
     uint64_t seed;
     uint32_t layer_id;
     uint32_t draw_offset;
     uint32_t token_offset;
-    uint32_t reserved; /* must be 0 */
+    uint32_t channel_offset;
 } dust_noise_key;
 
 /*
@@ -89,6 +93,26 @@ dust_status dust_noisy_linear_fwd(const void* x, const void* W, const void* u, d
                                   float sigma, dust_noise_key key, float* dloss,
                                   int64_t ld_dloss, void* workspace, size_t ws_bytes,
                                   void* stream);
+
+/*
+ * LM-head perturbation on cached logits (Dust page, section "간섭(interference) 줄이기": the
+ * LM head is perturbed on the cached logits and only the cross-entropy is recomputed, on a
+ * slab of the vocabulary).  For each draw i and token t, with noise sigma a_t^(i)[v] added to
+ * the logits of the slab v in [v0, v0 + S) (v is the noise channel; key.channel_offset must
+ * be 0):
+ *   dloss[i * ld_dloss + t] = CE(z_t + noise) - CE(z_t),  CE(z) = log sum_v exp(z_v) - z_{y_t},
+ *                           = log(1 + X / E) - sigma a_t^(i)[y_t] [y_t in slab],
+ *   E = sum_v exp(z_v - max z),  X = sum_{v in slab} exp(z_v - max z) (exp(sigma a) - 1).
+ * z: logits [N, ld_z] of dtype dt (fp32 or bf16) with V valid columns; y: DEVICE int32 [N]
+ * targets (a target outside [0, V) gives NaN for its token).  v0 and S multiples of 4,
+ * v0 + S <= V.  The output feeds dust_credit, then dust_weight_grad with d_out = S and
+ * key.channel_offset = v0 gives g on the slab and the slab's rows of the head weight estimate.
+ * workspace: dust_workspace_size(DUST_OP_LOGITS_CE, dt, N, V, S, K) bytes.
+ */
+dust_status dust_noisy_logits_ce(const void* z, int64_t ld_z, dust_dtype dt, const int32_t* y,
+                                 int64_t N, int32_t V, int32_t v0, int32_t S, int32_t K,
+                                 float sigma, dust_noise_key key, float* dloss, int64_t ld_dloss,
+                                 void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * Centred loss and discounted credit (centred-loss and credit equations).
@@ -144,6 +168,48 @@ dust_status dust_weight_grad(const float* r, int64_t ld_r, const void* x, dust_d
 dust_status dust_credit_no_alloc(const float* loss, int64_t ld_loss, int32_t K, int64_t N,
                                  const int32_t* cu_seqlens, int32_t n_seq, float gamma,
                                  float* r, int64_t ld_r, void* stream);
+
+/*
+ * Optimizer step on a weight estimate.  The Dust page trains with SGD and momentum (section
+ * "설정") and reports the same estimate fed to Adam (section "Adam에서도 통할까?"); it names
+ * the optimizers only, so their standard published forms are used, with decoupled weight
+ * decay applied first (W <- W - lr wd W):
+ *   DUST_OPT_SGD_MOMENTUM:  m <- momentum m + G;  W <- W - lr m
+ *   DUST_OPT_ADAM (Kingma & Ba, bias-corrected, step t >= 1):
+ *     m <- b1 m + (1 - b1) G;  v <- b2 v + (1 - b2) G^2;
+ *     W <- W - lr (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps)
+ * All state is fp32 and updated in place.
+ */
+typedef enum { DUST_OPT_SGD_MOMENTUM = 1, DUST_OPT_ADAM = 2 } dust_opt_kind;
+
+typedef struct {
+    int32_t kind;        /* dust_opt_kind */
+    int32_t step;        /* Adam: 1-based step count t */
+    float lr;            /* >= 0 */
+    float momentum;      /* SGD: 0 <= momentum < 1 */
+    float beta1, beta2;  /* Adam: 0 <= beta < 1 */
+    float eps;           /* Adam: > 0 */
+    float weight_decay;  /* >= 0, decoupled */
+} dust_opt_params;
+
+/* One step on n elements: G (read), W fp32 master weights, m (and v for Adam) state, all
+ * DEVICE fp32 [n], 16-byte aligned, updated in place; W_bf16 (DEVICE, optional, NULL to skip)
+ * receives the updated W rounded to bf16 (for the next forward).  `opt` is a HOST pointer. */
+dust_status dust_optimizer_step(const dust_opt_params* opt, const float* G, float* W,
+                                void* W_bf16, float* m, float* v, int64_t n, void* stream);
+
+/* dust_weight_grad with the optimizer step fused into the pass that finishes G_W (the
+ * contraction's epilogue, or the split-K reduction): the weight estimate is not written and
+ * read back before the step.  Same arguments as dust_weight_grad (bf16 only), plus the step:
+ * W, W_bf16, m, v as in dust_optimizer_step with n = d_out * d_in.  G_W may be NULL (then it
+ * is not stored; accumulate must be 0).  The result equals dust_weight_grad followed by
+ * dust_optimizer_step. */
+dust_status dust_weight_grad_step(const float* r, int64_t ld_r, const void* x, dust_dtype dt,
+                                  int64_t N, int32_t d_in, int32_t d_out, int32_t K_chunk,
+                                  int32_t K_total, float sigma, dust_noise_key key, float* G_W,
+                                  int accumulate, float* g_out, const dust_opt_params* opt,
+                                  float* W, void* W_bf16, float* m, float* v, void* workspace,
+                                  size_t ws_bytes, void* stream);
 
 /*
  * Grouped forms: the same three steps for many bf16 layers that share the token batch

@@ -1,0 +1,93 @@
+"""LM-head perturbation on cached logits (Dust page, "간섭(interference) 줄이기"): the CUDA
+cross-entropy loss change against the oracle, and the whole head estimate (credit, g on the
+slab, slab rows of the head weight estimate) against the oracle chain.  Tolerances as for the
+linear forward: the loss change is a short fp32 computation on exactly read inputs with
+fp32 normals (element error <= 1e-3 x RMS, relative Frobenius <= 1e-4); g and G_W 2e-3."""
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from tests import _dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def z():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import zeroth_order_transformer_b200 as zz
+    zz.lib()
+    return zz
+
+
+def _case(seed, N, V, dtype):
+    import torch
+    rng = np.random.default_rng(seed)
+    logits = (rng.standard_normal((N, V)) * 2.0).astype(np.float32)
+    y = rng.integers(0, V, size=N).astype(np.int32)
+    if dtype == "bf16":
+        bits = workloads.to_bf16_bits(logits)
+        z64 = workloads.bf16_bits_to_f64(bits)
+        zt = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+    else:
+        z64 = logits.astype(np.float64)
+        zt = torch.from_numpy(logits).cuda()
+    return zt, torch.from_numpy(y).cuda(), z64, y
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("N,V,v0,S,K,sigma", [
+    (300, 512, 0, 512, 4, 1e-2),      # the whole vocabulary, series path
+    (257, 1000, 128, 256, 3, 5e-2),   # a slab, expm1 path, ragged tokens
+    (64, 4096, 1024, 1024, 2, 1e-3),
+    (10, 96, 4, 20, 2, 1e-2),         # slab not a multiple of 16
+])
+def test_logits_ce_matches_oracle(z, dtype, N, V, v0, S, K, sigma):
+    import torch
+    zt, yt, z64, y = _case(N + V, N, V, dtype)
+    key = z.NoiseKey(0x5EED0006, layer_id=48, draw_offset=5, token_offset=77)
+    dl = z.dust_noisy_logits_ce(zt, yt, v0, S, K, sigma, key)
+    torch.cuda.synchronize()
+    loss, clean = oracle.noisy_logits_ce(z64, y, v0, S, K, sigma, key.seed, 48, 5, 77)
+    _dev.assert_fp32_close(_dev.host(dl), loss - clean, "lm-head dloss")
+
+
+def test_logits_ce_targets_outside_the_slab_and_invalid(z):
+    import torch
+    zt, yt, z64, y = _case(3, 40, 256, "f32")
+    y[:20] = 5           # outside the slab [64, 192)
+    y[20:] = 100         # inside
+    yt = torch.from_numpy(y).cuda()
+    dl = z.dust_noisy_logits_ce(zt, yt, 64, 128, 3, 1e-2, z.NoiseKey(9))
+    torch.cuda.synchronize()
+    loss, clean = oracle.noisy_logits_ce(z64, y, 64, 128, 3, 1e-2, 9)
+    _dev.assert_fp32_close(_dev.host(dl), loss - clean, "targets in/out")
+    y[7] = 256           # not a vocabulary index: NaN for that token only
+    dl = z.dust_noisy_logits_ce(zt, torch.from_numpy(y).cuda(), 64, 128, 3, 1e-2, z.NoiseKey(9))
+    h = _dev.host(dl)
+    assert np.isnan(h[:, 7]).all() and np.isfinite(np.delete(h, 7, axis=1)).all()
+
+
+def test_lm_head_estimate_matches_oracle_chain(z):
+    """Cross-entropy loss change -> credit (gamma = 0: the head only changes its own token's
+    loss) -> g on the slab and the slab's rows of the head weight estimate G_W = sum g h^T."""
+    import torch
+    N, V, d_model, v0, S, K, sigma = 512, 1024, 64, 256, 256, 8, 1e-2
+    zt, yt, z64, y = _case(11, N, V, "bf16")
+    H = workloads.custom_layer(12, N, d_model, 16, "bf16", 0.02)   # hidden states x = h
+    h = _dev.to_device(H.x_store, "bf16")
+    key = z.NoiseKey(0x5EED0006, layer_id=48)
+    cu = np.array([0, N], dtype=np.int32)
+    dl = z.dust_noisy_logits_ce(zt, yt, v0, S, K, sigma, key)
+    r = z.dust_credit(dl, _dev.cu_to_device(cu), 0.0)
+    GW, g = z.dust_weight_grad(r, h, S, K, sigma, key._replace(channel_offset=v0), g_out=True)
+    torch.cuda.synchronize()
+    loss, clean = oracle.noisy_logits_ce(z64, y, v0, S, K, sigma, key.seed, 48)
+    r_ref = oracle.credit(loss, cu, 0.0)
+    g_ref = oracle.output_error(r_ref, K, sigma, key.seed, V, 48, chans=np.arange(v0, v0 + S))
+    GW_ref = oracle.weight_grad(g_ref, H.x_f64)
+    assert _dev.rel_fro(_dev.host(g), g_ref) <= _dev.GW_FRO
+    assert _dev.rel_fro(_dev.host(GW), GW_ref) <= _dev.GW_FRO

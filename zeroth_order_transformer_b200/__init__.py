@@ -33,6 +33,7 @@ DUST_BF16 = 1
 DUST_OP_NOISY_LINEAR_FWD = 0
 DUST_OP_CREDIT = 1
 DUST_OP_WEIGHT_GRAD = 2
+DUST_OP_LOGITS_CE = 3
 
 EXPORTED_SYMBOLS = (
     "dust_noisy_linear_fwd", "dust_credit", "dust_weight_grad", "dust_workspace_size",
@@ -40,7 +41,11 @@ EXPORTED_SYMBOLS = (
     "dust_debug_credit_skip_publish", "dust_profile_enable", "dust_profile_disable",
     "dust_profile_read", "dust_credit_no_alloc", "dust_noisy_linear_fwd_grouped",
     "dust_credit_grouped", "dust_weight_grad_grouped", "dust_workspace_size_grouped",
+    "dust_optimizer_step", "dust_weight_grad_step", "dust_noisy_logits_ce",
 )
+
+DUST_OPT_SGD_MOMENTUM = 1
+DUST_OPT_ADAM = 2
 
 
 class DustError(RuntimeError):
@@ -52,7 +57,7 @@ class DustError(RuntimeError):
 class dust_noise_key(ctypes.Structure):
     _fields_ = [("seed", ctypes.c_uint64), ("layer_id", ctypes.c_uint32),
                 ("draw_offset", ctypes.c_uint32), ("token_offset", ctypes.c_uint32),
-                ("reserved", ctypes.c_uint32)]
+                ("channel_offset", ctypes.c_uint32)]
 
 
 class dust_layer_desc(ctypes.Structure):
@@ -63,15 +68,31 @@ class dust_layer_desc(ctypes.Structure):
                 ("G_W", ctypes.c_void_p), ("g_out", ctypes.c_void_p)]
 
 
+class dust_opt_params(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("step", ctypes.c_int32), ("lr", ctypes.c_float),
+                ("momentum", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float)]
+
+
+def sgd_momentum(lr: float, momentum: float, weight_decay: float = 0.0) -> dust_opt_params:
+    return dust_opt_params(DUST_OPT_SGD_MOMENTUM, 0, lr, momentum, 0.0, 0.0, 0.0, weight_decay)
+
+
+def adam(lr: float, step: int, beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8,
+         weight_decay: float = 0.0) -> dust_opt_params:
+    return dust_opt_params(DUST_OPT_ADAM, step, lr, 0.0, beta1, beta2, eps, weight_decay)
+
+
 class NoiseKey(NamedTuple):
     seed: int
     layer_id: int = 0
     draw_offset: int = 0
     token_offset: int = 0
+    channel_offset: int = 0
 
     def c(self) -> dust_noise_key:
         return dust_noise_key(self.seed & 0xFFFFFFFFFFFFFFFF, self.layer_id, self.draw_offset,
-                              self.token_offset, 0)
+                              self.token_offset, self.channel_offset)
 
 
 _lib = None
@@ -105,6 +126,16 @@ def lib() -> ctypes.CDLL:
         for name in ("dust_noisy_linear_fwd_grouped", "dust_credit_grouped",
                      "dust_weight_grad_grouped"):
             getattr(L, name).restype = ctypes.c_int
+        op = ctypes.POINTER(dust_opt_params)
+        L.dust_optimizer_step.argtypes = [op, vp, vp, vp, vp, vp, i64, vp]
+        L.dust_optimizer_step.restype = ctypes.c_int
+        L.dust_weight_grad_step.argtypes = [vp, i64, vp, ctypes.c_int, i64, i32, i32, i32, i32,
+                                            f32, dust_noise_key, vp, ctypes.c_int, vp, op, vp, vp,
+                                            vp, vp, vp, sz, vp]
+        L.dust_weight_grad_step.restype = ctypes.c_int
+        L.dust_noisy_logits_ce.argtypes = [vp, i64, ctypes.c_int, vp, i64, i32, i32, i32, i32,
+                                           f32, dust_noise_key, vp, i64, vp, sz, vp]
+        L.dust_noisy_logits_ce.restype = ctypes.c_int
         L.dust_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, i64, i32, i32, i32]
         L.dust_workspace_size.restype = sz
         L.dust_status_string.argtypes = [ctypes.c_int]
@@ -201,6 +232,28 @@ def dust_noisy_linear_fwd(x, W, u, K: int, sigma: float, key: NoiseKey, dloss=No
     return dloss
 
 
+def dust_noisy_logits_ce(z, y, v0: int, S: int, K: int, sigma: float, key: NoiseKey,
+                         dloss=None, workspace=None, stream=None):
+    """Per-draw change of the full-vocabulary cross-entropy dloss[K, N] when noise is added to
+    the cached logits of the slab [v0, v0 + S) (LM-head perturbation)."""
+    torch = _torch()
+    _cuda(z, "z"), _cuda(y, "y")
+    if y.dtype != torch.int32:
+        raise TypeError("y must be int32")
+    N, V = z.shape
+    dt = _dtype_code(z)
+    if dloss is None:
+        dloss = torch.empty((K, N), dtype=torch.float32, device=z.device)
+    ws, nb = _workspace(workspace, dust_workspace_size(DUST_OP_LOGITS_CE, dt, N, V, S, K),
+                        z.device)
+    st = lib().dust_noisy_logits_ce(z.data_ptr(), z.stride(0), dt, y.data_ptr(), N, V, v0, S, K,
+                                    float(sigma), key.c(), dloss.data_ptr(), dloss.stride(0),
+                                    ws.data_ptr() if ws is not None else None, nb,
+                                    _stream(z.device, stream))
+    _check(st, "dust_noisy_logits_ce")
+    return dloss
+
+
 def dust_credit(loss, cu_seqlens, gamma: float, r=None, workspace=None, stream=None):
     """Credit r[K, N] from losses [K, N] and int32 cu_seqlens [n_seq + 1] (device)."""
     torch = _torch()
@@ -266,6 +319,40 @@ def dust_weight_grad(r, x, d_out: int, K_total: int, sigma: float, key: NoiseKey
                                 _stream(x.device, stream))
     _check(st, "dust_weight_grad")
     return G_W, g_out
+
+
+def _ptr(t):
+    return t.data_ptr() if t is not None else None
+
+
+def dust_optimizer_step(opt: dust_opt_params, G, W, m, v=None, W_bf16=None, stream=None):
+    """One optimizer step in place on fp32 W, m (and v for Adam) from the estimate G."""
+    for t, nm in ((G, "G"), (W, "W"), (m, "m")):
+        _cuda(t, nm)
+    st = lib().dust_optimizer_step(ctypes.byref(opt), G.data_ptr(), W.data_ptr(), _ptr(W_bf16),
+                                   m.data_ptr(), _ptr(v), W.numel(), _stream(W.device, stream))
+    _check(st, "dust_optimizer_step")
+    return W
+
+
+def dust_weight_grad_step(r, x, d_out: int, K_total: int, sigma: float, key: NoiseKey,
+                          opt: dust_opt_params, W, m, v=None, W_bf16=None, G_W=None,
+                          accumulate: bool = False, g_out=None, workspace=None, stream=None):
+    """dust_weight_grad with the optimizer step fused into the pass that finishes G_W."""
+    _cuda(r, "r"), _cuda(x, "x"), _cuda(W, "W"), _cuda(m, "m")
+    K_chunk, N = r.shape
+    d_in = x.shape[1]
+    dt = _dtype_code(x)
+    ws, nb = _workspace(workspace, dust_workspace_size(DUST_OP_WEIGHT_GRAD, dt, N, d_in, d_out,
+                                                       K_chunk), x.device)
+    st = lib().dust_weight_grad_step(r.data_ptr(), r.stride(0), x.data_ptr(), dt, N, d_in, d_out,
+                                     K_chunk, K_total, float(sigma), key.c(), _ptr(G_W),
+                                     1 if accumulate else 0, _ptr(g_out), ctypes.byref(opt),
+                                     W.data_ptr(), _ptr(W_bf16), m.data_ptr(), _ptr(v),
+                                     ws.data_ptr() if ws is not None else None, nb,
+                                     _stream(x.device, stream))
+    _check(st, "dust_weight_grad_step")
+    return W
 
 
 def dust_last_device_error(stream=None, device=None) -> Tuple[int, int]:

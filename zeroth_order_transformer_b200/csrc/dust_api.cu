@@ -192,8 +192,30 @@ size_t dust_workspace_size(dust_op op, dust_dtype dt, int64_t N, int32_t d_in, i
         case DUST_OP_NOISY_LINEAR_FWD: return fwd_workspace_bytes(dt, N, d_out, K);
         case DUST_OP_CREDIT: return credit_workspace_bytes(N, K);
         case DUST_OP_WEIGHT_GRAD: return wgrad_workspace_bytes(dt, N, d_in, d_out);
+        case DUST_OP_LOGITS_CE: return lmhead_workspace_bytes(N, d_out, K);
     }
     return 0;
+}
+
+dust_status dust_noisy_logits_ce(const void* z, int64_t ld_z, dust_dtype dt, const int32_t* y,
+                                 int64_t N, int32_t V, int32_t v0, int32_t S, int32_t K,
+                                 float sigma, dust_noise_key key, float* dloss, int64_t ld_dloss,
+                                 void* workspace, size_t ws_bytes, void* stream) {
+    if (!valid_dtype(dt) || !z || !y || !dloss || N < 1 || V < 1 || K < 1 || ld_z < V ||
+        ld_dloss < N)
+        return DUST_ERR_INVALID_ARG;
+    if (v0 < 0 || S < 0 || v0 % 4 != 0 || S % 4 != 0 || static_cast<int64_t>(v0) + S > V)
+        return DUST_ERR_INVALID_ARG;
+    if (!std::isfinite(sigma) || key.channel_offset != 0 || (reinterpret_cast<uintptr_t>(y) & 3u))
+        return DUST_ERR_INVALID_ARG;
+    if (N > 0xFFFFFFFFLL) return DUST_ERR_UNSUPPORTED;
+    if (static_cast<uint64_t>(key.draw_offset) + static_cast<uint64_t>(K) > 0x100000000ull ||
+        static_cast<uint64_t>(key.token_offset) + static_cast<uint64_t>(N) > 0x100000000ull)
+        return DUST_ERR_INVALID_ARG;
+    dust_status st = check_ws(workspace, ws_bytes, lmhead_workspace_bytes(N, S, K));
+    if (st != DUST_OK) return st;
+    return lmhead_launch(z, ld_z, dt, y, N, V, v0, S, K, sigma, make_key(key), dloss, ld_dloss,
+                         workspace, static_cast<cudaStream_t>(stream));
 }
 
 dust_status dust_noisy_linear_fwd(const void* x, const void* W, const void* u, dust_dtype dt,
@@ -205,7 +227,7 @@ dust_status dust_noisy_linear_fwd(const void* x, const void* W, const void* u, d
     if (st != DUST_OK) return st;
     if (!W || !u || !dloss || !aligned16(W) || !aligned16(u) || !aligned16(dloss))
         return DUST_ERR_INVALID_ARG;
-    if (K < 1 || ld_dloss < N || !std::isfinite(sigma) || key.reserved != 0)
+    if (K < 1 || ld_dloss < N || !std::isfinite(sigma) || key.channel_offset % 4 != 0)
         return DUST_ERR_INVALID_ARG;
     if (static_cast<uint64_t>(key.draw_offset) + static_cast<uint64_t>(K) > 0x100000000ull ||
         static_cast<uint64_t>(key.token_offset) + static_cast<uint64_t>(N) > 0x100000000ull)
@@ -238,7 +260,7 @@ dust_status dust_weight_grad(const float* r, int64_t ld_r, const void* x, dust_d
     dust_status st = check_layer(x, dt, N, d_in, d_out);
     if (st != DUST_OK) return st;
     if (!r || !G_W || !aligned16(G_W) || (g_out && !aligned16(g_out))) return DUST_ERR_INVALID_ARG;
-    if (K_chunk < 1 || K_total < K_chunk || ld_r < N || key.reserved != 0)
+    if (K_chunk < 1 || K_total < K_chunk || ld_r < N || key.channel_offset % 4 != 0)
         return DUST_ERR_INVALID_ARG;
     if (!(sigma > 0.f) || !std::isfinite(sigma)) return DUST_ERR_INVALID_ARG;
     if (static_cast<uint64_t>(key.draw_offset) + static_cast<uint64_t>(K_chunk) > 0x100000000ull ||
@@ -250,6 +272,46 @@ dust_status dust_weight_grad(const float* r, int64_t ld_r, const void* x, dust_d
     if (st != DUST_OK) return st;
     return wgrad_launch(r, ld_r, x, dt, N, d_in, d_out, K_chunk, K_total, sigma, make_key(key),
                         G_W, accumulate, g_out, workspace, static_cast<cudaStream_t>(stream));
+}
+
+dust_status dust_optimizer_step(const dust_opt_params* opt, const float* G, float* W,
+                                void* W_bf16, float* m, float* v, int64_t n, void* stream) {
+    OptParams o;
+    if (!make_opt(opt, &o) || n < 0) return DUST_ERR_INVALID_ARG;
+    if (n > 0 && (!G || !W || !m || (o.kind == DUST_OPT_ADAM && !v))) return DUST_ERR_INVALID_ARG;
+    if (!aligned16(G) || !aligned16(W) || !aligned16(m) || (v && !aligned16(v)) ||
+        (W_bf16 && (reinterpret_cast<uintptr_t>(W_bf16) & 7u) != 0))
+        return DUST_ERR_INVALID_ARG;
+    return opt_launch(o, G, OptTargets{W, W_bf16, m, v}, n, static_cast<cudaStream_t>(stream));
+}
+
+dust_status dust_weight_grad_step(const float* r, int64_t ld_r, const void* x, dust_dtype dt,
+                                  int64_t N, int32_t d_in, int32_t d_out, int32_t K_chunk,
+                                  int32_t K_total, float sigma, dust_noise_key key, float* G_W,
+                                  int accumulate, float* g_out, const dust_opt_params* opt,
+                                  float* W, void* W_bf16, float* m, float* v, void* workspace,
+                                  size_t ws_bytes, void* stream) {
+    dust_status st = check_layer(x, dt, N, d_in, d_out);
+    if (st != DUST_OK) return st;
+    if (dt != DUST_BF16) return DUST_ERR_UNSUPPORTED;
+    OptParams o;
+    if (!make_opt(opt, &o)) return DUST_ERR_INVALID_ARG;
+    if (!r || (G_W && !aligned16(G_W)) || (accumulate && !G_W) || (g_out && !aligned16(g_out)))
+        return DUST_ERR_INVALID_ARG;
+    if (!W || !m || (o.kind == DUST_OPT_ADAM && !v) || !aligned16(W) || !aligned16(m) ||
+        (v && !aligned16(v)) || (W_bf16 && (reinterpret_cast<uintptr_t>(W_bf16) & 7u) != 0))
+        return DUST_ERR_INVALID_ARG;
+    if (K_chunk < 1 || K_total < K_chunk || ld_r < N || key.channel_offset % 4 != 0) return DUST_ERR_INVALID_ARG;
+    if (!(sigma > 0.f) || !std::isfinite(sigma)) return DUST_ERR_INVALID_ARG;
+    if (static_cast<uint64_t>(key.draw_offset) + static_cast<uint64_t>(K_chunk) > 0x100000000ull ||
+        static_cast<uint64_t>(key.token_offset) + static_cast<uint64_t>(N) > 0x100000000ull)
+        return DUST_ERR_INVALID_ARG;
+    st = check_ws(workspace, ws_bytes, wgrad_workspace_bytes(dt, N, d_in, d_out));
+    if (st != DUST_OK) return st;
+    const OptTargets t{W, W_bf16, m, v};
+    return wgrad_launch(r, ld_r, x, dt, N, d_in, d_out, K_chunk, K_total, sigma, make_key(key),
+                        G_W, accumulate, g_out, workspace, static_cast<cudaStream_t>(stream), &o,
+                        &t);
 }
 
 dust_status dust_last_device_error(void* stream, int32_t* info) {
@@ -285,7 +347,7 @@ namespace {
 
 dust_status check_group(const dust_layer_desc* layers, int32_t n_layers, int64_t N, int32_t K,
                         dust_noise_key key, int step) {
-    if (!layers || n_layers < 1 || N < 1 || K < 1 || key.reserved != 0) return DUST_ERR_INVALID_ARG;
+    if (!layers || n_layers < 1 || N < 1 || K < 1 || key.channel_offset % 4 != 0) return DUST_ERR_INVALID_ARG;
     if (N > 0xFFFFFFFFLL) return DUST_ERR_UNSUPPORTED;
     if (static_cast<uint64_t>(key.draw_offset) + static_cast<uint64_t>(K) > 0x100000000ull ||
         static_cast<uint64_t>(key.token_offset) + static_cast<uint64_t>(N) > 0x100000000ull)

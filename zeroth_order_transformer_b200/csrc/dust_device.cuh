@@ -161,6 +161,49 @@ __device__ __forceinline__ F4 normal_quad(uint32_t q, uint32_t t, uint32_t i, ui
 }
 
 // ----------------------------------------------------------------------------------------
+// Optimizer step on one element of the weight estimate g (decoupled weight decay first):
+//   SGD with momentum:  m <- mu m + g;  w <- w - lr m
+//   Adam (bias-corrected): m <- b1 m + (1-b1) g;  v <- b2 v + (1-b2) g^2;
+//                          w <- w - lr (m / c1) / (sqrt(v / c2) + eps),  c = 1 - beta^t
+// ----------------------------------------------------------------------------------------
+__device__ __forceinline__ void opt_update(const OptParams& o, float g, float& w, float& m,
+                                           float& v) {
+    w = fmaf(-o.lr_wd, w, w);
+    if (o.kind == DUST_OPT_SGD_MOMENTUM) {
+        m = fmaf(o.mu, m, g);
+        w = fmaf(-o.lr, m, w);
+    } else {
+        m = fmaf(o.b1, m, o.omb1 * g);
+        v = fmaf(o.b2, v, o.omb2 * (g * g));
+        w = w - o.lr * (m / o.c1) / (sqrtf(v / o.c2) + o.eps);
+    }
+}
+
+// Applies the step to 4 consecutive elements at index e (a multiple of 4) of the targets.
+__device__ __forceinline__ void opt_update4(const OptParams& o, const OptTargets& t, int64_t e,
+                                            float4 g) {
+    float4 w = *reinterpret_cast<const float4*>(t.W + e);
+    float4 m = *reinterpret_cast<const float4*>(t.m + e);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (o.kind == DUST_OPT_ADAM) v = *reinterpret_cast<const float4*>(t.v + e);
+    opt_update(o, g.x, w.x, m.x, v.x);
+    opt_update(o, g.y, w.y, m.y, v.y);
+    opt_update(o, g.z, w.z, m.z, v.z);
+    opt_update(o, g.w, w.w, m.w, v.w);
+    *reinterpret_cast<float4*>(t.W + e) = w;
+    *reinterpret_cast<float4*>(t.m + e) = m;
+    if (o.kind == DUST_OPT_ADAM) *reinterpret_cast<float4*>(t.v + e) = v;
+    if (t.W_bf16) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(w.x, w.y);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(w.z, w.w);
+        uint2 b;
+        b.x = *reinterpret_cast<uint32_t*>(&lo);
+        b.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(t.W_bf16) + e) = b;
+    }
+}
+
+// ----------------------------------------------------------------------------------------
 // Shared-memory addresses, mbarriers, TMA.
 // ----------------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -8,8 +8,10 @@
 // turns the accumulator into s_e = sigma (y - u) in place; then the CTA's twelve warps share
 // (draw, channel-half) work units: each thread owns one token, regenerates the normals of the
 // unit's 128 channels (never stored) and sums sigma a e + sigma^2 a^2 / 2 into a per-unit
-// partial.  The last tile of each token block (an atomic ticket) adds the partials of all
-// units in a fixed order, so the result is deterministic.
+// partial.  Tiles of the last, partial wave of CTAs are split into unit ranges (each computing
+// the tile's GEMM) so that the wave ends together.  The CTA that completes a token block (a
+// counter of finished units) adds the partials of all units in a fixed order, so the result is
+// deterministic.
 //
 // fp32 layers: a SIMT kernel (one warp per token, one quad of channels per lane) and a
 // partial-sum reduction kernel.
@@ -52,6 +54,9 @@ struct FwdTable {
     FwdLayer layer[kMax];
     ErrorWord* ew;
     int64_t N;
+    int64_t total_tiles;
+    int64_t n_full;  // tiles processed whole, one CTA each (CTAs 0 .. n_full-1)
+    int split;       // unit ranges per tile of the remaining tiles
     int n_layers, m_tiles, K;
     float sigma, half_sigma2;
     NoiseKey key;
@@ -78,24 +83,11 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_bf16_kernel(const __grid_cons
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
     int* is_last = reinterpret_cast<int*>(tmem_slot + 1);
 
-    // this CTA's layer and tile (tiles are numbered layer by layer, token tile fastest)
-    int l = 0;
-    const int tile = blockIdx.x;
-    while (l + 1 < T.n_layers && tile >= T.layer[l + 1].tile_begin) ++l;
-    const FwdLayer& L = T.layer[l];
-    const CUtensorMap* tmx = &T.tmx[l];
-    const CUtensorMap* tmw = &T.tmw[l];
-    const int local = tile - L.tile_begin;
-    const int m_tile = local % T.m_tiles;
-    const int n_tile = local / T.m_tiles;
-    const int64_t N = T.N;
-    const int K = T.K;
-
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t m0 = static_cast<int64_t>(m_tile) * kBM;
-    const int n0 = n_tile * kBN;
-    const int nk = (L.d_in + kBK - 1) / kBK;
+    const int64_t N = T.N;
+    const int K = T.K;
+    const int U = 2 * K;  // work units per tile: (draw, channel half)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -103,7 +95,6 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_bf16_kernel(const __grid_cons
             mbar_init(&empty[s], 1);
         }
         mbar_init(acc_full, 1);
-        *is_last = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -115,137 +106,171 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_bf16_kernel(const __grid_cons
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0 && lane == 0) {
-        // TMA producer
-        prefetch_tensormap(tmx);
-        prefetch_tensormap(tmw);
-        for (int kb = 0; kb < nk; ++kb) {
-            const int s = kb % kStages;
-            if (kb >= kStages &&
-                !mbar_wait_bounded(&empty[s], ((kb / kStages) - 1) & 1, T.ew, 101))
-                break;
-            uint8_t* a = smem + s * kStageBytes;
-            mbar_arrive_expect_tx(&full[s], kStageBytes);
-            tma_load_2d(a, tmx, &full[s], kb * kBK, static_cast<int32_t>(m0));
-            tma_load_2d(a + kABytes, tmw, &full[s], kb * kBK, n0);
-        }
-    } else if (warp == 1 && lane == 0) {
-        // MMA issuer: 4 MMAs of K = 16 per stage; operands K-major, 128-byte swizzle,
-        // 8-row core groups 1024 bytes apart.
-        constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, 0, 0);
-        for (int kb = 0; kb < nk; ++kb) {
-            const int s = kb % kStages;
-            if (!mbar_wait_bounded(&full[s], (kb / kStages) & 1, T.ew, 102)) break;
-            tc_fence_after();
-            const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
-            const uint32_t b_addr = a_addr + kABytes;
-#pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk) {
-                const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
-                const uint64_t bd = sdesc_sw128(b_addr + kk * 32, 16, 1024);
-                umma_bf16(tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+    // This CTA's tile and unit range: the tiles of the full waves take one CTA each (all
+    // units); the tiles of the last, partial wave are split into T.split unit ranges, each
+    // computing the tile's GEMM, so that the last wave ends nearly together.
+    int tile, u_begin, u_end;
+    if (static_cast<int64_t>(blockIdx.x) < T.n_full) {
+        tile = blockIdx.x;
+        u_begin = 0;
+        u_end = U;
+    } else {
+        const int r = blockIdx.x - static_cast<int>(T.n_full);
+        const int part = r % T.split;
+        tile = static_cast<int>(T.n_full) + r / T.split;
+        u_begin = U * part / T.split;
+        u_end = U * (part + 1) / T.split;
+    }
+    uint32_t kc_prod = 0, kc_mma = 0;
+    const uint32_t acc_phase = 0;
+    int l = 0;
+    {
+        while (l + 1 < T.n_layers && tile >= T.layer[l + 1].tile_begin) ++l;
+        const FwdLayer& L = T.layer[l];
+        const CUtensorMap* tmx = &T.tmx[l];
+        const CUtensorMap* tmw = &T.tmw[l];
+        const int local = tile - L.tile_begin;
+        const int m_tile = local % T.m_tiles;
+        const int n_tile = local / T.m_tiles;
+        const int64_t m0 = static_cast<int64_t>(m_tile) * kBM;
+        const int n0 = n_tile * kBN;
+        const int nk = (L.d_in + kBK - 1) / kBK;
+
+        if (warp == 0 && lane == 0) {
+            // TMA producer
+            prefetch_tensormap(tmx);
+            prefetch_tensormap(tmw);
+            for (int kb = 0; kb < nk; ++kb, ++kc_prod) {
+                const int s = kc_prod % kStages;
+                if (kc_prod >= kStages &&
+                    !mbar_wait_bounded(&empty[s], ((kc_prod / kStages) - 1) & 1, T.ew, 101))
+                    break;
+                uint8_t* a = smem + s * kStageBytes;
+                mbar_arrive_expect_tx(&full[s], kStageBytes);
+                tma_load_2d(a, tmx, &full[s], kb * kBK, static_cast<int32_t>(m0));
+                tma_load_2d(a + kABytes, tmw, &full[s], kb * kBK, n0);
             }
-            umma_commit(&empty[s]);
-        }
-        umma_commit(acc_full);
-    }
-
-    mbar_wait_bounded(acc_full, 0, T.ew, 103);
-    __syncwarp();
-    tc_fence_after();
-
-    // ---------------- epilogue: every warp; TMEM lane quarter = warp % 4, and the kGroups
-    // warps that share a lane quarter split the work (chunks in phase 1, units in phase 2).
-    const int lq = warp & 3;
-    const int grp = warp >> 2;
-    const int row = lq * 32 + lane;
-    const int64_t t = m0 + row;
-    const bool valid = t < N;
-    const uint32_t trow = tmem + (static_cast<uint32_t>(lq * 32) << 16);
-    const int nchunks = min(kBN, L.d_out - n0) / 16;
-
-    // Phase 1: s_e = sigma (y - u), written back in place.
-    for (int c = grp; c < nchunks; c += kGroups) {
-        float v[16];
-        tmem_ld16(trow + c * 16, v);
-        tmem_wait_ld();
-        if (valid) {
-            const uint4* up =
-                reinterpret_cast<const uint4*>(L.u + t * L.d_out + n0 + c * 16);
-            float uf[16];
-            unpack_bf16x8(__ldg(up), uf);
-            unpack_bf16x8(__ldg(up + 1), uf + 8);
+        } else if (warp == 1 && lane == 0) {
+            // MMA issuer: 4 MMAs of K = 16 per stage; operands K-major, 128-byte swizzle,
+            // 8-row core groups 1024 bytes apart.
+            constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, 0, 0);
+            for (int kb = 0; kb < nk; ++kb, ++kc_mma) {
+                const int s = kc_mma % kStages;
+                if (!mbar_wait_bounded(&full[s], (kc_mma / kStages) & 1, T.ew, 102)) break;
+                tc_fence_after();
+                const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
+                const uint32_t b_addr = a_addr + kABytes;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = T.sigma * (v[j] - uf[j]);
-        } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = 0.f;
+                for (int kk = 0; kk < kBK / 16; ++kk) {
+                    const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(b_addr + kk * 32, 16, 1024);
+                    umma_bf16(tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                }
+                umma_commit(&empty[s]);
+            }
+            umma_commit(acc_full);
         }
-        tmem_st16(trow + c * 16, v);
-    }
-    tmem_wait_st();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
 
-    // Phase 2: work units are (draw, half of the tile's channels), dealt round-robin to the
-    // warp groups so that they finish together.  Per unit: regenerate the noise and sum the
-    // loss change over the half's channels.  In polar form a pair (z, z') = -rho (cos, sin)
-    // contributes sigma (z e + z' e') + sigma^2 / 2 (z^2 + z'^2)
-    //           = -rho (cos s_e + sin s_e') + h x,   with x = rho^2 = -2 ln u.
-    const uint32_t tg = T.key.token_offset + static_cast<uint32_t>(t);
-    const uint32_t qbase = static_cast<uint32_t>(n0 >> 2);
-    const float h = T.half_sigma2;
-    const int half_chunks = (nchunks + 1) / 2;
-    for (int unit = grp; unit < 2 * K; unit += kGroups) {
-        const int i = unit >> 1;
-        const int hf = unit & 1;
-        const uint32_t di = T.key.draw_offset + static_cast<uint32_t>(i);
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        const int c_end = hf ? nchunks : half_chunks;
-        for (int c = hf ? half_chunks : 0; c < c_end; ++c) {
-            float se[16];
-            tmem_ld16(trow + c * 16, se);
+        mbar_wait_bounded(acc_full, acc_phase, T.ew, 103);
+        __syncwarp();
+        tc_fence_after();
+
+        // ---------------- epilogue: every warp; TMEM lane quarter = warp % 4, and the kGroups
+        // warps that share a lane quarter split the work (chunks in phase 1, units in phase 2).
+        const int lq = warp & 3;
+        const int grp = warp >> 2;
+        const int row = lq * 32 + lane;
+        const int64_t t = m0 + row;
+        const bool valid = t < N;
+        const uint32_t trow = tmem + (static_cast<uint32_t>(lq * 32) << 16);
+        const int nchunks = min(kBN, L.d_out - n0) / 16;
+
+        // Phase 1: s_e = sigma (y - u), written back in place.
+        for (int c = grp; c < nchunks; c += kGroups) {
+            float v[16];
+            tmem_ld16(trow + c * 16, v);
             tmem_wait_ld();
+            if (valid) {
+                const uint4* up =
+                    reinterpret_cast<const uint4*>(L.u + t * L.d_out + n0 + c * 16);
+                float uf[16];
+                unpack_bf16x8(__ldg(up), uf);
+                unpack_bf16x8(__ldg(up + 1), uf + 8);
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                const Polar4 z = normal_quad_polar(qbase + c * 4 + qq, tg, di, L.layer_id, T.key);
-                const float l0 = fmaf(z.s0, se[4 * qq + 1], z.c0 * se[4 * qq + 0]);
-                const float l1 = fmaf(z.s1, se[4 * qq + 3], z.c1 * se[4 * qq + 2]);
-                acc[qq] = fmaf(-z.r0, l0, acc[qq]);
-                acc[qq] = fmaf(-z.r1, l1, acc[qq]);
-                acc[qq] = fmaf(h, z.x0 + z.x1, acc[qq]);
+                for (int j = 0; j < 16; ++j) v[j] = T.sigma * (v[j] - uf[j]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] = 0.f;
             }
+            tmem_st16(trow + c * 16, v);
         }
-        if (valid)
-            L.partial[((static_cast<int64_t>(n_tile) * 2 + hf) * K + i) * N + t] =
-                (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // Phase 2: this CTA's units of the tile, dealt round-robin to the warp groups.  A unit
+        // is (draw, half of the tile's channels): regenerate the noise and sum the loss change
+        // over the half's channels.  In polar form a pair (z, z') = -rho (cos, sin) contributes
+        // sigma (z e + z' e') + sigma^2 / 2 (z^2 + z'^2) = -rho (cos s_e + sin s_e') + h x,
+        // with x = rho^2 = -2 ln u.
+        const uint32_t tg = T.key.token_offset + static_cast<uint32_t>(t);
+        const uint32_t qbase = static_cast<uint32_t>(n0 >> 2) + T.key.quad_offset;
+        const float h = T.half_sigma2;
+        const int half_chunks = (nchunks + 1) / 2;
+        for (int unit = u_begin + grp; unit < u_end; unit += kGroups) {
+            const int i = unit >> 1;
+            const int hf = unit & 1;
+            const uint32_t di = T.key.draw_offset + static_cast<uint32_t>(i);
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            const int c_end = hf ? nchunks : half_chunks;
+            for (int c = hf ? half_chunks : 0; c < c_end; ++c) {
+                float se[16];
+                tmem_ld16(trow + c * 16, se);
+                tmem_wait_ld();
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const Polar4 z = normal_quad_polar(qbase + c * 4 + qq, tg, di, L.layer_id, T.key);
+                    const float l0 = fmaf(z.s0, se[4 * qq + 1], z.c0 * se[4 * qq + 0]);
+                    const float l1 = fmaf(z.s1, se[4 * qq + 3], z.c1 * se[4 * qq + 2]);
+                    acc[qq] = fmaf(-z.r0, l0, acc[qq]);
+                    acc[qq] = fmaf(-z.r1, l1, acc[qq]);
+                    acc[qq] = fmaf(h, z.x0 + z.x1, acc[qq]);
+                }
+            }
+            if (valid)
+                L.partial[((static_cast<int64_t>(n_tile) * 2 + hf) * K + i) * N + t] =
+                    (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        }
+
+        // Done with the accumulator.  Count the finished units of the token block; the CTA
+        // that completes it adds the partials of every unit in a fixed order.
+        tc_fence_before();
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            const int done = u_end - u_begin;
+            const int old = atomicAdd(&L.counters[m_tile], done);
+            *is_last = (old + done == L.n_tiles * U);
+        }
+        __syncthreads();
+        if (*is_last) {
+            __threadfence();
+            for (int idx = threadIdx.x; idx < K * kBM; idx += kThreads) {
+                const int i = idx / kBM;
+                const int64_t tt = m0 + (idx % kBM);
+                if (tt < N) {
+                    float s = 0.f;
+                    for (int pp = 0; pp < 2 * L.n_tiles; ++pp)
+                        s += __ldcg(&L.partial[(static_cast<int64_t>(pp) * K + i) * N + tt]);
+                    L.dloss[static_cast<int64_t>(i) * L.ld + tt] = s;
+                }
+            }
+            if (threadIdx.x == 0) L.counters[m_tile] = 0;
+        }
     }
 
-    // Release tensor memory early, then the last channel tile of this token block reduces.
-    tc_fence_before();
-    __threadfence();
-    __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
-    if (threadIdx.x == 0) {
-        const int old = atomicAdd(&L.counters[m_tile], 1);
-        *is_last = (old == L.n_tiles - 1);
-    }
-    __syncthreads();
-    if (*is_last) {
-        __threadfence();
-        for (int idx = threadIdx.x; idx < K * kBM; idx += kThreads) {
-            const int i = idx / kBM;
-            const int64_t tt = m0 + (idx % kBM);
-            if (tt < N) {
-                float s = 0.f;
-                for (int pp = 0; pp < 2 * L.n_tiles; ++pp)
-                    s += __ldcg(&L.partial[(static_cast<int64_t>(pp) * K + i) * N + tt]);
-                L.dloss[static_cast<int64_t>(i) * L.ld + tt] = s;
-            }
-        }
-        if (threadIdx.x == 0) L.counters[m_tile] = 0;
-    }
 }
 
 size_t bf16_layer_ws(int64_t N, int32_t d_out, int32_t K) {
@@ -253,6 +278,28 @@ size_t bf16_layer_ws(int64_t N, int32_t d_out, int32_t K) {
     const int64_t m_tiles = (N + kBM - 1) / kBM;
     return align_up(static_cast<size_t>(2 * n_tiles * K * N) * 4, 256) +
            align_up(static_cast<size_t>(m_tiles) * 4, 256);
+}
+
+// How many unit ranges to cut each of the `rem` tiles of the last partial wave into, so that
+// the wave's CTAs finish nearly together.  A range of u units takes ceil(u / kGroups) rounds
+// of its warp groups; the cost minimised is (CTA waves of the tail) x (rounds per range as a
+// share of a whole tile's rounds + the GEMM share of a tile, about 6%).
+int tail_split(int64_t rem, int64_t slots, int units) {
+    if (rem == 0) return 1;
+    int best = 1;
+    double best_t = 1e30;
+    const double full_rounds = static_cast<double>((units + kGroups - 1) / kGroups);
+    for (int f = 1; f <= 8 && units / f >= 2; ++f) {
+        const double waves = static_cast<double>((rem * f + slots - 1) / slots);
+        const int max_units = (units + f - 1) / f;
+        const double rounds = static_cast<double>((max_units + kGroups - 1) / kGroups);
+        const double t = waves * (rounds / full_rounds + 0.06);
+        if (t < best_t - 1e-9) {
+            best_t = t;
+            best = f;
+        }
+    }
+    return best;
 }
 
 // Fills and launches one table of up to kMax layers.
@@ -303,8 +350,15 @@ dust_status launch_bf16_table(const FwdLayerArgs* layers, int n, int64_t N, int 
             return DUST_ERR_CUDA;
         if (dev < 64) attr_done[dev] = true;
     }
+    // Full waves of two CTAs per SM take whole tiles; the remainder is split (see the kernel).
+    T.total_tiles = tiles;
+    const int64_t slots = 2LL * num_sms();
+    T.n_full = tiles / slots * slots;
+    T.split = tail_split(tiles - T.n_full, slots, 2 * K);
+    const int64_t grid = T.n_full + (tiles - T.n_full) * T.split;
+    if (grid > 2147483647LL) return DUST_ERR_UNSUPPORTED;
     prof_begin(s);
-    fwd_bf16_kernel<kMax><<<static_cast<unsigned>(tiles), kThreads, kSmemBytes, s>>>(T);
+    fwd_bf16_kernel<kMax><<<static_cast<unsigned>(grid), kThreads, kSmemBytes, s>>>(T);
     prof_end(s, kMax == 1 ? "fwd_bf16_noise_loss" : "fwd_bf16_noise_loss_grouped");
     return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
 }
@@ -350,7 +404,7 @@ __global__ void __launch_bounds__(256) fwd_f32_kernel(const FwdF32Params p) {
     for (int i = 0; i < p.K; ++i) {
         float acc = 0.f;
         if (ch_ok[0]) {
-            const F4 z = normal_quad(static_cast<uint32_t>(q), tg,
+            const F4 z = normal_quad(static_cast<uint32_t>(q) + p.key.quad_offset, tg,
                                      p.key.draw_offset + static_cast<uint32_t>(i), p.key.layer, p.key);
             const float zz[4] = {z.x, z.y, z.z, z.w};
 #pragma unroll

@@ -24,12 +24,13 @@ struct NoiseKey {
     uint32_t layer;         // fourth counter word
     uint32_t draw_offset;   // added to the draw index (third counter word)
     uint32_t token_offset;  // added to the token index (second counter word)
+    uint32_t quad_offset;   // added to the channel-quad index (first counter word)
     uint32_t rk[20];        // round keys: rk[2r] = k0 + r W0, rk[2r+1] = k1 + r W1
 };
 
 inline NoiseKey make_key(const dust_noise_key& k) {
     NoiseKey n{static_cast<uint32_t>(k.seed & 0xffffffffu), static_cast<uint32_t>(k.seed >> 32),
-               k.layer_id, k.draw_offset, k.token_offset, {}};
+               k.layer_id, k.draw_offset, k.token_offset, k.channel_offset / 4, {}};
     for (uint32_t r = 0; r < 10; ++r) {
         n.rk[2 * r] = n.k0 + r * kPhiloxWeyl0;
         n.rk[2 * r + 1] = n.k1 + r * kPhiloxWeyl1;
@@ -63,6 +64,12 @@ dust_status fwd_launch(const void* x, const void* W, const void* u, dust_dtype d
                        int32_t d_in, int32_t d_out, int32_t K, float sigma, NoiseKey key,
                        float* dloss, int64_t ld, void* ws, cudaStream_t s);
 
+// ---- LM head on cached logits (dust_lmhead.cu)
+size_t lmhead_workspace_bytes(int64_t N, int32_t S, int32_t K);
+dust_status lmhead_launch(const void* z, int64_t ld_z, dust_dtype dt, const int32_t* y, int64_t N,
+                          int32_t V, int32_t v0, int32_t S, int32_t K, float sigma, NoiseKey key,
+                          float* dloss, int64_t ld, void* ws, cudaStream_t s);
+
 // ---- credit (dust_credit.cu)
 size_t credit_workspace_bytes(int64_t N, int32_t K);
 dust_status credit_launch(const float* loss, int64_t ld_loss, int32_t K, int64_t N,
@@ -79,6 +86,23 @@ size_t credit_grouped_workspace_bytes(int n_layers, int64_t N, int32_t K);
 dust_status credit_grouped_launch(const CreditLayerArgs* layers, int n, int32_t K, int64_t N,
                                   const int32_t* cu, int32_t n_seq, float gamma, void* ws,
                                   cudaStream_t s);
+
+// ---- optimizer step on the weight estimate (dust_opt.cu, and fused in dust_wgrad.cu)
+struct OptParams {
+    int kind;             // 0: none, DUST_OPT_SGD_MOMENTUM, DUST_OPT_ADAM
+    float lr, lr_wd;      // learning rate; lr * decoupled weight decay
+    float mu;             // SGD momentum
+    float b1, omb1, b2, omb2, eps, c1, c2;  // Adam: betas, 1 - betas, eps, 1 - beta^t
+};
+struct OptTargets {
+    float* W;      // fp32 master weights (updated in place)
+    void* W_bf16;  // optional bf16 copy of the updated weights
+    float* m;      // first moment / momentum
+    float* v;      // second moment (Adam)
+};
+bool make_opt(const dust_opt_params* p, OptParams* o);
+dust_status opt_launch(const OptParams& o, const float* G, const OptTargets& t, int64_t n,
+                       cudaStream_t s);
 
 // ---- weight estimate (dust_wgrad.cu)
 struct WgradLayerArgs {
@@ -98,7 +122,8 @@ size_t wgrad_workspace_bytes(dust_dtype dt, int64_t N, int32_t d_in, int32_t d_o
 dust_status wgrad_launch(const float* r, int64_t ld_r, const void* x, dust_dtype dt, int64_t N,
                          int32_t d_in, int32_t d_out, int32_t K_chunk, int32_t K_total,
                          float sigma, NoiseKey key, float* G_W, int accumulate, float* g_out,
-                         void* ws, cudaStream_t s);
+                         void* ws, cudaStream_t s, const OptParams* opt = nullptr,
+                         const OptTargets* targets = nullptr);
 
 // ---- generator test export (dust_api.cu)
 dust_status philox_debug_launch(const uint32_t* ctr, int64_t n, NoiseKey key, uint32_t* words,

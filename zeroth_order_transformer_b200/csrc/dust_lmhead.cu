@@ -1,0 +1,236 @@
+// LM-head perturbation on cached logits (Dust review page, section "간섭(interference)
+// 줄이기", third point: the LM head is perturbed directly on the cached logits; only the
+// cross-entropy is recomputed, on a slab of the vocabulary, so populations far larger than
+// one forward pass cost stay cheap).
+//
+// For token t, draw i and the slab [v0, v0 + S):
+//   l^(i) - l^clean = log(1 + X^(i) / E) - sigma a^(i)[y] [y in slab],
+//   E = sum_v exp(z_v - zmax)  (the whole vocabulary, clean),
+//   X^(i) = sum_{v in slab} exp(z_v - zmax) (exp(sigma a^(i)[v]) - 1).
+// Three kernels:
+//   ce_stats_kernel    per token: zmax and E over the vocabulary (online max / rescaled sum).
+//   ce_noise_kernel    per (128-channel chunk, 128 tokens): w = exp(z - zmax) staged in shared
+//                      memory, then per draw the normals of the chunk are regenerated and
+//                      sum w (exp(sigma a) - 1) goes into a per-chunk partial.
+//   ce_finish_kernel   per (draw, token): log1p(sum of partials / E) minus the target's term.
+// exp(x) - 1 for |x| <= 0.1 is its Taylor series to degree 5 (relative error below
+// x^5 / 720 < 2e-8); larger noise scales use expm1f.
+#include <algorithm>
+#include <cmath>
+
+#include "dust_device.cuh"
+#include "dust_internal.h"
+
+namespace dust {
+namespace {
+
+constexpr int kChunk = 128;   // slab channels per noise block
+constexpr int kTokB = 128;    // tokens per noise block
+constexpr int kNoiseThreads = 256;
+constexpr int kStride = kTokB + 1;  // padded row of the staged weights (conflict-free)
+
+template <typename T>
+__device__ __forceinline__ float load_logit(const T* p);
+template <>
+__device__ __forceinline__ float load_logit<float>(const float* p) {
+    return __ldg(p);
+}
+template <>
+__device__ __forceinline__ float load_logit<__nv_bfloat16>(const __nv_bfloat16* p) {
+    return __bfloat162float(*p);
+}
+
+struct CeArgs {
+    const void* z;
+    const int32_t* y;
+    float4* stats;    // [N]: zmax, E, target valid (1/0), unused
+    float* partial;   // [n_chunks, K, N]
+    float* dloss;     // [K, ld]
+    int64_t ld_z, ld, N;
+    int V, v0, S, K, n_chunks;
+    float sigma;
+    NoiseKey key;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) ce_stats_kernel(const CeArgs a) {
+    const int64_t t = blockIdx.x;
+    const T* zt = static_cast<const T*>(a.z) + t * a.ld_z;
+    float m = -INFINITY, s = 0.f;
+    for (int v = threadIdx.x; v < a.V; v += blockDim.x) {
+        const float zv = load_logit<T>(zt + v);
+        if (zv > m) {
+            s = s * __expf(m - zv) + 1.f;
+            m = zv;
+        } else {
+            s += __expf(zv - m);
+        }
+    }
+    // combine (m, s) pairs: warp shuffles, then the warps through shared memory
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+        const float s2 = __shfl_xor_sync(0xffffffffu, s, off);
+        const float mm = fmaxf(m, m2);
+        s = (m == -INFINITY ? 0.f : s * __expf(m - mm)) + (m2 == -INFINITY ? 0.f : s2 * __expf(m2 - mm));
+        m = mm;
+    }
+    __shared__ float sm_m[32], sm_s[32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        sm_m[warp] = m;
+        sm_s[warp] = s;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int nw = blockDim.x >> 5;
+        m = lane < nw ? sm_m[lane] : -INFINITY;
+        s = lane < nw ? sm_s[lane] : 0.f;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+            const float s2 = __shfl_xor_sync(0xffffffffu, s, off);
+            const float mm = fmaxf(m, m2);
+            s = (m == -INFINITY ? 0.f : s * __expf(m - mm)) + (m2 == -INFINITY ? 0.f : s2 * __expf(m2 - mm));
+            m = mm;
+        }
+        if (lane == 0) {
+            const int y = a.y[t];
+            a.stats[t] = make_float4(m, s, (y >= 0 && y < a.V) ? 1.f : 0.f, 0.f);
+        }
+    }
+}
+
+// exp(x) - 1: degree-5 Taylor series for |x| <= 0.1, else the library expm1f.
+template <bool kSeries>
+__device__ __forceinline__ float em1(float x) {
+    if (kSeries) {
+        float p = fmaf(x, 1.f / 120.f, 1.f / 24.f);
+        p = fmaf(x, p, 1.f / 6.f);
+        p = fmaf(x, p, 0.5f);
+        p = fmaf(x, p, 1.f);
+        return x * p;
+    }
+    return expm1f(x);
+}
+
+template <typename T, bool kSeries>
+__global__ void __launch_bounds__(kNoiseThreads) ce_noise_kernel(const CeArgs a) {
+    extern __shared__ float w[];  // [kChunk][kStride]: exp(z - zmax), channel-major
+    const int chunk = blockIdx.x;
+    const int64_t t0 = static_cast<int64_t>(blockIdx.y) * kTokB;
+    const int c0 = a.v0 + chunk * kChunk;                 // first vocabulary index of the chunk
+    const int nch = min(kChunk, a.v0 + a.S - c0);         // channels of this chunk (multiple of 4)
+    // stage w: a warp reads 32 consecutive channels of one token row
+    for (int idx = threadIdx.x; idx < kTokB * kChunk; idx += kNoiseThreads) {
+        const int r = idx / kChunk, j = idx % kChunk;
+        const int64_t t = t0 + r;
+        float v = 0.f;
+        if (t < a.N && j < nch) {
+            const float zmax = a.stats[t].x;
+            v = __expf(load_logit<T>(static_cast<const T*>(a.z) + t * a.ld_z + c0 + j) - zmax);
+        }
+        w[j * kStride + r] = v;
+    }
+    __syncthreads();
+    const int lt = threadIdx.x % kTokB;
+    const int half = threadIdx.x / kTokB;
+    const int64_t t = t0 + lt;
+    const uint32_t tg = a.key.token_offset + static_cast<uint32_t>(t);
+    const uint32_t q0 = static_cast<uint32_t>(c0 >> 2);
+    const int nq = nch >> 2;
+    const float sigma = a.sigma;
+    for (int i = half; i < a.K; i += kNoiseThreads / kTokB) {
+        const uint32_t di = a.key.draw_offset + static_cast<uint32_t>(i);
+        float acc0 = 0.f, acc1 = 0.f;
+        for (int q = 0; q < nq; ++q) {
+            const F4 z = normal_quad(q0 + q, tg, di, a.key.layer, a.key);
+            const float* wq = w + (4 * q) * kStride + lt;
+            acc0 = fmaf(wq[0], em1<kSeries>(sigma * z.x), acc0);
+            acc1 = fmaf(wq[kStride], em1<kSeries>(sigma * z.y), acc1);
+            acc0 = fmaf(wq[2 * kStride], em1<kSeries>(sigma * z.z), acc0);
+            acc1 = fmaf(wq[3 * kStride], em1<kSeries>(sigma * z.w), acc1);
+        }
+        if (t < a.N) a.partial[(static_cast<int64_t>(chunk) * a.K + i) * a.N + t] = acc0 + acc1;
+    }
+}
+
+__global__ void ce_finish_kernel(const CeArgs a) {
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= static_cast<int64_t>(a.K) * a.N) return;
+    const int i = static_cast<int>(idx / a.N);
+    const int64_t t = idx % a.N;
+    float X = 0.f;
+    for (int c = 0; c < a.n_chunks; ++c) X += a.partial[(static_cast<int64_t>(c) * a.K + i) * a.N + t];
+    const float4 st = a.stats[t];
+    float dl = log1pf(X / st.y);
+    const int y = a.y[t];
+    if (st.z == 0.f) {
+        dl = __int_as_float(0x7fc00000);  // target outside the vocabulary
+    } else if (y >= a.v0 && y < a.v0 + a.S) {
+        const F4 z = normal_quad(static_cast<uint32_t>(y) >> 2, a.key.token_offset + static_cast<uint32_t>(t),
+                                 a.key.draw_offset + static_cast<uint32_t>(i), a.key.layer, a.key);
+        const float ay = (y & 3) == 0 ? z.x : (y & 3) == 1 ? z.y : (y & 3) == 2 ? z.z : z.w;
+        dl -= a.sigma * ay;
+    }
+    a.dloss[static_cast<int64_t>(i) * a.ld + t] = dl;
+}
+
+template <typename T>
+dust_status launch_typed(CeArgs& a, cudaStream_t s) {
+    prof_begin(s);
+    ce_stats_kernel<T><<<static_cast<unsigned>(a.N), 256, 0, s>>>(a);
+    prof_end(s, "lmhead_ce_stats");
+    const size_t smem = static_cast<size_t>(kChunk) * kStride * 4;
+    const bool series = std::fabs(a.sigma) * 5.8f <= 0.1f;
+    auto kern = series ? ce_noise_kernel<T, true> : ce_noise_kernel<T, false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return DUST_ERR_CUDA;
+    if (a.n_chunks > 0) {
+        const dim3 grid(static_cast<unsigned>(a.n_chunks),
+                        static_cast<unsigned>((a.N + kTokB - 1) / kTokB));
+        prof_begin(s);
+        kern<<<grid, kNoiseThreads, smem, s>>>(a);
+        prof_end(s, "lmhead_ce_noise");
+    }
+    const int64_t total = static_cast<int64_t>(a.K) * a.N;
+    prof_begin(s);
+    ce_finish_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(a);
+    prof_end(s, "lmhead_ce_finish");
+    return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
+}
+
+}  // namespace
+
+size_t lmhead_workspace_bytes(int64_t N, int32_t S, int32_t K) {
+    const int64_t n_chunks = (S + kChunk - 1) / kChunk;
+    return align_up(static_cast<size_t>(N) * 16, 256) +
+           align_up(static_cast<size_t>(n_chunks) * K * N * 4, 256);
+}
+
+dust_status lmhead_launch(const void* z, int64_t ld_z, dust_dtype dt, const int32_t* y, int64_t N,
+                          int32_t V, int32_t v0, int32_t S, int32_t K, float sigma, NoiseKey key,
+                          float* dloss, int64_t ld, void* ws, cudaStream_t s) {
+    if (N > 2147483647LL || (N + kTokB - 1) / kTokB > 65535) return DUST_ERR_UNSUPPORTED;
+    CeArgs a;
+    a.z = z;
+    a.y = y;
+    a.stats = static_cast<float4*>(ws);
+    a.partial = reinterpret_cast<float*>(static_cast<char*>(ws) + align_up(static_cast<size_t>(N) * 16, 256));
+    a.dloss = dloss;
+    a.ld_z = ld_z;
+    a.ld = ld;
+    a.N = N;
+    a.V = V;
+    a.v0 = v0;
+    a.S = S;
+    a.K = K;
+    a.n_chunks = (S + kChunk - 1) / kChunk;
+    a.sigma = sigma;
+    a.key = key;
+    if (S == 0) a.n_chunks = 0;
+    return dt == DUST_BF16 ? launch_typed<__nv_bfloat16>(a, s) : launch_typed<float>(a, s);
+}
+
+}  // namespace dust

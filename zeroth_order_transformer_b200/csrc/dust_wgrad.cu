@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kGThreads) ghat_kernel(const __grid_constant__
 #pragma unroll 2
         for (int i = 0; i < T.K; ++i) {
             const float ri = __ldg(rt + static_cast<int64_t>(i) * L.ld_r);
-            const Polar4 z = normal_quad_polar(static_cast<uint32_t>(q), tg,
+            const Polar4 z = normal_quad_polar(static_cast<uint32_t>(q) + T.key.quad_offset, tg,
                                                T.key.draw_offset + static_cast<uint32_t>(i),
                                                L.layer_id, T.key);
             // r a = -(r rho) (cos, sin) per pair
@@ -103,7 +103,9 @@ constexpr uint32_t kGSmem = kGStages * kGStageBytes + 1024 + 256;
 constexpr uint32_t kGTmemCols = 256;
 
 struct GwLayer {
-    float* out;  // G_W (splits == 1) or partial [S, d_out, d_in]
+    float* out;  // G_W (splits == 1; may be null when an optimizer step consumes it) or
+                 // partial [S, d_out, d_in]
+    OptTargets opt;  // used when the table's optimizer kind is set and splits == 1
     int64_t tokens_per_split;
     int d_in, d_out, o_tiles, k_tiles, splits, tile_begin, accumulate;
 };
@@ -113,6 +115,7 @@ struct GwTable {
     CUtensorMap tmg[kMax];
     CUtensorMap tmx[kMax];
     GwLayer layer[kMax];
+    OptParams opt;  // kind 0: no optimizer step
     ErrorWord* ew;
     int64_t N;
     int n_layers;
@@ -209,7 +212,7 @@ __global__ void __launch_bounds__(kGWThreads, 1) gw_bf16_kernel(const __grid_con
     const int o = o0 + warp * 32 + lane;
     const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const int ncols = min(kGN, L.d_in - k0);
-    float* dst = L.out + static_cast<int64_t>(split) * L.d_out * L.d_in;
+    float* dst = L.out ? L.out + static_cast<int64_t>(split) * L.d_out * L.d_in : nullptr;
     for (int c = 0; c < ncols / 16; ++c) {
         float v[16];
         tmem_ld16(trow + c * 16, v);
@@ -219,7 +222,8 @@ __global__ void __launch_bounds__(kGWThreads, 1) gw_bf16_kernel(const __grid_con
             for (int j = 0; j < 16; ++j) v[j] = 0.f;
         }
         if (o < L.d_out) {
-            float4* d4 = reinterpret_cast<float4*>(dst + static_cast<int64_t>(o) * L.d_in + k0 + c * 16);
+            const int64_t e0 = static_cast<int64_t>(o) * L.d_in + k0 + c * 16;
+            float4* d4 = dst ? reinterpret_cast<float4*>(dst + e0) : nullptr;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 float4 w = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
@@ -230,7 +234,8 @@ __global__ void __launch_bounds__(kGWThreads, 1) gw_bf16_kernel(const __grid_con
                     w.z += old.z;
                     w.w += old.w;
                 }
-                d4[j] = w;
+                if (d4) d4[j] = w;
+                if (T.opt.kind != 0 && L.splits == 1) opt_update4(T.opt, L.opt, e0 + 4 * j, w);
             }
         }
     }
@@ -241,7 +246,8 @@ __global__ void __launch_bounds__(kGWThreads, 1) gw_bf16_kernel(const __grid_con
 
 struct SplitLayer {
     const float4* part;  // [S, n4]
-    float4* out;         // [n4]
+    float4* out;         // [n4], or null when an optimizer step consumes the sum
+    OptTargets opt;
     int64_t n4;
     int S, accumulate;
 };
@@ -249,9 +255,11 @@ struct SplitLayer {
 template <int kMax>
 struct SplitTable {
     SplitLayer layer[kMax];
+    OptParams opt;
 };
 
-// out = (accumulate ? out : 0) + sum_s part[s] in order s = 0 .. S-1; blockIdx.y = layer.
+// out = (accumulate ? out : 0) + sum_s part[s] in order s = 0 .. S-1, then the optimizer step
+// on that sum when one is set; blockIdx.y = layer.
 template <int kMax>
 __global__ void splitk_reduce_kernel(const __grid_constant__ SplitTable<kMax> T) {
     const SplitLayer& L = T.layer[blockIdx.y];
@@ -265,7 +273,8 @@ __global__ void splitk_reduce_kernel(const __grid_constant__ SplitTable<kMax> T)
             s.z += v.z;
             s.w += v.w;
         }
-        L.out[idx] = s;
+        if (L.out) L.out[idx] = s;
+        if (T.opt.kind != 0) opt_update4(T.opt, L.opt, 4 * idx, s);
     }
 }
 
@@ -340,7 +349,8 @@ size_t bf16_layer_ws(int64_t N, int32_t d_in, int32_t d_out, int S) {
 template <int kMax>
 dust_status launch_bf16_tables(const WgradLayerArgs* layers, int n, int64_t N, int32_t K_chunk,
                                int32_t K_total, float sigma, const NoiseKey& key, int accumulate,
-                               char* ws, cudaStream_t s) {
+                               char* ws, cudaStream_t s, const OptParams* opt = nullptr,
+                               const OptTargets* targets = nullptr) {
     int64_t tiles0 = 0;
     for (int l = 0; l < n; ++l) tiles0 += gw_tiles(layers[l].d_in, layers[l].d_out);
     const int S = choose_splits(tiles0, N);
@@ -377,10 +387,12 @@ dust_status launch_bf16_tables(const WgradLayerArgs* layers, int n, int64_t N, i
 
     // stage 2: G_W for every layer
     GwTable<kMax> W;
+    W.opt = opt ? *opt : OptParams{};
     W.ew = device_error_word();
     W.N = N;
     W.n_layers = n;
     SplitTable<kMax> R;
+    R.opt = W.opt;
     int n_split_layers = 0;
     int64_t max_n4 = 0;
     int64_t tiles = 0;
@@ -398,6 +410,7 @@ dust_status launch_bf16_tables(const WgradLayerArgs* layers, int n, int64_t N, i
         L.d_in = a.d_in;
         L.d_out = a.d_out;
         L.tile_begin = static_cast<int>(tiles);
+        L.opt = targets ? targets[l] : OptTargets{};
         tiles += static_cast<int64_t>(L.o_tiles) * L.k_tiles * S;
         if (tiles > 2147483647LL) return DUST_ERR_UNSUPPORTED;
         if (S == 1) {
@@ -409,6 +422,7 @@ dust_status launch_bf16_tables(const WgradLayerArgs* layers, int n, int64_t N, i
             SplitLayer& Rl = R.layer[n_split_layers++];
             Rl.part = reinterpret_cast<const float4*>(L.out);
             Rl.out = reinterpret_cast<float4*>(a.G_W);
+            Rl.opt = L.opt;
             Rl.n4 = static_cast<int64_t>(a.d_out) * a.d_in / 4;
             Rl.S = S;
             Rl.accumulate = accumulate;
@@ -475,12 +489,14 @@ dust_status wgrad_grouped_launch(const WgradLayerArgs* layers, int n, int64_t N,
 dust_status wgrad_launch(const float* r, int64_t ld_r, const void* x, dust_dtype dt, int64_t N,
                          int32_t d_in, int32_t d_out, int32_t K_chunk, int32_t K_total,
                          float sigma, NoiseKey key, float* G_W, int accumulate, float* g_out,
-                         void* ws, cudaStream_t s) {
+                         void* ws, cudaStream_t s, const OptParams* opt,
+                         const OptTargets* targets) {
     if (dt == DUST_BF16) {
         WgradLayerArgs a{r, ld_r, x, d_in, d_out, key.layer, G_W, g_out};
         return launch_bf16_tables<1>(&a, 1, N, K_chunk, K_total, sigma, key, accumulate,
-                                     static_cast<char*>(ws), s);
+                                     static_cast<char*>(ws), s, opt, targets);
     }
+    if (opt) return DUST_ERR_UNSUPPORTED;  // fp32 layers: call dust_optimizer_step
     // fp32: g in fp32 (into g_out when given, else the workspace), SIMT contraction.
     float* gf = g_out ? g_out : static_cast<float*>(ws);
     GhatTable<1> G;
