@@ -25,6 +25,10 @@ def z():
     return zz
 
 
+def _f32(x: float) -> float:
+    return float(np.float32(x))
+
+
 def _t(a):
     import torch
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
@@ -43,12 +47,14 @@ def test_optimizer_step_matches_oracle(z, kind, n):
     for t in range(1, 4):
         G = (rng.standard_normal(n) * 0.1).astype(np.float32)
         M = (0.9 * M + np.abs(G)) if kind == "sgd" else (0.9 * M + 0.1 * np.abs(G))
+        # the call's hyper-parameters are fp32 (dust_opt_params); the oracle reads those values
         if kind == "sgd":
             z.dust_optimizer_step(z.sgd_momentum(0.05, 0.9, 0.01), _t(G), W, m, W_bf16=Wb)
-            Wr, mr = oracle.sgd_momentum(Wr, mr, G, 0.05, 0.9, 0.01)
+            Wr, mr = oracle.sgd_momentum(Wr, mr, G, _f32(0.05), _f32(0.9), _f32(0.01))
         else:
             z.dust_optimizer_step(z.adam(1e-3, t, weight_decay=0.01), _t(G), W, m, v, W_bf16=Wb)
-            Wr, mr, vr = oracle.adam(Wr, mr, vr, G, 1e-3, 0.9, 0.999, 1e-8, t, 0.01)
+            Wr, mr, vr = oracle.adam(Wr, mr, vr, G, _f32(1e-3), _f32(0.9), _f32(0.999),
+                                     _f32(1e-8), t, _f32(0.01))
     torch.cuda.synchronize()
     np.testing.assert_allclose(_dev.host(W), Wr, rtol=2e-6, atol=1e-7)
     assert np.all(np.abs(_dev.host(m) - mr) <= 8 * 2.0**-24 * M)
