@@ -41,7 +41,11 @@ L2_FLUSH_BYTES = 256 << 20
 # consumer FMAs: 2 per normal in the forward, 1 in the draw reduction).
 LANES_PER_SM = 128
 OPS_PER_NORMAL = {"fwd_bf16_noise_loss": 20.0, "ghat_reduce_draws": 19.0,
-                  "fwd_bf16_noise_loss_grouped": 20.0, "ghat_reduce_draws_grouped": 19.0}
+                  "fwd_bf16_noise_loss_grouped": 20.0, "ghat_reduce_draws_grouped": 19.0,
+                  # LM head: generator 18 (Philox 10, uniform 3, Box-Muller 5), sigma a (1),
+                  # exp(sigma a) - 1 as a degree-5 series (5), the weighted sum (1)
+                  "lmhead_ce_noise": 25.0}
+HEAD_METRIC = "Dust LM-head estimator tokens*draws/s"
 
 
 def measured_peaks():
@@ -178,6 +182,24 @@ def kernel_work(name, wl, shapes):
     if name.startswith("credit_scan"):
         return "hbm", 8.0 * K * N * len(shapes), "bytes"
     return None, None, None
+
+
+def generator_ceiling(dust, torch, dev, reps: int = 10) -> float:
+    """Gnormal/s of the generator-only probe (generate and add, nothing else) over a grid of
+    8 x 256 threads per SM, 1024 normals each: what the noise kernels' generator can reach."""
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    n, nq = sms * 8 * 256, 256
+    out = torch.empty(n, dtype=torch.float32, device=dev)
+    key = dust.NoiseKey(0x5EED0000, 0)
+    for _ in range(3):
+        dust.dust_debug_normal_sum(key, n, nq, out)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        dust.dust_debug_normal_sum(key, n, nq, out)
+    b.record()
+    torch.cuda.synchronize(dev)
+    return 4.0 * n * nq * reps / (a.elapsed_time(b) / 1e3) / 1e9
 
 
 def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
@@ -334,6 +356,10 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                         "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None}
         if roofline is not None:
             roofline["peak_source"] = peaks["source"]
+            if bound == "alu":
+                gc = generator_ceiling(dust, torch, dev)
+                roofline["generator_ceiling"] = round(gc, 2)
+                roofline["frac_of_generator_ceiling"] = round(roofline["achieved"] / gc, 4)
 
     # ---- end to end through the public API, host buffers, copies inside the timed region
     e2e = None
@@ -451,6 +477,184 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     print(json.dumps(line), flush=True)
 
 
+def head_kernel_work(name, hw):
+    """Algorithmic work of one launch of the LM-head step's kernels."""
+    N, K = hw.N, hw.K
+    zb = 2 if hw.dtype == "bf16" else 4
+    if name in ("lmhead_ce_noise", "ghat_reduce_draws"):
+        return "alu", N * hw.S * K, "normals"
+    if name == "lmhead_ce_stats":
+        return "hbm", N * hw.V * zb + N * 16, "bytes"
+    if name.startswith("gw_bf16_tcgen05"):
+        return "tensor", 2.0 * N * hw.d_model * hw.S, "flops"
+    if name.startswith("credit_scan"):
+        return "hbm", 8.0 * K * N, "bytes"
+    return None, None, None
+
+
+def run_head(args) -> None:
+    """The LM-head estimator on cached logits: dust_noisy_logits_ce (cross-entropy change with
+    noise on the vocabulary slab) -> dust_credit -> dust_weight_grad on the slab's channels
+    (g and the slab's rows of the head weight estimate).  One GPU; one JSON line."""
+    import torch
+
+    import zeroth_order_transformer_b200 as dust
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    hw = workloads.HEAD_WORKLOADS[args.head]
+    data = workloads.generate_head(hw)
+    peaks = measured_peaks()
+
+    def dev_t(store):
+        if hw.dtype == "f32":
+            return torch.from_numpy(np.ascontiguousarray(store)).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(store).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+
+    z, h = dev_t(data.z_store), dev_t(data.h_store)
+    y = torch.from_numpy(data.y).to(dev)
+    cu = torch.from_numpy(data.cu_seqlens).to(dev)
+    dt = 1 if hw.dtype == "bf16" else 0
+    ws_bytes = max(dust.dust_workspace_size(dust.DUST_OP_LOGITS_CE, dt, hw.N, hw.V, hw.S, hw.K),
+                   dust.dust_workspace_size(dust.DUST_OP_CREDIT, 0, hw.N, 0, 0, hw.K),
+                   dust.dust_workspace_size(dust.DUST_OP_WEIGHT_GRAD, dt, hw.N, hw.d_model,
+                                            hw.S, hw.K))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    dloss = torch.empty((hw.K, hw.N), dtype=torch.float32, device=dev)
+    r = torch.empty_like(dloss)
+    GW = torch.empty((hw.S, hw.d_model), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    key = dust.NoiseKey(hw.seed, 48)
+    slab_key = key._replace(channel_offset=hw.v0)
+
+    def step(zz=z, yy=y, hh=h):
+        dust.dust_noisy_logits_ce(zz, yy, hw.v0, hw.S, hw.K, hw.sigma, key, dloss, ws)
+        dust.dust_credit(dloss, cu, hw.gamma, r, ws)
+        dust.dust_weight_grad(r, hh, hw.S, hw.K, hw.sigma, slab_key, GW, False, None, ws)
+        return GW
+
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    dust.dust_profile_enable(1 << 16)
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    prof = dust.dust_profile_read()
+    dust.dust_profile_disable()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    units = hw.N * hw.K
+    per = {}
+    for name, t in prof:
+        d = per.setdefault(name, [0, 0.0])
+        d[0] += 1
+        d[1] += t
+    tot = sum(v[1] for v in per.values())
+    kernels = {n: {"launches": c, "ms_total": round(t, 4), "ms_avg": round(t / c, 5),
+                   "share": round(t / tot, 4)}
+               for n, (c, t) in sorted(per.items(), key=lambda kv: -kv[1][1])}
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    roofline = None
+    for n, info in kernels.items():
+        bound, amount, what = head_kernel_work(n, hw)
+        if amount is None:
+            continue
+        rate = amount / (info["ms_avg"] / 1e3)
+        info[{"normals": "gnormals_per_s", "flops": "tflops", "bytes": "gbs"}[what]] = round(
+            rate / (1e12 if what == "flops" else 1e9), 2)
+        if roofline is None:
+            if bound == "alu":
+                ops = OPS_PER_NORMAL.get(n, 19.0)
+                peak = sms * LANES_PER_SM * peaks["sm_max_mhz"] * 1e6 / ops / 1e9
+                ach = rate / 1e9
+                roofline = {"kernel": n, "bound": "alu", "achieved": round(ach, 2),
+                            "peak": round(peak, 2), "unit": "Gnormal/s",
+                            "frac": round(ach / peak, 4), "traffic": None,
+                            "peak_basis": f"{sms} SMs x {LANES_PER_SM} lanes x "
+                                          f"{peaks['sm_max_mhz']:.0f} MHz / {ops:.0f} ops per "
+                                          f"normal", "peak_source": peaks["source"]}
+            elif bound == "hbm":
+                roofline = {"kernel": n, "bound": "hbm", "achieved": round(rate / 1e9, 2),
+                            "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": round(rate / 1e9 / peaks["hbm_gbs"], 4), "traffic": None,
+                            "peak_source": peaks["source"]}
+    if roofline is not None and roofline["bound"] == "alu":
+        gc = generator_ceiling(dust, torch, dev)
+        roofline["generator_ceiling"] = round(gc, 2)
+        roofline["frac_of_generator_ceiling"] = round(roofline["achieved"] / gc, 4)
+    # end to end: logits, targets and hidden states from pinned host memory, G_W back
+    e2e = None
+    if not args.no_e2e:
+        hz, hy, hh = (t.cpu().pin_memory() for t in (z, y, h))
+        dz, dy, dh = torch.empty_like(z), torch.empty_like(y), torch.empty_like(h)
+        hG = torch.empty(GW.shape, dtype=GW.dtype, pin_memory=True)
+
+        def e2e_step():
+            dz.copy_(hz, non_blocking=True)
+            dy.copy_(hy, non_blocking=True)
+            dh.copy_(hh, non_blocking=True)
+            hG.copy_(step(dz, dy, dh), non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for a, b in ee:
+            flush.zero_()
+            a.record(stream)
+            e2e_step()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = sum(a.elapsed_time(b) for a, b in ee) / args.steps
+        e2e = {"value": units / (e_ms / 1e3), "unit": UNIT, "ms_per_step": e_ms,
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (hz, hy, hh)),
+               "d2h_bytes_per_step": hG.numel() * hG.element_size()}
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        n_tok, done, t0 = 8, 0, time.perf_counter()
+        while time.perf_counter() - t0 < args.cpu_seconds:
+            t0_blk = (done // hw.K) % (hw.N - n_tok + 1)
+            idx = np.arange(t0_blk, t0_blk + n_tok)
+            loss, _ = oracle.noisy_logits_ce(data.z_f64, data.y, hw.v0, hw.S, hw.K, hw.sigma,
+                                             hw.seed, 48, tokens=idx)
+            rr = oracle.credit(loss, np.array([0, n_tok], dtype=np.int32), hw.gamma)
+            g = oracle.output_error(rr, hw.K, hw.sigma, hw.seed, hw.V, 48,
+                                    token_offset=int(t0_blk),
+                                    chans=np.arange(hw.v0, hw.v0 + hw.S))
+            oracle.weight_grad(g, data.h_f64[idx])
+            done += n_tok * hw.K
+        el = time.perf_counter() - t0
+        cpu = {"value": done / el, "unit": UNIT, "cores": oracle.get_threads(),
+               "kind": "oracle", "seconds": round(el, 2),
+               "sample": f"oracle (fp64 C, OpenMP) head estimator on blocks of {n_tok} tokens "
+                         f"(gamma = 0: tokens are independent) for about {args.cpu_seconds:.0f} s"}
+    line = {
+        "metric": HEAD_METRIC, "value": units / (ms / 1e3), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": f"{hw.dtype} logits, f32/u32 noise",
+        "data": "synthetic (seeded; the Dust page's head shape)",
+        "config": {"workload": f"{hw.name}: {hw.n_seq}x{hw.seq_len} tokens, vocabulary {hw.V}, "
+                               f"slab [{hw.v0}, {hw.v0 + hw.S}), width {hw.d_model}, K={hw.K}, "
+                               f"sigma={hw.sigma}, gamma={hw.gamma}",
+                   "l2": "flushed (256 MiB write) before every timed step"},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": sum(v["launches"] for v in kernels.values()), "clocks": clocks,
+        "kernels": kernels,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_credit_stress(args) -> None:
     """The credit step alone on a stress shape larger than L2 (default K = 64 draws x 4 Mi
     tokens: 1 GiB of losses in, 1 GiB of credit out), packed sequences U[256, 2048]; prints
@@ -508,9 +712,14 @@ def main():
                     help="time dust_credit alone on a shape larger than L2 and exit")
     ap.add_argument("--stress-K", type=int, default=64)
     ap.add_argument("--stress-N", type=int, default=1 << 22)
+    ap.add_argument("--head", choices=sorted(workloads.HEAD_WORKLOADS), default=None,
+                    help="time the LM-head estimator on cached logits instead and exit")
     args = ap.parse_args()
     if args.credit_stress:
         run_credit_stress(args)
+        return
+    if args.head:
+        run_head(args)
         return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -287,6 +287,14 @@ int32_t dust_profile_read(const char** names, float* ms, int32_t max);
 dust_status dust_debug_philox(const uint32_t* ctr, int64_t n, uint64_t seed, uint32_t* words,
                               float* normals, void* stream);
 
+/* Test and measurement support: the generator's throughput ceiling.  out[g] (DEVICE fp32
+ * [n]) = the sum of the normals a_t^(i)[o] of token t = key.token_offset + g, draw
+ * i = key.draw_offset, layer key.layer_id, channels o = key.channel_offset + 0 .. 4 n_quads - 1
+ * (the estimator's mapping).  The kernel only generates and adds (one add per normal), so
+ * its rate bounds what the noise kernels can reach.  key.channel_offset a multiple of 4. */
+dust_status dust_debug_normal_sum(dust_noise_key key, int64_t n, int32_t n_quads, float* out,
+                                  void* stream);
+
 /* Test support: the next dust_credit launch on any stream skips publishing the look-back
  * status of token block `block` (-1: none), so that the block before it waits until its
  * bounded wait runs out.  Used to test the timeout path; never set in normal use. */

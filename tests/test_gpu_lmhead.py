@@ -91,3 +91,40 @@ def test_lm_head_estimate_matches_oracle_chain(z):
     GW_ref = oracle.weight_grad(g_ref, H.x_f64)
     assert _dev.rel_fro(_dev.host(g), g_ref) <= _dev.GW_FRO
     assert _dev.rel_fro(_dev.host(GW), GW_ref) <= _dev.GW_FRO
+
+
+def test_head_workload_full_size_sampled(z):
+    """The benchmarked head workload (16k tokens, vocabulary 4096, slab of 1024, K = 256) in
+    the bench's launch configuration.  The oracle computes blocks of sampled tokens one by one
+    (gamma = 0, so a token's credit needs only its own draws): loss change, credit and g on
+    every slab channel.  G_W is checked through its definition against the GPU's own fp32 g
+    (the sampled rows of which are pinned above), with the bf16 rounding bound of g."""
+    import torch
+    hw = workloads.HEAD_WORKLOADS["head-4096-slab1024"]
+    data = workloads.generate_head(hw)
+    zt = _dev.to_device(data.z_store, hw.dtype)
+    h = _dev.to_device(data.h_store, hw.dtype)
+    y = torch.from_numpy(data.y).cuda()
+    cu = _dev.cu_to_device(data.cu_seqlens)
+    key = z.NoiseKey(hw.seed, 48)
+    dl = z.dust_noisy_logits_ce(zt, y, hw.v0, hw.S, hw.K, hw.sigma, key)
+    r = z.dust_credit(dl, cu, hw.gamma)
+    GW, g = z.dust_weight_grad(r, h, hw.S, hw.K, hw.sigma, key._replace(channel_offset=hw.v0),
+                               g_out=True)
+    torch.cuda.synchronize()
+    assert z.dust_last_device_error()[0] == 0
+    dl_h, r_h, g_h = _dev.host(dl), _dev.host(r), _dev.host(g)
+    chans = np.arange(hw.v0, hw.v0 + hw.S)
+    for t0 in (0, 2047, 9000, hw.N - 8):          # sequence starts, a boundary, the tail
+        idx = np.arange(t0, t0 + 8)
+        loss, clean = oracle.noisy_logits_ce(data.z_f64, data.y, hw.v0, hw.S, hw.K, hw.sigma,
+                                             hw.seed, 48, tokens=idx)
+        _dev.assert_fp32_close(dl_h[:, idx], loss - clean, f"dloss @{t0}")
+        rr = oracle.credit(loss, np.array([0, 8], dtype=np.int32), hw.gamma)
+        _dev.assert_fp32_close(r_h[:, idx], rr, f"r @{t0}")
+        gr = oracle.output_error(rr, hw.K, hw.sigma, hw.seed, hw.V, 48, token_offset=t0,
+                                 chans=chans)
+        _dev.assert_fp32_close(g_h[idx], gr, f"g @{t0}")
+    g64 = g.double()
+    ref = (g64.t() @ h.double()).cpu().numpy()
+    assert _dev.rel_fro(_dev.host(GW), ref) <= _dev.GW_FRO

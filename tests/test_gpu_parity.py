@@ -2,9 +2,11 @@
 
 Tolerances, from the arithmetic:
   * Philox words and all integer/segment logic: bit-exact.
-  * Normals: the kernels evaluate Box-Muller in fp32 with logf (about 1 ulp), x * rsqrtf(x)
-    (2 ulp) and the fast sine/cosine on (-pi, pi) (absolute error 2^-21.41); with |z| <= 5.77
-    the bound is a few 1e-6, tested at 1e-5 absolute.
+  * Normals: the kernels evaluate Box-Muller in fp32: the hardware base-2 logarithm (absolute
+    error about 2^-22, replaced by an exact-input series for u > 1 - 2^-10), y * rsqrt(y)
+    (2 ulp), the angle in one FMA (at most 3.5e-7 rad) and the hardware sine/cosine on
+    [-pi, pi) (absolute error about 2^-21); with |z| <= 5.77 the bound is a few 1e-6, tested
+    at 1e-5 absolute.
   * Loss change and fp32 g: sums of d_out (or K) terms in fp32 whose inputs carry the normal
     error above: element error <= 1e-3 x RMS, relative Frobenius error <= 1e-4.
   * G_W (bf16): g enters the tensor cores rounded to bf16 (relative rounding error up to 2^-9,
@@ -69,6 +71,17 @@ def test_normals_near_u_one_and_u_zero():
     err = np.abs(zn[extreme] - z_ref[extreme]).max()
     print(f"max error at u0 < 0.001 or u0 > 0.999: {err:.3e}")
     assert err <= _dev.NORMAL_ATOL
+
+
+def test_generator_throughput_probe_sums_the_mapped_normals():
+    """dust_debug_normal_sum (the generator-only rate probe) adds exactly the estimator's
+    normals: token offset, draw offset, layer and channel offset all enter the counter."""
+    n, nq, c0 = 300, 17, 8
+    key = z.NoiseKey(0x5EED0002, layer_id=9, draw_offset=5, token_offset=1000, channel_offset=c0)
+    got = _dev.host(z.dust_debug_normal_sum(key, n, nq)).astype(np.float64)
+    a = oracle.noise(key.seed, 9, n, c0 + 4 * nq, 1, draw_offset=5, token_offset=1000)
+    ref = a[0, :, c0:].sum(axis=1)
+    assert np.abs(got - ref).max() <= 4 * nq * _dev.NORMAL_ATOL
 
 
 # ------------------------------------------------------------------------- forward

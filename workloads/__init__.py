@@ -194,3 +194,59 @@ def dyadic_losses(seed: int, K: int, N: int, scale_bits: int = 8, max_abs: int =
 def gaussian_losses(seed: int, K: int, N: int, scale: float = 1.0) -> np.ndarray:
     rng = np.random.default_rng(seed)
     return (rng.standard_normal((K, N)) * scale).astype(np.float32)
+
+
+# ------------------------------------------------------------------------------ LM head
+@dataclasses.dataclass(frozen=True)
+class HeadWorkload:
+    """The output layer perturbed on its cached logits: N tokens of hidden width d_model, a
+    vocabulary of V entries, noise on the slab [v0, v0 + S), K draws, noise scale sigma,
+    discount gamma (0: the head's noise changes only its own token's loss)."""
+    name: str
+    n_seq: int
+    seq_len: int
+    d_model: int
+    V: int
+    v0: int
+    S: int
+    K: int
+    sigma: float
+    gamma: float
+    dtype: str
+    seed: int
+    logit_std: float = 2.0
+
+    @property
+    def N(self) -> int:
+        return self.n_seq * self.seq_len
+
+
+# The Dust page's setting (section "설정": 4096-entry BPE vocabulary, width 512, batches of
+# 8 x 2048 tokens), with a quarter of the vocabulary as the noisy slab and a population of
+# 256 draws, larger than the hidden layers' because the head's draws cost no forward pass.
+HEAD_WORKLOADS = {
+    "head-4096-slab1024": HeadWorkload("head-4096-slab1024", 8, 2048, 512, 4096, 1024, 1024,
+                                       256, 1e-2, 0.0, "bf16", NOISE_SEED_BASE + 6),
+}
+
+
+@dataclasses.dataclass
+class HeadData:
+    wl: HeadWorkload
+    z_store: np.ndarray   # logits [N, V] (bf16 bits or float32)
+    z_f64: np.ndarray
+    y: np.ndarray         # int32 [N] targets, uniform over the vocabulary
+    h_store: np.ndarray   # hidden states [N, d_model] (the head's input)
+    h_f64: np.ndarray
+    cu_seqlens: np.ndarray
+
+
+def generate_head(wl: HeadWorkload, data_seed: int = 1006) -> HeadData:
+    """Logits ~ N(0, logit_std^2), targets uniform on [0, V), hidden states ~ N(0, 1); draw
+    order logits, targets, hidden states; sequences of seq_len tokens."""
+    rng = np.random.default_rng(data_seed)
+    zs, z64 = _draw(rng, (wl.N, wl.V), wl.logit_std, wl.dtype)
+    y = rng.integers(0, wl.V, size=wl.N).astype(np.int32)
+    hs, h64 = _draw(rng, (wl.N, wl.d_model), 1.0, wl.dtype)
+    cu = cu_seqlens_from_lengths([wl.seq_len] * wl.n_seq)
+    return HeadData(wl, zs, z64, y, hs, h64, cu)

@@ -42,6 +42,7 @@ EXPORTED_SYMBOLS = (
     "dust_profile_read", "dust_credit_no_alloc", "dust_noisy_linear_fwd_grouped",
     "dust_credit_grouped", "dust_weight_grad_grouped", "dust_workspace_size_grouped",
     "dust_optimizer_step", "dust_weight_grad_step", "dust_noisy_logits_ce",
+    "dust_debug_normal_sum",
 )
 
 DUST_OPT_SGD_MOMENTUM = 1
@@ -142,6 +143,8 @@ def lib() -> ctypes.CDLL:
         L.dust_status_string.restype = ctypes.c_char_p
         L.dust_last_device_error.argtypes = [vp, ctypes.POINTER(i32)]
         L.dust_debug_philox.argtypes = [vp, i64, ctypes.c_uint64, vp, vp, vp]
+        L.dust_debug_normal_sum.argtypes = [dust_noise_key, i64, i32, vp, vp]
+        L.dust_debug_normal_sum.restype = ctypes.c_int
         L.dust_debug_credit_skip_publish.argtypes = [i32]
         L.dust_debug_credit_skip_publish.restype = None
         L.dust_profile_enable.argtypes = [i32]
@@ -375,6 +378,20 @@ def dust_debug_philox(ctr, seed: int, stream=None):
                                  normals.data_ptr(), _stream(ctr.device, stream))
     _check(st, "dust_debug_philox")
     return words, normals
+
+
+def dust_debug_normal_sum(key: NoiseKey, n: int, n_quads: int, out=None, device=None,
+                          stream=None):
+    """out[g] = sum of the 4 n_quads normals of token key.token_offset + g (draw
+    key.draw_offset, channels from key.channel_offset): the generator-only throughput probe."""
+    torch = _torch()
+    if out is None:
+        out = torch.empty(n, dtype=torch.float32, device=device or "cuda")
+    _cuda(out, "out")
+    st = lib().dust_debug_normal_sum(key.c(), n, n_quads, out.data_ptr(),
+                                     _stream(out.device, stream))
+    _check(st, "dust_debug_normal_sum")
+    return out
 
 
 def dust_debug_credit_skip_publish(block: int) -> None:

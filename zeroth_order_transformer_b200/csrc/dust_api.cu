@@ -38,6 +38,26 @@ __global__ void philox_debug_kernel(const uint32_t* __restrict__ ctr, int64_t n,
     }
 }
 
+// Generator throughput probe: thread g sums the normals of the quads (j, g, 0, layer) for
+// j < n_quads.  Generation plus one add per normal and nothing else, so its rate is the
+// ceiling that the noise kernels' generator reaches on the device.
+__global__ void __launch_bounds__(256) normal_sum_kernel(const __grid_constant__ NoiseKey key,
+                                                         int64_t n, int32_t n_quads, float* out) {
+    for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < n;
+         g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const uint32_t t = key.token_offset + static_cast<uint32_t>(g);
+        float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 2
+        for (int32_t j = 0; j < n_quads; ++j) {
+            const Polar4 z = normal_quad_polar(key.quad_offset + static_cast<uint32_t>(j), t,
+                                               key.draw_offset, key.layer, key);
+            acc0 = fmaf(z.q0, z.c0 + z.s0, acc0);
+            acc1 = fmaf(z.q1, z.c1 + z.s1, acc1);
+        }
+        out[g] = -kKappa * (acc0 + acc1);
+    }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -143,6 +163,16 @@ dust_status philox_debug_launch(const uint32_t* ctr, int64_t n, NoiseKey key, ui
     prof_begin(s);
     philox_debug_kernel<<<blocks, 256, 0, s>>>(ctr, n, key, words, normals);
     prof_end(s, "philox_debug");
+    return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
+}
+
+dust_status normal_sum_launch(NoiseKey key, int64_t n, int32_t n_quads, float* out,
+                              cudaStream_t s) {
+    if (n == 0) return DUST_OK;
+    const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, static_cast<int64_t>(num_sms()) * 8));
+    prof_begin(s);
+    normal_sum_kernel<<<blocks, 256, 0, s>>>(key, n, n_quads, out);
+    prof_end(s, "normal_sum_probe");
     return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
 }
 
@@ -337,6 +367,17 @@ dust_status dust_debug_philox(const uint32_t* ctr, int64_t n, uint64_t seed, uin
     dust_noise_key k{seed, 0, 0, 0, 0};
     return philox_debug_launch(ctr, n, make_key(k), words, normals,
                                static_cast<cudaStream_t>(stream));
+}
+
+dust_status dust_debug_normal_sum(dust_noise_key key, int64_t n, int32_t n_quads, float* out,
+                                  void* stream) {
+    if (n < 0 || n_quads < 0 || (n > 0 && !out) || key.channel_offset % 4 != 0)
+        return DUST_ERR_INVALID_ARG;
+    if (static_cast<uint64_t>(key.token_offset) + static_cast<uint64_t>(n) > 0x100000000ull ||
+        static_cast<uint64_t>(key.channel_offset / 4) + static_cast<uint64_t>(n_quads) >
+            0x100000000ull)
+        return DUST_ERR_INVALID_ARG;
+    return normal_sum_launch(make_key(key), n, n_quads, out, static_cast<cudaStream_t>(stream));
 }
 
 void dust_debug_credit_skip_publish(int32_t block) { g_credit_skip_publish = block; }

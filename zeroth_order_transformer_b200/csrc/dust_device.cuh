@@ -94,53 +94,62 @@ __device__ __forceinline__ float cos_approx(float x) {
     return y;
 }
 
-// X = -2 ln u for u in [2^-24, 1 - 2^-24], from the hardware base-2 logarithm.  Its small
-// absolute error is amplified in rho = sqrt(X) by 1 / (2 rho), which matters only for u close
-// to 1; there (u > 1 - 2^-10) the Taylor series of
-// -2 ln(1 - v) = 2v + v^2 + (2/3) v^3 + (1/2) v^4 + ... in the exact v = 1 - u replaces it (the
-// omitted terms are below v^3 / 4 relative, i.e. under 2^-32).
-__device__ __forceinline__ float neg2_ln_fast(float u) {
-    return -1.3862943611198906f * lg2_approx(u);  // -2 ln(2) log2(u)
-}
-__device__ __forceinline__ float neg2_ln_near_one(float u, float x_fast) {
+// y = -log2 u for u in [2^-24, 1 - 2^-24], from the hardware base-2 logarithm.  Its small
+// absolute error is amplified in q = sqrt(y) by 1 / (2 q), which matters only for u close to
+// 1; there (u > 1 - 2^-10) the Taylor series -log2(1 - v) = (v + v^2/2 + v^3/3 + ...) / ln 2
+// in the exact v = 1 - u replaces it (the omitted terms are below v^3 / 4 relative, i.e.
+// under 2^-32).
+__device__ __forceinline__ float neg_lg2_near_one(float u, float y_fast) {
     if (u > 0.9990234375f) {
         const float v = 1.0f - u;
-        return v * fmaf(v, fmaf(v, 0.6666666667f, 1.0f), 2.0f);
+        return v * fmaf(v, fmaf(v, 0.48089834696298783f, 0.72134752044448170f),
+                        1.4426950408889634f);  // 1/(3 ln 2), 1/(2 ln 2), 1/ln 2
     }
-    return x_fast;
+    return y_fast;
 }
 // Words whose uniform exceeds 1 - 2^-10 have their top ten bits set.
 constexpr uint32_t kNearOneWord = 0xFFC00000u;
+
+// rho = sqrt(-2 ln u) = kKappa sqrt(-log2 u), kKappa = sqrt(2 ln 2).
+constexpr float kKappa = 1.1774100225154747f;
+
+// Box-Muller angle shifted by -pi, from the word in one FMA: with m = w >> 9 the float
+// f = 2 + m 2^-22 (exponent 1, mantissa m) gives 2 pi u(w) - pi = pi f - 3 pi + 2 pi 2^-24,
+// which lies in [-pi, pi).  (Largest error over all m: 3.5e-7 rad.)
+__device__ __forceinline__ float angle_from_word(uint32_t w) {
+    return fmaf(3.14159265358979323846f, __uint_as_float(0x40000000u | (w >> 9)),
+                -9.4247775872730683f);  // -3 pi + 2 pi 2^-24
+}
 
 struct F4 {
     float x, y, z, w;
 };
 
-// Box-Muller on one Philox block in polar form: pair p (words 2p, 2p+1) has radius
-// rho_p = sqrt(x_p), x_p = -2 ln u(w_2p), and angle 2 pi u(w_2p+1).  The angle is shifted by
-// -pi into (-pi, pi), where the hardware sine/cosine keep their absolute error bound; the
-// shift flips both signs, cos(x - pi) = -cos x and sin(x - pi) = -sin x, so
-//     z_2p = -rho_p cos_p,   z_2p+1 = -rho_p sin_p,   z_2p^2 + z_2p+1^2 = x_p.
-// Consumers that need sums of a and a^2 use this form directly.
+// Box-Muller on one Philox block in scaled polar form: pair p (words 2p, 2p+1) has
+// y_p = -log2 u(w_2p) >= 0, q_p = sqrt(y_p) (so the radius is rho_p = kKappa q_p and
+// rho_p^2 = 2 ln 2 y_p) and angle 2 pi u(w_2p+1) - pi, where the hardware sine and cosine keep
+// their absolute error bound.  The -pi shift flips both signs, so
+//     z_2p = -kKappa q_p cos_p,   z_2p+1 = -kKappa q_p sin_p.
+// Consumers fold kKappa (and 2 ln 2) into their own coefficients.
 struct Polar4 {
-    float x0, r0, c0, s0;  // pair 0: channels 4q, 4q+1
-    float x1, r1, c1, s1;  // pair 1: channels 4q+2, 4q+3
+    float y0, q0, c0, s0;  // pair 0: channels 4q, 4q+1
+    float y1, q1, c1, s1;  // pair 1: channels 4q+2, 4q+3
 };
 
 __device__ __forceinline__ Polar4 box_muller_polar(const U4& w) {
     const float u0 = uniform_from_word(w.x);
     const float u2 = uniform_from_word(w.z);
     Polar4 p;
-    p.x0 = neg2_ln_fast(u0);
-    p.x1 = neg2_ln_fast(u2);
+    p.y0 = -lg2_approx(u0);
+    p.y1 = -lg2_approx(u2);
     if (max(w.x, w.z) >= kNearOneWord) {  // rare: about 1 block in 500
-        p.x0 = neg2_ln_near_one(u0, p.x0);
-        p.x1 = neg2_ln_near_one(u2, p.x1);
+        p.y0 = neg_lg2_near_one(u0, p.y0);
+        p.y1 = neg_lg2_near_one(u2, p.y1);
     }
-    p.r0 = p.x0 * rsqrt_approx(p.x0);
-    p.r1 = p.x1 * rsqrt_approx(p.x1);
-    const float a1 = fmaf(uniform_from_word(w.y), 6.28318530717958647692f, -3.14159265358979323846f);
-    const float a3 = fmaf(uniform_from_word(w.w), 6.28318530717958647692f, -3.14159265358979323846f);
+    p.q0 = p.y0 * rsqrt_approx(p.y0);
+    p.q1 = p.y1 * rsqrt_approx(p.y1);
+    const float a1 = angle_from_word(w.y);
+    const float a3 = angle_from_word(w.w);
     p.c0 = cos_approx(a1);
     p.s0 = sin_approx(a1);
     p.c1 = cos_approx(a3);
@@ -157,7 +166,8 @@ __device__ __forceinline__ Polar4 normal_quad_polar(uint32_t q, uint32_t t, uint
 __device__ __forceinline__ F4 normal_quad(uint32_t q, uint32_t t, uint32_t i, uint32_t layer,
                                           const NoiseKey& key) {
     const Polar4 p = normal_quad_polar(q, t, i, layer, key);
-    return F4{-p.r0 * p.c0, -p.r0 * p.s0, -p.r1 * p.c1, -p.r1 * p.s1};
+    const float r0 = -kKappa * p.q0, r1 = -kKappa * p.q1;
+    return F4{r0 * p.c0, r0 * p.s0, r1 * p.c1, r1 * p.s1};
 }
 
 // ----------------------------------------------------------------------------------------

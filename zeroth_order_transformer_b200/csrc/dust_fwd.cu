@@ -58,7 +58,8 @@ struct FwdTable {
     int64_t n_full;  // tiles processed whole, one CTA each (CTAs 0 .. n_full-1)
     int split;       // unit ranges per tile of the remaining tiles
     int n_layers, m_tiles, K;
-    float sigma, half_sigma2;
+    float sigma_k;  // kKappa sigma: scales the residual so the noise radius needs no kKappa
+    float h_lg2;    // sigma^2 ln 2: the quadratic term per unit of -log2 u
     NoiseKey key;
 };
 
@@ -185,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_bf16_kernel(const __grid_cons
         const uint32_t trow = tmem + (static_cast<uint32_t>(lq * 32) << 16);
         const int nchunks = min(kBN, L.d_out - n0) / 16;
 
-        // Phase 1: s_e = sigma (y - u), written back in place.
+        // Phase 1: s_e = kKappa sigma (y - u), written back in place.
         for (int c = grp; c < nchunks; c += kGroups) {
             float v[16];
             tmem_ld16(trow + c * 16, v);
@@ -197,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_bf16_kernel(const __grid_cons
                 unpack_bf16x8(__ldg(up), uf);
                 unpack_bf16x8(__ldg(up + 1), uf + 8);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) v[j] = T.sigma * (v[j] - uf[j]);
+                for (int j = 0; j < 16; ++j) v[j] = T.sigma_k * (v[j] - uf[j]);
             } else {
 #pragma unroll
                 for (int j = 0; j < 16; ++j) v[j] = 0.f;
@@ -211,12 +212,12 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_bf16_kernel(const __grid_cons
 
         // Phase 2: this CTA's units of the tile, dealt round-robin to the warp groups.  A unit
         // is (draw, half of the tile's channels): regenerate the noise and sum the loss change
-        // over the half's channels.  In polar form a pair (z, z') = -rho (cos, sin) contributes
-        // sigma (z e + z' e') + sigma^2 / 2 (z^2 + z'^2) = -rho (cos s_e + sin s_e') + h x,
-        // with x = rho^2 = -2 ln u.
+        // over the half's channels.  In polar form a pair (z, z') = -kKappa q (cos, sin)
+        // contributes sigma (z e + z' e') + sigma^2 / 2 (z^2 + z'^2)
+        //   = -q (cos s_e + sin s_e') + h y,   h = sigma^2 ln 2,  y = q^2 = -log2 u.
         const uint32_t tg = T.key.token_offset + static_cast<uint32_t>(t);
         const uint32_t qbase = static_cast<uint32_t>(n0 >> 2) + T.key.quad_offset;
-        const float h = T.half_sigma2;
+        const float h = T.h_lg2;
         const int half_chunks = (nchunks + 1) / 2;
         for (int unit = u_begin + grp; unit < u_end; unit += kGroups) {
             const int i = unit >> 1;
@@ -233,9 +234,9 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_bf16_kernel(const __grid_cons
                     const Polar4 z = normal_quad_polar(qbase + c * 4 + qq, tg, di, L.layer_id, T.key);
                     const float l0 = fmaf(z.s0, se[4 * qq + 1], z.c0 * se[4 * qq + 0]);
                     const float l1 = fmaf(z.s1, se[4 * qq + 3], z.c1 * se[4 * qq + 2]);
-                    acc[qq] = fmaf(-z.r0, l0, acc[qq]);
-                    acc[qq] = fmaf(-z.r1, l1, acc[qq]);
-                    acc[qq] = fmaf(h, z.x0 + z.x1, acc[qq]);
+                    acc[qq] = fmaf(-z.q0, l0, acc[qq]);
+                    acc[qq] = fmaf(-z.q1, l1, acc[qq]);
+                    acc[qq] = fmaf(h, z.y0 + z.y1, acc[qq]);
                 }
             }
             if (valid)
@@ -312,8 +313,8 @@ dust_status launch_bf16_table(const FwdLayerArgs* layers, int n, int64_t N, int 
     T.n_layers = n;
     T.m_tiles = static_cast<int>((N + kBM - 1) / kBM);
     T.K = K;
-    T.sigma = sigma;
-    T.half_sigma2 = 0.5f * sigma * sigma;
+    T.sigma_k = kKappa * sigma;
+    T.h_lg2 = static_cast<float>(0.69314718055994531 * sigma * sigma);
     T.key = key;
     int64_t tiles = 0;
     size_t off = 0;

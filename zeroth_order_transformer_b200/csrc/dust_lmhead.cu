@@ -139,17 +139,19 @@ __global__ void __launch_bounds__(kNoiseThreads) ce_noise_kernel(const CeArgs a)
     const uint32_t tg = a.key.token_offset + static_cast<uint32_t>(t);
     const uint32_t q0 = static_cast<uint32_t>(c0 >> 2);
     const int nq = nch >> 2;
-    const float sigma = a.sigma;
+    const float sk = -kKappa * a.sigma;
     for (int i = half; i < a.K; i += kNoiseThreads / kTokB) {
         const uint32_t di = a.key.draw_offset + static_cast<uint32_t>(i);
         float acc0 = 0.f, acc1 = 0.f;
         for (int q = 0; q < nq; ++q) {
-            const F4 z = normal_quad(q0 + q, tg, di, a.key.layer, a.key);
+            // sigma a = -(kKappa sigma q) (cos, sin) per pair
+            const Polar4 z = normal_quad_polar(q0 + q, tg, di, a.key.layer, a.key);
             const float* wq = w + (4 * q) * kStride + lt;
-            acc0 = fmaf(wq[0], em1<kSeries>(sigma * z.x), acc0);
-            acc1 = fmaf(wq[kStride], em1<kSeries>(sigma * z.y), acc1);
-            acc0 = fmaf(wq[2 * kStride], em1<kSeries>(sigma * z.z), acc0);
-            acc1 = fmaf(wq[3 * kStride], em1<kSeries>(sigma * z.w), acc1);
+            const float r0 = sk * z.q0, r1 = sk * z.q1;
+            acc0 = fmaf(wq[0], em1<kSeries>(r0 * z.c0), acc0);
+            acc1 = fmaf(wq[kStride], em1<kSeries>(r0 * z.s0), acc1);
+            acc0 = fmaf(wq[2 * kStride], em1<kSeries>(r1 * z.c1), acc0);
+            acc1 = fmaf(wq[3 * kStride], em1<kSeries>(r1 * z.s1), acc1);
         }
         if (t < a.N) a.partial[(static_cast<int64_t>(chunk) * a.K + i) * a.N + t] = acc0 + acc1;
     }

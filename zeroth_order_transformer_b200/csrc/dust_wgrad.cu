@@ -64,18 +64,19 @@ __global__ void __launch_bounds__(kGThreads) ghat_kernel(const __grid_constant__
             const Polar4 z = normal_quad_polar(static_cast<uint32_t>(q) + T.key.quad_offset, tg,
                                                T.key.draw_offset + static_cast<uint32_t>(i),
                                                L.layer_id, T.key);
-            // r a = -(r rho) (cos, sin) per pair
-            const float rr0 = ri * z.r0;
-            const float rr1 = ri * z.r1;
+            // r a = -kKappa (r q) (cos, sin) per pair; kKappa is applied with the scale
+            const float rr0 = ri * z.q0;
+            const float rr1 = ri * z.q1;
             a0 = fmaf(-rr0, z.c0, a0);
             a1 = fmaf(-rr0, z.s0, a1);
             a2 = fmaf(-rr1, z.c1, a2);
             a3 = fmaf(-rr1, z.s1, a3);
         }
-        a0 *= T.scale;
-        a1 *= T.scale;
-        a2 *= T.scale;
-        a3 *= T.scale;
+        const float sk = T.scale * kKappa;
+        a0 *= sk;
+        a1 *= sk;
+        a2 *= sk;
+        a3 *= sk;
         const int64_t off = t * L.d_out + 4 * q;
         if (L.gb) {
             __nv_bfloat162 lo = __floats2bfloat162_rn(a0, a1);
