@@ -75,6 +75,9 @@ def lib():
             _c_f64p, _c_i32p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
             ctypes.c_int32, ctypes.c_double, ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32,
             ctypes.c_uint32, _c_i64p, ctypes.c_int64, _c_f64p, _c_f64p]
+        L.oracle_attn_reward.argtypes = [_c_f64p, _c_f64p, ctypes.c_int32, ctypes.c_int64,
+                                         ctypes.c_int32, _c_f64p]
+        L.oracle_discounted_credit.argtypes = L.oracle_credit.argtypes
         L.oracle_set_threads.argtypes = [ctypes.c_int]
         L.oracle_get_threads.restype = ctypes.c_int
         _lib = L
@@ -164,6 +167,29 @@ def credit(loss, cu_seqlens, gamma: float, route: str = "double_sum") -> np.ndar
     r = np.zeros((K, N), dtype=np.float64)
     fn = lib().oracle_credit if route == "double_sum" else lib().oracle_credit_recurrence
     fn(_p(loss, _c_f64p), K, N, _p(cu, _c_i32p), cu.shape[0] - 1, float(gamma), _p(r, _c_f64p))
+    return r
+
+
+def attn_reward(ghat, dO) -> np.ndarray:
+    """c[K, N] = -<ghat_t, dO[i, t]>: the attention-internal reward (Dust page, "간섭 줄이기")."""
+    ghat, dO = _f64(ghat), _f64(dO)
+    N, d = ghat.shape
+    K = dO.shape[0]
+    assert dO.shape == (K, N, d)
+    c = np.zeros((K, N), dtype=np.float64)
+    lib().oracle_attn_reward(_p(ghat, _c_f64p), _p(dO, _c_f64p), K, N, d, _p(c, _c_f64p))
+    return c
+
+
+def discounted_credit(c, cu_seqlens, gamma: float) -> np.ndarray:
+    """r[K, N] = sum_{s >= t, same segment} gamma^(s-t) c_s: the credit equation on a given
+    reward, without centring."""
+    c = _f64(c)
+    K, N = c.shape
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    r = np.zeros((K, N), dtype=np.float64)
+    lib().oracle_discounted_credit(_p(c, _c_f64p), K, N, _p(cu, _c_i32p), cu.shape[0] - 1,
+                                   float(gamma), _p(r, _c_f64p))
     return r
 
 

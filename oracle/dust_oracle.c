@@ -14,6 +14,9 @@
  *   credit equation         r_t = sum_{s >= t} gamma^(s-t) c_s  (later tokens of the sequence)
  *   output-error equation   g_t = -(1/(K sigma)) sum_i r_t^(i) a_t^(i)
  *   weight-estimate eq.     G_W = sum_t g_t x_t^T
+ * and, for the "next" rows: the optimizer steps on G_W (section "설정", section "Adam에서도
+ * 통할까?"), the LM-head cross-entropy on cached logits and the attention-internal reward
+ * c_s = -<ghat_s, delta_o_s> (section "간섭(interference) 줄이기").
  * The page fixes no random generator.  The one used here is Philox4x32-10
  * (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as 1, 2, 3",
  * SC'11), written from that paper's description, with the Box-Muller transform
@@ -374,4 +377,50 @@ void oracle_noisy_logits_ce(const double* z, const int32_t* y, int64_t N, int32_
         }
         free(zp);
     }
+}
+
+/*
+ * Attention-internal reward (Dust page, section "간섭(interference) 줄이기", second point):
+ * a perturbation of the attention's internal projections (Q, K, V, gate) barely shows in
+ * the token loss, so draw i is rewarded at token s by how well the output-error estimate at
+ * the attention output, ghat_s, lines up with the change of that output under the draw:
+ *   c_s^(i) = -<ghat_s, delta_o_s^(i)>.
+ * The reward replaces the centred loss of the credit equation (no centring).
+ * ghat: [N][d]; dO: [K][N][d] (draw-major); c: [K][N].
+ */
+void oracle_attn_reward(const double* ghat, const double* dO, int32_t K, int64_t N, int32_t d,
+                        double* c)
+{
+#pragma omp parallel for schedule(static) collapse(2)
+    for (int32_t i = 0; i < K; ++i) {
+        for (int64_t t = 0; t < N; ++t) {
+            double acc = 0.0;
+            for (int32_t k = 0; k < d; ++k)
+                acc += ghat[t * d + k] * dO[((int64_t)i * N + t) * d + k];
+            c[(int64_t)i * N + t] = -acc;
+        }
+    }
+}
+
+/*
+ * The credit equation applied to a given reward c (no centring):
+ *   r_t^(i) = sum_{s = t}^{end(seg(t)) - 1} gamma^(s - t) c_s^(i)
+ * as the explicit double sum.  c, r: [K][N].
+ */
+void oracle_discounted_credit(const double* c, int32_t K, int64_t N, const int32_t* cu,
+                              int32_t n_seq, double gamma, double* r)
+{
+    int32_t* end = segment_end_of(cu, n_seq, N);
+#pragma omp parallel for schedule(dynamic, 16) collapse(2)
+    for (int32_t i = 0; i < K; ++i) {
+        for (int64_t t = 0; t < N; ++t) {
+            double acc = 0.0, g = 1.0;
+            for (int64_t s = t; s < end[t]; ++s) {
+                acc += g * c[(int64_t)i * N + s];
+                g *= gamma;
+            }
+            r[(int64_t)i * N + t] = acc;
+        }
+    }
+    free(end);
 }
