@@ -78,6 +78,16 @@ def lib():
         L.oracle_attn_reward.argtypes = [_c_f64p, _c_f64p, ctypes.c_int32, ctypes.c_int64,
                                          ctypes.c_int32, _c_f64p]
         L.oracle_discounted_credit.argtypes = L.oracle_credit.argtypes
+        L.oracle_spsa_directions.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32,
+                                             ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                             _c_f64p]
+        L.oracle_spsa_probe.argtypes = [
+            _c_f64p, _c_f64p, _c_f64p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+            ctypes.c_int32, ctypes.c_double, ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32,
+            _c_f64p, _c_f64p, _c_f64p]
+        L.oracle_spsa_estimate.argtypes = [_c_f64p, ctypes.c_int32, ctypes.c_int32,
+                                           ctypes.c_int32, ctypes.c_int32, ctypes.c_uint64,
+                                           ctypes.c_uint32, ctypes.c_uint32, _c_f64p]
         L.oracle_set_threads.argtypes = [ctypes.c_int]
         L.oracle_get_threads.restype = ctypes.c_int
         _lib = L
@@ -261,3 +271,36 @@ def noisy_logits_ce(z, y, v0: int, S: int, K: int, sigma: float, seed: int, laye
                                  int(seed), layer_id, draw_offset, token_offset, _p(tk, _c_i64p),
                                  n_tok, _p(loss, _c_f64p), _p(clean, _c_f64p))
     return loss, clean
+
+
+# --------------------------------------------------------------------------- SPSA / MeZO
+def spsa_directions(seed: int, layer_id: int, P: int, d_out: int, d_in: int,
+                    probe_offset: int = 0) -> np.ndarray:
+    """The probes' weight-space directions z_j [P, d_out, d_in] (bf16 values, as float64)."""
+    Z = np.zeros((P, d_out, d_in), dtype=np.float64)
+    lib().oracle_spsa_directions(int(seed), layer_id, probe_offset, P, d_out, d_in,
+                                 _p(Z, _c_f64p))
+    return Z
+
+
+def spsa_probe(x, W, u, P: int, eps: float, seed: int, layer_id: int = 0, probe_offset: int = 0):
+    """p_j = (L_+ - L_-) / (2 eps) from the two perturbed forwards of each probe; returns
+    (p [P], L_+ [P], L_- [P])."""
+    x, W, u = _f64(x), _f64(W), _f64(u)
+    N, d_in = x.shape
+    d_out = W.shape[0]
+    p, Lp, Lm = (np.zeros(P, dtype=np.float64) for _ in range(3))
+    lib().oracle_spsa_probe(_p(x, _c_f64p), _p(W, _c_f64p), _p(u, _c_f64p), N, d_in, d_out, P,
+                            float(eps), int(seed), layer_id, probe_offset, _p(p, _c_f64p),
+                            _p(Lp, _c_f64p), _p(Lm, _c_f64p))
+    return p, Lp, Lm
+
+
+def spsa_estimate(p, P_total: int, d_out: int, d_in: int, seed: int, layer_id: int = 0,
+                  probe_offset: int = 0) -> np.ndarray:
+    """(1/P_total) sum_j p_j z_j [d_out, d_in]."""
+    p = _f64(p)
+    G = np.zeros((d_out, d_in), dtype=np.float64)
+    lib().oracle_spsa_estimate(_p(p, _c_f64p), p.shape[0], P_total, d_out, d_in, int(seed),
+                               layer_id, probe_offset, _p(G, _c_f64p))
+    return G

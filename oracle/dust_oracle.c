@@ -424,3 +424,95 @@ void oracle_discounted_credit(const double* c, int32_t K, int64_t N, const int32
     }
     free(end);
 }
+
+/*
+ * SPSA / MeZO weight-space probe, the contrast estimator (thakicloud page, the SPSA paragraph:
+ * two forwards, with the perturbation added and subtracted, estimate the gradient of every
+ * parameter; gist.science 2605.15622 and the FedSPZO page: the perturbation is regenerated
+ * from a shared seed, so only scalars travel).  Probe j moves the whole weight matrix along
+ * z_j, drawn from the same generator in a separate counter space and stored at the weights'
+ * precision (bf16):
+ *   z_j[o][k] = bf16( normal of counter (k >> 2, o, probe_offset + j, layer_id | 2^31), index k & 3 )
+ * The two perturbed forwards give
+ *   L_+-^(j) = sum_t 1/2 || (W +- eps z_j) x_t - u_t ||^2,   p_j = (L_+ - L_-) / (2 eps),
+ * and the weight estimate is (1/P_total) sum_j p_j z_j.
+ */
+static double bf16_round(double v)
+{
+    /* round to nearest, ties to even, at 8 significant bits (bf16 keeps fp32's exponent range) */
+    if (v == 0.0) return 0.0;
+    int e;
+    frexp(v, &e);
+    const double s = ldexp(1.0, 8 - e);
+    return nearbyint(v * s) / s;
+}
+
+static double spsa_direction_at(uint64_t seed, uint32_t layer_id, uint32_t j, int32_t o, int32_t k)
+{
+    double z[4];
+    oracle_normal_quad(seed, (uint32_t)k >> 2, (uint32_t)o, j, layer_id | 0x80000000u, z);
+    return bf16_round(z[k & 3]);
+}
+
+/* z_j for j = probe_offset .. probe_offset + P - 1: Z [P][d_out][d_in]. */
+void oracle_spsa_directions(uint64_t seed, uint32_t layer_id, uint32_t probe_offset, int32_t P,
+                            int32_t d_out, int32_t d_in, double* Z)
+{
+#pragma omp parallel for collapse(2)
+    for (int32_t j = 0; j < P; ++j)
+        for (int32_t o = 0; o < d_out; ++o)
+            for (int32_t k = 0; k < d_in; ++k)
+                Z[((int64_t)j * d_out + o) * d_in + k] =
+                    spsa_direction_at(seed, layer_id, probe_offset + (uint32_t)j, o, k);
+}
+
+/* p: [P]; Lp, Lm: [P] (may be NULL). */
+void oracle_spsa_probe(const double* x, const double* W, const double* u, int64_t N, int32_t d_in,
+                       int32_t d_out, int32_t P, double eps, uint64_t seed, uint32_t layer_id,
+                       uint32_t probe_offset, double* p, double* Lp, double* Lm)
+{
+#pragma omp parallel
+    {
+        double* z = (double*)malloc(sizeof(double) * (size_t)d_out * (size_t)d_in);
+#pragma omp for schedule(dynamic, 1)
+        for (int32_t j = 0; j < P; ++j) {
+            for (int32_t o = 0; o < d_out; ++o)
+                for (int32_t k = 0; k < d_in; ++k)
+                    z[(int64_t)o * d_in + k] =
+                        spsa_direction_at(seed, layer_id, probe_offset + (uint32_t)j, o, k);
+            double lp = 0.0, lm = 0.0;
+            for (int64_t t = 0; t < N; ++t) {
+                const double* xt = x + t * d_in;
+                for (int32_t o = 0; o < d_out; ++o) {
+                    double yp = 0.0, ym = 0.0;
+                    for (int32_t k = 0; k < d_in; ++k) {
+                        const double w = W[(int64_t)o * d_in + k], dz = eps * z[(int64_t)o * d_in + k];
+                        yp += (w + dz) * xt[k];
+                        ym += (w - dz) * xt[k];
+                    }
+                    const double ep = yp - u[t * d_out + o], em = ym - u[t * d_out + o];
+                    lp += 0.5 * ep * ep;
+                    lm += 0.5 * em * em;
+                }
+            }
+            p[j] = (lp - lm) / (2.0 * eps);
+            if (Lp) Lp[j] = lp;
+            if (Lm) Lm[j] = lm;
+        }
+        free(z);
+    }
+}
+
+/* G [d_out][d_in] = (1/P_total) sum_{j < P} p_j z_j. */
+void oracle_spsa_estimate(const double* p, int32_t P, int32_t P_total, int32_t d_out, int32_t d_in,
+                          uint64_t seed, uint32_t layer_id, uint32_t probe_offset, double* G)
+{
+#pragma omp parallel for schedule(static)
+    for (int32_t o = 0; o < d_out; ++o)
+        for (int32_t k = 0; k < d_in; ++k) {
+            double acc = 0.0;
+            for (int32_t j = 0; j < P; ++j)
+                acc += p[j] * spsa_direction_at(seed, layer_id, probe_offset + (uint32_t)j, o, k);
+            G[(int64_t)o * d_in + k] = acc / (double)P_total;
+        }
+}
