@@ -2,18 +2,23 @@
 // draws of l_s minus l_s; r_t = sum_{s >= t} gamma^(s-t) c_s over later tokens of the same
 // sequence).
 //
-// One block per 128 tokens and a group of up to 128 draw rows.  The block brings its
-// [rows, 128] slab of losses into shared memory with bulk asynchronous copies, centres every
-// token over the draws, and runs, per draw row, a reverse scan of the affine maps
-// r_t = c_t + g_t r_{t+1} (g_t = gamma, or 0 at a segment's last token): each lane composes 4
-// consecutive tokens serially and the warp composes the 32 lane maps with shuffles.  Blocks
-// are chained from the end of the stream to its start by decoupled look-back: a block
-// publishes its aggregate map (A, G), r_first = A + G r_next, then its inclusive value once its
-// successor's is known.  Block indices come from an atomic ticket in reverse order, so a block
-// only ever waits for blocks that started before it.  Waits are bounded; a wait that runs out
-// records the error, writes NaN and still publishes, so no other block waits forever.
-// With more than 128 draws, a first kernel computes the per-token mean over all draws and the
-// rows are split into groups with independent look-back chains.
+// One block per 128 tokens and a group of up to 128 draw rows.  TMA brings the [rows, 128]
+// slab of losses into shared memory as four 32-token sub-slabs whose 128-byte lines are
+// swizzled (16-byte chunk c of row i sits at chunk c ^ (i mod 8)); the per-token mean over the
+// draws is taken by one thread per token.  Then four threads own each draw row, 32 tokens
+// each, held in registers: a thread centres its tokens and composes their affine maps
+// r_t = c_t + g_t r_{t+1} (g_t = gamma, or 0 at a segment's last token) serially, and the four
+// maps of a row are composed with shuffles.  Eight consecutive lanes hold eight different rows
+// of the same sub-slab, so every 16-byte shared access of a warp is conflict-free.  Blocks are
+// chained from the end of the stream to its start by decoupled look-back: each warp publishes
+// its rows' aggregate maps (A, G), r_first = A + G r_next, then their inclusive values once
+// the carry from the following blocks is known.  Block indices come from an atomic ticket in
+// reverse order, so a block only waits for blocks that started before it.  Waits are bounded;
+// a wait that runs out records the error, writes NaN and still publishes, so no other block
+// waits forever.  The credit is written back into the slab and stored by TMA.  With more than
+// 128 draws, a first kernel computes the per-token mean over all draws and the rows are split
+// into groups with independent look-back chains.  Leading dimensions that TMA cannot describe
+// fall back to plain loads and stores into the same layout.
 #include <algorithm>
 
 #include "dust_device.cuh"
@@ -25,15 +30,17 @@ int g_credit_skip_publish = -1;
 
 namespace {
 
-constexpr int kCB = 128;       // tokens per block
-constexpr int kThreads = 128;  // 4 warps; thread j centres token j
-constexpr int kRowsMax = 128;  // draw rows per block (row group)
-constexpr int kTPL = kCB / 32; // tokens per lane
-constexpr int kWarps = kThreads / 32;
-constexpr unsigned kAgg = 1u, kInc = 2u;
+constexpr int kCB = 128;          // tokens per block
+constexpr int kSeg = 4;           // threads per draw row
+constexpr int kTPT = kCB / kSeg;  // tokens per thread: one 128-byte line
+constexpr int kRowsMax = 128;     // draw rows per block (row group)
+constexpr int kRowsPerWarp = 8;
+constexpr int kMaxThreads = kRowsMax * kSeg;  // 512
 constexpr int kMaxGroup = 64;
 
 struct CreditLayer {
+    CUtensorMap tm_loss;  // [K, N] losses, 32 x rows_p boxes, 128-byte swizzle
+    CUtensorMap tm_r;     // [K, N] credit, same boxes
     const float* loss;
     float* r;
     float* mean;  // [N] per-token mean over all draws (only with several row groups)
@@ -50,96 +57,97 @@ struct CreditTable {
     ErrorWord* ew;
     int64_t N;
     size_t state_stride;
-    int n_seq, K, rows, n_groups, nblk, skip_publish, bulk;
+    int n_seq, K, rows, rows_p, n_groups, nblk, skip_publish, tma;
+    int centre;  // 1: centre the losses over the draws first; 0: scan the given reward
     float gamma;
 };
 
+int padded_rows(int rows) { return (rows + kRowsPerWarp - 1) / kRowsPerWarp * kRowsPerWarp; }
+
+// Look-back state of one row group: a ticket, then per (block, row) two self-validating 64-bit
+// words, so that no fence or separate flag is needed (a naturally aligned 64-bit store is seen
+// whole or not at all):
+//   aggregate  {A, -G}: published when the sign bit of the high word is set (G >= 0, so -G
+//              always has it, -0.0 included); all-zero bits mean "not yet";
+//   inclusive  {r_first, 1}: published when the high word is 1.
 size_t state_bytes(int64_t nblk, int rows) {
-    return 256 + align_up(static_cast<size_t>(nblk) * kWarps * 4, 256) +
-           align_up(static_cast<size_t>(nblk) * rows * 8, 256) +
-           align_up(static_cast<size_t>(nblk) * rows * 4, 256);
+    return 256 + 2 * align_up(static_cast<size_t>(nblk) * rows * 8, 256);
 }
 
-__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+size_t smem_bytes(int rows_p) {
+    return 1024 + static_cast<size_t>(rows_p) * kCB * 4 + 2 * kCB * 4 +
+           static_cast<size_t>(rows_p) * 4 * 3 + 16;
+}
+
+__device__ __forceinline__ uint64_t ld_relaxed64(const uint64_t* p) {
+    uint64_t v;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
-__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+__device__ __forceinline__ void st_relaxed64(uint64_t* p, uint64_t v) {
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
-// Bulk asynchronous copy of `bytes` (multiple of 16, 16-byte aligned) global -> shared.
-__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes,
-                                          uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(smem_dst)),
-        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-// Bulk asynchronous copy shared -> global, tracked by the thread's bulk group.
-__device__ __forceinline__ void bulk_store(void* dst, const void* smem_src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
-                     reinterpret_cast<uint64_t>(dst)),
-                 "r"(smem_u32(smem_src)), "r"(bytes)
-                 : "memory");
+__device__ __forceinline__ uint64_t pack2(float lo, uint32_t hi) {
+    return static_cast<uint64_t>(__float_as_uint(lo)) | (static_cast<uint64_t>(hi) << 32);
 }
 
-size_t smem_bytes(int rows) {
-    return static_cast<size_t>(rows) * kCB * 4 + static_cast<size_t>(rows) * 4 * 3 + kCB * 4 + 64;
+// Offset (floats) of (row i, token j) in the slab: sub-slab j / 32 of rows_p 128-byte lines,
+// 16-byte chunk (j % 32) / 4 of line i stored at chunk ((j % 32) / 4) ^ (i % 8).
+__device__ __forceinline__ int slab_at(int i, int j, int rows_p) {
+    return (j >> 5) * rows_p * kTPT + i * kTPT + ((((j & 31) >> 2) ^ (i & 7)) << 2) + (j & 3);
 }
 
-// Composes the affine maps of this lane's kTPL tokens (last token first): r_first = A + G r_next.
-__device__ __forceinline__ void lane_map(const float4& c, const float4& g, float& A, float& G) {
-    A = c.w;
-    G = g.w;
-    A = fmaf(g.z, A, c.z);
-    G = g.z * G;
-    A = fmaf(g.y, A, c.y);
-    G = g.y * G;
-    A = fmaf(g.x, A, c.x);
-    G = g.x * G;
-}
-
-// Inclusive reverse scan over lanes: lane l ends with the composition of lanes l .. 31.
-__device__ __forceinline__ void warp_suffix_scan(int lane, float& A, float& G) {
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const float A2 = __shfl_down_sync(0xffffffffu, A, off);
-        const float G2 = __shfl_down_sync(0xffffffffu, G, off);
-        if (lane + off < 32) {
-            A = fmaf(G, A2, A);
-            G = G * G2;
+// First s in [lo, n_seq] with cu[s] > x (n_seq + 1 if there is none), found by the whole
+// warp: each step probes 32 evenly spaced entries of the bracket at once and keeps the part
+// that holds the answer, so the dependent loads number log32 of the bracket, not log2.
+// cu is non-decreasing and every s < lo has cu[s] <= x.
+__device__ __forceinline__ int warp_upper_bound(const int32_t* cu, int n_seq, int64_t x, int lo,
+                                                int lane) {
+    int hi = n_seq + 1;  // the answer lies in [lo, hi]
+    while (lo < hi) {
+        const int p = lo + static_cast<int>((static_cast<int64_t>(hi - lo) * lane) >> 5);
+        const unsigned m = __ballot_sync(0xffffffffu, static_cast<int64_t>(__ldg(&cu[p])) > x);
+        if (m == 0) {
+            lo = __shfl_sync(0xffffffffu, p, 31) + 1;
+        } else {
+            const int k = __ffs(m) - 1;
+            const int pk = __shfl_sync(0xffffffffu, p, k);
+            const int pprev = __shfl_sync(0xffffffffu, p, k > 0 ? k - 1 : 0);
+            lo = k > 0 ? pprev + 1 : lo;
+            hi = pk;
         }
     }
+    return lo;
 }
 
 template <int kMax>
-__global__ void __launch_bounds__(kThreads) credit_kernel(const __grid_constant__ CreditTable<kMax> T) {
+__global__ void __launch_bounds__(kMaxThreads, 2) credit_kernel(const __grid_constant__ CreditTable<kMax> T) {
     const int lyr = blockIdx.y / T.n_groups;
     const int grp = blockIdx.y % T.n_groups;
     const CreditLayer& L = T.layer[lyr];
     char* state = L.state + static_cast<size_t>(grp) * T.state_stride;
     unsigned* ticket = reinterpret_cast<unsigned*>(state);
-    unsigned* flags = reinterpret_cast<unsigned*>(state + 256);  // [nblk][kWarps]
-    const size_t off_agg = 256 + align_up(static_cast<size_t>(T.nblk) * kWarps * 4, 256);
-    float2* agg = reinterpret_cast<float2*>(state + off_agg);
-    float* inc = reinterpret_cast<float*>(
-        state + off_agg + align_up(static_cast<size_t>(T.nblk) * T.rows * 8, 256));
+    uint64_t* aggw = reinterpret_cast<uint64_t*>(state + 256);  // [nblk][rows]
+    uint64_t* incw = reinterpret_cast<uint64_t*>(
+        state + 256 + align_up(static_cast<size_t>(T.nblk) * T.rows * 8, 256));  // [nblk][rows]
     const int row0 = grp * T.rows;
     const int R = min(T.rows, T.K - row0);
+    const int Rp = T.rows_p;
 
-    extern __shared__ float sm[];
-    float* slab = sm;                  // [R][kCB]: loss, then c, then r (16-byte rows)
-    float* gval = slab + R * kCB;      // [kCB]: gamma, or 0 at a segment's last token
-    float* aggA = gval + kCB;          // [R]
-    float* aggG = aggA + R;            // [R]
-    float* carry = aggG + R;           // [R]: r at the first token after the block
+    extern __shared__ uint8_t smem_raw[];
+    float* slab = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+    float* gval = slab + Rp * kCB;  // [kCB]: gamma, or 0 at a segment's last token
+    float* mean = gval + kCB;       // [kCB]
+    float* aggA = mean + kCB;       // [Rp]
+    float* aggG = aggA + Rp;        // [Rp]
+    float* carry = aggG + Rp;       // [Rp]: r at the first token after the block
     uint64_t* bar = reinterpret_cast<uint64_t*>(
-        (reinterpret_cast<uintptr_t>(carry + R) + 7) & ~static_cast<uintptr_t>(7));
-    __shared__ int s_blk;
+        (reinterpret_cast<uintptr_t>(carry + Rp) + 7) & ~static_cast<uintptr_t>(7));
+    __shared__ int s_blk, s_jend;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nthr = blockDim.x;
     if (tid == 0) {
         s_blk = T.nblk - 1 - static_cast<int>(atomicAdd(ticket, 1u));
         mbar_init(bar, 1);
@@ -149,194 +157,235 @@ __global__ void __launch_bounds__(kThreads) credit_kernel(const __grid_constant_
     const int b = s_blk;
     const int64_t t0 = static_cast<int64_t>(b) * kCB;
     const int nb = static_cast<int>(min(static_cast<int64_t>(kCB), T.N - t0));
-    const bool bulk = T.bulk && nb == kCB;
-    const float* src = L.loss + static_cast<int64_t>(row0) * L.ld_loss + t0;
 
-    if (bulk) {
+    if (T.tma) {
         if (tid == 0) {
-            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(R) * kCB * 4);
-            for (int i = 0; i < R; ++i) bulk_load(slab + i * kCB, src + i * L.ld_loss, kCB * 4, bar);
+            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(Rp) * kCB * 4);
+#pragma unroll
+            for (int sg = 0; sg < kSeg; ++sg)
+                tma_load_2d(slab + sg * Rp * kTPT, &L.tm_loss, bar,
+                            static_cast<int32_t>(t0) + sg * kTPT, row0);
         }
     } else {
-        for (int idx = tid; idx < R * kCB; idx += kThreads) {
+        const float* src = L.loss + static_cast<int64_t>(row0) * L.ld_loss + t0;
+        for (int idx = tid; idx < Rp * kCB; idx += nthr) {
             const int i = idx / kCB, j = idx % kCB;
-            slab[idx] = (j < nb) ? __ldg(src + static_cast<int64_t>(i) * L.ld_loss + j) : 0.f;
+            slab[slab_at(i, j, Rp)] =
+                (i < R && j < nb) ? __ldg(src + static_cast<int64_t>(i) * L.ld_loss + j) : 0.f;
         }
     }
-    // segment ends (while the copies are in flight)
-    gval[tid] = (tid >= nb || t0 + tid == T.N - 1) ? 0.f : T.gamma;
+    for (int j = tid; j < kCB; j += nthr) gval[j] = (j >= nb || t0 + j == T.N - 1) ? 0.f : T.gamma;
     __syncthreads();
     if (warp == 0) {
         // segment ends e = cu[s] with t0 < e <= t0 + nb end token e - 1 of this block
-        int lo = 0, hi = T.n_seq + 1;
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (static_cast<int64_t>(__ldg(&T.cu[mid])) > t0) hi = mid;
-            else lo = mid + 1;
-        }
+        const int lo = warp_upper_bound(T.cu, T.n_seq, t0, 0, lane);
         for (int s = lo + lane; s <= T.n_seq; s += 32) {
             const int64_t e = __ldg(&T.cu[s]);
             if (e > t0 + nb) break;
-            if (e > t0) gval[e - 1 - t0] = 0.f;
+            gval[e - 1 - t0] = 0.f;
         }
+        // the block of the first segment end at or after the first token of block b + 1: no
+        // look-back reaches past it
+        const int hi = warp_upper_bound(T.cu, T.n_seq, t0 + kCB, lo, lane);
+        const int64_t e = hi <= T.n_seq ? static_cast<int64_t>(__ldg(&T.cu[hi])) : T.N;
+        if (lane == 0)
+            s_jend = static_cast<int>(min((e - 1) / kCB, static_cast<int64_t>(T.nblk - 1)));
     }
-    if (bulk) mbar_wait_bounded(bar, 0, T.ew, 301);
+    if (T.tma) mbar_wait_bounded(bar, 0, T.ew, 301);
     __syncthreads();
 
-    // centring over the draws: mean over all K draws (in this block, or from the mean pass)
-    {
-        const int j = tid;
-        float m;
-        if (T.n_groups == 1) {
-            m = 0.f;
-            for (int i = 0; i < R; ++i) m += slab[i * kCB + j];
-            m = m / static_cast<float>(T.K);
-        } else {
-            m = (j < nb) ? L.mean[t0 + j] : 0.f;
+    // per-token mean over all K draws (of this block's rows, or from the mean pass)
+    if (T.centre) {
+        for (int j = tid; j < kCB; j += nthr) {
+            float m;
+            if (T.n_groups == 1) {
+                m = 0.f;
+                for (int i = 0; i < R; ++i) m += slab[slab_at(i, j, Rp)];
+                m = m / static_cast<float>(T.K);
+            } else {
+                m = (j < nb) ? L.mean[t0 + j] : 0.f;
+            }
+            mean[j] = m;
         }
-        for (int i = 0; i < R; ++i) slab[i * kCB + j] = m - slab[i * kCB + j];
+        __syncthreads();
     }
-    __syncthreads();
 
-    // From here each warp owns the rows i = warp + 4 k (one per lane at most) and works on its
-    // own: pass 1 (aggregate map per row), look-back with the same warp of the following
-    // blocks (its own status flag), pass 2 (the credit).  No block-wide barrier until the store.
-    const float4 g4 = *reinterpret_cast<const float4*>(gval + lane * kTPL);
-    for (int i = warp; i < R; i += kWarps) {
-        const float4 c4 = *reinterpret_cast<const float4*>(slab + i * kCB + lane * kTPL);
-        float A, G;
-        lane_map(c4, g4, A, G);
-        warp_suffix_scan(lane, A, G);
-        if (lane == 0) {
-            aggA[i] = A;
-            aggG[i] = G;
-            agg[static_cast<int64_t>(b) * T.rows + i] = make_float2(A, G);
+    // Pass 1.  Thread (row i, part sg) holds tokens 32 sg .. 32 sg + 31 of row i.
+    const int i = warp * kRowsPerWarp + (lane & 7);
+    const int sg = lane >> 3;
+    float* line = slab + sg * Rp * kTPT + i * kTPT;
+    float v[kTPT];
+#pragma unroll
+    for (int c = 0; c < kTPT / 4; ++c) {
+        const float4 q = *reinterpret_cast<const float4*>(line + ((c ^ (i & 7)) << 2));
+        v[4 * c] = q.x;
+        v[4 * c + 1] = q.y;
+        v[4 * c + 2] = q.z;
+        v[4 * c + 3] = q.w;
+    }
+    if (T.centre) {
+#pragma unroll
+        for (int c = 0; c < kTPT / 4; ++c) {
+            const float4 m = *reinterpret_cast<const float4*>(mean + sg * kTPT + 4 * c);
+            v[4 * c] = m.x - v[4 * c];
+            v[4 * c + 1] = m.y - v[4 * c + 1];
+            v[4 * c + 2] = m.z - v[4 * c + 2];
+            v[4 * c + 3] = m.w - v[4 * c + 3];
         }
     }
-    __syncwarp();
+    // this thread's map, last token first: r_first = A + G r_next
+    float A = 0.f, G = 1.f;
+#pragma unroll
+    for (int c = kTPT / 4 - 1; c >= 0; --c) {
+        const float4 g = *reinterpret_cast<const float4*>(gval + sg * kTPT + 4 * c);
+        A = fmaf(g.w, A, v[4 * c + 3]);
+        G = g.w * G;
+        A = fmaf(g.z, A, v[4 * c + 2]);
+        G = g.z * G;
+        A = fmaf(g.y, A, v[4 * c + 1]);
+        G = g.y * G;
+        A = fmaf(g.x, A, v[4 * c]);
+        G = g.x * G;
+    }
+    // suffix over the row's four parts (lanes sg, sg + 8, sg + 16, sg + 24 of the warp)
+    float sA = A, sG = G;
+#pragma unroll
+    for (int off = 8; off < 32; off <<= 1) {
+        const float A2 = __shfl_down_sync(0xffffffffu, sA, off);
+        const float G2 = __shfl_down_sync(0xffffffffu, sG, off);
+        if (lane + off < 32) {
+            sA = fmaf(sG, A2, sA);
+            sG = sG * G2;
+        }
+    }
+    // the map of the parts after this one (identity for the last part)
+    float eA = __shfl_down_sync(0xffffffffu, sA, 8);
+    float eG = __shfl_down_sync(0xffffffffu, sG, 8);
+    if (sg == kSeg - 1) {
+        eA = 0.f;
+        eG = 1.f;
+    }
 
-    // Look-back: carry[i] = r at token t0 + kCB of row i.  Only the blocks up to the first one
-    // after b that holds a segment end can reach block b (that block's map has G = 0 on every
-    // row), so the window of blocks to compose is known from cu_seqlens: their flags are polled
-    // in parallel (one lane per block) and their aggregates loaded together; the composition
-    // stops early at a block that already published its inclusive value.
-    const int my_row = warp + kWarps * lane;  // the row this lane composes
-    unsigned* my_flags = flags + warp;        // flag of (block j, this warp) at my_flags[j * kWarps]
+    // Look-back, per warp and row: only the blocks up to the first one after b that holds a
+    // segment end can reach block b (that block's map has G = 0 on every row), so the window
+    // b + 1 .. jend is known from cu_seqlens.  It is walked four blocks at a time: lane
+    // (row r, part q) polls the words of row r in block base + q, and the four lanes of a row
+    // compose the four answers in block order, stopping at the first inclusive value.
+    const bool row_ok = i < R;
     {
         const bool publish = (b != T.skip_publish);
-        if (b == T.nblk - 1 || T.gamma == 0.f) {
-            if (my_row < R) carry[my_row] = 0.f;
-        } else {
-            // the aggregates were written by lane 0 itself: its release store publishes them
-            if (lane == 0 && publish) st_release(&my_flags[static_cast<int64_t>(b) * kWarps], kAgg);
-            int jend;  // the block of the first segment end at or after the first token of b + 1
-            {
-                const int64_t first = t0 + kCB;
-                int lo = 0, hi = T.n_seq + 1;
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (static_cast<int64_t>(__ldg(&T.cu[mid])) > first) hi = mid;
-                    else lo = mid + 1;
-                }
-                const int64_t e = lo <= T.n_seq ? static_cast<int64_t>(__ldg(&T.cu[lo])) : T.N;
-                jend = static_cast<int>(min((e - 1) / kCB, static_cast<int64_t>(T.nblk - 1)));
-            }
+        if (sg == 0) {
+            aggA[i] = sA;
+            aggG[i] = sG;
+        }
+        float carry_i = 0.f;
+        if (b != T.nblk - 1 && T.gamma != 0.f) {
+            if (sg == 0 && row_ok && publish)
+                st_relaxed64(&aggw[static_cast<int64_t>(b) * T.rows + i],
+                             pack2(sA, __float_as_uint(-sG)));
+            const int jend = s_jend;
             float accA = 0.f, accG = 1.f;
+            bool done = !row_ok, failed = false;
             const uint64_t start = global_timer_ns();
-            bool done = false, failed = false;
-            for (int w0 = b + 1; w0 <= jend && !done; w0 += 32) {
-                const int j = w0 + lane;
-                const bool active = j <= jend;
-                unsigned st = 0;
-                int timed_out = 0;
-                if (active) {
-                    st = ld_acquire(&my_flags[static_cast<int64_t>(j) * kWarps]);
-                    while (st == 0) {
+            for (int base = b + 1; base <= jend; base += kSeg) {
+                const int j = base + sg;
+                int kind = 0;  // 1: aggregate (va, vg); 2: inclusive value va; 3: wait ran out
+                float va = 0.f, vg = 1.f;
+                if (!done && j <= jend) {
+                    const int64_t at = static_cast<int64_t>(j) * T.rows + i;
+                    while (true) {
+                        const uint64_t wi = ld_relaxed64(&incw[at]);
+                        if (static_cast<uint32_t>(wi >> 32) == 1u) {
+                            kind = 2;
+                            va = __uint_as_float(static_cast<uint32_t>(wi));
+                            break;
+                        }
+                        const uint64_t wa = ld_relaxed64(&aggw[at]);
+                        if (static_cast<uint32_t>(wa >> 32) & 0x80000000u) {
+                            kind = 1;
+                            va = __uint_as_float(static_cast<uint32_t>(wa));
+                            vg = -__uint_as_float(static_cast<uint32_t>(wa >> 32));
+                            break;
+                        }
                         if (global_timer_ns() - start > kWaitLimitNs) {
-                            timed_out = 1;
+                            kind = 3;
                             break;
                         }
                         __nanosleep(32);
-                        st = ld_acquire(&my_flags[static_cast<int64_t>(j) * kWarps]);
                     }
                 }
-                // each lane acquired its own flag; the warp barrier orders those acquires before
-                // every lane's loads of the aggregates below
-                __syncwarp();
-                if (__any_sync(0xffffffffu, timed_out)) {
-                    failed = true;
-                    break;
-                }
-                const unsigned inc_mask = __ballot_sync(0xffffffffu, active && st == kInc);
-                const int n_here = min(32, jend - w0 + 1);
-                const int stop = inc_mask ? __ffs(inc_mask) - 1 : n_here;  // first INC lane
-                if (my_row < R) {
-#pragma unroll 8
-                    for (int q = 0; q < stop; ++q) {
-                        const float2 a = __ldcg(&agg[static_cast<int64_t>(w0 + q) * T.rows + my_row]);
-                        accA = fmaf(accG, a.x, accA);
-                        accG = accG * a.y;
+#pragma unroll
+                for (int q = 0; q < kSeg; ++q) {
+                    const int src = (lane & 7) + 8 * q;
+                    const int kq = __shfl_sync(0xffffffffu, kind, src);
+                    const float aq = __shfl_sync(0xffffffffu, va, src);
+                    const float gq = __shfl_sync(0xffffffffu, vg, src);
+                    if (!done) {
+                        if (kq == 3) {
+                            failed = true;
+                            done = true;
+                        } else if (kq == 2) {
+                            accA = fmaf(accG, aq, accA);
+                            done = true;
+                        } else if (kq == 1) {
+                            accA = fmaf(accG, aq, accA);
+                            accG = accG * gq;
+                        }
                     }
-                    if (stop < n_here)
-                        accA = fmaf(accG, __ldcg(&inc[static_cast<int64_t>(w0 + stop) * T.rows + my_row]),
-                                    accA);
                 }
-                done = stop < n_here || w0 + 31 >= jend;
+                if (__all_sync(0xffffffffu, done)) break;
             }
             if (failed) {
-                if (lane == 0) report_error(T.ew, kDevTimeout, b);
-                if (my_row < R) carry[my_row] = __int_as_float(0x7fc00000);
-            } else if (my_row < R) {
-                carry[my_row] = accA;
+                if (sg == 0) report_error(T.ew, kDevTimeout, b);
+                carry_i = __int_as_float(0x7fc00000);
+            } else {
+                carry_i = accA;
             }
         }
-        if (my_row < R)
-            inc[static_cast<int64_t>(b) * T.rows + my_row] = fmaf(aggG[my_row], carry[my_row], aggA[my_row]);
-        __syncwarp();
-        if (lane == 0 && publish) {
-            // the inclusive values were written by every lane: order them before the release
-            asm volatile("fence.acq_rel.gpu;" ::: "memory");
-            st_release(&my_flags[static_cast<int64_t>(b) * kWarps], kInc);
+        if (sg == 0) {
+            carry[i] = carry_i;
+            if (row_ok && publish)
+                st_relaxed64(&incw[static_cast<int64_t>(b) * T.rows + i],
+                             pack2(fmaf(sG, carry_i, sA), 1u));
         }
+        __syncwarp();
     }
 
-    // pass 2: this warp's rows again, now with their carries
-    for (int i = warp; i < R; i += kWarps) {
-        float4 c4 = *reinterpret_cast<const float4*>(slab + i * kCB + lane * kTPL);
-        float A, G;
-        lane_map(c4, g4, A, G);
-        warp_suffix_scan(lane, A, G);
-        float eA = __shfl_down_sync(0xffffffffu, A, 1);
-        float eG = __shfl_down_sync(0xffffffffu, G, 1);
-        if (lane == 31) {
-            eA = 0.f;
-            eG = 1.f;
-        }
+    // Pass 2: the credit of this thread's tokens, from the carry of its row, back into the slab.
+    {
         float rn = fmaf(eG, carry[i], eA);
-        rn = fmaf(g4.w, rn, c4.w);
-        c4.w = rn;
-        rn = fmaf(g4.z, rn, c4.z);
-        c4.z = rn;
-        rn = fmaf(g4.y, rn, c4.y);
-        c4.y = rn;
-        rn = fmaf(g4.x, rn, c4.x);
-        c4.x = rn;
-        *reinterpret_cast<float4*>(slab + i * kCB + lane * kTPL) = c4;
+#pragma unroll
+        for (int c = kTPT / 4 - 1; c >= 0; --c) {
+            const float4 g = *reinterpret_cast<const float4*>(gval + sg * kTPT + 4 * c);
+            float4 q;
+            rn = fmaf(g.w, rn, v[4 * c + 3]);
+            q.w = rn;
+            rn = fmaf(g.z, rn, v[4 * c + 2]);
+            q.z = rn;
+            rn = fmaf(g.y, rn, v[4 * c + 1]);
+            q.y = rn;
+            rn = fmaf(g.x, rn, v[4 * c]);
+            q.x = rn;
+            *reinterpret_cast<float4*>(line + ((c ^ (i & 7)) << 2)) = q;
+        }
     }
-    float* dst = L.r + static_cast<int64_t>(row0) * L.ld_r + t0;
-    if (bulk) {
+    if (T.tma) {
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncthreads();
         if (tid == 0) {
-            for (int i = 0; i < R; ++i) bulk_store(dst + i * L.ld_r, slab + i * kCB, kCB * 4);
+#pragma unroll
+            for (int q = 0; q < kSeg; ++q)
+                tma_store_2d(&L.tm_r, slab + q * Rp * kTPT, static_cast<int32_t>(t0) + q * kTPT,
+                             row0);
             asm volatile("cp.async.bulk.commit_group;" ::: "memory");
             asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
         }
     } else {
         __syncthreads();
-        for (int idx = tid; idx < R * kCB; idx += kThreads) {
-            const int i = idx / kCB, j = idx % kCB;
-            if (j < nb) dst[static_cast<int64_t>(i) * L.ld_r + j] = slab[idx];
+        float* dst = L.r + static_cast<int64_t>(row0) * L.ld_r + t0;
+        for (int idx = tid; idx < R * kCB; idx += nthr) {
+            const int ii = idx / kCB, j = idx % kCB;
+            if (j < nb) dst[static_cast<int64_t>(ii) * L.ld_r + j] = slab[slab_at(ii, j, Rp)];
         }
     }
 }
@@ -369,31 +418,42 @@ namespace {
 
 template <int kMax>
 void fill_common(CreditTable<kMax>& T, const int32_t* cu, int32_t n_seq, int32_t K, int64_t N,
-                 float gamma, int skip, int64_t ld_loss, int64_t ld_r) {
+                 float gamma, int skip, int64_t ld_loss, int64_t ld_r, int centre = 1) {
     T.cu = cu;
+    T.centre = centre;
     T.ew = device_error_word();
     T.N = N;
     T.n_seq = n_seq;
     T.K = K;
     T.rows = group_rows(K);
+    T.rows_p = padded_rows(T.rows);
     T.n_groups = n_groups(K);
     T.nblk = static_cast<int>((N + kCB - 1) / kCB);
     T.state_stride = state_bytes(T.nblk, T.rows);
     T.skip_publish = skip;
     T.gamma = gamma;
-    T.bulk = (ld_loss % 4 == 0) && (ld_r % 4 == 0);
+    T.tma = (ld_loss % 4 == 0) && (ld_r % 4 == 0);
 }
 
-// Points a layer at its workspace region and clears every group's ticket and flags.
+// Points a layer at its workspace region, clears every group's ticket and look-back words, and encodes
+// its TMA descriptors (a table whose descriptors cannot all be encoded uses plain loads).
 template <int kMax>
 bool place_layer(CreditTable<kMax>& T, CreditLayer& L, char* base, cudaStream_t s) {
     L.state = base;
-    L.mean = T.n_groups > 1
+    if (T.tma &&
+        !(make_tmap_f32_2d_sw128(&L.tm_loss, L.loss, static_cast<uint64_t>(T.K),
+                                 static_cast<uint64_t>(T.N), static_cast<uint64_t>(L.ld_loss),
+                                 static_cast<uint32_t>(T.rows_p)) &&
+          make_tmap_f32_2d_sw128(&L.tm_r, L.r, static_cast<uint64_t>(T.K),
+                                 static_cast<uint64_t>(T.N), static_cast<uint64_t>(L.ld_r),
+                                 static_cast<uint32_t>(T.rows_p))))
+        T.tma = 0;
+    L.mean = T.n_groups > 1 && T.centre
                  ? reinterpret_cast<float*>(base + static_cast<size_t>(T.n_groups) * T.state_stride)
                  : nullptr;
     for (int g = 0; g < T.n_groups; ++g)
-        if (cudaMemsetAsync(base + static_cast<size_t>(g) * T.state_stride, 0,
-                            256 + static_cast<size_t>(T.nblk) * kWarps * 4, s) != cudaSuccess)
+        if (cudaMemsetAsync(base + static_cast<size_t>(g) * T.state_stride, 0, T.state_stride,
+                            s) != cudaSuccess)
             return false;
     return true;
 }
@@ -401,21 +461,21 @@ bool place_layer(CreditTable<kMax>& T, CreditLayer& L, char* base, cudaStream_t 
 template <int kMax>
 dust_status launch_credit_table(const CreditTable<kMax>& T, int n_layers, cudaStream_t s,
                                 const char* name) {
-    if (T.n_groups > 1) {
+    if (T.n_groups > 1 && T.centre) {
         const unsigned bx = static_cast<unsigned>(
             std::min<int64_t>((T.N + 255) / 256, static_cast<int64_t>(num_sms()) * 8));
         prof_begin(s);
         credit_mean_kernel<kMax><<<dim3(bx, n_layers), 256, 0, s>>>(T);
         prof_end(s, "credit_mean");
     }
-    const size_t smem = smem_bytes(T.rows);
+    const size_t smem = smem_bytes(T.rows_p);
     if (cudaFuncSetAttribute(credit_kernel<kMax>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return DUST_ERR_CUDA;
     if (static_cast<int64_t>(n_layers) * T.n_groups > 65535) return DUST_ERR_UNSUPPORTED;
     prof_begin(s);
     credit_kernel<kMax><<<dim3(static_cast<unsigned>(T.nblk), static_cast<unsigned>(n_layers * T.n_groups)),
-                          kThreads, smem, s>>>(T);
+                          kSeg * T.rows_p, smem, s>>>(T);
     prof_end(s, name);
     return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
 }
@@ -424,18 +484,18 @@ dust_status launch_credit_table(const CreditTable<kMax>& T, int n_layers, cudaSt
 
 dust_status credit_launch(const float* loss, int64_t ld_loss, int32_t K, int64_t N,
                           const int32_t* cu, int32_t n_seq, float gamma, float* r, int64_t ld_r,
-                          void* ws, cudaStream_t s) {
+                          void* ws, cudaStream_t s, int centre) {
     const int64_t nblk = (N + kCB - 1) / kCB;
     if (nblk > 2147483647LL) return DUST_ERR_UNSUPPORTED;
     CreditTable<1> T;
-    fill_common(T, cu, n_seq, K, N, gamma, g_credit_skip_publish, ld_loss, ld_r);
+    fill_common(T, cu, n_seq, K, N, gamma, g_credit_skip_publish, ld_loss, ld_r, centre);
     g_credit_skip_publish = -1;
     T.layer[0].loss = loss;
     T.layer[0].r = r;
     T.layer[0].ld_loss = ld_loss;
     T.layer[0].ld_r = ld_r;
     if (!place_layer(T, T.layer[0], static_cast<char*>(ws), s)) return DUST_ERR_CUDA;
-    return launch_credit_table(T, 1, s, "credit_scan");
+    return launch_credit_table(T, 1, s, centre ? "credit_scan" : "discounted_credit_scan");
 }
 
 size_t credit_grouped_workspace_bytes(int n_layers, int64_t N, int32_t K) {
@@ -475,7 +535,7 @@ dust_status credit_grouped_launch(const CreditLayerArgs* layers, int n, int32_t 
 // Credit without a caller workspace.  Some callers cannot allocate device memory at all: a
 // plugin run by a host engine that owns every buffer and forbids allocation while it executes,
 // or a process working under a fixed memory budget where a cudaMalloc could fail or stall the
-// device.  For them the look-back scratch (ticket, status flags, per-block aggregates) lives
+// device.  For them the look-back scratch (ticket and per-block look-back words) lives
 // in this fixed device array instead.  Each device that loads the library keeps it until the
 // process exits.
 // ------------------------------------------------------------------------------------------
@@ -525,7 +585,7 @@ extern "C" dust_status dust_credit_no_alloc(const float* loss, int64_t ld_loss, 
     T.layer[0].r = r;
     T.layer[0].ld_loss = ld_loss;
     T.layer[0].ld_r = ld_r;
-    // The tickets and the status flags must start at zero; the array keeps the previous
+    // The tickets and the look-back words must start at zero; the array keeps the previous
     // call's contents, so they are cleared on the stream before every launch.
     if (!place_layer(T, T.layer[0], static_cast<char*>(scratch), s)) return DUST_ERR_CUDA;
     return launch_credit_table(T, 1, s, "credit_scan_no_alloc");
