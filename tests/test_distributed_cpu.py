@@ -57,6 +57,21 @@ def _worker(rank, world, port, mode, q):
         L = workloads.custom_layer(21, 600, 12, 16, "f32", None)
         cu = workloads.random_segments(22, 600, 40, 200)
         K, sigma, gamma, seed = 6, 1e-2, 0.9, 0x5EED0009
+        if mode == "spsa":
+            # weight-space probes: each rank's tokens give partial p; one all-reduce of P
+            # scalars makes every rank's estimate the whole batch's
+            Lb = workloads.custom_layer(31, 90, 8, 8, "bf16", 0.05)
+            t0, t1 = (0, 40) if rank == 0 else (40, 90)
+            pp, _, _ = oracle.spsa_probe(Lb.x_f64[t0:t1], Lb.W_f64, Lb.u_f64[t0:t1], 5, 1e-3,
+                                         seed, 2)
+            pt = torch.from_numpy(pp.copy())
+            zd.allreduce_probe_scalars(pt)
+            whole, _, _ = oracle.spsa_probe(Lb.x_f64, Lb.W_f64, Lb.u_f64, 5, 1e-3, seed, 2)
+            G = oracle.spsa_estimate(pt.numpy(), 5, 8, 8, seed, 2)
+            Gw = oracle.spsa_estimate(whole, 5, 8, 8, seed, 2)
+            q.put((rank, float(max(np.abs(pt.numpy() - whole).max() / np.abs(whole).max(),
+                                   np.linalg.norm(G - Gw) / np.linalg.norm(Gw)))))
+            return
         if mode == "mismatch":
             try:
                 zd.check_same_problem(seed=seed + rank, K=K)
@@ -122,3 +137,10 @@ def test_rank_leaving_before_the_collective_fails_the_others():
     out = _run("dead")
     assert out[1] == "left"
     assert isinstance(out[0], str) and out[0].startswith("collective failed"), out[0]
+
+
+def test_two_ranks_spsa_exchange_only_probe_scalars():
+    out = _run("spsa")
+    assert set(out) == {0, 1}
+    for r, err in out.items():
+        assert isinstance(err, float) and err < 1e-9, (r, err)

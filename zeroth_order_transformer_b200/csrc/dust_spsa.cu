@@ -1,0 +1,387 @@
+// SPSA / MeZO weight-space probe, the contrast estimator (thakicloud page on zero-order
+// training, the SPSA paragraph: two forwards, with a perturbation of all weights added and
+// subtracted, estimate the gradient; gist.science 2605.15622 and the FedSPZO page: the
+// perturbation is regenerated from a shared seed, so only scalars travel).
+//
+// Probe j moves the weight matrix along z_j [d_out, d_in], drawn from the noise generator in
+// its own counter space, (k >> 2, o, probe, layer | 2^31), and stored at the weights' precision
+// (bf16).  For the quadratic readout the two perturbed forwards of a probe share y = W x:
+//   L_+- = sum_t 1/2 |e_t +- eps v_t|^2,  e_t = W x_t - u_t,  v_t = z_j x_t,
+// so L_+ - L_- = 2 eps sum_t <e_t, v_t> and L_+ + L_- = 2 L_0 + eps^2 sum_t |v_t|^2.  The
+// kernels evaluate both forwards through those sums, without the cancellation of subtracting
+// two large fp32 losses:
+//   spsa_dir_kernel     z_j for all probes, bf16, into the workspace [P, d_out_pad, d_in]
+//                       (rows d_out .. d_out_pad - 1 of each probe are zero).
+//   spsa_gemm_kernel    tcgen05 GEMM of x against W (residual mode: e = y - u and 1/2 |e|^2)
+//                       or against the stacked directions (probe mode: <e, v> and |v|^2 per
+//                       token and 256-row tile), TMA-fed, accumulator in tensor memory.  The
+//                       probe tiles are ordered probe-fastest so that the CTAs in flight share
+//                       the e and x tiles in L2.
+//   spsa_reduce_kernel  fixed-order sums over tokens and tiles: p_j = (L_+ - L_-) / (2 eps),
+//                       L_+ and L_-.
+//   spsa_estimate_kernel  G (+)= (1/P_total) sum_j p_j z_j, regenerating z (ALU-bound).
+#include <algorithm>
+
+#include "dust_device.cuh"
+#include "dust_internal.h"
+
+namespace dust {
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kBK = 64;
+constexpr int kStages = 4;
+constexpr int kThreads = 128;
+constexpr uint32_t kABytes = kBM * kBK * 2;
+constexpr uint32_t kBBytes = kBN * kBK * 2;
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 + 256;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kWeightSpace = 0x80000000u;
+
+int pad256(int d) { return (d + kBN - 1) / kBN * kBN; }
+
+// ---------------------------------------------------------------- directions
+__global__ void __launch_bounds__(256) spsa_dir_kernel(const __grid_constant__ NoiseKey key, int P,
+                                                       int d_out, int d_out_pad, int d_in,
+                                                       __nv_bfloat16* Z) {
+    const int nq = d_in >> 2;
+    const int64_t total = static_cast<int64_t>(P) * d_out_pad * nq;
+    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int q = static_cast<int>(idx % nq);
+        const int64_t row = idx / nq;  // j * d_out_pad + o
+        const int o = static_cast<int>(row % d_out_pad);
+        const int j = static_cast<int>(row / d_out_pad);
+        uint2 out = make_uint2(0u, 0u);
+        if (o < d_out) {
+            const F4 z = normal_quad(static_cast<uint32_t>(q), static_cast<uint32_t>(o),
+                                     key.draw_offset + static_cast<uint32_t>(j),
+                                     key.layer | kWeightSpace, key);
+            __nv_bfloat162 lo = __floats2bfloat162_rn(z.x, z.y);
+            __nv_bfloat162 hi = __floats2bfloat162_rn(z.z, z.w);
+            out.x = *reinterpret_cast<uint32_t*>(&lo);
+            out.y = *reinterpret_cast<uint32_t*>(&hi);
+        }
+        *reinterpret_cast<uint2*>(Z + row * d_in + 4 * q) = out;
+    }
+}
+
+// ---------------------------------------------------------------- GEMM with two epilogues
+struct GemmArgs {
+    CUtensorMap tmx;  // x [N, d_in], 64 x 128 boxes
+    CUtensorMap tmb;  // W [d_out, d_in] or Z [P d_out_pad, d_in], 64 x 256 boxes
+    const __nv_bfloat16* u;
+    float* e;         // [N, d_out] fp32: written in residual mode, read in probe mode
+    float* part_a;    // residual: [o_tiles, N] 1/2 |e|^2;  probe: [P o_tiles, N] <e, v>
+    float* part_b;    // probe: [P o_tiles, N] |v|^2
+    ErrorWord* ew;
+    int64_t N;
+    int d_in, d_out, o_tiles, P, m_tiles;
+};
+
+template <bool kProbe>
+__global__ void __launch_bounds__(kThreads, 1) spsa_gemm_kernel(const __grid_constant__ GemmArgs A) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+    uint64_t* empty = full + kStages;
+    uint64_t* acc_full = empty + kStages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // tile order: probe fastest, then the 256-row output tile, then the token tile
+    const int P = kProbe ? A.P : 1;
+    const int j = blockIdx.x % P;
+    const int o_tile = (blockIdx.x / P) % A.o_tiles;
+    const int m_tile = blockIdx.x / (P * A.o_tiles);
+    const int64_t m0 = static_cast<int64_t>(m_tile) * kBM;
+    const int o0 = o_tile * kBN;
+    const int b0 = kProbe ? (j * A.o_tiles + o_tile) * kBN : o0;  // first row of the B tile
+    const int nk = (A.d_in + kBK - 1) / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&A.tmx);
+        prefetch_tensormap(&A.tmb);
+        for (int kb = 0; kb < nk; ++kb) {
+            const int s = kb % kStages;
+            if (kb >= kStages && !mbar_wait_bounded(&empty[s], ((kb / kStages) - 1) & 1, A.ew, 401))
+                break;
+            uint8_t* a = smem + s * kStageBytes;
+            mbar_arrive_expect_tx(&full[s], kStageBytes);
+            tma_load_2d(a, &A.tmx, &full[s], kb * kBK, static_cast<int32_t>(m0));
+            tma_load_2d(a + kABytes, &A.tmb, &full[s], kb * kBK, b0);
+        }
+    } else if (warp == 1 && lane == 0) {
+        constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, 0, 0);
+        for (int kb = 0; kb < nk; ++kb) {
+            const int s = kb % kStages;
+            if (!mbar_wait_bounded(&full[s], (kb / kStages) & 1, A.ew, 402)) break;
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
+            const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+                const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
+                const uint64_t bd = sdesc_sw128(b_addr + kk * 32, 16, 1024);
+                umma_bf16(tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            }
+            umma_commit(&empty[s]);
+        }
+        umma_commit(acc_full);
+    }
+    mbar_wait_bounded(acc_full, 0, A.ew, 403);
+    __syncwarp();
+    tc_fence_after();
+
+    // epilogue: thread = token row (TMEM lane quarter = warp)
+    const int row = warp * 32 + lane;
+    const int64_t t = m0 + row;
+    const bool valid = t < A.N;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int nchunks = min(kBN, A.d_out - o0) / 16;
+    float sa = 0.f, sb = 0.f;
+    for (int c = 0; c < nchunks; ++c) {
+        float v[16];
+        tmem_ld16(trow + c * 16, v);
+        tmem_wait_ld();
+        if (!valid) continue;
+        const int64_t off = t * A.d_out + o0 + c * 16;
+        if (kProbe) {
+            const float4* e4 = reinterpret_cast<const float4*>(A.e + off);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 e = __ldg(e4 + q);
+                sa = fmaf(e.x, v[4 * q], sa);
+                sa = fmaf(e.y, v[4 * q + 1], sa);
+                sa = fmaf(e.z, v[4 * q + 2], sa);
+                sa = fmaf(e.w, v[4 * q + 3], sa);
+                sb = fmaf(v[4 * q], v[4 * q], sb);
+                sb = fmaf(v[4 * q + 1], v[4 * q + 1], sb);
+                sb = fmaf(v[4 * q + 2], v[4 * q + 2], sb);
+                sb = fmaf(v[4 * q + 3], v[4 * q + 3], sb);
+            }
+        } else {
+            const uint4* up = reinterpret_cast<const uint4*>(A.u + off);
+            float uf[16];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint4 w = __ldg(up + h);
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uf[8 * h + 2 * q] = __uint_as_float(ww[q] << 16);
+                    uf[8 * h + 2 * q + 1] = __uint_as_float(ww[q] & 0xFFFF0000u);
+                }
+            }
+            float4* e4 = reinterpret_cast<float4*>(A.e + off);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float4 e;
+                e.x = v[4 * q] - uf[4 * q];
+                e.y = v[4 * q + 1] - uf[4 * q + 1];
+                e.z = v[4 * q + 2] - uf[4 * q + 2];
+                e.w = v[4 * q + 3] - uf[4 * q + 3];
+                e4[q] = e;
+                sa = fmaf(e.x, e.x, sa);
+                sa = fmaf(e.y, e.y, sa);
+                sa = fmaf(e.z, e.z, sa);
+                sa = fmaf(e.w, e.w, sa);
+            }
+        }
+    }
+    if (valid) {
+        const int64_t slot = static_cast<int64_t>(kProbe ? j * A.o_tiles + o_tile : o_tile);
+        if (kProbe) {
+            A.part_a[slot * A.N + t] = sa;
+            A.part_b[slot * A.N + t] = sb;
+        } else {
+            A.part_a[slot * A.N + t] = 0.5f * sa;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---------------------------------------------------------------- reductions
+// Block b < P: probe b's sums; block P: the clean loss.  Tokens are summed per thread in order,
+// tiles in order, then the block's threads in a fixed tree.
+__global__ void __launch_bounds__(256) spsa_reduce_kernel(const float* part_l0, const float* part_ev,
+                                                          const float* part_vv, int64_t N,
+                                                          int o_tiles, int P, float eps, float* p,
+                                                          float* Lp, float* Lm, float* l0_out) {
+    __shared__ float sa[256], sb[256], sc[256];
+    const int j = blockIdx.x;  // a probe
+    float a = 0.f, b = 0.f, c = 0.f;
+    for (int ot = 0; ot < o_tiles; ++ot) {
+        const int64_t slot = static_cast<int64_t>(j) * o_tiles + ot;
+        for (int64_t t = threadIdx.x; t < N; t += blockDim.x) {
+            a += part_ev[slot * N + t];
+            b += part_vv[slot * N + t];
+            c += part_l0[static_cast<int64_t>(ot) * N + t];
+        }
+    }
+    sa[threadIdx.x] = a;
+    sb[threadIdx.x] = b;
+    sc[threadIdx.x] = c;
+    __syncthreads();
+    for (int w = 128; w > 0; w >>= 1) {
+        if (threadIdx.x < w) {
+            sa[threadIdx.x] += sa[threadIdx.x + w];
+            sb[threadIdx.x] += sb[threadIdx.x + w];
+            sc[threadIdx.x] += sc[threadIdx.x + w];
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        const float ev = sa[0], vv = sb[0], l0 = sc[0];
+        p[j] = ev;  // (L_+ - L_-) / (2 eps) = sum_t <e_t, v_t>
+        const float curv = 0.5f * eps * eps * vv;
+        if (Lp) Lp[j] = l0 + eps * ev + curv;
+        if (Lm) Lm[j] = l0 - eps * ev + curv;
+        if (l0_out && j == 0) *l0_out = l0;
+    }
+}
+
+// G[o][k] (+)= scale * sum_j p_j z_j[o][k]: one thread per (o, channel quad), probes in order.
+__global__ void __launch_bounds__(256) spsa_estimate_kernel(const __grid_constant__ NoiseKey key,
+                                                            const float* __restrict__ p, int P,
+                                                            int d_out, int d_in, float scale,
+                                                            float* G, int accumulate) {
+    const int nq = d_in >> 2;
+    const int64_t total = static_cast<int64_t>(d_out) * nq;
+    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int q = static_cast<int>(idx % nq);
+        const int o = static_cast<int>(idx / nq);
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        for (int j = 0; j < P; ++j) {
+            const float pj = __ldg(p + j);
+            const F4 z = normal_quad(static_cast<uint32_t>(q), static_cast<uint32_t>(o),
+                                     key.draw_offset + static_cast<uint32_t>(j),
+                                     key.layer | kWeightSpace, key);
+            // the direction is the bf16 value of the normal
+            a0 = fmaf(pj, __bfloat162float(__float2bfloat16_rn(z.x)), a0);
+            a1 = fmaf(pj, __bfloat162float(__float2bfloat16_rn(z.y)), a1);
+            a2 = fmaf(pj, __bfloat162float(__float2bfloat16_rn(z.z)), a2);
+            a3 = fmaf(pj, __bfloat162float(__float2bfloat16_rn(z.w)), a3);
+        }
+        float4* g = reinterpret_cast<float4*>(G + static_cast<int64_t>(o) * d_in + 4 * q);
+        float4 r = make_float4(scale * a0, scale * a1, scale * a2, scale * a3);
+        if (accumulate) {
+            const float4 old = *g;
+            r.x += old.x;
+            r.y += old.y;
+            r.z += old.z;
+            r.w += old.w;
+        }
+        *g = r;
+    }
+}
+
+}  // namespace
+
+size_t spsa_workspace_bytes(int64_t N, int32_t d_in, int32_t d_out, int32_t P) {
+    const int o_tiles = pad256(d_out) / kBN;
+    return align_up(static_cast<size_t>(P) * pad256(d_out) * d_in * 2, 256) +  // Z
+           align_up(static_cast<size_t>(N) * d_out * 4, 256) +                    // e
+           align_up(static_cast<size_t>(o_tiles) * N * 4, 256) +                  // 1/2 |e|^2
+           2 * align_up(static_cast<size_t>(P) * o_tiles * N * 4, 256);           // <e,v>, |v|^2
+}
+
+dust_status spsa_probe_launch(const void* x, const void* W, const void* u, int64_t N, int32_t d_in,
+                              int32_t d_out, int32_t P, float eps, NoiseKey key, float* p,
+                              float* Lp, float* Lm, void* ws, cudaStream_t s) {
+    const int dpad = pad256(d_out);
+    const int o_tiles = dpad / kBN;
+    const int m_tiles = static_cast<int>((N + kBM - 1) / kBM);
+    char* w = static_cast<char*>(ws);
+    __nv_bfloat16* Z = reinterpret_cast<__nv_bfloat16*>(w);
+    w += align_up(static_cast<size_t>(P) * dpad * d_in * 2, 256);
+    float* e = reinterpret_cast<float*>(w);
+    w += align_up(static_cast<size_t>(N) * d_out * 4, 256);
+    float* pl0 = reinterpret_cast<float*>(w);
+    w += align_up(static_cast<size_t>(o_tiles) * N * 4, 256);
+    float* pev = reinterpret_cast<float*>(w);
+    w += align_up(static_cast<size_t>(P) * o_tiles * N * 4, 256);
+    float* pvv = reinterpret_cast<float*>(w);
+
+    GemmArgs R{};
+    R.u = static_cast<const __nv_bfloat16*>(u);
+    R.e = e;
+    R.part_a = pl0;
+    R.part_b = nullptr;
+    R.ew = device_error_word();
+    R.N = N;
+    R.d_in = d_in;
+    R.d_out = d_out;
+    R.o_tiles = o_tiles;
+    R.P = P;
+    R.m_tiles = m_tiles;
+    if (!make_tmap_bf16_2d(&R.tmx, x, static_cast<uint64_t>(N), d_in, kBM, kBK) ||
+        !make_tmap_bf16_2d(&R.tmb, W, static_cast<uint64_t>(d_out), d_in, kBN, kBK))
+        return DUST_ERR_CUDA;
+    GemmArgs Q = R;
+    Q.part_a = pev;
+    Q.part_b = pvv;
+    if (!make_tmap_bf16_2d(&Q.tmb, Z, static_cast<uint64_t>(P) * dpad, d_in, kBN, kBK))
+        return DUST_ERR_CUDA;
+    if (cudaFuncSetAttribute(spsa_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes)) != cudaSuccess ||
+        cudaFuncSetAttribute(spsa_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+        return DUST_ERR_CUDA;
+    const int64_t dir_total = static_cast<int64_t>(P) * dpad * (d_in / 4);
+    prof_begin(s);
+    spsa_dir_kernel<<<static_cast<unsigned>(std::min<int64_t>((dir_total + 255) / 256,
+                                                              static_cast<int64_t>(num_sms()) * 16)),
+                      256, 0, s>>>(key, P, d_out, dpad, d_in, Z);
+    prof_end(s, "spsa_directions");
+    prof_begin(s);
+    spsa_gemm_kernel<false><<<static_cast<unsigned>(m_tiles * o_tiles), kThreads, kSmemBytes, s>>>(R);
+    prof_end(s, "spsa_residual_gemm");
+    prof_begin(s);
+    spsa_gemm_kernel<true><<<static_cast<unsigned>(static_cast<int64_t>(m_tiles) * o_tiles * P),
+                             kThreads, kSmemBytes, s>>>(Q);
+    prof_end(s, "spsa_probe_gemm");
+    prof_begin(s);
+    spsa_reduce_kernel<<<static_cast<unsigned>(P), 256, 0, s>>>(pl0, pev, pvv, N, o_tiles, P, eps,
+                                                               p, Lp, Lm, nullptr);
+    prof_end(s, "spsa_reduce");
+    return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
+}
+
+dust_status spsa_estimate_launch(const float* p, int32_t P, int32_t P_total, int32_t d_in,
+                                 int32_t d_out, NoiseKey key, float* G, int accumulate,
+                                 cudaStream_t s) {
+    const int64_t total = static_cast<int64_t>(d_out) * (d_in / 4);
+    prof_begin(s);
+    spsa_estimate_kernel<<<static_cast<unsigned>(std::min<int64_t>((total + 255) / 256,
+                                                                   static_cast<int64_t>(num_sms()) * 16)),
+                           256, 0, s>>>(key, p, P, d_out, d_in, 1.0f / static_cast<float>(P_total),
+                                        G, accumulate);
+    prof_end(s, "spsa_estimate");
+    return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
+}
+
+}  // namespace dust

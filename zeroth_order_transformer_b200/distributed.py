@@ -80,3 +80,23 @@ def estimate_sharded(x, W, u, cu_local, K: int, sigma: float, gamma: float, seed
     key = NoiseKey(seed, layer_id, 0, token_offset)
     G_W = layer.estimate(x, W, u, cu, sigma, gamma, key)
     return allreduce_weight_estimate(G_W, group)
+
+
+def allreduce_probe_scalars(p, group=None):
+    """SPSA / MeZO: the sum over ranks of the per-rank projected gradients p [P] (and of the
+    perturbed losses, if given the same way).  P scalars per step: the weight-space probes'
+    directions are regenerated from the seed on every rank, never sent."""
+    import torch.distributed as dist
+    dist.all_reduce(p, op=dist.ReduceOp.SUM, group=group)
+    return p
+
+
+def spsa_sharded(x, W, u, P: int, eps: float, seed: int, layer_id: int = 0,
+                 probe_offset: int = 0, group=None):
+    """The SPSA weight estimate of one layer from this rank's tokens (CUDA path): local probes,
+    one all-reduce of P scalars, then the estimate (identical on every rank)."""
+    from . import NoiseKey, dust_spsa_estimate, dust_spsa_probe
+    key = NoiseKey(seed, layer_id, probe_offset)
+    p = dust_spsa_probe(x, W, u, P, eps, key)
+    allreduce_probe_scalars(p, group)
+    return dust_spsa_estimate(p, P, W.shape[0], W.shape[1], key), p
