@@ -46,6 +46,7 @@ OPS_PER_NORMAL = {"fwd_bf16_noise_loss": 20.0, "ghat_reduce_draws": 19.0,
                   # exp(sigma a) - 1 as a degree-5 series (5), the weighted sum (1)
                   "lmhead_ce_noise": 25.0}
 HEAD_METRIC = "Dust LM-head estimator tokens*draws/s"
+ATTN_METRIC = "Dust attention-reward estimator tokens*draws/s"
 
 
 def measured_peaks():
@@ -477,6 +478,304 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     print(json.dumps(line), flush=True)
 
 
+def kernel_table(prof, work, peaks, sms):
+    """Per-kernel launches, times, shares and achieved rates from the profile records, and the
+    roofline object of the dominant kernel (the largest total time with a defined work)."""
+    per = {}
+    for name, t in prof:
+        d = per.setdefault(name, [0, 0.0])
+        d[0] += 1
+        d[1] += t
+    tot = sum(v[1] for v in per.values())
+    kernels = {n: {"launches": c, "ms_total": round(t, 4), "ms_avg": round(t / c, 5),
+                   "share": round(t / tot, 4)}
+               for n, (c, t) in sorted(per.items(), key=lambda kv: -kv[1][1])}
+    roofline = None
+    for n, info in kernels.items():
+        bound, amount, what = work(n)
+        if amount is None:
+            continue
+        rate = amount / (info["ms_avg"] / 1e3)
+        info[{"normals": "gnormals_per_s", "flops": "tflops", "bytes": "gbs"}[what]] = round(
+            rate / (1e12 if what == "flops" else 1e9), 2)
+        if roofline is not None:
+            continue
+        if bound == "alu":
+            ops = OPS_PER_NORMAL.get(n, 19.0)
+            peak = sms * LANES_PER_SM * peaks["sm_max_mhz"] * 1e6 / ops / 1e9
+            roofline = {"kernel": n, "bound": "alu", "achieved": round(rate / 1e9, 2),
+                        "peak": round(peak, 2), "unit": "Gnormal/s",
+                        "frac": round(rate / 1e9 / peak, 4), "traffic": None,
+                        "peak_basis": f"{sms} SMs x {LANES_PER_SM} lanes x "
+                                      f"{peaks['sm_max_mhz']:.0f} MHz / {ops:.0f} ops per normal"}
+        elif bound == "hbm":
+            roofline = {"kernel": n, "bound": "hbm", "achieved": round(rate / 1e9, 2),
+                        "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": round(rate / 1e9 / peaks["hbm_gbs"], 4), "traffic": None}
+        elif bound == "tensor":
+            roofline = {"kernel": n, "bound": "tensor", "achieved": round(rate / 1e12, 2),
+                        "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                        "frac": round(rate / 1e12 / peaks["bf16_tflops"], 4), "traffic": None}
+        roofline["peak_source"] = peaks["source"]
+    return kernels, roofline
+
+
+def attn_kernel_work(name, aw):
+    """Algorithmic work of one launch of the attention-reward step's kernels."""
+    N, K = aw.N, aw.K
+    if name == "attn_reward":
+        return "hbm", 2.0 * K * N * aw.d + 4.0 * N * aw.d + 4.0 * K * N, "bytes"
+    if name.startswith("discounted_credit_scan"):
+        return "hbm", 8.0 * K * N, "bytes"
+    if name == "ghat_reduce_draws":
+        return "alu", N * aw.d * K, "normals"
+    if name.startswith("gw_bf16_tcgen05"):
+        return "tensor", 2.0 * N * aw.d_model * aw.d, "flops"
+    return None, None, None
+
+
+def run_attn(args) -> None:
+    """The estimate of an attention projection from the attention-internal reward:
+    dust_attn_reward (c = -<ghat, delta_o>) -> dust_discounted_credit -> dust_weight_grad of
+    the perturbed projection.  One GPU; one JSON line."""
+    import torch
+
+    import zeroth_order_transformer_b200 as dust
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    aw = workloads.ATTN_WORKLOADS[args.attn]
+    data = workloads.generate_attn(aw)
+    peaks = measured_peaks()
+    G = torch.from_numpy(data.ghat).to(dev)
+    dO = torch.from_numpy(data.dO_store.view(np.int16)).view(torch.bfloat16).to(dev)
+    x = torch.from_numpy(data.x_store.view(np.int16)).view(torch.bfloat16).to(dev)
+    cu = torch.from_numpy(data.cu_seqlens).to(dev)
+    ws = torch.empty(max(dust.dust_workspace_size(dust.DUST_OP_CREDIT, 0, aw.N, 0, 0, aw.K),
+                         dust.dust_workspace_size(dust.DUST_OP_WEIGHT_GRAD, 1, aw.N, aw.d_model,
+                                                  aw.d, aw.K)), dtype=torch.uint8, device=dev)
+    c = torch.empty((aw.K, aw.N), dtype=torch.float32, device=dev)
+    r = torch.empty_like(c)
+    GW = torch.empty((aw.d, aw.d_model), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    key = dust.NoiseKey(aw.seed, 2)
+
+    def step(GG=G, DD=dO, XX=x):
+        dust.dust_attn_reward(GG, DD, c)
+        dust.dust_discounted_credit(c, cu, aw.gamma, r, ws)
+        dust.dust_weight_grad(r, XX, aw.d, aw.K, aw.sigma, key, GW, False, None, ws)
+        return GW
+
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    dust.dust_profile_enable(1 << 16)
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    prof = dust.dust_profile_read()
+    dust.dust_profile_disable()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    units = aw.N * aw.K
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    kernels, roofline = kernel_table(prof, lambda n: attn_kernel_work(n, aw), peaks, sms)
+    if roofline is not None and roofline["bound"] == "alu":
+        gc = generator_ceiling(dust, torch, dev)
+        roofline["generator_ceiling"] = round(gc, 2)
+        roofline["frac_of_generator_ceiling"] = round(roofline["achieved"] / gc, 4)
+    e2e = None
+    if not args.no_e2e:
+        hG, hD, hx = (t.cpu().pin_memory() for t in (G, dO, x))
+        dG, dD, dx = torch.empty_like(G), torch.empty_like(dO), torch.empty_like(x)
+        hW = torch.empty(GW.shape, dtype=GW.dtype, pin_memory=True)
+
+        def e2e_step():
+            dG.copy_(hG, non_blocking=True)
+            dD.copy_(hD, non_blocking=True)
+            dx.copy_(hx, non_blocking=True)
+            hW.copy_(step(dG, dD, dx), non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for a, b in ee:
+            flush.zero_()
+            a.record(stream)
+            e2e_step()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = sum(a.elapsed_time(b) for a, b in ee) / args.steps
+        e2e = {"value": units / (e_ms / 1e3), "unit": UNIT, "ms_per_step": e_ms,
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (hG, hD, hx)),
+               "d2h_bytes_per_step": hW.numel() * hW.element_size()}
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        n_tok = 256
+        G64 = data.ghat[:n_tok].astype(np.float64)
+        D64 = workloads.bf16_bits_to_f64(data.dO_store[:, :n_tok])
+        X64 = workloads.bf16_bits_to_f64(data.x_store[:n_tok])
+        done, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < args.cpu_seconds:
+            cc = oracle.attn_reward(G64, D64)
+            rr = oracle.discounted_credit(cc, np.array([0, n_tok], dtype=np.int32), aw.gamma)
+            g = oracle.output_error(rr, aw.K, aw.sigma, aw.seed, aw.d, 2)
+            oracle.weight_grad(g, X64)
+            done += n_tok * aw.K
+        el = time.perf_counter() - t0
+        cpu = {"value": done / el, "unit": UNIT, "cores": oracle.get_threads(), "kind": "oracle",
+               "seconds": round(el, 2),
+               "sample": f"oracle (fp64 C, OpenMP) reward-based estimate on the first {n_tok} "
+                         f"tokens (credit truncated to the sample), repeated for about "
+                         f"{args.cpu_seconds:.0f} s"}
+    line = {
+        "metric": ATTN_METRIC, "value": units / (ms / 1e3), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 delta_o and x, f32 ghat",
+        "data": "synthetic (seeded; GPT-2-small attention shape)",
+        "config": {"workload": f"{aw.name}: {aw.n_seq}x{aw.seq_len} tokens, projection "
+                               f"{aw.d_model}->{aw.d}, K={aw.K}, sigma={aw.sigma}, "
+                               f"gamma={aw.gamma}",
+                   "l2": "flushed (256 MiB write) before every timed step"},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": sum(v["launches"] for v in kernels.values()), "clocks": clocks,
+        "kernels": kernels,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def spsa_kernel_work(name, wl, P):
+    """Algorithmic work of one launch of the SPSA probe step's kernels (one layer)."""
+    N, s = wl.N, wl.layers[0]
+    if name == "spsa_probe_gemm":
+        return "tensor", 2.0 * N * s.d_in * s.d_out * P, "flops"
+    if name == "spsa_residual_gemm":
+        return "tensor", 2.0 * N * s.d_in * s.d_out, "flops"
+    if name in ("spsa_directions", "spsa_estimate"):
+        return "alu", s.d_out * s.d_in * P, "normals"
+    return None, None, None
+
+
+def run_spsa(args) -> None:
+    """The SPSA / MeZO contrast estimator on a workload's first layer: dust_spsa_probe (the two
+    perturbed forwards of P probes) -> dust_spsa_estimate (the weight estimate).  One GPU."""
+    import torch
+
+    import zeroth_order_transformer_b200 as dust
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    data = workloads.generate(args.workload, n_layers=1)
+    wl = data.wl
+    L = data.layers[0]
+    s0 = L.shape
+    P = args.spsa_probes
+    peaks = measured_peaks()
+
+    def dev_t(store):
+        return torch.from_numpy(np.ascontiguousarray(store).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+
+    x, W, u = dev_t(L.x_store), dev_t(L.W_store), dev_t(L.u_store)
+    ws = torch.empty(dust.dust_workspace_size(dust.DUST_OP_SPSA_PROBE, 1, wl.N, s0.d_in, s0.d_out,
+                                              P), dtype=torch.uint8, device=dev)
+    p = torch.empty(P, dtype=torch.float32, device=dev)
+    G = torch.empty((s0.d_out, s0.d_in), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    key = dust.NoiseKey(wl.seed, s0.layer_id)
+
+    def step(xx=x, WW=W, uu=u):
+        dust.dust_spsa_probe(xx, WW, uu, P, 1e-3, key, p, workspace=ws)
+        dust.dust_spsa_estimate(p, P, s0.d_out, s0.d_in, key, G)
+        return G
+
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    dust.dust_profile_enable(1 << 16)
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    prof = dust.dust_profile_read()
+    dust.dust_profile_disable()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    kernels, roofline = kernel_table(prof, lambda n: spsa_kernel_work(n, wl, P), peaks, sms)
+    units = wl.N * P
+    e2e = None
+    if not args.no_e2e:
+        hx, hW, hu = (t.cpu().pin_memory() for t in (x, W, u))
+        dx, dW, du = torch.empty_like(x), torch.empty_like(W), torch.empty_like(u)
+        hG = torch.empty(G.shape, dtype=G.dtype, pin_memory=True)
+
+        def e2e_step():
+            dx.copy_(hx, non_blocking=True)
+            dW.copy_(hW, non_blocking=True)
+            du.copy_(hu, non_blocking=True)
+            hG.copy_(step(dx, dW, du), non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for a, b in ee:
+            flush.zero_()
+            a.record(stream)
+            e2e_step()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = sum(a.elapsed_time(b) for a, b in ee) / args.steps
+        e2e = {"value": units / (e_ms / 1e3), "unit": "tokens*probes/s", "ms_per_step": e_ms,
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (hx, hW, hu)),
+               "d2h_bytes_per_step": hG.numel() * hG.element_size()}
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        n_tok = 64
+        done, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < args.cpu_seconds:
+            pp, _, _ = oracle.spsa_probe(L.x_f64[:n_tok], L.W_f64, L.u_f64[:n_tok], 1, 1e-3,
+                                         wl.seed, s0.layer_id, done // n_tok % P)
+            done += n_tok
+        el = time.perf_counter() - t0
+        cpu = {"value": done / el, "unit": "tokens*probes/s", "cores": oracle.get_threads(),
+               "kind": "oracle", "seconds": round(el, 2),
+               "sample": f"oracle (fp64 C) two perturbed forwards of one probe on {n_tok} tokens, "
+                         f"repeated for about {args.cpu_seconds:.0f} s (the estimate step not "
+                         f"included)"}
+    line = {
+        "metric": "SPSA/MeZO contrast estimator tokens*probes/s", "value": units / (ms / 1e3),
+        "unit": "tokens*probes/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 in, f32 accumulate", "data": "synthetic (seeded)",
+        "config": {"workload": f"{describe(wl)}; first layer; P={P} probes, eps=1e-3",
+                   "l2": "flushed (256 MiB write) before every timed step"},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": sum(v["launches"] for v in kernels.values()), "clocks": clocks,
+        "kernels": kernels,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def head_kernel_work(name, hw):
     """Algorithmic work of one launch of the LM-head step's kernels."""
     N, K = hw.N, hw.K
@@ -554,40 +853,8 @@ def run_head(args) -> None:
     dust.dust_profile_disable()
     ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
     units = hw.N * hw.K
-    per = {}
-    for name, t in prof:
-        d = per.setdefault(name, [0, 0.0])
-        d[0] += 1
-        d[1] += t
-    tot = sum(v[1] for v in per.values())
-    kernels = {n: {"launches": c, "ms_total": round(t, 4), "ms_avg": round(t / c, 5),
-                   "share": round(t / tot, 4)}
-               for n, (c, t) in sorted(per.items(), key=lambda kv: -kv[1][1])}
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    roofline = None
-    for n, info in kernels.items():
-        bound, amount, what = head_kernel_work(n, hw)
-        if amount is None:
-            continue
-        rate = amount / (info["ms_avg"] / 1e3)
-        info[{"normals": "gnormals_per_s", "flops": "tflops", "bytes": "gbs"}[what]] = round(
-            rate / (1e12 if what == "flops" else 1e9), 2)
-        if roofline is None:
-            if bound == "alu":
-                ops = OPS_PER_NORMAL.get(n, 19.0)
-                peak = sms * LANES_PER_SM * peaks["sm_max_mhz"] * 1e6 / ops / 1e9
-                ach = rate / 1e9
-                roofline = {"kernel": n, "bound": "alu", "achieved": round(ach, 2),
-                            "peak": round(peak, 2), "unit": "Gnormal/s",
-                            "frac": round(ach / peak, 4), "traffic": None,
-                            "peak_basis": f"{sms} SMs x {LANES_PER_SM} lanes x "
-                                          f"{peaks['sm_max_mhz']:.0f} MHz / {ops:.0f} ops per "
-                                          f"normal", "peak_source": peaks["source"]}
-            elif bound == "hbm":
-                roofline = {"kernel": n, "bound": "hbm", "achieved": round(rate / 1e9, 2),
-                            "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                            "frac": round(rate / 1e9 / peaks["hbm_gbs"], 4), "traffic": None,
-                            "peak_source": peaks["source"]}
+    kernels, roofline = kernel_table(prof, lambda n: head_kernel_work(n, hw), peaks, sms)
     if roofline is not None and roofline["bound"] == "alu":
         gc = generator_ceiling(dust, torch, dev)
         roofline["generator_ceiling"] = round(gc, 2)
@@ -714,12 +981,23 @@ def main():
     ap.add_argument("--stress-N", type=int, default=1 << 22)
     ap.add_argument("--head", choices=sorted(workloads.HEAD_WORKLOADS), default=None,
                     help="time the LM-head estimator on cached logits instead and exit")
+    ap.add_argument("--attn", choices=sorted(workloads.ATTN_WORKLOADS), default=None,
+                    help="time the attention-reward estimate of a projection instead and exit")
+    ap.add_argument("--spsa", action="store_true",
+                    help="time the SPSA/MeZO contrast estimator on the workload's first layer")
+    ap.add_argument("--spsa-probes", type=int, default=16)
     args = ap.parse_args()
     if args.credit_stress:
         run_credit_stress(args)
         return
     if args.head:
         run_head(args)
+        return
+    if args.attn:
+        run_attn(args)
+        return
+    if args.spsa:
+        run_spsa(args)
         return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -58,7 +58,8 @@ typedef enum {
     DUST_OP_NOISY_LINEAR_FWD = 0,
     DUST_OP_CREDIT = 1,
     DUST_OP_WEIGHT_GRAD = 2,
-    DUST_OP_LOGITS_CE = 3 /* d_in = vocabulary size V, d_out = slab size S */
+    DUST_OP_LOGITS_CE = 3, /* d_in = vocabulary size V, d_out = slab size S */
+    DUST_OP_SPSA_PROBE = 4 /* K = number of probes P */
 } dust_op;
 
 /* Identifies the noise of one call.  seed: generator key; layer_id: fourth counter word, so
@@ -131,6 +132,69 @@ dust_status dust_noisy_logits_ce(const void* z, int64_t ld_z, dust_dtype dt, con
 dust_status dust_credit(const float* loss, int64_t ld_loss, int32_t K, int64_t N,
                         const int32_t* cu_seqlens, int32_t n_seq, float gamma, float* r,
                         int64_t ld_r, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Attention-internal reward (Dust page, section "간섭(interference) 줄이기", second point): the
+ * perturbations of an attention layer's internal projections (Q, K, V, gate) barely show in
+ * the token loss, so each draw is rewarded by the alignment of the output-error estimate at
+ * the attention output with the change that the draw caused there:
+ *   c[i * ld_c + t] = -<ghat_t, delta_o_t^(i)>
+ * ghat: fp32 [N, ld_g], the output-error estimate at the attention output (for instance the g
+ *       of the output projection from dust_weight_grad); delta_o: [K, N, ld_delta_o] of dtype
+ *       dt (draw-major; row (i, t) starts at (i * N + t) * ld_delta_o), the change of the
+ *       attention output under draw i, computed by the caller's attention recomputation.
+ * c: fp32 [K, ld_c], ld_c >= N.  16-byte aligned ghat and delta_o, ld_g a multiple of 4,
+ * ld_delta_o and d multiples of 8 (bf16) or 4 (fp32); d <= 6144.  The reward feeds
+ * dust_discounted_credit (no centring), then dust_weight_grad of the perturbed projection.
+ * Deterministic (fixed-order sums).
+ */
+dust_status dust_attn_reward(const float* ghat, int64_t ld_g, const void* delta_o,
+                             int64_t ld_delta_o, dust_dtype dt, int64_t N, int32_t d, int32_t K,
+                             float* c, int64_t ld_c, void* stream);
+
+/*
+ * The credit equation on a given reward (no centring): r[i][t] = c[i][t] + gamma * r[i][t+1],
+ * restarted at the last token of each segment.  Same arguments, layout, workspace
+ * (dust_workspace_size(DUST_OP_CREDIT, ...)) and bounded waits as dust_credit; K >= 1.
+ */
+dust_status dust_discounted_credit(const float* c, int64_t ld_c, int32_t K, int64_t N,
+                                   const int32_t* cu_seqlens, int32_t n_seq, float gamma,
+                                   float* r, int64_t ld_r, void* workspace, size_t ws_bytes,
+                                   void* stream);
+
+/*
+ * SPSA / MeZO weight-space probe, the contrast estimator (thakicloud page on zero-order
+ * training, the SPSA paragraph: two forwards with a perturbation of all weights added and
+ * subtracted; gist.science 2605.15622 and the FedSPZO page: the perturbation is regenerated
+ * from a shared seed, so only scalars travel).  Probe j moves W along z_j [d_out, d_in]:
+ *   z_j[o][k] = bf16 of the normal of counter (k >> 2, o, key.draw_offset + j,
+ *               key.layer_id | 2^31), element k & 3 (the noise generator in its own space).
+ * For each probe j in [0, P), with the quadratic readout l_t = 1/2 |y_t - u_t|^2:
+ *   L_+-[j] = sum_t 1/2 |(W +- eps z_j) x_t - u_t|^2,   p[j] = (L_+[j] - L_-[j]) / (2 eps).
+ * The two forwards share y = W x; they are evaluated through sum_t <W x_t - u_t, z_j x_t> and
+ * sum_t |z_j x_t|^2, so p carries no cancellation error.
+ * x [N, d_in], W [d_out, d_in], u [N, d_out]: bf16, 16-byte aligned; d_in and d_out multiples
+ * of 16.  p: DEVICE fp32 [P]; L_plus, L_minus: optional DEVICE fp32 [P] (NULL to skip).
+ * With tokens sharded over devices, p, L_plus and L_minus are sums over the local tokens:
+ * summing them over the devices (P scalars each) gives the whole batch's values.
+ * workspace: dust_workspace_size(DUST_OP_SPSA_PROBE, DUST_BF16, N, d_in, d_out, P) bytes.
+ * key.token_offset and key.channel_offset must be 0 and key.layer_id below 2^31 (the top bit
+ * marks the weight-space stream).  Deterministic.
+ */
+dust_status dust_spsa_probe(const void* x, const void* W, const void* u, dust_dtype dt, int64_t N,
+                            int32_t d_in, int32_t d_out, int32_t P, float eps,
+                            dust_noise_key key, float* p, float* L_plus, float* L_minus,
+                            void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * The SPSA weight estimate: G (+)= (1 / P_total) sum_{j < P} p[j] z_j (z_j as in
+ * dust_spsa_probe, regenerated from key).  p: DEVICE fp32 [P]; G: DEVICE fp32 [d_out, d_in],
+ * 16-byte aligned; accumulate != 0 adds to G (probe chunks of one population).  d_in a
+ * multiple of 4.  Deterministic (probes summed in order).
+ */
+dust_status dust_spsa_estimate(const float* p, int32_t P, int32_t P_total, int32_t d_in,
+                               int32_t d_out, dust_noise_key key, float* G, int accumulate,
+                               void* stream);
 
 /*
  * Output-error estimate and weight estimate (output-error and weight-estimate equations).

@@ -44,6 +44,7 @@ def _case(seed, N, V, dtype):
     (257, 1000, 128, 256, 3, 5e-2),   # a slab, expm1 path, ragged tokens
     (64, 4096, 1024, 1024, 2, 1e-3),
     (10, 96, 4, 20, 2, 1e-2),         # slab not a multiple of 16
+    (50, 1002, 500, 500, 2, 1e-2),    # rows not a multiple of 16 bytes (bf16): scalar stats
 ])
 def test_logits_ce_matches_oracle(z, dtype, N, V, v0, S, K, sigma):
     import torch

@@ -250,3 +250,50 @@ def generate_head(wl: HeadWorkload, data_seed: int = 1006) -> HeadData:
     hs, h64 = _draw(rng, (wl.N, wl.d_model), 1.0, wl.dtype)
     cu = cu_seqlens_from_lengths([wl.seq_len] * wl.n_seq)
     return HeadData(wl, zs, z64, y, hs, h64, cu)
+
+
+# ------------------------------------------------------------------------------ attention
+@dataclasses.dataclass(frozen=True)
+class AttnWorkload:
+    """A value (or key / gate) projection d_model -> d inside attention, estimated from the
+    attention-internal reward: N tokens, K draws, noise scale sigma, discount gamma (close to
+    1 for the projections that later tokens read)."""
+    name: str
+    n_seq: int
+    seq_len: int
+    d_model: int
+    d: int
+    K: int
+    sigma: float
+    gamma: float
+    seed: int
+
+    @property
+    def N(self) -> int:
+        return self.n_seq * self.seq_len
+
+
+ATTN_WORKLOADS = {
+    "attn-v-768": AttnWorkload("attn-v-768", 8, 1024, 768, 768, 16, 1e-3, 0.99,
+                               NOISE_SEED_BASE + 7),
+}
+
+
+@dataclasses.dataclass
+class AttnData:
+    wl: AttnWorkload
+    ghat: np.ndarray       # float32 [N, d]: output-error estimate at the attention output
+    dO_store: np.ndarray   # bf16 bits [K, N, d]: change of the attention output per draw
+    x_store: np.ndarray    # bf16 bits [N, d_model]: the projection's input
+    cu_seqlens: np.ndarray
+
+
+def generate_attn(wl: AttnWorkload, data_seed: int = 1007) -> AttnData:
+    """ghat ~ N(0, 1), delta_o ~ N(0, sigma^2) (what the caller's attention recomputation
+    would hand over), x ~ N(0, 1); draw order ghat, delta_o, x; sequences of seq_len tokens."""
+    rng = np.random.default_rng(data_seed)
+    ghat = rng.standard_normal((wl.N, wl.d)).astype(np.float32)
+    dO = (rng.standard_normal((wl.K, wl.N, wl.d)) * wl.sigma).astype(np.float32)
+    xs, _ = _draw(rng, (wl.N, wl.d_model), 1.0, "bf16")
+    return AttnData(wl, ghat, to_bf16_bits(dO), xs,
+                    cu_seqlens_from_lengths([wl.seq_len] * wl.n_seq))

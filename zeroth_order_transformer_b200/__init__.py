@@ -34,6 +34,7 @@ DUST_OP_NOISY_LINEAR_FWD = 0
 DUST_OP_CREDIT = 1
 DUST_OP_WEIGHT_GRAD = 2
 DUST_OP_LOGITS_CE = 3
+DUST_OP_SPSA_PROBE = 4
 
 EXPORTED_SYMBOLS = (
     "dust_noisy_linear_fwd", "dust_credit", "dust_weight_grad", "dust_workspace_size",
@@ -42,7 +43,8 @@ EXPORTED_SYMBOLS = (
     "dust_profile_read", "dust_credit_no_alloc", "dust_noisy_linear_fwd_grouped",
     "dust_credit_grouped", "dust_weight_grad_grouped", "dust_workspace_size_grouped",
     "dust_optimizer_step", "dust_weight_grad_step", "dust_noisy_logits_ce",
-    "dust_debug_normal_sum",
+    "dust_debug_normal_sum", "dust_attn_reward", "dust_discounted_credit",
+    "dust_spsa_probe", "dust_spsa_estimate",
 )
 
 DUST_OPT_SGD_MOMENTUM = 1
@@ -143,6 +145,18 @@ def lib() -> ctypes.CDLL:
         L.dust_status_string.restype = ctypes.c_char_p
         L.dust_last_device_error.argtypes = [vp, ctypes.POINTER(i32)]
         L.dust_debug_philox.argtypes = [vp, i64, ctypes.c_uint64, vp, vp, vp]
+        L.dust_attn_reward.argtypes = [vp, i64, vp, i64, ctypes.c_int, i64, i32, i32, vp, i64,
+                                       vp]
+        L.dust_attn_reward.restype = ctypes.c_int
+        L.dust_discounted_credit.argtypes = [vp, i64, i32, i64, vp, i32, f32, vp, i64, vp, sz,
+                                             vp]
+        L.dust_discounted_credit.restype = ctypes.c_int
+        L.dust_spsa_probe.argtypes = [vp, vp, vp, ctypes.c_int, i64, i32, i32, i32, f32,
+                                      dust_noise_key, vp, vp, vp, vp, sz, vp]
+        L.dust_spsa_probe.restype = ctypes.c_int
+        L.dust_spsa_estimate.argtypes = [vp, i32, i32, i32, i32, dust_noise_key, vp, ctypes.c_int,
+                                         vp]
+        L.dust_spsa_estimate.restype = ctypes.c_int
         L.dust_debug_normal_sum.argtypes = [dust_noise_key, i64, i32, vp, vp]
         L.dust_debug_normal_sum.restype = ctypes.c_int
         L.dust_debug_credit_skip_publish.argtypes = [i32]
@@ -275,6 +289,85 @@ def dust_credit(loss, cu_seqlens, gamma: float, r=None, workspace=None, stream=N
                            _stream(loss.device, stream))
     _check(st, "dust_credit")
     return r
+
+
+def dust_attn_reward(ghat, delta_o, c=None, stream=None):
+    """Attention-internal reward c[K, N] = -<ghat_t, delta_o[i, t]> from the fp32 output-error
+    estimate ghat [N, d] at the attention output and delta_o [K, N, d] (bf16 or fp32)."""
+    torch = _torch()
+    _cuda(ghat, "ghat")
+    if not delta_o.is_cuda:
+        raise ValueError("delta_o must be a CUDA tensor")
+    if ghat.dtype != torch.float32:
+        raise TypeError("ghat must be float32")
+    K, N, d = delta_o.shape
+    if tuple(ghat.shape) != (N, d) or delta_o.stride(2) != 1 or delta_o.stride(0) != N * delta_o.stride(1):
+        raise ValueError("ghat must be [N, d] and delta_o [K, N, d] with rows N * ld apart")
+    if c is None:
+        c = torch.empty((K, N), dtype=torch.float32, device=ghat.device)
+    st = lib().dust_attn_reward(ghat.data_ptr(), ghat.stride(0), delta_o.data_ptr(),
+                                delta_o.stride(1), _dtype_code(delta_o), N, d, K, c.data_ptr(),
+                                c.stride(0), _stream(ghat.device, stream))
+    _check(st, "dust_attn_reward")
+    return c
+
+
+def dust_discounted_credit(c, cu_seqlens, gamma: float, r=None, workspace=None, stream=None):
+    """The credit equation on a given reward c [K, N] (no centring): r[K, N]."""
+    torch = _torch()
+    _cuda(c, "c"), _cuda(cu_seqlens, "cu_seqlens")
+    if c.dtype != torch.float32 or cu_seqlens.dtype != torch.int32:
+        raise TypeError("c must be float32 and cu_seqlens int32")
+    K, N = c.shape
+    if r is None:
+        r = torch.empty((K, N), dtype=torch.float32, device=c.device)
+    _cuda(r, "r")
+    ws, nb = _workspace(workspace, dust_workspace_size(DUST_OP_CREDIT, DUST_F32, N, 0, 0, K),
+                        c.device)
+    st = lib().dust_discounted_credit(c.data_ptr(), c.stride(0), K, N, cu_seqlens.data_ptr(),
+                                      cu_seqlens.numel() - 1, float(gamma), r.data_ptr(),
+                                      r.stride(0), ws.data_ptr() if ws is not None else None,
+                                      nb, _stream(c.device, stream))
+    _check(st, "dust_discounted_credit")
+    return r
+
+
+def dust_spsa_probe(x, W, u, P: int, eps: float, key: NoiseKey, p=None, losses: bool = False,
+                    workspace=None, stream=None):
+    """SPSA / MeZO probe: p[P] = (L_+ - L_-) / (2 eps) for the weight directions z_j of
+    draws key.draw_offset .. + P; with losses=True also returns L_+ and L_- [P]."""
+    torch = _torch()
+    _cuda(x, "x"), _cuda(W, "W"), _cuda(u, "u")
+    N, d_in = x.shape
+    d_out = W.shape[0]
+    dt = _dtype_code(x)
+    if p is None:
+        p = torch.empty(P, dtype=torch.float32, device=x.device)
+    Lp = torch.empty(P, dtype=torch.float32, device=x.device) if losses else None
+    Lm = torch.empty(P, dtype=torch.float32, device=x.device) if losses else None
+    ws, nb = _workspace(workspace, dust_workspace_size(DUST_OP_SPSA_PROBE, dt, N, d_in, d_out, P),
+                        x.device)
+    st = lib().dust_spsa_probe(x.data_ptr(), W.data_ptr(), u.data_ptr(), dt, N, d_in, d_out, P,
+                               float(eps), key.c(), p.data_ptr(), _ptr(Lp), _ptr(Lm),
+                               ws.data_ptr() if ws is not None else None, nb,
+                               _stream(x.device, stream))
+    _check(st, "dust_spsa_probe")
+    return (p, Lp, Lm) if losses else p
+
+
+def dust_spsa_estimate(p, P_total: int, d_out: int, d_in: int, key: NoiseKey, G=None,
+                       accumulate: bool = False, stream=None):
+    """G [d_out, d_in] (+)= (1/P_total) sum_j p[j] z_j."""
+    torch = _torch()
+    _cuda(p, "p")
+    if G is None:
+        G = torch.empty((d_out, d_in), dtype=torch.float32, device=p.device)
+        accumulate = False
+    _cuda(G, "G")
+    st = lib().dust_spsa_estimate(p.data_ptr(), p.numel(), P_total, d_in, d_out, key.c(),
+                                  G.data_ptr(), 1 if accumulate else 0, _stream(p.device, stream))
+    _check(st, "dust_spsa_estimate")
+    return G
 
 
 def dust_credit_no_alloc(loss, cu_seqlens, gamma: float, r, stream=None):

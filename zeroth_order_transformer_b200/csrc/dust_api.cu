@@ -115,6 +115,19 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tmap_f32_2d_sw128(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols,
+                            uint64_t ld, uint32_t box_rows) {
+    auto fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld * 4};
+    cuuint32_t box[2] = {32, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 namespace {
 struct ProfRecord {
     const char* name;
@@ -223,6 +236,7 @@ size_t dust_workspace_size(dust_op op, dust_dtype dt, int64_t N, int32_t d_in, i
         case DUST_OP_CREDIT: return credit_workspace_bytes(N, K);
         case DUST_OP_WEIGHT_GRAD: return wgrad_workspace_bytes(dt, N, d_in, d_out);
         case DUST_OP_LOGITS_CE: return lmhead_workspace_bytes(N, d_out, K);
+        case DUST_OP_SPSA_PROBE: return spsa_workspace_bytes(N, d_in, d_out, K);
     }
     return 0;
 }
@@ -280,6 +294,69 @@ dust_status dust_credit(const float* loss, int64_t ld_loss, int32_t K, int64_t N
     if (st != DUST_OK) return st;
     return credit_launch(loss, ld_loss, K, N, cu_seqlens, n_seq, gamma, r, ld_r, workspace,
                          static_cast<cudaStream_t>(stream));
+}
+
+dust_status dust_spsa_probe(const void* x, const void* W, const void* u, dust_dtype dt, int64_t N,
+                            int32_t d_in, int32_t d_out, int32_t P, float eps,
+                            dust_noise_key key, float* p, float* L_plus, float* L_minus,
+                            void* workspace, size_t ws_bytes, void* stream) {
+    if (!x || !W || !u || !p || N < 1 || d_in < 1 || d_out < 1 || P < 1 || !valid_dtype(dt))
+        return DUST_ERR_INVALID_ARG;
+    if (!(eps > 0.f) || !std::isfinite(eps) || key.token_offset != 0 || key.channel_offset != 0 ||
+        key.layer_id >= 0x80000000u)
+        return DUST_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(W) || !aligned16(u)) return DUST_ERR_INVALID_ARG;
+    if (static_cast<uint64_t>(key.draw_offset) + static_cast<uint64_t>(P) > 0x100000000ull)
+        return DUST_ERR_INVALID_ARG;
+    if (dt != DUST_BF16 || d_in % 16 != 0 || d_out % 16 != 0 || N > 2147483647LL ||
+        static_cast<int64_t>(P) * ((d_out + 255) / 256 * 256) > 2147483647LL)
+        return DUST_ERR_UNSUPPORTED;
+    dust_status st = check_ws(workspace, ws_bytes, spsa_workspace_bytes(N, d_in, d_out, P));
+    if (st != DUST_OK) return st;
+    return spsa_probe_launch(x, W, u, N, d_in, d_out, P, eps, make_key(key), p, L_plus, L_minus,
+                             workspace, static_cast<cudaStream_t>(stream));
+}
+
+dust_status dust_spsa_estimate(const float* p, int32_t P, int32_t P_total, int32_t d_in,
+                               int32_t d_out, dust_noise_key key, float* G, int accumulate,
+                               void* stream) {
+    if (!p || !G || P < 1 || P_total < P || d_in < 1 || d_out < 1 || d_in % 4 != 0 ||
+        !aligned16(G) || key.token_offset != 0 || key.channel_offset != 0 ||
+        key.layer_id >= 0x80000000u)
+        return DUST_ERR_INVALID_ARG;
+    if (static_cast<uint64_t>(key.draw_offset) + static_cast<uint64_t>(P) > 0x100000000ull)
+        return DUST_ERR_INVALID_ARG;
+    return spsa_estimate_launch(p, P, P_total, d_in, d_out, make_key(key), G, accumulate,
+                                static_cast<cudaStream_t>(stream));
+}
+
+dust_status dust_attn_reward(const float* ghat, int64_t ld_g, const void* delta_o,
+                             int64_t ld_delta_o, dust_dtype dt, int64_t N, int32_t d, int32_t K,
+                             float* c, int64_t ld_c, void* stream) {
+    if (!valid_dtype(dt) || !ghat || !delta_o || !c || N < 1 || d < 1 || K < 1 || ld_g < d ||
+        ld_delta_o < d || ld_c < N)
+        return DUST_ERR_INVALID_ARG;
+    const int E = dt == DUST_BF16 ? 8 : 4;  // elements per 16 bytes
+    if (!aligned16(ghat) || !aligned16(delta_o) || ld_g % 4 != 0 || ld_delta_o % E != 0)
+        return DUST_ERR_INVALID_ARG;
+    if (d % E != 0 || d > 6144) return DUST_ERR_UNSUPPORTED;
+    return attn_reward_launch(ghat, ld_g, delta_o, ld_delta_o, dt, N, d, K, c, ld_c,
+                              static_cast<cudaStream_t>(stream));
+}
+
+dust_status dust_discounted_credit(const float* c, int64_t ld_c, int32_t K, int64_t N,
+                                   const int32_t* cu_seqlens, int32_t n_seq, float gamma,
+                                   float* r, int64_t ld_r, void* workspace, size_t ws_bytes,
+                                   void* stream) {
+    if (!c || !r || !cu_seqlens || N < 1 || K < 1 || n_seq < 1 || ld_c < N || ld_r < N)
+        return DUST_ERR_INVALID_ARG;
+    if (!(gamma >= 0.f && gamma <= 1.f)) return DUST_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0 || !aligned16(c) || !aligned16(r))
+        return DUST_ERR_INVALID_ARG;
+    dust_status st = check_ws(workspace, ws_bytes, credit_workspace_bytes(N, K));
+    if (st != DUST_OK) return st;
+    return credit_launch(c, ld_c, K, N, cu_seqlens, n_seq, gamma, r, ld_r, workspace,
+                         static_cast<cudaStream_t>(stream), 0);
 }
 
 dust_status dust_weight_grad(const float* r, int64_t ld_r, const void* x, dust_dtype dt,

@@ -46,6 +46,11 @@ int num_sms();                   // of the current device
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                        uint32_t box_rows, uint32_t box_cols);
 
+// Encodes a 2-D row-major fp32 tensor [rows, cols] with leading dimension ld (elements) for
+// TMA with a (32 x box_rows) box and 128-byte swizzle: 32 floats make one 128-byte line.
+bool make_tmap_f32_2d_sw128(CUtensorMap* map, const float* base, uint64_t rows, uint64_t cols,
+                            uint64_t ld, uint32_t box_rows);
+
 // ---- noisy linear forward (dust_fwd.cu)
 struct FwdLayerArgs {
     const void* x;
@@ -74,7 +79,21 @@ dust_status lmhead_launch(const void* z, int64_t ld_z, dust_dtype dt, const int3
 size_t credit_workspace_bytes(int64_t N, int32_t K);
 dust_status credit_launch(const float* loss, int64_t ld_loss, int32_t K, int64_t N,
                           const int32_t* cu, int32_t n_seq, float gamma, float* r, int64_t ld_r,
-                          void* ws, cudaStream_t s);
+                          void* ws, cudaStream_t s, int centre = 1);
+
+// ---- SPSA / MeZO weight-space probe (dust_spsa.cu)
+size_t spsa_workspace_bytes(int64_t N, int32_t d_in, int32_t d_out, int32_t P);
+dust_status spsa_probe_launch(const void* x, const void* W, const void* u, int64_t N, int32_t d_in,
+                              int32_t d_out, int32_t P, float eps, NoiseKey key, float* p,
+                              float* Lp, float* Lm, void* ws, cudaStream_t s);
+dust_status spsa_estimate_launch(const float* p, int32_t P, int32_t P_total, int32_t d_in,
+                                 int32_t d_out, NoiseKey key, float* G, int accumulate,
+                                 cudaStream_t s);
+
+// ---- attention-internal reward (dust_attn.cu)
+dust_status attn_reward_launch(const float* ghat, int64_t ld_g, const void* dO, int64_t ld_dO,
+                               dust_dtype dt, int64_t N, int32_t d, int32_t K, float* c,
+                               int64_t ld_c, cudaStream_t s);
 extern int g_credit_skip_publish;
 struct CreditLayerArgs {
     const float* loss;

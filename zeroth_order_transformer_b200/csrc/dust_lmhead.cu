@@ -101,6 +101,61 @@ __global__ void __launch_bounds__(256) ce_stats_kernel(const CeArgs a) {
     }
 }
 
+// Online (max, rescaled sum) update with one value.
+__device__ __forceinline__ void lse_push(float zv, float& m, float& s) {
+    if (zv > m) {
+        s = s * __expf(m - zv) + 1.f;
+        m = zv;
+    } else {
+        s += __expf(zv - m);
+    }
+}
+
+__device__ __forceinline__ void lse_warp_combine(float& m, float& s) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+        const float s2 = __shfl_xor_sync(0xffffffffu, s, off);
+        const float mm = fmaxf(m, m2);
+        s = (m == -INFINITY ? 0.f : s * __expf(m - mm)) + (m2 == -INFINITY ? 0.f : s2 * __expf(m2 - mm));
+        m = mm;
+    }
+}
+
+// The same statistics with one warp per token and 16-byte loads (rows whose start and length
+// are multiples of 16 bytes): HBM-bound.
+template <typename T>
+__global__ void __launch_bounds__(256) ce_stats_vec_kernel(const CeArgs a) {
+    constexpr int E = 16 / sizeof(T);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * 8;
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + warp; t < a.N; t += stride) {
+        const T* zt = static_cast<const T*>(a.z) + t * a.ld_z;
+        float m = -INFINITY, s = 0.f;
+        for (int v = lane * E; v < a.V; v += 32 * E) {
+            const uint4 q = __ldcs(reinterpret_cast<const uint4*>(zt + v));
+            if (sizeof(T) == 2) {
+                const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    lse_push(__uint_as_float(w[j] << 16), m, s);
+                    lse_push(__uint_as_float(w[j] & 0xFFFF0000u), m, s);
+                }
+            } else {
+                lse_push(__uint_as_float(q.x), m, s);
+                lse_push(__uint_as_float(q.y), m, s);
+                lse_push(__uint_as_float(q.z), m, s);
+                lse_push(__uint_as_float(q.w), m, s);
+            }
+        }
+        lse_warp_combine(m, s);
+        if (lane == 0) {
+            const int y = a.y[t];
+            a.stats[t] = make_float4(m, s, (y >= 0 && y < a.V) ? 1.f : 0.f, 0.f);
+        }
+    }
+}
+
 // exp(x) - 1: degree-5 Taylor series for |x| <= 0.1, else the library expm1f.
 template <bool kSeries>
 __device__ __forceinline__ float em1(float x) {
@@ -180,8 +235,15 @@ __global__ void ce_finish_kernel(const CeArgs a) {
 
 template <typename T>
 dust_status launch_typed(CeArgs& a, cudaStream_t s) {
+    const int E = 16 / static_cast<int>(sizeof(T));
+    const bool vec = (reinterpret_cast<uintptr_t>(a.z) & 15u) == 0 && a.V % E == 0 && a.ld_z % E == 0;
     prof_begin(s);
-    ce_stats_kernel<T><<<static_cast<unsigned>(a.N), 256, 0, s>>>(a);
+    if (vec)
+        ce_stats_vec_kernel<T><<<static_cast<unsigned>(std::min<int64_t>((a.N + 7) / 8,
+                                                                       static_cast<int64_t>(num_sms()) * 16)),
+                                 256, 0, s>>>(a);
+    else
+        ce_stats_kernel<T><<<static_cast<unsigned>(a.N), 256, 0, s>>>(a);
     prof_end(s, "lmhead_ce_stats");
     const size_t smem = static_cast<size_t>(kChunk) * kStride * 4;
     const bool series = std::fabs(a.sigma) * 5.8f <= 0.1f;
