@@ -3,8 +3,8 @@
 //
 // Stage 1 (ghat_kernel): one thread per (token, channel quad) regenerates the quad's normals
 // for every draw and accumulates the reward-weighted sum; g is written as bf16 (the tensor
-// core operand) and optionally as fp32.  A grid-stride loop over (layer, token, 128-quad
-// block) units keeps every SM busy to the end.
+// core operand) and optionally as fp32.  A grid-stride loop over units of 128 consecutive
+// (token, quad) pairs of a layer keeps every SM busy to the end.
 // Stage 2 (gw_bf16_kernel): G_W = g^T x on the tensor cores.  Both operands are MN-major
 // (tokens are the contraction index and the slow index of g [N, d_out] and x [N, d_in]):
 // TMA loads 64-token x 64-element boxes with 128-byte swizzle, one thread issues
@@ -31,7 +31,8 @@ struct GhatLayer {
     __nv_bfloat16* gb;  // [N, d_out] or null
     float* gf;          // [N, d_out] or null
     int64_t ld_r, unit_begin;
-    int d_out, nqb;
+    int64_t n_flat;  // N * d_out / 4: (token, channel quad) pairs, token-major
+    int d_out;
     uint32_t layer_id;
 };
 
@@ -50,10 +51,13 @@ __global__ void __launch_bounds__(kGThreads) ghat_kernel(const __grid_constant__
     for (int64_t u = blockIdx.x; u < T.total_units; u += gridDim.x) {
         while (l + 1 < T.n_layers && u >= T.layer[l + 1].unit_begin) ++l;
         const GhatLayer& L = T.layer[l];
-        const int64_t local = u - L.unit_begin;
-        const int64_t t = local / L.nqb;
-        const int q = static_cast<int>(local % L.nqb) * kGThreads + threadIdx.x;
-        if (q >= (L.d_out >> 2)) continue;
+        // a unit is 128 consecutive (token, quad) pairs, so no lane idles when d_out / 4 is
+        // not a multiple of 128
+        const int64_t f = (u - L.unit_begin) * kGThreads + threadIdx.x;
+        if (f >= L.n_flat) continue;
+        const int nq = L.d_out >> 2;
+        const int64_t t = f / nq;
+        const int q = static_cast<int>(f - t * nq);
         const uint32_t tg = T.key.token_offset + static_cast<uint32_t>(t);
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
         const float* rt = L.r + t;
@@ -374,10 +378,10 @@ dust_status launch_bf16_tables(const WgradLayerArgs* layers, int n, int64_t N, i
         L.gb = reinterpret_cast<__nv_bfloat16*>(ws + off);
         L.gf = a.g_out;
         L.d_out = a.d_out;
-        L.nqb = (a.d_out / 4 + kGThreads - 1) / kGThreads;
+        L.n_flat = N * (a.d_out / 4);
         L.unit_begin = units;
         L.layer_id = a.layer_id;
-        units += N * L.nqb;
+        units += (L.n_flat + kGThreads - 1) / kGThreads;
         off += bf16_layer_ws(N, a.d_in, a.d_out, S);
     }
     G.total_units = units;
@@ -505,9 +509,8 @@ dust_status wgrad_launch(const float* r, int64_t ld_r, const void* x, dust_dtype
     G.K = K_chunk;
     G.scale = -1.0f / (static_cast<float>(K_total) * sigma);
     G.key = key;
-    G.layer[0] = GhatLayer{r, nullptr, gf, ld_r, 0, d_out, (d_out / 4 + kGThreads - 1) / kGThreads,
-                           key.layer};
-    G.total_units = N * G.layer[0].nqb;
+    G.layer[0] = GhatLayer{r, nullptr, gf, ld_r, 0, N * (d_out / 4), d_out, key.layer};
+    G.total_units = (G.layer[0].n_flat + kGThreads - 1) / kGThreads;
     const int64_t max_blocks = static_cast<int64_t>(num_sms()) * 16;
     prof_begin(s);
     ghat_kernel<1><<<static_cast<unsigned>(std::min(G.total_units, max_blocks)), kGThreads, 0, s>>>(G);
