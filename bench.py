@@ -45,6 +45,17 @@ OPS_PER_NORMAL = {"fwd_bf16_noise_loss": 20.0, "ghat_reduce_draws": 19.0,
                   # LM head: generator 18 (Philox 10, uniform 3, Box-Muller 5), sigma a (1),
                   # exp(sigma a) - 1 as a degree-5 series (5), the weighted sum (1)
                   "lmhead_ce_noise": 25.0}
+# DRAM bytes (read + write) per launch of a dominant kernel, from one ncu capture of the
+# current build of that kernel on that workload (profiles/ holds the capture summaries);
+# absent entries are reported as null.
+MEASURED_TRAFFIC = {
+    ("fwd_bf16_noise_loss", "gpt2s-mlp-win-768x3072"): (67.83e6 + 3.70e6,
+                                                       "profiles/ncu_full_gpt2s_mlp_win_768x3072.md"),
+    ("ghat_reduce_draws", "gpt2s-mlp-win-768x3072"): (0.54e6 + 0.29e6,
+                                                     "profiles/ncu_full_gpt2s_mlp_win_768x3072.md"),
+    ("lmhead_ce_noise", "head-4096-slab1024"): (34.64e6 + 75.64e6,
+                                                "profiles/ncu_full_lmhead_head-4096-slab1024.md"),
+}
 HEAD_METRIC = "Dust LM-head estimator tokens*draws/s"
 ATTN_METRIC = "Dust attention-reward estimator tokens*draws/s"
 
@@ -357,6 +368,10 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                         "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None}
         if roofline is not None:
             roofline["peak_source"] = peaks["source"]
+            tr = MEASURED_TRAFFIC.get((dominant, wl.name))
+            if tr is not None:
+                roofline["traffic"] = tr[0]
+                roofline["traffic_source"] = tr[1]
             if bound == "alu":
                 gc = generator_ceiling(dust, torch, dev)
                 roofline["generator_ceiling"] = round(gc, 2)
@@ -855,6 +870,8 @@ def run_head(args) -> None:
     units = hw.N * hw.K
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     kernels, roofline = kernel_table(prof, lambda n: head_kernel_work(n, hw), peaks, sms)
+    if roofline is not None and (roofline["kernel"], hw.name) in MEASURED_TRAFFIC:
+        roofline["traffic"], roofline["traffic_source"] = MEASURED_TRAFFIC[(roofline["kernel"], hw.name)]
     if roofline is not None and roofline["bound"] == "alu":
         gc = generator_ceiling(dust, torch, dev)
         roofline["generator_ceiling"] = round(gc, 2)

@@ -129,3 +129,18 @@ def test_head_workload_full_size_sampled(z):
     g64 = g.double()
     ref = (g64.t() @ h.double()).cpu().numpy()
     assert _dev.rel_fro(_dev.host(GW), ref) <= _dev.GW_FRO
+
+
+def test_empty_slab_gives_zero_change_and_bad_slabs_are_rejected(z):
+    """S = 0: no logit is perturbed, so every draw's loss change is exactly 0 (the oracle's
+    special case); slabs that are not quad-aligned or leave the vocabulary are refused."""
+    import torch
+    zt, yt, z64, y = _case(5, 33, 64, "f32")
+    dl = z.dust_noisy_logits_ce(zt, yt, 16, 0, 3, 1e-2, z.NoiseKey(4))
+    torch.cuda.synchronize()
+    assert np.array_equal(_dev.host(dl), np.zeros((3, 33), dtype=np.float32))
+    loss, clean = oracle.noisy_logits_ce(z64, y, 16, 0, 3, 1e-2, 4)
+    assert np.array_equal(loss - clean, np.zeros((3, 33)))
+    for v0, S in ((2, 8), (0, 6), (60, 8)):
+        with pytest.raises(z.DustError):
+            z.dust_noisy_logits_ce(zt, yt, v0, S, 3, 1e-2, z.NoiseKey(4))

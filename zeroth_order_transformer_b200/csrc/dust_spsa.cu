@@ -14,9 +14,9 @@
 //                       (rows d_out .. d_out_pad - 1 of each probe are zero).
 //   spsa_gemm_kernel    tcgen05 GEMM of x against W (residual mode: e = y - u and 1/2 |e|^2)
 //                       or against the stacked directions (probe mode: <e, v> and |v|^2 per
-//                       token and 256-row tile), TMA-fed, accumulator in tensor memory.  The
-//                       probe tiles are ordered probe-fastest so that the CTAs in flight share
-//                       the e and x tiles in L2.
+//                       token and 256-row tile), TMA-fed, accumulator in tensor memory, two
+//                       CTAs per SM.  Tiles run token-tile fastest, so each B tile is read
+//                       once and one output tile's e stays in L2 across the probes.
 //   spsa_reduce_kernel  fixed-order sums over tokens and tiles: p_j = (L_+ - L_-) / (2 eps),
 //                       L_+ and L_-.
 //   spsa_estimate_kernel  G (+)= (1/P_total) sum_j p_j z_j, regenerating z (ALU-bound).
@@ -31,7 +31,7 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBN = 256;
 constexpr int kBK = 64;
-constexpr int kStages = 4;
+constexpr int kStages = 2;  // two CTAs per SM: one's epilogue overlaps the other's mainloop
 constexpr int kThreads = 128;
 constexpr uint32_t kABytes = kBM * kBK * 2;
 constexpr uint32_t kBBytes = kBN * kBK * 2;
@@ -82,7 +82,7 @@ struct GemmArgs {
 };
 
 template <bool kProbe>
-__global__ void __launch_bounds__(kThreads, 1) spsa_gemm_kernel(const __grid_constant__ GemmArgs A) {
+__global__ void __launch_bounds__(kThreads, 2) spsa_gemm_kernel(const __grid_constant__ GemmArgs A) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -92,11 +92,13 @@ __global__ void __launch_bounds__(kThreads, 1) spsa_gemm_kernel(const __grid_con
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // tile order: probe fastest, then the 256-row output tile, then the token tile
+    // tile order: token tile fastest, then the probe, then the 256-row output tile, so that
+    // a B tile (W or one probe's directions) is read from memory once and reused by every
+    // token tile, and one output tile's e (all token tiles) stays in L2 across the probes
     const int P = kProbe ? A.P : 1;
-    const int j = blockIdx.x % P;
-    const int o_tile = (blockIdx.x / P) % A.o_tiles;
-    const int m_tile = blockIdx.x / (P * A.o_tiles);
+    const int m_tile = blockIdx.x % A.m_tiles;
+    const int j = (blockIdx.x / A.m_tiles) % P;
+    const int o_tile = blockIdx.x / (A.m_tiles * P);
     const int64_t m0 = static_cast<int64_t>(m_tile) * kBM;
     const int o0 = o_tile * kBN;
     const int b0 = kProbe ? (j * A.o_tiles + o_tile) * kBN : o0;  // first row of the B tile
@@ -224,43 +226,49 @@ __global__ void __launch_bounds__(kThreads, 1) spsa_gemm_kernel(const __grid_con
 }
 
 // ---------------------------------------------------------------- reductions
-// Block b < P: probe b's sums; block P: the clean loss.  Tokens are summed per thread in order,
-// tiles in order, then the block's threads in a fixed tree.
-__global__ void __launch_bounds__(256) spsa_reduce_kernel(const float* part_l0, const float* part_ev,
-                                                          const float* part_vv, int64_t N,
-                                                          int o_tiles, int P, float eps, float* p,
-                                                          float* Lp, float* Lm, float* l0_out) {
-    __shared__ float sa[256], sb[256], sc[256];
-    const int j = blockIdx.x;  // a probe
-    float a = 0.f, b = 0.f, c = 0.f;
-    for (int ot = 0; ot < o_tiles; ++ot) {
-        const int64_t slot = static_cast<int64_t>(j) * o_tiles + ot;
-        for (int64_t t = threadIdx.x; t < N; t += blockDim.x) {
-            a += part_ev[slot * N + t];
-            b += part_vv[slot * N + t];
-            c += part_l0[static_cast<int64_t>(ot) * N + t];
-        }
-    }
-    sa[threadIdx.x] = a;
-    sb[threadIdx.x] = b;
-    sc[threadIdx.x] = c;
+// Stage 1: block (slot, chunk) sums its chunk of tokens of one partial row in a fixed order
+// (per thread in token order, then the threads in a fixed tree).  Slots: P o_tiles rows of
+// <e, v>, then as many of |v|^2, then o_tiles rows of 1/2 |e|^2.
+constexpr int kRedChunk = 4096;
+__global__ void __launch_bounds__(256) spsa_reduce_kernel(const float* part_ev, const float* part_vv,
+                                                          const float* part_l0, int64_t N,
+                                                          int n_pv, int o_tiles, int n_chunks,
+                                                          float* sums) {
+    __shared__ float sh[256];
+    const int slot = blockIdx.x / n_chunks, chunk = blockIdx.x % n_chunks;
+    const float* row = slot < n_pv ? part_ev + static_cast<int64_t>(slot) * N
+                       : slot < 2 * n_pv ? part_vv + static_cast<int64_t>(slot - n_pv) * N
+                                         : part_l0 + static_cast<int64_t>(slot - 2 * n_pv) * N;
+    const int64_t t_end = min(N, static_cast<int64_t>(chunk + 1) * kRedChunk);
+    float a = 0.f;
+    for (int64_t t = static_cast<int64_t>(chunk) * kRedChunk + threadIdx.x; t < t_end; t += 256)
+        a += row[t];
+    sh[threadIdx.x] = a;
     __syncthreads();
     for (int w = 128; w > 0; w >>= 1) {
-        if (threadIdx.x < w) {
-            sa[threadIdx.x] += sa[threadIdx.x + w];
-            sb[threadIdx.x] += sb[threadIdx.x + w];
-            sc[threadIdx.x] += sc[threadIdx.x + w];
-        }
+        if (threadIdx.x < w) sh[threadIdx.x] += sh[threadIdx.x + w];
         __syncthreads();
     }
-    if (threadIdx.x == 0) {
-        const float ev = sa[0], vv = sb[0], l0 = sc[0];
-        p[j] = ev;  // (L_+ - L_-) / (2 eps) = sum_t <e_t, v_t>
-        const float curv = 0.5f * eps * eps * vv;
-        if (Lp) Lp[j] = l0 + eps * ev + curv;
-        if (Lm) Lm[j] = l0 - eps * ev + curv;
-        if (l0_out && j == 0) *l0_out = l0;
-    }
+    if (threadIdx.x == 0) sums[blockIdx.x] = sh[0];
+}
+
+// Stage 2: one thread per probe adds its tiles' chunk sums in order; p, L_+, L_-.
+__global__ void spsa_finish_kernel(const float* sums, int P, int o_tiles, int n_chunks, float eps,
+                                   float* p, float* Lp, float* Lm) {
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= P) return;
+    const int n_pv = P * o_tiles;
+    float ev = 0.f, vv = 0.f, l0 = 0.f;
+    for (int ot = 0; ot < o_tiles; ++ot)
+        for (int c = 0; c < n_chunks; ++c) {
+            ev += sums[(static_cast<int64_t>(j) * o_tiles + ot) * n_chunks + c];
+            vv += sums[(static_cast<int64_t>(n_pv + j * o_tiles + ot)) * n_chunks + c];
+            l0 += sums[(static_cast<int64_t>(2 * n_pv + ot)) * n_chunks + c];
+        }
+    p[j] = ev;  // (L_+ - L_-) / (2 eps) = sum_t <e_t, v_t>
+    const float curv = 0.5f * eps * eps * vv;
+    if (Lp) Lp[j] = l0 + eps * ev + curv;
+    if (Lm) Lm[j] = l0 - eps * ev + curv;
 }
 
 // G[o][k] (+)= scale * sum_j p_j z_j[o][k]: one thread per (o, channel quad), probes in order.
@@ -306,7 +314,8 @@ size_t spsa_workspace_bytes(int64_t N, int32_t d_in, int32_t d_out, int32_t P) {
     return align_up(static_cast<size_t>(P) * pad256(d_out) * d_in * 2, 256) +  // Z
            align_up(static_cast<size_t>(N) * d_out * 4, 256) +                    // e
            align_up(static_cast<size_t>(o_tiles) * N * 4, 256) +                  // 1/2 |e|^2
-           2 * align_up(static_cast<size_t>(P) * o_tiles * N * 4, 256);           // <e,v>, |v|^2
+           2 * align_up(static_cast<size_t>(P) * o_tiles * N * 4, 256) +          // <e,v>, |v|^2
+           align_up(static_cast<size_t>(2 * P + 1) * o_tiles * ((N + 4095) / 4096) * 4, 256);
 }
 
 dust_status spsa_probe_launch(const void* x, const void* W, const void* u, int64_t N, int32_t d_in,
@@ -325,6 +334,8 @@ dust_status spsa_probe_launch(const void* x, const void* W, const void* u, int64
     float* pev = reinterpret_cast<float*>(w);
     w += align_up(static_cast<size_t>(P) * o_tiles * N * 4, 256);
     float* pvv = reinterpret_cast<float*>(w);
+    w += align_up(static_cast<size_t>(P) * o_tiles * N * 4, 256);
+    float* sums = reinterpret_cast<float*>(w);
 
     GemmArgs R{};
     R.u = static_cast<const __nv_bfloat16*>(u);
@@ -364,9 +375,13 @@ dust_status spsa_probe_launch(const void* x, const void* W, const void* u, int64
     spsa_gemm_kernel<true><<<static_cast<unsigned>(static_cast<int64_t>(m_tiles) * o_tiles * P),
                              kThreads, kSmemBytes, s>>>(Q);
     prof_end(s, "spsa_probe_gemm");
+    const int n_chunks = static_cast<int>((N + kRedChunk - 1) / kRedChunk);
+    const int n_pv = P * o_tiles;
     prof_begin(s);
-    spsa_reduce_kernel<<<static_cast<unsigned>(P), 256, 0, s>>>(pl0, pev, pvv, N, o_tiles, P, eps,
-                                                               p, Lp, Lm, nullptr);
+    spsa_reduce_kernel<<<static_cast<unsigned>((2 * n_pv + o_tiles) * n_chunks), 256, 0, s>>>(
+        pev, pvv, pl0, N, n_pv, o_tiles, n_chunks, sums);
+    spsa_finish_kernel<<<static_cast<unsigned>((P + 127) / 128), 128, 0, s>>>(sums, P, o_tiles,
+                                                                            n_chunks, eps, p, Lp, Lm);
     prof_end(s, "spsa_reduce");
     return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
 }
