@@ -6,9 +6,9 @@
 // slab of losses into shared memory as four 32-token sub-slabs whose 128-byte lines are
 // swizzled (16-byte chunk c of row i sits at chunk c ^ (i mod 8)); the per-token mean over the
 // draws is taken by one thread per token.  Then four threads own each draw row, 32 tokens
-// each, held in registers: a thread centres its tokens and composes their affine maps
-// r_t = c_t + g_t r_{t+1} (g_t = gamma, or 0 at a segment's last token) serially, and the four
-// maps of a row are composed with shuffles.  Eight consecutive lanes hold eight different rows
+// each, streamed from the slab in 16-byte chunks: a thread centres its tokens and composes
+// their affine maps r_t = c_t + g_t r_{t+1} (g_t = gamma, or 0 at a segment's last token)
+// serially, and the four maps of a row are composed with shuffles.  Eight consecutive lanes hold eight different rows
 // of the same sub-slab, so every 16-byte shared access of a warp is conflict-free.  Blocks are
 // chained from the end of the stream to its start by decoupled look-back: each warp publishes
 // its rows' aggregate maps (A, G), r_first = A + G r_next, then their inclusive values once
@@ -120,8 +120,8 @@ __device__ __forceinline__ int warp_upper_bound(const int32_t* cu, int n_seq, in
     return lo;
 }
 
-template <int kMax>
-__global__ void __launch_bounds__(kMaxThreads, 2) credit_kernel(const __grid_constant__ CreditTable<kMax> T) {
+template <int kMax, int kThr, int kMinBlocks>
+__global__ void __launch_bounds__(kThr, kMinBlocks) credit_kernel(const __grid_constant__ CreditTable<kMax> T) {
     const int lyr = blockIdx.y / T.n_groups;
     const int grp = blockIdx.y % T.n_groups;
     const CreditLayer& L = T.layer[lyr];
@@ -210,41 +210,34 @@ __global__ void __launch_bounds__(kMaxThreads, 2) credit_kernel(const __grid_con
         __syncthreads();
     }
 
-    // Pass 1.  Thread (row i, part sg) holds tokens 32 sg .. 32 sg + 31 of row i.
+    // Pass 1.  Thread (row i, part sg) owns tokens 32 sg .. 32 sg + 31 of row i and composes
+    // their maps from the last token to the first, streaming 16-byte chunks from the slab (the
+    // values are not kept in registers, so six CTAs fit on an SM).
     const int i = warp * kRowsPerWarp + (lane & 7);
     const int sg = lane >> 3;
     float* line = slab + sg * Rp * kTPT + i * kTPT;
-    float v[kTPT];
-#pragma unroll
-    for (int c = 0; c < kTPT / 4; ++c) {
-        const float4 q = *reinterpret_cast<const float4*>(line + ((c ^ (i & 7)) << 2));
-        v[4 * c] = q.x;
-        v[4 * c + 1] = q.y;
-        v[4 * c + 2] = q.z;
-        v[4 * c + 3] = q.w;
-    }
-    if (T.centre) {
-#pragma unroll
-        for (int c = 0; c < kTPT / 4; ++c) {
-            const float4 m = *reinterpret_cast<const float4*>(mean + sg * kTPT + 4 * c);
-            v[4 * c] = m.x - v[4 * c];
-            v[4 * c + 1] = m.y - v[4 * c + 1];
-            v[4 * c + 2] = m.z - v[4 * c + 2];
-            v[4 * c + 3] = m.w - v[4 * c + 3];
+    // the centred values c = mean - loss of chunk cc of this thread's tokens
+    auto centred = [&](int cc) {
+        float4 q = *reinterpret_cast<const float4*>(line + ((cc ^ (i & 7)) << 2));
+        if (T.centre) {
+            const float4 m = *reinterpret_cast<const float4*>(mean + sg * kTPT + 4 * cc);
+            q = make_float4(m.x - q.x, m.y - q.y, m.z - q.z, m.w - q.w);
         }
-    }
+        return q;
+    };
     // this thread's map, last token first: r_first = A + G r_next
     float A = 0.f, G = 1.f;
-#pragma unroll
+#pragma unroll 2
     for (int c = kTPT / 4 - 1; c >= 0; --c) {
         const float4 g = *reinterpret_cast<const float4*>(gval + sg * kTPT + 4 * c);
-        A = fmaf(g.w, A, v[4 * c + 3]);
+        const float4 q = centred(c);
+        A = fmaf(g.w, A, q.w);
         G = g.w * G;
-        A = fmaf(g.z, A, v[4 * c + 2]);
+        A = fmaf(g.z, A, q.z);
         G = g.z * G;
-        A = fmaf(g.y, A, v[4 * c + 1]);
+        A = fmaf(g.y, A, q.y);
         G = g.y * G;
-        A = fmaf(g.x, A, v[4 * c]);
+        A = fmaf(g.x, A, q.x);
         G = g.x * G;
     }
     // suffix over the row's four parts (lanes sg, sg + 8, sg + 16, sg + 24 of the warp)
@@ -351,20 +344,22 @@ __global__ void __launch_bounds__(kMaxThreads, 2) credit_kernel(const __grid_con
         __syncwarp();
     }
 
-    // Pass 2: the credit of this thread's tokens, from the carry of its row, back into the slab.
+    // Pass 2: the credit of this thread's tokens, from the carry of its row, back into the slab
+    // (the centred values are formed again from the slab, in the same arithmetic).
     {
         float rn = fmaf(eG, carry[i], eA);
-#pragma unroll
+#pragma unroll 2
         for (int c = kTPT / 4 - 1; c >= 0; --c) {
             const float4 g = *reinterpret_cast<const float4*>(gval + sg * kTPT + 4 * c);
+            const float4 cv = centred(c);
             float4 q;
-            rn = fmaf(g.w, rn, v[4 * c + 3]);
+            rn = fmaf(g.w, rn, cv.w);
             q.w = rn;
-            rn = fmaf(g.z, rn, v[4 * c + 2]);
+            rn = fmaf(g.z, rn, cv.z);
             q.z = rn;
-            rn = fmaf(g.y, rn, v[4 * c + 1]);
+            rn = fmaf(g.y, rn, cv.y);
             q.y = rn;
-            rn = fmaf(g.x, rn, v[4 * c]);
+            rn = fmaf(g.x, rn, cv.x);
             q.x = rn;
             *reinterpret_cast<float4*>(line + ((c ^ (i & 7)) << 2)) = q;
         }
@@ -469,13 +464,16 @@ dust_status launch_credit_table(const CreditTable<kMax>& T, int n_layers, cudaSt
         prof_end(s, "credit_mean");
     }
     const size_t smem = smem_bytes(T.rows_p);
-    if (cudaFuncSetAttribute(credit_kernel<kMax>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const int threads = kSeg * T.rows_p;
+    // up to 64 rows (256 threads): six resident blocks (42 registers each); 128 rows: two
+    auto kern = threads <= 256 ? credit_kernel<kMax, 256, 6> : credit_kernel<kMax, kMaxThreads, 2>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return DUST_ERR_CUDA;
     if (static_cast<int64_t>(n_layers) * T.n_groups > 65535) return DUST_ERR_UNSUPPORTED;
     prof_begin(s);
-    credit_kernel<kMax><<<dim3(static_cast<unsigned>(T.nblk), static_cast<unsigned>(n_layers * T.n_groups)),
-                          kSeg * T.rows_p, smem, s>>>(T);
+    kern<<<dim3(static_cast<unsigned>(T.nblk), static_cast<unsigned>(n_layers * T.n_groups)),
+           threads, smem, s>>>(T);
     prof_end(s, name);
     return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
 }
