@@ -475,7 +475,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, f32/u32 noise",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "operands": "bf16 x, W, u; u32 Philox words",
         "data": "synthetic (seeded; shapes of the Dust page's transformer layers)",
         "config": {"workload": describe(wl), "tokens_per_gpu": wl.N, "d_in": s0.d_in,
                    "d_out": s0.d_out, "K": wl.K, "layers": len(layers),
@@ -656,7 +656,7 @@ def run_attn(args) -> None:
     line = {
         "metric": ATTN_METRIC, "value": units / (ms / 1e3), "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 delta_o and x, f32 ghat",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "operands": "bf16 delta_o and x, f32 ghat",
         "data": "synthetic (seeded; GPT-2-small attention shape)",
         "config": {"workload": f"{aw.name}: {aw.n_seq}x{aw.seq_len} tokens, projection "
                                f"{aw.d_model}->{aw.d}, K={aw.K}, sigma={aw.sigma}, "
@@ -781,7 +781,7 @@ def run_spsa(args) -> None:
         "metric": "SPSA/MeZO contrast estimator tokens*probes/s", "value": units / (ms / 1e3),
         "unit": "tokens*probes/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16 in, f32 accumulate", "data": "synthetic (seeded)",
+        "dtype": "f32", "operands": "bf16 x, W, u and directions", "data": "synthetic (seeded)",
         "config": {"workload": f"{describe(wl)}; first layer; P={P} probes, eps=1e-3",
                    "l2": "flushed (256 MiB write) before every timed step"},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
@@ -926,7 +926,7 @@ def run_head(args) -> None:
     line = {
         "metric": HEAD_METRIC, "value": units / (ms / 1e3), "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": f"{hw.dtype} logits, f32/u32 noise",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "operands": f"{hw.dtype} logits and hidden states",
         "data": "synthetic (seeded; the Dust page's head shape)",
         "config": {"workload": f"{hw.name}: {hw.n_seq}x{hw.seq_len} tokens, vocabulary {hw.V}, "
                                f"slab [{hw.v0}, {hw.v0 + hw.S}), width {hw.d_model}, K={hw.K}, "

@@ -12,10 +12,12 @@
 // two large fp32 losses:
 //   spsa_dir_kernel     z_j for all probes, bf16, into the workspace [P, d_out_pad, d_in]
 //                       (rows d_out .. d_out_pad - 1 of each probe are zero).
-//   spsa_gemm_kernel    tcgen05 GEMM of x against W (residual mode: e = y - u and 1/2 |e|^2)
-//                       or against the stacked directions (probe mode: <e, v> and |v|^2 per
-//                       token and 256-row tile), TMA-fed, accumulator in tensor memory, two
-//                       CTAs per SM.  Tiles run token-tile fastest, so each B tile is read
+//   spsa_gemm_kernel    tcgen05 GEMM of x against W (residual mode: e = y - u and 1/2 |e|^2),
+//                       TMA-fed, accumulator in tensor memory, two CTAs per SM.
+//   spsa_probe_gemm_kernel  the same against the stacked directions (probe mode: <e, v> and
+//                       |v|^2 per token and 256-row tile), persistent and warp-specialised with
+//                       two accumulators, so each tile's epilogue overlaps the next tile's
+//                       mainloop.  Tiles run token-tile fastest, so each direction tile is read
 //                       once and one output tile's e stays in L2 across the probes.
 //   spsa_reduce_kernel  fixed-order sums over tokens and tiles: p_j = (L_+ - L_-) / (2 eps),
 //                       L_+ and L_-.
@@ -81,7 +83,6 @@ struct GemmArgs {
     int d_in, d_out, o_tiles, P, m_tiles;
 };
 
-template <bool kProbe>
 __global__ void __launch_bounds__(kThreads, 2) spsa_gemm_kernel(const __grid_constant__ GemmArgs A) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -92,16 +93,12 @@ __global__ void __launch_bounds__(kThreads, 2) spsa_gemm_kernel(const __grid_con
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // tile order: token tile fastest, then the probe, then the 256-row output tile, so that
-    // a B tile (W or one probe's directions) is read from memory once and reused by every
-    // token tile, and one output tile's e (all token tiles) stays in L2 across the probes
-    const int P = kProbe ? A.P : 1;
+    // tile order: token tile fastest, so a tile of W is read once for all token tiles
     const int m_tile = blockIdx.x % A.m_tiles;
-    const int j = (blockIdx.x / A.m_tiles) % P;
-    const int o_tile = blockIdx.x / (A.m_tiles * P);
+    const int o_tile = blockIdx.x / A.m_tiles;
     const int64_t m0 = static_cast<int64_t>(m_tile) * kBM;
     const int o0 = o_tile * kBN;
-    const int b0 = kProbe ? (j * A.o_tiles + o_tile) * kBN : o0;  // first row of the B tile
+    const int b0 = o0;  // first row of the B tile
     const int nk = (A.d_in + kBK - 1) / kBK;
 
     if (threadIdx.x == 0) {
@@ -161,74 +158,209 @@ __global__ void __launch_bounds__(kThreads, 2) spsa_gemm_kernel(const __grid_con
     const bool valid = t < A.N;
     const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const int nchunks = min(kBN, A.d_out - o0) / 16;
-    float sa = 0.f, sb = 0.f;
+    float sa = 0.f;
     for (int c = 0; c < nchunks; ++c) {
         float v[16];
         tmem_ld16(trow + c * 16, v);
         tmem_wait_ld();
         if (!valid) continue;
         const int64_t off = t * A.d_out + o0 + c * 16;
-        if (kProbe) {
-            const float4* e4 = reinterpret_cast<const float4*>(A.e + off);
+        const uint4* up = reinterpret_cast<const uint4*>(A.u + off);
+        float uf[16];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint4 w = __ldg(up + h);
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const float4 e = __ldg(e4 + q);
-                sa = fmaf(e.x, v[4 * q], sa);
-                sa = fmaf(e.y, v[4 * q + 1], sa);
-                sa = fmaf(e.z, v[4 * q + 2], sa);
-                sa = fmaf(e.w, v[4 * q + 3], sa);
-                sb = fmaf(v[4 * q], v[4 * q], sb);
-                sb = fmaf(v[4 * q + 1], v[4 * q + 1], sb);
-                sb = fmaf(v[4 * q + 2], v[4 * q + 2], sb);
-                sb = fmaf(v[4 * q + 3], v[4 * q + 3], sb);
-            }
-        } else {
-            const uint4* up = reinterpret_cast<const uint4*>(A.u + off);
-            float uf[16];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint4 w = __ldg(up + h);
-                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uf[8 * h + 2 * q] = __uint_as_float(ww[q] << 16);
-                    uf[8 * h + 2 * q + 1] = __uint_as_float(ww[q] & 0xFFFF0000u);
-                }
-            }
-            float4* e4 = reinterpret_cast<float4*>(A.e + off);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float4 e;
-                e.x = v[4 * q] - uf[4 * q];
-                e.y = v[4 * q + 1] - uf[4 * q + 1];
-                e.z = v[4 * q + 2] - uf[4 * q + 2];
-                e.w = v[4 * q + 3] - uf[4 * q + 3];
-                e4[q] = e;
-                sa = fmaf(e.x, e.x, sa);
-                sa = fmaf(e.y, e.y, sa);
-                sa = fmaf(e.z, e.z, sa);
-                sa = fmaf(e.w, e.w, sa);
+                uf[8 * h + 2 * q] = __uint_as_float(ww[q] << 16);
+                uf[8 * h + 2 * q + 1] = __uint_as_float(ww[q] & 0xFFFF0000u);
             }
         }
-    }
-    if (valid) {
-        const int64_t slot = static_cast<int64_t>(kProbe ? j * A.o_tiles + o_tile : o_tile);
-        if (kProbe) {
-            A.part_a[slot * A.N + t] = sa;
-            A.part_b[slot * A.N + t] = sb;
-        } else {
-            A.part_a[slot * A.N + t] = 0.5f * sa;
+        float4* e4 = reinterpret_cast<float4*>(A.e + off);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float4 e;
+            e.x = v[4 * q] - uf[4 * q];
+            e.y = v[4 * q + 1] - uf[4 * q + 1];
+            e.z = v[4 * q + 2] - uf[4 * q + 2];
+            e.w = v[4 * q + 3] - uf[4 * q + 3];
+            e4[q] = e;
+            sa = fmaf(e.x, e.x, sa);
+            sa = fmaf(e.y, e.y, sa);
+            sa = fmaf(e.z, e.z, sa);
+            sa = fmaf(e.w, e.w, sa);
         }
     }
+    if (valid) A.part_a[static_cast<int64_t>(o_tile) * A.N + t] = 0.5f * sa;
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+// ---------------------------------------------------------------- persistent probe GEMM
+// The probe mode as a persistent, warp-specialised kernel: one CTA per SM walks the tiles in the
+// same order; warp 0 feeds a 4-stage TMA ring, warp 1 issues the MMAs into one of two
+// 256-column accumulators, and warps 2-9 run the epilogue of the previous tile from the other
+// accumulator meanwhile: warp w reads TMEM lanes 32 (w % 4) .. + 31 (its tokens) and the
+// columns of half (w - 2) / 4 of the tile, so each (token, half) has its own partial sums.
+constexpr int kPStages = 4;
+constexpr int kPThreads = 320;  // producer, MMA issuer, eight epilogue warps
+constexpr uint32_t kPSmemBytes = kPStages * kStageBytes + 1024 + 256;
+
+__global__ void __launch_bounds__(kPThreads, 1) spsa_probe_gemm_kernel(const __grid_constant__ GemmArgs A) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPStages * kStageBytes);
+    uint64_t* empty = full + kPStages;
+    uint64_t* acc_full = empty + kPStages;  // [2]
+    uint64_t* acc_empty = acc_full + 2;     // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_tiles = A.m_tiles * A.P * A.o_tiles;
+    const int nk = (A.d_in + kBK - 1) / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 8);  // one arrival per epilogue warp
+        }
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 2 * kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tensormap(&A.tmx);
+            prefetch_tensormap(&A.tmb);
+            uint32_t kc = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+                const int m_tile = tile % A.m_tiles;
+                const int j = (tile / A.m_tiles) % A.P;
+                const int o_tile = tile / (A.m_tiles * A.P);
+                const int b0 = (j * A.o_tiles + o_tile) * kBN;
+                for (int kb = 0; kb < nk; ++kb, ++kc) {
+                    const int s = kc % kPStages;
+                    if (kc >= kPStages &&
+                        !mbar_wait_bounded(&empty[s], ((kc / kPStages) - 1) & 1, A.ew, 411)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* a = smem + s * kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], kStageBytes);
+                    tma_load_2d(a, &A.tmx, &full[s], kb * kBK, m_tile * kBM);
+                    tma_load_2d(a + kABytes, &A.tmb, &full[s], kb * kBK, b0);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, 0, 0);
+            uint32_t kc = 0;
+            int lt = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++lt) {
+                const int buf = lt & 1;
+                // the epilogue of the tile that last used this accumulator has read it
+                if (lt >= 2 && !mbar_wait_bounded(&acc_empty[buf], ((lt >> 1) - 1) & 1, A.ew, 412))
+                    break;
+                tc_fence_after();
+                const uint32_t d = tmem + static_cast<uint32_t>(buf * kTmemCols);
+                for (int kb = 0; kb < nk; ++kb, ++kc) {
+                    const int s = kc % kPStages;
+                    if (!mbar_wait_bounded(&full[s], (kc / kPStages) & 1, A.ew, 413)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
+                    const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
+                        const uint64_t bd = sdesc_sw128(b_addr + kk * 32, 16, 1024);
+                        umma_bf16(d, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(&empty[s]);
+                }
+                umma_commit(&acc_full[buf]);
+            }
+        }
+    } else {
+        // epilogue warps 2..9: TMEM lane quarter q = warp % 4, column half hf
+        const int q = warp & 3;
+        const int hf = (warp - 2) >> 2;
+        int lt = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++lt) {
+            const int buf = lt & 1;
+            const int m_tile = tile % A.m_tiles;
+            const int j = (tile / A.m_tiles) % A.P;
+            const int o_tile = tile / (A.m_tiles * A.P);
+            const int o0 = o_tile * kBN;
+            if (!mbar_wait_bounded(&acc_full[buf], (lt >> 1) & 1, A.ew, 414)) break;
+            __syncwarp();
+            tc_fence_after();
+            const int row = q * 32 + lane;
+            const int64_t t = static_cast<int64_t>(m_tile) * kBM + row;
+            const bool valid = t < A.N;
+            const uint32_t trow = tmem + static_cast<uint32_t>(buf * kTmemCols) +
+                                  (static_cast<uint32_t>(q * 32) << 16);
+            const int nchunks = min(kBN, A.d_out - o0) / 16;
+            const int c_end = min(nchunks, (hf + 1) * (kBN / 32));
+            float sa = 0.f, sb = 0.f;
+            for (int c = hf * (kBN / 32); c < c_end; ++c) {
+                float v[16];
+                tmem_ld16(trow + c * 16, v);
+                tmem_wait_ld();
+                if (!valid) continue;
+                const float4* e4 = reinterpret_cast<const float4*>(A.e + t * A.d_out + o0 + c * 16);
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const float4 e = __ldg(e4 + qq);
+                    sa = fmaf(e.x, v[4 * qq], sa);
+                    sa = fmaf(e.y, v[4 * qq + 1], sa);
+                    sa = fmaf(e.z, v[4 * qq + 2], sa);
+                    sa = fmaf(e.w, v[4 * qq + 3], sa);
+                    sb = fmaf(v[4 * qq], v[4 * qq], sb);
+                    sb = fmaf(v[4 * qq + 1], v[4 * qq + 1], sb);
+                    sb = fmaf(v[4 * qq + 2], v[4 * qq + 2], sb);
+                    sb = fmaf(v[4 * qq + 3], v[4 * qq + 3], sb);
+                }
+            }
+            // the accumulator may be refilled once every epilogue warp has read it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            if (valid) {
+                const int64_t slot = (static_cast<int64_t>(j) * A.o_tiles + o_tile) * 2 + hf;
+                A.part_a[slot * A.N + t] = sa;
+                A.part_b[slot * A.N + t] = sb;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, 2 * kTmemCols);
+}
+
 // ---------------------------------------------------------------- reductions
 // Stage 1: block (slot, chunk) sums its chunk of tokens of one partial row in a fixed order
-// (per thread in token order, then the threads in a fixed tree).  Slots: P o_tiles rows of
-// <e, v>, then as many of |v|^2, then o_tiles rows of 1/2 |e|^2.
+// (per thread in token order, then the threads in a fixed tree).  Slots: 2 P o_tiles rows of
+// <e, v> (probe, output tile, column half), then as many of |v|^2, then o_tiles rows of
+// 1/2 |e|^2.
 constexpr int kRedChunk = 4096;
 __global__ void __launch_bounds__(256) spsa_reduce_kernel(const float* part_ev, const float* part_vv,
                                                           const float* part_l0, int64_t N,
@@ -257,14 +389,18 @@ __global__ void spsa_finish_kernel(const float* sums, int P, int o_tiles, int n_
                                    float* p, float* Lp, float* Lm) {
     const int j = blockIdx.x * blockDim.x + threadIdx.x;
     if (j >= P) return;
-    const int n_pv = P * o_tiles;
+    const int n_pv = P * o_tiles * 2;  // (probe, output tile, column half) slots
     float ev = 0.f, vv = 0.f, l0 = 0.f;
-    for (int ot = 0; ot < o_tiles; ++ot)
-        for (int c = 0; c < n_chunks; ++c) {
-            ev += sums[(static_cast<int64_t>(j) * o_tiles + ot) * n_chunks + c];
-            vv += sums[(static_cast<int64_t>(n_pv + j * o_tiles + ot)) * n_chunks + c];
+    for (int ot = 0; ot < o_tiles; ++ot) {
+        for (int h = 0; h < 2; ++h)
+            for (int c = 0; c < n_chunks; ++c) {
+                const int64_t sl = (static_cast<int64_t>(j) * o_tiles + ot) * 2 + h;
+                ev += sums[sl * n_chunks + c];
+                vv += sums[(n_pv + sl) * n_chunks + c];
+            }
+        for (int c = 0; c < n_chunks; ++c)
             l0 += sums[(static_cast<int64_t>(2 * n_pv + ot)) * n_chunks + c];
-        }
+    }
     p[j] = ev;  // (L_+ - L_-) / (2 eps) = sum_t <e_t, v_t>
     const float curv = 0.5f * eps * eps * vv;
     if (Lp) Lp[j] = l0 + eps * ev + curv;
@@ -314,8 +450,8 @@ size_t spsa_workspace_bytes(int64_t N, int32_t d_in, int32_t d_out, int32_t P) {
     return align_up(static_cast<size_t>(P) * pad256(d_out) * d_in * 2, 256) +  // Z
            align_up(static_cast<size_t>(N) * d_out * 4, 256) +                    // e
            align_up(static_cast<size_t>(o_tiles) * N * 4, 256) +                  // 1/2 |e|^2
-           2 * align_up(static_cast<size_t>(P) * o_tiles * N * 4, 256) +          // <e,v>, |v|^2
-           align_up(static_cast<size_t>(2 * P + 1) * o_tiles * ((N + 4095) / 4096) * 4, 256);
+           2 * align_up(static_cast<size_t>(2 * P) * o_tiles * N * 4, 256) +      // <e,v>, |v|^2
+           align_up(static_cast<size_t>(4 * P + 1) * o_tiles * ((N + 4095) / 4096) * 4, 256);
 }
 
 dust_status spsa_probe_launch(const void* x, const void* W, const void* u, int64_t N, int32_t d_in,
@@ -324,6 +460,7 @@ dust_status spsa_probe_launch(const void* x, const void* W, const void* u, int64
     const int dpad = pad256(d_out);
     const int o_tiles = dpad / kBN;
     const int m_tiles = static_cast<int>((N + kBM - 1) / kBM);
+    if (static_cast<int64_t>(m_tiles) * o_tiles * P > 2147483647LL) return DUST_ERR_UNSUPPORTED;
     char* w = static_cast<char*>(ws);
     __nv_bfloat16* Z = reinterpret_cast<__nv_bfloat16*>(w);
     w += align_up(static_cast<size_t>(P) * dpad * d_in * 2, 256);
@@ -332,9 +469,9 @@ dust_status spsa_probe_launch(const void* x, const void* W, const void* u, int64
     float* pl0 = reinterpret_cast<float*>(w);
     w += align_up(static_cast<size_t>(o_tiles) * N * 4, 256);
     float* pev = reinterpret_cast<float*>(w);
-    w += align_up(static_cast<size_t>(P) * o_tiles * N * 4, 256);
+    w += align_up(static_cast<size_t>(2 * P) * o_tiles * N * 4, 256);
     float* pvv = reinterpret_cast<float*>(w);
-    w += align_up(static_cast<size_t>(P) * o_tiles * N * 4, 256);
+    w += align_up(static_cast<size_t>(2 * P) * o_tiles * N * 4, 256);
     float* sums = reinterpret_cast<float*>(w);
 
     GemmArgs R{};
@@ -357,10 +494,10 @@ dust_status spsa_probe_launch(const void* x, const void* W, const void* u, int64
     Q.part_b = pvv;
     if (!make_tmap_bf16_2d(&Q.tmb, Z, static_cast<uint64_t>(P) * dpad, d_in, kBN, kBK))
         return DUST_ERR_CUDA;
-    if (cudaFuncSetAttribute(spsa_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(spsa_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBytes)) != cudaSuccess ||
-        cudaFuncSetAttribute(spsa_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+        cudaFuncSetAttribute(spsa_probe_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kPSmemBytes)) != cudaSuccess)
         return DUST_ERR_CUDA;
     const int64_t dir_total = static_cast<int64_t>(P) * dpad * (d_in / 4);
     prof_begin(s);
@@ -369,14 +506,15 @@ dust_status spsa_probe_launch(const void* x, const void* W, const void* u, int64
                       256, 0, s>>>(key, P, d_out, dpad, d_in, Z);
     prof_end(s, "spsa_directions");
     prof_begin(s);
-    spsa_gemm_kernel<false><<<static_cast<unsigned>(m_tiles * o_tiles), kThreads, kSmemBytes, s>>>(R);
+    spsa_gemm_kernel<<<static_cast<unsigned>(m_tiles * o_tiles), kThreads, kSmemBytes, s>>>(R);
     prof_end(s, "spsa_residual_gemm");
     prof_begin(s);
-    spsa_gemm_kernel<true><<<static_cast<unsigned>(static_cast<int64_t>(m_tiles) * o_tiles * P),
-                             kThreads, kSmemBytes, s>>>(Q);
+    const int64_t probe_tiles = static_cast<int64_t>(m_tiles) * o_tiles * P;
+    spsa_probe_gemm_kernel<<<static_cast<unsigned>(std::min<int64_t>(probe_tiles, num_sms())),
+                             kPThreads, kPSmemBytes, s>>>(Q);
     prof_end(s, "spsa_probe_gemm");
     const int n_chunks = static_cast<int>((N + kRedChunk - 1) / kRedChunk);
-    const int n_pv = P * o_tiles;
+    const int n_pv = 2 * P * o_tiles;
     prof_begin(s);
     spsa_reduce_kernel<<<static_cast<unsigned>((2 * n_pv + o_tiles) * n_chunks), 256, 0, s>>>(
         pev, pvv, pl0, N, n_pv, o_tiles, n_chunks, sums);
