@@ -96,6 +96,22 @@ dust_status dust_noisy_linear_fwd(const void* x, const void* W, const void* u, d
                                   void* stream);
 
 /*
+ * The perturbed layer outputs themselves, for callers that evaluate their own loss downstream
+ * (for instance by recomputing the later blocks of a model for each draw, as the Dust page's
+ * section "간섭(interference) 줄이기" describes for a perturbed block):
+ *   y_out[(i * N + t) * ld_out + o] = (W x_t)[o] + sigma a_t^(i)[o],  i < K, t < N, o < d_out
+ * with the same noise as dust_noisy_linear_fwd for the same key.  x [N, d_in], W [d_out, d_in]:
+ * bf16 (d_in, d_out multiples of 16), 16-byte aligned.  y_out: DEVICE, out_dt fp32 or bf16
+ * (rounded to nearest even), 16-byte aligned; ld_out >= d_out, a multiple of 16 bytes'
+ * elements.  K N d_out values are written: this materialises what the fused forward never
+ * stores.  Deterministic.
+ */
+dust_status dust_noisy_linear_output(const void* x, const void* W, dust_dtype dt, int64_t N,
+                                     int32_t d_in, int32_t d_out, int32_t K, float sigma,
+                                     dust_noise_key key, void* y_out, dust_dtype out_dt,
+                                     int64_t ld_out, void* stream);
+
+/*
  * LM-head perturbation on cached logits (Dust page, section "간섭(interference) 줄이기": the
  * LM head is perturbed on the cached logits and only the cross-entropy is recomputed, on a
  * slab of the vocabulary).  For each draw i and token t, with noise sigma a_t^(i)[v] added to

@@ -296,6 +296,25 @@ dust_status dust_credit(const float* loss, int64_t ld_loss, int32_t K, int64_t N
                          static_cast<cudaStream_t>(stream));
 }
 
+dust_status dust_noisy_linear_output(const void* x, const void* W, dust_dtype dt, int64_t N,
+                                     int32_t d_in, int32_t d_out, int32_t K, float sigma,
+                                     dust_noise_key key, void* y_out, dust_dtype out_dt,
+                                     int64_t ld_out, void* stream) {
+    dust_status st = check_layer(x, dt, N, d_in, d_out);
+    if (st != DUST_OK) return st;
+    if (!W || !y_out || !aligned16(W) || !aligned16(y_out) || K < 1 || ld_out < d_out ||
+        !valid_dtype(out_dt) || !std::isfinite(sigma) || key.channel_offset % 4 != 0)
+        return DUST_ERR_INVALID_ARG;
+    if (ld_out % (out_dt == DUST_BF16 ? 8 : 4) != 0) return DUST_ERR_INVALID_ARG;
+    if (static_cast<uint64_t>(key.draw_offset) + static_cast<uint64_t>(K) > 0x100000000ull ||
+        static_cast<uint64_t>(key.token_offset) + static_cast<uint64_t>(N) > 0x100000000ull)
+        return DUST_ERR_INVALID_ARG;
+    if (dt != DUST_BF16 || N > 2147483647LL) return DUST_ERR_UNSUPPORTED;
+    return noisy_output_launch(x, W, N, d_in, d_out, K, sigma, make_key(key), y_out,
+                               out_dt == DUST_BF16 ? 1 : 0, ld_out,
+                               static_cast<cudaStream_t>(stream));
+}
+
 dust_status dust_spsa_probe(const void* x, const void* W, const void* u, dust_dtype dt, int64_t N,
                             int32_t d_in, int32_t d_out, int32_t P, float eps,
                             dust_noise_key key, float* p, float* L_plus, float* L_minus,

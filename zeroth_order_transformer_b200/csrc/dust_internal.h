@@ -86,6 +86,9 @@ size_t spsa_workspace_bytes(int64_t N, int32_t d_in, int32_t d_out, int32_t P);
 dust_status spsa_probe_launch(const void* x, const void* W, const void* u, int64_t N, int32_t d_in,
                               int32_t d_out, int32_t P, float eps, NoiseKey key, float* p,
                               float* Lp, float* Lm, void* ws, cudaStream_t s);
+dust_status noisy_output_launch(const void* x, const void* W, int64_t N, int32_t d_in,
+                               int32_t d_out, int32_t K, float sigma, NoiseKey key, void* y_out,
+                               int out_bf16, int64_t ld_out, cudaStream_t s);
 dust_status spsa_estimate_launch(const float* p, int32_t P, int32_t P_total, int32_t d_in,
                                  int32_t d_out, NoiseKey key, float* G, int accumulate,
                                  cudaStream_t s);

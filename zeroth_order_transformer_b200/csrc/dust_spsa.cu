@@ -13,7 +13,9 @@
 //   spsa_dir_kernel     z_j for all probes, bf16, into the workspace [P, d_out_pad, d_in]
 //                       (rows d_out .. d_out_pad - 1 of each probe are zero).
 //   spsa_gemm_kernel    tcgen05 GEMM of x against W (residual mode: e = y - u and 1/2 |e|^2),
-//                       TMA-fed, accumulator in tensor memory, two CTAs per SM.
+//                       TMA-fed, accumulator in tensor memory, two CTAs per SM.  Its second
+//                       epilogue writes the perturbed outputs y + sigma a of every draw
+//                       (dust_noisy_linear_output).
 //   spsa_probe_gemm_kernel  the same against the stacked directions (probe mode: <e, v> and
 //                       |v|^2 per token and 256-row tile), persistent and warp-specialised with
 //                       two accumulators, so each tile's epilogue overlaps the next tile's
@@ -76,13 +78,23 @@ struct GemmArgs {
     CUtensorMap tmb;  // W [d_out, d_in] or Z [P d_out_pad, d_in], 64 x 256 boxes
     const __nv_bfloat16* u;
     float* e;         // [N, d_out] fp32: written in residual mode, read in probe mode
-    float* part_a;    // residual: [o_tiles, N] 1/2 |e|^2;  probe: [P o_tiles, N] <e, v>
-    float* part_b;    // probe: [P o_tiles, N] |v|^2
+    float* part_a;    // residual: [o_tiles, N] 1/2 |e|^2;  probe: [2 P o_tiles, N] <e, v>
+    float* part_b;    // probe: [2 P o_tiles, N] |v|^2
+    void* y_out;      // noisy-output mode: [K, N, ld_out] of y + sigma a, fp32 or bf16
     ErrorWord* ew;
-    int64_t N;
+    int64_t N, ld_out;
     int d_in, d_out, o_tiles, P, m_tiles;
+    int K, out_bf16;
+    float sigma;
+    NoiseKey key;
 };
 
+// Epilogues of the one-tile GEMM y = x W^T: kResidual writes e = y - u and 1/2 |e|^2 per
+// token and tile; kNoisyOut writes y + sigma a_t^(i) for every draw i (the perturbed layer
+// outputs, for callers that evaluate their own loss downstream).
+enum GemmMode { kResidual = 0, kNoisyOut = 1 };
+
+template <int kMode>
 __global__ void __launch_bounds__(kThreads, 2) spsa_gemm_kernel(const __grid_constant__ GemmArgs A) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -164,6 +176,41 @@ __global__ void __launch_bounds__(kThreads, 2) spsa_gemm_kernel(const __grid_con
         tmem_ld16(trow + c * 16, v);
         tmem_wait_ld();
         if (!valid) continue;
+        if (kMode == kNoisyOut) {
+            const uint32_t tg = A.key.token_offset + static_cast<uint32_t>(t);
+            const uint32_t q0 = static_cast<uint32_t>((o0 + c * 16) >> 2) + A.key.quad_offset;
+            for (int i = 0; i < A.K; ++i) {
+                const int64_t at = (static_cast<int64_t>(i) * A.N + t) * A.ld_out + o0 + c * 16;
+                float o[16];
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const F4 a = normal_quad(q0 + qq, tg, A.key.draw_offset + static_cast<uint32_t>(i),
+                                             A.key.layer, A.key);
+                    o[4 * qq] = fmaf(A.sigma, a.x, v[4 * qq]);
+                    o[4 * qq + 1] = fmaf(A.sigma, a.y, v[4 * qq + 1]);
+                    o[4 * qq + 2] = fmaf(A.sigma, a.z, v[4 * qq + 2]);
+                    o[4 * qq + 3] = fmaf(A.sigma, a.w, v[4 * qq + 3]);
+                }
+                if (A.out_bf16) {
+                    uint4 w[2];
+                    uint32_t* wb = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) {
+                        __nv_bfloat162 b2 = __floats2bfloat162_rn(o[2 * h], o[2 * h + 1]);
+                        wb[h] = *reinterpret_cast<uint32_t*>(&b2);
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(A.y_out) + at);
+                    dst[0] = w[0];
+                    dst[1] = w[1];
+                } else {
+                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(A.y_out) + at);
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq)
+                        dst[qq] = make_float4(o[4 * qq], o[4 * qq + 1], o[4 * qq + 2], o[4 * qq + 3]);
+                }
+            }
+            continue;
+        }
         const int64_t off = t * A.d_out + o0 + c * 16;
         const uint4* up = reinterpret_cast<const uint4*>(A.u + off);
         float uf[16];
@@ -192,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 2) spsa_gemm_kernel(const __grid_con
             sa = fmaf(e.w, e.w, sa);
         }
     }
-    if (valid) A.part_a[static_cast<int64_t>(o_tile) * A.N + t] = 0.5f * sa;
+    if (kMode == kResidual && valid) A.part_a[static_cast<int64_t>(o_tile) * A.N + t] = 0.5f * sa;
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
@@ -494,7 +541,7 @@ dust_status spsa_probe_launch(const void* x, const void* W, const void* u, int64
     Q.part_b = pvv;
     if (!make_tmap_bf16_2d(&Q.tmb, Z, static_cast<uint64_t>(P) * dpad, d_in, kBN, kBK))
         return DUST_ERR_CUDA;
-    if (cudaFuncSetAttribute(spsa_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(spsa_gemm_kernel<kResidual>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBytes)) != cudaSuccess ||
         cudaFuncSetAttribute(spsa_probe_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kPSmemBytes)) != cudaSuccess)
@@ -506,7 +553,7 @@ dust_status spsa_probe_launch(const void* x, const void* W, const void* u, int64
                       256, 0, s>>>(key, P, d_out, dpad, d_in, Z);
     prof_end(s, "spsa_directions");
     prof_begin(s);
-    spsa_gemm_kernel<<<static_cast<unsigned>(m_tiles * o_tiles), kThreads, kSmemBytes, s>>>(R);
+    spsa_gemm_kernel<kResidual><<<static_cast<unsigned>(m_tiles * o_tiles), kThreads, kSmemBytes, s>>>(R);
     prof_end(s, "spsa_residual_gemm");
     prof_begin(s);
     const int64_t probe_tiles = static_cast<int64_t>(m_tiles) * o_tiles * P;
@@ -521,6 +568,36 @@ dust_status spsa_probe_launch(const void* x, const void* W, const void* u, int64
     spsa_finish_kernel<<<static_cast<unsigned>((P + 127) / 128), 128, 0, s>>>(sums, P, o_tiles,
                                                                             n_chunks, eps, p, Lp, Lm);
     prof_end(s, "spsa_reduce");
+    return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
+}
+
+dust_status noisy_output_launch(const void* x, const void* W, int64_t N, int32_t d_in,
+                               int32_t d_out, int32_t K, float sigma, NoiseKey key, void* y_out,
+                               int out_bf16, int64_t ld_out, cudaStream_t s) {
+    GemmArgs G{};
+    G.y_out = y_out;
+    G.ew = device_error_word();
+    G.N = N;
+    G.ld_out = ld_out;
+    G.d_in = d_in;
+    G.d_out = d_out;
+    G.o_tiles = pad256(d_out) / kBN;
+    G.P = 1;
+    G.m_tiles = static_cast<int>((N + kBM - 1) / kBM);
+    G.K = K;
+    G.out_bf16 = out_bf16;
+    G.sigma = sigma;
+    G.key = key;
+    if (!make_tmap_bf16_2d(&G.tmx, x, static_cast<uint64_t>(N), d_in, kBM, kBK) ||
+        !make_tmap_bf16_2d(&G.tmb, W, static_cast<uint64_t>(d_out), d_in, kBN, kBK))
+        return DUST_ERR_CUDA;
+    if (cudaFuncSetAttribute(spsa_gemm_kernel<kNoisyOut>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+        return DUST_ERR_CUDA;
+    prof_begin(s);
+    spsa_gemm_kernel<kNoisyOut><<<static_cast<unsigned>(G.m_tiles * G.o_tiles), kThreads,
+                                  kSmemBytes, s>>>(G);
+    prof_end(s, "noisy_linear_output");
     return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
 }
 
