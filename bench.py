@@ -391,14 +391,27 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         host_out = [torch.empty(G.shape, dtype=G.dtype, pin_memory=True) for G in GWs]
         d2h = sum(G.numel() * G.element_size() for G in GWs)
 
-        def e2e_step():
-            for (s, hx, hW, hu), (_, dx, dW, du) in zip(host_in, dev_in):
-                dx.copy_(hx, non_blocking=True)
-                dW.copy_(hW, non_blocking=True)
-                du.copy_(hu, non_blocking=True)
-            out = step(dev_in)
-            for G, hG in zip(out, host_out):
-                hG.copy_(G, non_blocking=True)
+        if len(layers) == 1:
+            # one layer: the public host-input call, upload pipelined with the compute
+            s1 = layers[0][0]
+            host_layer = dust.DustLayer(wl.N, s1.d_in, s1.d_out, wl.K, tdt, dev)
+            red = (lambda G: dist.all_reduce(G)) if world > 1 else None
+
+            def e2e_step():
+                _, hx, hW, hu = host_in[0]
+                host_layer.estimate_from_host(
+                    hx, hW, hu, data.cu_seqlens, wl.sigma, gamma,
+                    dust.NoiseKey(wl.seed, s1.layer_id, 0, rank * wl.N), host_out[0],
+                    chunks=4, reduce=red)
+        else:
+            def e2e_step():
+                for (s, hx, hW, hu), (_, dx, dW, du) in zip(host_in, dev_in):
+                    dx.copy_(hx, non_blocking=True)
+                    dW.copy_(hW, non_blocking=True)
+                    du.copy_(hu, non_blocking=True)
+                out = step(dev_in)
+                for G, hG in zip(out, host_out):
+                    hG.copy_(G, non_blocking=True)
 
         for _ in range(max(1, args.warmup // 2)):
             flush.zero_()

@@ -363,3 +363,26 @@ def test_chain_bf16_ragged_packed():
     assert _dev.rel_fro(got["G_W"], ref["G_W"]) <= _dev.GW_FRO
     # the credit sums to zero over draws at every token (centring), to fp32 rounding
     assert np.abs(got["r"].sum(axis=0)).max() <= 1e-4 * np.abs(got["r"]).max()
+
+
+def test_estimate_from_host_pipelined_matches_oracle():
+    """DustLayer.estimate_from_host: pinned host inputs uploaded in runs of whole sequences
+    while earlier runs are estimated; the noise keeps the whole batch's token indices."""
+    import torch
+    N, d_in, d_out, K, sigma, gamma = 1000, 128, 256, 8, 1e-3, 0.9
+    L = workloads.custom_layer(31, N, d_in, d_out, "bf16", 0.02)
+    cu = np.array([0, 240, 500, 764, 1000], dtype=np.int32)
+    key = z.NoiseKey(0x5EED00C1, layer_id=4, token_offset=77)
+
+    def pinned(store):
+        return torch.from_numpy(np.ascontiguousarray(store).view(np.int16)).view(
+            torch.bfloat16).pin_memory()
+
+    layer = z.DustLayer(N, d_in, d_out, K, torch.bfloat16, "cuda")
+    G = layer.estimate_from_host(pinned(L.x_store), pinned(L.W_store), pinned(L.u_store), cu,
+                                 sigma, gamma, key, chunks=3)
+    ref = oracle.dust_layer(L.x_f64, L.W_f64, L.u_f64, K, sigma, gamma, cu, key.seed, 4,
+                            token_offset=77)
+    _dev.assert_fp32_close(_dev.host(layer.dloss), ref["loss"] - ref["clean"], "dloss")
+    assert _dev.rel_fro(_dev.host(layer.r), ref["r"]) <= 1e-4
+    assert _dev.rel_fro(G.numpy(), ref["G_W"]) <= _dev.GW_FRO

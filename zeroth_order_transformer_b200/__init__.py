@@ -44,7 +44,7 @@ EXPORTED_SYMBOLS = (
     "dust_credit_grouped", "dust_weight_grad_grouped", "dust_workspace_size_grouped",
     "dust_optimizer_step", "dust_weight_grad_step", "dust_noisy_logits_ce",
     "dust_debug_normal_sum", "dust_attn_reward", "dust_discounted_credit",
-    "dust_spsa_probe", "dust_spsa_estimate",
+    "dust_spsa_probe", "dust_spsa_estimate", "dust_noisy_linear_output",
 )
 
 DUST_OPT_SGD_MOMENTUM = 1
@@ -151,6 +151,9 @@ def lib() -> ctypes.CDLL:
         L.dust_discounted_credit.argtypes = [vp, i64, i32, i64, vp, i32, f32, vp, i64, vp, sz,
                                              vp]
         L.dust_discounted_credit.restype = ctypes.c_int
+        L.dust_noisy_linear_output.argtypes = [vp, vp, ctypes.c_int, i64, i32, i32, i32, f32,
+                                               dust_noise_key, vp, ctypes.c_int, i64, vp]
+        L.dust_noisy_linear_output.restype = ctypes.c_int
         L.dust_spsa_probe.argtypes = [vp, vp, vp, ctypes.c_int, i64, i32, i32, i32, f32,
                                       dust_noise_key, vp, vp, vp, vp, sz, vp]
         L.dust_spsa_probe.restype = ctypes.c_int
@@ -206,6 +209,16 @@ def _cuda(t, name: str):
     return t
 
 
+def _cuda_rows(t, name: str):
+    """A CUDA matrix whose rows are contiguous; rows may be further apart (the row stride is
+    passed as the leading dimension)."""
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be a matrix with contiguous rows")
+    return t
+
+
 def _stream(device, stream) -> int:
     torch = _torch()
     if stream is None:
@@ -238,7 +251,7 @@ def dust_noisy_linear_fwd(x, W, u, K: int, sigma: float, key: NoiseKey, dloss=No
     dt = _dtype_code(x)
     if dloss is None:
         dloss = torch.empty((K, N), dtype=torch.float32, device=x.device)
-    _cuda(dloss, "dloss")
+    _cuda_rows(dloss, "dloss")
     ws, nb = _workspace(workspace, dust_workspace_size(DUST_OP_NOISY_LINEAR_FWD, dt, N, d_in,
                                                        d_out, K), x.device)
     st = lib().dust_noisy_linear_fwd(x.data_ptr(), W.data_ptr(), u.data_ptr(), dt, N, d_in,
@@ -274,13 +287,13 @@ def dust_noisy_logits_ce(z, y, v0: int, S: int, K: int, sigma: float, key: Noise
 def dust_credit(loss, cu_seqlens, gamma: float, r=None, workspace=None, stream=None):
     """Credit r[K, N] from losses [K, N] and int32 cu_seqlens [n_seq + 1] (device)."""
     torch = _torch()
-    _cuda(loss, "loss"), _cuda(cu_seqlens, "cu_seqlens")
+    _cuda_rows(loss, "loss"), _cuda(cu_seqlens, "cu_seqlens")
     if loss.dtype != torch.float32 or cu_seqlens.dtype != torch.int32:
         raise TypeError("loss must be float32 and cu_seqlens int32")
     K, N = loss.shape
     if r is None:
         r = torch.empty((K, N), dtype=torch.float32, device=loss.device)
-    _cuda(r, "r")
+    _cuda_rows(r, "r")
     ws, nb = _workspace(workspace, dust_workspace_size(DUST_OP_CREDIT, DUST_F32, N, 0, 0, K),
                         loss.device)
     st = lib().dust_credit(loss.data_ptr(), loss.stride(0), K, N, cu_seqlens.data_ptr(),
@@ -330,6 +343,25 @@ def dust_discounted_credit(c, cu_seqlens, gamma: float, r=None, workspace=None, 
                                       nb, _stream(c.device, stream))
     _check(st, "dust_discounted_credit")
     return r
+
+
+def dust_noisy_linear_output(x, W, K: int, sigma: float, key: NoiseKey, y_out=None,
+                             out_dtype=None, stream=None):
+    """The perturbed outputs y_out[K, N, d_out] = W x_t + sigma a_t^(i) (fp32 by default, or
+    out_dtype=torch.bfloat16), with the noise of dust_noisy_linear_fwd for the same key."""
+    torch = _torch()
+    _cuda(x, "x"), _cuda(W, "W")
+    N, d_in = x.shape
+    d_out = W.shape[0]
+    if y_out is None:
+        y_out = torch.empty((K, N, d_out), dtype=out_dtype or torch.float32, device=x.device)
+    _cuda(y_out, "y_out")
+    st = lib().dust_noisy_linear_output(x.data_ptr(), W.data_ptr(), _dtype_code(x), N, d_in,
+                                        d_out, K, float(sigma), key.c(), y_out.data_ptr(),
+                                        _dtype_code(y_out), y_out.stride(1),
+                                        _stream(x.device, stream))
+    _check(st, "dust_noisy_linear_output")
+    return y_out
 
 
 def dust_spsa_probe(x, W, u, P: int, eps: float, key: NoiseKey, p=None, losses: bool = False,
@@ -391,7 +423,7 @@ def dust_weight_grad(r, x, d_out: int, K_total: int, sigma: float, key: NoiseKey
                      ) -> Tuple[object, Optional[object]]:
     """G_W[d_out, d_in] (fp32) and, if g_out is a tensor or True, g[N, d_out] (fp32)."""
     torch = _torch()
-    _cuda(r, "r"), _cuda(x, "x")
+    _cuda_rows(r, "r"), _cuda(x, "x")
     K_chunk, N = r.shape
     d_in = x.shape[1]
     dt = _dtype_code(x)
@@ -582,3 +614,66 @@ class DustLayer:
         dust_weight_grad(self.r, x, self.d_out, self.K, sigma, key, self.G_W, False, None,
                          self.ws, stream)
         return self.G_W
+
+    def estimate_from_host(self, hx, hW, hu, cu_seqlens, sigma: float, gamma: float,
+                           key: NoiseKey, G_host=None, chunks: int = 4, reduce=None):
+        """The estimate from inputs in pinned host memory, with the upload overlapped: the
+        tokens are cut into ``chunks`` runs of whole sequences; each run is copied on a copy
+        stream while the previous one goes through the forward, the credit and the weight
+        estimate (accumulated over the runs, token offsets keeping the noise of the whole
+        batch).  ``reduce`` (optional) is applied to the device G_W before it is copied back
+        (for instance the all-reduce over data-parallel ranks).  G_W comes back into
+        ``G_host`` (pinned, allocated if None).  Synchronises."""
+        import numpy as np
+        torch = _torch()
+        dev = self.ws.device
+        cu = np.asarray(cu_seqlens, dtype=np.int64)
+        N = int(cu[-1])
+        if N != self.N:
+            raise ValueError("cu_seqlens does not cover the layer's N tokens")
+        if not hasattr(self, "_x"):
+            self._x = torch.empty((N, self.d_in), dtype=hx.dtype, device=dev)
+            self._u = torch.empty((N, self.d_out), dtype=hu.dtype, device=dev)
+            self._W = torch.empty((self.d_out, self.d_in), dtype=hW.dtype, device=dev)
+            self._copy = torch.cuda.Stream(device=dev)
+        # cuts at sequence ends that keep the per-run views 16-byte aligned
+        ends = cu[(cu % 4 == 0) & (cu > 0) & (cu < N)]
+        cuts = [0]
+        for c in range(1, chunks):
+            if ends.size == 0:
+                break
+            e = int(ends[int(np.argmin(np.abs(ends - N * c / chunks)))])
+            if e > cuts[-1]:
+                cuts.append(e)
+        cuts.append(N)
+        # every run's local cu_seqlens, uploaded once
+        locs = [(cu[(cu >= a) & (cu <= b)] - a).astype(np.int32) for a, b in zip(cuts[:-1], cuts[1:])]
+        cu_all = torch.from_numpy(np.concatenate(locs)).pin_memory().to(dev, non_blocking=True)
+        offs = np.cumsum([0] + [len(l) for l in locs])
+        comp = torch.cuda.current_stream(dev)
+        ready = []
+        self._copy.wait_stream(comp)  # the uploads start after the work already queued
+        with torch.cuda.stream(self._copy):
+            self._W.copy_(hW, non_blocking=True)
+            for a, b in zip(cuts[:-1], cuts[1:]):
+                self._x[a:b].copy_(hx[a:b], non_blocking=True)
+                self._u[a:b].copy_(hu[a:b], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(self._copy)
+                ready.append(ev)
+        for n, ((a, b), ev) in enumerate(zip(zip(cuts[:-1], cuts[1:]), ready)):
+            comp.wait_event(ev)
+            cu_d = cu_all[int(offs[n]):int(offs[n + 1])]
+            k = key._replace(token_offset=key.token_offset + a)
+            x, u = self._x[a:b], self._u[a:b]
+            dl, r = self.dloss[:, a:b], self.r[:, a:b]
+            dust_noisy_linear_fwd(x, self._W, u, self.K, sigma, k, dl, self.ws)
+            dust_credit(dl, cu_d, gamma, r, self.ws)
+            dust_weight_grad(r, x, self.d_out, self.K, sigma, k, self.G_W, n > 0, None, self.ws)
+        if reduce is not None:
+            reduce(self.G_W)
+        if G_host is None:
+            G_host = torch.empty(self.G_W.shape, dtype=self.G_W.dtype, pin_memory=True)
+        G_host.copy_(self.G_W, non_blocking=True)
+        torch.cuda.current_stream(dev).synchronize()
+        return G_host
