@@ -46,7 +46,7 @@ struct GhatTable {
 };
 
 template <int kMax>
-__global__ void __launch_bounds__(kGThreads) ghat_kernel(const __grid_constant__ GhatTable<kMax> T) {
+__global__ void __launch_bounds__(kGThreads, 8) ghat_kernel(const __grid_constant__ GhatTable<kMax> T) {
     int l = 0;
     for (int64_t u = blockIdx.x; u < T.total_units; u += gridDim.x) {
         while (l + 1 < T.n_layers && u >= T.layer[l + 1].unit_begin) ++l;
@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(kGThreads) ghat_kernel(const __grid_constant__
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
         const float* rt = L.r + t;
         // unrolled so that independent Philox chains of consecutive draws interleave
-#pragma unroll 2
+#pragma unroll 4
         for (int i = 0; i < T.K; ++i) {
             const float ri = __ldg(rt + static_cast<int64_t>(i) * L.ld_r);
             const Polar4 z = normal_quad_polar(static_cast<uint32_t>(q) + T.key.quad_offset, tg,
