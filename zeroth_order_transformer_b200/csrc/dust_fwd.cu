@@ -28,7 +28,7 @@ constexpr int kBM = 128;  // tokens per tile
 constexpr int kBN = 256;  // channels per tile
 constexpr int kBK = 64;   // d_in per pipeline stage (128 bytes of bf16: one swizzle row)
 constexpr int kStages = 2;
-constexpr int kThreads = 384;  // 3 groups of 4 warps
+constexpr int kThreads = 512;  // 4 groups of 4 warps
 constexpr int kGroups = kThreads / 128;
 constexpr uint32_t kABytes = kBM * kBK * 2;
 constexpr uint32_t kBBytes = kBN * kBK * 2;
@@ -224,19 +224,25 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_bf16_kernel(const __grid_cons
             const int hf = unit & 1;
             const uint32_t di = T.key.draw_offset + static_cast<uint32_t>(i);
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            // s_e in 8-column pieces (two quads); a 16-channel chunk is two pieces
             const int c_end = hf ? nchunks : half_chunks;
             for (int c = hf ? half_chunks : 0; c < c_end; ++c) {
-                float se[16];
-                tmem_ld16(trow + c * 16, se);
-                tmem_wait_ld();
 #pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    const Polar4 z = normal_quad_polar(qbase + c * 4 + qq, tg, di, L.layer_id, T.key);
-                    const float l0 = fmaf(z.s0, se[4 * qq + 1], z.c0 * se[4 * qq + 0]);
-                    const float l1 = fmaf(z.s1, se[4 * qq + 3], z.c1 * se[4 * qq + 2]);
-                    acc[qq] = fmaf(-z.q0, l0, acc[qq]);
-                    acc[qq] = fmaf(-z.q1, l1, acc[qq]);
-                    acc[qq] = fmaf(h, z.y0 + z.y1, acc[qq]);
+                for (int piece = 0; piece < 2; ++piece) {
+                    float se[8];
+                    tmem_ld8(trow + c * 16 + piece * 8, se);
+                    tmem_wait_ld8(se);
+#pragma unroll
+                    for (int qq = 0; qq < 2; ++qq) {
+                        const Polar4 z = normal_quad_polar(qbase + c * 4 + piece * 2 + qq, tg, di,
+                                                           L.layer_id, T.key);
+                        const float l0 = fmaf(z.s0, se[4 * qq + 1], z.c0 * se[4 * qq + 0]);
+                        const float l1 = fmaf(z.s1, se[4 * qq + 3], z.c1 * se[4 * qq + 2]);
+                        float& a = acc[2 * piece + qq];
+                        a = fmaf(-z.q0, l0, a);
+                        a = fmaf(-z.q1, l1, a);
+                        a = fmaf(h, z.y0 + z.y1, a);
+                    }
                 }
             }
             if (valid)
