@@ -9,7 +9,7 @@
 //   X^(i) = sum_{v in slab} exp(z_v - zmax) (exp(sigma a^(i)[v]) - 1).
 // Three kernels:
 //   ce_stats_kernel    per token: zmax and E over the vocabulary (online max / rescaled sum).
-//   ce_noise_kernel    per (128-channel chunk, 128 tokens): w = exp(z - zmax) staged in shared
+//   ce_noise_kernel    per (128-channel chunk, 64 tokens): w = exp(z - zmax) staged in shared
 //                      memory, then per draw the normals of the chunk are regenerated and
 //                      sum w (exp(sigma a) - 1) goes into a per-chunk partial.
 //   ce_finish_kernel   per (draw, token): log1p(sum of partials / E) minus the target's term.
@@ -25,7 +25,7 @@ namespace dust {
 namespace {
 
 constexpr int kChunk = 128;   // slab channels per noise block
-constexpr int kTokB = 128;    // tokens per noise block
+constexpr int kTokB = 64;     // tokens per noise block (33 KB of staged weights: six blocks per SM)
 constexpr int kNoiseThreads = 256;
 constexpr int kStride = kTokB + 1;  // padded row of the staged weights (conflict-free)
 
