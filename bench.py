@@ -53,8 +53,6 @@ MEASURED_TRAFFIC = {
                                                        "profiles/ncu_full_gpt2s_mlp_win_768x3072.md"),
     ("ghat_reduce_draws", "gpt2s-mlp-win-768x3072"): (0.54e6 + 0.52e6,
                                                      "profiles/ncu_full_gpt2s_mlp_win_768x3072.md"),
-    ("lmhead_ce_noise", "head-4096-slab1024"): (34.64e6 + 75.64e6,
-                                                "profiles/ncu_full_lmhead_head-4096-slab1024.md"),
 }
 HEAD_METRIC = "Dust LM-head estimator tokens*draws/s"
 ATTN_METRIC = "Dust attention-reward estimator tokens*draws/s"
