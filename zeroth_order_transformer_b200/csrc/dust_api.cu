@@ -46,15 +46,14 @@ __global__ void __launch_bounds__(256) normal_sum_kernel(const __grid_constant__
     for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < n;
          g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const uint32_t t = key.token_offset + static_cast<uint32_t>(g);
-        float acc0 = 0.f, acc1 = 0.f;
+        F2 acc{0.f, 0.f};  // lanes: the quad's two polar pairs
 #pragma unroll 2
         for (int32_t j = 0; j < n_quads; ++j) {
-            const Polar4 z = normal_quad_polar(key.quad_offset + static_cast<uint32_t>(j), t,
-                                               key.draw_offset, key.layer, key);
-            acc0 = fmaf(z.q0, z.c0 + z.s0, acc0);
-            acc1 = fmaf(z.q1, z.c1 + z.s1, acc1);
+            const PolarPairs z = normal_quad_pairs(key.quad_offset + static_cast<uint32_t>(j), t,
+                                                   key.draw_offset, key.layer, key);
+            acc = fma2(z.nq, add2(z.c, z.s), acc);
         }
-        out[g] = -kKappa * (acc0 + acc1);
+        out[g] = kKappa * (acc.x + acc.y);
     }
 }
 

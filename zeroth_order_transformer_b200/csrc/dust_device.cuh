@@ -65,10 +65,10 @@ __device__ __forceinline__ U4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c
     return U4{c0, c1, c2, c3};
 }
 
-// u(w) = (2 (w >> 9) + 1) 2^-24, exact: 1 + m 2^-23 has the 23 bits m = w >> 9 as mantissa,
-// and subtracting 1 - 2^-24 leaves (2m + 1) 2^-24, which fits in 24 bits.
-__device__ __forceinline__ float uniform_from_word(uint32_t w) {
-    return __uint_as_float(0x3f800000u | (w >> 9)) - 0.99999994f;
+// The float with the given sign and exponent bits and the word's top 23 bits m = w >> 9 as
+// mantissa (written as an add: the two bit fields do not overlap).
+__device__ __forceinline__ float mantissa_float(uint32_t exp_bits, uint32_t w) {
+    return __uint_as_float(exp_bits + (w >> 9));
 }
 
 // Hardware approximations (PTX .approx with flush-to-zero; every input here is a normal
@@ -113,48 +113,97 @@ constexpr uint32_t kNearOneWord = 0xFFC00000u;
 // rho = sqrt(-2 ln u) = kKappa sqrt(-log2 u), kKappa = sqrt(2 ln 2).
 constexpr float kKappa = 1.1774100225154747f;
 
-// Box-Muller angle shifted by -pi, from the word in one FMA: with m = w >> 9 the float
-// f = 2 + m 2^-22 (exponent 1, mantissa m) gives 2 pi u(w) - pi = pi f - 3 pi + 2 pi 2^-24,
-// which lies in [-pi, pi).  (Largest error over all m: 3.5e-7 rad.)
-__device__ __forceinline__ float angle_from_word(uint32_t w) {
-    return fmaf(3.14159265358979323846f, __uint_as_float(0x40000000u | (w >> 9)),
-                -9.4247775872730683f);  // -3 pi + 2 pi 2^-24
-}
-
 struct F4 {
     float x, y, z, w;
 };
 
-// Box-Muller on one Philox block in scaled polar form: pair p (words 2p, 2p+1) has
-// y_p = -log2 u(w_2p) >= 0, q_p = sqrt(y_p) (so the radius is rho_p = kKappa q_p and
-// rho_p^2 = 2 ln 2 y_p) and angle 2 pi u(w_2p+1) - pi, where the hardware sine and cosine keep
-// their absolute error bound.  The -pi shift flips both signs, so
-//     z_2p = -kKappa q_p cos_p,   z_2p+1 = -kKappa q_p sin_p.
-// Consumers fold kKappa (and 2 ln 2) into their own coefficients.
+// Two-wide fp32 arithmetic: sm_100's packed f32x2 instructions do two independent,
+// correctly rounded operations (the same results as two scalar ones) in one issue slot.
+struct F2 {
+    float x, y;
+};
+__device__ __forceinline__ F2 fma2(F2 a, F2 b, F2 c) {
+    F2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ F2 mul2(F2 a, F2 b) {
+    F2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ F2 add2(F2 a, F2 b) {
+    F2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// Box-Muller on one Philox block in scaled polar form, as packed pairs: pair p (words 2p,
+// 2p+1) has the radius word's L_p = log2 u(w_2p) <= 0, so y_p = -L_p and q_p = sqrt(y_p) (the
+// radius is rho_p = kKappa q_p, rho_p^2 = 2 ln 2 y_p), and the angle 2 pi u(w_2p+1) - pi, where
+// the hardware sine and cosine keep their absolute error bound.  The -pi shift flips both
+// signs, so
+//     z_2p = -kKappa q_p cos_p = kKappa nq_p cos_p,   z_2p+1 = kKappa nq_p sin_p,
+// with nq_p = -q_p = L_p rsqrt(-L_p).  Lane x of each pair is pair 0 (channels 4q, 4q+1),
+// lane y pair 1 (channels 4q+2, 4q+3).  Consumers fold kKappa (and 2 ln 2) into their own
+// coefficients.
+struct PolarPairs {
+    F2 L;   // log2 u of the radius words
+    F2 nq;  // -sqrt(-L)
+    F2 c;   // cosines of the two angles
+    F2 s;   // sines
+};
+
+__device__ __forceinline__ PolarPairs box_muller_pairs(const U4& w) {
+    // u(w) = (2m + 1) 2^-24 with m = w >> 9, exact: 1 + m 2^-23 (exponent 0, mantissa m) minus
+    // 1 - 2^-24 leaves (2m + 1) 2^-24, which fits in 24 bits; both radius words at once
+    const F2 u = add2(F2{mantissa_float(0x3f800000u, w.x), mantissa_float(0x3f800000u, w.z)},
+                      F2{-0.99999994f, -0.99999994f});
+    PolarPairs p;
+    p.L.x = lg2_approx(u.x);
+    p.L.y = lg2_approx(u.y);
+    if (max(w.x, w.z) >= kNearOneWord) {  // rare: about 1 block in 500
+        p.L.x = -neg_lg2_near_one(u.x, -p.L.x);
+        p.L.y = -neg_lg2_near_one(u.y, -p.L.y);
+    }
+    p.nq = mul2(p.L, F2{rsqrt_approx(-p.L.x), rsqrt_approx(-p.L.y)});
+    // Box-Muller angle shifted by -pi, one FMA per angle word: the float f = 2 + m 2^-22
+    // (exponent 1, mantissa m) gives 2 pi u(w) - pi = pi f - 3 pi + 2 pi 2^-24, which lies in
+    // [-pi, pi) (largest error over all m: 3.5e-7 rad)
+    const F2 a = fma2(F2{3.14159265358979323846f, 3.14159265358979323846f},
+                      F2{mantissa_float(0x40000000u, w.y), mantissa_float(0x40000000u, w.w)},
+                      F2{-9.4247775872730683f, -9.4247775872730683f});  // -3 pi + 2 pi 2^-24
+    p.c = F2{cos_approx(a.x), cos_approx(a.y)};
+    p.s = F2{sin_approx(a.x), sin_approx(a.y)};
+    return p;
+}
+
+__device__ __forceinline__ PolarPairs normal_quad_pairs(uint32_t q, uint32_t t, uint32_t i,
+                                                        uint32_t layer, const NoiseKey& key) {
+    return box_muller_pairs(philox4x32_10(q, t, i, layer, key));
+}
+
+// The same block with scalar fields: y_p = -L_p >= 0 and q_p = sqrt(y_p).
 struct Polar4 {
     float y0, q0, c0, s0;  // pair 0: channels 4q, 4q+1
     float y1, q1, c1, s1;  // pair 1: channels 4q+2, 4q+3
 };
 
 __device__ __forceinline__ Polar4 box_muller_polar(const U4& w) {
-    const float u0 = uniform_from_word(w.x);
-    const float u2 = uniform_from_word(w.z);
-    Polar4 p;
-    p.y0 = -lg2_approx(u0);
-    p.y1 = -lg2_approx(u2);
-    if (max(w.x, w.z) >= kNearOneWord) {  // rare: about 1 block in 500
-        p.y0 = neg_lg2_near_one(u0, p.y0);
-        p.y1 = neg_lg2_near_one(u2, p.y1);
-    }
-    p.q0 = p.y0 * rsqrt_approx(p.y0);
-    p.q1 = p.y1 * rsqrt_approx(p.y1);
-    const float a1 = angle_from_word(w.y);
-    const float a3 = angle_from_word(w.w);
-    p.c0 = cos_approx(a1);
-    p.s0 = sin_approx(a1);
-    p.c1 = cos_approx(a3);
-    p.s1 = sin_approx(a3);
-    return p;
+    const PolarPairs p = box_muller_pairs(w);
+    return Polar4{-p.L.x, -p.nq.x, p.c.x, p.s.x, -p.L.y, -p.nq.y, p.c.y, p.s.y};
 }
 
 __device__ __forceinline__ Polar4 normal_quad_polar(uint32_t q, uint32_t t, uint32_t i,

@@ -203,7 +203,18 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_bf16_kernel(const __grid_cons
 #pragma unroll
                 for (int j = 0; j < 16; ++j) v[j] = 0.f;
             }
-            tmem_st16(trow + c * 16, v);
+            // stored per channel quad as (e0, e2, e1, e3): phase 2 then loads the pairs
+            // (e0, e2) and (e1, e3) that go with the cosines and the sines of the quad's two
+            // polar pairs
+            float w[16];
+#pragma unroll
+            for (int j = 0; j < 16; j += 4) {
+                w[j] = v[j];
+                w[j + 1] = v[j + 2];
+                w[j + 2] = v[j + 1];
+                w[j + 3] = v[j + 3];
+            }
+            tmem_st16(trow + c * 16, w);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -212,18 +223,19 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_bf16_kernel(const __grid_cons
 
         // Phase 2: this CTA's units of the tile, dealt round-robin to the warp groups.  A unit
         // is (draw, half of the tile's channels): regenerate the noise and sum the loss change
-        // over the half's channels.  In polar form a pair (z, z') = -kKappa q (cos, sin)
+        // over the half's channels.  In polar form a pair (z, z') = kKappa nq (cos, sin)
         // contributes sigma (z e + z' e') + sigma^2 / 2 (z^2 + z'^2)
-        //   = -q (cos s_e + sin s_e') + h y,   h = sigma^2 ln 2,  y = q^2 = -log2 u.
+        //   = nq (cos s_e + sin s_e') - h L,   h = sigma^2 ln 2,  L = log2 u = -nq^2;
+        // the quad's two pairs are the two lanes of packed f32x2 operations.
         const uint32_t tg = T.key.token_offset + static_cast<uint32_t>(t);
         const uint32_t qbase = static_cast<uint32_t>(n0 >> 2) + T.key.quad_offset;
-        const float h = T.h_lg2;
+        const F2 mh{-T.h_lg2, -T.h_lg2};
         const int half_chunks = (nchunks + 1) / 2;
         for (int unit = u_begin + grp; unit < u_end; unit += kGroups) {
             const int i = unit >> 1;
             const int hf = unit & 1;
             const uint32_t di = T.key.draw_offset + static_cast<uint32_t>(i);
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            F2 acc[2] = {{0.f, 0.f}, {0.f, 0.f}};
             // s_e in 8-column pieces (two quads); a 16-channel chunk is two pieces
             const int c_end = hf ? nchunks : half_chunks;
             for (int c = hf ? half_chunks : 0; c < c_end; ++c) {
@@ -234,20 +246,18 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_bf16_kernel(const __grid_cons
                     tmem_wait_ld8(se);
 #pragma unroll
                     for (int qq = 0; qq < 2; ++qq) {
-                        const Polar4 z = normal_quad_polar(qbase + c * 4 + piece * 2 + qq, tg, di,
-                                                           L.layer_id, T.key);
-                        const float l0 = fmaf(z.s0, se[4 * qq + 1], z.c0 * se[4 * qq + 0]);
-                        const float l1 = fmaf(z.s1, se[4 * qq + 3], z.c1 * se[4 * qq + 2]);
-                        float& a = acc[2 * piece + qq];
-                        a = fmaf(-z.q0, l0, a);
-                        a = fmaf(-z.q1, l1, a);
-                        a = fmaf(h, z.y0 + z.y1, a);
+                        const PolarPairs z = normal_quad_pairs(qbase + c * 4 + piece * 2 + qq, tg,
+                                                               di, L.layer_id, T.key);
+                        const F2 lc = fma2(z.s, F2{se[4 * qq + 2], se[4 * qq + 3]},
+                                           mul2(z.c, F2{se[4 * qq + 0], se[4 * qq + 1]}));
+                        acc[qq] = fma2(z.nq, lc, acc[qq]);
+                        acc[qq] = fma2(mh, z.L, acc[qq]);
                     }
                 }
             }
             if (valid)
                 L.partial[((static_cast<int64_t>(n_tile) * 2 + hf) * K + i) * N + t] =
-                    (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                    (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
         }
 
         // Done with the accumulator.  Count the finished units of the token block; the CTA

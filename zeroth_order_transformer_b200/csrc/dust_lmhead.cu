@@ -156,17 +156,14 @@ __global__ void __launch_bounds__(256) ce_stats_vec_kernel(const CeArgs a) {
     }
 }
 
-// exp(x) - 1: degree-5 Taylor series for |x| <= 0.1, else the library expm1f.
-template <bool kSeries>
-__device__ __forceinline__ float em1(float x) {
-    if (kSeries) {
-        float p = fmaf(x, 1.f / 120.f, 1.f / 24.f);
-        p = fmaf(x, p, 1.f / 6.f);
-        p = fmaf(x, p, 0.5f);
-        p = fmaf(x, p, 1.f);
-        return x * p;
-    }
-    return expm1f(x);
+// exp(x) - 1 for |x| <= 0.1: the degree-5 Taylor series, on two lanes (packed f32x2
+// operations); larger noise scales call expm1f per element.
+__device__ __forceinline__ F2 em1_series2(F2 x) {
+    F2 p = fma2(x, F2{1.f / 120.f, 1.f / 120.f}, F2{1.f / 24.f, 1.f / 24.f});
+    p = fma2(x, p, F2{1.f / 6.f, 1.f / 6.f});
+    p = fma2(x, p, F2{0.5f, 0.5f});
+    p = fma2(x, p, F2{1.f, 1.f});
+    return mul2(x, p);
 }
 
 template <typename T, bool kSeries>
@@ -194,20 +191,29 @@ __global__ void __launch_bounds__(kNoiseThreads) ce_noise_kernel(const CeArgs a)
     const uint32_t tg = a.key.token_offset + static_cast<uint32_t>(t);
     const uint32_t q0 = static_cast<uint32_t>(c0 >> 2);
     const int nq = nch >> 2;
-    const float sk = -kKappa * a.sigma;
+    const float sk = kKappa * a.sigma;
     for (int i = half; i < a.K; i += kNoiseThreads / kTokB) {
         const uint32_t di = a.key.draw_offset + static_cast<uint32_t>(i);
-        float acc0 = 0.f, acc1 = 0.f;
+        // lanes: the quad's two polar pairs; accc takes the cosine channels (4q, 4q+2),
+        // accs the sine channels (4q+1, 4q+3)
+        F2 accc{0.f, 0.f}, accs{0.f, 0.f};
         for (int q = 0; q < nq; ++q) {
-            // sigma a = -(kKappa sigma q) (cos, sin) per pair
-            const Polar4 z = normal_quad_polar(q0 + q, tg, di, a.key.layer, a.key);
+            // sigma a = (kKappa sigma nq) (cos, sin) per pair
+            const PolarPairs z = normal_quad_pairs(q0 + q, tg, di, a.key.layer, a.key);
             const float* wq = w + (4 * q) * kStride + lt;
-            const float r0 = sk * z.q0, r1 = sk * z.q1;
-            acc0 = fmaf(wq[0], em1<kSeries>(r0 * z.c0), acc0);
-            acc1 = fmaf(wq[kStride], em1<kSeries>(r0 * z.s0), acc1);
-            acc0 = fmaf(wq[2 * kStride], em1<kSeries>(r1 * z.c1), acc0);
-            acc1 = fmaf(wq[3 * kStride], em1<kSeries>(r1 * z.s1), acc1);
+            const F2 r = mul2(F2{sk, sk}, z.nq);
+            const F2 xc = mul2(r, z.c), xs = mul2(r, z.s);
+            if (kSeries) {
+                accc = fma2(F2{wq[0], wq[2 * kStride]}, em1_series2(xc), accc);
+                accs = fma2(F2{wq[kStride], wq[3 * kStride]}, em1_series2(xs), accs);
+            } else {
+                accc.x = fmaf(wq[0], expm1f(xc.x), accc.x);
+                accc.y = fmaf(wq[2 * kStride], expm1f(xc.y), accc.y);
+                accs.x = fmaf(wq[kStride], expm1f(xs.x), accs.x);
+                accs.y = fmaf(wq[3 * kStride], expm1f(xs.y), accs.y);
+            }
         }
+        const float acc0 = accc.x + accc.y, acc1 = accs.x + accs.y;
         if (t < a.N) a.partial[(static_cast<int64_t>(chunk) * a.K + i) * a.N + t] = acc0 + acc1;
     }
 }

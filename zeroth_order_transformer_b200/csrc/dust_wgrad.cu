@@ -59,28 +59,23 @@ __global__ void __launch_bounds__(kGThreads, 8) ghat_kernel(const __grid_constan
         const int64_t t = f / nq;
         const int q = static_cast<int>(f - t * nq);
         const uint32_t tg = T.key.token_offset + static_cast<uint32_t>(t);
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        // channel pairs (4q, 4q+2) and (4q+1, 4q+3): the lanes of packed f32x2 operations
+        F2 a02{0.f, 0.f}, a13{0.f, 0.f};
         const float* rt = L.r + t;
         // unrolled so that independent Philox chains of consecutive draws interleave
 #pragma unroll 4
         for (int i = 0; i < T.K; ++i) {
             const float ri = __ldg(rt + static_cast<int64_t>(i) * L.ld_r);
-            const Polar4 z = normal_quad_polar(static_cast<uint32_t>(q) + T.key.quad_offset, tg,
-                                               T.key.draw_offset + static_cast<uint32_t>(i),
-                                               L.layer_id, T.key);
-            // r a = -kKappa (r q) (cos, sin) per pair; kKappa is applied with the scale
-            const float rr0 = ri * z.q0;
-            const float rr1 = ri * z.q1;
-            a0 = fmaf(-rr0, z.c0, a0);
-            a1 = fmaf(-rr0, z.s0, a1);
-            a2 = fmaf(-rr1, z.c1, a2);
-            a3 = fmaf(-rr1, z.s1, a3);
+            const PolarPairs z = normal_quad_pairs(static_cast<uint32_t>(q) + T.key.quad_offset, tg,
+                                                   T.key.draw_offset + static_cast<uint32_t>(i),
+                                                   L.layer_id, T.key);
+            // r a = kKappa (r nq) (cos, sin) per pair; kKappa is applied with the scale
+            const F2 rr{ri * z.nq.x, ri * z.nq.y};
+            a02 = fma2(rr, z.c, a02);
+            a13 = fma2(rr, z.s, a13);
         }
         const float sk = T.scale * kKappa;
-        a0 *= sk;
-        a1 *= sk;
-        a2 *= sk;
-        a3 *= sk;
+        const float a0 = a02.x * sk, a1 = a13.x * sk, a2 = a02.y * sk, a3 = a13.y * sk;
         const int64_t off = t * L.d_out + 4 * q;
         if (L.gb) {
             __nv_bfloat162 lo = __floats2bfloat162_rn(a0, a1);
