@@ -91,3 +91,31 @@ def test_product_package_does_not_import_the_oracle():
                 src = open(os.path.join(dirpath, fn)).read()
                 assert "import oracle" not in src and "from oracle" not in src, fn
                 assert "dust_oracle" not in src, fn
+
+
+def test_forward_tiling_choice():
+    """The bf16 forward's tile width and tail split (host logic, 2 x 148 CTA slots)."""
+    slots = 296
+    # 8 x 1024 tokens, 768 -> 3072, K = 16: 768 tiles of 256 channels leave 176 for a third
+    # wave; 1024 tiles of 192 leave 136, split in two unit ranges that end nearly together
+    assert z.dust_debug_fwd_tiling(8192, 16, [3072], slots) == (192, 2)
+    assert z.dust_debug_fwd_tiling(32768, 32, [1024], slots)[0] == 256
+    assert z.dust_debug_fwd_tiling(16384, 64, [8192], slots)[0] == 256
+    assert z.dust_debug_fwd_tiling(8192, 16, [2304, 768, 3072, 768] * 12, slots)[0] == 256
+    # a single tile's worth of work: the narrowest tiles, cut until a range of units is one
+    # round of the four warp groups (8 units: two ranges of four)
+    assert z.dust_debug_fwd_tiling(128, 4, [256], slots) == (128, 2)
+    rng = __import__("random").Random(3)
+    for _ in range(200):
+        N, K = rng.randrange(1, 40000), rng.randrange(1, 70)
+        d = [16 * rng.randrange(1, 600) for _ in range(rng.randrange(1, 5))]
+        w, split = z.dust_debug_fwd_tiling(N, K, d, slots)
+        assert w in (128, 192, 256) and 1 <= split <= 8 and (2 * K) // split >= 1
+
+
+@pytest.mark.parametrize("args", [
+    (0, 4, [256], 296), (128, 0, [256], 296), (128, 4, [0], 296), (128, 4, [256], 0),
+])
+def test_forward_tiling_rejects_bad_arguments(args):
+    with pytest.raises(z.DustError):
+        z.dust_debug_fwd_tiling(*args)

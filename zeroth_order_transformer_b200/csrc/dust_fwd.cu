@@ -1,17 +1,19 @@
 // Noisy linear forward with the per-draw loss change (Dust review page, section "신용 할당",
 // noise equation y_t -> y_t + sigma a_t, with the quadratic readout l = 1/2 |y + sigma a - u|^2).
 //
-// bf16 layers: one tcgen05 kernel; each CTA owns a 128-token x 256-channel tile of one layer
+// bf16 layers: one tcgen05 kernel; each CTA owns a 128-token x kBN-channel tile of one layer
 // (a launch may hold the tiles of up to kMaxGroup layers, described by a table in parameter
-// space).  TMA brings x and W tiles (128-byte swizzle, 2-stage ring) into shared memory, one
-// thread issues tcgen05.mma into a 128 x 256 fp32 accumulator in tensor memory.  The epilogue
-// turns the accumulator into s_e = sigma (y - u) in place; then the CTA's twelve warps share
-// (draw, channel-half) work units: each thread owns one token, regenerates the normals of the
-// unit's 128 channels (never stored) and sums sigma a e + sigma^2 a^2 / 2 into a per-unit
-// partial.  Tiles of the last, partial wave of CTAs are split into unit ranges (each computing
-// the tile's GEMM) so that the wave ends together.  The CTA that completes a token block (a
-// counter of finished units) adds the partials of all units in a fixed order, so the result is
-// deterministic.
+// space; kBN = 256, 192 or 128, chosen per launch so that the tiles fill the last wave of CTAs
+// best).  TMA brings x and W tiles (128-byte swizzle, 2-stage ring) into shared memory, one
+// thread issues tcgen05.mma into a 128 x kBN fp32 accumulator in tensor memory.  The epilogue
+// turns the accumulator into s_e = kKappa sigma (y - u) in place; then the CTA's sixteen warps
+// (four groups of four, one warp per TMEM lane quarter in each group) share (draw,
+// channel-half) work units: each thread owns one token, regenerates the normals of the unit's
+// channels (never stored) and sums sigma a e + sigma^2 a^2 / 2 into a per-unit partial.
+// Tiles of the last, partial wave of CTAs are split into unit ranges (each computing the
+// tile's GEMM) so that the wave ends together.  The CTA that completes a token block (a
+// counter of finished units) adds the partials of all units in a fixed order, so the result
+// is deterministic.
 //
 // fp32 layers: a SIMT kernel (one warp per token, one quad of channels per lane) and a
 // partial-sum reduction kernel.
@@ -25,16 +27,20 @@ namespace dust {
 namespace {
 
 constexpr int kBM = 128;  // tokens per tile
-constexpr int kBN = 256;  // channels per tile
 constexpr int kBK = 64;   // d_in per pipeline stage (128 bytes of bf16: one swizzle row)
 constexpr int kStages = 2;
 constexpr int kThreads = 512;  // 4 groups of 4 warps
 constexpr int kGroups = kThreads / 128;
 constexpr uint32_t kABytes = kBM * kBK * 2;
-constexpr uint32_t kBBytes = kBN * kBK * 2;
-constexpr uint32_t kStageBytes = kABytes + kBBytes;
-constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 + 256;
 constexpr uint32_t kTmemCols = 256;
+// Channels per tile (the MMA's N): 256, 192 or 128, chosen per launch so that the tiles fill
+// the last wave of CTAs best; the workspace is sized for the narrowest.
+constexpr int kMinBN = 128;
+template <int kBN>
+struct TileBytes {
+    static constexpr uint32_t kStage = kABytes + kBN * kBK * 2;
+    static constexpr uint32_t kSmem = kStages * kStage + 1024 + 256;
+};
 constexpr int kMaxGroup = 64;  // layers per grouped launch (parameter space holds their table)
 
 struct FwdLayer {
@@ -73,8 +79,9 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& v, float* f) {
     }
 }
 
-template <int kMax>
+template <int kMax, int kBN>
 __global__ void __launch_bounds__(kThreads, 2) fwd_bf16_kernel(const __grid_constant__ FwdTable<kMax> T) {
+    constexpr uint32_t kStageBytes = TileBytes<kBN>::kStage;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -291,38 +298,65 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_bf16_kernel(const __grid_cons
 }
 
 size_t bf16_layer_ws(int64_t N, int32_t d_out, int32_t K) {
-    const int64_t n_tiles = (d_out + kBN - 1) / kBN;
+    const int64_t n_tiles = (d_out + kMinBN - 1) / kMinBN;
     const int64_t m_tiles = (N + kBM - 1) / kBM;
     return align_up(static_cast<size_t>(2 * n_tiles * K * N) * 4, 256) +
            align_up(static_cast<size_t>(m_tiles) * 4, 256);
 }
 
-// How many unit ranges to cut each of the `rem` tiles of the last partial wave into, so that
-// the wave's CTAs finish nearly together.  A range of u units takes ceil(u / kGroups) rounds
-// of its warp groups; the cost minimised is (CTA waves of the tail) x (rounds per range as a
-// share of a whole tile's rounds + the GEMM share of a tile, about 6%).
-int tail_split(int64_t rem, int64_t slots, int units) {
-    if (rem == 0) return 1;
-    int best = 1;
-    double best_t = 1e30;
+// The tile width and the tail split of a launch.  Model (in units of a 256-channel tile's
+// noise time; the GEMM and s_e phase of a tile cost about 6% of that at 256 channels, in
+// proportion to the x and W rows it loads): the full waves of 2 CTAs per SM take whole tiles;
+// each of the `rem` tiles of the last, partial wave is cut into f unit ranges, a range of u
+// units taking ceil(u / kGroups) rounds of its warp groups.  The width and f with the
+// smallest modelled time win (ties to the wider tile and the smaller f).
+struct Tiling {
+    int width, split;
+    int64_t tiles;
+};
+
+Tiling choose_tiling(const FwdLayerArgs* layers, int n, int64_t N, int K, int64_t slots) {
+    const int units = 2 * K;
+    const int64_t m_tiles = (N + kBM - 1) / kBM;
     const double full_rounds = static_cast<double>((units + kGroups - 1) / kGroups);
-    for (int f = 1; f <= 8 && units / f >= 2; ++f) {
-        const double waves = static_cast<double>((rem * f + slots - 1) / slots);
-        const int max_units = (units + f - 1) / f;
-        const double rounds = static_cast<double>((max_units + kGroups - 1) / kGroups);
-        const double t = waves * (rounds / full_rounds + 0.06);
+    Tiling best{256, 1, 0};
+    double best_t = 1e300;
+    for (int w : {256, 192, 128}) {
+        int64_t tiles = 0;
+        for (int l = 0; l < n; ++l) tiles += m_tiles * ((layers[l].d_out + w - 1) / w);
+        const double tn = w / 256.0;
+        const double tg = 0.06 * (kBM + w) / (kBM + 256.0);
+        const int64_t n_full = tiles / slots * slots;
+        const int64_t rem = tiles - n_full;
+        double t = static_cast<double>(n_full / slots) * (tn + tg);
+        int split = 1;
+        if (rem > 0) {
+            double best_tail = 1e300;
+            for (int f = 1; f <= 8 && units / f >= 2; ++f) {
+                const double waves = static_cast<double>((rem * f + slots - 1) / slots);
+                const int max_units = (units + f - 1) / f;
+                const double rounds = static_cast<double>((max_units + kGroups - 1) / kGroups);
+                const double tt = waves * (rounds / full_rounds * tn + tg);
+                if (tt < best_tail - 1e-9) {
+                    best_tail = tt;
+                    split = f;
+                }
+            }
+            t += best_tail;
+        }
         if (t < best_t - 1e-9) {
             best_t = t;
-            best = f;
+            best = Tiling{w, split, tiles};
         }
     }
     return best;
 }
 
-// Fills and launches one table of up to kMax layers.
-template <int kMax>
+// Fills and launches one table of up to kMax layers with tiles of kBN channels.
+template <int kMax, int kBN>
 dust_status launch_bf16_table(const FwdLayerArgs* layers, int n, int64_t N, int K, float sigma,
-                              const NoiseKey& key, char* ws, cudaStream_t s) {
+                              const NoiseKey& key, int split, char* ws, cudaStream_t s) {
+    constexpr uint32_t kSmemBytes = TileBytes<kBN>::kSmem;
     FwdTable<kMax> T;  // copied into the launch's parameter space
     T.ew = device_error_word();
     T.N = N;
@@ -362,7 +396,7 @@ dust_status launch_bf16_table(const FwdLayerArgs* layers, int n, int64_t N, int 
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !attr_done[dev]) {
-        if (cudaFuncSetAttribute(fwd_bf16_kernel<kMax>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(fwd_bf16_kernel<kMax, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kSmemBytes) != cudaSuccess)
             return DUST_ERR_CUDA;
         if (dev < 64) attr_done[dev] = true;
@@ -371,13 +405,24 @@ dust_status launch_bf16_table(const FwdLayerArgs* layers, int n, int64_t N, int 
     T.total_tiles = tiles;
     const int64_t slots = 2LL * num_sms();
     T.n_full = tiles / slots * slots;
-    T.split = tail_split(tiles - T.n_full, slots, 2 * K);
+    T.split = split;
     const int64_t grid = T.n_full + (tiles - T.n_full) * T.split;
     if (grid > 2147483647LL) return DUST_ERR_UNSUPPORTED;
     prof_begin(s);
-    fwd_bf16_kernel<kMax><<<static_cast<unsigned>(grid), kThreads, kSmemBytes, s>>>(T);
+    fwd_bf16_kernel<kMax, kBN><<<static_cast<unsigned>(grid), kThreads, kSmemBytes, s>>>(T);
     prof_end(s, kMax == 1 ? "fwd_bf16_noise_loss" : "fwd_bf16_noise_loss_grouped");
     return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
+}
+
+template <int kMax>
+dust_status launch_bf16(const FwdLayerArgs* layers, int n, int64_t N, int K, float sigma,
+                        const NoiseKey& key, char* ws, cudaStream_t s) {
+    const Tiling tl = choose_tiling(layers, n, N, K, 2LL * num_sms());
+    switch (tl.width) {
+        case 256: return launch_bf16_table<kMax, 256>(layers, n, N, K, sigma, key, tl.split, ws, s);
+        case 192: return launch_bf16_table<kMax, 192>(layers, n, N, K, sigma, key, tl.split, ws, s);
+        default: return launch_bf16_table<kMax, 128>(layers, n, N, K, sigma, key, tl.split, ws, s);
+    }
 }
 
 // ------------------------------------------------------------------------------ fp32 path
@@ -453,6 +498,15 @@ size_t fwd_workspace_bytes(dust_dtype dt, int64_t N, int32_t d_out, int32_t K) {
     return align_up(static_cast<size_t>(n_cb * K * N) * 4, 256);
 }
 
+void fwd_tiling(const int32_t* d_out, int n, int64_t N, int32_t K, int64_t slots, int32_t* width,
+                int32_t* split) {
+    std::vector<FwdLayerArgs> a(static_cast<size_t>(n), FwdLayerArgs{});
+    for (int l = 0; l < n; ++l) a[l].d_out = d_out[l];
+    const Tiling t = choose_tiling(a.data(), n, N, K, slots);
+    *width = t.width;
+    *split = t.split;
+}
+
 size_t fwd_grouped_workspace_bytes(const FwdLayerArgs* layers, int n, int64_t N, int32_t K) {
     size_t total = 0;
     for (int l = 0; l < n; ++l) total += bf16_layer_ws(N, layers[l].d_out, K);
@@ -464,7 +518,7 @@ dust_status fwd_grouped_launch(const FwdLayerArgs* layers, int n, int64_t N, int
     char* base = static_cast<char*>(ws);
     for (int l0 = 0; l0 < n; l0 += kMaxGroup) {
         const int cnt = std::min(kMaxGroup, n - l0);
-        const dust_status st = launch_bf16_table<kMaxGroup>(layers + l0, cnt, N, K, sigma, key, base, s);
+        const dust_status st = launch_bf16<kMaxGroup>(layers + l0, cnt, N, K, sigma, key, base, s);
         if (st != DUST_OK) return st;
         base += fwd_grouped_workspace_bytes(layers + l0, cnt, N, K);
     }
@@ -475,10 +529,10 @@ dust_status fwd_launch(const void* x, const void* W, const void* u, dust_dtype d
                        int32_t d_in, int32_t d_out, int32_t K, float sigma, NoiseKey key,
                        float* dloss, int64_t ld, void* ws, cudaStream_t s) {
     if (dt == DUST_BF16) {
-        const int64_t tiles = (N + kBM - 1) / kBM * ((d_out + kBN - 1) / kBN);
+        const int64_t tiles = (N + kBM - 1) / kBM * ((d_out + kMinBN - 1) / kMinBN);
         if (tiles > 2147483647LL) return DUST_ERR_UNSUPPORTED;
         FwdLayerArgs a{x, W, u, d_in, d_out, key.layer, dloss, ld};
-        return launch_bf16_table<1>(&a, 1, N, K, sigma, key, static_cast<char*>(ws), s);
+        return launch_bf16<1>(&a, 1, N, K, sigma, key, static_cast<char*>(ws), s);
     }
     const int n_cb = (d_out + 4 * kF32Quads - 1) / (4 * kF32Quads);
     FwdF32Params p;

@@ -65,6 +65,10 @@ size_t fwd_grouped_workspace_bytes(const FwdLayerArgs* layers, int n, int64_t N,
 dust_status fwd_grouped_launch(const FwdLayerArgs* layers, int n, int64_t N, int32_t K,
                                float sigma, NoiseKey key, void* ws, cudaStream_t s);
 size_t fwd_workspace_bytes(dust_dtype dt, int64_t N, int32_t d_out, int32_t K);
+// The bf16 forward's tile width and tail split for layers of these widths on `slots` CTA slots
+// (host only).
+void fwd_tiling(const int32_t* d_out, int n, int64_t N, int32_t K, int64_t slots, int32_t* width,
+                int32_t* split);
 dust_status fwd_launch(const void* x, const void* W, const void* u, dust_dtype dt, int64_t N,
                        int32_t d_in, int32_t d_out, int32_t K, float sigma, NoiseKey key,
                        float* dloss, int64_t ld, void* ws, cudaStream_t s);
@@ -156,5 +160,18 @@ void prof_begin(cudaStream_t s);
 void prof_end(cudaStream_t s, const char* name);
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Division of 0 <= f by a divisor d >= 1 fixed at launch, without a 64-bit divide in the
+// kernel: with M = floor((2^64 - 1) / d) + 1 = 2^64 / d + e, 0 <= e < 1, the high word of f M
+// is floor(f / d + f e 2^-64), and f e 2^-64 < 1 / d whenever f d < 2^64, so it cannot carry
+// past the next multiple of 1 / d.  (d = 1 needs M = 2^64 and is handled apart.)
+inline uint64_t div_magic(int64_t d) {
+    return d > 1 ? ~0ull / static_cast<uint64_t>(d) + 1 : 0;
+}
+#ifdef __CUDACC__
+__device__ __forceinline__ int64_t div_by_magic(int64_t f, int64_t d, uint64_t magic) {
+    return d == 1 ? f : static_cast<int64_t>(__umul64hi(static_cast<uint64_t>(f), magic));
+}
+#endif
 
 }  // namespace dust

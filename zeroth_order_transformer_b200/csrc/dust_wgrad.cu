@@ -32,6 +32,7 @@ struct GhatLayer {
     float* gf;          // [N, d_out] or null
     int64_t ld_r, unit_begin;
     int64_t n_flat;  // N * d_out / 4: (token, channel quad) pairs, token-major
+    uint64_t nq_magic;  // div_magic(d_out / 4)
     int d_out;
     uint32_t layer_id;
 };
@@ -56,7 +57,7 @@ __global__ void __launch_bounds__(kGThreads, 8) ghat_kernel(const __grid_constan
         const int64_t f = (u - L.unit_begin) * kGThreads + threadIdx.x;
         if (f >= L.n_flat) continue;
         const int nq = L.d_out >> 2;
-        const int64_t t = f / nq;
+        const int64_t t = div_by_magic(f, nq, L.nq_magic);
         const int q = static_cast<int>(f - t * nq);
         const uint32_t tg = T.key.token_offset + static_cast<uint32_t>(t);
         // channel pairs (4q, 4q+2) and (4q+1, 4q+3): the lanes of packed f32x2 operations
@@ -374,6 +375,7 @@ dust_status launch_bf16_tables(const WgradLayerArgs* layers, int n, int64_t N, i
         L.gf = a.g_out;
         L.d_out = a.d_out;
         L.n_flat = N * (a.d_out / 4);
+        L.nq_magic = div_magic(a.d_out / 4);
         L.unit_begin = units;
         L.layer_id = a.layer_id;
         units += (L.n_flat + kGThreads - 1) / kGThreads;
@@ -504,7 +506,7 @@ dust_status wgrad_launch(const float* r, int64_t ld_r, const void* x, dust_dtype
     G.K = K_chunk;
     G.scale = -1.0f / (static_cast<float>(K_total) * sigma);
     G.key = key;
-    G.layer[0] = GhatLayer{r, nullptr, gf, ld_r, 0, N * (d_out / 4), d_out, key.layer};
+    G.layer[0] = GhatLayer{r, nullptr, gf, ld_r, 0, N * (d_out / 4), div_magic(d_out / 4), d_out, key.layer};
     G.total_units = (G.layer[0].n_flat + kGThreads - 1) / kGThreads;
     const int64_t max_blocks = static_cast<int64_t>(num_sms()) * 16;
     prof_begin(s);
