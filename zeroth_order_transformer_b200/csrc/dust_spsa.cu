@@ -36,39 +36,48 @@ constexpr int kBM = 128;
 constexpr int kBN = 256;
 constexpr int kBK = 64;
 constexpr int kStages = 2;  // two CTAs per SM: one's epilogue overlaps the other's mainloop
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;  // two warp groups share the epilogue's 16-column chunks
 constexpr uint32_t kABytes = kBM * kBK * 2;
 constexpr uint32_t kBBytes = kBN * kBK * 2;
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
-constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 + 256;
+constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 + 256 + kBM * 4;
+constexpr uint32_t kEBoxBytes = 32 * kBM * 4;  // one staged 32-column box of e
+static_assert(4 * kEBoxBytes <= kStages * kStageBytes, "e staging reuses the pipeline buffers");
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kWeightSpace = 0x80000000u;
 
 int pad256(int d) { return (d + kBN - 1) / kBN * kBN; }
 
 // ---------------------------------------------------------------- directions
+// One warp per row (probe j, output channel o) of the stacked directions, its lanes over the
+// row's channel quads: 256 contiguous bytes per warp store, and 32-bit index arithmetic (the
+// host guarantees P d_out_pad < 2^31).
 __global__ void __launch_bounds__(256) spsa_dir_kernel(const __grid_constant__ NoiseKey key, int P,
                                                        int d_out, int d_out_pad, int d_in,
                                                        __nv_bfloat16* Z) {
     const int nq = d_in >> 2;
-    const int64_t total = static_cast<int64_t>(P) * d_out_pad * nq;
-    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
-         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int q = static_cast<int>(idx % nq);
-        const int64_t row = idx / nq;  // j * d_out_pad + o
-        const int o = static_cast<int>(row % d_out_pad);
-        const int j = static_cast<int>(row / d_out_pad);
-        uint2 out = make_uint2(0u, 0u);
-        if (o < d_out) {
-            const F4 z = normal_quad(static_cast<uint32_t>(q), static_cast<uint32_t>(o),
-                                     key.draw_offset + static_cast<uint32_t>(j),
-                                     key.layer | kWeightSpace, key);
-            __nv_bfloat162 lo = __floats2bfloat162_rn(z.x, z.y);
-            __nv_bfloat162 hi = __floats2bfloat162_rn(z.z, z.w);
-            out.x = *reinterpret_cast<uint32_t*>(&lo);
-            out.y = *reinterpret_cast<uint32_t*>(&hi);
+    const int rows = P * d_out_pad;
+    const int lane = threadIdx.x & 31;
+    const int wpb = blockDim.x >> 5;
+    for (int row = blockIdx.x * wpb + (threadIdx.x >> 5); row < rows; row += gridDim.x * wpb) {
+        const int o = row % d_out_pad;
+        const uint32_t di = key.draw_offset + static_cast<uint32_t>(row / d_out_pad);
+        uint2* zr = reinterpret_cast<uint2*>(Z + static_cast<int64_t>(row) * d_in);
+        for (int q = lane; q < nq; q += 32) {
+            uint2 out = make_uint2(0u, 0u);
+            if (o < d_out) {
+                // z = kKappa nq (cos, sin) per pair; lanes: the quad's two pairs
+                const PolarPairs z = normal_quad_pairs(static_cast<uint32_t>(q), static_cast<uint32_t>(o),
+                                                       di, key.layer | kWeightSpace, key);
+                const F2 r = mul2(F2{kKappa, kKappa}, z.nq);
+                const F2 zc = mul2(r, z.c), zs = mul2(r, z.s);  // (z0, z2), (z1, z3)
+                __nv_bfloat162 lo = __floats2bfloat162_rn(zc.x, zs.x);
+                __nv_bfloat162 hi = __floats2bfloat162_rn(zc.y, zs.y);
+                out.x = *reinterpret_cast<uint32_t*>(&lo);
+                out.y = *reinterpret_cast<uint32_t*>(&hi);
+            }
+            zr[q] = out;
         }
-        *reinterpret_cast<uint2*>(Z + row * d_in + 4 * q) = out;
     }
 }
 
@@ -76,6 +85,7 @@ __global__ void __launch_bounds__(256) spsa_dir_kernel(const __grid_constant__ N
 struct GemmArgs {
     CUtensorMap tmx;  // x [N, d_in], 64 x 128 boxes
     CUtensorMap tmb;  // W [d_out, d_in] or Z [P d_out_pad, d_in], 64 x 256 boxes
+    CUtensorMap tme;  // residual mode: e [N, d_out] fp32, 32 x 128 boxes, 128-byte swizzle
     const __nv_bfloat16* u;
     float* e;         // [N, d_out] fp32: written in residual mode, read in probe mode
     float* part_a;    // residual: [o_tiles, N] 1/2 |e|^2;  probe: [2 P o_tiles, N] <e, v>
@@ -103,6 +113,7 @@ __global__ void __launch_bounds__(kThreads, 2) spsa_gemm_kernel(const __grid_con
     uint64_t* empty = full + kStages;
     uint64_t* acc_full = empty + kStages;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+    float* red = reinterpret_cast<float*>(smem + kStages * kStageBytes + 256);  // [kBM]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     // tile order: token tile fastest, so a tile of W is read once for all token tiles
@@ -164,19 +175,103 @@ __global__ void __launch_bounds__(kThreads, 2) spsa_gemm_kernel(const __grid_con
     __syncwarp();
     tc_fence_after();
 
-    // epilogue: thread = token row (TMEM lane quarter = warp)
-    const int row = warp * 32 + lane;
+    // epilogue: thread = token row (TMEM lane quarter = warp % 4)
+    const int lq = warp & 3;
+    const int grp = warp >> 2;
+    const int row = lq * 32 + lane;
     const int64_t t = m0 + row;
     const bool valid = t < A.N;
-    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t trow = tmem + (static_cast<uint32_t>(lq * 32) << 16);
     const int nchunks = min(kBN, A.d_out - o0) / 16;
-    float sa = 0.f;
-    for (int c = 0; c < nchunks; ++c) {
-        float v[16];
-        tmem_ld16(trow + c * 16, v);
-        tmem_wait_ld();
-        if (!valid) continue;
-        if (kMode == kNoisyOut) {
+    if (kMode == kResidual) {
+        // e = y - u leaves through shared memory: each warp group stages 32-column boxes of the
+        // tile's 128 rows in the freed pipeline buffers (128-byte swizzle: 16-byte chunk j of
+        // row i at position j ^ (i mod 8), conflict-free), and one thread of the group stores
+        // each box with TMA (rows past N and columns past d_out are clipped).  The groups take
+        // alternate boxes, two buffers each.  u is read one box ahead.
+        const int nboxes = (nchunks + 1) / 2;
+        const bool issuer = lq == 0 && lane == 0;
+        auto group_sync = [grp]() {  // the group's four warps (barriers 1 and 2)
+            if (grp == 0)
+                named_bar_sync(1, 128);
+            else
+                named_bar_sync(2, 128);
+        };
+        const uint4* urow = reinterpret_cast<const uint4*>(A.u + (valid ? t * A.d_out + o0 : 0));
+        uint4 un[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) un[h] = make_uint4(0u, 0u, 0u, 0u);
+        if (valid && grp < nboxes) {
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+                if (2 * grp + (h >> 1) < nchunks) un[h] = __ldg(urow + 4 * grp + h);
+        }
+        float sa = 0.f;
+        int k = 0;
+        for (int b = grp; b < nboxes; b += 2, ++k) {
+            float* buf = reinterpret_cast<float*>(smem + (grp * 2 + (k & 1)) * kEBoxBytes);
+            if (k >= 2) {
+                // the store that last read this buffer (two boxes ago) is done with it
+                if (issuer) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                group_sync();
+            }
+            uint4 uc[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) uc[h] = un[h];
+            if (valid && b + 2 < nboxes) {
+#pragma unroll
+                for (int h = 0; h < 4; ++h)
+                    if (2 * (b + 2) + (h >> 1) < nchunks) un[h] = __ldg(urow + 4 * (b + 2) + h);
+            }
+#pragma unroll
+            for (int hc = 0; hc < 2; ++hc) {
+                const int c = 2 * b + hc;
+                if (c >= nchunks) break;  // warp-uniform
+                float v[16];
+                tmem_ld16(trow + c * 16, v);
+                tmem_wait_ld();
+                float e[16];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint4 w = uc[2 * hc + h];
+                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        e[8 * h + 2 * q] = v[8 * h + 2 * q] - __uint_as_float(ww[q] << 16);
+                        e[8 * h + 2 * q + 1] = v[8 * h + 2 * q + 1] - __uint_as_float(ww[q] & 0xFFFF0000u);
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float4 e4 = make_float4(e[4 * q], e[4 * q + 1], e[4 * q + 2], e[4 * q + 3]);
+                    if (!valid) e4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                    sa = fmaf(e4.x, e4.x, sa);
+                    sa = fmaf(e4.y, e4.y, sa);
+                    sa = fmaf(e4.z, e4.z, sa);
+                    sa = fmaf(e4.w, e4.w, sa);
+                    const int j = (4 * hc + q) ^ (row & 7);
+                    *reinterpret_cast<float4*>(buf + row * 32 + 4 * j) = e4;
+                }
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            group_sync();
+            if (issuer) {
+                tma_store_2d(&A.tme, buf, o0 + 32 * b, static_cast<int32_t>(m0));
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            }
+        }
+        if (issuer) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        // the two groups' partial sums of a token, added in a fixed order
+        if (grp == 1) red[row] = sa;
+        __syncthreads();
+        if (grp == 0 && valid) A.part_a[static_cast<int64_t>(o_tile) * A.N + t] = 0.5f * (sa + red[row]);
+    } else {
+        // the perturbed outputs of every draw; the two warp groups take alternate 16-column chunks
+        for (int c = grp; c < nchunks; c += 2) {
+            float v[16];
+            tmem_ld16(trow + c * 16, v);
+            tmem_wait_ld();
+            if (!valid) continue;
             const uint32_t tg = A.key.token_offset + static_cast<uint32_t>(t);
             const uint32_t q0 = static_cast<uint32_t>((o0 + c * 16) >> 2) + A.key.quad_offset;
             for (int i = 0; i < A.K; ++i) {
@@ -209,37 +304,8 @@ __global__ void __launch_bounds__(kThreads, 2) spsa_gemm_kernel(const __grid_con
                         dst[qq] = make_float4(o[4 * qq], o[4 * qq + 1], o[4 * qq + 2], o[4 * qq + 3]);
                 }
             }
-            continue;
-        }
-        const int64_t off = t * A.d_out + o0 + c * 16;
-        const uint4* up = reinterpret_cast<const uint4*>(A.u + off);
-        float uf[16];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const uint4 w = __ldg(up + h);
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uf[8 * h + 2 * q] = __uint_as_float(ww[q] << 16);
-                uf[8 * h + 2 * q + 1] = __uint_as_float(ww[q] & 0xFFFF0000u);
-            }
-        }
-        float4* e4 = reinterpret_cast<float4*>(A.e + off);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            float4 e;
-            e.x = v[4 * q] - uf[4 * q];
-            e.y = v[4 * q + 1] - uf[4 * q + 1];
-            e.z = v[4 * q + 2] - uf[4 * q + 2];
-            e.w = v[4 * q + 3] - uf[4 * q + 3];
-            e4[q] = e;
-            sa = fmaf(e.x, e.x, sa);
-            sa = fmaf(e.y, e.y, sa);
-            sa = fmaf(e.z, e.z, sa);
-            sa = fmaf(e.w, e.w, sa);
         }
     }
-    if (kMode == kResidual && valid) A.part_a[static_cast<int64_t>(o_tile) * A.N + t] = 0.5f * sa;
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
@@ -458,27 +524,32 @@ __global__ void spsa_finish_kernel(const float* sums, int P, int o_tiles, int n_
 __global__ void __launch_bounds__(256) spsa_estimate_kernel(const __grid_constant__ NoiseKey key,
                                                             const float* __restrict__ p, int P,
                                                             int d_out, int d_in, float scale,
-                                                            float* G, int accumulate) {
+                                                            float* G, int accumulate,
+                                                            uint64_t nq_magic) {
     const int nq = d_in >> 2;
     const int64_t total = static_cast<int64_t>(d_out) * nq;
     for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
          idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int q = static_cast<int>(idx % nq);
-        const int o = static_cast<int>(idx / nq);
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        const int o = static_cast<int>(div_by_magic(idx, nq, nq_magic));
+        const int q = static_cast<int>(idx - static_cast<int64_t>(o) * nq);
+        F2 a02{0.f, 0.f}, a13{0.f, 0.f};  // channels (4q, 4q+2) and (4q+1, 4q+3)
+        // unrolled so that independent Philox chains of consecutive probes interleave
+#pragma unroll 4
         for (int j = 0; j < P; ++j) {
             const float pj = __ldg(p + j);
-            const F4 z = normal_quad(static_cast<uint32_t>(q), static_cast<uint32_t>(o),
-                                     key.draw_offset + static_cast<uint32_t>(j),
-                                     key.layer | kWeightSpace, key);
+            const PolarPairs z = normal_quad_pairs(static_cast<uint32_t>(q), static_cast<uint32_t>(o),
+                                                   key.draw_offset + static_cast<uint32_t>(j),
+                                                   key.layer | kWeightSpace, key);
+            const F2 r = mul2(F2{kKappa, kKappa}, z.nq);
+            const F2 zc = mul2(r, z.c), zs = mul2(r, z.s);
             // the direction is the bf16 value of the normal
-            a0 = fmaf(pj, __bfloat162float(__float2bfloat16_rn(z.x)), a0);
-            a1 = fmaf(pj, __bfloat162float(__float2bfloat16_rn(z.y)), a1);
-            a2 = fmaf(pj, __bfloat162float(__float2bfloat16_rn(z.z)), a2);
-            a3 = fmaf(pj, __bfloat162float(__float2bfloat16_rn(z.w)), a3);
+            const __nv_bfloat162 bc = __floats2bfloat162_rn(zc.x, zc.y);
+            const __nv_bfloat162 bs = __floats2bfloat162_rn(zs.x, zs.y);
+            a02 = fma2(F2{pj, pj}, F2{__low2float(bc), __high2float(bc)}, a02);
+            a13 = fma2(F2{pj, pj}, F2{__low2float(bs), __high2float(bs)}, a13);
         }
         float4* g = reinterpret_cast<float4*>(G + static_cast<int64_t>(o) * d_in + 4 * q);
-        float4 r = make_float4(scale * a0, scale * a1, scale * a2, scale * a3);
+        float4 r = make_float4(scale * a02.x, scale * a13.x, scale * a02.y, scale * a13.y);
         if (accumulate) {
             const float4 old = *g;
             r.x += old.x;
@@ -534,7 +605,8 @@ dust_status spsa_probe_launch(const void* x, const void* W, const void* u, int64
     R.P = P;
     R.m_tiles = m_tiles;
     if (!make_tmap_bf16_2d(&R.tmx, x, static_cast<uint64_t>(N), d_in, kBM, kBK) ||
-        !make_tmap_bf16_2d(&R.tmb, W, static_cast<uint64_t>(d_out), d_in, kBN, kBK))
+        !make_tmap_bf16_2d(&R.tmb, W, static_cast<uint64_t>(d_out), d_in, kBN, kBK) ||
+        !make_tmap_f32_2d_sw128(&R.tme, e, static_cast<uint64_t>(N), d_out, d_out, kBM))
         return DUST_ERR_CUDA;
     GemmArgs Q = R;
     Q.part_a = pev;
@@ -546,10 +618,10 @@ dust_status spsa_probe_launch(const void* x, const void* W, const void* u, int64
         cudaFuncSetAttribute(spsa_probe_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kPSmemBytes)) != cudaSuccess)
         return DUST_ERR_CUDA;
-    const int64_t dir_total = static_cast<int64_t>(P) * dpad * (d_in / 4);
+    const int64_t dir_rows = static_cast<int64_t>(P) * dpad;  // one warp each, 8 per block
     prof_begin(s);
-    spsa_dir_kernel<<<static_cast<unsigned>(std::min<int64_t>((dir_total + 255) / 256,
-                                                              static_cast<int64_t>(num_sms()) * 16)),
+    spsa_dir_kernel<<<static_cast<unsigned>(std::min<int64_t>((dir_rows + 7) / 8,
+                                                              static_cast<int64_t>(num_sms()) * 8)),
                       256, 0, s>>>(key, P, d_out, dpad, d_in, Z);
     prof_end(s, "spsa_directions");
     prof_begin(s);
@@ -609,7 +681,7 @@ dust_status spsa_estimate_launch(const float* p, int32_t P, int32_t P_total, int
     spsa_estimate_kernel<<<static_cast<unsigned>(std::min<int64_t>((total + 255) / 256,
                                                                    static_cast<int64_t>(num_sms()) * 16)),
                            256, 0, s>>>(key, p, P, d_out, d_in, 1.0f / static_cast<float>(P_total),
-                                        G, accumulate);
+                                        G, accumulate, div_magic(d_in / 4));
     prof_end(s, "spsa_estimate");
     return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
 }
