@@ -49,10 +49,10 @@ OPS_PER_NORMAL = {"fwd_bf16_noise_loss": 20.0, "ghat_reduce_draws": 19.0,
 # current build of that kernel on that workload (profiles/ holds the capture summaries);
 # absent entries are reported as null.
 MEASURED_TRAFFIC = {
-    ("fwd_bf16_noise_loss", "gpt2s-mlp-win-768x3072"): (67.84e6 + 4.06e6,
-                                                       "profiles/ncu_full_gpt2s_mlp_win_768x3072.md"),
-    ("ghat_reduce_draws", "gpt2s-mlp-win-768x3072"): (0.54e6 + 0.52e6,
-                                                     "profiles/ncu_full_gpt2s_mlp_win_768x3072.md"),
+    ("fwd_bf16_noise_loss", "gpt2s-mlp-win-768x3072"): (68.49e6 + 2.45e6,
+                                                       "profiles/ncu_full_fwd_persistent_gpt2s_mlp_win_768x3072.md"),
+    ("ghat_reduce_draws", "gpt2s-mlp-win-768x3072"): (0.54e6 + 0.49e6,
+                                                     "profiles/ncu_full_fwd_persistent_gpt2s_mlp_win_768x3072.md"),
 }
 HEAD_METRIC = "Dust LM-head estimator tokens*draws/s"
 ATTN_METRIC = "Dust attention-reward estimator tokens*draws/s"

@@ -380,15 +380,14 @@ dust_status dust_debug_normal_sum(dust_noise_key key, int64_t n, int32_t n_quads
  * bounded wait runs out.  Used to test the timeout path; never set in normal use. */
 void dust_debug_credit_skip_publish(int32_t block);
 
-/* Test support: the tiling the bf16 forward (dust_noisy_linear_fwd and its grouped form) chooses
+/* Test support: the form the bf16 forward (dust_noisy_linear_fwd and its grouped form) takes
  * for N tokens, K draws and n_layers layers of output widths d_out[0 .. n_layers-1] (HOST
- * int32) when `slots` CTAs run at once (2 per SM).  Writes the tile width in channels (256,
- * 192 or 128: the one whose tiles fill the last wave of CTAs best under a cost model of the
- * kernel) and the number of unit ranges each tile of the last, partial wave is cut into.
- * Host-only: touches no device.  DUST_ERR_INVALID_ARG on a non-positive size or a NULL
- * pointer. */
-dust_status dust_debug_fwd_tiling(int64_t N, int32_t K, int32_t n_layers, const int32_t* d_out,
-                                  int32_t slots, int32_t* width, int32_t* split);
+ * int32) on a device with `sms` SMs.  *persistent = 1: one CTA per SM walks a balanced range
+ * of (tile, draw, channel half) items (*split = 0); 0: one 128 x 256 tile per CTA, two CTAs per
+ * SM, each tile of the last, partial wave cut into *split unit ranges.  Host-only: touches no
+ * device.  DUST_ERR_INVALID_ARG on a non-positive size or a NULL pointer. */
+dust_status dust_debug_fwd_plan(int64_t N, int32_t K, int32_t n_layers, const int32_t* d_out,
+                                int32_t sms, int32_t* persistent, int32_t* split);
 
 #ifdef __cplusplus
 }

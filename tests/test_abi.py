@@ -93,29 +93,37 @@ def test_product_package_does_not_import_the_oracle():
                 assert "dust_oracle" not in src, fn
 
 
-def test_forward_tiling_choice():
-    """The bf16 forward's tile width and tail split (host logic, 2 x 148 CTA slots)."""
-    slots = 296
-    # 8 x 1024 tokens, 768 -> 3072, K = 16: 768 tiles of 256 channels leave 176 for a third
-    # wave; 1024 tiles of 192 leave 136, split in two unit ranges that end nearly together
-    assert z.dust_debug_fwd_tiling(8192, 16, [3072], slots) == (192, 2)
-    assert z.dust_debug_fwd_tiling(32768, 32, [1024], slots)[0] == 256
-    assert z.dust_debug_fwd_tiling(16384, 64, [8192], slots)[0] == 256
-    assert z.dust_debug_fwd_tiling(8192, 16, [2304, 768, 3072, 768] * 12, slots)[0] == 256
-    # a single tile's worth of work: the narrowest tiles, cut until a range of units is one
-    # round of the four warp groups (8 units: two ranges of four)
-    assert z.dust_debug_fwd_tiling(128, 4, [256], slots) == (128, 2)
+def test_forward_plan():
+    """The bf16 forward's form and tail split (host logic, 148 SMs: 296 CTA slots of the
+    one-tile kernel)."""
+    sms = 148
+    # 8 x 1024 tokens, 768 -> 3072: 768 tiles, under three waves of 296: persistent
+    assert z.dust_debug_fwd_plan(8192, 16, [3072], sms) == (True, 0)
+    assert z.dust_debug_fwd_plan(1024, 16, [3072], sms) == (True, 0)
+    assert z.dust_debug_fwd_plan(128, 4, [256], sms) == (True, 0)
+    # 887 tiles persistent, 888 (three waves) one tile per CTA
+    assert z.dust_debug_fwd_plan(887 * 128, 8, [256], sms)[0]
+    assert not z.dust_debug_fwd_plan(888 * 128, 8, [256], sms)[0]
+    # 32k tokens x 1024 -> 1024, K = 32: 1024 tiles; the 136 of the last wave in two ranges
+    # of 32 units (eight rounds of the four warp groups: one wave of 272 CTAs)
+    assert z.dust_debug_fwd_plan(32768, 32, [1024], sms) == (False, 2)
+    # 16k x 2048 -> 8192, K = 64: 4096 tiles, 248 in the last wave, whole
+    assert z.dust_debug_fwd_plan(16384, 64, [8192], sms) == (False, 1)
+    # the 48-layer group: 20736 tiles
+    assert not z.dust_debug_fwd_plan(8192, 16, [2304, 768, 3072, 768] * 12, sms)[0]
     rng = __import__("random").Random(3)
     for _ in range(200):
-        N, K = rng.randrange(1, 40000), rng.randrange(1, 70)
+        N, K = rng.randrange(1, 200000), rng.randrange(1, 70)
         d = [16 * rng.randrange(1, 600) for _ in range(rng.randrange(1, 5))]
-        w, split = z.dust_debug_fwd_tiling(N, K, d, slots)
-        assert w in (128, 192, 256) and 1 <= split <= 8 and (2 * K) // split >= 1
+        persistent, split = z.dust_debug_fwd_plan(N, K, d, sms)
+        tiles = sum(-(-N // 128) * -(-dd // 256) for dd in d)
+        assert persistent == (tiles < 3 * 2 * sms)
+        assert (split == 0) if persistent else (1 <= split <= 8 and (2 * K) // split >= 1)
 
 
 @pytest.mark.parametrize("args", [
-    (0, 4, [256], 296), (128, 0, [256], 296), (128, 4, [0], 296), (128, 4, [256], 0),
+    (0, 4, [256], 148), (128, 0, [256], 148), (128, 4, [0], 148), (128, 4, [256], 0),
 ])
-def test_forward_tiling_rejects_bad_arguments(args):
+def test_forward_plan_rejects_bad_arguments(args):
     with pytest.raises(z.DustError):
-        z.dust_debug_fwd_tiling(*args)
+        z.dust_debug_fwd_plan(*args)

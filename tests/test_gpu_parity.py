@@ -109,30 +109,20 @@ def test_fwd_bf16_matches_oracle(N, d_in, d_out, K):
     _dev.assert_fp32_close(got, ref, "dloss")
 
 
-def _tile_width_cases():
-    """The cheapest shape (N x d_out x K, d_in = 64) for which the forward chooses each tile
-    width on this device, with whole and with ragged last tiles."""
+def test_fwd_bf16_both_forms_match_oracle():
+    """Layers large enough for the one-tile-per-CTA form (three waves of two CTAs per SM) and
+    just below it (the persistent form), with ragged token and channel tails."""
     import torch
-    slots = 2 * torch.cuda.get_device_properties(0).multi_processor_count
-    found = {}
-    for N in (2048, 2047, 4096, 4000, 5120, 8192):
-        for d_out in (768, 784, 1024, 1040, 1536, 1552, 2048, 3072):
-            for K in (2, 4, 8):
-                w, _ = z.dust_debug_fwd_tiling(N, K, [d_out], slots)
-                case = (w, N % 128 != 0 or d_out % w != 0)
-                if case not in found or N * d_out * K < found[case][0]:
-                    found[case] = (N * d_out * K, N, d_out, K)
-    return found
-
-
-def test_fwd_bf16_every_tile_width_matches_oracle():
-    found = _tile_width_cases()
-    assert {w for w, _ in found} == {128, 192, 256}
-    for (w, ragged), (_, N, d_out, K) in sorted(found.items()):
-        L = workloads.custom_layer(77 + N + d_out, N, 64, d_out, "bf16", 0.02)
-        key = z.NoiseKey(0x5EED00A0 + w, layer_id=1, draw_offset=3, token_offset=5)
-        got, ref = _fwd_case(L, K, 1e-3, key)
-        _dev.assert_fp32_close(got, ref, f"dloss, {w}-channel tiles, ragged {ragged}")
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for d_out, K in ((1040, 2), (784, 3)):
+        n_t = -(-d_out // 256)
+        for m_tiles, persistent in ((-(-6 * sms // n_t)), False), ((6 * sms - 1) // n_t, True):
+            N = 128 * m_tiles - 37
+            assert z.dust_debug_fwd_plan(N, K, [d_out], sms)[0] == persistent
+            L = workloads.custom_layer(90 + N + d_out, N, 64, d_out, "bf16", 0.02)
+            key = z.NoiseKey(0x5EED00B0 + K, layer_id=1, draw_offset=3, token_offset=5)
+            got, ref = _fwd_case(L, K, 1e-3, key)
+            _dev.assert_fp32_close(got, ref, f"dloss, persistent {persistent}, {N} x {d_out}")
 
 
 def test_fwd_f32_tiny_workload_matches_oracle():

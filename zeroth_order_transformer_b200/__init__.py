@@ -43,7 +43,7 @@ EXPORTED_SYMBOLS = (
     "dust_profile_read", "dust_credit_no_alloc", "dust_noisy_linear_fwd_grouped",
     "dust_credit_grouped", "dust_weight_grad_grouped", "dust_workspace_size_grouped",
     "dust_optimizer_step", "dust_weight_grad_step", "dust_noisy_logits_ce",
-    "dust_debug_normal_sum", "dust_debug_fwd_tiling", "dust_attn_reward", "dust_discounted_credit",
+    "dust_debug_normal_sum", "dust_debug_fwd_plan", "dust_attn_reward", "dust_discounted_credit",
     "dust_spsa_probe", "dust_spsa_estimate", "dust_noisy_linear_output",
 )
 
@@ -164,9 +164,9 @@ def lib() -> ctypes.CDLL:
         L.dust_debug_normal_sum.restype = ctypes.c_int
         L.dust_debug_credit_skip_publish.argtypes = [i32]
         L.dust_debug_credit_skip_publish.restype = None
-        L.dust_debug_fwd_tiling.argtypes = [i64, i32, i32, vp, i32, ctypes.POINTER(i32),
-                                            ctypes.POINTER(i32)]
-        L.dust_debug_fwd_tiling.restype = ctypes.c_int
+        L.dust_debug_fwd_plan.argtypes = [i64, i32, i32, vp, i32, ctypes.POINTER(i32),
+                                          ctypes.POINTER(i32)]
+        L.dust_debug_fwd_plan.restype = ctypes.c_int
         L.dust_profile_enable.argtypes = [i32]
         L.dust_profile_enable.restype = ctypes.c_int
         L.dust_profile_disable.argtypes = []
@@ -522,15 +522,15 @@ def dust_debug_normal_sum(key: NoiseKey, n: int, n_quads: int, out=None, device=
     return out
 
 
-def dust_debug_fwd_tiling(N: int, K: int, d_outs, slots: int):
-    """(tile width, tail split) that the bf16 forward chooses for layers of output widths
-    `d_outs` when `slots` CTAs run at once (host only; no device needed)."""
+def dust_debug_fwd_plan(N: int, K: int, d_outs, sms: int):
+    """(persistent, tail split) of the bf16 forward for layers of output widths `d_outs` on a
+    device with `sms` SMs (host only; no device needed)."""
     arr = (ctypes.c_int32 * len(d_outs))(*[int(d) for d in d_outs])
-    w, sp = ctypes.c_int32(0), ctypes.c_int32(0)
-    st = lib().dust_debug_fwd_tiling(int(N), int(K), len(d_outs), ctypes.cast(arr, ctypes.c_void_p),
-                                     int(slots), ctypes.byref(w), ctypes.byref(sp))
-    _check(st, "dust_debug_fwd_tiling")
-    return w.value, sp.value
+    p, sp = ctypes.c_int32(0), ctypes.c_int32(0)
+    st = lib().dust_debug_fwd_plan(int(N), int(K), len(d_outs), ctypes.cast(arr, ctypes.c_void_p),
+                                   int(sms), ctypes.byref(p), ctypes.byref(sp))
+    _check(st, "dust_debug_fwd_plan")
+    return bool(p.value), sp.value
 
 
 def dust_debug_credit_skip_publish(block: int) -> None:

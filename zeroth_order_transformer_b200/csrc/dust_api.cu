@@ -477,13 +477,13 @@ dust_status dust_debug_normal_sum(dust_noise_key key, int64_t n, int32_t n_quads
 
 void dust_debug_credit_skip_publish(int32_t block) { g_credit_skip_publish = block; }
 
-dust_status dust_debug_fwd_tiling(int64_t N, int32_t K, int32_t n_layers, const int32_t* d_out,
-                                  int32_t slots, int32_t* width, int32_t* split) {
-    if (N < 1 || K < 1 || n_layers < 1 || !d_out || slots < 1 || !width || !split)
+dust_status dust_debug_fwd_plan(int64_t N, int32_t K, int32_t n_layers, const int32_t* d_out,
+                                int32_t sms, int32_t* persistent, int32_t* split) {
+    if (N < 1 || K < 1 || n_layers < 1 || !d_out || sms < 1 || !persistent || !split)
         return DUST_ERR_INVALID_ARG;
     for (int32_t l = 0; l < n_layers; ++l)
         if (d_out[l] < 1) return DUST_ERR_INVALID_ARG;
-    fwd_tiling(d_out, n_layers, N, K, slots, width, split);
+    fwd_plan(d_out, n_layers, N, K, sms, persistent, split);
     return DUST_OK;
 }
 

@@ -316,6 +316,22 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// The same for waits expected to be long, by warps that share their SM with busy ones: sleeps
+// `ns` between polls so that the waiting warp takes few issue slots.
+__device__ __forceinline__ bool mbar_wait_bounded_sleep(uint64_t* bar, uint32_t parity, ErrorWord* ew,
+                                                        int site, uint32_t ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        __nanosleep(ns);
+        if (mbar_try_wait(bar, parity)) return true;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            report_error(ew, kDevTimeout, site);
+            return false;
+        }
+    }
+}
+
 // 2-D tiled TMA load of box (x, y) into shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map,
                                             uint64_t* bar, int32_t x, int32_t y) {

@@ -33,14 +33,9 @@ constexpr int kThreads = 512;  // 4 groups of 4 warps
 constexpr int kGroups = kThreads / 128;
 constexpr uint32_t kABytes = kBM * kBK * 2;
 constexpr uint32_t kTmemCols = 256;
-// Channels per tile (the MMA's N): 256, 192 or 128, chosen per launch so that the tiles fill
-// the last wave of CTAs best; the workspace is sized for the narrowest.
-constexpr int kMinBN = 128;
-template <int kBN>
-struct TileBytes {
-    static constexpr uint32_t kStage = kABytes + kBN * kBK * 2;
-    static constexpr uint32_t kSmem = kStages * kStage + 1024 + 256;
-};
+constexpr int kBN = 256;  // channels per tile (the MMA's N)
+constexpr uint32_t kStageBytes = kABytes + kBN * kBK * 2;
+constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 + 256;
 constexpr int kMaxGroup = 64;  // layers per grouped launch (parameter space holds their table)
 
 struct FwdLayer {
@@ -79,9 +74,8 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& v, float* f) {
     }
 }
 
-template <int kMax, int kBN>
+template <int kMax>
 __global__ void __launch_bounds__(kThreads, 2) fwd_bf16_kernel(const __grid_constant__ FwdTable<kMax> T) {
-    constexpr uint32_t kStageBytes = TileBytes<kBN>::kStage;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -298,65 +292,57 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_bf16_kernel(const __grid_cons
 }
 
 size_t bf16_layer_ws(int64_t N, int32_t d_out, int32_t K) {
-    const int64_t n_tiles = (d_out + kMinBN - 1) / kMinBN;
+    const int64_t n_tiles = (d_out + kBN - 1) / kBN;
     const int64_t m_tiles = (N + kBM - 1) / kBM;
     return align_up(static_cast<size_t>(2 * n_tiles * K * N) * 4, 256) +
            align_up(static_cast<size_t>(m_tiles) * 4, 256);
 }
 
-// The tile width and the tail split of a launch.  Model (in units of a 256-channel tile's
-// noise time; the GEMM and s_e phase of a tile cost about 6% of that at 256 channels, in
-// proportion to the x and W rows it loads): the full waves of 2 CTAs per SM take whole tiles;
-// each of the `rem` tiles of the last, partial wave is cut into f unit ranges, a range of u
-// units taking ceil(u / kGroups) rounds of its warp groups.  The width and f with the
-// smallest modelled time win (ties to the wider tile and the smaller f).
-struct Tiling {
-    int width, split;
-    int64_t tiles;
+// The form of a launch.  With fewer tiles than three waves of the one-tile kernel (two CTAs
+// per SM), the persistent kernel below wins: its GEMM and s_e pass hide behind the noise work
+// and its ranges end together (+2% at 8k tokens x 768->3072 in the bench, +43% at 1k tokens).
+// With more, the one-tile kernel's 32 noise warps per SM beat the persistent kernel's 28
+// (-3% at 32k x 1024^2, -7% for the 48-layer group) and its waves desynchronise by themselves.
+// The one-tile kernel cuts each tile of its last, partial wave into `split` unit ranges: a
+// range of u units takes ceil(u / kGroups) rounds of its warp groups, and the cost minimised is
+// (CTA waves of the tail) x (rounds per range as a share of a whole tile's + the GEMM share of
+// a tile, about 6%).
+constexpr int kPersistentMaxWaves = 3;
+
+struct FwdPlan {
+    bool persistent;
+    int split;
 };
 
-Tiling choose_tiling(const FwdLayerArgs* layers, int n, int64_t N, int K, int64_t slots) {
-    const int units = 2 * K;
+FwdPlan plan_forward(const FwdLayerArgs* layers, int n, int64_t N, int K, int64_t sms) {
     const int64_t m_tiles = (N + kBM - 1) / kBM;
-    const double full_rounds = static_cast<double>((units + kGroups - 1) / kGroups);
-    Tiling best{256, 1, 0};
+    int64_t tiles = 0;
+    for (int l = 0; l < n; ++l) tiles += m_tiles * ((layers[l].d_out + kBN - 1) / kBN);
+    const int64_t slots = 2 * sms;
+    if (tiles < kPersistentMaxWaves * slots) return FwdPlan{true, 0};
+    const int units = 2 * K;
+    const int64_t rem = tiles % slots;
+    if (rem == 0) return FwdPlan{false, 1};
+    int best = 1;
     double best_t = 1e300;
-    for (int w : {256, 192, 128}) {
-        int64_t tiles = 0;
-        for (int l = 0; l < n; ++l) tiles += m_tiles * ((layers[l].d_out + w - 1) / w);
-        const double tn = w / 256.0;
-        const double tg = 0.06 * (kBM + w) / (kBM + 256.0);
-        const int64_t n_full = tiles / slots * slots;
-        const int64_t rem = tiles - n_full;
-        double t = static_cast<double>(n_full / slots) * (tn + tg);
-        int split = 1;
-        if (rem > 0) {
-            double best_tail = 1e300;
-            for (int f = 1; f <= 8 && units / f >= 2; ++f) {
-                const double waves = static_cast<double>((rem * f + slots - 1) / slots);
-                const int max_units = (units + f - 1) / f;
-                const double rounds = static_cast<double>((max_units + kGroups - 1) / kGroups);
-                const double tt = waves * (rounds / full_rounds * tn + tg);
-                if (tt < best_tail - 1e-9) {
-                    best_tail = tt;
-                    split = f;
-                }
-            }
-            t += best_tail;
-        }
+    const double full_rounds = static_cast<double>((units + kGroups - 1) / kGroups);
+    for (int f = 1; f <= 8 && units / f >= 2; ++f) {
+        const double waves = static_cast<double>((rem * f + slots - 1) / slots);
+        const int max_units = (units + f - 1) / f;
+        const double rounds = static_cast<double>((max_units + kGroups - 1) / kGroups);
+        const double t = waves * (rounds / full_rounds + 0.06);
         if (t < best_t - 1e-9) {
             best_t = t;
-            best = Tiling{w, split, tiles};
+            best = f;
         }
     }
-    return best;
+    return FwdPlan{false, best};
 }
 
-// Fills and launches one table of up to kMax layers with tiles of kBN channels.
-template <int kMax, int kBN>
+// Fills and launches one table of up to kMax layers, one tile per CTA.
+template <int kMax>
 dust_status launch_bf16_table(const FwdLayerArgs* layers, int n, int64_t N, int K, float sigma,
                               const NoiseKey& key, int split, char* ws, cudaStream_t s) {
-    constexpr uint32_t kSmemBytes = TileBytes<kBN>::kSmem;
     FwdTable<kMax> T;  // copied into the launch's parameter space
     T.ew = device_error_word();
     T.N = N;
@@ -396,7 +382,7 @@ dust_status launch_bf16_table(const FwdLayerArgs* layers, int n, int64_t N, int 
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !attr_done[dev]) {
-        if (cudaFuncSetAttribute(fwd_bf16_kernel<kMax, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(fwd_bf16_kernel<kMax>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kSmemBytes) != cudaSuccess)
             return DUST_ERR_CUDA;
         if (dev < 64) attr_done[dev] = true;
@@ -409,20 +395,345 @@ dust_status launch_bf16_table(const FwdLayerArgs* layers, int n, int64_t N, int 
     const int64_t grid = T.n_full + (tiles - T.n_full) * T.split;
     if (grid > 2147483647LL) return DUST_ERR_UNSUPPORTED;
     prof_begin(s);
-    fwd_bf16_kernel<kMax, kBN><<<static_cast<unsigned>(grid), kThreads, kSmemBytes, s>>>(T);
+    fwd_bf16_kernel<kMax><<<static_cast<unsigned>(grid), kThreads, kSmemBytes, s>>>(T);
     prof_end(s, kMax == 1 ? "fwd_bf16_noise_loss" : "fwd_bf16_noise_loss_grouped");
     return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
 }
 
 template <int kMax>
+dust_status launch_persistent(const FwdLayerArgs* layers, int n, int64_t N, int K, float sigma,
+                              const NoiseKey& key, char* ws, cudaStream_t s);
+
+template <int kMax>
 dust_status launch_bf16(const FwdLayerArgs* layers, int n, int64_t N, int K, float sigma,
                         const NoiseKey& key, char* ws, cudaStream_t s) {
-    const Tiling tl = choose_tiling(layers, n, N, K, 2LL * num_sms());
-    switch (tl.width) {
-        case 256: return launch_bf16_table<kMax, 256>(layers, n, N, K, sigma, key, tl.split, ws, s);
-        case 192: return launch_bf16_table<kMax, 192>(layers, n, N, K, sigma, key, tl.split, ws, s);
-        default: return launch_bf16_table<kMax, 128>(layers, n, N, K, sigma, key, tl.split, ws, s);
+    const FwdPlan plan = plan_forward(layers, n, N, K, num_sms());
+    if (plan.persistent) return launch_persistent<kMax>(layers, n, N, K, sigma, key, ws, s);
+    return launch_bf16_table<kMax>(layers, n, N, K, sigma, key, plan.split, ws, s);
+}
+
+// ------------------------------------------------------------------------ persistent form
+// One CTA per SM walks a balanced, contiguous range of the launch's (tile, unit) items, tiles of
+// 128 tokens x 256 channels in token-block-major order.  Two 256-column accumulators let the
+// next tile's GEMM and s_e pass run while the noise warps work on the current tile:
+//   warps 0-3   the control group: warp 0 lane 0 feeds a 4-stage TMA ring, warp 1 lane 0 issues
+//               the MMAs into accumulator jj % 2, then all four warps (one per TMEM lane
+//               quarter) rewrite it in place to s_e and signal se_ready; the accumulator of
+//               tile jj is reused for tile jj + 2 once the noise warps signal acc_empty;
+//   warps 4-31  seven groups of four noise warps: group g takes the CTA's units g, g + 7, ...
+//               (draw, channel half), each as in the one-tile kernel above.
+// The per-unit partials are added by fwd_reduce_kernel afterwards, in a fixed order.
+constexpr int kPThreads = 1024;
+constexpr int kPNoiseGroups = (kPThreads - 128) / 128;  // 7
+constexpr int kPStages = 4;
+constexpr uint32_t kPStageBytes = kStageBytes;
+constexpr uint32_t kPSmemBytes = kPStages * kPStageBytes + 1024 + 256;
+
+template <int kMax>
+__global__ void __launch_bounds__(kPThreads, 1) fwd_persistent_kernel(const __grid_constant__ FwdTable<kMax> T) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPStages * kPStageBytes);
+    uint64_t* empty = full + kPStages;
+    uint64_t* acc_full = empty + kPStages;  // [2]
+    uint64_t* se_ready = acc_full + 2;      // [2]
+    uint64_t* acc_empty = se_ready + 2;     // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t N = T.N;
+    const int K = T.K;
+    const int U = 2 * K;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < kPStages; ++st) {
+            mbar_init(&full[st], 1);
+            mbar_init(&empty[st], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&se_ready[b], 128);
+            mbar_init(&acc_empty[b], kPNoiseGroups * 4);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
     }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 2 * kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // waits give up together: the first that times out sets the flag, later ones return at once
+    auto wait = [&](uint64_t* bar, uint32_t parity, int site) -> bool {
+        if (*abort_flag) return false;
+        if (mbar_wait_bounded(bar, parity, T.ew, site)) return true;
+        *abort_flag = 1;
+        return false;
+    };
+    // the control group's long waits (for the noise warps, and for the GEMM) poll every 256 ns
+    auto wait_idle = [&](uint64_t* bar, uint32_t parity, int site) -> bool {
+        if (*abort_flag) return false;
+        if (mbar_wait_bounded_sleep(bar, parity, T.ew, site, 256)) return true;
+        *abort_flag = 1;
+        return false;
+    };
+
+    // this CTA's items: [ub, ue) of the launch's total_tiles * U (tile-major)
+    const int64_t total = T.total_tiles * U;
+    const int64_t ub = total * blockIdx.x / gridDim.x;
+    const int64_t ue = total * (blockIdx.x + 1) / gridDim.x;
+    if (ub < ue) {
+        const int64_t tile_first = ub / U;
+        const int nt = static_cast<int>((ue - 1) / U - tile_first + 1);
+        int l = 0;
+        if (warp < 4) {
+            // ------------------------------------------------------------ control group
+            uint32_t kc_prod = 0, kc_mma = 0;
+            const int row = warp * 32 + lane;
+            const uint32_t trow0 = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+            for (int jj = 0; jj < nt; ++jj) {
+                const int64_t gt = tile_first + jj;
+                while (l + 1 < T.n_layers && gt >= T.layer[l + 1].tile_begin) ++l;
+                const FwdLayer& L = T.layer[l];
+                const int local = static_cast<int>(gt - L.tile_begin);
+                const int m_tile = local / L.n_tiles;
+                const int n_tile = local - m_tile * L.n_tiles;
+                const int64_t m0 = static_cast<int64_t>(m_tile) * kBM;
+                const int n0 = n_tile * kBN;
+                const int nk = (L.d_in + kBK - 1) / kBK;
+                const int b = jj & 1;
+                if (jj >= 2) {
+                    wait_idle(&acc_empty[b], ((jj >> 1) - 1) & 1, 111);
+                    tc_fence_after();
+                }
+                if (warp == 0 && lane == 0) {
+                    const CUtensorMap* tmx = &T.tmx[l];
+                    const CUtensorMap* tmw = &T.tmw[l];
+                    for (int kb = 0; kb < nk; ++kb, ++kc_prod) {
+                        const int st = kc_prod % kPStages;
+                        if (kc_prod >= kPStages && !wait(&empty[st], ((kc_prod / kPStages) - 1) & 1, 112))
+                            break;
+                        uint8_t* a = smem + st * kPStageBytes;
+                        mbar_arrive_expect_tx(&full[st], kPStageBytes);
+                        tma_load_2d(a, tmx, &full[st], kb * kBK, static_cast<int32_t>(m0));
+                        tma_load_2d(a + kABytes, tmw, &full[st], kb * kBK, n0);
+                    }
+                } else if (warp == 1 && lane == 0) {
+                    constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, 0, 0);
+                    const uint32_t acc = tmem + static_cast<uint32_t>(b * kTmemCols);
+                    for (int kb = 0; kb < nk; ++kb, ++kc_mma) {
+                        const int st = kc_mma % kPStages;
+                        if (!wait(&full[st], (kc_mma / kPStages) & 1, 113)) break;
+                        tc_fence_after();
+                        const uint32_t a_addr = smem_u32(smem + st * kPStageBytes);
+                        const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+                        for (int kk = 0; kk < kBK / 16; ++kk) {
+                            const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
+                            const uint64_t bd = sdesc_sw128(b_addr + kk * 32, 16, 1024);
+                            umma_bf16(acc, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        }
+                        umma_commit(&empty[st]);
+                    }
+                    umma_commit(&acc_full[b]);
+                }
+                // s_e = kKappa sigma (y - u) in place, each channel quad as (e0, e2, e1, e3);
+                // u is read one chunk ahead
+                if (warp == 1 && lane == 0)
+                    wait(&acc_full[b], (jj >> 1) & 1, 114);
+                else
+                    wait_idle(&acc_full[b], (jj >> 1) & 1, 114);
+                __syncwarp();
+                tc_fence_after();
+                const int64_t t = m0 + row;
+                const bool valid = t < N;
+                const uint32_t trow = trow0 + static_cast<uint32_t>(b * kTmemCols);
+                const int nchunks = min(kBN, L.d_out - n0) / 16;
+                const uint4* up = reinterpret_cast<const uint4*>(L.u + (valid ? t * L.d_out + n0 : 0));
+                uint4 un0 = make_uint4(0u, 0u, 0u, 0u), un1 = un0;
+                if (valid) {
+                    un0 = __ldg(up);
+                    un1 = __ldg(up + 1);
+                }
+                for (int c = 0; c < nchunks; ++c) {
+                    float v[16];
+                    tmem_ld16(trow + c * 16, v);
+                    const uint4 uc0 = un0, uc1 = un1;
+                    if (valid && c + 1 < nchunks) {
+                        un0 = __ldg(up + 2 * (c + 1));
+                        un1 = __ldg(up + 2 * (c + 1) + 1);
+                    }
+                    tmem_wait_ld();
+                    float uf[16];
+                    unpack_bf16x8(uc0, uf);
+                    unpack_bf16x8(uc1, uf + 8);
+                    float w[16];
+#pragma unroll
+                    for (int j = 0; j < 16; j += 4) {
+                        w[j] = valid ? T.sigma_k * (v[j] - uf[j]) : 0.f;
+                        w[j + 1] = valid ? T.sigma_k * (v[j + 2] - uf[j + 2]) : 0.f;
+                        w[j + 2] = valid ? T.sigma_k * (v[j + 1] - uf[j + 1]) : 0.f;
+                        w[j + 3] = valid ? T.sigma_k * (v[j + 3] - uf[j + 3]) : 0.f;
+                    }
+                    tmem_st16(trow + c * 16, w);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&se_ready[b]);
+            }
+        } else {
+            // ------------------------------------------------------------ noise warps
+            const int gi = (warp - 4) >> 2;
+            const int lq = warp & 3;
+            const int row = lq * 32 + lane;
+            const uint32_t trow0 = tmem + (static_cast<uint32_t>(lq * 32) << 16);
+            const F2 mh{-T.h_lg2, -T.h_lg2};
+            for (int jj = 0; jj < nt; ++jj) {
+                const int64_t gt = tile_first + jj;
+                while (l + 1 < T.n_layers && gt >= T.layer[l + 1].tile_begin) ++l;
+                const FwdLayer& L = T.layer[l];
+                const int local = static_cast<int>(gt - L.tile_begin);
+                const int m_tile = local / L.n_tiles;
+                const int n_tile = local - m_tile * L.n_tiles;
+                const int64_t t = static_cast<int64_t>(m_tile) * kBM + row;
+                const bool valid = t < N;
+                const int n0 = n_tile * kBN;
+                const int nchunks = min(kBN, L.d_out - n0) / 16;
+                const int half_chunks = (nchunks + 1) / 2;
+                const int b = jj & 1;
+                const uint32_t trow = trow0 + static_cast<uint32_t>(b * kTmemCols);
+                const uint32_t tg = T.key.token_offset + static_cast<uint32_t>(t);
+                const uint32_t qbase = static_cast<uint32_t>(n0 >> 2) + T.key.quad_offset;
+                // this group's units of the tile: u in [max(ub, gt U), min(ue, (gt + 1) U)) with
+                // (u - ub) % 7 == gi
+                const int64_t lo = max(ub, gt * U), hi = min(ue, (gt + 1) * U);
+                const int64_t first = lo + (gi - (lo - ub) % kPNoiseGroups + kPNoiseGroups) % kPNoiseGroups;
+                wait(&se_ready[b], (jj >> 1) & 1, 115);
+                tc_fence_after();
+                for (int64_t u = first; u < hi; u += kPNoiseGroups) {
+                    const int unit = static_cast<int>(u - gt * U);
+                    const int i = unit >> 1;
+                    const int hf = unit & 1;
+                    const uint32_t di = T.key.draw_offset + static_cast<uint32_t>(i);
+                    F2 acc[2] = {{0.f, 0.f}, {0.f, 0.f}};
+                    const int c_end = hf ? nchunks : half_chunks;
+                    for (int c = hf ? half_chunks : 0; c < c_end; ++c) {
+#pragma unroll
+                        for (int piece = 0; piece < 2; ++piece) {
+                            float se[8];
+                            tmem_ld8(trow + c * 16 + piece * 8, se);
+                            tmem_wait_ld8(se);
+#pragma unroll
+                            for (int qq = 0; qq < 2; ++qq) {
+                                const PolarPairs z = normal_quad_pairs(qbase + c * 4 + piece * 2 + qq,
+                                                                       tg, di, L.layer_id, T.key);
+                                const F2 lc = fma2(z.s, F2{se[4 * qq + 2], se[4 * qq + 3]},
+                                                   mul2(z.c, F2{se[4 * qq + 0], se[4 * qq + 1]}));
+                                acc[qq] = fma2(z.nq, lc, acc[qq]);
+                                acc[qq] = fma2(mh, z.L, acc[qq]);
+                            }
+                        }
+                    }
+                    if (valid)
+                        L.partial[((static_cast<int64_t>(n_tile) * 2 + hf) * K + i) * N + t] =
+                            (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[b]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 2 * kTmemCols);
+}
+
+// dloss[i][t] = the sum over the 2 n_tiles unit partials of (draw i, token t), in order.
+template <int kMax>
+__global__ void __launch_bounds__(256) fwd_reduce_kernel(const __grid_constant__ FwdTable<kMax> T) {
+    const FwdLayer& L = T.layer[blockIdx.y];
+    const int64_t total = static_cast<int64_t>(T.K) * T.N;
+    const int parts = 2 * L.n_tiles;
+    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int i = static_cast<int>(idx / T.N);
+        const int64_t t = idx - static_cast<int64_t>(i) * T.N;
+        const float* p = L.partial + static_cast<int64_t>(i) * T.N + t;
+        const int64_t stride = static_cast<int64_t>(T.K) * T.N;
+        float s = 0.f;
+        for (int pp = 0; pp < parts; ++pp) s += __ldcs(p + pp * stride);
+        L.dloss[static_cast<int64_t>(i) * L.ld + t] = s;
+    }
+}
+
+template <int kMax>
+dust_status launch_persistent(const FwdLayerArgs* layers, int n, int64_t N, int K, float sigma,
+                              const NoiseKey& key, char* ws, cudaStream_t s) {
+    FwdTable<kMax> T;  // copied into the launch's parameter space
+    T.ew = device_error_word();
+    T.N = N;
+    T.n_layers = n;
+    T.m_tiles = static_cast<int>((N + kBM - 1) / kBM);
+    T.K = K;
+    T.sigma_k = kKappa * sigma;
+    T.h_lg2 = static_cast<float>(0.69314718055994531 * sigma * sigma);
+    T.key = key;
+    T.n_full = 0;
+    T.split = 1;
+    int64_t tiles = 0;
+    size_t off = 0;
+    for (int l = 0; l < n; ++l) {
+        const FwdLayerArgs& a = layers[l];
+        if (!make_tmap_bf16_2d(&T.tmx[l], a.x, static_cast<uint64_t>(N), a.d_in, kBM, kBK) ||
+            !make_tmap_bf16_2d(&T.tmw[l], a.W, static_cast<uint64_t>(a.d_out), a.d_in, kBN, kBK))
+            return DUST_ERR_CUDA;
+        FwdLayer& L = T.layer[l];
+        const int n_tiles = (a.d_out + kBN - 1) / kBN;
+        L.u = static_cast<const __nv_bfloat16*>(a.u);
+        L.partial = reinterpret_cast<float*>(ws + off);
+        L.counters = nullptr;
+        L.dloss = a.dloss;
+        L.ld = a.ld;
+        L.d_in = a.d_in;
+        L.d_out = a.d_out;
+        L.n_tiles = n_tiles;
+        L.tile_begin = static_cast<int>(tiles);
+        L.layer_id = a.layer_id;
+        tiles += static_cast<int64_t>(n_tiles) * T.m_tiles;
+        if (tiles > 2147483647LL) return DUST_ERR_UNSUPPORTED;
+        off += bf16_layer_ws(N, a.d_out, K);
+    }
+    T.total_tiles = tiles;
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !attr_done[dev]) {
+        if (cudaFuncSetAttribute(fwd_persistent_kernel<kMax>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kPSmemBytes) != cudaSuccess)
+            return DUST_ERR_CUDA;
+        if (dev < 64) attr_done[dev] = true;
+    }
+    const int64_t grid = std::min<int64_t>(num_sms(), tiles * 2 * K);
+    prof_begin(s);
+    fwd_persistent_kernel<kMax><<<static_cast<unsigned>(grid), kPThreads, kPSmemBytes, s>>>(T);
+    prof_end(s, kMax == 1 ? "fwd_bf16_noise_loss" : "fwd_bf16_noise_loss_grouped");
+    const int64_t outs = static_cast<int64_t>(K) * N;
+    prof_begin(s);
+    fwd_reduce_kernel<kMax><<<dim3(static_cast<unsigned>(std::min<int64_t>((outs + 255) / 256,
+                                                                           num_sms() * 8LL)),
+                                   static_cast<unsigned>(n)),
+                              256, 0, s>>>(T);
+    prof_end(s, kMax == 1 ? "fwd_reduce_partials" : "fwd_reduce_partials_grouped");
+    return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------------------ fp32 path
@@ -498,13 +809,13 @@ size_t fwd_workspace_bytes(dust_dtype dt, int64_t N, int32_t d_out, int32_t K) {
     return align_up(static_cast<size_t>(n_cb * K * N) * 4, 256);
 }
 
-void fwd_tiling(const int32_t* d_out, int n, int64_t N, int32_t K, int64_t slots, int32_t* width,
-                int32_t* split) {
+void fwd_plan(const int32_t* d_out, int n, int64_t N, int32_t K, int64_t sms, int32_t* persistent,
+              int32_t* split) {
     std::vector<FwdLayerArgs> a(static_cast<size_t>(n), FwdLayerArgs{});
     for (int l = 0; l < n; ++l) a[l].d_out = d_out[l];
-    const Tiling t = choose_tiling(a.data(), n, N, K, slots);
-    *width = t.width;
-    *split = t.split;
+    const FwdPlan p = plan_forward(a.data(), n, N, K, sms);
+    *persistent = p.persistent ? 1 : 0;
+    *split = p.split;
 }
 
 size_t fwd_grouped_workspace_bytes(const FwdLayerArgs* layers, int n, int64_t N, int32_t K) {
@@ -529,7 +840,7 @@ dust_status fwd_launch(const void* x, const void* W, const void* u, dust_dtype d
                        int32_t d_in, int32_t d_out, int32_t K, float sigma, NoiseKey key,
                        float* dloss, int64_t ld, void* ws, cudaStream_t s) {
     if (dt == DUST_BF16) {
-        const int64_t tiles = (N + kBM - 1) / kBM * ((d_out + kMinBN - 1) / kMinBN);
+        const int64_t tiles = (N + kBM - 1) / kBM * ((d_out + kBN - 1) / kBN);
         if (tiles > 2147483647LL) return DUST_ERR_UNSUPPORTED;
         FwdLayerArgs a{x, W, u, d_in, d_out, key.layer, dloss, ld};
         return launch_bf16<1>(&a, 1, N, K, sigma, key, static_cast<char*>(ws), s);

@@ -65,10 +65,10 @@ size_t fwd_grouped_workspace_bytes(const FwdLayerArgs* layers, int n, int64_t N,
 dust_status fwd_grouped_launch(const FwdLayerArgs* layers, int n, int64_t N, int32_t K,
                                float sigma, NoiseKey key, void* ws, cudaStream_t s);
 size_t fwd_workspace_bytes(dust_dtype dt, int64_t N, int32_t d_out, int32_t K);
-// The bf16 forward's tile width and tail split for layers of these widths on `slots` CTA slots
-// (host only).
-void fwd_tiling(const int32_t* d_out, int n, int64_t N, int32_t K, int64_t slots, int32_t* width,
-                int32_t* split);
+// The bf16 forward's form (persistent or one tile per CTA) and tail split for layers of these
+// widths on `sms` SMs (host only).
+void fwd_plan(const int32_t* d_out, int n, int64_t N, int32_t K, int64_t sms, int32_t* persistent,
+              int32_t* split);
 dust_status fwd_launch(const void* x, const void* W, const void* u, dust_dtype dt, int64_t N,
                        int32_t d_in, int32_t d_out, int32_t K, float sigma, NoiseKey key,
                        float* dloss, int64_t ld, void* ws, cudaStream_t s);
