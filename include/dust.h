@@ -237,8 +237,8 @@ dust_status dust_weight_grad(const float* r, int64_t ld_r, const void* x, dust_d
  * every device that loads the library holds until the process exits.  The call allocates
  * nothing (no cudaMalloc, no allocating library routine).
  *   - Sizes whose scratch (dust_workspace_size(DUST_OP_CREDIT, ...)) exceeds 4 MiB are
- *     rejected with DUST_ERR_WORKSPACE; the scratch is about 12 K + 16 bytes per 128 tokens
- *     (K <= 128), so K = 32 allows N up to about 1.34 million tokens and K = 64 about 680,000.
+ *     rejected with DUST_ERR_WORKSPACE; the scratch is 16 K bytes per 128 tokens plus 256
+ *     (K <= 128), so K = 32 allows N up to about 1.05 million tokens and K = 64 about 520,000.
  *   - The first call on a device looks up the array's device address (once per device, with
  *     that device current); make that first call before any stream capture.
  *   - Every call shares the one array, and the ticket and flags are cleared on `stream` before
