@@ -324,6 +324,15 @@ def test_weight_grad_f32_matches_oracle():
     _dev.assert_fp32_close(GW, GW_ref, "G_W f32")
 
 
+def test_weight_grad_f32_odd_quad_count_matches_oracle():
+    # d_out = 36: nine channel quads per token, so the last thread of every row owns one quad
+    L = workloads.custom_layer(4, 77, 40, 36, "f32", None)
+    key = z.NoiseKey(0x5EED0004, layer_id=2, draw_offset=5, token_offset=9)
+    GW, g, GW_ref, g_ref = _wgrad_case(L, 5, 7, 1e-2, key, 91, "f32")
+    _dev.assert_fp32_close(g, g_ref, "g f32, odd quad count")
+    _dev.assert_fp32_close(GW, GW_ref, "G_W f32, odd quad count")
+
+
 def test_weight_grad_accumulates_draw_chunks():
     """Two chunks (draw offsets 0 and K1) with accumulate give the full-population G_W."""
     import torch

@@ -1,10 +1,10 @@
 // Output-error estimate and weight estimate (Dust review page, section "신용 할당":
 // g_t = -(1/(K sigma)) sum_i r_t^(i) a_t^(i) and G_W = sum_t g_t x_t^T).
 //
-// Stage 1 (ghat_kernel): one thread per (token, channel quad) regenerates the quad's normals
-// for every draw and accumulates the reward-weighted sum; g is written as bf16 (the tensor
-// core operand) and optionally as fp32.  A grid-stride loop over units of 128 consecutive
-// (token, quad) pairs of a layer keeps every SM busy to the end.
+// Stage 1 (ghat_kernel): one thread per (token, two channel quads) regenerates the quads'
+// normals for every draw and accumulates the reward-weighted sum; g is written as bf16 (the
+// tensor core operand) and optionally as fp32.  A grid-stride loop over units of 128
+// consecutive (token, quad pair) items of a layer keeps every SM busy to the end.
 // Stage 2 (gw_bf16_kernel): G_W = g^T x on the tensor cores.  Both operands are MN-major
 // (tokens are the contraction index and the slow index of g [N, d_out] and x [N, d_in]):
 // TMA loads 64-token x 64-element boxes with 128-byte swizzle, one thread issues
@@ -31,8 +31,8 @@ struct GhatLayer {
     __nv_bfloat16* gb;  // [N, d_out] or null
     float* gf;          // [N, d_out] or null
     int64_t ld_r, unit_begin;
-    int64_t n_flat;  // N * d_out / 4: (token, channel quad) pairs, token-major
-    uint64_t nq_magic;  // div_magic(d_out / 4)
+    int64_t n_flat;  // N * ceil(d_out / 8): (token, pair of channel quads) items, token-major
+    uint64_t np_magic;  // div_magic(ceil(d_out / 8))
     int d_out;
     uint32_t layer_id;
 };
@@ -46,47 +46,61 @@ struct GhatTable {
     NoiseKey key;
 };
 
+// Each thread owns one token and two consecutive channel quads (the second absent at the end
+// of a row with an odd number of quads), so the credit of a draw is loaded once for eight
+// channels and the two quads' Philox chains interleave.  (Unrolling the draws as well spills
+// at 64 registers; two quads at 53 registers beat one quad with four draws unrolled by 3-7%.)
 template <int kMax>
 __global__ void __launch_bounds__(kGThreads, 8) ghat_kernel(const __grid_constant__ GhatTable<kMax> T) {
     int l = 0;
     for (int64_t u = blockIdx.x; u < T.total_units; u += gridDim.x) {
         while (l + 1 < T.n_layers && u >= T.layer[l + 1].unit_begin) ++l;
         const GhatLayer& L = T.layer[l];
-        // a unit is 128 consecutive (token, quad) pairs, so no lane idles when d_out / 4 is
-        // not a multiple of 128
+        // a unit is 128 consecutive (token, quad pair) items, so no lane idles when the row's
+        // pair count is not a multiple of 128
         const int64_t f = (u - L.unit_begin) * kGThreads + threadIdx.x;
         if (f >= L.n_flat) continue;
         const int nq = L.d_out >> 2;
-        const int64_t t = div_by_magic(f, nq, L.nq_magic);
-        const int q = static_cast<int>(f - t * nq);
+        const int np = (nq + 1) >> 1;
+        const int64_t t = div_by_magic(f, np, L.np_magic);
+        const int q = 2 * static_cast<int>(f - t * np);
+        const bool two = q + 1 < nq;
         const uint32_t tg = T.key.token_offset + static_cast<uint32_t>(t);
-        // channel pairs (4q, 4q+2) and (4q+1, 4q+3): the lanes of packed f32x2 operations
-        F2 a02{0.f, 0.f}, a13{0.f, 0.f};
+        const uint32_t qg = static_cast<uint32_t>(q) + T.key.quad_offset;
+        // per quad, channel pairs (4q, 4q+2) and (4q+1, 4q+3): the lanes of packed f32x2 operations
+        F2 a02{0.f, 0.f}, a13{0.f, 0.f}, b02{0.f, 0.f}, b13{0.f, 0.f};
         const float* rt = L.r + t;
-        // unrolled so that independent Philox chains of consecutive draws interleave
-#pragma unroll 4
+#pragma unroll 1
         for (int i = 0; i < T.K; ++i) {
             const float ri = __ldg(rt + static_cast<int64_t>(i) * L.ld_r);
-            const PolarPairs z = normal_quad_pairs(static_cast<uint32_t>(q) + T.key.quad_offset, tg,
-                                                   T.key.draw_offset + static_cast<uint32_t>(i),
-                                                   L.layer_id, T.key);
+            const uint32_t di = T.key.draw_offset + static_cast<uint32_t>(i);
+            const PolarPairs z = normal_quad_pairs(qg, tg, di, L.layer_id, T.key);
+            const PolarPairs w = normal_quad_pairs(qg + 1, tg, di, L.layer_id, T.key);
             // r a = kKappa (r nq) (cos, sin) per pair; kKappa is applied with the scale
-            const F2 rr{ri * z.nq.x, ri * z.nq.y};
-            a02 = fma2(rr, z.c, a02);
-            a13 = fma2(rr, z.s, a13);
+            const F2 rz{ri * z.nq.x, ri * z.nq.y};
+            const F2 rw{ri * w.nq.x, ri * w.nq.y};
+            a02 = fma2(rz, z.c, a02);
+            a13 = fma2(rz, z.s, a13);
+            b02 = fma2(rw, w.c, b02);
+            b13 = fma2(rw, w.s, b13);
         }
         const float sk = T.scale * kKappa;
-        const float a0 = a02.x * sk, a1 = a13.x * sk, a2 = a02.y * sk, a3 = a13.y * sk;
+        const float4 ga = make_float4(a02.x * sk, a13.x * sk, a02.y * sk, a13.y * sk);
+        const float4 gb = make_float4(b02.x * sk, b13.x * sk, b02.y * sk, b13.y * sk);
         const int64_t off = t * L.d_out + 4 * q;
         if (L.gb) {
-            __nv_bfloat162 lo = __floats2bfloat162_rn(a0, a1);
-            __nv_bfloat162 hi = __floats2bfloat162_rn(a2, a3);
-            uint2 v;
-            v.x = *reinterpret_cast<uint32_t*>(&lo);
-            v.y = *reinterpret_cast<uint32_t*>(&hi);
-            *reinterpret_cast<uint2*>(L.gb + off) = v;
+            __nv_bfloat162 h[4] = {__floats2bfloat162_rn(ga.x, ga.y), __floats2bfloat162_rn(ga.z, ga.w),
+                                   __floats2bfloat162_rn(gb.x, gb.y), __floats2bfloat162_rn(gb.z, gb.w)};
+            const uint32_t* hv = reinterpret_cast<const uint32_t*>(h);
+            if (two)
+                *reinterpret_cast<uint4*>(L.gb + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+            else
+                *reinterpret_cast<uint2*>(L.gb + off) = make_uint2(hv[0], hv[1]);
         }
-        if (L.gf) *reinterpret_cast<float4*>(L.gf + off) = make_float4(a0, a1, a2, a3);
+        if (L.gf) {
+            *reinterpret_cast<float4*>(L.gf + off) = ga;
+            if (two) *reinterpret_cast<float4*>(L.gf + off + 4) = gb;
+        }
     }
 }
 
@@ -374,8 +388,8 @@ dust_status launch_bf16_tables(const WgradLayerArgs* layers, int n, int64_t N, i
         L.gb = reinterpret_cast<__nv_bfloat16*>(ws + off);
         L.gf = a.g_out;
         L.d_out = a.d_out;
-        L.n_flat = N * (a.d_out / 4);
-        L.nq_magic = div_magic(a.d_out / 4);
+        L.n_flat = N * ((a.d_out / 4 + 1) / 2);
+        L.np_magic = div_magic((a.d_out / 4 + 1) / 2);
         L.unit_begin = units;
         L.layer_id = a.layer_id;
         units += (L.n_flat + kGThreads - 1) / kGThreads;
@@ -506,7 +520,8 @@ dust_status wgrad_launch(const float* r, int64_t ld_r, const void* x, dust_dtype
     G.K = K_chunk;
     G.scale = -1.0f / (static_cast<float>(K_total) * sigma);
     G.key = key;
-    G.layer[0] = GhatLayer{r, nullptr, gf, ld_r, 0, N * (d_out / 4), div_magic(d_out / 4), d_out, key.layer};
+    G.layer[0] = GhatLayer{r, nullptr, gf, ld_r, 0, N * ((d_out / 4 + 1) / 2),
+                           div_magic((d_out / 4 + 1) / 2), d_out, key.layer};
     G.total_units = (G.layer[0].n_flat + kGThreads - 1) / kGThreads;
     const int64_t max_blocks = static_cast<int64_t>(num_sms()) * 16;
     prof_begin(s);
