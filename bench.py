@@ -51,8 +51,8 @@ OPS_PER_NORMAL = {"fwd_bf16_noise_loss": 20.0, "ghat_reduce_draws": 19.0,
 MEASURED_TRAFFIC = {
     ("fwd_bf16_noise_loss", "gpt2s-mlp-win-768x3072"): (68.49e6 + 2.45e6,
                                                        "profiles/ncu_full_fwd_persistent_gpt2s_mlp_win_768x3072.md"),
-    ("ghat_reduce_draws", "gpt2s-mlp-win-768x3072"): (0.54e6 + 0.49e6,
-                                                     "profiles/ncu_full_fwd_persistent_gpt2s_mlp_win_768x3072.md"),
+    ("lmhead_ce_noise", "head-4096-slab1024"): (33.85e6 + 75.21e6,
+                                                "profiles/ncu_full_lmhead_head-4096-slab1024.md"),
 }
 HEAD_METRIC = "Dust LM-head estimator tokens*draws/s"
 ATTN_METRIC = "Dust attention-reward estimator tokens*draws/s"
