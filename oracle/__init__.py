@@ -51,6 +51,9 @@ def lib():
         L.oracle_uniform.restype = ctypes.c_double
         L.oracle_philox_batch.argtypes = [_c_u32p, ctypes.c_int64, ctypes.c_uint64, _c_u32p,
                                           _c_f64p]
+        L.oracle_normal_stats.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32,
+                                          ctypes.c_int64, ctypes.c_int32, ctypes.c_double,
+                                          ctypes.c_double, _c_f64p, _c_i64p]
         L.oracle_normal_quad.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32,
                                          ctypes.c_uint32, ctypes.c_uint32, _c_f64p]
         L.oracle_noisy_linear_loss.argtypes = [
@@ -136,6 +139,17 @@ def philox_batch(ctr: np.ndarray, seed: int, want_normals: bool = True):
     lib().oracle_philox_batch(_p(c, _c_u32p), n, int(seed), _p(words, _c_u32p),
                               _p(normals, _c_f64p))
     return words, normals
+
+
+def normal_stats(seed: int, draw: int, layer: int, n_blocks: int, n_bins: int, lo: float,
+                 hi: float):
+    """(sum z, sum z^2) and the histogram [n_bins + 2] (under, bins of [lo, hi), over) of the
+    4 n_blocks normals of counters (j mod 1024, j / 1024, draw, layer), streamed."""
+    sums = np.zeros(2, dtype=np.float64)
+    hist = np.zeros(n_bins + 2, dtype=np.int64)
+    lib().oracle_normal_stats(int(seed), draw, layer, int(n_blocks), int(n_bins), float(lo),
+                              float(hi), _p(sums, _c_f64p), _p(hist, _c_i64p))
+    return sums, hist
 
 
 def noise(seed: int, layer_id: int, N: int, d_out: int, K: int, draw_offset: int = 0,

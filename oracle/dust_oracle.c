@@ -115,6 +115,49 @@ void oracle_normal_quad(uint64_t seed, uint32_t q, uint32_t t, uint32_t i, uint3
     oracle_box_muller4(w, z);
 }
 
+/* Streaming statistics of the generator's normals, for the distribution pins at sizes whose
+ * samples would not fit in memory: blocks j = 0 .. n_blocks-1 with counter
+ * (j mod 1024, j / 1024, draw, layer) give 4 n_blocks normals.  sums[0] = sum z, sums[1] =
+ * sum z^2; hist[0] counts z < lo, hist[1 + b] counts z in bin b of n_bins equal bins of
+ * [lo, hi), hist[n_bins + 1] counts z >= hi. */
+void oracle_normal_stats(uint64_t seed, uint32_t draw, uint32_t layer, int64_t n_blocks,
+                         int32_t n_bins, double lo, double hi, double* sums, int64_t* hist)
+{
+    const double scale = (double)n_bins / (hi - lo);
+    sums[0] = 0.0;
+    sums[1] = 0.0;
+    memset(hist, 0, sizeof(int64_t) * (size_t)(n_bins + 2));
+#pragma omp parallel
+    {
+        int64_t* h = calloc((size_t)(n_bins + 2), sizeof(int64_t));
+        double s1 = 0.0, s2 = 0.0;
+#pragma omp for schedule(static)
+        for (int64_t j = 0; j < n_blocks; ++j) {
+            double z[4];
+            oracle_normal_quad(seed, (uint32_t)(j % 1024), (uint32_t)(j / 1024), draw, layer, z);
+            for (int k = 0; k < 4; ++k) {
+                s1 += z[k];
+                s2 += z[k] * z[k];
+                int64_t b;
+                if (z[k] < lo) b = 0;
+                else if (z[k] >= hi) b = n_bins + 1;
+                else {
+                    b = 1 + (int64_t)floor((z[k] - lo) * scale);
+                    if (b > n_bins) b = n_bins;
+                }
+                h[b] += 1;
+            }
+        }
+#pragma omp critical
+        {
+            sums[0] += s1;
+            sums[1] += s2;
+            for (int32_t b = 0; b < n_bins + 2; ++b) hist[b] += h[b];
+        }
+        free(h);
+    }
+}
+
 /* Batch of Philox blocks for arbitrary counters (n x 4 words in, n x 4 words and normals out). */
 void oracle_philox_batch(const uint32_t* ctr, int64_t n, uint64_t seed, uint32_t* words,
                          double* normals)

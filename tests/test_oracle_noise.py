@@ -2,11 +2,12 @@
 
 The Dust page (koala.ai.kr, "Dust: 역전파 없이 트랜스포머를 사전학습하다", section "신용 할당")
 only fixes a_t ~ N(0, I), independent per token and draw.  The generator is Philox4x32-10
-(Salmon et al., SC'11) with Box-Muller.  Philox words are pinned by cross-implementation
-against PyTorch's header-only CPU engine (called, not copied); the published known-answer
-vectors are not available in this environment.  Normals are pinned by exact invariants of
-Box-Muller and by distribution tests.
+(Salmon et al., SC'11) with Box-Muller.  Philox words are pinned by the published
+known-answer vectors (tests/golden/philox_kat.json) and by cross-implementation against
+PyTorch's header-only CPU engine (called, not copied).  Normals are pinned by exact invariants
+of Box-Muller and by distribution tests.
 """
+import json
 import math
 import os
 import subprocess
@@ -34,6 +35,26 @@ def torch_philox(tmp_path_factory):
         return np.array([[int(v) for v in ln.split()] for ln in out.stdout.strip().splitlines()],
                         dtype=np.uint64).astype(np.uint32)
     return run
+
+
+def kat_vectors():
+    """The published Philox4x32-10 known-answer vectors: [(ctr[4], key[2], out[4])]."""
+    with open(os.path.join(HERE, "golden", "philox_kat.json")) as f:
+        d = json.load(f)
+    return [(np.array([int(v, 16) for v in e["ctr"]], dtype=np.uint32),
+             np.array([int(v, 16) for v in e["key"]], dtype=np.uint32),
+             np.array([int(v, 16) for v in e["out"]], dtype=np.uint32)) for e in d["vectors"]]
+
+
+def test_philox_words_match_published_known_answers():
+    vecs = kat_vectors()
+    assert len(vecs) == 3
+    for ctr, key, out in vecs:
+        assert np.array_equal(oracle.philox4x32_10(ctr, key), out), (ctr, key)
+        # the batch route under the 64-bit seed (key0 = low word, key1 = high word)
+        seed = int(key[0]) | (int(key[1]) << 32)
+        words, _ = oracle.philox_batch(ctr.reshape(1, 4), seed, want_normals=False)
+        assert np.array_equal(words[0], out)
 
 
 def test_philox_words_match_independent_implementation(torch_philox):
@@ -106,6 +127,27 @@ def test_normals_distribution():
     c = np.corrcoef(z.T)
     assert np.max(np.abs(c - np.eye(4))) < 5.0 / math.sqrt(n_blocks)
     assert np.max(np.abs(flat)) <= math.sqrt(2 * 24 * math.log(2)) + 1e-12
+
+
+def test_normals_distribution_at_2_28():
+    """2^28 normals, streamed: |mean| < 5/sqrt(n), variance within 5 standard errors of 1, and
+    the Kolmogorov-Smirnov distance to the standard normal CDF, evaluated at the 2^16 + 1 edges
+    of a histogram over [-6, 6) (a lower bound of the exact distance), below the 1e-3 critical
+    value 1.9495/sqrt(n)."""
+    from scipy import special
+    n_blocks, n_bins, lo, hi = 1 << 26, 1 << 16, -6.0, 6.0
+    sums, hist = oracle.normal_stats(0x5EED0002, 3, 1, n_blocks, n_bins, lo, hi)
+    n = 4 * n_blocks
+    assert int(hist.sum()) == n
+    mean = sums[0] / n
+    var = sums[1] / n - mean * mean
+    assert abs(mean) < 5.0 / math.sqrt(n), mean
+    assert abs(var - 1.0) < 5.0 * math.sqrt(2.0 / n), var
+    edges = np.linspace(lo, hi, n_bins + 1)
+    F = np.cumsum(hist)[: n_bins + 1] / n
+    D = float(np.max(np.abs(F - special.ndtr(edges))))
+    assert D < 1.9495 / math.sqrt(n), D
+    assert hist[0] == 0 and hist[-1] == 0          # |z| <= sqrt(48 ln 2) = 5.77 < 6
 
 
 def test_noise_mapping_channels_tokens_draws_layers():
