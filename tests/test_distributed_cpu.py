@@ -72,6 +72,34 @@ def _worker(rank, world, port, mode, q):
             q.put((rank, float(max(np.abs(pt.numpy() - whole).max() / np.abs(whole).max(),
                                    np.linalg.norm(G - Gw) / np.linalg.norm(Gw)))))
             return
+        if mode == "stack":
+            # a stack of layers of different shapes: each rank's partial weight estimates
+            # go into one flat buffer, summed over ranks in buckets of consecutive layers
+            shapes = [(12, 16), (16, 8), (8, 24), (24, 12), (12, 12)]   # (d_in, d_out)
+            lays = [workloads.custom_layer(40 + l, 600, di, do, "f32", None, layer_id=l)
+                    for l, (di, do) in enumerate(shapes)]
+            layout, total = zd.flat_layout([(do, di) for di, do in shapes])
+            t0, t1, cu_local = zd.local_problem(cu, world, rank)
+            flat = torch.zeros(total, dtype=torch.float64)
+            for l, Ll in enumerate(lays):
+                res = oracle.dust_layer(Ll.x_f64[t0:t1], Ll.W_f64, Ll.u_f64[t0:t1], K, sigma,
+                                        gamma, cu_local, seed, layer_id=l, token_offset=t0)
+                o, m = layout[l]
+                flat[o:o + m] = torch.from_numpy(res["G_W"].reshape(-1))
+            plan = zd.plan_buckets([m for _, m in layout], 3)
+            covered = [l for a, b in plan for l in range(a, b)]
+            assert covered == list(range(len(lays))), plan
+            for bucket in plan:
+                zd.allreduce_bucket(flat, layout, bucket)
+            err = 0.0
+            for l, Ll in enumerate(lays):
+                whole = oracle.dust_layer(Ll.x_f64, Ll.W_f64, Ll.u_f64, K, sigma, gamma, cu, seed,
+                                          layer_id=l)["G_W"]
+                o, m = layout[l]
+                got = flat[o:o + m].numpy().reshape(whole.shape)
+                err = max(err, float(np.linalg.norm(got - whole) / np.linalg.norm(whole)))
+            q.put((rank, err))
+            return
         if mode == "mismatch":
             try:
                 zd.check_same_problem(seed=seed + rank, K=K)
@@ -137,6 +165,30 @@ def test_rank_leaving_before_the_collective_fails_the_others():
     out = _run("dead")
     assert out[1] == "left"
     assert isinstance(out[0], str) and out[0].startswith("collective failed"), out[0]
+
+
+def test_flat_layout_and_bucket_plan():
+    layout, total = zd.flat_layout([(2304, 768), (768, 768), (3072, 768), (768, 3072)] * 12)
+    assert all(o % 64 == 0 for o, _ in layout)              # 256-byte aligned views
+    assert all(a[0] + a[1] <= b[0] for a, b in zip(layout, layout[1:]))
+    assert total >= layout[-1][0] + layout[-1][1]
+    sizes = [m for _, m in layout]
+    for nb in (1, 2, 3, 4, 7, 48, 100):
+        plan = zd.plan_buckets(sizes, nb)
+        assert [l for a, b in plan for l in range(a, b)] == list(range(48))
+        assert len(plan) == min(nb, 48)
+    per = [sum(sizes[a:b]) for a, b in zd.plan_buckets(sizes, 4)]
+    assert max(per) <= 1.2 * sum(sizes) / 4                 # whole blocks: even buckets
+    a, b = zd.bucket_span(layout, (12, 24))
+    assert a == layout[12][0] and b == layout[23][0] + layout[23][1]
+    assert zd.plan_buckets([], 3) == [] and zd.plan_buckets([5, 1], 9) == [(0, 1), (1, 2)]
+
+
+def test_two_ranks_stack_bucketed_sum_equals_whole_batch():
+    out = _run("stack")
+    assert set(out) == {0, 1}
+    for r, err in out.items():
+        assert isinstance(err, float) and err < 1e-10, (r, err)
 
 
 def test_two_ranks_spsa_exchange_only_probe_scalars():

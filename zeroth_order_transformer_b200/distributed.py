@@ -3,7 +3,9 @@
 The estimator shards by tokens.  Each rank takes whole sequences (the credit scan never
 crosses a sequence end), generates the noise of its tokens with their GLOBAL index
 (token_offset), so no noise and no loss is ever exchanged.  The only exchange is the sum
-of the partial weight estimates G_W over ranks: one all-reduce per layer.  This follows the
+of the partial weight estimates G_W over ranks: one all-reduce per layer, or, for a stack of
+layers, one per bucket of consecutive layers issued while the later buckets are still being
+estimated.  This follows the
 pages' remark that zeroth-order training needs to share only seeds and scalars
 (gist.science 2605.15622, seed-based communication; gist.science 2502.10239, seed and scalar
 upload), and the weight-estimate equation of the Dust page (G_W = sum over ALL tokens).
@@ -65,6 +67,55 @@ def allreduce_weight_estimate(G_W, group=None):
     import torch.distributed as dist
     dist.all_reduce(G_W, op=dist.ReduceOp.SUM, group=group)
     return G_W
+
+
+def flat_layout(shapes: Sequence[Tuple[int, int]], align: int = 64):
+    """Where each layer's weight estimate G_W [d_out, d_in] sits in one flat fp32 buffer:
+    ([(offset, size)] per layer, total elements).  Offsets are multiples of ``align`` elements
+    (256 bytes), so every layer's view is aligned for the kernels and a bucket of consecutive
+    layers is one contiguous span for one collective."""
+    out, o = [], 0
+    for d_out, d_in in shapes:
+        n = int(d_out) * int(d_in)
+        out.append((o, n))
+        o += -(-n // align) * align
+    return out, o
+
+
+def plan_buckets(sizes: Sequence[int], n_buckets: int) -> List[Tuple[int, int]]:
+    """Consecutive layer ranges [l0, l1) with element counts as even as the layer boundaries
+    allow (cut where the running total is nearest k/n_buckets of the whole).  Every range is
+    non-empty; fewer ranges come back when there are fewer layers than buckets."""
+    n = len(sizes)
+    if n == 0:
+        return []
+    if n_buckets < 1:
+        raise ValueError("n_buckets must be >= 1")
+    cum = np.cumsum(np.asarray(sizes, dtype=np.float64))
+    total = cum[-1]
+    cuts = [0]
+    for k in range(1, min(n_buckets, n)):
+        j = int(np.argmin(np.abs(cum - k * total / n_buckets))) + 1
+        j = min(max(j, cuts[-1] + 1), n - (min(n_buckets, n) - k))
+        cuts.append(j)
+    cuts.append(n)
+    return [(a, b) for a, b in zip(cuts[:-1], cuts[1:]) if b > a]
+
+
+def bucket_span(layout, bucket: Tuple[int, int]) -> Tuple[int, int]:
+    """Element range [a, b) of the flat buffer covered by the layers of ``bucket``."""
+    l0, l1 = bucket
+    return layout[l0][0], layout[l1 - 1][0] + layout[l1 - 1][1]
+
+
+def allreduce_bucket(flat, layout, bucket: Tuple[int, int], group=None):
+    """Sum over ranks (in place) of one bucket of the flat weight-estimate buffer: one
+    collective for all its layers.  The stack calls it on a side stream as soon as the
+    bucket's estimates are complete, so the exchange overlaps the remaining layers' work."""
+    import torch.distributed as dist
+    a, b = bucket_span(layout, bucket)
+    dist.all_reduce(flat[a:b], op=dist.ReduceOp.SUM, group=group)
+    return flat
 
 
 def estimate_sharded(x, W, u, cu_local, K: int, sigma: float, gamma: float, seed: int,
