@@ -33,29 +33,65 @@ import workloads  # noqa: E402
 METRIC = "Dust estimator tokens*draws/s per layer"
 UNIT = "tokens*draws/s"
 L2_FLUSH_BYTES = 256 << 20
+# The 48-layer stack is the largest single-GPU workload; its gamma is swept over {0, 0.9,
+# 0.99}, and the headline takes the middle value.
+HEADLINE_GAMMA = 0.9
 
-# ALU roofline of the noise kernels: issue slots of all SMs at the maximum SM clock divided by
-# the algorithm's minimal per-normal operation count (one Philox4x32-10 block = 10 rounds x
-# (2 wide multiplies + 2 three-input XORs) per 4 normals; 3 ops per uniform; Box-Muller 10 ops
-# per pair: log, scale, rsqrt, multiply, angle FMA, range scale, sin, cos, 2 products; plus the
-# consumer FMAs: 2 per normal in the forward, 1 in the draw reduction).
-LANES_PER_SM = 128
-OPS_PER_NORMAL = {"fwd_bf16_noise_loss": 20.0, "ghat_reduce_draws": 19.0,
-                  "fwd_bf16_noise_loss_grouped": 20.0, "ghat_reduce_draws_grouped": 19.0,
-                  # LM head: generator 18 (Philox 10, uniform 3, Box-Muller 5), sigma a (1),
-                  # exp(sigma a) - 1 as a degree-5 series (5), the weighted sum (1)
-                  "lmhead_ce_noise": 25.0}
-# DRAM bytes (read + write) per launch of a dominant kernel, from one ncu capture of the
-# current build of that kernel on that workload (profiles/ holds the capture summaries);
-# absent entries are reported as null.
-MEASURED_TRAFFIC = {
-    ("fwd_bf16_noise_loss", "gpt2s-mlp-win-768x3072"): (68.49e6 + 2.45e6,
-                                                       "profiles/ncu_full_fwd_persistent_gpt2s_mlp_win_768x3072.md"),
-    ("lmhead_ce_noise", "head-4096-slab1024"): (33.85e6 + 75.21e6,
-                                                "profiles/ncu_full_lmhead_head-4096-slab1024.md"),
-}
+# ALU roofline of the noise kernels, per pipe.  Rates are operations per clock per SM (the
+# CUDA C programming guide's arithmetic-throughput table): 32-bit integer multiply 64 (a
+# 32x32->64 widening multiply gives two results), special functions (lg2, rsqrt, sin, cos)
+# 16, logical/shift/integer add 64, fp32 add/multiply/fma 128 on the two FMA pipes that the
+# integer multiplies share, and one warp instruction per clock per scheduler (128 lanes).
+PIPE_RATE = {"imad": 64.0, "xu": 16.0, "alu": 64.0, "fma_pipes": 128.0, "issue": 128.0}
+# Per-normal operation counts, from the algorithm (not from compiled code):
+#   Philox4x32-10: per 4 normals, 10 rounds x (2 widening multiplies + 2 three-input XORs)
+#     -> imad 10 results, alu 5;  uniforms: the word's mantissa field (shift, add) -> alu 2;
+#     the near-one test once per block (max, compare, branch) -> alu 0.75
+#   Box-Muller per pair: lg2, rsqrt, sin, cos -> xu 2;  radius uniform, angle, -sqrt as
+#     packed f32x2 pairs -> fp32 1.5 (0.75 instructions)
+#   consumer: forward 2 fp32 per normal (1 packed instruction); draw reduction r x nq per
+#     pair and 1 fma per normal -> 1.5 (0.75 instructions); LM head sigma a, a degree-5 series
+#     of exp(sigma a) - 1 and the weighted sum -> 7 (4 instructions)
+_GEN = {"imad": 10.0, "xu": 2.0, "alu": 7.75, "fp32": 1.5, "instr": 14.5}
+#   SPSA directions: rho x (cos or sin) and the bf16 pair conversion -> 1 fp32 (1 instruction);
+#     SPSA estimate: the same product and p_j z -> 2 fp32 (1 packed instruction)
+_CONSUMER = {"fwd": (2.0, 1.0), "ghat": (1.5, 0.75), "lmhead": (7.0, 4.0), "spsa_dir": (1.0, 1.0),
+             "spsa_est": (2.0, 1.0)}
+ALU_KERNELS = {"fwd_bf16_noise_loss": "fwd", "fwd_bf16_noise_loss_grouped": "fwd",
+               "ghat_reduce_draws": "ghat", "ghat_reduce_draws_grouped": "ghat",
+               "lmhead_ce_noise": "lmhead", "spsa_directions": "spsa_dir",
+               "spsa_estimate": "spsa_est"}
+
+# DRAM bytes (read + write) per launch of a dominant kernel from one ncu capture, with the
+# digest of the CUDA sources that were captured: a value is reported only while the sources
+# still have that digest (a changed kernel reports null until it is captured again).  Each
+# entry: (kernel, workload) -> (bytes per launch, source digest, profile summary).
+MEASURED_TRAFFIC = {}
 HEAD_METRIC = "Dust LM-head estimator tokens*draws/s"
 ATTN_METRIC = "Dust attention-reward estimator tokens*draws/s"
+
+
+def source_digest() -> str:
+    """sha256 (first 16 hex digits) of the library's CUDA sources and header."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "zeroth_order_transformer_b200", "csrc")
+    files = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))
+                   + glob.glob(os.path.join(csrc, "*.h"))
+                   + glob.glob(os.path.join(ROOT, "include", "*.h")))
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, workload: str):
+    e = MEASURED_TRAFFIC.get((kernel, workload))
+    if e is None or e[1] != source_digest():
+        return None, None
+    return e[0], e[2]
 
 
 def measured_peaks():
@@ -70,20 +106,51 @@ def measured_peaks():
                 sm_max_mhz=1965.0, source="fallback")
 
 
-def describe(wl) -> str:
+def alu_bounds(kind: str, sms: int, mhz: float):
+    """Gnormal/s that each pipe allows a noise kernel of the given consumer kind, and the
+    binding (smallest) one."""
+    c_fp32, c_instr = _CONSUMER[kind]
+    ops = {"imad": _GEN["imad"], "xu": _GEN["xu"], "alu": _GEN["alu"],
+           "fma_pipes": _GEN["imad"] + _GEN["fp32"] + c_fp32, "issue": _GEN["instr"] + c_instr}
+    clk = sms * mhz * 1e6
+    bounds = {p: round(clk * PIPE_RATE[p] / n / 1e9, 1) for p, n in ops.items()}
+    binding = min(bounds, key=bounds.get)
+    return bounds, binding, ops
+
+
+def alu_roofline(kernel: str, achieved: float, sms: int, peaks) -> dict:
+    bounds, binding, ops = alu_bounds(ALU_KERNELS[kernel], sms, peaks["sm_max_mhz"])
+    peak = bounds[binding]
+    return {"kernel": kernel, "bound": "alu", "achieved": round(achieved, 2), "peak": peak,
+            "unit": "Gnormal/s", "frac": round(achieved / peak, 4), "traffic": None,
+            "peak_source": "derived", "binding_pipe": binding, "pipe_bounds": bounds,
+            "peak_basis": (f"min over pipes of {sms} SMs x {peaks['sm_max_mhz']:.0f} MHz x "
+                           f"(pipe ops per clock per SM) / (that pipe's ops per normal); ops "
+                           f"per normal {ops}; clock from MEASURED_PEAKS.json")}
+
+
+def describe(wl, gamma=None) -> str:
     shapes = sorted({(l.d_in, l.d_out) for l in wl.layers})
     s = ", ".join(f"{a}->{b}" for a, b in shapes)
+    g = wl.gamma if gamma is None else gamma
     return (f"{wl.name} (cfg {wl.cfg_id}): {wl.n_seq}x{wl.seq_len} tokens"
             f"{' packed' if wl.packed else ''}, {len(wl.layers)} layer(s) {s}, K={wl.K}, "
-            f"sigma={wl.sigma}, gamma={wl.gamma}, {wl.dtype}")
+            f"sigma={wl.sigma}, gamma={g}, {wl.dtype}")
+
+
+def headline_gamma(wl, arg):
+    if arg is not None:
+        return float(arg)
+    return HEADLINE_GAMMA if HEADLINE_GAMMA in wl.gammas else wl.gamma
 
 
 # ------------------------------------------------------------------------------ CPU oracle
-def oracle_sample(data, n_tokens: int, max_seconds: float):
+def oracle_sample(data, n_tokens: int, max_seconds: float, gamma=None):
     """Run the oracle's whole estimator on the first n_tokens of each layer until max_seconds
     of work; returns (token*draws processed per layer, seconds, threads, description)."""
     import oracle
     wl = data.wl
+    g = wl.gamma if gamma is None else gamma
     done = 0
     t0 = time.perf_counter()
     layers_run = 0
@@ -92,7 +159,7 @@ def oracle_sample(data, n_tokens: int, max_seconds: float):
         n = min(n_tokens, wl.N)
         cu = np.asarray(data.cu_seqlens, dtype=np.int64)
         cu = np.unique(np.clip(cu, 0, n)).astype(np.int32)
-        oracle.dust_layer(L.x_f64[:n], L.W_f64, L.u_f64[:n], wl.K, wl.sigma, wl.gamma, cu,
+        oracle.dust_layer(L.x_f64[:n], L.W_f64, L.u_f64[:n], wl.K, wl.sigma, g, cu,
                           wl.seed, L.shape.layer_id)
         done += n * wl.K
         layers_run += 1
@@ -100,20 +167,23 @@ def oracle_sample(data, n_tokens: int, max_seconds: float):
         if el >= max_seconds or layers_run >= 64:
             break
     desc = (f"oracle (fp64 C, OpenMP) whole estimator on the first {min(n_tokens, wl.N)} tokens "
-            f"of {layers_run} layer pass(es) of the workload (credit segments truncated to the "
-            f"sample)")
+            f"of {layers_run} layer pass(es) of the workload, cycling through its layers "
+            f"(credit segments truncated to the sample)")
     return done, el, oracle.get_threads(), desc
 
 
 def run_reference(args, rank: int, world: int) -> None:
     if rank != 0:
         return
-    data = workloads.generate(args.workload, n_layers=1)
+    wl0 = workloads.WORKLOADS[args.workload]
+    # enough layers for the sample to visit every layer shape of the workload
+    data = workloads.generate(args.workload, n_layers=min(len(wl0.layers), 4))
     wl = data.wl
+    gamma = headline_gamma(wl, args.gamma)
     n_tok = args.ref_tokens
     times = []
     for k in range(args.warmup + args.steps):
-        done, el, cores, desc = oracle_sample(data, n_tok, 0.0)
+        done, el, cores, desc = oracle_sample(data, n_tok, 0.0, gamma)
         if k >= args.warmup:
             times.append(el)
     tot = sum(times)
@@ -122,7 +192,7 @@ def run_reference(args, rank: int, world: int) -> None:
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": describe(wl), "sample_tokens": min(n_tok, wl.N)},
+        "config": {"workload": describe(wl0, gamma), "sample_tokens": min(n_tok, wl.N)},
         "impl": "reference",
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": desc},
@@ -185,7 +255,7 @@ class ClockSampler:
 def kernel_work(name, wl, shapes):
     """Algorithmic work of one launch over the given layer shapes: (bound, amount, what)."""
     N, K = wl.N, wl.K
-    if name in OPS_PER_NORMAL:
+    if name in ALU_KERNELS:
         return "alu", sum(N * s.d_out * K for s in shapes), "normals"
     if name.startswith("gw_bf16_tcgen05"):
         return "tensor", sum(2.0 * N * s.d_in * s.d_out for s in shapes), "flops"
@@ -194,22 +264,162 @@ def kernel_work(name, wl, shapes):
     return None, None, None
 
 
-def generator_ceiling(dust, torch, dev, reps: int = 10) -> float:
-    """Gnormal/s of the generator-only probe (generate and add, nothing else) over a grid of
-    8 x 256 threads per SM, 1024 normals each: what the noise kernels' generator can reach."""
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    n, nq = sms * 8 * 256, 256
-    out = torch.empty(n, dtype=torch.float32, device=dev)
-    key = dust.NoiseKey(0x5EED0000, 0)
+def _time_probe(fn, torch, reps: int = 10) -> float:
+    """Milliseconds per call of fn (3 untimed calls, then reps between CUDA events on the
+    current stream)."""
     for _ in range(3):
-        dust.dust_debug_normal_sum(key, n, nq, out)
+        fn()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     for _ in range(reps):
-        dust.dust_debug_normal_sum(key, n, nq, out)
+        fn()
     b.record()
-    torch.cuda.synchronize(dev)
-    return 4.0 * n * nq * reps / (a.elapsed_time(b) / 1e3) / 1e9
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def generator_ceiling(dust, torch, dev) -> dict:
+    """Rates of the generator-only probe (Philox, Box-Muller and one add per normal) and of
+    the Philox-only probe (the words XORed together), over a grid of 8 x 256 threads per SM,
+    1024 normals (256 blocks) per thread: what the noise kernels' generator, and its integer
+    part alone, reach on the device."""
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    n, nq = sms * 8 * 256, 256
+    out = torch.empty(n, dtype=torch.float32, device=dev)
+    wout = torch.empty(n, dtype=torch.int32, device=dev)
+    key = dust.NoiseKey(0x5EED0000, 0)
+    ms_n = _time_probe(lambda: dust.dust_debug_normal_sum(key, n, nq, out), torch)
+    ms_w = _time_probe(lambda: dust.dust_debug_word_sum(key, n, nq, wout), torch)
+    return {"generator_gnormal_s": round(4.0 * n * nq / (ms_n / 1e3) / 1e9, 2),
+            "philox_gword_s": round(4.0 * n * nq / (ms_w / 1e3) / 1e9, 2)}
+
+
+def _prof_avg(prof, prefix):
+    t = [ms for name, ms in prof if name.startswith(prefix)]
+    return (sum(t) / len(t), len(t)) if t else (None, 0)
+
+
+def _single_layer_inputs(dust, torch, dev, cfg):
+    data = workloads.generate(cfg)
+    L = data.layers[0]
+
+    def to_dev(st):
+        return torch.from_numpy(np.ascontiguousarray(st).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+
+    x, W, u = to_dev(L.x_store), to_dev(L.W_store), to_dev(L.u_store)
+    return data, L, x, W, u, torch.from_numpy(data.cu_seqlens).to(dev)
+
+
+def measure_targets(dust, torch, dev, peaks, flush, reps: int) -> dict:
+    """The hot path's numeric targets, each measured here with CUDA events on the launching
+    stream (the library's per-launch profile records):
+      gw_cfg3            the weight-estimate contraction on the packed 32k x 1024 -> 1024
+                         workload, TFLOP/s against the measured dense bf16 peak (target 0.6);
+      credit_stress      the credit scan on K = 64 x 4 Mi tokens (larger than L2), GB/s of
+                         its 8 K N algorithmic bytes against the measured HBM copy bandwidth;
+      reduction_streams  the draw reduction on the 16k x 2048 -> 8192, K = 64 workload: its
+                         HBM streams (credit read 4 K N + bf16 g write 2 N d_out bytes) in GB/s
+                         against the HBM peak, and its normals against the ALU bound that in
+                         fact binds it;
+      credit_latency     the credit step of each workload (its own K, N and segments)."""
+    out = {}
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+
+    def run_wgrad(cfg):
+        data, L, x, W, u, cu = _single_layer_inputs(dust, torch, dev, cfg)
+        wl, s = data.wl, L.shape
+        ws = torch.empty(max(dust.dust_workspace_size(op, 1, wl.N, s.d_in, s.d_out, wl.K)
+                             for op in range(3)), dtype=torch.uint8, device=dev)
+        key = dust.NoiseKey(wl.seed, s.layer_id)
+        dl = dust.dust_noisy_linear_fwd(x, W, u, wl.K, wl.sigma, key, workspace=ws)
+        r = dust.dust_credit(dl, cu, wl.gamma, workspace=ws)
+        G = torch.empty((s.d_out, s.d_in), dtype=torch.float32, device=dev)
+        for _ in range(3):
+            dust.dust_weight_grad(r, x, s.d_out, wl.K, wl.sigma, key, G, False, None, ws)
+        torch.cuda.synchronize(dev)
+        dust.dust_profile_read()
+        dust.dust_profile_enable(1 << 12)
+        for _ in range(reps):
+            flush.zero_()
+            dust.dust_weight_grad(r, x, s.d_out, wl.K, wl.sigma, key, G, False, None, ws)
+        prof = dust.dust_profile_read()
+        dust.dust_profile_disable()
+        st = dust.dust_last_device_error()[0]
+        return wl, s, prof, st
+
+    wl, s, prof, st = run_wgrad(3)
+    gw_ms, n = _prof_avg(prof, "gw_bf16_tcgen05")
+    sk_ms, _ = _prof_avg(prof, "gw_splitk_reduce")
+    flops = 2.0 * wl.N * s.d_in * s.d_out
+    tf = flops / (gw_ms / 1e3) / 1e12
+    out["gw_cfg3"] = {"workload": describe(wl), "kernel": "gw_bf16_tcgen05", "launches": n,
+                      "ms": round(gw_ms, 5), "tflops": round(tf, 1),
+                      "peak": peaks["bf16_tflops"], "frac": round(tf / peaks["bf16_tflops"], 4),
+                      "target": 0.6, "splitk_reduce_ms": None if sk_ms is None else round(sk_ms, 5),
+                      "status": st, "peak_source": peaks["source"] + " (burst)"}
+
+    wl, s, prof, st = run_wgrad(4)
+    gh_ms, n = _prof_avg(prof, "ghat_reduce_draws")
+    gw4_ms, _ = _prof_avg(prof, "gw_bf16_tcgen05")
+    streams = 4.0 * wl.K * wl.N + 2.0 * wl.N * s.d_out
+    gbs = streams / (gh_ms / 1e3) / 1e9
+    gn = wl.N * s.d_out * wl.K / (gh_ms / 1e3) / 1e9
+    roof = alu_roofline("ghat_reduce_draws", gn, sms, peaks)
+    out["reduction_streams"] = {
+        "workload": describe(wl), "kernel": "ghat_reduce_draws", "launches": n,
+        "ms": round(gh_ms, 4), "stream_bytes": streams, "gbs": round(gbs, 2),
+        "frac_hbm": round(gbs / peaks["hbm_gbs"], 5), "target_hbm": 0.7,
+        "gnormal_s": round(gn, 2), "alu_bound": roof["peak"], "binding_pipe": roof["binding_pipe"],
+        "frac_alu": roof["frac"],
+        "note": "the noise regeneration (ALU) bounds this kernel; its HBM streams are "
+                f"{streams / 1e6:.0f} MB per launch",
+        "gw_cfg4_tflops": round(2.0 * wl.N * s.d_in * s.d_out / (gw4_ms / 1e3) / 1e12, 1),
+        "status": st}
+    torch.cuda.empty_cache()
+
+    # credit scan on a shape larger than L2
+    K, N = 64, 1 << 22
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234)
+    loss = torch.randn((K, N), generator=g, device=dev, dtype=torch.float32)
+    r = torch.empty_like(loss)
+    cu = torch.from_numpy(workloads.random_segments(77, N, 256, 2048)).to(dev)
+    ws = torch.empty(dust.dust_workspace_size(dust.DUST_OP_CREDIT, dust.DUST_F32, N, 0, 0, K),
+                     dtype=torch.uint8, device=dev)
+    ms = _time_probe(lambda: dust.dust_credit(loss, cu, 0.99, r, ws), torch, reps=max(reps, 10))
+    gbs = 8.0 * K * N / (ms / 1e3) / 1e9
+    out["credit_stress"] = {"K": K, "N": N, "segments": "packed U[256, 2048]", "gamma": 0.99,
+                            "ms": round(ms, 4), "gbs": round(gbs, 1),
+                            "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "target": 0.7,
+                            "status": dust.dust_last_device_error()[0],
+                            "note": "2 GiB moved per launch, larger than L2: no flush needed"}
+    del loss, r, ws
+    torch.cuda.empty_cache()
+
+    # credit latency at each workload's own size (L2-resident; the flush precedes each call)
+    lat = {}
+    for cfg in (2, 3, 4):
+        wl = workloads.WORKLOADS[cfg]
+        cu_np = workloads.generate(cfg, n_layers=0).cu_seqlens if wl.packed else \
+            workloads.cu_seqlens_from_lengths([wl.seq_len] * wl.n_seq)
+        loss = torch.from_numpy(workloads.gaussian_losses(cfg, wl.K, wl.N)).to(dev)
+        r = torch.empty_like(loss)
+        cu = torch.from_numpy(cu_np).to(dev)
+        ws = torch.empty(dust.dust_workspace_size(dust.DUST_OP_CREDIT, 0, wl.N, 0, 0, wl.K),
+                         dtype=torch.uint8, device=dev)
+        dust.dust_credit(loss, cu, wl.gamma, r, ws)
+        torch.cuda.synchronize(dev)
+        dust.dust_profile_enable(1 << 10)
+        for _ in range(reps):
+            flush.zero_()
+            dust.dust_credit(loss, cu, wl.gamma, r, ws)
+        t, _ = _prof_avg(dust.dust_profile_read(), "credit_scan")
+        dust.dust_profile_disable()
+        lat[f"cfg{cfg}"] = {"K": wl.K, "N": wl.N, "us": round(t * 1e3, 2),
+                            "gbs": round(8.0 * wl.K * wl.N / (t / 1e3) / 1e9, 1)}
+    out["credit_latency"] = lat
+    return out
 
 
 def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
@@ -217,6 +427,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     import torch.distributed as dist
 
     import zeroth_order_transformer_b200 as dust
+    from zeroth_order_transformer_b200 import distributed as zd
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -225,6 +436,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                                 device_id=dev)
     data = workloads.generate(args.workload)
     wl = data.wl
+    gamma = headline_gamma(wl, args.gamma)
     peaks = measured_peaks()
 
     def dev_t(store, dtype):
@@ -238,41 +450,61 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         layers.append((L.shape, x, W, u))
     cu = torch.from_numpy(data.cu_seqlens).to(dev)
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
-    max_in = max(s.d_in for s, *_ in layers)
-    max_out = max(s.d_out for s, *_ in layers)
-    ws_bytes = max(dust.dust_workspace_size(op, 1 if wl.dtype == "bf16" else 0, wl.N, s.d_in,
-                                            s.d_out, wl.K)
-                   for op in range(3) for s, *_ in layers)
-    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
-    dloss = torch.empty((wl.K, wl.N), dtype=torch.float32, device=dev)
-    r = torch.empty((wl.K, wl.N), dtype=torch.float32, device=dev)
-    GWs = [torch.empty((s.d_out, s.d_in), dtype=torch.float32, device=dev) for s, *_ in layers]
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    gamma = wl.gamma
+    stack = len(layers) > 1
+    red = (lambda G: dist.all_reduce(G)) if world > 1 else None
 
-    stacks = {}
+    if stack:
+        st = dust.DustStack([(x, W, u, s.layer_id) for s, x, W, u in layers], wl.K)
+        GWs = st.G_W
+    else:
+        s1, x1, W1, u1 = layers[0]
+        ws_bytes = max(dust.dust_workspace_size(op, 1 if wl.dtype == "bf16" else 0, wl.N,
+                                                s1.d_in, s1.d_out, wl.K) for op in range(3))
+        ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+        dloss = torch.empty((wl.K, wl.N), dtype=torch.float32, device=dev)
+        r = torch.empty((wl.K, wl.N), dtype=torch.float32, device=dev)
+        GWs = [torch.empty((s1.d_out, s1.d_in), dtype=torch.float32, device=dev)]
 
-    def step(inputs=None):
-        inputs = inputs or layers
-        if len(inputs) > 1:
-            # a block stack: the grouped calls, one launch per step for all layers
-            st = stacks.get(id(inputs))
-            if st is None:
-                st = dust.DustStack([(x, W, u, s.layer_id) for s, x, W, u in inputs], wl.K)
-                stacks[id(inputs)] = st
-            st.estimate(cu, wl.sigma, gamma, wl.seed, 0, rank * wl.N)
-            out = st.G_W
-        else:
-            s, x, W, u = inputs[0]
-            key = dust.NoiseKey(wl.seed, s.layer_id, 0, rank * wl.N)
-            dust.dust_noisy_linear_fwd(x, W, u, wl.K, wl.sigma, key, dloss, ws)
-            dust.dust_credit(dloss, cu, gamma, r, ws)
-            dust.dust_weight_grad(r, x, s.d_out, wl.K, wl.sigma, key, GWs[0], False, None, ws)
-            out = GWs
+    def step(g=gamma):
+        if stack:
+            # the grouped calls, one launch per step for all layers; on several GPUs the
+            # weight estimates are summed in buckets overlapped with the later layers' work
+            st.estimate(cu, wl.sigma, g, wl.seed, 0, rank * wl.N, reduce=red,
+                        buckets=args.buckets)
+            return GWs
+        key = dust.NoiseKey(wl.seed, s1.layer_id, 0, rank * wl.N)
+        dust.dust_noisy_linear_fwd(x1, W1, u1, wl.K, wl.sigma, key, dloss, ws)
+        dust.dust_credit(dloss, cu, g, r, ws)
+        dust.dust_weight_grad(r, x1, s1.d_out, wl.K, wl.sigma, key, GWs[0], False, None, ws)
+        if red is not None:
+            red(GWs[0])
+        return GWs
+
+    def timed(n_steps, g=gamma, profile=False):
+        """Device milliseconds per step (max over ranks) of n_steps steps, L2 flushed before
+        each, bracketed by barriers and device synchronisation."""
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(n_steps)]
+        stops = [torch.cuda.Event(enable_timing=True) for _ in range(n_steps)]
+        torch.cuda.synchronize(dev)
         if world > 1:
-            for G in out:
-                dist.all_reduce(G)
-        return out
+            dist.barrier()
+        if profile:
+            dust.dust_profile_enable(1 << 16)
+        for k in range(n_steps):
+            flush.zero_()
+            starts[k].record(stream)
+            step(g)
+            stops[k].record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        total = sum(a.elapsed_time(b) for a, b in zip(starts, stops))
+        if world > 1:
+            t = torch.tensor([total], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            total = float(t.item())
+        return total / n_steps
 
     stream = torch.cuda.current_stream(dev)
     for _ in range(args.warmup):
@@ -283,34 +515,25 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         dist.barrier()
 
     # ---- timed region
-    dust.dust_profile_enable(1 << 16)
     sampler = ClockSampler(local_rank) if rank == 0 else None
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    for k in range(args.steps):
-        flush.zero_()
-        starts[k].record(stream)
-        step()
-        stops[k].record(stream)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
+    ms_per_step = timed(args.steps, profile=True)
     clocks = sampler.stop() if sampler else None
     prof = dust.dust_profile_read()
     dust.dust_profile_disable()
-    step_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    ms_per_step = total_ms / args.steps
+    dev_status = dust.dust_last_device_error()[0]
     units = wl.N * wl.K * len(layers) * world
     # tokens*draws per layer processed per second: N K n_layers n_gpus / step time
     value = units / (ms_per_step / 1e3)
+
+    # ---- the other discounts of the workload (the stack sweeps gamma over {0, 0.9, 0.99})
+    sweep = None
+    if len(wl.gammas) > 1 and not args.no_sweep:
+        sweep = []
+        for g in wl.gammas:
+            step(g)
+            ms = timed(max(3, min(args.steps, 10)), g)
+            sweep.append({"gamma": g, "ms_per_step": round(ms, 4),
+                          "value": units / (ms / 1e3)})
 
     # ---- per-kernel statistics (rank 0's launches)
     per = {}
@@ -325,55 +548,48 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     s0 = layers[0][0]
     shapes = [s for s, *_ in layers]
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    for n, info in kernels.items():
-        bound, amount, what = kernel_work(n, wl, shapes if n.endswith("_grouped") else [s0])
-        if amount is None or (len(layers) > 1 and not n.endswith("_grouped")):
-            continue
-        per_s = amount / (info["ms_avg"] / 1e3)
-        if what == "normals":
-            info["gnormals_per_s"] = round(per_s / 1e9, 2)
-        elif what == "flops":
-            info["tflops"] = round(per_s / 1e12, 2)
-        else:
-            info["gbs"] = round(per_s / 1e9, 2)
-    # dominant kernel: the largest total time among kernels with a defined algorithmic work
+
     def work_of(n):
+        if stack and not n.endswith("_grouped"):
+            return None, None, None
         return kernel_work(n, wl, shapes if n.endswith("_grouped") else [s0])
 
+    for n, info in kernels.items():
+        bound, amount, what = work_of(n)
+        if amount is None:
+            continue
+        per_s = amount / (info["ms_avg"] / 1e3)
+        info[{"normals": "gnormals_per_s", "flops": "tflops", "bytes": "gbs"}[what]] = round(
+            per_s / (1e12 if what == "flops" else 1e9), 2)
+    # dominant kernel: the largest total time among kernels with a defined algorithmic work
     dominant = next((n for n in kernels if work_of(n)[1] is not None), None)
     roofline = None
     if dominant:
         bound, amount, what = work_of(dominant)
         avg_s = kernels[dominant]["ms_avg"] / 1e3
         if bound == "alu":
-            peak = sms * LANES_PER_SM * peaks["sm_max_mhz"] * 1e6 / OPS_PER_NORMAL[dominant] / 1e9
-            ach = amount / avg_s / 1e9
-            roofline = {"kernel": dominant, "bound": "alu", "achieved": round(ach, 2),
-                        "peak": round(peak, 2), "unit": "Gnormal/s", "frac": round(ach / peak, 4),
-                        "traffic": None,
-                        "peak_basis": f"{sms} SMs x {LANES_PER_SM} lanes x "
-                                      f"{peaks['sm_max_mhz']:.0f} MHz / "
-                                      f"{OPS_PER_NORMAL[dominant]:.0f} ops per normal"}
+            roofline = alu_roofline(dominant, amount / avg_s / 1e9, sms, peaks)
+            roofline.update(generator_ceiling(dust, torch, dev))
+            roofline["frac_of_generator"] = round(
+                roofline["achieved"] / roofline["generator_gnormal_s"], 4)
         elif bound == "tensor":
             ach = amount / avg_s / 1e12
             roofline = {"kernel": dominant, "bound": "tensor", "achieved": round(ach, 2),
-                        "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                        "frac": round(ach / peaks["bf16_tflops"], 4), "traffic": None}
+                        "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                        "frac": round(ach / peaks["bf16_tflops_sustained"], 4), "traffic": None,
+                        "peak_source": peaks["source"] + " (sustained)"}
         elif bound == "hbm":
             ach = amount / avg_s / 1e9
             roofline = {"kernel": dominant, "bound": "hbm", "achieved": round(ach, 2),
                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                        "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None}
+                        "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None,
+                        "peak_source": peaks["source"]}
         if roofline is not None:
-            roofline["peak_source"] = peaks["source"]
-            tr = MEASURED_TRAFFIC.get((dominant, wl.name))
-            if tr is not None:
-                roofline["traffic"] = tr[0]
-                roofline["traffic_source"] = tr[1]
-            if bound == "alu":
-                gc = generator_ceiling(dust, torch, dev)
-                roofline["generator_ceiling"] = round(gc, 2)
-                roofline["frac_of_generator_ceiling"] = round(roofline["achieved"] / gc, 4)
+            roofline["units_per_launch"] = amount
+            tr, src = measured_traffic(dominant, wl.name)
+            roofline["traffic"] = tr
+            roofline["traffic_source"] = src or ("null: no ncu capture of the current sources "
+                                                 "of this kernel on this workload")
 
     # ---- end to end through the public API, host buffers, copies inside the timed region
     e2e = None
@@ -382,34 +598,27 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         h2d = 0
         for s, x, W, u in layers:
             hx, hW, hu = (t.cpu().pin_memory() for t in (x, W, u))
-            host_in.append((s, hx, hW, hu))
+            host_in.append((hx, hW, hu))
             h2d += sum(t.numel() * t.element_size() for t in (hx, hW, hu))
-        dev_in = [(s, torch.empty_like(x), torch.empty_like(W), torch.empty_like(u))
-                  for s, x, W, u in layers]
-        host_out = [torch.empty(G.shape, dtype=G.dtype, pin_memory=True) for G in GWs]
-        d2h = sum(G.numel() * G.element_size() for G in GWs)
-
-        if len(layers) == 1:
-            # one layer: the public host-input call, upload pipelined with the compute
-            s1 = layers[0][0]
-            host_layer = dust.DustLayer(wl.N, s1.d_in, s1.d_out, wl.K, tdt, dev)
-            red = (lambda G: dist.all_reduce(G)) if world > 1 else None
+        if stack:
+            G_host = torch.empty(st.G_W_flat.shape, dtype=torch.float32, pin_memory=True)
+            d2h = G_host.numel() * 4
 
             def e2e_step():
-                _, hx, hW, hu = host_in[0]
+                st.estimate_from_host(host_in, data.cu_seqlens, wl.sigma, gamma, wl.seed,
+                                      G_host, chunks=4, reduce=red, buckets=args.buckets,
+                                      token_offset=rank * wl.N)
+        else:
+            host_layer = dust.DustLayer(wl.N, s1.d_in, s1.d_out, wl.K, tdt, dev)
+            G_host = torch.empty(GWs[0].shape, dtype=torch.float32, pin_memory=True)
+            d2h = G_host.numel() * 4
+
+            def e2e_step():
+                hx, hW, hu = host_in[0]
                 host_layer.estimate_from_host(
                     hx, hW, hu, data.cu_seqlens, wl.sigma, gamma,
-                    dust.NoiseKey(wl.seed, s1.layer_id, 0, rank * wl.N), host_out[0],
+                    dust.NoiseKey(wl.seed, s1.layer_id, 0, rank * wl.N), G_host,
                     chunks=4, reduce=red)
-        else:
-            def e2e_step():
-                for (s, hx, hW, hu), (_, dx, dW, du) in zip(host_in, dev_in):
-                    dx.copy_(hx, non_blocking=True)
-                    dW.copy_(hW, non_blocking=True)
-                    du.copy_(hu, non_blocking=True)
-                out = step(dev_in)
-                for G, hG in zip(out, host_out):
-                    hG.copy_(G, non_blocking=True)
 
         for _ in range(max(1, args.warmup // 2)):
             flush.zero_()
@@ -432,12 +641,15 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
             e_ms = float(t.item())
         e2e = {"value": units / (e_ms / args.steps / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": e_ms / args.steps}
+               "ms_per_step": e_ms / args.steps,
+               "note": "inputs uploaded from pinned host memory in four runs of whole "
+                       "sequences, each run's upload overlapped with the previous run's "
+                       "estimate; G_W read back"}
+        del host_in
 
     # ---- optional: the optimizer step fused into the weight estimate (single-layer workloads)
     opt_line = None
-    if args.optimizer != "none" and len(layers) == 1:
-        s1, x1, W1, u1 = layers[0]
+    if args.optimizer != "none" and not stack:
         Wm = torch.zeros((s1.d_out, s1.d_in), dtype=torch.float32, device=dev)
         mm = torch.zeros_like(Wm)
         vv = torch.zeros_like(Wm) if args.optimizer == "adam" else None
@@ -470,14 +682,19 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                     "weight_grad_with_step_ms": round(t_step, 5),
                     "step_overhead_ms": round(t_step - t_plain, 5)}
 
+    # ---- the path's numeric targets, measured in this run (one GPU)
+    targets = None
+    if world == 1 and not args.no_targets:
+        targets = measure_targets(dust, torch, dev, peaks, flush, reps=max(5, min(args.steps, 20)))
+
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        done, el, cores, desc = oracle_sample(data, args.cpu_tokens, args.cpu_seconds)
+        done, el, cores, desc = oracle_sample(data, args.cpu_tokens, args.cpu_seconds, gamma)
         cpu = {"value": done / el, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": desc, "seconds": round(el, 2)}
 
-    n_launch_per_step = sum(c for c in (v["launches"] for v in kernels.values())) / args.steps
+    n_launch = sum(v["launches"] for v in kernels.values())
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -486,18 +703,27 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "operands": "bf16 x, W, u; u32 Philox words",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "operands": "bf16 x, W, u; u32 Philox words",
         "data": "synthetic (seeded; shapes of the Dust page's transformer layers)",
-        "config": {"workload": describe(wl), "tokens_per_gpu": wl.N, "d_in": s0.d_in,
-                   "d_out": s0.d_out, "K": wl.K, "layers": len(layers),
-                   "parallelism": f"dp{world}: one batch per GPU, NCCL all-reduce of G_W",
+        "config": {"workload": describe(wl, gamma), "tokens_per_gpu": wl.N, "K": wl.K,
+                   "layers": len(layers),
+                   "layer_shapes": sorted({f"{s.d_in}->{s.d_out}" for s in shapes}),
+                   "gamma": gamma,
+                   "parallelism": (f"dp{world}: one batch per GPU, NCCL all-reduce of G_W"
+                                   + (f" in {args.buckets} buckets overlapped with the weight "
+                                      "estimate" if stack else "")),
                    "l2": "flushed (256 MiB write) before every timed step"},
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": int(round(n_launch_per_step * args.steps)),
+        "gpu_launches": n_launch,
+        "device_status": dev_status,
         "clocks": clocks,
+        "gamma_sweep": sweep,
+        "targets": targets,
         "kernels": kernels,
+        "source_digest": source_digest(),
     }
     if opt_line is not None:
         line["optimizer"] = opt_line
@@ -527,13 +753,7 @@ def kernel_table(prof, work, peaks, sms):
         if roofline is not None:
             continue
         if bound == "alu":
-            ops = OPS_PER_NORMAL.get(n, 19.0)
-            peak = sms * LANES_PER_SM * peaks["sm_max_mhz"] * 1e6 / ops / 1e9
-            roofline = {"kernel": n, "bound": "alu", "achieved": round(rate / 1e9, 2),
-                        "peak": round(peak, 2), "unit": "Gnormal/s",
-                        "frac": round(rate / 1e9 / peak, 4), "traffic": None,
-                        "peak_basis": f"{sms} SMs x {LANES_PER_SM} lanes x "
-                                      f"{peaks['sm_max_mhz']:.0f} MHz / {ops:.0f} ops per normal"}
+            roofline = alu_roofline(n, rate / 1e9, sms, peaks)
         elif bound == "hbm":
             roofline = {"kernel": n, "bound": "hbm", "achieved": round(rate / 1e9, 2),
                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -542,7 +762,7 @@ def kernel_table(prof, work, peaks, sms):
             roofline = {"kernel": n, "bound": "tensor", "achieved": round(rate / 1e12, 2),
                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                         "frac": round(rate / 1e12 / peaks["bf16_tflops"], 4), "traffic": None}
-        roofline["peak_source"] = peaks["source"]
+        roofline.setdefault("peak_source", peaks["source"])
     return kernels, roofline
 
 
@@ -615,9 +835,9 @@ def run_attn(args) -> None:
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     kernels, roofline = kernel_table(prof, lambda n: attn_kernel_work(n, aw), peaks, sms)
     if roofline is not None and roofline["bound"] == "alu":
-        gc = generator_ceiling(dust, torch, dev)
-        roofline["generator_ceiling"] = round(gc, 2)
-        roofline["frac_of_generator_ceiling"] = round(roofline["achieved"] / gc, 4)
+        roofline.update(generator_ceiling(dust, torch, dev))
+        roofline["frac_of_generator"] = round(roofline["achieved"] / roofline["generator_gnormal_s"],
+                                              4)
     e2e = None
     if not args.no_e2e:
         hG, hD, hx = (t.cpu().pin_memory() for t in (G, dO, x))
@@ -881,12 +1101,13 @@ def run_head(args) -> None:
     units = hw.N * hw.K
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     kernels, roofline = kernel_table(prof, lambda n: head_kernel_work(n, hw), peaks, sms)
-    if roofline is not None and (roofline["kernel"], hw.name) in MEASURED_TRAFFIC:
-        roofline["traffic"], roofline["traffic_source"] = MEASURED_TRAFFIC[(roofline["kernel"], hw.name)]
+    if roofline is not None:
+        roofline["traffic"], roofline["traffic_source"] = measured_traffic(roofline["kernel"],
+                                                                           hw.name)
     if roofline is not None and roofline["bound"] == "alu":
-        gc = generator_ceiling(dust, torch, dev)
-        roofline["generator_ceiling"] = round(gc, 2)
-        roofline["frac_of_generator_ceiling"] = round(roofline["achieved"] / gc, 4)
+        roofline.update(generator_ceiling(dust, torch, dev))
+        roofline["frac_of_generator"] = round(roofline["achieved"] / roofline["generator_gnormal_s"],
+                                              4)
     # end to end: logits, targets and hidden states from pinned host memory, G_W back
     e2e = None
     if not args.no_e2e:
@@ -993,7 +1214,16 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", type=int, default=2, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", type=int, default=5, choices=sorted(workloads.WORKLOADS),
+                    help="workload id (default 5: the 48 linear layers of a 12-block stack)")
+    ap.add_argument("--gamma", type=float, default=None,
+                    help="credit discount of the headline (default 0.9 for the stack, else the "
+                         "workload's own)")
+    ap.add_argument("--buckets", type=int, default=4,
+                    help="buckets of consecutive layers for the stack's G_W all-reduce (N > 1)")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the gamma sweep")
+    ap.add_argument("--no-targets", action="store_true",
+                    help="skip the contraction / scan / reduction target measurements")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

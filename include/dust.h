@@ -219,14 +219,21 @@ dust_status dust_spsa_estimate(const float* p, int32_t P, int32_t P_total, int32
  * r: fp32 [K_chunk, ld_r] holds the credit rows of draws key.draw_offset .. +K_chunk.
  * x: [N, d_in] of dtype dt.  G_W: fp32 [d_out, d_in]; accumulate != 0 adds to it (chunks of
  * one population), accumulate == 0 overwrites it.  g_out: optional fp32 [N, d_out] copy of g
- * (NULL to skip).  For bf16, g enters the tensor-core contraction rounded to bf16 (fp32
- * accumulation).  Deterministic (split-K partials are reduced in a fixed order).
+ * (NULL to skip).  For bf16 x the contraction runs on the tensor cores with fp32
+ * accumulation, and g enters it as g_terms bf16 terms:
+ *   g_terms = 1: g rounded once to bf16 (relative rounding error up to 2^-9 per element;
+ *                about 1.7e-3 relative Frobenius error of G_W when g is noise-dominated);
+ *   g_terms = 2: hi = bf16(g) and lo = bf16(g - hi), both multiplied by x into the same
+ *                accumulator (about 16 significant bits of g; twice the tensor-core work).
+ * fp32 layers contract the fp32 g and accept either value.  2 N must fit in 31 bits.
+ * Deterministic (split-K partials are reduced in a fixed order).  The workspace size does
+ * not depend on g_terms.
  */
 dust_status dust_weight_grad(const float* r, int64_t ld_r, const void* x, dust_dtype dt,
                              int64_t N, int32_t d_in, int32_t d_out, int32_t K_chunk,
                              int32_t K_total, float sigma, dust_noise_key key, float* G_W,
-                             int accumulate, float* g_out, void* workspace, size_t ws_bytes,
-                             void* stream);
+                             int accumulate, float* g_out, int32_t g_terms, void* workspace,
+                             size_t ws_bytes, void* stream);
 
 /*
  * dust_credit without a caller workspace (the paper has no counterpart: this is a packaging
@@ -236,11 +243,16 @@ dust_status dust_weight_grad(const float* r, int64_t ld_r, const void* x, dust_d
  * workspace: the look-back scratch lives in a 4 MiB static device array of the library, which
  * every device that loads the library holds until the process exits.  The call allocates
  * nothing (no cudaMalloc, no allocating library routine).
- *   - Sizes whose scratch (dust_workspace_size(DUST_OP_CREDIT, ...)) exceeds 4 MiB are
- *     rejected with DUST_ERR_WORKSPACE; the scratch is 16 K bytes per 128 tokens plus 256
- *     (K <= 128), so K = 32 allows N up to about 1.05 million tokens and K = 64 about 520,000.
- *   - The first call on a device looks up the array's device address (once per device, with
- *     that device current); make that first call before any stream capture.
+ *   - Sizes whose scratch exceeds 4 MiB are rejected with DUST_ERR_WORKSPACE.  The scratch is
+ *     exactly dust_workspace_size(DUST_OP_CREDIT, DUST_F32, N, 0, 0, K) bytes, so a caller
+ *     checks a size by comparing that value with 4 MiB (4194304).  For K <= 128 it is
+ *     about 16 K bytes per 128 tokens plus 256, so K = 32 allows N up to about 1.05 million
+ *     tokens and K = 64 about 520,000.  For K > 128 the draws form ceil(K / 128) groups of
+ *     up to 128 rows, each with its own look-back state, plus a 4 N byte per-token mean:
+ *     K = 256 allows N up to about 116,000 tokens.
+ *   - The first call on a device (and the first after that device's context was reset) looks
+ *     up the array's device address, with that device current; make that first call before
+ *     any stream capture.  Concurrent first calls from several host threads are safe.
  *   - Every call shares the one array, and the ticket and flags are cleared on `stream` before
  *     each launch.  Calls whose kernels overlap on the GPU (other streams, other threads)
  *     race on the scratch and give wrong results: serialize them.
@@ -287,9 +299,9 @@ dust_status dust_optimizer_step(const dust_opt_params* opt, const float* G, floa
 dust_status dust_weight_grad_step(const float* r, int64_t ld_r, const void* x, dust_dtype dt,
                                   int64_t N, int32_t d_in, int32_t d_out, int32_t K_chunk,
                                   int32_t K_total, float sigma, dust_noise_key key, float* G_W,
-                                  int accumulate, float* g_out, const dust_opt_params* opt,
-                                  float* W, void* W_bf16, float* m, float* v, void* workspace,
-                                  size_t ws_bytes, void* stream);
+                                  int accumulate, float* g_out, int32_t g_terms,
+                                  const dust_opt_params* opt, float* W, void* W_bf16, float* m,
+                                  float* v, void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * Grouped forms: the same three steps for many bf16 layers that share the token batch
@@ -330,11 +342,11 @@ dust_status dust_credit_grouped(const dust_layer_desc* layers, int32_t n_layers,
                                 int64_t N, const int32_t* cu_seqlens, int32_t n_seq, float gamma,
                                 void* workspace, size_t ws_bytes, void* stream);
 /* dust_weight_grad for every layer: reads r (K_chunk rows) and x; writes (or adds to) G_W and,
- * where not NULL, g_out. */
+ * where not NULL, g_out; g_terms (1 or 2) as in dust_weight_grad, for every layer. */
 dust_status dust_weight_grad_grouped(const dust_layer_desc* layers, int32_t n_layers, int64_t N,
                                      int32_t K_chunk, int32_t K_total, float sigma,
-                                     dust_noise_key key, int accumulate, void* workspace,
-                                     size_t ws_bytes, void* stream);
+                                     dust_noise_key key, int accumulate, int32_t g_terms,
+                                     void* workspace, size_t ws_bytes, void* stream);
 /* Workspace bytes of a grouped call of step `op`. */
 size_t dust_workspace_size_grouped(dust_op op, const dust_layer_desc* layers, int32_t n_layers,
                                    int64_t N, int32_t K);
@@ -374,6 +386,14 @@ dust_status dust_debug_philox(const uint32_t* ctr, int64_t n, uint64_t seed, uin
  * its rate bounds what the noise kernels can reach.  key.channel_offset a multiple of 4. */
 dust_status dust_debug_normal_sum(dust_noise_key key, int64_t n, int32_t n_quads, float* out,
                                   void* stream);
+
+/* Measurement support: the generator's integer part alone.  out[g] (DEVICE uint32 [n]) = the
+ * XOR of the four Philox4x32-10 words of every block (key.channel_offset / 4 + j,
+ * key.token_offset + g, key.draw_offset, key.layer_id), j < n_blocks, under the estimator's
+ * key.  Its rate (4 n n_blocks words per launch) shows what the widening multiplies alone
+ * allow the noise kernels.  key.channel_offset a multiple of 4; out 4-byte aligned. */
+dust_status dust_debug_word_sum(dust_noise_key key, int64_t n, int32_t n_blocks, uint32_t* out,
+                                void* stream);
 
 /* Test support: the next dust_credit launch on any stream skips publishing the look-back
  * status of token block `block` (-1: none), so that the block before it waits until its

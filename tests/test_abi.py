@@ -75,12 +75,16 @@ def test_credit_and_weight_grad_reject_bad_arguments():
     key = z.NoiseKey(1).c()
     # sigma must be > 0 (division by sigma); K_total >= K_chunk
     assert L.dust_weight_grad(0x1000, 256, 0x1000, 1, 256, 64, 64, 4, 4, 0.0, key, 0x1000, 0,
-                              None, None, 0, None) == 1
+                              None, 2, None, 0, None) == 1
     assert L.dust_weight_grad(0x1000, 256, 0x1000, 1, 256, 64, 64, 4, 2, 1e-3, key, 0x1000, 0,
-                              None, None, 0, None) == 1
+                              None, 2, None, 0, None) == 1
     bad = z.dust_noise_key(1, 0, 0xFFFFFFFF, 0, 0)   # draw index would wrap
     assert L.dust_weight_grad(0x1000, 256, 0x1000, 1, 256, 64, 64, 4, 4, 1e-3, bad, 0x1000, 0,
-                              None, None, 0, None) == 1
+                              None, 2, None, 0, None) == 1
+    # g enters the contraction as one or two bf16 terms, nothing else
+    for terms in (0, 3, -1):
+        assert L.dust_weight_grad(0x1000, 256, 0x1000, 1, 256, 64, 64, 4, 4, 1e-3, key, 0x1000,
+                                  0, None, terms, None, 0, None) == 1
 
 
 def test_product_package_does_not_import_the_oracle():

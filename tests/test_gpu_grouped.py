@@ -69,6 +69,51 @@ def test_grouped_stack_matches_oracle(z):
         assert _dev.rel_fro(_dev.host(st.G_W[l]), ref["G_W"]) <= _dev.GW_FRO, l
 
 
+def test_stack_bucketed_reduce_sees_every_layer_once(z):
+    """The stack's weight estimate in buckets of consecutive layers, each bucket's span of the
+    flat G_W buffer handed to a collective on a side stream (here a stand-in that doubles it on
+    the current stream): every layer comes out doubled, once."""
+    import torch
+    N, K, sigma, gamma, seed = 640, 6, 1e-3, 0.9, 0x5EED0005
+    layers = _stack(N, 64, 7)
+    cu_d = _dev.cu_to_device(workloads.random_segments(8, N, 50, 300))
+    dev_layers = [(*_dev.layer_to_device(L), L.shape.layer_id) for L in layers]
+    st = z.DustStack(dev_layers, K)
+    ref = [g.clone() for g in st.estimate(cu_d, sigma, gamma, seed)]
+    for buckets in (1, 3, 8):
+        seen = []
+
+        def reduce(G):
+            seen.append(G.numel())
+            G.mul_(2.0)
+
+        st.estimate(cu_d, sigma, gamma, seed, reduce=reduce, buckets=buckets)
+        torch.cuda.synchronize()
+        assert sum(seen) == sum(m for _, m in st.layout) and len(seen) == min(buckets, 8)
+        for l in range(len(layers)):
+            assert _dev.rel_fro(_dev.host(st.G_W[l]), 2.0 * _dev.host(ref[l])) < 1e-6, (buckets, l)
+
+
+def test_stack_estimate_from_host_matches_device_inputs(z):
+    """The stack from pinned host inputs (uploaded in runs of whole sequences, each run's
+    estimate overlapped with the next run's upload, G_W accumulated over the runs) gives the
+    estimate of the device inputs."""
+    import torch
+    N, K, sigma, gamma, seed = 1024, 8, 1e-3, 0.99, 0x5EED0005
+    layers = _stack(N, 32, 9)
+    cu = workloads.random_segments(10, N, 60, 200)
+    dev_layers = [(*_dev.layer_to_device(L), L.shape.layer_id) for L in layers]
+    st = z.DustStack(dev_layers, K)
+    ref = [_dev.host(g).copy() for g in st.estimate(_dev.cu_to_device(cu), sigma, gamma, seed)]
+    host = [tuple(t.cpu().pin_memory() for t in (x, W, u)) for x, W, u, _ in dev_layers]
+    for x, W, u, _ in dev_layers:
+        for t in (x, W, u):
+            t.zero_()
+    G = st.estimate_from_host(host, cu, sigma, gamma, seed, chunks=4).numpy()
+    for l, (o, m) in enumerate(st.layout):
+        assert _dev.rel_fro(G[o:o + m].reshape(ref[l].shape), ref[l]) < 1e-5, l
+
+
 def test_grouped_rejects_bad_descriptors(z):
     import ctypes
     d = (z.dust_layer_desc * 1)()

@@ -56,6 +56,40 @@ def test_philox_words_bit_exact_and_normals_close():
     assert err.max() <= _dev.NORMAL_ATOL, err.max()
 
 
+def test_philox_words_match_published_known_answers():
+    """The device generator on the published Philox4x32-10 known-answer vectors."""
+    import torch
+    from tests.test_oracle_noise import kat_vectors
+    for ctr, key, out in kat_vectors():
+        seed = int(key[0]) | (int(key[1]) << 32)
+        w, _ = z.dust_debug_philox(torch.from_numpy(ctr.reshape(1, 4).view(np.int32)).cuda(), seed)
+        assert np.array_equal(_dev.host(w).view(np.uint32)[0], out), (ctr, key)
+
+
+def test_philox_words_bit_exact_over_1e8_counters():
+    """Words are integers: the device equals the oracle bit for bit over 2^27 (1.3e8) sampled
+    counters in chunks of 2^24, each chunk with its own 64-bit seed: uniform random words (every
+    counter word >= 2^31 in about half the blocks, all four in 1/16), counters shaped like the
+    estimator's (small quad, token, draw and layer words), and all-high words."""
+    import torch
+    rng = np.random.default_rng(4242)
+    chunk, n_chunks, total = 1 << 24, 8, 0
+    for c in range(n_chunks):
+        ctr = rng.integers(0, 2**32, size=(chunk, 4), dtype=np.uint64).astype(np.uint32)
+        if c % 4 == 1:
+            ctr &= np.array([0xFFF, 0xFFFFF, 0xFFFF, 0x3F], dtype=np.uint32)
+        elif c % 4 == 2:
+            ctr |= np.uint32(0x80000000)
+        seed = int(rng.integers(0, 2**63, dtype=np.int64)) * 2 + c % 2
+        ref, _ = oracle.philox_batch(ctr, seed, want_normals=False)
+        w, _ = z.dust_debug_philox(torch.from_numpy(ctr.view(np.int32)).cuda(), seed)
+        got = _dev.host(w).view(np.uint32)
+        assert np.array_equal(got, ref), (c, int(np.count_nonzero(np.any(got != ref, axis=1))))
+        total += chunk
+        del w
+    assert total >= 10**8
+
+
 def test_normals_near_u_one_and_u_zero():
     """Words whose uniforms sit at the ends of (0, 1): rho -> 0 and rho -> 5.77."""
     import torch
@@ -71,6 +105,20 @@ def test_normals_near_u_one_and_u_zero():
     err = np.abs(zn[extreme] - z_ref[extreme]).max()
     print(f"max error at u0 < 0.001 or u0 > 0.999: {err:.3e}")
     assert err <= _dev.NORMAL_ATOL
+
+
+def test_philox_only_probe_xors_the_mapped_words():
+    """dust_debug_word_sum (the Philox-only rate probe) XORs exactly the words of the
+    estimator's counters: channel quad, token offset, draw and layer."""
+    n, nb, c0 = 300, 13, 8
+    key = z.NoiseKey(0x5EED0002, layer_id=9, draw_offset=5, token_offset=1000, channel_offset=c0)
+    got = _dev.host(z.dust_debug_word_sum(key, n, nb)).view(np.uint32)
+    q, t = np.meshgrid(np.arange(nb, dtype=np.uint32) + np.uint32(c0 // 4),
+                       np.arange(n, dtype=np.uint32) + np.uint32(1000), indexing="ij")
+    ctr = np.stack([q, t, np.full_like(q, 5), np.full_like(q, 9)], axis=-1).reshape(-1, 4)
+    words, _ = oracle.philox_batch(ctr, 0x5EED0002, want_normals=False)
+    ref = np.bitwise_xor.reduce(words.reshape(nb, n, 4), axis=(0, 2))
+    assert np.array_equal(got, ref)
 
 
 def test_generator_throughput_probe_sums_the_mapped_normals():
@@ -287,14 +335,14 @@ def test_credit_unaligned_leading_dimension():
 
 
 # ------------------------------------------------------------------------- weight estimate
-def _wgrad_case(L, K_chunk, K_total, sigma, key, r_seed, dtype):
+def _wgrad_case(L, K_chunk, K_total, sigma, key, r_seed, dtype, g_terms=2):
     import torch
     N = L.x_store.shape[0]
     d_out = L.W_store.shape[0]
     r = workloads.gaussian_losses(r_seed, K_chunk, N, scale=0.05)
     x = _dev.to_device(L.x_store, dtype)
     GW, g = z.dust_weight_grad(torch.from_numpy(r).cuda(), x, d_out, K_total, sigma, key,
-                               g_out=True)
+                               g_out=True, g_terms=g_terms)
     torch.cuda.synchronize()
     g_ref = oracle.output_error(r, K_total, sigma, key.seed, d_out, key.layer_id,
                                 key.draw_offset, key.token_offset)
@@ -302,18 +350,23 @@ def _wgrad_case(L, K_chunk, K_total, sigma, key, r_seed, dtype):
     return _dev.host(GW), _dev.host(g), GW_ref, g_ref
 
 
+@pytest.mark.parametrize("g_terms", [1, 2])
 @pytest.mark.parametrize("N,d_in,d_out,K", [
     (256, 256, 128, 4),
     (300, 272, 144, 6),      # ragged tokens, columns and rows
     (4100, 768, 512, 8),     # several token tiles: split-K
     (16, 16, 16, 2),
 ])
-def test_weight_grad_bf16_matches_oracle(N, d_in, d_out, K):
+def test_weight_grad_bf16_matches_oracle(N, d_in, d_out, K, g_terms):
+    """Random credit makes g pure noise, the worst case for the bf16 rounding of g: one term
+    stays within the required 2e-3, two terms (hi + lo) within the fp32 bound 1e-4."""
     L = workloads.custom_layer(2000 + N, N, d_in, d_out, "bf16", 0.02)
     key = z.NoiseKey(0x5EED0003, layer_id=1, draw_offset=40, token_offset=3)
-    GW, g, GW_ref, g_ref = _wgrad_case(L, K, K + 40, 1e-3, key, 80 + N, "bf16")
+    GW, g, GW_ref, g_ref = _wgrad_case(L, K, K + 40, 1e-3, key, 80 + N, "bf16", g_terms)
     _dev.assert_fp32_close(g, g_ref, "g")
-    assert _dev.rel_fro(GW, GW_ref) <= _dev.GW_FRO, _dev.rel_fro(GW, GW_ref)
+    e = _dev.rel_fro(GW, GW_ref)
+    print(f"G_W rel-Fro with {g_terms} bf16 term(s) of g: {e:.3e}")
+    assert e <= (_dev.GW_FRO if g_terms == 1 else _dev.FP32_FRO), e
 
 
 def test_weight_grad_f32_matches_oracle():

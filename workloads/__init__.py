@@ -9,8 +9,8 @@ Recipe (every workload):
     segment lengths; for the 48-layer stack the order repeats per layer in the order
     layer_id = 4*block + {0: QKV, 1: O, 2: W_in, 3: W_out}.
   * x ~ N(0, 1), u ~ N(0, 1), W ~ N(0, w_std^2), drawn in float64, rounded to float32 by
-    numpy (round to nearest even) and, for bf16 workloads, from float32 to bf16 by torch
-    (round to nearest even).  The oracle reads the rounded values exactly.
+    numpy (round to nearest even) and, for bf16 workloads, from float32 to bf16 (round to
+    nearest even, the same values as torch's conversion).  The oracle reads the rounded values exactly.
   * noise seed 0x5EED0000 + cfg_id, draw_offset 0, token_offset 0.
   * packed variable-length sequences (the attention-projection workload): lengths are iid
     integers uniform on [256, 2048] drawn until the stream of N tokens is full; the last
@@ -23,6 +23,7 @@ tokens); FineWeb and trained weights are not used, only their shapes.
 from __future__ import annotations
 
 import dataclasses
+import functools
 from typing import List, Optional, Sequence
 
 import numpy as np
@@ -109,46 +110,69 @@ def cu_seqlens_from_lengths(lengths: Sequence[int]) -> np.ndarray:
 
 
 def to_bf16_bits(a32: np.ndarray) -> np.ndarray:
-    """float32 -> bf16 bit patterns (uint16), round to nearest even, via torch."""
-    import torch
-    t = torch.from_numpy(np.ascontiguousarray(a32, dtype=np.float32)).to(torch.bfloat16)
-    return t.view(torch.int16).numpy().view(np.uint16)
+    """float32 -> bf16 bit patterns (uint16), round to nearest even: the top 16 bits after
+    adding 0x7fff plus the lowest kept bit (ties go to the even neighbour); a NaN stays a quiet
+    NaN.  The same values as torch's float32 -> bfloat16 conversion (checked by a test)."""
+    a = np.ascontiguousarray(a32, dtype=np.float32)
+    b = a.view(np.uint32)
+    out = ((b + (np.uint32(0x7FFF) + ((b >> np.uint32(16)) & np.uint32(1))))
+           >> np.uint32(16)).astype(np.uint16)
+    nan = np.isnan(a)
+    if nan.any():
+        out[nan] = ((b[nan] >> np.uint32(16)) | np.uint32(0x40)).astype(np.uint16)
+    return out
 
 
 def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
+def _widen(store: np.ndarray, dtype: str) -> np.ndarray:
+    """The stored values (float32, or bf16 bit patterns) widened exactly to float64."""
+    return store.astype(np.float64) if dtype == "f32" else bf16_bits_to_f64(store)
+
+
 @dataclasses.dataclass
 class LayerData:
     """One layer's inputs. ``*_store`` is what the device receives (float32 array, or bf16
-    bit patterns as uint16); ``*_f64`` is the same stored value widened exactly."""
+    bit patterns as uint16); ``*_f64`` is the same stored value widened exactly (made on first
+    use, so that a large stack that only goes to the device holds no float64 copy)."""
     shape: LayerShape
     dtype: str
     x_store: np.ndarray
     W_store: np.ndarray
     u_store: np.ndarray
-    x_f64: np.ndarray
-    W_f64: np.ndarray
-    u_f64: np.ndarray
+
+    @functools.cached_property
+    def x_f64(self) -> np.ndarray:
+        return _widen(self.x_store, self.dtype)
+
+    @functools.cached_property
+    def W_f64(self) -> np.ndarray:
+        return _widen(self.W_store, self.dtype)
+
+    @functools.cached_property
+    def u_f64(self) -> np.ndarray:
+        return _widen(self.u_store, self.dtype)
+
+
+def _store(rng, shape, std, dtype):
+    a32 = (rng.standard_normal(shape) * std).astype(np.float32)
+    return a32 if dtype == "f32" else to_bf16_bits(a32)
 
 
 def _draw(rng, shape, std, dtype):
-    a = rng.standard_normal(shape) * std
-    a32 = a.astype(np.float32)
-    if dtype == "f32":
-        return a32, a32.astype(np.float64)
-    bits = to_bf16_bits(a32)
-    return bits, bf16_bits_to_f64(bits)
+    s = _store(rng, shape, std, dtype)
+    return s, _widen(s, dtype)
 
 
 def make_layer(rng: np.random.Generator, shape: LayerShape, N: int, dtype: str,
                w_std: Optional[float]) -> LayerData:
     std_w = (1.0 / np.sqrt(shape.d_in)) if w_std is None else w_std
-    xs, x64 = _draw(rng, (N, shape.d_in), 1.0, dtype)
-    Ws, W64 = _draw(rng, (shape.d_out, shape.d_in), std_w, dtype)
-    us, u64 = _draw(rng, (N, shape.d_out), 1.0, dtype)
-    return LayerData(shape, dtype, xs, Ws, us, x64, W64, u64)
+    xs = _store(rng, (N, shape.d_in), 1.0, dtype)
+    Ws = _store(rng, (shape.d_out, shape.d_in), std_w, dtype)
+    us = _store(rng, (N, shape.d_out), 1.0, dtype)
+    return LayerData(shape, dtype, xs, Ws, us)
 
 
 @dataclasses.dataclass

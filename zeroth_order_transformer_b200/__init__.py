@@ -44,7 +44,7 @@ EXPORTED_SYMBOLS = (
     "dust_credit_grouped", "dust_weight_grad_grouped", "dust_workspace_size_grouped",
     "dust_optimizer_step", "dust_weight_grad_step", "dust_noisy_logits_ce",
     "dust_debug_normal_sum", "dust_debug_fwd_plan", "dust_attn_reward", "dust_discounted_credit",
-    "dust_spsa_probe", "dust_spsa_estimate", "dust_noisy_linear_output",
+    "dust_spsa_probe", "dust_spsa_estimate", "dust_noisy_linear_output", "dust_debug_word_sum",
 )
 
 DUST_OPT_SGD_MOMENTUM = 1
@@ -115,7 +115,7 @@ def lib() -> ctypes.CDLL:
                                             dust_noise_key, vp, i64, vp, sz, vp]
         L.dust_credit.argtypes = [vp, i64, i32, i64, vp, i32, f32, vp, i64, vp, sz, vp]
         L.dust_weight_grad.argtypes = [vp, i64, vp, ctypes.c_int, i64, i32, i32, i32, i32, f32,
-                                       dust_noise_key, vp, ctypes.c_int, vp, vp, sz, vp]
+                                       dust_noise_key, vp, ctypes.c_int, vp, i32, vp, sz, vp]
         L.dust_credit_no_alloc.argtypes = [vp, i64, i32, i64, vp, i32, f32, vp, i64, vp]
         L.dust_credit_no_alloc.restype = ctypes.c_int
         dp = ctypes.POINTER(dust_layer_desc)
@@ -123,7 +123,7 @@ def lib() -> ctypes.CDLL:
                                                     sz, vp]
         L.dust_credit_grouped.argtypes = [dp, i32, i32, i64, vp, i32, f32, vp, sz, vp]
         L.dust_weight_grad_grouped.argtypes = [dp, i32, i64, i32, i32, f32, dust_noise_key,
-                                               ctypes.c_int, vp, sz, vp]
+                                               ctypes.c_int, i32, vp, sz, vp]
         L.dust_workspace_size_grouped.argtypes = [ctypes.c_int, dp, i32, i64, i32]
         L.dust_workspace_size_grouped.restype = sz
         for name in ("dust_noisy_linear_fwd_grouped", "dust_credit_grouped",
@@ -133,8 +133,8 @@ def lib() -> ctypes.CDLL:
         L.dust_optimizer_step.argtypes = [op, vp, vp, vp, vp, vp, i64, vp]
         L.dust_optimizer_step.restype = ctypes.c_int
         L.dust_weight_grad_step.argtypes = [vp, i64, vp, ctypes.c_int, i64, i32, i32, i32, i32,
-                                            f32, dust_noise_key, vp, ctypes.c_int, vp, op, vp, vp,
-                                            vp, vp, vp, sz, vp]
+                                            f32, dust_noise_key, vp, ctypes.c_int, vp, i32, op, vp,
+                                            vp, vp, vp, vp, sz, vp]
         L.dust_weight_grad_step.restype = ctypes.c_int
         L.dust_noisy_logits_ce.argtypes = [vp, i64, ctypes.c_int, vp, i64, i32, i32, i32, i32,
                                            f32, dust_noise_key, vp, i64, vp, sz, vp]
@@ -162,6 +162,8 @@ def lib() -> ctypes.CDLL:
         L.dust_spsa_estimate.restype = ctypes.c_int
         L.dust_debug_normal_sum.argtypes = [dust_noise_key, i64, i32, vp, vp]
         L.dust_debug_normal_sum.restype = ctypes.c_int
+        L.dust_debug_word_sum.argtypes = [dust_noise_key, i64, i32, vp, vp]
+        L.dust_debug_word_sum.restype = ctypes.c_int
         L.dust_debug_credit_skip_publish.argtypes = [i32]
         L.dust_debug_credit_skip_publish.restype = None
         L.dust_debug_fwd_plan.argtypes = [i64, i32, i32, vp, i32, ctypes.POINTER(i32),
@@ -407,13 +409,16 @@ def dust_spsa_estimate(p, P_total: int, d_out: int, d_in: int, key: NoiseKey, G=
 
 def dust_credit_no_alloc(loss, cu_seqlens, gamma: float, r, stream=None):
     """dust_credit with the library's static 4 MiB scratch instead of a workspace, for callers
-    that cannot allocate device memory; ``r`` must be given (float32 [K, N]).  Calls that
-    overlap on the GPU share the scratch and race: serialize them."""
+    that cannot allocate device memory; ``r`` must be given (float32 [K, N], rows contiguous,
+    rows may be further apart, as may those of ``loss``).  Calls that overlap on the GPU share
+    the scratch and race: serialize them."""
     torch = _torch()
-    _cuda(loss, "loss"), _cuda(cu_seqlens, "cu_seqlens"), _cuda(r, "r")
+    _cuda_rows(loss, "loss"), _cuda(cu_seqlens, "cu_seqlens"), _cuda_rows(r, "r")
     if loss.dtype != torch.float32 or r.dtype != torch.float32 or cu_seqlens.dtype != torch.int32:
         raise TypeError("loss and r must be float32 and cu_seqlens int32")
     K, N = loss.shape
+    if tuple(r.shape) != (K, N):
+        raise ValueError(f"r must be [K, N] = [{K}, {N}] like loss, got {tuple(r.shape)}")
     st = lib().dust_credit_no_alloc(loss.data_ptr(), loss.stride(0), K, N, cu_seqlens.data_ptr(),
                                     cu_seqlens.numel() - 1, float(gamma), r.data_ptr(),
                                     r.stride(0), _stream(loss.device, stream))
@@ -421,10 +426,14 @@ def dust_credit_no_alloc(loss, cu_seqlens, gamma: float, r, stream=None):
     return r
 
 
+G_TERMS = 2  # default: g enters the bf16 contraction as hi + lo terms
+
+
 def dust_weight_grad(r, x, d_out: int, K_total: int, sigma: float, key: NoiseKey, G_W=None,
-                     accumulate: bool = False, g_out=None, workspace=None, stream=None
-                     ) -> Tuple[object, Optional[object]]:
-    """G_W[d_out, d_in] (fp32) and, if g_out is a tensor or True, g[N, d_out] (fp32)."""
+                     accumulate: bool = False, g_out=None, workspace=None, stream=None,
+                     g_terms: int = G_TERMS) -> Tuple[object, Optional[object]]:
+    """G_W[d_out, d_in] (fp32) and, if g_out is a tensor or True, g[N, d_out] (fp32).  For bf16
+    x, g enters the tensor cores as ``g_terms`` bf16 terms (2: hi + lo; 1: rounded once)."""
     torch = _torch()
     _cuda_rows(r, "r"), _cuda(x, "x")
     K_chunk, N = r.shape
@@ -445,7 +454,7 @@ def dust_weight_grad(r, x, d_out: int, K_total: int, sigma: float, key: NoiseKey
     st = lib().dust_weight_grad(r.data_ptr(), r.stride(0), x.data_ptr(), dt, N, d_in, d_out,
                                 K_chunk, K_total, float(sigma), key.c(), G_W.data_ptr(),
                                 1 if accumulate else 0,
-                                g_out.data_ptr() if g_out is not None else None,
+                                g_out.data_ptr() if g_out is not None else None, int(g_terms),
                                 ws.data_ptr() if ws is not None else None, nb,
                                 _stream(x.device, stream))
     _check(st, "dust_weight_grad")
@@ -468,7 +477,8 @@ def dust_optimizer_step(opt: dust_opt_params, G, W, m, v=None, W_bf16=None, stre
 
 def dust_weight_grad_step(r, x, d_out: int, K_total: int, sigma: float, key: NoiseKey,
                           opt: dust_opt_params, W, m, v=None, W_bf16=None, G_W=None,
-                          accumulate: bool = False, g_out=None, workspace=None, stream=None):
+                          accumulate: bool = False, g_out=None, workspace=None, stream=None,
+                          g_terms: int = G_TERMS):
     """dust_weight_grad with the optimizer step fused into the pass that finishes G_W."""
     _cuda(r, "r"), _cuda(x, "x"), _cuda(W, "W"), _cuda(m, "m")
     K_chunk, N = r.shape
@@ -478,7 +488,8 @@ def dust_weight_grad_step(r, x, d_out: int, K_total: int, sigma: float, key: Noi
                                                        K_chunk), x.device)
     st = lib().dust_weight_grad_step(r.data_ptr(), r.stride(0), x.data_ptr(), dt, N, d_in, d_out,
                                      K_chunk, K_total, float(sigma), key.c(), _ptr(G_W),
-                                     1 if accumulate else 0, _ptr(g_out), ctypes.byref(opt),
+                                     1 if accumulate else 0, _ptr(g_out), int(g_terms),
+                                     ctypes.byref(opt),
                                      W.data_ptr(), _ptr(W_bf16), m.data_ptr(), _ptr(v),
                                      ws.data_ptr() if ws is not None else None, nb,
                                      _stream(x.device, stream))
@@ -522,6 +533,21 @@ def dust_debug_normal_sum(key: NoiseKey, n: int, n_quads: int, out=None, device=
     return out
 
 
+def dust_debug_word_sum(key: NoiseKey, n: int, n_blocks: int, out=None, device=None,
+                        stream=None):
+    """out[g] (int32 bits of uint32) = XOR of the words of the Philox blocks (channel quad
+    key.channel_offset / 4 + j, token key.token_offset + g, draw key.draw_offset), j < n_blocks:
+    the generator's integer part alone, as a throughput probe."""
+    torch = _torch()
+    if out is None:
+        out = torch.empty(n, dtype=torch.int32, device=device or "cuda")
+    _cuda(out, "out")
+    st = lib().dust_debug_word_sum(key.c(), n, n_blocks, out.data_ptr(),
+                                   _stream(out.device, stream))
+    _check(st, "dust_debug_word_sum")
+    return out
+
+
 def dust_debug_fwd_plan(N: int, K: int, d_outs, sms: int):
     """(persistent, tail split) of the bf16 forward for layers of output widths `d_outs` on a
     device with `sms` SMs (host only; no device needed)."""
@@ -553,14 +579,34 @@ def dust_profile_read(max_records: int = 1 << 16):
     return [(names[i].decode(), float(ms[i])) for i in range(n)]
 
 
+def _sequence_cuts(cu, N: int, chunks: int):
+    """Token cuts [0, ..., N] at sequence ends near k N / chunks, kept at multiples of 4 tokens
+    so that every run's row and column views stay 16-byte aligned."""
+    import numpy as np
+    ends = cu[(cu % 4 == 0) & (cu > 0) & (cu < N)]
+    cuts = [0]
+    for c in range(1, chunks):
+        if ends.size == 0:
+            break
+        e = int(ends[int(np.argmin(np.abs(ends - N * c / chunks)))])
+        if e > cuts[-1]:
+            cuts.append(e)
+    cuts.append(N)
+    return cuts
+
+
 class DustStack:
     """Many bf16 layers sharing one token batch (a transformer block stack), estimated with the
     grouped calls: one launch per step for up to 64 layers.  ``layers`` is a list of
-    (x, W, u, layer_id) device tensors; outputs live in ``dloss[l]``, ``r[l]``, ``G_W[l]``."""
+    (x, W, u, layer_id) device tensors; outputs live in ``dloss[l]``, ``r[l]``, ``G_W[l]``.
+    The weight estimates are views of one flat fp32 buffer ``G_W_flat`` (layer l at
+    ``layout[l]``), so that consecutive layers can be exchanged between ranks in one call."""
 
-    def __init__(self, layers, K: int, want_g: bool = False):
+    def __init__(self, layers, K: int, want_g: bool = False, g_terms: int = G_TERMS):
+        from . import distributed
         torch = _torch()
         self.K = K
+        self.g_terms = g_terms
         self.layers = layers
         x0 = layers[0][0]
         self.N = x0.shape[0]
@@ -568,8 +614,11 @@ class DustStack:
         n = len(layers)
         self.dloss = [torch.empty((K, self.N), dtype=torch.float32, device=dev) for _ in range(n)]
         self.r = [torch.empty((K, self.N), dtype=torch.float32, device=dev) for _ in range(n)]
-        self.G_W = [torch.empty((W.shape[0], W.shape[1]), dtype=torch.float32, device=dev)
-                    for (_, W, _, _) in layers]
+        self.layout, total = distributed.flat_layout([(W.shape[0], W.shape[1])
+                                                      for (_, W, _, _) in layers])
+        self.G_W_flat = torch.empty(total, dtype=torch.float32, device=dev)
+        self.G_W = [self.G_W_flat[o:o + m].view(W.shape[0], W.shape[1])
+                    for (o, m), (_, W, _, _) in zip(self.layout, layers)]
         self.g = ([torch.empty((self.N, W.shape[0]), dtype=torch.float32, device=dev)
                    for (_, W, _, _) in layers] if want_g else None)
         self.desc = (dust_layer_desc * n)()
@@ -578,6 +627,8 @@ class DustStack:
                 _cuda(t, nm)
                 if t.dtype != torch.bfloat16:
                     raise TypeError("grouped calls take bf16 layers")
+            if x.shape[0] != self.N or u.shape != (self.N, W.shape[0]) or x.shape[1] != W.shape[1]:
+                raise ValueError("layer shapes: x [N, d_in], W [d_out, d_in], u [N, d_out]")
             d = self.desc[l]
             d.x, d.W, d.u = x.data_ptr(), W.data_ptr(), u.data_ptr()
             d.d_in, d.d_out = x.shape[1], W.shape[0]
@@ -586,15 +637,71 @@ class DustStack:
             d.r, d.ld_r = self.r[l].data_ptr(), self.N
             d.G_W = self.G_W[l].data_ptr()
             d.g_out = self.g[l].data_ptr() if want_g else None
-        nbytes = max(int(lib().dust_workspace_size_grouped(op, self.desc, n, self.N, K))
-                     for op in range(3))
-        self.ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+        self.ws = torch.empty(max(self._ws_need(self.desc, n, self.N), 256), dtype=torch.uint8,
+                              device=dev)
+        self._comm = None
+
+    def _ws_need(self, desc, n: int, N: int) -> int:
+        return max(int(lib().dust_workspace_size_grouped(op, desc, n, N, self.K))
+                   for op in range(3))
+
+    @staticmethod
+    def _sub(desc, l0: int):
+        """Pointer to descriptor l0 of a descriptor array (a bucket of consecutive layers)."""
+        return ctypes.cast(ctypes.addressof(desc) + l0 * ctypes.sizeof(dust_layer_desc),
+                           ctypes.POINTER(dust_layer_desc))
+
+    def _weight_grad(self, desc, N: int, key, accumulate: bool, s: int, reduce, buckets: int):
+        """The grouped weight estimate; with ``reduce``, in buckets of consecutive layers, each
+        bucket's span of G_W_flat handed to ``reduce`` on a side stream as soon as its launch
+        is queued, so the exchange overlaps the later buckets' work."""
+        from . import distributed
+        torch = _torch()
+        n = len(self.layers)
+        nb = self.ws.numel()
+        if reduce is None:
+            _check(lib().dust_weight_grad_grouped(desc, n, N, self.K, self.K, float(self.sigma),
+                                                  key, 1 if accumulate else 0, self.g_terms,
+                                                  self.ws.data_ptr(), nb, s),
+                   "dust_weight_grad_grouped")
+            return
+        dev = self.ws.device
+        comp = torch.cuda.current_stream(dev)
+        if self._comm is None:
+            self._comm = torch.cuda.Stream(device=dev)
+        plan = distributed.plan_buckets([m for _, m in self.layout], buckets)
+        for l0, l1 in plan:
+            sub = self._sub(desc, l0)
+            need = int(lib().dust_workspace_size_grouped(DUST_OP_WEIGHT_GRAD, sub, l1 - l0, N,
+                                                         self.K))
+            if need > nb:
+                raise RuntimeError("stack workspace too small for a bucket")
+            _check(lib().dust_weight_grad_grouped(sub, l1 - l0, N, self.K, self.K,
+                                                  float(self.sigma), key,
+                                                  1 if accumulate else 0, self.g_terms,
+                                                  self.ws.data_ptr(), nb, s),
+                   "dust_weight_grad_grouped")
+            ev = torch.cuda.Event()
+            ev.record(comp)
+            self._comm.wait_event(ev)
+            with torch.cuda.stream(self._comm):
+                a, b = distributed.bucket_span(self.layout, (l0, l1))
+                reduce(self.G_W_flat[a:b])
+        comp.wait_stream(self._comm)
 
     def estimate(self, cu_seqlens, sigma: float, gamma: float, seed: int, draw_offset: int = 0,
-                 token_offset: int = 0, stream=None):
+                 token_offset: int = 0, stream=None, reduce=None, buckets: int = 4):
+        """Forward, credit and weight estimate of every layer on the device inputs.  ``reduce``
+        (optional, e.g. a sum over data-parallel ranks) is applied to G_W_flat in ``buckets``
+        spans of consecutive layers, overlapped with the remaining weight estimates; it must
+        run on the current stream (torch collectives do).  ``stream`` must be None (the
+        current stream) when ``reduce`` is given."""
+        if reduce is not None and stream is not None:
+            raise ValueError("reduce runs against the current stream; pass stream=None")
         n = len(self.layers)
         s = _stream(self.ws.device, stream)
         nb = self.ws.numel()
+        self.sigma = sigma
         key = NoiseKey(seed, 0, draw_offset, token_offset).c()
         _check(lib().dust_noisy_linear_fwd_grouped(self.desc, n, self.N, self.K, float(sigma), key,
                                                    self.ws.data_ptr(), nb, s),
@@ -602,10 +709,80 @@ class DustStack:
         _check(lib().dust_credit_grouped(self.desc, n, self.K, self.N, cu_seqlens.data_ptr(),
                                          cu_seqlens.numel() - 1, float(gamma), self.ws.data_ptr(),
                                          nb, s), "dust_credit_grouped")
-        _check(lib().dust_weight_grad_grouped(self.desc, n, self.N, self.K, self.K, float(sigma),
-                                              key, 0, self.ws.data_ptr(), nb, s),
-               "dust_weight_grad_grouped")
+        self._weight_grad(self.desc, self.N, key, False, s, reduce, buckets)
         return self.G_W
+
+    def estimate_from_host(self, host_layers, cu_seqlens, sigma: float, gamma: float,
+                           seed: int, G_host=None, chunks: int = 4, reduce=None,
+                           buckets: int = 4, draw_offset: int = 0, token_offset: int = 0):
+        """The estimate from inputs in pinned host memory (``host_layers``: one (x, W, u) per
+        layer, the shapes of the stack's device tensors, which receive them), with the upload
+        overlapped: the tokens are cut into ``chunks`` runs of whole sequences; each run of
+        every layer is copied on a copy stream while the previous run goes through the grouped
+        forward, credit and weight estimate (accumulated over the runs; token offsets keep the
+        whole batch's noise).  ``reduce`` as in ``estimate``, on the last run.  The flat G_W
+        comes back into ``G_host`` (pinned, allocated if None).  Synchronises."""
+        import numpy as np
+        torch = _torch()
+        dev = self.ws.device
+        cu = np.asarray(cu_seqlens, dtype=np.int64)
+        N = int(cu[-1])
+        if N != self.N or len(host_layers) != len(self.layers):
+            raise ValueError("host inputs do not match the stack")
+        self.sigma = sigma
+        cuts = _sequence_cuts(cu, N, chunks)
+        locs = [(cu[(cu >= a) & (cu <= b)] - a).astype(np.int32)
+                for a, b in zip(cuts[:-1], cuts[1:])]
+        cu_all = torch.from_numpy(np.concatenate(locs)).pin_memory().to(dev, non_blocking=True)
+        offs = np.cumsum([0] + [len(v) for v in locs])
+        if not hasattr(self, "_copy"):
+            self._copy = torch.cuda.Stream(device=dev)
+        comp = torch.cuda.current_stream(dev)
+        ready = []
+        self._copy.wait_stream(comp)
+        with torch.cuda.stream(self._copy):
+            for (_, W, _, _), (_, hW, _) in zip(self.layers, host_layers):
+                W.copy_(hW, non_blocking=True)
+            for a, b in zip(cuts[:-1], cuts[1:]):
+                for (x, _, u, _), (hx, _, hu) in zip(self.layers, host_layers):
+                    x[a:b].copy_(hx[a:b], non_blocking=True)
+                    u[a:b].copy_(hu[a:b], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(self._copy)
+                ready.append(ev)
+        n = len(self.layers)
+        nb = self.ws.numel()
+        s = _stream(dev, None)
+        for c, ((a, b), ev) in enumerate(zip(zip(cuts[:-1], cuts[1:]), ready)):
+            comp.wait_event(ev)
+            m = b - a
+            desc = (dust_layer_desc * n)()
+            for l in range(n):
+                d, src = desc[l], self.desc[l]
+                ctypes.memmove(ctypes.byref(d), ctypes.byref(src), ctypes.sizeof(dust_layer_desc))
+                d.x = src.x + a * src.d_in * 2
+                d.u = src.u + a * src.d_out * 2
+                d.dloss = src.dloss + a * 4
+                d.r = src.r + a * 4
+                if src.g_out:
+                    d.g_out = src.g_out + a * src.d_out * 4
+            if self._ws_need(desc, n, m) > nb:
+                raise RuntimeError("stack workspace too small for a run")
+            key = NoiseKey(seed, 0, draw_offset, token_offset + a).c()
+            cu_d = cu_all[int(offs[c]):int(offs[c + 1])]
+            _check(lib().dust_noisy_linear_fwd_grouped(desc, n, m, self.K, float(sigma), key,
+                                                       self.ws.data_ptr(), nb, s),
+                   "dust_noisy_linear_fwd_grouped")
+            _check(lib().dust_credit_grouped(desc, n, self.K, m, cu_d.data_ptr(),
+                                             cu_d.numel() - 1, float(gamma), self.ws.data_ptr(),
+                                             nb, s), "dust_credit_grouped")
+            last = c == len(ready) - 1
+            self._weight_grad(desc, m, key, c > 0, s, reduce if last else None, buckets)
+        if G_host is None:
+            G_host = torch.empty(self.G_W_flat.shape, dtype=torch.float32, pin_memory=True)
+        G_host.copy_(self.G_W_flat, non_blocking=True)
+        comp.synchronize()
+        return G_host
 
 
 class DustLayer:
@@ -651,15 +828,7 @@ class DustLayer:
             self._W = torch.empty((self.d_out, self.d_in), dtype=hW.dtype, device=dev)
             self._copy = torch.cuda.Stream(device=dev)
         # cuts at sequence ends that keep the per-run views 16-byte aligned
-        ends = cu[(cu % 4 == 0) & (cu > 0) & (cu < N)]
-        cuts = [0]
-        for c in range(1, chunks):
-            if ends.size == 0:
-                break
-            e = int(ends[int(np.argmin(np.abs(ends - N * c / chunks)))])
-            if e > cuts[-1]:
-                cuts.append(e)
-        cuts.append(N)
+        cuts = _sequence_cuts(cu, N, chunks)
         # every run's local cu_seqlens, uploaded once
         locs = [(cu[(cu >= a) & (cu <= b)] - a).astype(np.int32) for a, b in zip(cuts[:-1], cuts[1:])]
         cu_all = torch.from_numpy(np.concatenate(locs)).pin_memory().to(dev, non_blocking=True)

@@ -57,6 +57,26 @@ __global__ void __launch_bounds__(256) normal_sum_kernel(const __grid_constant__
     }
 }
 
+// Philox-only throughput probe: thread g XORs together the words of the blocks
+// (j, g, draw, layer) for j < n_blocks.  The generator's integer part alone (its widening
+// multiplies and XORs), so its rate shows what the multiply pipe allows the noise kernels.
+__global__ void __launch_bounds__(256) word_sum_kernel(const __grid_constant__ NoiseKey key,
+                                                       int64_t n, int32_t n_blocks,
+                                                       uint32_t* out) {
+    for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < n;
+         g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const uint32_t t = key.token_offset + static_cast<uint32_t>(g);
+        uint32_t acc = 0;
+#pragma unroll 2
+        for (int32_t j = 0; j < n_blocks; ++j) {
+            const U4 w = philox4x32_10(key.quad_offset + static_cast<uint32_t>(j), t,
+                                       key.draw_offset, key.layer, key);
+            acc ^= w.x ^ w.y ^ w.z ^ w.w;
+        }
+        out[g] = acc;
+    }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -76,16 +96,29 @@ bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) 
 
 }  // namespace
 
-ErrorWord* device_error_word() {
-    static ErrorWord* addr[kMaxDevices] = {};
-    const int dev = current_device();
-    if (dev < 0 || dev >= kMaxDevices) return nullptr;
-    if (!addr[dev]) {
+void* current_context() {
+    using CtxGetCurrent = CUresult (*)(CUcontext*);
+    static CtxGetCurrent fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
-        addr[dev] = static_cast<ErrorWord*>(p);
-    }
-    return addr[dev];
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrent>(p);
+    });
+    CUcontext c = nullptr;
+    if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
+
+ErrorWord* device_error_word() {
+    static SymbolAddressCache cache;
+    return static_cast<ErrorWord*>(cache.get([] {
+        void* p = nullptr;
+        return cudaGetSymbolAddress(&p, g_error_word) == cudaSuccess ? p : nullptr;
+    }));
 }
 
 int num_sms() {
@@ -185,6 +218,16 @@ dust_status normal_sum_launch(NoiseKey key, int64_t n, int32_t n_quads, float* o
     prof_begin(s);
     normal_sum_kernel<<<blocks, 256, 0, s>>>(key, n, n_quads, out);
     prof_end(s, "normal_sum_probe");
+    return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
+}
+
+dust_status word_sum_launch(NoiseKey key, int64_t n, int32_t n_blocks, uint32_t* out,
+                            cudaStream_t s) {
+    if (n == 0) return DUST_OK;
+    const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, static_cast<int64_t>(num_sms()) * 8));
+    prof_begin(s);
+    word_sum_kernel<<<blocks, 256, 0, s>>>(key, n, n_blocks, out);
+    prof_end(s, "word_sum_probe");
     return cudaGetLastError() == cudaSuccess ? DUST_OK : DUST_ERR_CUDA;
 }
 
@@ -380,11 +423,13 @@ dust_status dust_discounted_credit(const float* c, int64_t ld_c, int32_t K, int6
 dust_status dust_weight_grad(const float* r, int64_t ld_r, const void* x, dust_dtype dt,
                              int64_t N, int32_t d_in, int32_t d_out, int32_t K_chunk,
                              int32_t K_total, float sigma, dust_noise_key key, float* G_W,
-                             int accumulate, float* g_out, void* workspace, size_t ws_bytes,
-                             void* stream) {
+                             int accumulate, float* g_out, int32_t g_terms, void* workspace,
+                             size_t ws_bytes, void* stream) {
     dust_status st = check_layer(x, dt, N, d_in, d_out);
     if (st != DUST_OK) return st;
     if (!r || !G_W || !aligned16(G_W) || (g_out && !aligned16(g_out))) return DUST_ERR_INVALID_ARG;
+    if (g_terms != 1 && g_terms != 2) return DUST_ERR_INVALID_ARG;
+    if (2 * N > 2147483647LL) return DUST_ERR_UNSUPPORTED;  // operand row index is 32-bit
     if (K_chunk < 1 || K_total < K_chunk || ld_r < N || key.channel_offset % 4 != 0)
         return DUST_ERR_INVALID_ARG;
     if (!(sigma > 0.f) || !std::isfinite(sigma)) return DUST_ERR_INVALID_ARG;
@@ -396,7 +441,8 @@ dust_status dust_weight_grad(const float* r, int64_t ld_r, const void* x, dust_d
     st = check_ws(workspace, ws_bytes, need);
     if (st != DUST_OK) return st;
     return wgrad_launch(r, ld_r, x, dt, N, d_in, d_out, K_chunk, K_total, sigma, make_key(key),
-                        G_W, accumulate, g_out, workspace, static_cast<cudaStream_t>(stream));
+                        G_W, accumulate, g_out, g_terms, workspace,
+                        static_cast<cudaStream_t>(stream));
 }
 
 dust_status dust_optimizer_step(const dust_opt_params* opt, const float* G, float* W,
@@ -413,12 +459,14 @@ dust_status dust_optimizer_step(const dust_opt_params* opt, const float* G, floa
 dust_status dust_weight_grad_step(const float* r, int64_t ld_r, const void* x, dust_dtype dt,
                                   int64_t N, int32_t d_in, int32_t d_out, int32_t K_chunk,
                                   int32_t K_total, float sigma, dust_noise_key key, float* G_W,
-                                  int accumulate, float* g_out, const dust_opt_params* opt,
-                                  float* W, void* W_bf16, float* m, float* v, void* workspace,
-                                  size_t ws_bytes, void* stream) {
+                                  int accumulate, float* g_out, int32_t g_terms,
+                                  const dust_opt_params* opt, float* W, void* W_bf16, float* m,
+                                  float* v, void* workspace, size_t ws_bytes, void* stream) {
     dust_status st = check_layer(x, dt, N, d_in, d_out);
     if (st != DUST_OK) return st;
     if (dt != DUST_BF16) return DUST_ERR_UNSUPPORTED;
+    if (g_terms != 1 && g_terms != 2) return DUST_ERR_INVALID_ARG;
+    if (2 * N > 2147483647LL) return DUST_ERR_UNSUPPORTED;
     OptParams o;
     if (!make_opt(opt, &o)) return DUST_ERR_INVALID_ARG;
     if (!r || (G_W && !aligned16(G_W)) || (accumulate && !G_W) || (g_out && !aligned16(g_out)))
@@ -435,8 +483,8 @@ dust_status dust_weight_grad_step(const float* r, int64_t ld_r, const void* x, d
     if (st != DUST_OK) return st;
     const OptTargets t{W, W_bf16, m, v};
     return wgrad_launch(r, ld_r, x, dt, N, d_in, d_out, K_chunk, K_total, sigma, make_key(key),
-                        G_W, accumulate, g_out, workspace, static_cast<cudaStream_t>(stream), &o,
-                        &t);
+                        G_W, accumulate, g_out, g_terms, workspace,
+                        static_cast<cudaStream_t>(stream), &o, &t);
 }
 
 dust_status dust_last_device_error(void* stream, int32_t* info) {
@@ -473,6 +521,18 @@ dust_status dust_debug_normal_sum(dust_noise_key key, int64_t n, int32_t n_quads
             0x100000000ull)
         return DUST_ERR_INVALID_ARG;
     return normal_sum_launch(make_key(key), n, n_quads, out, static_cast<cudaStream_t>(stream));
+}
+
+dust_status dust_debug_word_sum(dust_noise_key key, int64_t n, int32_t n_blocks, uint32_t* out,
+                                void* stream) {
+    if (n < 0 || n_blocks < 0 || (n > 0 && !out) || key.channel_offset % 4 != 0)
+        return DUST_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(out) & 3u) != 0) return DUST_ERR_INVALID_ARG;
+    if (static_cast<uint64_t>(key.token_offset) + static_cast<uint64_t>(n) > 0x100000000ull ||
+        static_cast<uint64_t>(key.channel_offset / 4) + static_cast<uint64_t>(n_blocks) >
+            0x100000000ull)
+        return DUST_ERR_INVALID_ARG;
+    return word_sum_launch(make_key(key), n, n_blocks, out, static_cast<cudaStream_t>(stream));
 }
 
 void dust_debug_credit_skip_publish(int32_t block) { g_credit_skip_publish = block; }
@@ -585,16 +645,18 @@ dust_status dust_credit_grouped(const dust_layer_desc* layers, int32_t n_layers,
 
 dust_status dust_weight_grad_grouped(const dust_layer_desc* layers, int32_t n_layers, int64_t N,
                                      int32_t K_chunk, int32_t K_total, float sigma,
-                                     dust_noise_key key, int accumulate, void* workspace,
-                                     size_t ws_bytes, void* stream) {
+                                     dust_noise_key key, int accumulate, int32_t g_terms,
+                                     void* workspace, size_t ws_bytes, void* stream) {
     dust_status st = check_group(layers, n_layers, N, K_chunk, key, 2);
     if (st != DUST_OK) return st;
     if (K_total < K_chunk || !(sigma > 0.f) || !std::isfinite(sigma)) return DUST_ERR_INVALID_ARG;
+    if (g_terms != 1 && g_terms != 2) return DUST_ERR_INVALID_ARG;
+    if (2 * N > 2147483647LL) return DUST_ERR_UNSUPPORTED;
     auto a = wgrad_args(layers, n_layers);
     st = check_ws(workspace, ws_bytes, wgrad_grouped_workspace_bytes(a.data(), n_layers, N));
     if (st != DUST_OK) return st;
     return wgrad_grouped_launch(a.data(), n_layers, N, K_chunk, K_total, sigma, make_key(key),
-                                accumulate, workspace, static_cast<cudaStream_t>(stream));
+                                accumulate, g_terms, workspace, static_cast<cudaStream_t>(stream));
 }
 
 dust_status dust_profile_enable(int32_t capacity) {

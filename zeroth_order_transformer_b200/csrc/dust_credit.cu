@@ -545,18 +545,14 @@ namespace {
 
 // Device address of g_credit_scratch on the current device.  Host code cannot pass the
 // array's name to a kernel (on the host it is only a stand-in symbol), so the address is
-// looked up once per device, with that device current, and cached.
+// looked up with cudaGetSymbolAddress once per device, with that device current, and cached
+// (thread-safe; looked up again if the device's context was reset).
 void* static_credit_scratch() {
-    constexpr int kMaxDev = 64;
-    static void* addr[kMaxDev] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
-    if (!addr[dev]) {
+    static SymbolAddressCache cache;
+    return cache.get([] {
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_credit_scratch) != cudaSuccess) return nullptr;
-        addr[dev] = p;
-    }
-    return addr[dev];
+        return cudaGetSymbolAddress(&p, g_credit_scratch) == cudaSuccess ? p : nullptr;
+    });
 }
 
 }  // namespace

@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/dust.h"
 
 namespace dust {
@@ -40,6 +42,49 @@ inline NoiseKey make_key(const dust_noise_key& k) {
 
 ErrorWord* device_error_word();  // of the current device
 int num_sms();                   // of the current device
+
+// The CUDA context current on the calling thread (driver handle), or nullptr.
+void* current_context();
+
+// Device address of a file-scope __device__ array, per device context.  Host code only holds
+// a stand-in for such an array, so its device address is looked up (by `lookup`, which must
+// call cudaGetSymbolAddress in the file that defines the array) once per device, with that
+// device current, and kept.  The entry is looked up again if the device's context changed
+// (after cudaDeviceReset the module is loaded again, possibly at another address).  Calls
+// from several host threads are serialised by a mutex.
+class SymbolAddressCache {
+  public:
+    template <class Lookup>
+    void* get(Lookup lookup) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+        void* ctx = current_context();
+        std::lock_guard<std::mutex> guard(mu_);
+        int slot = -1;
+        for (int i = 0; i < n_; ++i)
+            if (e_[i].dev == dev) slot = i;
+        if (slot >= 0 && ctx && e_[slot].ctx == ctx) return e_[slot].ptr;
+        void* p = lookup();
+        if (!p) return nullptr;
+        if (slot < 0) {
+            if (n_ == kMax) return p;  // not cached; still correct
+            slot = n_++;
+        }
+        e_[slot] = Entry{dev, current_context(), p};
+        return p;
+    }
+
+  private:
+    static constexpr int kMax = 64;
+    struct Entry {
+        int dev;
+        void* ctx;
+        void* ptr;
+    };
+    std::mutex mu_;
+    Entry e_[kMax] = {};
+    int n_ = 0;
+};
 
 // Encodes a 2-D row-major bf16 tensor [rows, cols] for TMA with a (box_cols x box_rows) box
 // and 128-byte swizzle.  Returns false if the driver rejects it.
@@ -141,14 +186,15 @@ struct WgradLayerArgs {
     float* g_out;
 };
 size_t wgrad_grouped_workspace_bytes(const WgradLayerArgs* layers, int n, int64_t N);
+// g_terms: 1 (g rounded once to bf16) or 2 (hi + lo bf16 terms) for the bf16 contraction.
 dust_status wgrad_grouped_launch(const WgradLayerArgs* layers, int n, int64_t N, int32_t K_chunk,
                                  int32_t K_total, float sigma, NoiseKey key, int accumulate,
-                                 void* ws, cudaStream_t s);
+                                 int g_terms, void* ws, cudaStream_t s);
 size_t wgrad_workspace_bytes(dust_dtype dt, int64_t N, int32_t d_in, int32_t d_out);
 dust_status wgrad_launch(const float* r, int64_t ld_r, const void* x, dust_dtype dt, int64_t N,
                          int32_t d_in, int32_t d_out, int32_t K_chunk, int32_t K_total,
                          float sigma, NoiseKey key, float* G_W, int accumulate, float* g_out,
-                         void* ws, cudaStream_t s, const OptParams* opt = nullptr,
+                         int g_terms, void* ws, cudaStream_t s, const OptParams* opt = nullptr,
                          const OptTargets* targets = nullptr);
 
 // ---- generator test export (dust_api.cu)

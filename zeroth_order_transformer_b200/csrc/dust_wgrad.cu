@@ -3,17 +3,22 @@
 //
 // Stage 1 (ghat_kernel): one thread per (token, two channel quads) regenerates the quads'
 // normals for every draw and accumulates the reward-weighted sum; g is written as bf16 (the
-// tensor core operand) and optionally as fp32.  A grid-stride loop over units of 128
-// consecutive (token, quad pair) items of a layer keeps every SM busy to the end.
+// tensor core operand) and optionally as fp32.  With two terms the operand is g's bf16
+// rounding hi = bf16(g) in rows [0, N) and the rounding of the remainder lo = bf16(g - hi)
+// in rows [N, 2N): hi + lo carries about 16 significant bits instead of 8.  A grid-stride
+// loop over units of 128 consecutive (token, quad pair) items of a layer keeps every SM busy
+// to the end.
 // Stage 2 (gw_bf16_kernel): G_W = g^T x on the tensor cores.  Both operands are MN-major
 // (tokens are the contraction index and the slow index of g [N, d_out] and x [N, d_in]):
 // TMA loads 64-token x 64-element boxes with 128-byte swizzle, one thread issues
 // tcgen05.mma (M = 128 output rows, N = 256 output columns, K = 16 tokens per instruction)
-// into a TMEM accumulator.  When the outputs have fewer tiles than SMs the token range is
+// into a TMEM accumulator; with two terms each 16-token step issues hi x and lo x into the
+// same accumulator (x is loaded once per stage for both).  When the outputs have fewer tiles than SMs the token range is
 // split (split-K) and a fixed-order reduction adds the partials, so the result is
 // deterministic.  One launch covers up to kMaxGroup layers (tables in parameter space).
 // fp32 layers use a SIMT tiled contraction on the fp32 g.
 #include <algorithm>
+#include <mutex>
 
 #include "dust_device.cuh"
 #include "dust_internal.h"
@@ -28,7 +33,8 @@ constexpr int kGThreads = 128;
 
 struct GhatLayer {
     const float* r;
-    __nv_bfloat16* gb;  // [N, d_out] or null
+    __nv_bfloat16* gb;  // [N, d_out] (hi) or null
+    __nv_bfloat16* gl;  // [N, d_out] (lo, two terms) or null
     float* gf;          // [N, d_out] or null
     int64_t ld_r, unit_begin;
     int64_t n_flat;  // N * ceil(d_out / 8): (token, pair of channel quads) items, token-major
@@ -96,6 +102,20 @@ __global__ void __launch_bounds__(kGThreads, 8) ghat_kernel(const __grid_constan
                 *reinterpret_cast<uint4*>(L.gb + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
             else
                 *reinterpret_cast<uint2*>(L.gb + off) = make_uint2(hv[0], hv[1]);
+            if (L.gl) {
+                // the remainder g - hi is exact in fp32 (|g - hi| <= half a bf16 ulp of g)
+                const float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
+                const float2 f2 = __bfloat1622float2(h[2]), f3 = __bfloat1622float2(h[3]);
+                __nv_bfloat162 lo[4] = {__floats2bfloat162_rn(ga.x - f0.x, ga.y - f0.y),
+                                        __floats2bfloat162_rn(ga.z - f1.x, ga.w - f1.y),
+                                        __floats2bfloat162_rn(gb.x - f2.x, gb.y - f2.y),
+                                        __floats2bfloat162_rn(gb.z - f3.x, gb.w - f3.y)};
+                const uint32_t* lv = reinterpret_cast<const uint32_t*>(lo);
+                if (two)
+                    *reinterpret_cast<uint4*>(L.gl + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+                else
+                    *reinterpret_cast<uint2*>(L.gl + off) = make_uint2(lv[0], lv[1]);
+            }
         }
         if (L.gf) {
             *reinterpret_cast<float4*>(L.gf + off) = ga;
@@ -108,14 +128,19 @@ __global__ void __launch_bounds__(kGThreads, 8) ghat_kernel(const __grid_constan
 constexpr int kGM = 128;  // output rows (o) per tile
 constexpr int kGN = 256;  // output columns (k) per tile
 constexpr int kGK = 64;   // tokens per stage
-constexpr int kGStages = 4;
 constexpr int kGWThreads = 128;
 constexpr uint32_t kBox = 64 * 64 * 2;  // one 64-token x 64-element box
 constexpr uint32_t kGABytes = kGM / 64 * kBox;
 constexpr uint32_t kGBBytes = kGN / 64 * kBox;
-constexpr uint32_t kGStageBytes = kGABytes + kGBBytes;
-constexpr uint32_t kGSmem = kGStages * kGStageBytes + 1024 + 256;
 constexpr uint32_t kGTmemCols = 256;
+// Pipeline shape for one or two g terms: a stage holds the terms' A tiles and the x tile.
+template <int kTerms>
+struct GwShape {
+    static constexpr int kStages = kTerms == 1 ? 4 : 3;
+    static constexpr uint32_t kStageBytes = kTerms * kGABytes + kGBBytes;
+    static constexpr uint32_t kSmem = kStages * kStageBytes + 1024 + 256;
+};
+static_assert(GwShape<2>::kSmem <= 227 * 1024, "two-term pipeline exceeds shared memory");
 
 struct GwLayer {
     float* out;  // G_W (splits == 1; may be null when an optimizer step consumes it) or
@@ -136,8 +161,10 @@ struct GwTable {
     int n_layers;
 };
 
-template <int kMax>
+template <int kMax, int kTerms>
 __global__ void __launch_bounds__(kGWThreads, 1) gw_bf16_kernel(const __grid_constant__ GwTable<kMax> T) {
+    constexpr int kGStages = GwShape<kTerms>::kStages;
+    constexpr uint32_t kGStageBytes = GwShape<kTerms>::kStageBytes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -189,11 +216,19 @@ __global__ void __launch_bounds__(kGWThreads, 1) gw_bf16_kernel(const __grid_con
                 !mbar_wait_bounded(&empty[s], ((kb / kGStages) - 1) & 1, T.ew, 201))
                 break;
             uint8_t* a = smem + s * kGStageBytes;
-            uint8_t* bsm = a + kGABytes;
+            uint8_t* bsm = a + kTerms * kGABytes;
             const int32_t tok = static_cast<int32_t>(t_begin + static_cast<int64_t>(kb) * kGK);
             mbar_arrive_expect_tx(&full[s], kGStageBytes);
 #pragma unroll
             for (int j = 0; j < kGM / 64; ++j) tma_load_2d(a + j * kBox, tmg, &full[s], o0 + 64 * j, tok);
+            if (kTerms == 2) {
+                // lo rows N + tok; rows past 2N read zeros, and hi rows past N (the lo block)
+                // meet x rows past N, which read zeros
+                const int32_t tlo = static_cast<int32_t>(T.N) + tok;
+#pragma unroll
+                for (int j = 0; j < kGM / 64; ++j)
+                    tma_load_2d(a + kGABytes + j * kBox, tmg, &full[s], o0 + 64 * j, tlo);
+            }
 #pragma unroll
             for (int j = 0; j < kGN / 64; ++j)
                 tma_load_2d(bsm + j * kBox, tmx, &full[s], k0 + 64 * j, tok);
@@ -208,12 +243,16 @@ __global__ void __launch_bounds__(kGWThreads, 1) gw_bf16_kernel(const __grid_con
             if (!mbar_wait_bounded(&full[s], (kb / kGStages) & 1, T.ew, 202)) break;
             tc_fence_after();
             const uint32_t a_addr = smem_u32(smem + s * kGStageBytes);
-            const uint32_t b_addr = a_addr + kGABytes;
+            const uint32_t b_addr = a_addr + kTerms * kGABytes;
 #pragma unroll
             for (int kk = 0; kk < kGK / 16; ++kk) {
                 const uint64_t ad = sdesc_sw128(a_addr + kk * 2048, kBox, 1024);
                 const uint64_t bd = sdesc_sw128(b_addr + kk * 2048, kBox, 1024);
                 umma_bf16(tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                if (kTerms == 2) {
+                    const uint64_t ld = sdesc_sw128(a_addr + kGABytes + kk * 2048, kBox, 1024);
+                    umma_bf16(tmem, ld, bd, idesc, 1u);
+                }
             }
             umma_commit(&empty[s]);
         }
@@ -356,15 +395,44 @@ int choose_splits(int64_t tiles, int64_t N) {
     return static_cast<int>(std::max<int64_t>(S, 1));
 }
 
+// bf16 g operand: always room for two terms (hi rows [0, N), lo rows [N, 2N)), so a workspace
+// sized once serves either form.
+size_t g_operand_bytes(int64_t N, int32_t d_out) {
+    return align_up(static_cast<size_t>(2 * N) * d_out * 2, 256);
+}
+
 size_t bf16_layer_ws(int64_t N, int32_t d_in, int32_t d_out, int S) {
-    return align_up(static_cast<size_t>(N) * d_out * 2, 256) +
+    return g_operand_bytes(N, d_out) +
            (S > 1 ? align_up(static_cast<size_t>(S) * d_out * d_in * 4, 256) : 0);
+}
+
+template <int kMax, int kTerms>
+dust_status launch_gw(const GwTable<kMax>& W, int64_t tiles, cudaStream_t s) {
+    static std::once_flag once[64];
+    static cudaError_t attr[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DUST_ERR_CUDA;
+    auto set = [] {
+        return cudaFuncSetAttribute(gw_bf16_kernel<kMax, kTerms>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    GwShape<kTerms>::kSmem);
+    };
+    if (dev < 64) {
+        std::call_once(once[dev], [&] { attr[dev] = set(); });
+        if (attr[dev] != cudaSuccess) return DUST_ERR_CUDA;
+    } else if (set() != cudaSuccess) {
+        return DUST_ERR_CUDA;
+    }
+    gw_bf16_kernel<kMax, kTerms><<<static_cast<unsigned>(tiles), kGWThreads,
+                                   GwShape<kTerms>::kSmem, s>>>(W);
+    return DUST_OK;
 }
 
 template <int kMax>
 dust_status launch_bf16_tables(const WgradLayerArgs* layers, int n, int64_t N, int32_t K_chunk,
                                int32_t K_total, float sigma, const NoiseKey& key, int accumulate,
-                               char* ws, cudaStream_t s, const OptParams* opt = nullptr,
+                               int g_terms, char* ws, cudaStream_t s,
+                               const OptParams* opt = nullptr,
                                const OptTargets* targets = nullptr) {
     int64_t tiles0 = 0;
     for (int l = 0; l < n; ++l) tiles0 += gw_tiles(layers[l].d_in, layers[l].d_out);
@@ -386,6 +454,7 @@ dust_status launch_bf16_tables(const WgradLayerArgs* layers, int n, int64_t N, i
         L.r = a.r;
         L.ld_r = a.ld_r;
         L.gb = reinterpret_cast<__nv_bfloat16*>(ws + off);
+        L.gl = g_terms == 2 ? L.gb + N * a.d_out : nullptr;
         L.gf = a.g_out;
         L.d_out = a.d_out;
         L.n_flat = N * ((a.d_out / 4 + 1) / 2);
@@ -415,7 +484,8 @@ dust_status launch_bf16_tables(const WgradLayerArgs* layers, int n, int64_t N, i
     off = 0;
     for (int l = 0; l < n; ++l) {
         const WgradLayerArgs& a = layers[l];
-        if (!make_tmap_bf16_2d(&W.tmg[l], ws + off, static_cast<uint64_t>(N), a.d_out, kGK, 64) ||
+        if (!make_tmap_bf16_2d(&W.tmg[l], ws + off, static_cast<uint64_t>(g_terms * N), a.d_out,
+                               kGK, 64) ||
             !make_tmap_bf16_2d(&W.tmx[l], a.x, static_cast<uint64_t>(N), a.d_in, kGK, 64))
             return DUST_ERR_CUDA;
         GwLayer& L = W.layer[l];
@@ -433,7 +503,7 @@ dust_status launch_bf16_tables(const WgradLayerArgs* layers, int n, int64_t N, i
             L.out = a.G_W;
             L.accumulate = accumulate;
         } else {
-            L.out = reinterpret_cast<float*>(ws + off + align_up(static_cast<size_t>(N) * a.d_out * 2, 256));
+            L.out = reinterpret_cast<float*>(ws + off + g_operand_bytes(N, a.d_out));
             L.accumulate = 0;
             SplitLayer& Rl = R.layer[n_split_layers++];
             Rl.part = reinterpret_cast<const float4*>(L.out);
@@ -446,18 +516,11 @@ dust_status launch_bf16_tables(const WgradLayerArgs* layers, int n, int64_t N, i
         }
         off += bf16_layer_ws(N, a.d_in, a.d_out, S);
     }
-    static bool attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 64 || !attr_done[dev]) {
-        if (cudaFuncSetAttribute(gw_bf16_kernel<kMax>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kGSmem) != cudaSuccess)
-            return DUST_ERR_CUDA;
-        if (dev < 64) attr_done[dev] = true;
-    }
     prof_begin(s);
-    gw_bf16_kernel<kMax><<<static_cast<unsigned>(tiles), kGWThreads, kGSmem, s>>>(W);
+    const dust_status gst = g_terms == 2 ? launch_gw<kMax, 2>(W, tiles, s)
+                                         : launch_gw<kMax, 1>(W, tiles, s);
     prof_end(s, kMax == 1 ? "gw_bf16_tcgen05" : "gw_bf16_tcgen05_grouped");
+    if (gst != DUST_OK) return gst;
     if (n_split_layers > 0) {
         const unsigned bx = static_cast<unsigned>(
             std::min<int64_t>((max_n4 + 255) / 256, std::max<int64_t>(1, max_blocks / n_split_layers)));
@@ -490,12 +553,13 @@ size_t wgrad_grouped_workspace_bytes(const WgradLayerArgs* layers, int n, int64_
 
 dust_status wgrad_grouped_launch(const WgradLayerArgs* layers, int n, int64_t N, int32_t K_chunk,
                                  int32_t K_total, float sigma, NoiseKey key, int accumulate,
-                                 void* ws, cudaStream_t s) {
+                                 int g_terms, void* ws, cudaStream_t s) {
     char* base = static_cast<char*>(ws);
     for (int l0 = 0; l0 < n; l0 += kMaxGroup) {
         const int cnt = std::min(kMaxGroup, n - l0);
         const dust_status st = launch_bf16_tables<kMaxGroup>(layers + l0, cnt, N, K_chunk, K_total,
-                                                             sigma, key, accumulate, base, s);
+                                                             sigma, key, accumulate, g_terms, base,
+                                                             s);
         if (st != DUST_OK) return st;
         base += wgrad_grouped_workspace_bytes(layers + l0, cnt, N);
     }
@@ -505,11 +569,11 @@ dust_status wgrad_grouped_launch(const WgradLayerArgs* layers, int n, int64_t N,
 dust_status wgrad_launch(const float* r, int64_t ld_r, const void* x, dust_dtype dt, int64_t N,
                          int32_t d_in, int32_t d_out, int32_t K_chunk, int32_t K_total,
                          float sigma, NoiseKey key, float* G_W, int accumulate, float* g_out,
-                         void* ws, cudaStream_t s, const OptParams* opt,
+                         int g_terms, void* ws, cudaStream_t s, const OptParams* opt,
                          const OptTargets* targets) {
     if (dt == DUST_BF16) {
         WgradLayerArgs a{r, ld_r, x, d_in, d_out, key.layer, G_W, g_out};
-        return launch_bf16_tables<1>(&a, 1, N, K_chunk, K_total, sigma, key, accumulate,
+        return launch_bf16_tables<1>(&a, 1, N, K_chunk, K_total, sigma, key, accumulate, g_terms,
                                      static_cast<char*>(ws), s, opt, targets);
     }
     if (opt) return DUST_ERR_UNSUPPORTED;  // fp32 layers: call dust_optimizer_step
@@ -520,7 +584,7 @@ dust_status wgrad_launch(const float* r, int64_t ld_r, const void* x, dust_dtype
     G.K = K_chunk;
     G.scale = -1.0f / (static_cast<float>(K_total) * sigma);
     G.key = key;
-    G.layer[0] = GhatLayer{r, nullptr, gf, ld_r, 0, N * ((d_out / 4 + 1) / 2),
+    G.layer[0] = GhatLayer{r, nullptr, nullptr, gf, ld_r, 0, N * ((d_out / 4 + 1) / 2),
                            div_magic((d_out / 4 + 1) / 2), d_out, key.layer};
     G.total_units = (G.layer[0].n_flat + kGThreads - 1) / kGThreads;
     const int64_t max_blocks = static_cast<int64_t>(num_sms()) * 16;
