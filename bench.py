@@ -619,7 +619,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
 
             def e2e_step():
                 st.estimate_from_host(host_in, data.cu_seqlens, wl.sigma, gamma, wl.seed,
-                                      G_host, chunks=4, reduce=red, buckets=args.buckets,
+                                      G_host, chunks=args.buckets, reduce=red,
                                       token_offset=rank * wl.N)
         else:
             host_layer = dust.DustLayer(wl.N, s1.d_in, s1.d_out, wl.K, tdt, dev)
@@ -655,9 +655,9 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         e2e = {"value": units / (e_ms / args.steps / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e_ms / args.steps,
-               "note": "inputs uploaded from pinned host memory in four runs of whole "
-                       "sequences, each run's upload overlapped with the previous run's "
-                       "estimate; G_W read back"}
+               "note": ("inputs uploaded from pinned host memory in buckets of layers (the "
+                        "stack) or runs of whole sequences (one layer), each overlapped with the "
+                        "previous one's estimate; G_W read back, bucket by bucket for the stack")}
         del host_in
 
     # ---- optional: the optimizer step fused into the weight estimate (single-layer workloads)

@@ -98,9 +98,9 @@ def test_stack_bucketed_reduce_sees_every_layer_once(z):
 
 
 def test_stack_estimate_from_host_matches_device_inputs(z):
-    """The stack from pinned host inputs (uploaded in runs of whole sequences, each run's
-    estimate overlapped with the next run's upload, G_W accumulated over the runs) gives the
-    estimate of the device inputs."""
+    """The stack from pinned host inputs (uploaded in buckets of layers, each bucket's estimate
+    overlapped with the next bucket's upload and its G_W copied back while later buckets run)
+    gives the estimate of the device inputs."""
     import torch
     N, K, sigma, gamma, seed = 1024, 8, 1e-3, 0.99, 0x5EED0005
     layers = _stack(N, 32, 9)

@@ -714,14 +714,17 @@ class DustStack:
 
     def estimate_from_host(self, host_layers, cu_seqlens, sigma: float, gamma: float,
                            seed: int, G_host=None, chunks: int = 4, reduce=None,
-                           buckets: int = 4, draw_offset: int = 0, token_offset: int = 0):
+                           draw_offset: int = 0, token_offset: int = 0):
         """The estimate from inputs in pinned host memory (``host_layers``: one (x, W, u) per
-        layer, the shapes of the stack's device tensors, which receive them), with the upload
-        overlapped: the tokens are cut into ``chunks`` runs of whole sequences; each run of
-        every layer is copied on a copy stream while the previous run goes through the grouped
-        forward, credit and weight estimate (accumulated over the runs; token offsets keep the
-        whole batch's noise).  ``reduce`` as in ``estimate``, on the last run.  The flat G_W
-        comes back into ``G_host`` (pinned, allocated if None).  Synchronises."""
+        layer, the shapes of the stack's device tensors, which receive them), pipelined over
+        ``chunks`` buckets of consecutive layers of about equal input bytes: a copy stream
+        uploads bucket after bucket; each bucket goes through the grouped forward, credit and
+        weight estimate as soon as its inputs are in; its span of G_W_flat is copied back on a
+        third stream (into ``G_host``, pinned, allocated if None) while the later buckets are
+        uploaded and estimated.  ``reduce`` (optional, e.g. the sum over data-parallel ranks)
+        is applied to each bucket's span on a side stream before it is copied back.
+        Synchronises."""
+        from . import distributed
         import numpy as np
         torch = _torch()
         dev = self.ws.device
@@ -730,57 +733,59 @@ class DustStack:
         if N != self.N or len(host_layers) != len(self.layers):
             raise ValueError("host inputs do not match the stack")
         self.sigma = sigma
-        cuts = _sequence_cuts(cu, N, chunks)
-        locs = [(cu[(cu >= a) & (cu <= b)] - a).astype(np.int32)
-                for a, b in zip(cuts[:-1], cuts[1:])]
-        cu_all = torch.from_numpy(np.concatenate(locs)).pin_memory().to(dev, non_blocking=True)
-        offs = np.cumsum([0] + [len(v) for v in locs])
         if not hasattr(self, "_copy"):
             self._copy = torch.cuda.Stream(device=dev)
+            self._back = torch.cuda.Stream(device=dev)
         comp = torch.cuda.current_stream(dev)
+        cu_d = torch.from_numpy(cu.astype(np.int32)).pin_memory().to(dev, non_blocking=True)
+        sizes = [sum(t.numel() * t.element_size() for t in h) for h in host_layers]
+        plan = distributed.plan_buckets(sizes, chunks)
         ready = []
-        self._copy.wait_stream(comp)
+        self._copy.wait_stream(comp)  # the uploads start after the work already queued
         with torch.cuda.stream(self._copy):
-            for (_, W, _, _), (_, hW, _) in zip(self.layers, host_layers):
-                W.copy_(hW, non_blocking=True)
-            for a, b in zip(cuts[:-1], cuts[1:]):
-                for (x, _, u, _), (hx, _, hu) in zip(self.layers, host_layers):
-                    x[a:b].copy_(hx[a:b], non_blocking=True)
-                    u[a:b].copy_(hu[a:b], non_blocking=True)
+            for l0, l1 in plan:
+                for (x, W, u, _), (hx, hW, hu) in zip(self.layers[l0:l1], host_layers[l0:l1]):
+                    W.copy_(hW, non_blocking=True)
+                    x.copy_(hx, non_blocking=True)
+                    u.copy_(hu, non_blocking=True)
                 ev = torch.cuda.Event()
                 ev.record(self._copy)
                 ready.append(ev)
-        n = len(self.layers)
-        nb = self.ws.numel()
-        s = _stream(dev, None)
-        for c, ((a, b), ev) in enumerate(zip(zip(cuts[:-1], cuts[1:]), ready)):
-            comp.wait_event(ev)
-            m = b - a
-            desc = (dust_layer_desc * n)()
-            for l in range(n):
-                d, src = desc[l], self.desc[l]
-                ctypes.memmove(ctypes.byref(d), ctypes.byref(src), ctypes.sizeof(dust_layer_desc))
-                d.x = src.x + a * src.d_in * 2
-                d.u = src.u + a * src.d_out * 2
-                d.dloss = src.dloss + a * 4
-                d.r = src.r + a * 4
-                if src.g_out:
-                    d.g_out = src.g_out + a * src.d_out * 4
-            if self._ws_need(desc, n, m) > nb:
-                raise RuntimeError("stack workspace too small for a run")
-            key = NoiseKey(seed, 0, draw_offset, token_offset + a).c()
-            cu_d = cu_all[int(offs[c]):int(offs[c + 1])]
-            _check(lib().dust_noisy_linear_fwd_grouped(desc, n, m, self.K, float(sigma), key,
-                                                       self.ws.data_ptr(), nb, s),
-                   "dust_noisy_linear_fwd_grouped")
-            _check(lib().dust_credit_grouped(desc, n, self.K, m, cu_d.data_ptr(),
-                                             cu_d.numel() - 1, float(gamma), self.ws.data_ptr(),
-                                             nb, s), "dust_credit_grouped")
-            last = c == len(ready) - 1
-            self._weight_grad(desc, m, key, c > 0, s, reduce if last else None, buckets)
         if G_host is None:
             G_host = torch.empty(self.G_W_flat.shape, dtype=torch.float32, pin_memory=True)
-        G_host.copy_(self.G_W_flat, non_blocking=True)
+        nb = self.ws.numel()
+        s = _stream(dev, None)
+        key = NoiseKey(seed, 0, draw_offset, token_offset).c()
+        if reduce is not None and self._comm is None:
+            self._comm = torch.cuda.Stream(device=dev)
+        for (l0, l1), ev in zip(plan, ready):
+            comp.wait_event(ev)
+            n = l1 - l0
+            sub = self._sub(self.desc, l0)
+            if self._ws_need(sub, n, N) > nb:
+                raise RuntimeError("stack workspace too small for a bucket")
+            _check(lib().dust_noisy_linear_fwd_grouped(sub, n, N, self.K, float(sigma), key,
+                                                       self.ws.data_ptr(), nb, s),
+                   "dust_noisy_linear_fwd_grouped")
+            _check(lib().dust_credit_grouped(sub, n, self.K, N, cu_d.data_ptr(), cu_d.numel() - 1,
+                                             float(gamma), self.ws.data_ptr(), nb, s),
+                   "dust_credit_grouped")
+            _check(lib().dust_weight_grad_grouped(sub, n, N, self.K, self.K, float(sigma), key, 0,
+                                                  self.g_terms, self.ws.data_ptr(), nb, s),
+                   "dust_weight_grad_grouped")
+            a, b = distributed.bucket_span(self.layout, (l0, l1))
+            done = torch.cuda.Event()
+            done.record(comp)
+            src = comp
+            if reduce is not None:
+                self._comm.wait_event(done)
+                with torch.cuda.stream(self._comm):
+                    reduce(self.G_W_flat[a:b])
+                src = self._comm
+            self._back.wait_stream(src)
+            with torch.cuda.stream(self._back):
+                G_host[a:b].copy_(self.G_W_flat[a:b], non_blocking=True)
+        comp.wait_stream(self._back)
         comp.synchronize()
         return G_host
 

@@ -125,22 +125,25 @@ __global__ void __launch_bounds__(kGThreads, 8) ghat_kernel(const __grid_constan
 }
 
 // ------------------------------------------------------------------ stage 2: G_W (bf16)
-constexpr int kGM = 128;  // output rows (o) per tile
+constexpr int kGH = 128;  // output rows (o) per MMA (one TMEM accumulator)
+constexpr int kGM = 256;  // output rows per tile: two MMA halves that share the x tile
 constexpr int kGN = 256;  // output columns (k) per tile
 constexpr int kGK = 64;   // tokens per stage
 constexpr int kGWThreads = 128;
 constexpr uint32_t kBox = 64 * 64 * 2;  // one 64-token x 64-element box
-constexpr uint32_t kGABytes = kGM / 64 * kBox;
+constexpr uint32_t kGHBytes = kGH / 64 * kBox;  // one half's g tile of one term
 constexpr uint32_t kGBBytes = kGN / 64 * kBox;
-constexpr uint32_t kGTmemCols = 256;
-// Pipeline shape for one or two g terms: a stage holds the terms' A tiles and the x tile.
+constexpr uint32_t kGTmemCols = 512;  // two 128 x 256 fp32 accumulators
+// Pipeline shape for one or two g terms: a stage holds both halves' g tiles of every term and
+// the x tile (64 KB or 96 KB), three or two stages in about 192 KB of shared memory.
 template <int kTerms>
 struct GwShape {
-    static constexpr int kStages = kTerms == 1 ? 4 : 3;
-    static constexpr uint32_t kStageBytes = kTerms * kGABytes + kGBBytes;
+    static constexpr uint32_t kStageBytes = kTerms * 2 * kGHBytes + kGBBytes;
+    static constexpr int kStages = kTerms == 1 ? 3 : 2;
     static constexpr uint32_t kSmem = kStages * kStageBytes + 1024 + 256;
 };
-static_assert(GwShape<2>::kSmem <= 227 * 1024, "two-term pipeline exceeds shared memory");
+static_assert(GwShape<1>::kSmem <= 227 * 1024 && GwShape<2>::kSmem <= 227 * 1024,
+              "pipeline exceeds shared memory");
 
 struct GwLayer {
     float* out;  // G_W (splits == 1; may be null when an optimizer step consumes it) or
@@ -207,27 +210,32 @@ __global__ void __launch_bounds__(kGWThreads, 1) gw_bf16_kernel(const __grid_con
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    // rows o0 .. o0 + 127 (half 0) and o0 + 128 .. o0 + 255 (half 1, skipped when the layer
+    // ends before it)
+    const int halves = o0 + kGH < L.d_out ? 2 : 1;
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(tmg);
         prefetch_tensormap(tmx);
+        const uint32_t bytes = static_cast<uint32_t>(kTerms * halves) * kGHBytes + kGBBytes;
         for (int kb = 0; kb < nk; ++kb) {
             const int s = kb % kGStages;
             if (kb >= kGStages &&
                 !mbar_wait_bounded(&empty[s], ((kb / kGStages) - 1) & 1, T.ew, 201))
                 break;
             uint8_t* a = smem + s * kGStageBytes;
-            uint8_t* bsm = a + kTerms * kGABytes;
+            uint8_t* bsm = a + kTerms * 2 * kGHBytes;
             const int32_t tok = static_cast<int32_t>(t_begin + static_cast<int64_t>(kb) * kGK);
-            mbar_arrive_expect_tx(&full[s], kGStageBytes);
+            mbar_arrive_expect_tx(&full[s], bytes);
+            // term tm's half h at a + (tm * 2 + h) * kGHBytes; the lo term's rows start at N
+            // (rows past 2N read zeros, and hi rows past N, the lo block, meet x rows past N,
+            // which read zeros)
+            for (int tm = 0; tm < kTerms; ++tm) {
+                const int32_t trow = tm == 0 ? tok : static_cast<int32_t>(T.N) + tok;
+                for (int h = 0; h < halves; ++h)
 #pragma unroll
-            for (int j = 0; j < kGM / 64; ++j) tma_load_2d(a + j * kBox, tmg, &full[s], o0 + 64 * j, tok);
-            if (kTerms == 2) {
-                // lo rows N + tok; rows past 2N read zeros, and hi rows past N (the lo block)
-                // meet x rows past N, which read zeros
-                const int32_t tlo = static_cast<int32_t>(T.N) + tok;
-#pragma unroll
-                for (int j = 0; j < kGM / 64; ++j)
-                    tma_load_2d(a + kGABytes + j * kBox, tmg, &full[s], o0 + 64 * j, tlo);
+                    for (int j = 0; j < kGH / 64; ++j)
+                        tma_load_2d(a + (tm * 2 + h) * kGHBytes + j * kBox, tmg, &full[s],
+                                    o0 + kGH * h + 64 * j, trow);
             }
 #pragma unroll
             for (int j = 0; j < kGN / 64; ++j)
@@ -236,23 +244,26 @@ __global__ void __launch_bounds__(kGWThreads, 1) gw_bf16_kernel(const __grid_con
     } else if (warp == 1 && lane == 0) {
         // MN-major operands: 64-element (128-byte) rows, one row per token; 8-token core
         // groups 1024 bytes apart (SBO); successive 64-element column blocks one box apart
-        // (LBO); 16 tokens per instruction = 2048 bytes.
-        constexpr uint32_t idesc = idesc_bf16_f32(kGM, kGN, 1, 1);
+        // (LBO); 16 tokens per instruction = 2048 bytes.  Half h accumulates in columns
+        // [256 h, 256 h + 256) of the CTA's tensor memory.
+        constexpr uint32_t idesc = idesc_bf16_f32(kGH, kGN, 1, 1);
         for (int kb = 0; kb < nk; ++kb) {
             const int s = kb % kGStages;
             if (!mbar_wait_bounded(&full[s], (kb / kGStages) & 1, T.ew, 202)) break;
             tc_fence_after();
             const uint32_t a_addr = smem_u32(smem + s * kGStageBytes);
-            const uint32_t b_addr = a_addr + kTerms * kGABytes;
+            const uint32_t b_addr = a_addr + kTerms * 2 * kGHBytes;
 #pragma unroll
             for (int kk = 0; kk < kGK / 16; ++kk) {
-                const uint64_t ad = sdesc_sw128(a_addr + kk * 2048, kBox, 1024);
                 const uint64_t bd = sdesc_sw128(b_addr + kk * 2048, kBox, 1024);
-                umma_bf16(tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
-                if (kTerms == 2) {
-                    const uint64_t ld = sdesc_sw128(a_addr + kGABytes + kk * 2048, kBox, 1024);
-                    umma_bf16(tmem, ld, bd, idesc, 1u);
-                }
+                for (int h = 0; h < halves; ++h)
+#pragma unroll
+                    for (int tm = 0; tm < kTerms; ++tm) {
+                        const uint64_t ad = sdesc_sw128(
+                            a_addr + (tm * 2 + h) * kGHBytes + kk * 2048, kBox, 1024);
+                        umma_bf16(tmem + static_cast<uint32_t>(h * 256), ad, bd, idesc,
+                                  (kb | kk | tm) != 0 ? 1u : 0u);
+                    }
             }
             umma_commit(&empty[s]);
         }
@@ -263,33 +274,37 @@ __global__ void __launch_bounds__(kGWThreads, 1) gw_bf16_kernel(const __grid_con
     __syncwarp();
     tc_fence_after();
 
-    const int o = o0 + warp * 32 + lane;
-    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const int ncols = min(kGN, L.d_in - k0);
     float* dst = L.out ? L.out + static_cast<int64_t>(split) * L.d_out * L.d_in : nullptr;
-    for (int c = 0; c < ncols / 16; ++c) {
-        float v[16];
-        tmem_ld16(trow + c * 16, v);
-        tmem_wait_ld();
-        if (nk == 0) {
+    for (int h = 0; h < halves; ++h) {
+        const int o = o0 + kGH * h + warp * 32 + lane;
+        const uint32_t trow =
+            tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(h * 256);
+        for (int c = 0; c < ncols / 16; ++c) {
+            float v[16];
+            tmem_ld16(trow + c * 16, v);
+            tmem_wait_ld();
+            if (nk == 0) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = 0.f;
-        }
-        if (o < L.d_out) {
-            const int64_t e0 = static_cast<int64_t>(o) * L.d_in + k0 + c * 16;
-            float4* d4 = dst ? reinterpret_cast<float4*>(dst + e0) : nullptr;
+                for (int j = 0; j < 16; ++j) v[j] = 0.f;
+            }
+            if (o < L.d_out) {
+                const int64_t e0 = static_cast<int64_t>(o) * L.d_in + k0 + c * 16;
+                float4* d4 = dst ? reinterpret_cast<float4*>(dst + e0) : nullptr;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                float4 w = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-                if (L.accumulate) {
-                    const float4 old = d4[j];
-                    w.x += old.x;
-                    w.y += old.y;
-                    w.z += old.z;
-                    w.w += old.w;
+                for (int j = 0; j < 4; ++j) {
+                    float4 w = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                    if (L.accumulate) {
+                        const float4 old = d4[j];
+                        w.x += old.x;
+                        w.y += old.y;
+                        w.z += old.z;
+                        w.w += old.w;
+                    }
+                    if (d4) d4[j] = w;
+                    if (T.opt.kind != 0 && L.splits == 1)
+                        opt_update4(T.opt, L.opt, e0 + 4 * j, w);
                 }
-                if (d4) d4[j] = w;
-                if (T.opt.kind != 0 && L.splits == 1) opt_update4(T.opt, L.opt, e0 + 4 * j, w);
             }
         }
     }
