@@ -63,24 +63,34 @@ ALU_KERNELS = {"fwd_bf16_noise_loss": "fwd", "fwd_bf16_noise_loss_grouped": "fwd
                "spsa_estimate": "spsa_est"}
 
 # DRAM bytes (read + write) per launch of a dominant kernel from one ncu capture, with the
-# digest of the CUDA sources that were captured: a value is reported only while the sources
+# digest of the CUDA sources that build that kernel: a value is reported only while those files
 # still have that digest (a changed kernel reports null until it is captured again).  Each
-# entry: (kernel, workload) -> (bytes per launch, source digest, profile summary).
-MEASURED_TRAFFIC = {}
+# entry: (kernel, workload) -> (bytes per launch, source files, their digest, summary).
+_FWD_SOURCES = ("dust_fwd.cu", "dust_device.cuh", "dust_internal.h")
+MEASURED_TRAFFIC = {
+    # the full 48-layer launch, one pass (dram__bytes_read.sum + dram__bytes_write.sum)
+    ("fwd_bf16_noise_loss_grouped", "gpt2s-12-block-stack-48-layers"): (
+        2770000000 + 370430000, _FWD_SOURCES, "6b7c26f22d128cba",
+        "profiles/ncu_dram_stack_48_layers.md"),
+}
 HEAD_METRIC = "Dust LM-head estimator tokens*draws/s"
 ATTN_METRIC = "Dust attention-reward estimator tokens*draws/s"
 
 
-def source_digest() -> str:
-    """sha256 (first 16 hex digits) of the library's CUDA sources and header."""
+def source_digest(files=None) -> str:
+    """sha256 (first 16 hex digits) of the library's CUDA sources (all of them and the public
+    header, or only the named files of csrc/)."""
     import glob
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "zeroth_order_transformer_b200", "csrc")
-    files = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))
-                   + glob.glob(os.path.join(csrc, "*.h"))
-                   + glob.glob(os.path.join(ROOT, "include", "*.h")))
-    for f in files:
+    if files is None:
+        paths = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))
+                       + glob.glob(os.path.join(csrc, "*.h"))
+                       + glob.glob(os.path.join(ROOT, "include", "*.h")))
+    else:
+        paths = [os.path.join(csrc, f) for f in files]
+    for f in paths:
         h.update(os.path.basename(f).encode())
         with open(f, "rb") as fh:
             h.update(fh.read())
@@ -89,9 +99,9 @@ def source_digest() -> str:
 
 def measured_traffic(kernel: str, workload: str):
     e = MEASURED_TRAFFIC.get((kernel, workload))
-    if e is None or e[1] != source_digest():
+    if e is None or e[2] != source_digest(e[1]):
         return None, None
-    return e[0], e[2]
+    return e[0], e[3]
 
 
 def measured_peaks():
@@ -447,7 +457,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
                                 device_id=dev)
-    data = workloads.generate(args.workload)
+    data = workloads.generate(args.workload, n_layers=args.layers)
     wl = data.wl
     gamma = headline_gamma(wl, args.gamma)
     peaks = measured_peaks()
@@ -599,7 +609,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                         "peak_source": peaks["source"]}
         if roofline is not None:
             roofline["units_per_launch"] = amount
-            tr, src = measured_traffic(dominant, wl.name)
+            tr, src = (measured_traffic(dominant, wl.name) if len(layers) == len(wl.layers)
+                       else (None, None))
             roofline["traffic"] = tr
             roofline["traffic_source"] = src or ("null: no ncu capture of the current sources "
                                                  "of this kernel on this workload")
@@ -719,8 +730,9 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "operands": "bf16 x, W, u; u32 Philox words",
         "data": "synthetic (seeded; shapes of the Dust page's transformer layers)",
-        "config": {"workload": describe(wl, gamma), "tokens_per_gpu": wl.N, "K": wl.K,
-                   "layers": len(layers),
+        "config": {"workload": describe(wl, gamma)
+                   + (f"; first {len(layers)} layers only" if len(layers) < len(wl.layers) else ""),
+                   "tokens_per_gpu": wl.N, "K": wl.K, "layers": len(layers),
                    "layer_shapes": sorted({f"{s.d_in}->{s.d_out}" for s in shapes}),
                    "gamma": gamma,
                    "parallelism": (f"dp{world}: one batch per GPU, NCCL all-reduce of G_W"
@@ -1232,6 +1244,9 @@ def main():
     ap.add_argument("--gamma", type=float, default=None,
                     help="credit discount of the headline (default 0.9 for the stack, else the "
                          "workload's own)")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="only the first LAYERS layers of a stack workload (small profiling "
+                         "cases; the line then says so)")
     ap.add_argument("--buckets", type=int, default=4,
                     help="buckets of consecutive layers for the stack's G_W all-reduce (N > 1)")
     ap.add_argument("--no-sweep", action="store_true", help="skip the gamma sweep")
