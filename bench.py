@@ -155,9 +155,10 @@ def headline_gamma(wl, arg):
 
 
 # ------------------------------------------------------------------------------ CPU oracle
-def oracle_sample(data, n_tokens: int, max_seconds: float, gamma=None):
-    """Run the oracle's whole estimator on the first n_tokens of each layer until max_seconds
-    of work; returns (token*draws processed per layer, seconds, threads, description)."""
+def oracle_sample(data, n_tokens: int, max_seconds: float, gamma=None, first: int = 0):
+    """Run the oracle's whole estimator on the first n_tokens of each layer in turn (from layer
+    `first`) until max_seconds of work; returns (token*draws processed per layer, seconds,
+    threads, description)."""
     import oracle
     wl = data.wl
     g = wl.gamma if gamma is None else gamma
@@ -165,7 +166,7 @@ def oracle_sample(data, n_tokens: int, max_seconds: float, gamma=None):
     t0 = time.perf_counter()
     layers_run = 0
     while True:
-        L = data.layers[layers_run % len(data.layers)]
+        L = data.layers[(first + layers_run) % len(data.layers)]
         n = min(n_tokens, wl.N)
         cu = np.asarray(data.cu_seqlens, dtype=np.int64)
         cu = np.unique(np.clip(cu, 0, n)).astype(np.int32)
@@ -193,7 +194,7 @@ def run_reference(args, rank: int, world: int) -> None:
     n_tok = args.ref_tokens
     times = []
     for k in range(args.warmup + args.steps):
-        done, el, cores, desc = oracle_sample(data, n_tok, 0.0, gamma)
+        done, el, cores, desc = oracle_sample(data, n_tok, 0.0, gamma, first=k)
         if k >= args.warmup:
             times.append(el)
     tot = sum(times)
