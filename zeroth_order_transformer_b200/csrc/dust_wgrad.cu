@@ -83,8 +83,8 @@ __global__ void __launch_bounds__(kGThreads, 8) ghat_kernel(const __grid_constan
             const PolarPairs z = normal_quad_pairs(qg, tg, di, L.layer_id, T.key);
             const PolarPairs w = normal_quad_pairs(qg + 1, tg, di, L.layer_id, T.key);
             // r a = kKappa (r nq) (cos, sin) per pair; kKappa is applied with the scale
-            const F2 rz{ri * z.nq.x, ri * z.nq.y};
-            const F2 rw{ri * w.nq.x, ri * w.nq.y};
+            const F2 rz = mul2(F2{ri, ri}, z.nq);
+            const F2 rw = mul2(F2{ri, ri}, w.nq);
             a02 = fma2(rz, z.c, a02);
             a13 = fma2(rz, z.s, a13);
             b02 = fma2(rw, w.c, b02);
