@@ -34,7 +34,7 @@ constexpr int kCB = 128;          // tokens per block
 constexpr int kSeg = 4;           // threads per draw row
 constexpr int kTPT = kCB / kSeg;  // tokens per thread: one 128-byte line
 constexpr int kRowsMax = 128;     // draw rows per block (row group)
-constexpr int kRowsPerWarp = 8;
+constexpr int kRowsPerWarp = 32 / kSeg;  // a warp holds kSeg parts of kRowsPerWarp rows
 constexpr int kMaxThreads = kRowsMax * kSeg;  // 512
 constexpr int kMaxGroup = 64;
 
@@ -213,8 +213,8 @@ __global__ void __launch_bounds__(kThr, kMinBlocks) credit_kernel(const __grid_c
     // Pass 1.  Thread (row i, part sg) owns tokens 32 sg .. 32 sg + 31 of row i and composes
     // their maps from the last token to the first, streaming 16-byte chunks from the slab (the
     // values are not kept in registers, so six CTAs fit on an SM).
-    const int i = warp * kRowsPerWarp + (lane & 7);
-    const int sg = lane >> 3;
+    const int i = warp * kRowsPerWarp + lane % kRowsPerWarp;
+    const int sg = lane / kRowsPerWarp;
     float* line = slab + sg * Rp * kTPT + i * kTPT;
     // the centred values c = mean - loss of chunk cc of this thread's tokens
     auto centred = [&](int cc) {
@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(kThr, kMinBlocks) credit_kernel(const __grid_c
     // suffix over the row's four parts (lanes sg, sg + 8, sg + 16, sg + 24 of the warp)
     float sA = A, sG = G;
 #pragma unroll
-    for (int off = 8; off < 32; off <<= 1) {
+    for (int off = kRowsPerWarp; off < 32; off <<= 1) {
         const float A2 = __shfl_down_sync(0xffffffffu, sA, off);
         const float G2 = __shfl_down_sync(0xffffffffu, sG, off);
         if (lane + off < 32) {
@@ -252,8 +252,8 @@ __global__ void __launch_bounds__(kThr, kMinBlocks) credit_kernel(const __grid_c
         }
     }
     // the map of the parts after this one (identity for the last part)
-    float eA = __shfl_down_sync(0xffffffffu, sA, 8);
-    float eG = __shfl_down_sync(0xffffffffu, sG, 8);
+    float eA = __shfl_down_sync(0xffffffffu, sA, kRowsPerWarp);
+    float eG = __shfl_down_sync(0xffffffffu, sG, kRowsPerWarp);
     if (sg == kSeg - 1) {
         eA = 0.f;
         eG = 1.f;
@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(kThr, kMinBlocks) credit_kernel(const __grid_c
                 }
 #pragma unroll
                 for (int q = 0; q < kSeg; ++q) {
-                    const int src = (lane & 7) + 8 * q;
+                    const int src = lane % kRowsPerWarp + kRowsPerWarp * q;
                     const int kq = __shfl_sync(0xffffffffu, kind, src);
                     const float aq = __shfl_sync(0xffffffffu, va, src);
                     const float gq = __shfl_sync(0xffffffffu, vg, src);
