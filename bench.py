@@ -411,13 +411,19 @@ def measure_targets(dust, torch, dev, peaks, flush, reps: int) -> dict:
     cu = torch.from_numpy(workloads.random_segments(77, N, 256, 2048)).to(dev)
     ws = torch.empty(dust.dust_workspace_size(dust.DUST_OP_CREDIT, dust.DUST_F32, N, 0, 0, K),
                      dtype=torch.uint8, device=dev)
-    ms = _time_probe(lambda: dust.dust_credit(loss, cu, 0.99, r, ws), torch, reps=max(reps, 10))
+    # best of five groups of ten back-to-back launches, as the HBM copy peak is a best of ten
+    groups = [_time_probe(lambda: dust.dust_credit(loss, cu, 0.99, r, ws), torch, reps=10)
+              for _ in range(5)]
+    ms = min(groups)
     gbs = 8.0 * K * N / (ms / 1e3) / 1e9
     out["credit_stress"] = {"K": K, "N": N, "segments": "packed U[256, 2048]", "gamma": 0.99,
-                            "ms": round(ms, 4), "gbs": round(gbs, 1),
+                            "ms": round(ms, 4), "ms_mean_of_groups": round(sum(groups) / 5, 4),
+                            "gbs": round(gbs, 1),
                             "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "target": 0.7,
                             "status": dust.dust_last_device_error()[0],
-                            "note": "2 GiB moved per launch, larger than L2: no flush needed"}
+                            "note": "2 GiB moved per launch, larger than L2: no flush needed; "
+                                    "best of 5 groups of 10 launches (the HBM copy peak is "
+                                    "the best of 10 copies)"}
     del loss, r, ws
     torch.cuda.empty_cache()
 
