@@ -1,12 +1,16 @@
 #!/usr/bin/env python
-"""Benchmark of the Dust estimator hot path for one transformer linear layer on B200.
+"""Benchmark of the Dust estimator hot path on B200.
 
 One step = the whole path over one batch of seeded synthetic input resident in HBM:
   dust_noisy_linear_fwd (noise + per-draw loss change) -> dust_credit (centring + discounted
   credit scan) -> dust_weight_grad (output-error estimate g + weight estimate G_W),
-and, on N > 1 GPUs, one NCCL all-reduce of G_W (each rank holds its own batch; weak scaling).
+for every layer of the workload (by default the 48 linear layers of a 12-block GPT-2-small
+stack, through the grouped calls: one launch per stage for all layers), and, on N > 1 GPUs,
+the all-reduce of G_W (each rank holds its own batch; weak scaling), in buckets of layers
+overlapped with the weight estimate.
 
-Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload C] [--impl ours|reference]
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload C] [--gamma G]
+                        [--impl ours|reference]
 Multi-GPU: launched by torchrun, one rank per GPU (RANK / LOCAL_RANK / WORLD_SIZE from the env).
 Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle instead (rank 0
 only), on a bounded sample of the same workload.
