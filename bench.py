@@ -74,7 +74,7 @@ _FWD_SOURCES = ("dust_fwd.cu", "dust_device.cuh", "dust_internal.h")
 MEASURED_TRAFFIC = {
     # the full 48-layer launch, one pass (dram__bytes_read.sum + dram__bytes_write.sum)
     ("fwd_bf16_noise_loss_grouped", "gpt2s-12-block-stack-48-layers"): (
-        2770000000 + 370430000, _FWD_SOURCES, "6b7c26f22d128cba",
+        2780000000 + 372030000, _FWD_SOURCES, "d75ecd7afd8ba6ea",
         "profiles/ncu_dram_stack_48_layers.md"),
 }
 HEAD_METRIC = "Dust LM-head estimator tokens*draws/s"

@@ -117,6 +117,65 @@ def test_stack_estimate_from_host_matches_device_inputs(z):
         assert _dev.rel_fro(G[o:o + m].reshape(ref[l].shape), ref[l]) < 1e-5, l
 
 
+@pytest.mark.parametrize("g_terms", [1, 2])
+def test_grouped_more_layers_than_one_launch_holds(z, g_terms):
+    """70 small layers: every stage runs as two launches (64 layers is one launch's table).
+    Each layer equals its single-layer calls: loss change, credit and g bit for bit, G_W
+    within fp32 rounding, for either number of bf16 terms of g."""
+    import torch
+    N, K, sigma, gamma, seed = 256, 4, 1e-3, 0.9, 0x5EED0011
+    rng = np.random.default_rng(71)
+    shapes = [workloads.LayerShape(16 * (1 + l % 3), 16 * (1 + (l * 5) % 4), l) for l in range(70)]
+    layers = [workloads.make_layer(rng, sh, N, "bf16", 0.05) for sh in shapes]
+    cu = workloads.random_segments(72, N, 20, 120)
+    cu_d = _dev.cu_to_device(cu)
+    dev_layers = [(*_dev.layer_to_device(L), L.shape.layer_id) for L in layers]
+    st = z.DustStack(dev_layers, K, want_g=True, g_terms=g_terms)
+    st.estimate(cu_d, sigma, gamma, seed)
+    torch.cuda.synchronize()
+    assert z.dust_last_device_error()[0] == 0
+    for l in (0, 1, 33, 63, 64, 65, 69):
+        x, W, u, lid = dev_layers[l]
+        key = z.NoiseKey(seed, lid)
+        dl = z.dust_noisy_linear_fwd(x, W, u, K, sigma, key)
+        r = z.dust_credit(dl, cu_d, gamma)
+        GW, g = z.dust_weight_grad(r, x, W.shape[0], K, sigma, key, g_out=True, g_terms=g_terms)
+        torch.cuda.synchronize()
+        assert torch.equal(st.dloss[l], dl), l
+        assert torch.equal(st.r[l], r), l
+        assert torch.equal(st.g[l], g), l
+        assert _dev.rel_fro(_dev.host(st.G_W[l]), _dev.host(GW)) < 1e-6, l
+    # and against the oracle for the first and the last layer
+    for l in (0, 69):
+        L = layers[l]
+        ref = oracle.dust_layer(L.x_f64, L.W_f64, L.u_f64, K, sigma, gamma, cu, seed, l)
+        assert _dev.rel_fro(_dev.host(st.G_W[l]), ref["G_W"]) <= (
+            _dev.GW_FRO if g_terms == 1 else _dev.FP32_FRO), l
+
+
+def test_stack_estimate_from_host_with_bucketed_reduce(z):
+    """The host-input path with a reduction per bucket of layers (a stand-in collective that
+    doubles its span on the side stream) before each bucket is copied back."""
+    import torch
+    N, K, sigma, gamma, seed = 512, 6, 1e-3, 0.9, 0x5EED0005
+    layers = _stack(N, 32, 13)
+    cu = workloads.random_segments(14, N, 60, 200)
+    dev_layers = [(*_dev.layer_to_device(L), L.shape.layer_id) for L in layers]
+    st = z.DustStack(dev_layers, K)
+    ref = [_dev.host(g).copy() for g in st.estimate(_dev.cu_to_device(cu), sigma, gamma, seed)]
+    host = [tuple(t.cpu().pin_memory() for t in (x, W, u)) for x, W, u, _ in dev_layers]
+    seen = []
+
+    def reduce(G):
+        seen.append(G.numel())
+        G.mul_(2.0)
+
+    G = st.estimate_from_host(host, cu, sigma, gamma, seed, chunks=3, reduce=reduce).numpy()
+    assert sum(seen) == sum(m for _, m in st.layout) and len(seen) == 3
+    for l, (o, m) in enumerate(st.layout):
+        assert _dev.rel_fro(G[o:o + m].reshape(ref[l].shape), 2.0 * ref[l]) < 1e-5, l
+
+
 def test_grouped_rejects_bad_descriptors(z):
     import ctypes
     d = (z.dust_layer_desc * 1)()
