@@ -10,13 +10,15 @@
 // to the end.
 // Stage 2 (gw_bf16_kernel): G_W = g^T x on the tensor cores.  Both operands are MN-major
 // (tokens are the contraction index and the slow index of g [N, d_out] and x [N, d_in]):
-// TMA loads 64-token x 64-element boxes with 128-byte swizzle, one thread issues
+// TMA loads 64-token x 64-element boxes with 128-byte swizzle.  A CTA owns a 256 x 256
+// output tile as two halves of 128 rows, each in its own TMEM accumulator; one thread issues
 // tcgen05.mma (M = 128 output rows, N = 256 output columns, K = 16 tokens per instruction)
-// into a TMEM accumulator; with two terms each 16-token step issues hi x and lo x into the
-// same accumulator (x is loaded once per stage for both).  When the outputs have fewer tiles than SMs the token range is
-// split (split-K) and a fixed-order reduction adds the partials, so the result is
-// deterministic.  One launch covers up to kMaxGroup layers (tables in parameter space).
-// fp32 layers use a SIMT tiled contraction on the fp32 g.
+// for both halves against the same x tile, so x is loaded once per stage for 256 rows; with
+// two terms each 16-token step also issues the lo rows into the same accumulators.  When the
+// outputs have fewer tiles than SMs the token range is split (split-K) and a fixed-order
+// reduction adds the partials, so the result is deterministic.  One launch covers up to
+// kMaxGroup layers (tables in parameter space).  fp32 layers use a SIMT tiled contraction on
+// the fp32 g.
 #include <algorithm>
 #include <mutex>
 
