@@ -130,22 +130,28 @@ __global__ void __launch_bounds__(kGThreads, 8) ghat_kernel(const __grid_constan
 constexpr int kGH = 128;  // output rows (o) per MMA (one TMEM accumulator)
 constexpr int kGM = 256;  // output rows per tile: two MMA halves that share the x tile
 constexpr int kGN = 256;  // output columns (k) per tile
-constexpr int kGK = 64;   // tokens per stage
+constexpr int kGK = 64;   // token granularity of the split-K ranges (a multiple of every stage)
 constexpr int kGWThreads = 128;
-constexpr uint32_t kBox = 64 * 64 * 2;  // one 64-token x 64-element box
-constexpr uint32_t kGHBytes = kGH / 64 * kBox;  // one half's g tile of one term
-constexpr uint32_t kGBBytes = kGN / 64 * kBox;
 constexpr uint32_t kGTmemCols = 512;  // two 128 x 256 fp32 accumulators
-// Pipeline shape for one or two g terms: a stage holds both halves' g tiles of every term and
-// the x tile (64 KB or 96 KB), three or two stages in about 192 KB of shared memory.
+// Pipeline shape for one or two g terms.  A stage holds kK tokens of both halves' g tiles of
+// every term and of the x tile, in boxes of kK tokens x 64 elements: one term, 64-token stages
+// (64 KB, three of them); two terms, 32-token stages (48 KB, four of them), whose longer
+// look-ahead made the two-term contraction 3-4% faster while one term, with half the MMAs per
+// stage, lost 14% at 32 tokens.
 template <int kTerms>
 struct GwShape {
-    static constexpr uint32_t kStageBytes = kTerms * 2 * kGHBytes + kGBBytes;
-    static constexpr int kStages = kTerms == 1 ? 3 : 2;
+    static constexpr int kK = kTerms == 1 ? 64 : 32;
+    static constexpr uint32_t kBox = kK * 64 * 2;         // one kK-token x 64-element box
+    static constexpr uint32_t kHBytes = kGH / 64 * kBox;  // one half's g tile of one term
+    static constexpr uint32_t kBBytes = kGN / 64 * kBox;  // the x tile
+    static constexpr uint32_t kStageBytes = kTerms * 2 * kHBytes + kBBytes;
+    static constexpr int kStages = kTerms == 1 ? 3 : 4;
     static constexpr uint32_t kSmem = kStages * kStageBytes + 1024 + 256;
 };
 static_assert(GwShape<1>::kSmem <= 227 * 1024 && GwShape<2>::kSmem <= 227 * 1024,
               "pipeline exceeds shared memory");
+static_assert(kGK % GwShape<1>::kK == 0 && kGK % GwShape<2>::kK == 0,
+              "split-K ranges must hold whole stages");
 
 struct GwLayer {
     float* out;  // G_W (splits == 1; may be null when an optimizer step consumes it) or
@@ -170,6 +176,10 @@ template <int kMax, int kTerms>
 __global__ void __launch_bounds__(kGWThreads, 1) gw_bf16_kernel(const __grid_constant__ GwTable<kMax> T) {
     constexpr int kGStages = GwShape<kTerms>::kStages;
     constexpr uint32_t kGStageBytes = GwShape<kTerms>::kStageBytes;
+    constexpr int kK = GwShape<kTerms>::kK;
+    constexpr uint32_t kBox = GwShape<kTerms>::kBox;
+    constexpr uint32_t kGHBytes = GwShape<kTerms>::kHBytes;
+    constexpr uint32_t kGBBytes = GwShape<kTerms>::kBBytes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -193,7 +203,7 @@ __global__ void __launch_bounds__(kGWThreads, 1) gw_bf16_kernel(const __grid_con
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t_begin = static_cast<int64_t>(split) * L.tokens_per_split;
     const int64_t t_end = min(T.N, t_begin + L.tokens_per_split);
-    const int nk = t_end > t_begin ? static_cast<int>((t_end - t_begin + kGK - 1) / kGK) : 0;
+    const int nk = t_end > t_begin ? static_cast<int>((t_end - t_begin + kK - 1) / kK) : 0;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kGStages; ++s) {
@@ -226,7 +236,7 @@ __global__ void __launch_bounds__(kGWThreads, 1) gw_bf16_kernel(const __grid_con
                 break;
             uint8_t* a = smem + s * kGStageBytes;
             uint8_t* bsm = a + kTerms * 2 * kGHBytes;
-            const int32_t tok = static_cast<int32_t>(t_begin + static_cast<int64_t>(kb) * kGK);
+            const int32_t tok = static_cast<int32_t>(t_begin + static_cast<int64_t>(kb) * kK);
             mbar_arrive_expect_tx(&full[s], bytes);
             // term tm's half h at a + (tm * 2 + h) * kGHBytes; the lo term's rows start at N
             // (rows past 2N read zeros, and hi rows past N, the lo block, meet x rows past N,
@@ -256,7 +266,7 @@ __global__ void __launch_bounds__(kGWThreads, 1) gw_bf16_kernel(const __grid_con
             const uint32_t a_addr = smem_u32(smem + s * kGStageBytes);
             const uint32_t b_addr = a_addr + kTerms * 2 * kGHBytes;
 #pragma unroll
-            for (int kk = 0; kk < kGK / 16; ++kk) {
+            for (int kk = 0; kk < kK / 16; ++kk) {
                 const uint64_t bd = sdesc_sw128(b_addr + kk * 2048, kBox, 1024);
                 for (int h = 0; h < halves; ++h)
 #pragma unroll
@@ -501,9 +511,10 @@ dust_status launch_bf16_tables(const WgradLayerArgs* layers, int n, int64_t N, i
     off = 0;
     for (int l = 0; l < n; ++l) {
         const WgradLayerArgs& a = layers[l];
+        const uint32_t box = g_terms == 2 ? GwShape<2>::kK : GwShape<1>::kK;
         if (!make_tmap_bf16_2d(&W.tmg[l], ws + off, static_cast<uint64_t>(g_terms * N), a.d_out,
-                               kGK, 64) ||
-            !make_tmap_bf16_2d(&W.tmx[l], a.x, static_cast<uint64_t>(N), a.d_in, kGK, 64))
+                               box, 64) ||
+            !make_tmap_bf16_2d(&W.tmx[l], a.x, static_cast<uint64_t>(N), a.d_in, box, 64))
             return DUST_ERR_CUDA;
         GwLayer& L = W.layer[l];
         L.o_tiles = (a.d_out + kGM - 1) / kGM;
