@@ -1,6 +1,7 @@
 """Parity at the benchmarked sizes, in bench.py's launch configuration, against the oracle's
-own chain (workloads 2-4 whole; the 48-layer stack's shapes with two of its twelve blocks,
-grouped, at the three discounts of its sweep).
+own chain (workloads 2-4 whole; the whole 48-layer stack in one grouped launch per step, as
+benchmarked, at the headline discount 0.9; two of its twelve blocks, grouped, at the three
+discounts of its sweep with the fp32 g kept).
 
 For every workload the oracle evaluates the whole forward (every token, draw and channel),
 its centred loss and its credit over the real segments.  Compared:
@@ -51,8 +52,9 @@ def _credit_tol(r_ref, cu, gamma):
 
 
 def _check_chain(L, cu, K, sigma, gamma, seed, dl, r, g, GW, loss=None, full_gw=False):
-    """Compare the GPU's loss change, credit, fp32 g and G_W with the oracle's chain; loss
-    (the oracle's absolute losses and clean losses) may be passed in when it is reused."""
+    """Compare the GPU's loss change, credit, fp32 g (None: not kept by the GPU run) and G_W
+    with the oracle's chain; loss (the oracle's absolute losses and clean losses) may be passed
+    in when it is reused."""
     lid, d_out = L.shape.layer_id, L.shape.d_out
     if loss is None:
         loss = oracle.noisy_linear_loss(L.x_f64, L.W_f64, L.u_f64, K, sigma, seed, lid)
@@ -71,7 +73,8 @@ def _check_chain(L, cu, K, sigma, gamma, seed, dl, r, g, GW, loss=None, full_gw=
         return
     ch = _channels(d_out)
     g_ref = oracle.output_error(r_ref, K, sigma, seed, d_out, lid, chans=ch)
-    _dev.assert_fp32_close(g[:, ch], g_ref, f"g layer {lid} sampled channels")
+    if g is not None:
+        _dev.assert_fp32_close(g[:, ch], g_ref, f"g layer {lid} sampled channels")
     rows = oracle.weight_grad(g_ref, L.x_f64)
     e = _dev.rel_fro(GW[ch], rows)
     print(f"layer {lid} gamma {gamma}: G_W rel-Fro {e:.3e} over {ch.size} sampled rows")
@@ -126,3 +129,28 @@ def test_grouped_stack_against_oracle_chain(z):
             _check_chain(L, cu, wl.K, wl.sigma, gamma, wl.seed, _dev.host(st.dloss[l]),
                          _dev.host(st.r[l]), _dev.host(st.g[l]), _dev.host(st.G_W[l]),
                          loss=_LOSS[l])
+
+
+def test_whole_48_layer_stack_as_benchmarked_against_oracle_chain(z):
+    """All 48 layers of the 12-block stack, one grouped launch per kernel, no fp32 g kept,
+    gamma 0.9: the launch that bench.py times.  Checked against the oracle: the first block's
+    four layers and the last block's four (every layer shape, both ends of the layer table)."""
+    import torch
+    data = workloads.generate(5)
+    wl = data.wl
+    assert len(data.layers) == 48
+    layers = [(*_dev.layer_to_device(L), L.shape.layer_id) for L in data.layers]
+    st = z.DustStack(layers, wl.K)
+    cu = data.cu_seqlens
+    gamma = 0.9
+    st.estimate(_dev.cu_to_device(cu), wl.sigma, gamma, wl.seed)
+    torch.cuda.synchronize()
+    assert z.dust_last_device_error()[0] == 0
+    checked = (0, 1, 2, 3, 44, 45, 46, 47)
+    host = {l: (_dev.host(st.dloss[l]), _dev.host(st.r[l]), _dev.host(st.G_W[l]))
+            for l in checked}
+    del layers, st
+    torch.cuda.empty_cache()
+    for l in checked:
+        dl, r, GW = host[l]
+        _check_chain(data.layers[l], cu, wl.K, wl.sigma, gamma, wl.seed, dl, r, None, GW)

@@ -46,11 +46,12 @@ __global__ void __launch_bounds__(256) normal_sum_kernel(const __grid_constant__
     for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < n;
          g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const uint32_t t = key.token_offset + static_cast<uint32_t>(g);
+        const PhiloxRun run = philox_run_over_word0(t, key.draw_offset, key.layer, key);
         F2 acc{0.f, 0.f};  // lanes: the quad's two polar pairs
 #pragma unroll 2
         for (int32_t j = 0; j < n_quads; ++j) {
-            const PolarPairs z = normal_quad_pairs(key.quad_offset + static_cast<uint32_t>(j), t,
-                                                   key.draw_offset, key.layer, key);
+            const PolarPairs z =
+                box_muller_pairs(philox_word0(key.quad_offset + static_cast<uint32_t>(j), run, key));
             acc = fma2(z.nq, add2(z.c, z.s), acc);
         }
         out[g] = kKappa * (acc.x + acc.y);
@@ -66,11 +67,11 @@ __global__ void __launch_bounds__(256) word_sum_kernel(const __grid_constant__ N
     for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < n;
          g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const uint32_t t = key.token_offset + static_cast<uint32_t>(g);
+        const PhiloxRun run = philox_run_over_word0(t, key.draw_offset, key.layer, key);
         uint32_t acc = 0;
 #pragma unroll 2
         for (int32_t j = 0; j < n_blocks; ++j) {
-            const U4 w = philox4x32_10(key.quad_offset + static_cast<uint32_t>(j), t,
-                                       key.draw_offset, key.layer, key);
+            const U4 w = philox_word0(key.quad_offset + static_cast<uint32_t>(j), run, key);
             acc ^= w.x ^ w.y ^ w.z ^ w.w;
         }
         out[g] = acc;

@@ -65,6 +65,86 @@ __device__ __forceinline__ U4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c
     return U4{c0, c1, c2, c3};
 }
 
+// Runs of blocks whose counters differ in one word only.  The noise kernels walk either the
+// channel quads of one (token, draw, layer) (word 0 varies) or the draws of one (quad, token,
+// layer) (word 2 varies).  Then the first round's product of the fixed multiplied word and
+// the second round's product of the word it produces are the same for the whole run: they are
+// formed once, with the round keys and fixed words that are XORed into them, and each block of
+// the run costs 18 widening multiplies instead of 20.  The words are those of philox4x32_10.
+//
+// Word 0 varies, counter (q, c1, c2, c3):
+//   round 0:  (hi(M1 c2) ^ c1 ^ rk0,  lo(M1 c2),  hi(M0 q) ^ c3 ^ rk1,  lo(M0 q))
+//             = (a, b, hi(M0 q) ^ e, lo(M0 q))              a, b, e = c3 ^ rk1 fixed
+//   round 1:  (hi(M1 x2) ^ b ^ rk2,  lo(M1 x2),  hi(M0 a) ^ x3 ^ rk3,  lo(M0 a))
+//             = (hi(M1 x2) ^ f, lo(M1 x2), h ^ x3, d)       f = b ^ rk2, h = hi(M0 a) ^ rk3, d fixed
+// Word 2 varies, counter (c0, c1, i, c3):
+//   round 0:  (hi(M1 i) ^ g,  lo(M1 i),  E,  F)             g = c1 ^ rk0; E = hi(M0 c0) ^ c3 ^ rk1,
+//                                                           F = lo(M0 c0) fixed
+//   round 1:  (hi(M1 E) ^ x1 ^ rk2,  lo(M1 E),  hi(M0 x0) ^ F ^ rk3,  lo(M0 x0))
+//             = (h ^ x1, H, hi(M0 x0) ^ f, lo(M0 x0))       h = hi(M1 E) ^ rk2, H, f = F ^ rk3 fixed
+struct PhiloxRun {
+    uint32_t k1, k2, k3, k4;  // word 0 varies: e, f, h, d;  word 2 varies: g, h, H, f
+};
+
+__device__ __forceinline__ void philox_rounds_2_to_9(uint32_t& c0, uint32_t& c1, uint32_t& c2,
+                                                     uint32_t& c3, const NoiseKey& key) {
+#pragma unroll
+    for (int round = 2; round < 10; ++round) {
+        const uint64_t p0 = static_cast<uint64_t>(kPhiloxM0) * c0;
+        const uint64_t p1 = static_cast<uint64_t>(kPhiloxM1) * c2;
+        const uint32_t n0 = static_cast<uint32_t>(p1 >> 32) ^ c1 ^ key.rk[2 * round];
+        const uint32_t n2 = static_cast<uint32_t>(p0 >> 32) ^ c3 ^ key.rk[2 * round + 1];
+        c1 = static_cast<uint32_t>(p1);
+        c3 = static_cast<uint32_t>(p0);
+        c0 = n0;
+        c2 = n2;
+    }
+}
+
+__device__ __forceinline__ PhiloxRun philox_run_over_word0(uint32_t c1, uint32_t c2, uint32_t c3,
+                                                           const NoiseKey& key) {
+    const uint64_t p1 = static_cast<uint64_t>(kPhiloxM1) * c2;
+    const uint32_t a = static_cast<uint32_t>(p1 >> 32) ^ c1 ^ key.rk[0];
+    const uint64_t pa = static_cast<uint64_t>(kPhiloxM0) * a;
+    return PhiloxRun{c3 ^ key.rk[1], static_cast<uint32_t>(p1) ^ key.rk[2],
+                     static_cast<uint32_t>(pa >> 32) ^ key.rk[3], static_cast<uint32_t>(pa)};
+}
+
+__device__ __forceinline__ U4 philox_word0(uint32_t q, const PhiloxRun& R, const NoiseKey& key) {
+    const uint64_t p0 = static_cast<uint64_t>(kPhiloxM0) * q;
+    const uint32_t x2 = static_cast<uint32_t>(p0 >> 32) ^ R.k1;
+    const uint32_t x3 = static_cast<uint32_t>(p0);
+    const uint64_t p1 = static_cast<uint64_t>(kPhiloxM1) * x2;
+    uint32_t c0 = static_cast<uint32_t>(p1 >> 32) ^ R.k2;
+    uint32_t c1 = static_cast<uint32_t>(p1);
+    uint32_t c2 = R.k3 ^ x3;
+    uint32_t c3 = R.k4;
+    philox_rounds_2_to_9(c0, c1, c2, c3, key);
+    return U4{c0, c1, c2, c3};
+}
+
+__device__ __forceinline__ PhiloxRun philox_run_over_word2(uint32_t c0, uint32_t c1, uint32_t c3,
+                                                           const NoiseKey& key) {
+    const uint64_t p0 = static_cast<uint64_t>(kPhiloxM0) * c0;
+    const uint32_t E = static_cast<uint32_t>(p0 >> 32) ^ c3 ^ key.rk[1];
+    const uint64_t pE = static_cast<uint64_t>(kPhiloxM1) * E;
+    return PhiloxRun{c1 ^ key.rk[0], static_cast<uint32_t>(pE >> 32) ^ key.rk[2],
+                     static_cast<uint32_t>(pE), static_cast<uint32_t>(p0) ^ key.rk[3]};
+}
+
+__device__ __forceinline__ U4 philox_word2(uint32_t i, const PhiloxRun& R, const NoiseKey& key) {
+    const uint64_t p1 = static_cast<uint64_t>(kPhiloxM1) * i;
+    const uint32_t x0 = static_cast<uint32_t>(p1 >> 32) ^ R.k1;
+    const uint32_t x1 = static_cast<uint32_t>(p1);
+    const uint64_t p0 = static_cast<uint64_t>(kPhiloxM0) * x0;
+    uint32_t c0 = R.k2 ^ x1;
+    uint32_t c1 = R.k3;
+    uint32_t c2 = static_cast<uint32_t>(p0 >> 32) ^ R.k4;
+    uint32_t c3 = static_cast<uint32_t>(p0);
+    philox_rounds_2_to_9(c0, c1, c2, c3, key);
+    return U4{c0, c1, c2, c3};
+}
+
 // The float with the given sign and exponent bits and the word's top 23 bits m = w >> 9 as
 // mantissa (written as an add: the two bit fields do not overlap).
 __device__ __forceinline__ float mantissa_float(uint32_t exp_bits, uint32_t w) {

@@ -236,6 +236,7 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_bf16_kernel(const __grid_cons
             const int i = unit >> 1;
             const int hf = unit & 1;
             const uint32_t di = T.key.draw_offset + static_cast<uint32_t>(i);
+            const PhiloxRun run = philox_run_over_word0(tg, di, L.layer_id, T.key);
             F2 acc[2] = {{0.f, 0.f}, {0.f, 0.f}};
             const int c_end = hf ? nchunks : half_chunks;
             // s_e of a 16-channel chunk in one tensor-memory read, one wait per four quads (two
@@ -247,8 +248,7 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_bf16_kernel(const __grid_cons
                 tmem_wait_ld();
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
-                    const PolarPairs z = normal_quad_pairs(qbase + c * 4 + qq, tg, di, L.layer_id,
-                                                           T.key);
+                    const PolarPairs z = box_muller_pairs(philox_word0(qbase + c * 4 + qq, run, T.key));
                     const F2 lc = fma2(z.s, F2{se[4 * qq + 2], se[4 * qq + 3]},
                                        mul2(z.c, F2{se[4 * qq + 0], se[4 * qq + 1]}));
                     acc[qq & 1] = fma2(z.nq, lc, acc[qq & 1]);
@@ -621,6 +621,7 @@ __global__ void __launch_bounds__(kPThreads, 1) fwd_persistent_kernel(const __gr
                     const int i = unit >> 1;
                     const int hf = unit & 1;
                     const uint32_t di = T.key.draw_offset + static_cast<uint32_t>(i);
+                    const PhiloxRun run = philox_run_over_word0(tg, di, L.layer_id, T.key);
                     F2 acc[2] = {{0.f, 0.f}, {0.f, 0.f}};
                     const int c_end = hf ? nchunks : half_chunks;
                     for (int c = hf ? half_chunks : 0; c < c_end; ++c) {
@@ -631,8 +632,8 @@ __global__ void __launch_bounds__(kPThreads, 1) fwd_persistent_kernel(const __gr
                             tmem_wait_ld8(se);
 #pragma unroll
                             for (int qq = 0; qq < 2; ++qq) {
-                                const PolarPairs z = normal_quad_pairs(qbase + c * 4 + piece * 2 + qq,
-                                                                       tg, di, L.layer_id, T.key);
+                                const PolarPairs z = box_muller_pairs(
+                                    philox_word0(qbase + c * 4 + piece * 2 + qq, run, T.key));
                                 const F2 lc = fma2(z.s, F2{se[4 * qq + 2], se[4 * qq + 3]},
                                                    mul2(z.c, F2{se[4 * qq + 0], se[4 * qq + 1]}));
                                 acc[qq] = fma2(z.nq, lc, acc[qq]);

@@ -197,9 +197,10 @@ __global__ void __launch_bounds__(kNoiseThreads) ce_noise_kernel(const CeArgs a)
         // lanes: the quad's two polar pairs; accc takes the cosine channels (4q, 4q+2),
         // accs the sine channels (4q+1, 4q+3)
         F2 accc{0.f, 0.f}, accs{0.f, 0.f};
+        const PhiloxRun run = philox_run_over_word0(tg, di, a.key.layer, a.key);
         for (int q = 0; q < nq; ++q) {
             // sigma a = (kKappa sigma nq) (cos, sin) per pair
-            const PolarPairs z = normal_quad_pairs(q0 + q, tg, di, a.key.layer, a.key);
+            const PolarPairs z = box_muller_pairs(philox_word0(q0 + q, run, a.key));
             const float* wq = w + (4 * q) * kStride + lt;
             const F2 r = mul2(F2{sk, sk}, z.nq);
             const F2 xc = mul2(r, z.c), xs = mul2(r, z.s);

@@ -63,12 +63,13 @@ __global__ void __launch_bounds__(256) spsa_dir_kernel(const __grid_constant__ N
         const int o = row % d_out_pad;
         const uint32_t di = key.draw_offset + static_cast<uint32_t>(row / d_out_pad);
         uint2* zr = reinterpret_cast<uint2*>(Z + static_cast<int64_t>(row) * d_in);
+        const PhiloxRun run = philox_run_over_word0(static_cast<uint32_t>(o), di,
+                                                    key.layer | kWeightSpace, key);
         for (int q = lane; q < nq; q += 32) {
             uint2 out = make_uint2(0u, 0u);
             if (o < d_out) {
                 // z = kKappa nq (cos, sin) per pair; lanes: the quad's two pairs
-                const PolarPairs z = normal_quad_pairs(static_cast<uint32_t>(q), static_cast<uint32_t>(o),
-                                                       di, key.layer | kWeightSpace, key);
+                const PolarPairs z = box_muller_pairs(philox_word0(static_cast<uint32_t>(q), run, key));
                 const F2 r = mul2(F2{kKappa, kKappa}, z.nq);
                 const F2 zc = mul2(r, z.c), zs = mul2(r, z.s);  // (z0, z2), (z1, z3)
                 __nv_bfloat162 lo = __floats2bfloat162_rn(zc.x, zs.x);
@@ -533,13 +534,14 @@ __global__ void __launch_bounds__(256) spsa_estimate_kernel(const __grid_constan
         const int o = static_cast<int>(div_by_magic(idx, nq, nq_magic));
         const int q = static_cast<int>(idx - static_cast<int64_t>(o) * nq);
         F2 a02{0.f, 0.f}, a13{0.f, 0.f};  // channels (4q, 4q+2) and (4q+1, 4q+3)
+        const PhiloxRun run = philox_run_over_word2(static_cast<uint32_t>(q), static_cast<uint32_t>(o),
+                                                    key.layer | kWeightSpace, key);
         // unrolled so that independent Philox chains of consecutive probes interleave
 #pragma unroll 4
         for (int j = 0; j < P; ++j) {
             const float pj = __ldg(p + j);
-            const PolarPairs z = normal_quad_pairs(static_cast<uint32_t>(q), static_cast<uint32_t>(o),
-                                                   key.draw_offset + static_cast<uint32_t>(j),
-                                                   key.layer | kWeightSpace, key);
+            const PolarPairs z = box_muller_pairs(
+                philox_word2(key.draw_offset + static_cast<uint32_t>(j), run, key));
             const F2 r = mul2(F2{kKappa, kKappa}, z.nq);
             const F2 zc = mul2(r, z.c), zs = mul2(r, z.s);
             // the direction is the bf16 value of the normal

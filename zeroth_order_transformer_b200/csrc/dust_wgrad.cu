@@ -78,12 +78,14 @@ __global__ void __launch_bounds__(kGThreads, 8) ghat_kernel(const __grid_constan
         // per quad, channel pairs (4q, 4q+2) and (4q+1, 4q+3): the lanes of packed f32x2 operations
         F2 a02{0.f, 0.f}, a13{0.f, 0.f}, b02{0.f, 0.f}, b13{0.f, 0.f};
         const float* rt = L.r + t;
+        const PhiloxRun run_z = philox_run_over_word2(qg, tg, L.layer_id, T.key);
+        const PhiloxRun run_w = philox_run_over_word2(qg + 1, tg, L.layer_id, T.key);
 #pragma unroll 1
         for (int i = 0; i < T.K; ++i) {
             const float ri = __ldg(rt + static_cast<int64_t>(i) * L.ld_r);
             const uint32_t di = T.key.draw_offset + static_cast<uint32_t>(i);
-            const PolarPairs z = normal_quad_pairs(qg, tg, di, L.layer_id, T.key);
-            const PolarPairs w = normal_quad_pairs(qg + 1, tg, di, L.layer_id, T.key);
+            const PolarPairs z = box_muller_pairs(philox_word2(di, run_z, T.key));
+            const PolarPairs w = box_muller_pairs(philox_word2(di, run_w, T.key));
             // r a = kKappa (r nq) (cos, sin) per pair; kKappa is applied with the scale
             const F2 rz = mul2(F2{ri, ri}, z.nq);
             const F2 rw = mul2(F2{ri, ri}, w.nq);
