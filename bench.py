@@ -48,15 +48,18 @@ HEADLINE_GAMMA = 0.9
 # integer multiplies share, and one warp instruction per clock per scheduler (128 lanes).
 PIPE_RATE = {"imad": 64.0, "xu": 16.0, "alu": 64.0, "fma_pipes": 128.0, "issue": 128.0}
 # Per-normal operation counts, from the algorithm (not from compiled code):
-#   Philox4x32-10: per 4 normals, 10 rounds x (2 widening multiplies + 2 three-input XORs)
-#     -> imad 10 results, alu 5;  uniforms: the word's mantissa field (shift, add) -> alu 2;
+#   Philox4x32-10: per 4 normals, 10 rounds x (2 widening multiplies + 2 three-input XORs);
+#     the kernels walk runs of counters that differ in one word, where the first two rounds
+#     share one product each over the run: 18 multiplies and 19 XORs per block
+#     -> imad 9 results, alu 4.75;  uniforms: the word's mantissa field (shift, add) -> alu 2;
 #     the near-one test once per block (max, compare, branch) -> alu 0.75
+#   instructions: 4.5 multiplies + 4.75 XORs + 2 + 0.75 + 2 special functions + 0.75 packed fp32
 #   Box-Muller per pair: lg2, rsqrt, sin, cos -> xu 2;  radius uniform, angle, -sqrt as
 #     packed f32x2 pairs -> fp32 1.5 (0.75 instructions)
 #   consumer: forward 2 fp32 per normal (1 packed instruction); draw reduction r x nq per
 #     pair and 1 fma per normal -> 1.5 (0.75 instructions); LM head sigma a, a degree-5 series
 #     of exp(sigma a) - 1 and the weighted sum -> 7 (4 instructions)
-_GEN = {"imad": 10.0, "xu": 2.0, "alu": 7.75, "fp32": 1.5, "instr": 14.5}
+_GEN = {"imad": 9.0, "xu": 2.0, "alu": 7.5, "fp32": 1.5, "instr": 14.75}
 #   SPSA directions: rho x (cos or sin) and the bf16 pair conversion -> 1 fp32 (1 instruction);
 #     SPSA estimate: the same product and p_j z -> 2 fp32 (1 packed instruction)
 _CONSUMER = {"fwd": (2.0, 1.0), "ghat": (1.5, 0.75), "lmhead": (7.0, 4.0), "spsa_dir": (1.0, 1.0),
@@ -74,7 +77,7 @@ _FWD_SOURCES = ("dust_fwd.cu", "dust_device.cuh", "dust_internal.h")
 MEASURED_TRAFFIC = {
     # the full 48-layer launch, one pass (dram__bytes_read.sum + dram__bytes_write.sum)
     ("fwd_bf16_noise_loss_grouped", "gpt2s-12-block-stack-48-layers"): (
-        2780000000 + 372030000, _FWD_SOURCES, "d75ecd7afd8ba6ea",
+        2779759616 + 371725824, _FWD_SOURCES, "5510dfd7dcd2ce39",
         "profiles/ncu_dram_stack_48_layers.md"),
 }
 HEAD_METRIC = "Dust LM-head estimator tokens*draws/s"
@@ -1258,8 +1261,9 @@ def main():
     ap.add_argument("--layers", type=int, default=None,
                     help="only the first LAYERS layers of a stack workload (small profiling "
                          "cases; the line then says so)")
-    ap.add_argument("--buckets", type=int, default=4,
-                    help="buckets of consecutive layers for the stack's G_W all-reduce (N > 1)")
+    ap.add_argument("--buckets", type=int, default=12,
+                    help="buckets of consecutive layers: the stack's G_W all-reduce (N > 1) and "
+                         "the end-to-end leg's upload pipeline")
     ap.add_argument("--no-sweep", action="store_true", help="skip the gamma sweep")
     ap.add_argument("--no-targets", action="store_true",
                     help="skip the contraction / scan / reduction target measurements")

@@ -131,12 +131,17 @@ def test_grouped_stack_against_oracle_chain(z):
                          loss=_LOSS[l])
 
 
-def test_whole_48_layer_stack_as_benchmarked_against_oracle_chain(z):
+@pytest.fixture(scope="module")
+def stack5():
+    return workloads.generate(5)
+
+
+def test_whole_48_layer_stack_as_benchmarked_against_oracle_chain(z, stack5):
     """All 48 layers of the 12-block stack, one grouped launch per kernel, no fp32 g kept,
     gamma 0.9: the launch that bench.py times.  Checked against the oracle: the first block's
     four layers and the last block's four (every layer shape, both ends of the layer table)."""
     import torch
-    data = workloads.generate(5)
+    data = stack5
     wl = data.wl
     assert len(data.layers) == 48
     layers = [(*_dev.layer_to_device(L), L.shape.layer_id) for L in data.layers]
@@ -154,3 +159,27 @@ def test_whole_48_layer_stack_as_benchmarked_against_oracle_chain(z):
     for l in checked:
         dl, r, GW = host[l]
         _check_chain(data.layers[l], cu, wl.K, wl.sigma, gamma, wl.seed, dl, r, None, GW)
+
+
+def test_whole_48_layer_stack_from_host_inputs_as_benchmarked(z, stack5):
+    """The end-to-end form that bench.py times: the 48 layers' inputs in pinned host memory,
+    uploaded in the default buckets of layers, each bucket estimated while the next one is
+    uploaded, G_W read back bucket by bucket.  Every layer's G_W equals the estimate of the
+    same inputs already on the device (fp32 rounding of the split-K sums, whose plan depends
+    on the launch's tiles)."""
+    import torch
+    data = stack5
+    wl = data.wl
+    layers = [(*_dev.layer_to_device(L), L.shape.layer_id) for L in data.layers]
+    st = z.DustStack(layers, wl.K)
+    cu = data.cu_seqlens
+    ref = [_dev.host(g).copy() for g in st.estimate(_dev.cu_to_device(cu), wl.sigma, 0.9, wl.seed)]
+    host = [tuple(t.cpu().pin_memory() for t in (x, W, u)) for x, W, u, _ in layers]
+    for x, W, u, _ in layers:
+        for t in (x, W, u):
+            t.zero_()
+    G = st.estimate_from_host(host, cu, wl.sigma, 0.9, wl.seed).numpy()
+    assert z.dust_last_device_error()[0] == 0
+    for l, (o, m) in enumerate(st.layout):
+        e = _dev.rel_fro(G[o:o + m].reshape(ref[l].shape), ref[l])
+        assert e < 1e-5, (l, e)

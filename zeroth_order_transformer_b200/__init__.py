@@ -690,7 +690,7 @@ class DustStack:
         comp.wait_stream(self._comm)
 
     def estimate(self, cu_seqlens, sigma: float, gamma: float, seed: int, draw_offset: int = 0,
-                 token_offset: int = 0, stream=None, reduce=None, buckets: int = 4):
+                 token_offset: int = 0, stream=None, reduce=None, buckets: int = 12):
         """Forward, credit and weight estimate of every layer on the device inputs.  ``reduce``
         (optional, e.g. a sum over data-parallel ranks) is applied to G_W_flat in ``buckets``
         spans of consecutive layers, overlapped with the remaining weight estimates; it must
@@ -713,7 +713,7 @@ class DustStack:
         return self.G_W
 
     def estimate_from_host(self, host_layers, cu_seqlens, sigma: float, gamma: float,
-                           seed: int, G_host=None, chunks: int = 4, reduce=None,
+                           seed: int, G_host=None, chunks: int = 12, reduce=None,
                            draw_offset: int = 0, token_offset: int = 0):
         """The estimate from inputs in pinned host memory (``host_layers``: one (x, W, u) per
         layer, the shapes of the stack's device tensors, which receive them), pipelined over
