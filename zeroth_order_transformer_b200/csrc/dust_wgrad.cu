@@ -32,10 +32,12 @@ constexpr int kMaxGroup = 64;
 
 // ------------------------------------------------------------------ stage 1: g
 constexpr int kGThreads = 128;
-// Grid of the draw reduction: CTAs per SM, eight resident at a time.  The CTAs walk the units
-// grid-stride, so this only sets how many times the resident CTAs are replaced: six waves
-// desynchronise the warps of an SM (their Philox multiplies and Box-Muller special functions
-// then overlap better) and beat one wave by 11% and two by 3% on the 48-layer stack.
+// Grid of the draw reduction, in CTAs per SM.  The CTAs walk the units grid-stride, each with
+// an equal share; nine of them (56 registers per thread) fit on an SM at once, so a grid of one
+// wave of eight per SM can land unevenly, and a grid of several small waves lets the block
+// scheduler even out the SMs' loads as CTAs finish.  48 per SM beat one wave of 8 by 11% and 16
+// per SM by 3% on the 48-layer stack; a per-warp start stagger made no difference, so the gain
+// is the balance, not the warps' relative phase.
 constexpr int kGCtasPerSm = 48;
 
 struct GhatLayer {
