@@ -247,6 +247,38 @@ def _credit_tol(ref_c, cu, gamma):
     return 2e-6 * eff * np.max(np.abs(ref_c), axis=1, keepdims=True) + 1e-6
 
 
+@pytest.mark.parametrize("lo,hi", [(256, 2048), (4096, 4096), (7000, 8192)])
+def test_credit_repeats_bit_for_bit_up_to_8192_token_segments(lo, hi):
+    """With every segment at most 8192 tokens (64 look-back blocks) each block's carry is the
+    fixed-order composition of the aggregates of its window, so repeated calls agree bit for
+    bit, whatever the order in which the blocks ran (K = 64 x 1 Mi tokens, more blocks than
+    the GPU holds at once)."""
+    import torch
+    K, N = 64, 1 << 20
+    g = torch.Generator(device="cuda")
+    g.manual_seed(99)
+    loss = torch.randn((K, N), generator=g, device="cuda")
+    cu = _dev.cu_to_device(workloads.random_segments(98, N, lo, hi))
+    first = z.dust_credit(loss, cu, 0.99)
+    for _ in range(4):
+        again = z.dust_credit(loss, cu, 0.99)
+        torch.cuda.synchronize()
+        assert torch.equal(first, again)
+    assert z.dust_last_device_error()[0] == 0
+
+
+def test_credit_segments_longer_than_the_aggregate_window():
+    """Segments of 20k to 60k tokens (windows past 64 blocks, walked with inclusive values):
+    against the oracle within the scan's rounding bound."""
+    N = 1 << 17
+    cu = workloads.random_segments(97, N, 20000, 60000)
+    loss = workloads.gaussian_losses(96, 8, N)
+    got = _credit_gpu(loss, cu, 0.999)
+    ref = oracle.credit(loss.astype(np.float64), cu, 0.999)
+    assert np.all(np.abs(got - ref) <= _credit_tol(ref, cu, 0.999))
+    assert z.dust_last_device_error()[0] == 0
+
+
 @pytest.mark.parametrize("gamma", [0.5, 0.9, 0.95, 0.99])
 def test_credit_general_gamma(gamma):
     K, N = 16, 5000

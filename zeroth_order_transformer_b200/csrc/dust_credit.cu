@@ -12,7 +12,9 @@
 // of the same sub-slab, so every 16-byte shared access of a warp is conflict-free.  Blocks are
 // chained from the end of the stream to its start by decoupled look-back: each warp publishes
 // its rows' aggregate maps (A, G), r_first = A + G r_next, then their inclusive values once
-// the carry from the following blocks is known.  Block indices come from an atomic ticket in
+// the carry from the following blocks is known; a block composes its carry from the
+// aggregates of the blocks up to the next segment end (so the result repeats bit for bit) and
+// takes an inclusive value only beyond 64 blocks.  Block indices come from an atomic ticket in
 // reverse order, so a block only waits for blocks that started before it.  Waits are bounded;
 // a wait that runs out records the error, writes NaN and still publishes, so no other block
 // waits forever.  The credit is written back into the slab and stored by TMA.  With more than
@@ -37,6 +39,11 @@ constexpr int kRowsMax = 128;     // draw rows per block (row group)
 constexpr int kRowsPerWarp = 32 / kSeg;  // a warp holds kSeg parts of kRowsPerWarp rows
 constexpr int kMaxThreads = kRowsMax * kSeg;  // 512
 constexpr int kMaxGroup = 64;
+// Look-back: blocks read per sweep (one per lane of a row: wider sweeps put more polls on the
+// L2 and were slower, 8 blocks by 7% and 16 by 22% on 64 x 4 Mi), and the blocks after b that
+// are composed from aggregates alone (64: every segment of up to 8192 tokens).
+constexpr int kSweep = 4;
+constexpr int kDetBlocks = 64;
 
 struct CreditLayer {
     CUtensorMap tm_loss;  // [K, N] losses, 32 x rows_p boxes, 128-byte swizzle
@@ -261,9 +268,15 @@ __global__ void __launch_bounds__(kThr, kMinBlocks) credit_kernel(const __grid_c
 
     // Look-back, per warp and row: only the blocks up to the first one after b that holds a
     // segment end can reach block b (that block's map has G = 0 on every row), so the window
-    // b + 1 .. jend is known from cu_seqlens.  It is walked four blocks at a time: lane
-    // (row r, part q) polls the words of row r in block base + q, and the four lanes of a row
-    // compose the four answers in block order, stopping at the first inclusive value.
+    // b + 1 .. jend is known from cu_seqlens, and the aggregates of the window alone give the
+    // carry.  The blocks of the window took their tickets just before b, so their inclusive
+    // values are rarely out yet: up to kDetBlocks blocks after b are read as aggregates only, in
+    // sweeps of kSweep blocks, lane (row r, part q) polling blocks base + q + 4k (k < kSweep / 4),
+    // and the four lanes of a row compose the answers in block order.  The carry is then the
+    // same fixed-order composition in every run, and the credit repeats bit for bit.  A window
+    // longer than kDetBlocks (a segment of more than 8192 tokens) is walked on four blocks at a
+    // time, each polled for its inclusive value first, stopping at the first one found; its
+    // last bits then depend on which blocks had published.
     const bool row_ok = i < R;
     {
         const bool publish = (b != T.skip_publish);
@@ -272,15 +285,82 @@ __global__ void __launch_bounds__(kThr, kMinBlocks) credit_kernel(const __grid_c
             aggG[i] = sG;
         }
         float carry_i = 0.f;
+        // every block publishes its aggregate (the last one too: the aggregate-only sweep of
+        // the blocks before it reads it)
+        if (T.gamma != 0.f && sg == 0 && row_ok && publish)
+            st_relaxed64(&aggw[static_cast<int64_t>(b) * T.rows + i],
+                         pack2(sA, __float_as_uint(-sG)));
         if (b != T.nblk - 1 && T.gamma != 0.f) {
-            if (sg == 0 && row_ok && publish)
-                st_relaxed64(&aggw[static_cast<int64_t>(b) * T.rows + i],
-                             pack2(sA, __float_as_uint(-sG)));
             const int jend = s_jend;
             float accA = 0.f, accG = 1.f;
             bool done = !row_ok, failed = false;
             const uint64_t start = global_timer_ns();
-            for (int base = b + 1; base <= jend; base += kSeg) {
+            // sweeps of kSweep blocks read as aggregates only, up to kDetBlocks after b
+            const int det_end = min(jend, b + kDetBlocks);
+            int base = b + 1;
+            for (; base <= det_end && !__all_sync(0xffffffffu, done); base += kSweep) {
+                constexpr int kPer = kSweep / kSeg;  // blocks per lane
+                float va[kPer], vg[kPer];
+                bool pend[kPer];
+                int kind = 0;  // 0: answered; 3: a wait ran out
+#pragma unroll
+                for (int k = 0; k < kPer; ++k) {
+                    va[k] = 0.f;
+                    vg[k] = 1.f;
+                    pend[k] = !done && base + sg + kSeg * k <= det_end;
+                }
+                while (true) {
+                    uint64_t w[kPer];
+#pragma unroll
+                    for (int k = 0; k < kPer; ++k)
+                        if (pend[k])
+                            w[k] = ld_relaxed64(
+                                &aggw[static_cast<int64_t>(base + sg + kSeg * k) * T.rows + i]);
+                    bool any = false;
+#pragma unroll
+                    for (int k = 0; k < kPer; ++k) {
+                        if (pend[k] && (static_cast<uint32_t>(w[k] >> 32) & 0x80000000u)) {
+                            va[k] = __uint_as_float(static_cast<uint32_t>(w[k]));
+                            vg[k] = -__uint_as_float(static_cast<uint32_t>(w[k] >> 32));
+                            pend[k] = false;
+                        }
+                        any = any || pend[k];
+                    }
+                    if (!any) break;
+                    if (global_timer_ns() - start > kWaitLimitNs) {
+                        kind = 3;
+                        break;
+                    }
+                    __nanosleep(32);
+                }
+                // compose blocks base .. base + kSweep - 1 in order: block base + q + 4k is lane
+                // (r, q)'s slot k; blocks past det_end carry the identity map
+#pragma unroll
+                for (int k = 0; k < kPer; ++k) {
+#pragma unroll
+                    for (int q = 0; q < kSeg; ++q) {
+                        const int src = lane % kRowsPerWarp + kRowsPerWarp * q;
+                        const float aq = __shfl_sync(0xffffffffu, va[k], src);
+                        const float gq = __shfl_sync(0xffffffffu, vg[k], src);
+                        if (!done) {
+                            accA = fmaf(accG, aq, accA);
+                            accG = accG * gq;
+                        }
+                    }
+                }
+                int kq = kind;  // the row's: any of its four lanes ran out
+#pragma unroll
+                for (int q = 0; q < kSeg; ++q)
+                    kq = max(kq, __shfl_sync(0xffffffffu, kind,
+                                             lane % kRowsPerWarp + kRowsPerWarp * q));
+                if (kq == 3 && !done) {
+                    failed = true;
+                    done = true;
+                }
+            }
+            if (det_end == jend) done = true;  // the window was composed from aggregates alone
+            base = det_end + 1;
+            for (; base <= jend && !__all_sync(0xffffffffu, done); base += kSeg) {
                 const int j = base + sg;
                 int kind = 0;  // 1: aggregate (va, vg); 2: inclusive value va; 3: wait ran out
                 float va = 0.f, vg = 1.f;
@@ -326,7 +406,6 @@ __global__ void __launch_bounds__(kThr, kMinBlocks) credit_kernel(const __grid_c
                         }
                     }
                 }
-                if (__all_sync(0xffffffffu, done)) break;
             }
             if (failed) {
                 if (sg == 0) report_error(T.ew, kDevTimeout, b);
