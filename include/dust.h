@@ -143,7 +143,10 @@ dust_status dust_noisy_logits_ce(const void* z, int64_t ld_z, dust_dtype dt, con
  * 0 <= gamma <= 1.  K >= 2 (with K = 1 the centred loss is identically 0).
  * The reverse scan chains token blocks by decoupled look-back.  Every wait is bounded (about
  * one second); a wait that runs out writes NaN to its block and sets DUST_ERR_TIMEOUT in the
- * device error word.  Deterministic.
+ * device error word.  Bit-identical from call to call when no segment is longer than 8192
+ * tokens (each block's carry is then composed from its successors' aggregates in a fixed
+ * order); in a longer segment a block may take a successor's published inclusive value, and
+ * the last bits can differ between calls.
  */
 dust_status dust_credit(const float* loss, int64_t ld_loss, int32_t K, int64_t N,
                         const int32_t* cu_seqlens, int32_t n_seq, float gamma, float* r,
