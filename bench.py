@@ -1303,6 +1303,10 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and rank == 0:
+        print(f"bench.py: --gpus {args.gpus} but {world} rank(s) were launched; the line reports "
+              f"the {world} rank(s) that run (launch N > 1 with torch.distributed.run "
+              f"--nproc-per-node N)", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
