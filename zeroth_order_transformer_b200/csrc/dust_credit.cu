@@ -83,7 +83,7 @@ size_t state_bytes(int64_t nblk, int rows) {
 
 size_t smem_bytes(int rows_p) {
     return 1024 + static_cast<size_t>(rows_p) * kCB * 4 + 2 * kCB * 4 +
-           static_cast<size_t>(rows_p) * 4 * 3 + 16;
+           static_cast<size_t>(rows_p) * 4 + 16;
 }
 
 __device__ __forceinline__ uint64_t ld_relaxed64(const uint64_t* p) {
@@ -146,9 +146,7 @@ __global__ void __launch_bounds__(kThr, kMinBlocks) credit_kernel(const __grid_c
                                            ~static_cast<uintptr_t>(1023));
     float* gval = slab + Rp * kCB;  // [kCB]: gamma, or 0 at a segment's last token
     float* mean = gval + kCB;       // [kCB]
-    float* aggA = mean + kCB;       // [Rp]
-    float* aggG = aggA + Rp;        // [Rp]
-    float* carry = aggG + Rp;       // [Rp]: r at the first token after the block
+    float* carry = mean + kCB;      // [Rp]: r at the first token after the block
     uint64_t* bar = reinterpret_cast<uint64_t*>(
         (reinterpret_cast<uintptr_t>(carry + Rp) + 7) & ~static_cast<uintptr_t>(7));
     __shared__ int s_blk, s_jend;
@@ -280,10 +278,6 @@ __global__ void __launch_bounds__(kThr, kMinBlocks) credit_kernel(const __grid_c
     const bool row_ok = i < R;
     {
         const bool publish = (b != T.skip_publish);
-        if (sg == 0) {
-            aggA[i] = sA;
-            aggG[i] = sG;
-        }
         float carry_i = 0.f;
         // every block publishes its aggregate (the last one too: the aggregate-only sweep of
         // the blocks before it reads it)
