@@ -236,6 +236,21 @@ def test_credit_bit_exact_on_integer_losses(seg, gamma, K):
     assert np.array_equal(got.astype(np.float64), ref), np.abs(got - ref).max()
 
 
+@pytest.mark.parametrize("K", [2, 8])
+def test_credit_bit_exact_past_the_aggregate_window(K):
+    """Segments of 15k-25k tokens (look-back windows of more than 64 blocks, walked with
+    inclusive values), gamma = 1, integer losses in [-8, 8]: every partial sum is a multiple of
+    1/K below 2^19 (at most 25k tokens of |c| <= 16), exact in fp32 for K <= 8, so whichever
+    inclusive value a block takes the credit equals the oracle's bit for bit."""
+    N = 60000
+    cu = workloads.random_segments(34, N, 15000, 25000)
+    loss = workloads.dyadic_losses(50 + K, K, N, scale_bits=0, max_abs=8)
+    got = _credit_gpu(loss, cu, 1.0)
+    ref = oracle.credit(loss, cu, 1.0)
+    assert np.array_equal(got.astype(np.float64), ref), np.abs(got - ref).max()
+    assert z.dust_last_device_error()[0] == 0
+
+
 def _credit_tol(ref_c, cu, gamma):
     """fp32 rounding bound of the reverse scan: each step rounds by 2^-24 relative and the
     rounding errors decay by gamma, so the error is below a few 2^-24 times the discounted sum
