@@ -270,11 +270,6 @@ __device__ __forceinline__ PolarPairs box_muller_pairs(const U4& w) {
     return p;
 }
 
-__device__ __forceinline__ PolarPairs normal_quad_pairs(uint32_t q, uint32_t t, uint32_t i,
-                                                        uint32_t layer, const NoiseKey& key) {
-    return box_muller_pairs(philox4x32_10(q, t, i, layer, key));
-}
-
 // The same block with scalar fields: y_p = -L_p >= 0 and q_p = sqrt(y_p).
 struct Polar4 {
     float y0, q0, c0, s0;  // pair 0: channels 4q, 4q+1
