@@ -503,10 +503,12 @@ void fill_common(CreditTable<kMax>& T, const int32_t* cu, int32_t n_seq, int32_t
     T.tma = (ld_loss % 4 == 0) && (ld_r % 4 == 0);
 }
 
-// Points a layer at its workspace region, clears every group's ticket and look-back words, and encodes
-// its TMA descriptors (a table whose descriptors cannot all be encoded uses plain loads).
+// Points a layer at its workspace region, clears every group's ticket and look-back words (unless
+// the caller clears the regions of several layers at once), and encodes its TMA descriptors (a
+// table whose descriptors cannot all be encoded uses plain loads).
 template <int kMax>
-bool place_layer(CreditTable<kMax>& T, CreditLayer& L, char* base, cudaStream_t s) {
+bool place_layer(CreditTable<kMax>& T, CreditLayer& L, char* base, cudaStream_t s,
+                 bool clear = true) {
     L.state = base;
     if (T.tma &&
         !(make_tmap_f32_2d_sw128(&L.tm_loss, L.loss, static_cast<uint64_t>(T.K),
@@ -519,11 +521,9 @@ bool place_layer(CreditTable<kMax>& T, CreditLayer& L, char* base, cudaStream_t 
     L.mean = T.n_groups > 1 && T.centre
                  ? reinterpret_cast<float*>(base + static_cast<size_t>(T.n_groups) * T.state_stride)
                  : nullptr;
-    for (int g = 0; g < T.n_groups; ++g)
-        if (cudaMemsetAsync(base + static_cast<size_t>(g) * T.state_stride, 0, T.state_stride,
-                            s) != cudaSuccess)
-            return false;
-    return true;
+    // the groups' states are contiguous
+    return !clear || cudaMemsetAsync(base, 0, static_cast<size_t>(T.n_groups) * T.state_stride,
+                                     s) == cudaSuccess;
 }
 
 template <int kMax>
@@ -587,13 +587,17 @@ dust_status credit_grouped_launch(const CreditLayerArgs* layers, int n, int32_t 
         for (int l = 0; l < cnt; ++l)
             aligned = aligned && layers[l0 + l].ld_loss % 4 == 0 && layers[l0 + l].ld_r % 4 == 0;
         fill_common(T, cu, n_seq, K, N, gamma, -1, aligned ? 4 : 1, aligned ? 4 : 1);
+        // the table's layers' regions are contiguous: one memset clears their states (and the
+        // per-token means, which the mean pass rewrites)
+        if (cudaMemsetAsync(base, 0, static_cast<size_t>(cnt) * per, s) != cudaSuccess)
+            return DUST_ERR_CUDA;
         for (int l = 0; l < cnt; ++l) {
             CreditLayer& L = T.layer[l];
             L.loss = layers[l0 + l].loss;
             L.r = layers[l0 + l].r;
             L.ld_loss = layers[l0 + l].ld_loss;
             L.ld_r = layers[l0 + l].ld_r;
-            if (!place_layer(T, L, base, s)) return DUST_ERR_CUDA;
+            if (!place_layer(T, L, base, s, false)) return DUST_ERR_CUDA;
             base += per;
         }
         const dust_status st = launch_credit_table(T, cnt, s, "credit_scan_grouped");

@@ -352,7 +352,11 @@ dust_status launch_bf16_table(const FwdLayerArgs* layers, int n, int64_t N, int 
     T.h_lg2 = static_cast<float>(0.69314718055994531 * sigma * sigma);
     T.key = key;
     int64_t tiles = 0;
-    size_t off = 0;
+    // the layers' unit counters side by side at the start of the workspace (one memset clears
+    // them all), then the layers' partials; the same total as the sum of bf16_layer_ws
+    const size_t counters_bytes = align_up(static_cast<size_t>(T.m_tiles) * 4, 256);
+    size_t off = static_cast<size_t>(n) * counters_bytes;
+    if (cudaMemsetAsync(ws, 0, off, s) != cudaSuccess) return DUST_ERR_CUDA;
     for (int l = 0; l < n; ++l) {
         const FwdLayerArgs& a = layers[l];
         if (!make_tmap_bf16_2d(&T.tmx[l], a.x, static_cast<uint64_t>(N), a.d_in, kBM, kBK) ||
@@ -362,8 +366,7 @@ dust_status launch_bf16_table(const FwdLayerArgs* layers, int n, int64_t N, int 
         const int n_tiles = (a.d_out + kBN - 1) / kBN;
         L.u = static_cast<const __nv_bfloat16*>(a.u);
         L.partial = reinterpret_cast<float*>(ws + off);
-        L.counters = reinterpret_cast<int*>(
-            ws + off + align_up(static_cast<size_t>(2 * n_tiles) * K * N * 4, 256));
+        L.counters = reinterpret_cast<int*>(ws + static_cast<size_t>(l) * counters_bytes);
         L.dloss = a.dloss;
         L.ld = a.ld;
         L.d_in = a.d_in;
@@ -371,11 +374,9 @@ dust_status launch_bf16_table(const FwdLayerArgs* layers, int n, int64_t N, int 
         L.n_tiles = n_tiles;
         L.tile_begin = static_cast<int>(tiles);
         L.layer_id = a.layer_id;
-        if (cudaMemsetAsync(L.counters, 0, static_cast<size_t>(T.m_tiles) * 4, s) != cudaSuccess)
-            return DUST_ERR_CUDA;
         tiles += static_cast<int64_t>(n_tiles) * T.m_tiles;
         if (tiles > 2147483647LL) return DUST_ERR_UNSUPPORTED;
-        off += bf16_layer_ws(N, a.d_out, K);
+        off += align_up(static_cast<size_t>(2 * n_tiles) * K * N * 4, 256);
     }
     static bool attr_done[64] = {};
     int dev = 0;
