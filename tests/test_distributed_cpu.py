@@ -179,6 +179,8 @@ def test_flat_layout_and_bucket_plan():
         assert len(plan) == min(nb, 48)
     per = [sum(sizes[a:b]) for a, b in zd.plan_buckets(sizes, 4)]
     assert max(per) <= 1.2 * sum(sizes) / 4                 # whole blocks: even buckets
+    # the default of the stack's calls and of bench.py: twelve buckets, one transformer block each
+    assert zd.plan_buckets(sizes, 12) == [(4 * k, 4 * k + 4) for k in range(12)]
     a, b = zd.bucket_span(layout, (12, 24))
     assert a == layout[12][0] and b == layout[23][0] + layout[23][1]
     assert zd.plan_buckets([], 3) == [] and zd.plan_buckets([5, 1], 9) == [(0, 1), (1, 2)]
