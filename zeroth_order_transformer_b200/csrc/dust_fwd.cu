@@ -378,15 +378,13 @@ dust_status launch_bf16_table(const FwdLayerArgs* layers, int n, int64_t N, int 
         if (tiles > 2147483647LL) return DUST_ERR_UNSUPPORTED;
         off += align_up(static_cast<size_t>(2 * n_tiles) * K * N * 4, 256);
     }
-    static bool attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 64 || !attr_done[dev]) {
-        if (cudaFuncSetAttribute(fwd_bf16_kernel<kMax>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kSmemBytes) != cudaSuccess)
-            return DUST_ERR_CUDA;
-        if (dev < 64) attr_done[dev] = true;
-    }
+    static PerContextOnce attr;
+    if (!attr.run([] {
+            return cudaFuncSetAttribute(fwd_bf16_kernel<kMax>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kSmemBytes) == cudaSuccess;
+        }))
+        return DUST_ERR_CUDA;
     // Full waves of two CTAs per SM take whole tiles; the remainder is split (see the kernel).
     T.total_tiles = tiles;
     const int64_t slots = 2LL * num_sms();
@@ -714,15 +712,13 @@ dust_status launch_persistent(const FwdLayerArgs* layers, int n, int64_t N, int 
         off += bf16_layer_ws(N, a.d_out, K);
     }
     T.total_tiles = tiles;
-    static bool attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 64 || !attr_done[dev]) {
-        if (cudaFuncSetAttribute(fwd_persistent_kernel<kMax>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kPSmemBytes) != cudaSuccess)
-            return DUST_ERR_CUDA;
-        if (dev < 64) attr_done[dev] = true;
-    }
+    static PerContextOnce attr;
+    if (!attr.run([] {
+            return cudaFuncSetAttribute(fwd_persistent_kernel<kMax>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kPSmemBytes) == cudaSuccess;
+        }))
+        return DUST_ERR_CUDA;
     const int64_t grid = std::min<int64_t>(num_sms(), tiles * 2 * K);
     prof_begin(s);
     fwd_persistent_kernel<kMax><<<static_cast<unsigned>(grid), kPThreads, kPSmemBytes, s>>>(T);

@@ -86,6 +86,22 @@ class SymbolAddressCache {
     int n_ = 0;
 };
 
+// Runs `set` (returning true on success) once per device context: a kernel's function
+// attributes belong to the context, so after a context reset the next call sets them again.
+// Thread-safe; a failed `set` is tried again on the next call.
+class PerContextOnce {
+  public:
+    template <class Set>
+    bool run(Set set) {
+        return cache_.get([&]() -> void* {
+                   return set() ? reinterpret_cast<void*>(static_cast<uintptr_t>(1)) : nullptr;
+               }) != nullptr;
+    }
+
+  private:
+    SymbolAddressCache cache_;
+};
+
 // Encodes a 2-D row-major bf16 tensor [rows, cols] for TMA with a (box_cols x box_rows) box
 // and 128-byte swizzle.  Returns false if the driver rejects it.
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,

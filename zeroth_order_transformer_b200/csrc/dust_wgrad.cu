@@ -444,21 +444,13 @@ size_t bf16_layer_ws(int64_t N, int32_t d_in, int32_t d_out, int S) {
 
 template <int kMax, int kTerms>
 dust_status launch_gw(const GwTable<kMax>& W, int64_t tiles, cudaStream_t s) {
-    static std::once_flag once[64];
-    static cudaError_t attr[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return DUST_ERR_CUDA;
-    auto set = [] {
-        return cudaFuncSetAttribute(gw_bf16_kernel<kMax, kTerms>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    GwShape<kTerms>::kSmem);
-    };
-    if (dev < 64) {
-        std::call_once(once[dev], [&] { attr[dev] = set(); });
-        if (attr[dev] != cudaSuccess) return DUST_ERR_CUDA;
-    } else if (set() != cudaSuccess) {
+    static PerContextOnce attr;
+    if (!attr.run([] {
+            return cudaFuncSetAttribute(gw_bf16_kernel<kMax, kTerms>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        GwShape<kTerms>::kSmem) == cudaSuccess;
+        }))
         return DUST_ERR_CUDA;
-    }
     gw_bf16_kernel<kMax, kTerms><<<static_cast<unsigned>(tiles), kGWThreads,
                                    GwShape<kTerms>::kSmem, s>>>(W);
     return DUST_OK;
