@@ -77,7 +77,7 @@ _FWD_SOURCES = ("dust_fwd.cu", "dust_device.cuh", "dust_internal.h")
 MEASURED_TRAFFIC = {
     # the full 48-layer launch, one pass (dram__bytes_read.sum + dram__bytes_write.sum)
     ("fwd_bf16_noise_loss_grouped", "gpt2s-12-block-stack-48-layers"): (
-        2779303168 + 371896576, _FWD_SOURCES, "7df83608833ad37d",
+        2783402752 + 372459008, _FWD_SOURCES, "030dab1ab282d541",
         "profiles/ncu_dram_stack_48_layers.md"),
 }
 HEAD_METRIC = "Dust LM-head estimator tokens*draws/s"
