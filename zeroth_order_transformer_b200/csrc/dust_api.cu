@@ -3,6 +3,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <mutex>
 #include <vector>
@@ -123,16 +124,18 @@ ErrorWord* device_error_word() {
 }
 
 int num_sms() {
-    static int cache[kMaxDevices] = {};
+    // the count never changes for a device; several host threads may fill an entry at once
+    // and store the same value (atomic, so that is not a data race)
+    static std::atomic<int> cache[kMaxDevices];
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices) return 148;
-    if (!cache[dev]) {
-        int n = 0;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (!n) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
             n = 148;
-        cache[dev] = n;
+        cache[dev].store(n, std::memory_order_relaxed);
     }
-    return cache[dev];
+    return n;
 }
 
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
